@@ -1,0 +1,543 @@
+// C ABI of the bq library (declared in include/bq.h): argument validation on
+// the host, the mapping from a granularity to contiguous groups, and the
+// choice between the single-pass and two-pass paths. Nothing here computes
+// on the host; every result comes from the kernels, enqueued on the
+// caller's stream.
+#include <cstring>
+
+#include "bq.h"
+#include "bq_internal.h"
+
+using bq::DT;
+
+namespace {
+
+bool is_float(bq_dtype t) { return t == BQ_F32 || t == BQ_F64 || t == BQ_F16 || t == BQ_BF16; }
+bool is_half_or_f32(bq_dtype t) { return t == BQ_F32 || t == BQ_F16 || t == BQ_BF16; }
+DT to_dt(bq_dtype t) {
+    switch (t) {
+        case BQ_F32: return DT::F32;
+        case BQ_F64: return DT::F64;
+        case BQ_F16: return DT::F16;
+        default: return DT::BF16;
+    }
+}
+int64_t esize(bq_dtype t) {
+    switch (t) {
+        case BQ_F32: return 4;
+        case BQ_F64: return 8;
+        case BQ_F16: case BQ_BF16: return 2;
+        default: return 1;
+    }
+}
+bool aligned(const void* p, int64_t n) { return ((uintptr_t)p % (uintptr_t)n) == 0; }
+bq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA; }
+cudaStream_t S(void* s) { return (cudaStream_t)s; }
+
+// Granularities as the kernels see them (per-token is its own case).
+enum Gr { GR_TENSOR = 0, GR_CHANNEL = 1, GR_GROUP = 2, GR_TOKEN = 3 };
+
+struct Layout {
+    bq::SegView sv;   // n_seg groups of G contiguous elements
+};
+
+// Shape checks shared by every entry point: ndim in [0, 8], sizes >= 0 and
+// an element count that fits in 62 bits.
+bq_status shape_numel(const bq_qdesc* d, int64_t* numel) {
+    if (!d || d->ndim < 0 || d->ndim > 8) return BQ_ERR_INVALID_ARG;
+    int64_t n = 1;
+    for (int i = 0; i < d->ndim; ++i) {
+        const int64_t s = d->shape[i];
+        if (s < 0) return BQ_ERR_INVALID_ARG;
+        if (s != 0 && n > ((int64_t)1 << 62) / s) return BQ_ERR_INVALID_ARG;
+        n *= s;
+    }
+    *numel = n;
+    return BQ_OK;
+}
+
+// [granularity] (axis, group_size) -> contiguous groups. With x viewed as
+// [outer, L, inner], group g of outer index o covers axis indices
+// [g*gs, (g+1)*gs) and every inner index: gs*inner consecutive elements.
+bq_status make_layout(const bq_qdesc* d, int gr, int32_t axis, int64_t gs, Layout* out) {
+    int64_t numel;
+    bq_status st = shape_numel(d, &numel);
+    if (st != BQ_OK) return st;
+    bq::SegView sv;
+    sv.numel = numel;
+    if (gr == GR_TENSOR) {
+        sv.n_seg = 1;
+        sv.G = numel;
+    } else if (gr == GR_TOKEN) {
+        if (d->ndim < 1) return BQ_ERR_INVALID_ARG;
+        const int64_t last = d->shape[d->ndim - 1];
+        sv.G = last;
+        sv.n_seg = last ? numel / last : 0;
+    } else {
+        if (axis < 0 || axis >= d->ndim) return BQ_ERR_INVALID_ARG;
+        if (gr == GR_CHANNEL) gs = 1;
+        if (gs < 1) return BQ_ERR_INVALID_ARG;
+        int64_t outer = 1, inner = 1;
+        for (int i = 0; i < axis; ++i) outer *= d->shape[i];
+        for (int i = axis + 1; i < d->ndim; ++i) inner *= d->shape[i];
+        const int64_t L = d->shape[axis];
+        if (L % gs != 0) return BQ_ERR_INVALID_ARG;
+        sv.n_seg = outer * (L / gs);
+        sv.G = gs * inner;
+    }
+    out->sv = sv;
+    return BQ_OK;
+}
+
+// Code range: validates dtypes and resolves qmin = qmax = 0 to the defaults.
+bq_status make_cfg(const bq_qdesc* d, bool need_x, bq::IntCfg* c) {
+    if (need_x && !is_float(d->x_dtype)) return BQ_ERR_UNSUPPORTED;
+    if (d->q_dtype != BQ_S8 && d->q_dtype != BQ_U8) return BQ_ERR_UNSUPPORTED;
+    if (d->rnd != BQ_RNE && d->rnd != BQ_RHAZ) return BQ_ERR_INVALID_ARG;
+    int32_t lo, hi;
+    bq_default_q_range(d->q_dtype, &lo, &hi);
+    int32_t qmin = d->qmin, qmax = d->qmax;
+    if (qmin == 0 && qmax == 0) { qmin = lo; qmax = hi; }
+    if (qmin < lo || qmax > hi || qmin >= qmax) return BQ_ERR_INVALID_ARG;
+    if (d->symmetric && d->q_dtype == BQ_U8) return BQ_ERR_UNSUPPORTED;
+    if (d->symmetric && qmax <= 0) return BQ_ERR_INVALID_ARG;
+    c->qmin = qmin;
+    c->qmax = qmax;
+    c->symmetric = d->symmetric ? 1 : 0;
+    c->rhaz = d->rnd == BQ_RHAZ ? 1 : 0;
+    c->q_signed = d->q_dtype == BQ_S8 ? 1 : 0;
+    return BQ_OK;
+}
+
+// Whether the single-pass kernel can take this call, judged from shape,
+// dtype and rounding only (pointer alignment is checked at launch).
+bool single_pass_possible(const bq_qdesc* d, const bq::SegView& sv) {
+    if (d->x_dtype == BQ_F64 || d->rnd != BQ_RNE) return false;
+    const int64_t vec = d->x_dtype == BQ_F32 ? 4 : 8;
+    return sv.G > 0 && sv.G % vec == 0 && sv.G <= 4096 * vec;
+}
+
+// quantize / fake_quantize, every granularity and scale mode.
+bq_status quant_impl(int op, const void* x, const bq_qdesc* d, int gr, int32_t axis, int64_t gs,
+                     void* q, float* scale, void* zp, bq_scale_mode mode, void* y, void* ws,
+                     size_t ws_bytes, void* stream) {
+    Layout lay;
+    bq_status st = make_layout(d, gr, axis, gs, &lay);
+    if (st != BQ_OK) return st;
+    bq::IntCfg cfg;
+    if ((st = make_cfg(d, true, &cfg)) != BQ_OK) return st;
+    if (mode != BQ_SCALE_DYNAMIC && mode != BQ_SCALE_STATIC && mode != BQ_SCALE_FROM_RANGE)
+        return BQ_ERR_INVALID_ARG;
+    const bq::SegView sv = lay.sv;
+    const bool asym = !cfg.symmetric;
+    if (sv.numel > 0 && !x) return BQ_ERR_INVALID_ARG;
+    if (op == bq::OP_QUANT && sv.numel > 0 && !q) return BQ_ERR_INVALID_ARG;
+    if (op == bq::OP_FAKE && sv.numel > 0 && !y) return BQ_ERR_INVALID_ARG;
+    if (sv.n_seg > 0 && !scale) return BQ_ERR_INVALID_ARG;
+    if (mode == BQ_SCALE_STATIC && asym && sv.n_seg > 0 && !zp) return BQ_ERR_INVALID_ARG;
+    const int64_t es = esize(d->x_dtype);
+    if (!aligned(x, es) || !aligned(scale, 4) || (y && !aligned(y, es))) return BQ_ERR_MISALIGNED;
+    const size_t need_ranges = (size_t)sv.n_seg * 16;
+    if (mode == BQ_SCALE_FROM_RANGE) {
+        if (sv.n_seg > 0 && (!ws || ws_bytes < need_ranges)) return BQ_ERR_INVALID_ARG;
+        if (!aligned(ws, 8)) return BQ_ERR_MISALIGNED;
+    }
+    const DT dt = to_dt(d->x_dtype);
+    cudaStream_t s = S(stream);
+    if (sv.n_seg == 0) return BQ_OK;
+    if (mode == BQ_SCALE_DYNAMIC && sv.G == 0) {
+        return from_cuda(bq::empty_groups(sv.n_seg, cfg, scale, zp, s));
+    }
+    void* out = (op == bq::OP_QUANT) ? q : y;
+    if (mode == BQ_SCALE_STATIC) {
+        return from_cuda(bq::int_map(dt, op, bq::PS_STATIC, x, nullptr, sv, cfg, scale, zp,
+                                     nullptr, nullptr, nullptr, out, s));
+    }
+    if (mode == BQ_SCALE_FROM_RANGE) {
+        return from_cuda(bq::int_map(dt, op, bq::PS_RANGE, x, nullptr, sv, cfg, nullptr, nullptr,
+                                     (const unsigned long long*)ws, scale, zp, out, s));
+    }
+    // Dynamic: one pass when a register-resident configuration covers the group.
+    cudaError_t e = bq::int_dyn(dt, op, x, sv, cfg, q, y, scale, zp, s);
+    if (e != cudaErrorNotSupported) return from_cuda(e);
+    if (!ws || ws_bytes < need_ranges) {
+        return single_pass_possible(d, sv) ? BQ_ERR_MISALIGNED : BQ_ERR_INVALID_ARG;
+    }
+    if (!aligned(ws, 8)) return BQ_ERR_MISALIGNED;
+    unsigned long long* ranges = (unsigned long long*)ws;
+    if (cudaMemsetAsync(ranges, 0, need_ranges, s) != cudaSuccess) return BQ_ERR_CUDA;
+    e = (sv.n_seg == 1) ? bq::tensor_range(dt, x, sv.numel, cfg.symmetric, ranges, s)
+                        : bq::seg_range(dt, x, sv, cfg.symmetric, ranges, s);
+    if (e != cudaSuccess) return BQ_ERR_CUDA;
+    return from_cuda(bq::int_map(dt, op, bq::PS_RANGE, x, nullptr, sv, cfg, nullptr, nullptr,
+                                 ranges, scale, zp, out, s));
+}
+
+bq_status dequant_impl(const void* q, const float* scale, const void* zp, const bq_qdesc* d,
+                       int gr, int32_t axis, int64_t gs, void* y, bq_dtype y_dtype,
+                       void* stream) {
+    Layout lay;
+    bq_status st = make_layout(d, gr, axis, gs, &lay);
+    if (st != BQ_OK) return st;
+    bq::IntCfg cfg;
+    if ((st = make_cfg(d, false, &cfg)) != BQ_OK) return st;
+    if (!is_float(y_dtype)) return BQ_ERR_UNSUPPORTED;
+    cfg.symmetric = zp ? 0 : 1;                 // dequantize uses zp whenever it is given
+    const bq::SegView sv = lay.sv;
+    if (sv.numel == 0) return BQ_OK;
+    if (!q || !scale || !y) return BQ_ERR_INVALID_ARG;
+    if (!aligned(scale, 4) || !aligned(y, esize(y_dtype))) return BQ_ERR_MISALIGNED;
+    return from_cuda(bq::int_map(to_dt(y_dtype), bq::OP_DEQ, bq::PS_STATIC, q, nullptr, sv, cfg,
+                                 scale, zp, nullptr, nullptr, nullptr, y, S(stream)));
+}
+
+// Straight-Through Estimator backwards (quantize: op QBWD, fake: op FBWD).
+bq_status ste_impl(int op, const void* x, const void* dy, const float* scale, const void* zp,
+                   const bq_qdesc* d, int gr, int32_t axis, int64_t gs, void* dx, void* stream) {
+    Layout lay;
+    bq_status st = make_layout(d, gr, axis, gs, &lay);
+    if (st != BQ_OK) return st;
+    bq::IntCfg cfg;
+    if ((st = make_cfg(d, true, &cfg)) != BQ_OK) return st;
+    const bq::SegView sv = lay.sv;
+    if (sv.numel == 0) return BQ_OK;
+    if (!x || !dy || !scale || !dx) return BQ_ERR_INVALID_ARG;
+    if (!cfg.symmetric && !zp) return BQ_ERR_INVALID_ARG;
+    const int64_t es = esize(d->x_dtype);
+    if (!aligned(x, es) || !aligned(dy, es) || !aligned(dx, es) || !aligned(scale, 4))
+        return BQ_ERR_MISALIGNED;
+    return from_cuda(bq::int_map(to_dt(d->x_dtype), op, bq::PS_STATIC, x, dy, sv, cfg, scale, zp,
+                                 nullptr, nullptr, nullptr, dx, S(stream)));
+}
+
+bq_status dequant_bwd_impl(const void* dy, const float* scale, const bq_qdesc* d, int gr,
+                           int32_t axis, int64_t gs, void* dq, void* stream) {
+    Layout lay;
+    bq_status st = make_layout(d, gr, axis, gs, &lay);
+    if (st != BQ_OK) return st;
+    if (!is_float(d->x_dtype)) return BQ_ERR_UNSUPPORTED;
+    bq::IntCfg cfg{-128, 127, 1, 0, 1};
+    const bq::SegView sv = lay.sv;
+    if (sv.numel == 0) return BQ_OK;
+    if (!dy || !scale || !dq) return BQ_ERR_INVALID_ARG;
+    const int64_t es = esize(d->x_dtype);
+    if (!aligned(dy, es) || !aligned(dq, es) || !aligned(scale, 4)) return BQ_ERR_MISALIGNED;
+    return from_cuda(bq::int_map(to_dt(d->x_dtype), bq::OP_DBWD, bq::PS_STATIC, dy, nullptr, sv,
+                                 cfg, scale, nullptr, nullptr, nullptr, nullptr, dq, S(stream)));
+}
+
+int gran_to_gr(bq_gran g) {
+    switch (g) {
+        case BQ_GRAN_TENSOR: return GR_TENSOR;
+        case BQ_GRAN_CHANNEL: return GR_CHANNEL;
+        case BQ_GRAN_GROUP: return GR_GROUP;
+    }
+    return -1;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* bq_status_string(bq_status s) {
+    switch (s) {
+        case BQ_OK: return "ok";
+        case BQ_ERR_INVALID_ARG: return "invalid argument";
+        case BQ_ERR_UNSUPPORTED: return "unsupported dtype or mode";
+        case BQ_ERR_MISALIGNED: return "misaligned pointer";
+        case BQ_ERR_CUDA: return "CUDA launch error";
+        case BQ_ERR_TIMEOUT: return "timeout";
+    }
+    return "unknown status";
+}
+
+const char* bq_granularity_name(bq_gran g) {
+    switch (g) {
+        case BQ_GRAN_TENSOR: return "tensor";
+        case BQ_GRAN_CHANNEL: return "channel";
+        case BQ_GRAN_GROUP: return "group";
+    }
+    return nullptr;
+}
+
+bq_status bq_default_q_range(bq_dtype q_dtype, int32_t* qmin, int32_t* qmax) {
+    if (!qmin || !qmax) return BQ_ERR_INVALID_ARG;
+    if (q_dtype == BQ_S8) { *qmin = -128; *qmax = 127; return BQ_OK; }
+    if (q_dtype == BQ_U8) { *qmin = 0; *qmax = 255; return BQ_OK; }
+    return BQ_ERR_UNSUPPORTED;
+}
+
+bq_status bq_group_count(const bq_qdesc* d, bq_gran gran, int32_t axis, int64_t group_size,
+                         int64_t* n_groups, int64_t* group_elems) {
+    const int gr = gran_to_gr(gran);
+    if (gr < 0 || !n_groups || !group_elems) return BQ_ERR_INVALID_ARG;
+    Layout lay;
+    bq_status st = make_layout(d, gr, axis, group_size, &lay);
+    if (st != BQ_OK) return st;
+    *n_groups = lay.sv.n_seg;
+    *group_elems = lay.sv.G;
+    return BQ_OK;
+}
+
+size_t bq_quantize_workspace_size(const bq_qdesc* d, bq_gran gran, int32_t axis,
+                                  int64_t group_size, bq_scale_mode mode) {
+    const int gr = gran_to_gr(gran);
+    Layout lay;
+    if (gr < 0 || make_layout(d, gr, axis, group_size, &lay) != BQ_OK) return 0;
+    if (mode == BQ_SCALE_STATIC) return 0;
+    if (mode == BQ_SCALE_FROM_RANGE) return (size_t)lay.sv.n_seg * 16;
+    return single_pass_possible(d, lay.sv) ? 0 : (size_t)lay.sv.n_seg * 16;
+}
+
+bq_status bq_group_range(const void* x, const bq_qdesc* d, bq_gran gran, int32_t axis,
+                         int64_t group_size, void* ranges, void* stream) {
+    const int gr = gran_to_gr(gran);
+    if (gr < 0) return BQ_ERR_INVALID_ARG;
+    Layout lay;
+    bq_status st = make_layout(d, gr, axis, group_size, &lay);
+    if (st != BQ_OK) return st;
+    if (!is_float(d->x_dtype)) return BQ_ERR_UNSUPPORTED;
+    const bq::SegView sv = lay.sv;
+    if (sv.n_seg == 0) return BQ_OK;
+    if (!ranges || (sv.numel > 0 && !x)) return BQ_ERR_INVALID_ARG;
+    if (!aligned(ranges, 8) || !aligned(x, esize(d->x_dtype))) return BQ_ERR_MISALIGNED;
+    cudaStream_t s = S(stream);
+    if (cudaMemsetAsync(ranges, 0, (size_t)sv.n_seg * 16, s) != cudaSuccess) return BQ_ERR_CUDA;
+    // Both slots are always filled, so the records serve either scaling.
+    cudaError_t e = (sv.n_seg == 1)
+        ? bq::tensor_range(to_dt(d->x_dtype), x, sv.numel, false, (unsigned long long*)ranges, s)
+        : bq::seg_range(to_dt(d->x_dtype), x, sv, false, (unsigned long long*)ranges, s);
+    return from_cuda(e);
+}
+
+bq_status bq_tensor_amax(const void* x, bq_dtype dtype, int64_t n, float* amax, void* ws,
+                         void* stream) {
+    if (!is_half_or_f32(dtype)) return BQ_ERR_UNSUPPORTED;
+    if (n < 0 || !amax || !ws || (n > 0 && !x)) return BQ_ERR_INVALID_ARG;
+    if (!aligned(ws, 8) || !aligned(amax, 4) || !aligned(x, esize(dtype))) return BQ_ERR_MISALIGNED;
+    cudaStream_t s = S(stream);
+    if (cudaMemsetAsync(ws, 0, 16, s) != cudaSuccess) return BQ_ERR_CUDA;
+    cudaError_t e = bq::tensor_range(to_dt(dtype), x, n, true, (unsigned long long*)ws, s);
+    if (e != cudaSuccess) return BQ_ERR_CUDA;
+    return from_cuda(bq::range_to_amax((const unsigned long long*)ws, amax, s));
+}
+
+// ---- quantize
+bq_status bq_quantize_per_tensor(const void* x, const bq_qdesc* d, void* q, float* scale,
+                                 void* zp, bq_scale_mode mode, void* ws, size_t ws_bytes,
+                                 void* stream) {
+    return quant_impl(bq::OP_QUANT, x, d, GR_TENSOR, 0, 1, q, scale, zp, mode, nullptr, ws,
+                      ws_bytes, stream);
+}
+bq_status bq_quantize_per_channel(const void* x, const bq_qdesc* d, int32_t axis, void* q,
+                                  float* scale, void* zp, bq_scale_mode mode, void* ws,
+                                  size_t ws_bytes, void* stream) {
+    return quant_impl(bq::OP_QUANT, x, d, GR_CHANNEL, axis, 1, q, scale, zp, mode, nullptr, ws,
+                      ws_bytes, stream);
+}
+bq_status bq_quantize_per_token(const void* x, const bq_qdesc* d, void* q, float* scale,
+                                void* zp, bq_scale_mode mode, void* ws, size_t ws_bytes,
+                                void* stream) {
+    return quant_impl(bq::OP_QUANT, x, d, GR_TOKEN, 0, 1, q, scale, zp, mode, nullptr, ws,
+                      ws_bytes, stream);
+}
+bq_status bq_quantize_per_group(const void* x, const bq_qdesc* d, int32_t axis,
+                                int64_t group_size, void* q, float* scale, void* zp,
+                                bq_scale_mode mode, void* ws, size_t ws_bytes, void* stream) {
+    return quant_impl(bq::OP_QUANT, x, d, GR_GROUP, axis, group_size, q, scale, zp, mode,
+                      nullptr, ws, ws_bytes, stream);
+}
+
+// ---- dequantize
+bq_status bq_dequantize_per_tensor(const void* q, const float* scale, const void* zp,
+                                   const bq_qdesc* d, void* y, bq_dtype y_dtype, void* stream) {
+    return dequant_impl(q, scale, zp, d, GR_TENSOR, 0, 1, y, y_dtype, stream);
+}
+bq_status bq_dequantize_per_channel(const void* q, const float* scale, const void* zp,
+                                    const bq_qdesc* d, int32_t axis, void* y, bq_dtype y_dtype,
+                                    void* stream) {
+    return dequant_impl(q, scale, zp, d, GR_CHANNEL, axis, 1, y, y_dtype, stream);
+}
+bq_status bq_dequantize_per_token(const void* q, const float* scale, const void* zp,
+                                  const bq_qdesc* d, void* y, bq_dtype y_dtype, void* stream) {
+    return dequant_impl(q, scale, zp, d, GR_TOKEN, 0, 1, y, y_dtype, stream);
+}
+bq_status bq_dequantize_per_group(const void* q, const float* scale, const void* zp,
+                                  const bq_qdesc* d, int32_t axis, int64_t group_size, void* y,
+                                  bq_dtype y_dtype, void* stream) {
+    return dequant_impl(q, scale, zp, d, GR_GROUP, axis, group_size, y, y_dtype, stream);
+}
+
+// ---- fake quantize
+bq_status bq_fake_quantize(const void* x, const bq_qdesc* d, bq_gran gran, int32_t axis,
+                           int64_t group_size, float* scale, void* zp, bq_scale_mode mode,
+                           void* y, void* ws, size_t ws_bytes, void* stream) {
+    const int gr = gran_to_gr(gran);
+    if (gr < 0) return BQ_ERR_INVALID_ARG;
+    return quant_impl(bq::OP_FAKE, x, d, gr, axis, group_size, nullptr, scale, zp, mode, y, ws,
+                      ws_bytes, stream);
+}
+
+// ---- backwards
+bq_status bq_quantize_per_tensor_backward(const void* x, const void* dy, const float* scale,
+                                          const void* zp, const bq_qdesc* d, void* dx,
+                                          void* stream) {
+    return ste_impl(bq::OP_QBWD, x, dy, scale, zp, d, GR_TENSOR, 0, 1, dx, stream);
+}
+bq_status bq_quantize_per_channel_backward(const void* x, const void* dy, const float* scale,
+                                           const void* zp, const bq_qdesc* d, int32_t axis,
+                                           void* dx, void* stream) {
+    return ste_impl(bq::OP_QBWD, x, dy, scale, zp, d, GR_CHANNEL, axis, 1, dx, stream);
+}
+bq_status bq_quantize_per_token_backward(const void* x, const void* dy, const float* scale,
+                                         const void* zp, const bq_qdesc* d, void* dx,
+                                         void* stream) {
+    return ste_impl(bq::OP_QBWD, x, dy, scale, zp, d, GR_TOKEN, 0, 1, dx, stream);
+}
+bq_status bq_quantize_per_group_backward(const void* x, const void* dy, const float* scale,
+                                         const void* zp, const bq_qdesc* d, int32_t axis,
+                                         int64_t group_size, void* dx, void* stream) {
+    return ste_impl(bq::OP_QBWD, x, dy, scale, zp, d, GR_GROUP, axis, group_size, dx, stream);
+}
+bq_status bq_fake_quantize_backward(const void* x, const void* dy, const float* scale,
+                                    const void* zp, const bq_qdesc* d, bq_gran gran,
+                                    int32_t axis, int64_t group_size, void* dx, void* stream) {
+    const int gr = gran_to_gr(gran);
+    if (gr < 0) return BQ_ERR_INVALID_ARG;
+    return ste_impl(bq::OP_FBWD, x, dy, scale, zp, d, gr, axis, group_size, dx, stream);
+}
+
+bq_status bq_dequantize_per_tensor_backward(const void* dy, const float* scale,
+                                            const bq_qdesc* d, void* dq, void* stream) {
+    return dequant_bwd_impl(dy, scale, d, GR_TENSOR, 0, 1, dq, stream);
+}
+bq_status bq_dequantize_per_channel_backward(const void* dy, const float* scale,
+                                             const bq_qdesc* d, int32_t axis, void* dq,
+                                             void* stream) {
+    return dequant_bwd_impl(dy, scale, d, GR_CHANNEL, axis, 1, dq, stream);
+}
+bq_status bq_dequantize_per_token_backward(const void* dy, const float* scale,
+                                           const bq_qdesc* d, void* dq, void* stream) {
+    return dequant_bwd_impl(dy, scale, d, GR_TOKEN, 0, 1, dq, stream);
+}
+bq_status bq_dequantize_per_group_backward(const void* dy, const float* scale,
+                                           const bq_qdesc* d, int32_t axis, int64_t group_size,
+                                           void* dq, void* stream) {
+    return dequant_bwd_impl(dy, scale, d, GR_GROUP, axis, group_size, dq, stream);
+}
+
+// ---- NVFP4
+bq_status bq_nvfp4_quantize(const void* x, bq_dtype x_dtype, int64_t n, int64_t k,
+                            uint8_t* packed, uint8_t* scale_e4m3, float* global_scale,
+                            int32_t static_global, void* ws, size_t ws_bytes, void* stream) {
+    if (!is_half_or_f32(x_dtype)) return BQ_ERR_UNSUPPORTED;
+    if (n < 0 || k < 0 || k % 16 != 0) return BQ_ERR_INVALID_ARG;
+    if (!global_scale) return BQ_ERR_INVALID_ARG;
+    if (!static_global && (!ws || ws_bytes < 16)) return BQ_ERR_INVALID_ARG;
+    if (n * k > 0 && (!x || !packed || !scale_e4m3)) return BQ_ERR_INVALID_ARG;
+    if (!aligned(x, esize(x_dtype)) || !aligned(global_scale, 4) || (!static_global && !aligned(ws, 8)))
+        return BQ_ERR_MISALIGNED;
+    cudaStream_t s = S(stream);
+    const DT dt = to_dt(x_dtype);
+    unsigned long long* rec = (unsigned long long*)ws;
+    if (!static_global) {
+        if (cudaMemsetAsync(rec, 0, 16, s) != cudaSuccess) return BQ_ERR_CUDA;
+        if (n * k == 0) return from_cuda(bq::set_f32(global_scale, 1.0f, s));   // zero range
+        if (bq::tensor_range(dt, x, n * k, true, rec, s) != cudaSuccess) return BQ_ERR_CUDA;
+    }
+    if (n * k == 0) return BQ_OK;
+    return from_cuda(bq::mx_quant(dt, bq::MX_NVFP4, x, n, k, packed, scale_e4m3, rec, global_scale,
+                                  static_global ? 1 : 0, s));
+}
+
+bq_status bq_nvfp4_dequantize(const uint8_t* packed, const uint8_t* scale_e4m3,
+                              const float* global_scale, int64_t n, int64_t k, void* y,
+                              bq_dtype y_dtype, void* stream) {
+    if (!is_half_or_f32(y_dtype)) return BQ_ERR_UNSUPPORTED;
+    if (n < 0 || k < 0 || k % 16 != 0) return BQ_ERR_INVALID_ARG;
+    if (n * k == 0) return BQ_OK;
+    if (!packed || !scale_e4m3 || !global_scale || !y) return BQ_ERR_INVALID_ARG;
+    if (!aligned(global_scale, 4) || !aligned(y, esize(y_dtype))) return BQ_ERR_MISALIGNED;
+    return from_cuda(bq::mx_dequant(to_dt(y_dtype), bq::MX_NVFP4, packed, scale_e4m3,
+                                    global_scale, n, k, y, S(stream)));
+}
+
+// ---- MXFP8
+bq_status bq_mxfp8_quantize(const void* x, bq_dtype x_dtype, int64_t rows, int64_t k,
+                            uint8_t* e4m3, uint8_t* e8m0, void* stream) {
+    if (!is_half_or_f32(x_dtype)) return BQ_ERR_UNSUPPORTED;
+    if (rows < 0 || k < 0 || k % 32 != 0) return BQ_ERR_INVALID_ARG;
+    if (rows * k == 0) return BQ_OK;
+    if (!x || !e4m3 || !e8m0) return BQ_ERR_INVALID_ARG;
+    if (!aligned(x, esize(x_dtype))) return BQ_ERR_MISALIGNED;
+    return from_cuda(bq::mx_quant(to_dt(x_dtype), bq::MX_MXFP8, x, rows, k, e4m3, e8m0, nullptr,
+                                  nullptr, 0, S(stream)));
+}
+
+bq_status bq_mxfp8_dequantize(const uint8_t* e4m3, const uint8_t* e8m0, int64_t rows, int64_t k,
+                              void* y, bq_dtype y_dtype, void* stream) {
+    if (!is_half_or_f32(y_dtype)) return BQ_ERR_UNSUPPORTED;
+    if (rows < 0 || k < 0 || k % 32 != 0) return BQ_ERR_INVALID_ARG;
+    if (rows * k == 0) return BQ_OK;
+    if (!e4m3 || !e8m0 || !y) return BQ_ERR_INVALID_ARG;
+    if (!aligned(y, esize(y_dtype))) return BQ_ERR_MISALIGNED;
+    return from_cuda(bq::mx_dequant(to_dt(y_dtype), bq::MX_MXFP8, e4m3, e8m0, nullptr, rows, k, y,
+                                    S(stream)));
+}
+
+// ---- FP8 blocks
+bq_status bq_fp8_block_quantize(const void* x, bq_dtype x_dtype, int64_t rows, int64_t cols,
+                                int32_t block_rows, int32_t block_cols, uint8_t* e4m3,
+                                float* scale, void* stream) {
+    if (!is_half_or_f32(x_dtype)) return BQ_ERR_UNSUPPORTED;
+    if (rows < 0 || cols < 0) return BQ_ERR_INVALID_ARG;
+    if (block_cols != 128 || (block_rows != 1 && block_rows != 128)) return BQ_ERR_UNSUPPORTED;
+    if (rows * cols == 0) return BQ_OK;
+    if (!x || !e4m3 || !scale) return BQ_ERR_INVALID_ARG;
+    if (!aligned(x, esize(x_dtype)) || !aligned(scale, 4)) return BQ_ERR_MISALIGNED;
+    const DT dt = to_dt(x_dtype);
+    cudaStream_t s = S(stream);
+    if (block_rows == 1 && cols % 128 == 0 && aligned(x, 16))
+        return from_cuda(bq::mx_quant(dt, bq::MX_FP8_1x128, x, rows, cols, e4m3, scale, nullptr,
+                                      nullptr, 0, s));
+    return from_cuda(bq::fp8_tile_quant(dt, x, rows, cols, block_rows, block_cols, e4m3, scale, s));
+}
+
+bq_status bq_fp8_block_dequantize(const uint8_t* e4m3, const float* scale, int64_t rows,
+                                  int64_t cols, int32_t block_rows, int32_t block_cols, void* y,
+                                  bq_dtype y_dtype, void* stream) {
+    if (!is_half_or_f32(y_dtype)) return BQ_ERR_UNSUPPORTED;
+    if (rows < 0 || cols < 0) return BQ_ERR_INVALID_ARG;
+    if (block_cols != 128 || (block_rows != 1 && block_rows != 128)) return BQ_ERR_UNSUPPORTED;
+    if (rows * cols == 0) return BQ_OK;
+    if (!e4m3 || !scale || !y) return BQ_ERR_INVALID_ARG;
+    if (!aligned(scale, 4) || !aligned(y, esize(y_dtype))) return BQ_ERR_MISALIGNED;
+    return from_cuda(bq::fp8_block_dequant(to_dt(y_dtype), e4m3, scale, rows, cols, block_rows,
+                                           block_cols, y, S(stream)));
+}
+
+// ---- packed transpose
+int64_t bq_packed_transpose_stride(int64_t n, int64_t align) {
+    if (n < 0 || align < 1) return -1;
+    if (n > INT64_MAX - (align - 1)) return -1;
+    return (n + align - 1) / align * align;
+}
+
+bq_status bq_packed_transpose(const uint8_t* w, const uint8_t* sc, int64_t n, int64_t k,
+                              int64_t group_size, int64_t align, uint8_t* w_t, uint8_t* sc_t,
+                              int64_t* out_stride, void* stream) {
+    if (n < 0 || k < 0 || align < 1 || k % 2 != 0) return BQ_ERR_INVALID_ARG;
+    if ((sc == nullptr) != (sc_t == nullptr)) return BQ_ERR_INVALID_ARG;
+    if (sc && (group_size < 1 || k % group_size != 0)) return BQ_ERR_INVALID_ARG;
+    const int64_t stride = bq_packed_transpose_stride(n, align);
+    if (stride < 0) return BQ_ERR_INVALID_ARG;
+    if (out_stride) *out_stride = stride;
+    if (k == 0 || stride == 0) return BQ_OK;
+    if (!w_t || (n > 0 && !w)) return BQ_ERR_INVALID_ARG;
+    cudaStream_t s = S(stream);
+    if (bq::byte_transpose(w, n, k / 2, stride, w_t, s) != cudaSuccess) return BQ_ERR_CUDA;
+    if (sc) return from_cuda(bq::byte_transpose(sc, n, k / group_size, stride, sc_t, s));
+    return BQ_OK;
+}
+
+}  // extern "C"

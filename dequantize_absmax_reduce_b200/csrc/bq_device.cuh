@@ -1,0 +1,333 @@
+// Device helpers shared by the bq kernels: element types, 16-byte memory
+// access, correctly rounded division, integer-code rounding and the FP8 / FP4
+// encoders. sm_100a only.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include <type_traits>
+
+namespace bq {
+
+// ---------------------------------------------------------------- elements
+// Acc is the arithmetic type: f32 for f32/f16/bf16 storage, f64 for f64.
+template <class T> struct Traits;
+template <> struct Traits<float>          { using Acc = float;  static constexpr int VEC = 4; };
+template <> struct Traits<__half>         { using Acc = float;  static constexpr int VEC = 8; };
+template <> struct Traits<__nv_bfloat16>  { using Acc = float;  static constexpr int VEC = 8; };
+template <> struct Traits<double>         { using Acc = double; static constexpr int VEC = 2; };
+
+struct alignas(16) U4 { uint32_t x, y, z, w; };
+
+// Streaming 16-byte load: read once, keep it out of L1.
+__device__ __forceinline__ U4 ld16_stream(const void* p) {
+    U4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
+__device__ __forceinline__ void st16(void* p, const U4& v) {
+    asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};"
+                 :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+__device__ __forceinline__ void st8(void* p, uint32_t a, uint32_t b) {
+    asm volatile("st.global.v2.u32 [%0], {%1,%2};" :: "l"(p), "r"(a), "r"(b) : "memory");
+}
+__device__ __forceinline__ void st4(void* p, uint32_t a) {
+    asm volatile("st.global.u32 [%0], %1;" :: "l"(p), "r"(a) : "memory");
+}
+
+// Unpack one 16-byte vector into VEC arithmetic values (exact widening).
+__device__ __forceinline__ void unpack(const U4& u, float (&v)[4]) {
+    v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y);
+    v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
+}
+__device__ __forceinline__ void unpack_bf16x2(uint32_t w, float& lo, float& hi) {
+    lo = __uint_as_float(w << 16);
+    hi = __uint_as_float(w & 0xFFFF0000u);
+}
+__device__ __forceinline__ void unpack_f16x2(uint32_t w, float& lo, float& hi) {
+    __half2 h = *reinterpret_cast<__half2*>(&w);
+    float2 f = __half22float2(h);
+    lo = f.x; hi = f.y;
+}
+template <class T> __device__ __forceinline__ void unpack8(const U4& u, float (&v)[8]);
+template <> __device__ __forceinline__ void unpack8<__nv_bfloat16>(const U4& u, float (&v)[8]) {
+    unpack_bf16x2(u.x, v[0], v[1]); unpack_bf16x2(u.y, v[2], v[3]);
+    unpack_bf16x2(u.z, v[4], v[5]); unpack_bf16x2(u.w, v[6], v[7]);
+}
+template <> __device__ __forceinline__ void unpack8<__half>(const U4& u, float (&v)[8]) {
+    unpack_f16x2(u.x, v[0], v[1]); unpack_f16x2(u.y, v[2], v[3]);
+    unpack_f16x2(u.z, v[4], v[5]); unpack_f16x2(u.w, v[6], v[7]);
+}
+__device__ __forceinline__ void unpack(const U4& u, double (&v)[2]) {
+    v[0] = __hiloint2double((int)u.y, (int)u.x);
+    v[1] = __hiloint2double((int)u.w, (int)u.z);
+}
+
+// Generic: VEC values from one 16-byte vector.
+template <class T>
+__device__ __forceinline__ void load_vec(const U4& u, typename Traits<T>::Acc (&v)[Traits<T>::VEC]) {
+    if constexpr (sizeof(T) == 2) unpack8<T>(u, v); else unpack(u, v);
+}
+
+// Scalar element load / store with round-to-nearest-even narrowing.
+template <class T> __device__ __forceinline__ typename Traits<T>::Acc ld1(const T* p);
+template <> __device__ __forceinline__ float ld1<float>(const float* p) { return __ldg(p); }
+template <> __device__ __forceinline__ double ld1<double>(const double* p) { return __ldg(p); }
+template <> __device__ __forceinline__ float ld1<__half>(const __half* p) {
+    return __half2float(__ldg(p));
+}
+template <> __device__ __forceinline__ float ld1<__nv_bfloat16>(const __nv_bfloat16* p) {
+    unsigned short b = __ldg(reinterpret_cast<const unsigned short*>(p));
+    return __uint_as_float(((uint32_t)b) << 16);
+}
+
+template <class T> __device__ __forceinline__ T to_out(typename Traits<T>::Acc v);
+template <> __device__ __forceinline__ float to_out<float>(float v) { return v; }
+template <> __device__ __forceinline__ double to_out<double>(double v) { return v; }
+template <> __device__ __forceinline__ __half to_out<__half>(float v) { return __float2half_rn(v); }
+template <> __device__ __forceinline__ __nv_bfloat16 to_out<__nv_bfloat16>(float v) {
+    return __float2bfloat16_rn(v);
+}
+
+// Pack VEC arithmetic values into one 16-byte vector of T (RNE narrowing).
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+template <class T>
+__device__ __forceinline__ U4 pack_vec(const typename Traits<T>::Acc (&v)[Traits<T>::VEC]) {
+    U4 u;
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        u.x = pack_bf16x2(v[0], v[1]); u.y = pack_bf16x2(v[2], v[3]);
+        u.z = pack_bf16x2(v[4], v[5]); u.w = pack_bf16x2(v[6], v[7]);
+    } else if constexpr (std::is_same<T, __half>::value) {
+        u.x = pack_f16x2(v[0], v[1]); u.y = pack_f16x2(v[2], v[3]);
+        u.z = pack_f16x2(v[4], v[5]); u.w = pack_f16x2(v[6], v[7]);
+    } else if constexpr (std::is_same<T, float>::value) {
+        u.x = __float_as_uint(v[0]); u.y = __float_as_uint(v[1]);
+        u.z = __float_as_uint(v[2]); u.w = __float_as_uint(v[3]);
+    } else {
+        u.x = (uint32_t)__double2loint(v[0]); u.y = (uint32_t)__double2hiint(v[0]);
+        u.z = (uint32_t)__double2loint(v[1]); u.w = (uint32_t)__double2hiint(v[1]);
+    }
+    return u;
+}
+
+// ---------------------------------------------------------------- division
+// fl(x / s) for a per-group divisor s, correctly rounded, from the correctly
+// rounded reciprocal y = RN(1/s) and two remainder corrections:
+//   q0 = RN(x*y); q1 = RN(q0 + RN(x - s*q0)*y)  -> within one ulp of x/s;
+//   q2 = RN(q1 + (x - s*q1)*y)                  -> RN(x/s)
+// The last step is Markstein's theorem (P. Markstein, IBM J. Res. Dev. 34(1),
+// 1990; Muller et al., Handbook of Floating-Point Arithmetic, ch. 4): with y
+// within half an ulp of 1/s and q1 within one ulp of x/s, the remainder
+// x - s*q1 is exact in an FMA and RN(q1 + r*y) = RN(x/s). The hypotheses
+// need no overflow and a remainder above the subnormal range; `fast` holds
+// when 2^-64 <= |s| <= 2^64, which covers every quotient that can decide a
+// code (|x/s| >= 2^-12 needs |x| >= 2^-76). Outside that range, and for
+// x/s that overflow (only possible when x is not bounded by the group range),
+// callers use the IEEE division __fdiv_rn.
+struct Recip {
+    float s, y;
+    bool fast;
+};
+__device__ __forceinline__ Recip make_recip(float s) {
+    Recip r;
+    r.s = s;
+    r.y = __frcp_rn(s);
+    const float a = fabsf(s);
+    r.fast = (a >= 0x1p-64f) && (a <= 0x1p64f);
+    return r;
+}
+// Correct when r.fast and |x| is bounded by the group range (no overflow).
+__device__ __forceinline__ float div_chain(float x, const Recip& r) {
+    const float q0 = __fmul_rn(x, r.y);
+    const float e0 = __fmaf_rn(-r.s, q0, x);
+    const float q1 = __fmaf_rn(e0, r.y, q0);
+    const float e1 = __fmaf_rn(-r.s, q1, x);
+    return __fmaf_rn(e1, r.y, q1);
+}
+// Any x: falls back to IEEE division when the chain produced a NaN
+// (an infinite or overflowing operand); a NaN x stays NaN either way.
+__device__ __forceinline__ float div_any(float x, const Recip& r) {
+    if (!r.fast) return __fdiv_rn(x, r.s);
+    float q = div_chain(x, r);
+    if (q != q) q = __fdiv_rn(x, r.s);
+    return q;
+}
+// Sign of a quotient of zero: x/s keeps the sign of x * s. The chain returns
+// +0 for x = -0; encoders that keep the sign of zero restore it here.
+__device__ __forceinline__ float with_quotient_sign(float q, float x, float s) {
+    return __uint_as_float((__float_as_uint(q) & 0x7FFFFFFFu) |
+                           ((__float_as_uint(x) ^ __float_as_uint(s)) & 0x80000000u));
+}
+
+// ---------------------------------------------------------------- int codes
+// Rounding v (an exact f32 quotient) to an integer code with nearest-even:
+// for |v| <= 2^22, fl(v + 1.5*2^23) has unit spacing, so the addition itself
+// rounds v to the nearest integer (ties to even) and the integer sits in the
+// low mantissa bits. Adding (1.5*2^23 + zp) instead puts (round(v) + zp) mod
+// 256 in the low byte.
+constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
+
+struct IntParams {
+    float lo, hi;      // code range shifted by the zero-point: qmin - zp, qmax - zp
+    float magic;       // kMagic + zp
+};
+__device__ __forceinline__ IntParams make_int_params(int qmin, int qmax, int zp) {
+    IntParams p;
+    p.lo = (float)(qmin - zp);
+    p.hi = (float)(qmax - zp);
+    p.magic = kMagic + (float)zp;
+    return p;
+}
+// Low byte = clamp(rne(v) + zp, qmin, qmax); a NaN v gives qmin.
+__device__ __forceinline__ uint32_t code_rne(float v, const IntParams& p) {
+    v = fminf(fmaxf(v, p.lo), p.hi);            // fmaxf(NaN, lo) = lo
+    return __float_as_uint(__fadd_rn(v, p.magic));
+}
+// Ties away from zero.
+__device__ __forceinline__ uint32_t code_rhaz(float v, const IntParams& p) {
+    v = fminf(fmaxf(v, p.lo), p.hi);
+    const float t = truncf(v);
+    const float d = __fsub_rn(v, t);             // exact
+    const float k = (fabsf(d) >= 0.5f) ? __fadd_rn(t, copysignf(1.0f, v)) : t;
+    return __float_as_uint(__fadd_rn(k, p.magic));
+}
+template <bool RHAZ>
+__device__ __forceinline__ uint32_t code_of(float v, const IntParams& p) {
+    if constexpr (RHAZ) return code_rhaz(v, p); else return code_rne(v, p);
+}
+// round(v) as a float, for the STE mask; v is clamped to [lo-1, hi+1] first
+// so that the result stays exact (a NaN v gives lo - 1: masked).
+template <bool RHAZ>
+__device__ __forceinline__ float round_for_mask(float v, const IntParams& p) {
+    v = fminf(fmaxf(v, p.lo - 1.0f), p.hi + 1.0f);
+    if constexpr (RHAZ) {
+        const float t = truncf(v);
+        const float d = __fsub_rn(v, t);
+        return (fabsf(d) >= 0.5f) ? __fadd_rn(t, copysignf(1.0f, v)) : t;
+    } else {
+        return __fsub_rn(__fadd_rn(v, kMagic), kMagic);
+    }
+}
+
+// f64 versions (f64 inputs): IEEE f64 division and rounding.
+__device__ __forceinline__ double round_rne_d(double v) { return rint(v); }
+__device__ __forceinline__ double round_rhaz_d(double v) { return round(v); }
+
+// Pack four low bytes into one word: byte i of the result = low byte of w[i].
+__device__ __forceinline__ uint32_t pack4_lowbytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    const uint32_t ab = __byte_perm(a, b, 0x0040);   // [a0, b0, a0, a0]
+    const uint32_t cd = __byte_perm(c, d, 0x0040);   // [c0, d0, ...]
+    return __byte_perm(ab, cd, 0x5410);              // [a0, b0, c0, d0]
+}
+
+// ---------------------------------------------------------------- FP8 / FP4
+// E4M3 (OCP FP8, max 448, no infinities), round to nearest even, saturating.
+// Two values per instruction; `lo` lands in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+    return e4m3x2(a, b) | (e4m3x2(c, d) << 16);
+}
+// E2M1 (OCP FP4), round to nearest even, saturating to +-6: eight values
+// into one word, value i in nibble i (low nibble first).
+__device__ __forceinline__ uint32_t e2m1x8(const float (&v)[8]) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+    return r;
+}
+// Decode two E4M3 bytes (low byte first) to f32 exactly (via f16, which
+// holds every E4M3 value).
+__device__ __forceinline__ float2 e4m3x2_to_f32(uint32_t two) {
+    uint32_t h;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"((uint16_t)two));
+    __half2 hh = *reinterpret_cast<__half2*>(&h);
+    return __half22float2(hh);
+}
+// Decode one byte of two E2M1 codes (low nibble first) to f32.
+__device__ __forceinline__ float2 e2m1x2_to_f32(uint32_t byte) {
+    uint32_t h;
+    asm("{\n\t.reg .b8 lo, hi;\n\t"
+        "mov.b16 {lo, hi}, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, lo;\n\t}"
+        : "=r"(h) : "h"((uint16_t)byte));
+    __half2 hh = *reinterpret_cast<__half2*>(&h);
+    return __half22float2(hh);
+}
+__device__ __forceinline__ float e4m3_to_f32(uint32_t byte) { return e4m3x2_to_f32(byte & 0xFF).x; }
+
+// 2^e as f32 for e in [-149, 127], exact.
+__device__ __forceinline__ float exp2i(int e) {
+    return (e >= -126) ? __uint_as_float((uint32_t)(e + 127) << 23)
+                       : __uint_as_float(1u << (e + 149));
+}
+
+// ---------------------------------------------------------------- reductions
+__device__ __forceinline__ float warp_max(float v, int width = 32) {
+    for (int o = width / 2; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o, width));
+    return v;
+}
+__device__ __forceinline__ double warp_max(double v, int width = 32) {
+    for (int o = width / 2; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o, width));
+    return v;
+}
+
+// Range record bits: IEEE bits of a non-negative value, zero-extended.
+__device__ __forceinline__ unsigned long long range_bits(float v) {
+    return (unsigned long long)__float_as_uint(v);
+}
+__device__ __forceinline__ unsigned long long range_bits(double v) {
+    return (unsigned long long)__double_as_longlong(v);
+}
+__device__ __forceinline__ void range_from_bits(unsigned long long b, float& v) {
+    v = __uint_as_float((uint32_t)b);
+}
+__device__ __forceinline__ void range_from_bits(unsigned long long b, double& v) {
+    v = __longlong_as_double((long long)b);
+}
+
+// ---------------------------------------------------------------- fast divide
+// Unsigned 32-bit division by a runtime-invariant d (Granlund & Montgomery,
+// "Division by invariant integers using multiplication", PLDI 1994, §4):
+// with l = ceil(log2 d) and m = floor(2^32 * (2^l - d) / d) + 1,
+// n / d = (t + ((n - t) >> 1)) >> (l - 1) where t = mulhi(m, n), for l >= 1.
+struct FastDiv {
+    uint32_t d, m, l;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+    FastDiv f;
+    f.d = d;
+    uint32_t l = 0;
+    while (l < 32 && (1ull << l) < d) ++l;
+    f.l = l;
+    f.m = (uint32_t)(((1ull << 32) * ((1ull << l) - d)) / d + 1);
+    return f;
+}
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
+    if (f.l == 0) return n;                      // d == 1
+    const uint32_t t = __umulhi(f.m, n);
+    return (t + ((n - t) >> 1)) >> (f.l - 1);
+}
+
+}  // namespace bq

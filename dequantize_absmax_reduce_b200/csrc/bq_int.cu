@@ -1,0 +1,814 @@
+// Integer (s8 / u8) quantize, dequantize, fake-quantize and Straight-Through
+// Estimator kernels for every granularity (baracuda_kernels::quantize module
+// index: per_tensor, per_channel, per_token, per_group and their backwards;
+// teenygrad granularity.rs for the groups).
+//
+// Every granularity reaches these kernels as a view of n_seg contiguous
+// groups of G elements: with x viewed as [outer, L, inner], Group{axis, gs}
+// holds axis indices [g*gs, (g+1)*gs) and every inner index, which is one
+// contiguous run of gs*inner elements.
+//
+// Kernels:
+//   k_int_dyn_warp / k_int_dyn_cta  one HBM pass for dynamic scales: a team
+//       of lanes (part of a warp, a warp, or a CTA) holds a whole group in
+//       registers, reduces its range, derives scale / zero-point and writes
+//       the codes. 16-byte streaming loads.
+//   k_int_map  element-wise with per-group parameters: static scales,
+//       scales derived from range records (second pass of the two-pass path),
+//       dequantize, and the three backwards.
+//   k_tensor_range / k_seg_range  range records (max(0, max x),
+//       max(0, -min x)) with integer atomicMax on the IEEE bits.
+#include <type_traits>
+
+#include "bq_device.cuh"
+#include "bq_internal.h"
+
+namespace bq {
+
+// ------------------------------------------------------------ group params
+struct GroupF { float s; int zp; };
+struct GroupD { float s; int zp; };
+
+// Scale and zero-point from a group's range (f32 arithmetic). Symmetric:
+// s = fl(amax / qmax). Asymmetric: s = fl(fl(max' - min') / (qmax - qmin)),
+// zp = clamp(qmin - round(fl(min' / s)), qmin, qmax). 0 -> 1.
+__device__ __forceinline__ GroupF derive_f(float hi, float nlo, const IntCfg& c) {
+    GroupF g;
+    if (c.symmetric) {
+        float s = __fdiv_rn(fmaxf(hi, nlo), (float)c.qmax);
+        if (s == 0.0f) s = 1.0f;
+        g.s = s;
+        g.zp = 0;
+    } else {
+        const float span = __fadd_rn(hi, nlo);
+        float s = __fdiv_rn(span, (float)(c.qmax - c.qmin));
+        if (s == 0.0f) s = 1.0f;
+        const float m = __fdiv_rn(-nlo, s);
+        const float r = c.rhaz ? roundf(m) : rintf(m);
+        float z = __fsub_rn((float)c.qmin, r);
+        z = fminf(fmaxf(z, (float)c.qmin), (float)c.qmax);   // NaN -> qmin
+        g.s = s;
+        g.zp = (int)z;
+    }
+    return g;
+}
+// Same in f64 for f64 inputs; the stored scale is still f32.
+__device__ __forceinline__ GroupD derive_d(double hi, double nlo, const IntCfg& c) {
+    GroupD g;
+    if (c.symmetric) {
+        float s = __double2float_rn(fmax(hi, nlo) / (double)c.qmax);
+        if (s == 0.0f) s = 1.0f;
+        g.s = s;
+        g.zp = 0;
+    } else {
+        const double span = hi + nlo;
+        float s = __double2float_rn(span / (double)(c.qmax - c.qmin));
+        if (s == 0.0f) s = 1.0f;
+        const double m = -nlo / (double)s;
+        const double r = c.rhaz ? round(m) : rint(m);
+        double z = (double)c.qmin - r;
+        z = fmin(fmax(z, (double)c.qmin), (double)c.qmax);
+        g.s = s;
+        g.zp = (int)z;
+    }
+    return g;
+}
+
+__device__ __forceinline__ int load_zp(const void* zp, int64_t g, int q_signed) {
+    if (!zp) return 0;
+    const uint8_t b = __ldg((const uint8_t*)zp + g);
+    return q_signed ? (int)(int8_t)b : (int)b;
+}
+
+// ------------------------------------------------------------ dynamic, warp
+struct DynArgs {
+    const void* x;
+    int64_t n_seg;
+    int G;          // elements per group (multiple of VEC)
+    int team;       // lanes per group when NV == 1 (power of two <= 32)
+    IntCfg cfg;
+    uint8_t* q;
+    void* y;
+    float* scale;
+    uint8_t* zp;
+};
+
+// One group's codes (and fake-quantized values) from its vectors. `lane_vec`
+// gives the element offset of vector j for this lane.
+template <class T, int OP, bool FAST>
+__device__ __forceinline__ void emit_vec(const U4& raw, const Recip& R, const IntParams& ip,
+                                         int64_t off, const DynArgs& a) {
+    constexpr int VEC = Traits<T>::VEC;
+    float v[VEC];
+    load_vec<T>(raw, v);
+    uint32_t cw[VEC];
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) {
+        const float qv = FAST ? div_chain(v[i], R) : __fdiv_rn(v[i], R.s);
+        cw[i] = code_rne(qv, ip);
+    }
+    if constexpr (OP == OP_QUANT) {
+        if constexpr (VEC == 8) {
+            st8(a.q + off, pack4_lowbytes(cw[0], cw[1], cw[2], cw[3]),
+                pack4_lowbytes(cw[4], cw[5], cw[6], cw[7]));
+        } else {
+            st4(a.q + off, pack4_lowbytes(cw[0], cw[1], cw[2], cw[3]));
+        }
+    } else {
+        float o[VEC];
+#pragma unroll
+        for (int i = 0; i < VEC; ++i)
+            o[i] = __fmul_rn(__fsub_rn(__uint_as_float(cw[i]), ip.magic), R.s);
+        st16((T*)a.y + off, pack_vec<T>(o));
+    }
+}
+
+template <class T>
+__device__ __forceinline__ void range_vec(const U4& raw, bool sym, float& hi, float& nlo) {
+    constexpr int VEC = Traits<T>::VEC;
+    float v[VEC];
+    load_vec<T>(raw, v);
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) {
+        if (sym) {
+            hi = fmaxf(hi, fabsf(v[i]));
+        } else {
+            hi = fmaxf(hi, v[i]);
+            nlo = fmaxf(nlo, -v[i]);
+        }
+    }
+}
+
+// NV vectors per lane; NV == 1 allows teams of `a.team` lanes, NV > 1 uses
+// whole warps. SEGS groups per team per iteration keep several loads in
+// flight when groups are small.
+template <class T, int OP, int NV, int SEGS, bool SYM>
+__global__ void __launch_bounds__(256) k_int_dyn_warp(DynArgs a) {
+    constexpr int VEC = Traits<T>::VEC;
+    const T* __restrict__ x = (const T*)a.x;
+    const int team = (NV == 1) ? a.team : 32;
+    const int tpw = 32 / team;
+    const int lane = threadIdx.x & 31;
+    const int tm = lane / team;
+    const int l = lane % team;
+    const int64_t gwarp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t per_chunk = (int64_t)SEGS * tpw;
+    const int64_t n_chunks = (a.n_seg + per_chunk - 1) / per_chunk;
+
+    for (int64_t c = gwarp; c < n_chunks; c += nwarps) {
+        U4 raw[SEGS][NV];
+#pragma unroll
+        for (int r = 0; r < SEGS; ++r) {
+            const int64_t seg = c * per_chunk + (int64_t)r * tpw + tm;
+#pragma unroll
+            for (int j = 0; j < NV; ++j) {
+                const int e = (j * team + l) * VEC;
+                if (seg < a.n_seg && e < a.G) raw[r][j] = ld16_stream(x + seg * a.G + e);
+                else raw[r][j] = U4{0u, 0u, 0u, 0u};
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < SEGS; ++r) {
+            const int64_t seg = c * per_chunk + (int64_t)r * tpw + tm;
+            float hi = 0.0f, nlo = 0.0f;
+#pragma unroll
+            for (int j = 0; j < NV; ++j) range_vec<T>(raw[r][j], SYM, hi, nlo);
+            for (int o = team / 2; o > 0; o >>= 1) {
+                hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+                if (!SYM) nlo = fmaxf(nlo, __shfl_xor_sync(0xffffffffu, nlo, o));
+            }
+            const GroupF g = derive_f(hi, nlo, a.cfg);
+            const bool seg_ok = seg < a.n_seg;
+            if (seg_ok && l == 0) {
+                a.scale[seg] = g.s;
+                if (a.zp) a.zp[seg] = (uint8_t)g.zp;
+            }
+            const IntParams ip = make_int_params(a.cfg.qmin, a.cfg.qmax, g.zp);
+            const Recip R = make_recip(g.s);
+            if (R.fast) {
+#pragma unroll
+                for (int j = 0; j < NV; ++j) {
+                    const int e = (j * team + l) * VEC;
+                    if (seg_ok && e < a.G) emit_vec<T, OP, true>(raw[r][j], R, ip, seg * a.G + e, a);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < NV; ++j) {
+                    const int e = (j * team + l) * VEC;
+                    if (seg_ok && e < a.G) emit_vec<T, OP, false>(raw[r][j], R, ip, seg * a.G + e, a);
+                }
+            }
+        }
+    }
+}
+
+// A CTA of NTH threads per group, NV vectors per thread.
+template <class T, int OP, int NTH, int NV, bool SYM>
+__global__ void __launch_bounds__(NTH) k_int_dyn_cta(DynArgs a) {
+    constexpr int VEC = Traits<T>::VEC;
+    constexpr int NW = NTH / 32;
+    __shared__ float sh_hi[2][NW], sh_nlo[2][NW];
+    const T* __restrict__ x = (const T*)a.x;
+    const int tid = threadIdx.x, wid = tid >> 5, lane = tid & 31;
+    int par = 0;
+    for (int64_t seg = blockIdx.x; seg < a.n_seg; seg += gridDim.x, par ^= 1) {
+        U4 raw[NV];
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+            const int e = (j * NTH + tid) * VEC;
+            raw[j] = (e < a.G) ? ld16_stream(x + seg * a.G + e) : U4{0u, 0u, 0u, 0u};
+        }
+        float hi = 0.0f, nlo = 0.0f;
+#pragma unroll
+        for (int j = 0; j < NV; ++j) range_vec<T>(raw[j], SYM, hi, nlo);
+        hi = warp_max(hi);
+        if (!SYM) nlo = warp_max(nlo);
+        if (lane == 0) { sh_hi[par][wid] = hi; sh_nlo[par][wid] = nlo; }
+        __syncthreads();
+        hi = sh_hi[par][0];
+        nlo = sh_nlo[par][0];
+#pragma unroll
+        for (int w = 1; w < NW; ++w) {
+            hi = fmaxf(hi, sh_hi[par][w]);
+            if (!SYM) nlo = fmaxf(nlo, sh_nlo[par][w]);
+        }
+        if (SYM) nlo = 0.0f;
+        const GroupF g = derive_f(hi, nlo, a.cfg);
+        if (tid == 0) {
+            a.scale[seg] = g.s;
+            if (a.zp) a.zp[seg] = (uint8_t)g.zp;
+        }
+        const IntParams ip = make_int_params(a.cfg.qmin, a.cfg.qmax, g.zp);
+        const Recip R = make_recip(g.s);
+        if (R.fast) {
+#pragma unroll
+            for (int j = 0; j < NV; ++j) {
+                const int e = (j * NTH + tid) * VEC;
+                if (e < a.G) emit_vec<T, OP, true>(raw[j], R, ip, seg * a.G + e, a);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < NV; ++j) {
+                const int e = (j * NTH + tid) * VEC;
+                if (e < a.G) emit_vec<T, OP, false>(raw[j], R, ip, seg * a.G + e, a);
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------ element-wise
+struct MapArgs {
+    const void* a;      // x, q or dy
+    const void* b;      // dy (backwards)
+    int64_t numel, G, n_seg;
+    FastDiv fd;         // divide by G when numel < 2^32
+    int use_fd;
+    IntCfg cfg;
+    const float* scale_in;
+    const void* zp_in;
+    const unsigned long long* ranges;
+    float* scale_out;
+    uint8_t* zp_out;
+    void* out;
+};
+
+// Per-group state cached by a thread while it walks its elements.
+struct GState {
+    int64_t seg;
+    float s;
+    int zp;
+    Recip R;
+    IntParams ip;
+};
+
+template <class T, int PSRC>
+__device__ __forceinline__ void load_group(const MapArgs& a, int64_t seg, bool writer, GState& st) {
+    using Acc = typename Traits<T>::Acc;
+    st.seg = seg;
+    if (PSRC == PS_RANGE) {
+        Acc hi, nlo;
+        range_from_bits(a.ranges[2 * seg], hi);
+        range_from_bits(a.ranges[2 * seg + 1], nlo);
+        if constexpr (std::is_same<Acc, double>::value) {
+            const GroupD g = derive_d(hi, nlo, a.cfg);
+            st.s = g.s; st.zp = g.zp;
+        } else {
+            const GroupF g = derive_f(hi, nlo, a.cfg);
+            st.s = g.s; st.zp = g.zp;
+        }
+        if (writer) {
+            a.scale_out[seg] = st.s;
+            if (a.zp_out) a.zp_out[seg] = (uint8_t)st.zp;
+        }
+    } else {
+        st.s = __ldg(a.scale_in + seg);
+        st.zp = a.cfg.symmetric ? 0 : load_zp(a.zp_in, seg, a.cfg.q_signed);
+    }
+    st.R = make_recip(st.s);
+    st.ip = make_int_params(a.cfg.qmin, a.cfg.qmax, st.zp);
+}
+
+// One element, f32 arithmetic. Returns the output value (float ops) or the
+// code byte (QUANT) in the low byte of *code.
+template <int OP, bool RHAZ>
+__device__ __forceinline__ float elem_f(float xa, float xb, const GState& st, uint32_t* code) {
+    if constexpr (OP == OP_QUANT || OP == OP_FAKE) {
+        const float v = div_any(xa, st.R);
+        const uint32_t c = code_of<RHAZ>(v, st.ip);
+        *code = c;
+        if constexpr (OP == OP_FAKE) return __fmul_rn(__fsub_rn(__uint_as_float(c), st.ip.magic), st.s);
+        return 0.0f;
+    } else if constexpr (OP == OP_QBWD || OP == OP_FBWD) {
+        const float v = div_any(xa, st.R);
+        const float k = round_for_mask<RHAZ>(v, st.ip);
+        const float m = (k > st.ip.lo && k < st.ip.hi) ? 1.0f : 0.0f;
+        if constexpr (OP == OP_QBWD) {
+            const float g = with_quotient_sign(div_any(xb, st.R), xb, st.s);
+            return __fmul_rn(g, m);
+        } else {
+            return __fmul_rn(xb, m);
+        }
+    } else if constexpr (OP == OP_DBWD) {
+        return __fmul_rn(xa, st.s);
+    } else {
+        return 0.0f;
+    }
+}
+
+// f64 arithmetic (f64 tensors).
+template <int OP, bool RHAZ>
+__device__ __forceinline__ double elem_d(double xa, double xb, const GState& st, uint32_t* code) {
+    const double s = (double)st.s;
+    const double lo = (double)st.ip.lo, hi = (double)st.ip.hi;
+    if constexpr (OP == OP_QUANT || OP == OP_FAKE) {
+        const double v = xa / s;
+        double k = RHAZ ? round(v) : rint(v);
+        k = fmin(fmax(k, lo), hi);                  // NaN -> lo
+        *code = (uint32_t)((int)k + st.zp);
+        if constexpr (OP == OP_FAKE) return k * s;
+        return 0.0;
+    } else if constexpr (OP == OP_QBWD || OP == OP_FBWD) {
+        const double v = xa / s;
+        double k = RHAZ ? round(v) : rint(v);
+        if (v != v) k = lo;
+        const double m = (k > lo && k < hi) ? 1.0 : 0.0;
+        if constexpr (OP == OP_QBWD) return (xb / s) * m;
+        else return xb * m;
+    } else if constexpr (OP == OP_DBWD) {
+        return xa * s;
+    } else {
+        return 0.0;
+    }
+}
+
+// Dequantize one code: (q - zp) * s. The byte goes into the low mantissa of
+// 2^23 so that one f32 subtraction gives q - zp exactly.
+__device__ __forceinline__ float deq_code_f(uint32_t word, int i, const GState& st, int q_signed) {
+    if (q_signed) word ^= 0x80808080u;
+    const uint32_t sel = (uint32_t)i | (4u << 4) | (5u << 8) | (7u << 12);
+    const float f = __uint_as_float(__byte_perm(word, 0x4B000000u, sel));
+    const float off = 8388608.0f + (float)((q_signed ? 128 : 0) + st.zp);
+    return __fmul_rn(__fsub_rn(f, off), st.s);
+}
+
+template <class T, int OP, int PSRC, bool VECP, bool RHAZ>
+__global__ void __launch_bounds__(256) k_int_map(MapArgs a) {
+    using Acc = typename Traits<T>::Acc;
+    constexpr bool WIDE = std::is_same<Acc, double>::value;
+    constexpr int W = VECP ? Traits<T>::VEC : 1;
+    const int64_t n_items = a.numel / W;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    GState st;
+    st.seg = -1;
+    for (int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; it < n_items; it += stride) {
+        const int64_t e0 = it * W;
+        const int64_t seg = a.use_fd ? (int64_t)fdiv((uint32_t)e0, a.fd) : e0 / a.G;
+        if (seg != st.seg) load_group<T, PSRC>(a, seg, e0 == seg * a.G, st);
+
+        if constexpr (OP == OP_DEQ) {
+            // a: codes (bytes); out: T
+            const uint8_t* qb = (const uint8_t*)a.a + e0;
+            Acc o[W];
+            if constexpr (W == 8) {
+                const uint2 w2 = __ldg(reinterpret_cast<const uint2*>(qb));
+#pragma unroll
+                for (int i = 0; i < 4; ++i) o[i] = deq_code_f(w2.x, i, st, a.cfg.q_signed);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) o[4 + i] = deq_code_f(w2.y, i, st, a.cfg.q_signed);
+            } else if constexpr (W == 4) {
+                const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(qb));
+#pragma unroll
+                for (int i = 0; i < 4; ++i) o[i] = deq_code_f(w, i, st, a.cfg.q_signed);
+            } else {
+#pragma unroll
+                for (int i = 0; i < W; ++i) {
+                    const uint8_t b = __ldg(qb + i);
+                    const int qv = a.cfg.q_signed ? (int)(int8_t)b : (int)b;
+                    if constexpr (WIDE) o[i] = (double)(qv - st.zp) * (double)st.s;
+                    else o[i] = __fmul_rn((float)(qv - st.zp), st.s);
+                }
+            }
+            if constexpr (VECP) {
+                st16((T*)a.out + e0, pack_vec<T>(o));
+            } else {
+                ((T*)a.out)[e0] = to_out<T>(o[0]);
+            }
+        } else {
+            Acc xa[W], xb[W];
+            if constexpr (VECP) {
+                load_vec<T>(ld16_stream((const T*)a.a + e0), xa);
+                if constexpr (OP == OP_QBWD || OP == OP_FBWD)
+                    load_vec<T>(ld16_stream((const T*)a.b + e0), xb);
+            } else {
+                xa[0] = ld1<T>((const T*)a.a + e0);
+                if constexpr (OP == OP_QBWD || OP == OP_FBWD) xb[0] = ld1<T>((const T*)a.b + e0);
+            }
+            Acc o[W];
+            uint32_t cw[W];
+#pragma unroll
+            for (int i = 0; i < W; ++i) {
+                if constexpr (WIDE) o[i] = elem_d<OP, RHAZ>(xa[i], (OP == OP_QBWD || OP == OP_FBWD) ? xb[i] : 0.0, st, &cw[i]);
+                else o[i] = elem_f<OP, RHAZ>(xa[i], (OP == OP_QBWD || OP == OP_FBWD) ? xb[i] : 0.0f, st, &cw[i]);
+            }
+            if constexpr (OP == OP_QUANT) {
+                uint8_t* q = (uint8_t*)a.out + e0;
+                if constexpr (W == 8) {
+                    st8(q, pack4_lowbytes(cw[0], cw[1], cw[2], cw[3]),
+                        pack4_lowbytes(cw[4], cw[5], cw[6], cw[7]));
+                } else if constexpr (W == 4) {
+                    st4(q, pack4_lowbytes(cw[0], cw[1], cw[2], cw[3]));
+                } else {
+#pragma unroll
+                    for (int i = 0; i < W; ++i) q[i] = (uint8_t)cw[i];
+                }
+            } else {
+                if constexpr (VECP) st16((T*)a.out + e0, pack_vec<T>(o));
+                else ((T*)a.out)[e0] = to_out<T>(o[0]);
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------ ranges
+template <class Acc>
+__device__ __forceinline__ void acc_range(Acc v, bool sym, Acc& hi, Acc& nlo) {
+    if (sym) {
+        hi = fmax(hi, fabs(v));
+    } else {
+        hi = fmax(hi, v);
+        nlo = fmax(nlo, -v);
+    }
+}
+
+// Whole tensor: grid-stride 16-byte loads, CTA reduction, one atomicMax per
+// CTA and slot. Unaligned head / tail elements go through scalar loads.
+template <class T>
+__global__ void __launch_bounds__(512) k_tensor_range(const T* __restrict__ x, int64_t n,
+                                                      int64_t head, int sym,
+                                                      unsigned long long* rec) {
+    using Acc = typename Traits<T>::Acc;
+    constexpr int VEC = Traits<T>::VEC;
+    constexpr int UNR = 4;
+    __shared__ Acc sh[2][16];
+    Acc hi = 0, nlo = 0;
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
+    if (tid < head) acc_range<Acc>(ld1<T>(x + tid), sym, hi, nlo);
+    const T* body = x + head;
+    const int64_t nb = n - head;
+    const int64_t nvec = nb / VEC;
+    int64_t i = tid;
+    for (; i + (UNR - 1) * nthr < nvec; i += UNR * nthr) {
+        U4 r[UNR];
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) r[u] = ld16_stream(body + (i + u * nthr) * VEC);
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) {
+            Acc v[VEC];
+            load_vec<T>(r[u], v);
+#pragma unroll
+            for (int k = 0; k < VEC; ++k) acc_range<Acc>(v[k], sym, hi, nlo);
+        }
+    }
+    for (; i < nvec; i += nthr) {
+        Acc v[VEC];
+        load_vec<T>(ld16_stream(body + i * VEC), v);
+#pragma unroll
+        for (int k = 0; k < VEC; ++k) acc_range<Acc>(v[k], sym, hi, nlo);
+    }
+    const int64_t tail0 = nvec * VEC;
+    if (tid < nb - tail0) acc_range<Acc>(ld1<T>(body + tail0 + tid), sym, hi, nlo);
+
+    hi = warp_max(hi);
+    nlo = warp_max(nlo);
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) { sh[0][w] = hi; sh[1][w] = nlo; }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const int nw = blockDim.x >> 5;
+        for (int k = 1; k < nw; ++k) { hi = fmax(hi, sh[0][k]); nlo = fmax(nlo, sh[1][k]); }
+        atomicMax(rec, range_bits(hi));
+        if (!sym) atomicMax(rec + 1, range_bits(nlo));
+    }
+}
+
+// Many groups: the units (group, slice of UL elements) are split into one
+// contiguous block per warp; a warp flushes its running range with
+// atomicMax whenever the group changes and at the end.
+template <class T, bool VECP>
+__global__ void __launch_bounds__(256) k_seg_range(const T* __restrict__ x, int64_t n_seg,
+                                                   int64_t G, int64_t upg, int64_t per_warp,
+                                                   int sym, unsigned long long* ranges) {
+    using Acc = typename Traits<T>::Acc;
+    constexpr int W = VECP ? Traits<T>::VEC : 1;
+    constexpr int UNR = 4;
+    constexpr int64_t UL = 32 * W * UNR;
+    const int lane = threadIdx.x & 31;
+    const int64_t gwarp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t total = n_seg * upg;
+    const int64_t u0 = gwarp * per_warp;
+    const int64_t u1 = min(total, u0 + per_warp);
+    int64_t cur = -1;
+    Acc hi = 0, nlo = 0;
+    for (int64_t u = u0; u < u1; ++u) {
+        const int64_t seg = u / upg, part = u % upg;
+        if (seg != cur) {
+            if (cur >= 0) {
+                const Acc h = warp_max(hi), nl = warp_max(nlo);
+                if (lane == 0) {
+                    atomicMax(ranges + 2 * cur, range_bits(h));
+                    if (!sym) atomicMax(ranges + 2 * cur + 1, range_bits(nl));
+                }
+            }
+            cur = seg;
+            hi = 0; nlo = 0;
+        }
+        const int64_t base = seg * G + part * UL;
+        const int64_t lim = min(UL, G - part * UL);
+#pragma unroll
+        for (int k = 0; k < UNR; ++k) {
+            const int64_t e = (int64_t)(k * 32 + lane) * W;
+            if (e < lim) {
+                Acc v[W];
+                if constexpr (VECP) load_vec<T>(ld16_stream(x + base + e), v);
+                else v[0] = ld1<T>(x + base + e);
+#pragma unroll
+                for (int m = 0; m < W; ++m) acc_range<Acc>(v[m], sym, hi, nlo);
+            }
+        }
+    }
+    if (cur >= 0) {
+        const Acc h = warp_max(hi), nl = warp_max(nlo);
+        if (lane == 0) {
+            atomicMax(ranges + 2 * cur, range_bits(h));
+            if (!sym) atomicMax(ranges + 2 * cur + 1, range_bits(nl));
+        }
+    }
+}
+
+// Groups that hold no element (a zero-sized dimension after the axis): the
+// range is empty, so the parameters are those of a zero range.
+__global__ void k_empty_groups(int64_t n_seg, IntCfg cfg, float* scale, uint8_t* zp) {
+    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < n_seg;
+         g += (int64_t)gridDim.x * blockDim.x) {
+        const GroupF p = derive_f(0.0f, 0.0f, cfg);
+        scale[g] = p.s;
+        if (zp) zp[g] = (uint8_t)p.zp;
+    }
+}
+
+__global__ void k_range_to_amax(const unsigned long long* rec, float* amax) {
+    float h, n;
+    range_from_bits(rec[0], h);
+    range_from_bits(rec[1], n);
+    *amax = fmaxf(h, n);
+}
+
+// ------------------------------------------------------------ launchers
+static int g_sms[64];
+
+int sm_count() {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    int v = __atomic_load_n(&g_sms[dev], __ATOMIC_RELAXED);
+    if (v <= 0) {
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+            v = 148;
+        __atomic_store_n(&g_sms[dev], v, __ATOMIC_RELAXED);
+    }
+    return v;
+}
+
+static unsigned grid_for(int64_t work_items, int per_block, int blocks_per_sm) {
+    int64_t need = (work_items + per_block - 1) / per_block;
+    int64_t cap = (int64_t)sm_count() * blocks_per_sm;
+    if (need < 1) need = 1;
+    return (unsigned)(need < cap ? need : cap);
+}
+
+template <class T, int OP, bool SYM>
+static cudaError_t launch_dyn_t(const DynArgs& a0, cudaStream_t st) {
+    constexpr int VEC = Traits<T>::VEC;
+    DynArgs a = a0;
+    const int64_t U = a.G / VEC;          // vectors per group
+    if (U <= 32) {
+        int team = 1;
+        while (team < U) team <<= 1;
+        a.team = team;
+        const int64_t groups_per_warp = (32 / team) * 4;
+        const int64_t warps = (a.n_seg + groups_per_warp - 1) / groups_per_warp;
+        k_int_dyn_warp<T, OP, 1, 4, SYM><<<grid_for(warps * 32, 256, 8), 256, 0, st>>>(a);
+    } else if (U <= 64) {
+        a.team = 32;
+        k_int_dyn_warp<T, OP, 2, 2, SYM><<<grid_for(((a.n_seg + 1) / 2) * 32, 256, 8), 256, 0, st>>>(a);
+    } else if (U <= 128) {
+        a.team = 32;
+        k_int_dyn_warp<T, OP, 4, 1, SYM><<<grid_for(a.n_seg * 32, 256, 8), 256, 0, st>>>(a);
+    } else if (U <= 256) {
+        a.team = 32;
+        k_int_dyn_warp<T, OP, 8, 1, SYM><<<grid_for(a.n_seg * 32, 256, 8), 256, 0, st>>>(a);
+    } else if (U <= 512) {
+        a.team = 32;
+        k_int_dyn_warp<T, OP, 16, 1, SYM><<<grid_for(a.n_seg * 32, 256, 6), 256, 0, st>>>(a);
+    } else if (U <= 1024) {
+        k_int_dyn_cta<T, OP, 256, 4, SYM><<<grid_for(a.n_seg, 1, 8), 256, 0, st>>>(a);
+    } else if (U <= 2048) {
+        k_int_dyn_cta<T, OP, 256, 8, SYM><<<grid_for(a.n_seg, 1, 6), 256, 0, st>>>(a);
+    } else if (U <= 4096) {
+        k_int_dyn_cta<T, OP, 256, 16, SYM><<<grid_for(a.n_seg, 1, 3), 256, 0, st>>>(a);
+    } else {
+        return cudaErrorNotSupported;
+    }
+    return cudaGetLastError();
+}
+
+template <class T>
+static cudaError_t launch_dyn_dt(int op, bool sym, const DynArgs& a, cudaStream_t st) {
+    if (op == OP_QUANT) return sym ? launch_dyn_t<T, OP_QUANT, true>(a, st) : launch_dyn_t<T, OP_QUANT, false>(a, st);
+    return sym ? launch_dyn_t<T, OP_FAKE, true>(a, st) : launch_dyn_t<T, OP_FAKE, false>(a, st);
+}
+
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+cudaError_t int_dyn(DT dt, int op, const void* x, SegView sv, IntCfg cfg, void* q, void* y,
+                    float* scale, void* zp, cudaStream_t st) {
+    if (dt == DT::F64 || cfg.rhaz) return cudaErrorNotSupported;
+    if (op != OP_QUANT && op != OP_FAKE) return cudaErrorNotSupported;
+    const int VEC = (dt == DT::F32) ? 4 : 8;
+    if (sv.G % VEC != 0 || sv.G > (int64_t)4096 * VEC || !aligned16(x)) return cudaErrorNotSupported;
+    if (op == OP_QUANT && ((uintptr_t)q % VEC) != 0) return cudaErrorNotSupported;
+    if (op == OP_FAKE && !aligned16(y)) return cudaErrorNotSupported;
+    if (sv.n_seg == 0) return cudaSuccess;
+    DynArgs a;
+    a.x = x; a.n_seg = sv.n_seg; a.G = (int)sv.G; a.team = 32; a.cfg = cfg;
+    a.q = (uint8_t*)q; a.y = y; a.scale = scale; a.zp = (uint8_t*)zp;
+    const bool sym = cfg.symmetric != 0;
+    switch (dt) {
+        case DT::F32: return launch_dyn_dt<float>(op, sym, a, st);
+        case DT::F16: return launch_dyn_dt<__half>(op, sym, a, st);
+        case DT::BF16: return launch_dyn_dt<__nv_bfloat16>(op, sym, a, st);
+        default: return cudaErrorNotSupported;
+    }
+}
+
+template <class T, int OP, int PSRC, bool VECP>
+static cudaError_t launch_map4(const MapArgs& a, cudaStream_t st) {
+    const int W = VECP ? Traits<T>::VEC : 1;
+    const unsigned grid = grid_for(a.numel / W, 256, 8);
+    if (a.cfg.rhaz) k_int_map<T, OP, PSRC, VECP, true><<<grid, 256, 0, st>>>(a);
+    else k_int_map<T, OP, PSRC, VECP, false><<<grid, 256, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+template <class T, int OP, int PSRC>
+static cudaError_t launch_map3(const MapArgs& a, bool vecp, cudaStream_t st) {
+    return vecp ? launch_map4<T, OP, PSRC, true>(a, st) : launch_map4<T, OP, PSRC, false>(a, st);
+}
+
+template <class T>
+static cudaError_t launch_map_dt(int op, int psrc, const MapArgs& a, bool vecp, cudaStream_t st) {
+    switch (op) {
+        case OP_QUANT:
+            return psrc == PS_RANGE ? launch_map3<T, OP_QUANT, PS_RANGE>(a, vecp, st)
+                                    : launch_map3<T, OP_QUANT, PS_STATIC>(a, vecp, st);
+        case OP_FAKE:
+            return psrc == PS_RANGE ? launch_map3<T, OP_FAKE, PS_RANGE>(a, vecp, st)
+                                    : launch_map3<T, OP_FAKE, PS_STATIC>(a, vecp, st);
+        case OP_QBWD: return launch_map3<T, OP_QBWD, PS_STATIC>(a, vecp, st);
+        case OP_FBWD: return launch_map3<T, OP_FBWD, PS_STATIC>(a, vecp, st);
+        case OP_DEQ: return launch_map3<T, OP_DEQ, PS_STATIC>(a, vecp, st);
+        case OP_DBWD: return launch_map3<T, OP_DBWD, PS_STATIC>(a, vecp, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t int_map(DT dt, int op, int psrc, const void* a_ptr, const void* b_ptr, SegView sv,
+                    IntCfg cfg, const float* scale_in, const void* zp_in,
+                    const unsigned long long* ranges, float* scale_out, void* zp_out, void* out,
+                    cudaStream_t st) {
+    if (sv.numel == 0) return cudaSuccess;
+    MapArgs a;
+    a.a = a_ptr; a.b = b_ptr;
+    a.numel = sv.numel; a.G = sv.G; a.n_seg = sv.n_seg;
+    a.use_fd = (sv.numel < ((int64_t)1 << 32)) ? 1 : 0;
+    a.fd = make_fastdiv(a.use_fd ? (uint32_t)sv.G : 1u);
+    a.cfg = cfg;
+    a.scale_in = scale_in; a.zp_in = zp_in; a.ranges = ranges;
+    a.scale_out = scale_out; a.zp_out = (uint8_t*)zp_out; a.out = out;
+    const int esz = (dt == DT::F64) ? 8 : (dt == DT::F32 ? 4 : 2);
+    const int VEC = 16 / esz;
+    bool vecp = (sv.G % VEC == 0);
+    if (op == OP_DEQ) {
+        vecp = vecp && aligned16(out) && ((uintptr_t)a_ptr % VEC == 0);
+    } else {
+        vecp = vecp && aligned16(a_ptr);
+        if (op == OP_QBWD || op == OP_FBWD) vecp = vecp && aligned16(b_ptr);
+        if (op == OP_QUANT) vecp = vecp && ((uintptr_t)out % VEC == 0);
+        else vecp = vecp && aligned16(out);
+    }
+    switch (dt) {
+        case DT::F32: return launch_map_dt<float>(op, psrc, a, vecp, st);
+        case DT::F64: return launch_map_dt<double>(op, psrc, a, vecp, st);
+        case DT::F16: return launch_map_dt<__half>(op, psrc, a, vecp, st);
+        case DT::BF16: return launch_map_dt<__nv_bfloat16>(op, psrc, a, vecp, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+template <class T>
+static cudaError_t launch_seg_range_t(const void* x, SegView sv, bool sym, unsigned long long* r,
+                                      cudaStream_t st) {
+    constexpr int VEC = Traits<T>::VEC;
+    const bool vecp = (sv.G % VEC == 0) && aligned16(x);
+    const int64_t UL = 32 * (vecp ? VEC : 1) * 4;
+    const int64_t upg = (sv.G + UL - 1) / UL;
+    const int64_t total = sv.n_seg * upg;
+    const unsigned grid = grid_for(total * 32, 256, 8);
+    const int64_t nwarps = (int64_t)grid * 8;
+    const int64_t per_warp = (total + nwarps - 1) / nwarps;
+    if (vecp) k_seg_range<T, true><<<grid, 256, 0, st>>>((const T*)x, sv.n_seg, sv.G, upg, per_warp, sym, r);
+    else k_seg_range<T, false><<<grid, 256, 0, st>>>((const T*)x, sv.n_seg, sv.G, upg, per_warp, sym, r);
+    return cudaGetLastError();
+}
+
+cudaError_t seg_range(DT dt, const void* x, SegView sv, bool sym, unsigned long long* ranges,
+                      cudaStream_t st) {
+    if (sv.n_seg == 0 || sv.G == 0) return cudaSuccess;
+    switch (dt) {
+        case DT::F32: return launch_seg_range_t<float>(x, sv, sym, ranges, st);
+        case DT::F64: return launch_seg_range_t<double>(x, sv, sym, ranges, st);
+        case DT::F16: return launch_seg_range_t<__half>(x, sv, sym, ranges, st);
+        case DT::BF16: return launch_seg_range_t<__nv_bfloat16>(x, sv, sym, ranges, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+template <class T>
+static cudaError_t launch_tensor_range_t(const void* x, int64_t n, bool sym,
+                                         unsigned long long* rec, cudaStream_t st) {
+    constexpr int VEC = Traits<T>::VEC;
+    int64_t head = 0;
+    const uintptr_t p = (uintptr_t)x;
+    if (p % 16 != 0) {
+        head = (int64_t)((16 - p % 16) / sizeof(T));
+        if (head > n) head = n;
+    }
+    const int64_t nvec = (n - head) / VEC;
+    const unsigned grid = grid_for(nvec / 4 + 1, 512, 2);
+    k_tensor_range<T><<<grid, 512, 0, st>>>((const T*)x, n, head, sym ? 1 : 0, rec);
+    return cudaGetLastError();
+}
+
+cudaError_t tensor_range(DT dt, const void* x, int64_t n, bool sym, unsigned long long* rec,
+                         cudaStream_t st) {
+    if (n == 0) return cudaSuccess;
+    switch (dt) {
+        case DT::F32: return launch_tensor_range_t<float>(x, n, sym, rec, st);
+        case DT::F64: return launch_tensor_range_t<double>(x, n, sym, rec, st);
+        case DT::F16: return launch_tensor_range_t<__half>(x, n, sym, rec, st);
+        case DT::BF16: return launch_tensor_range_t<__nv_bfloat16>(x, n, sym, rec, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t empty_groups(int64_t n_seg, IntCfg cfg, float* scale, void* zp, cudaStream_t st) {
+    if (n_seg == 0) return cudaSuccess;
+    k_empty_groups<<<grid_for(n_seg, 256, 4), 256, 0, st>>>(n_seg, cfg, scale, (uint8_t*)zp);
+    return cudaGetLastError();
+}
+
+__global__ void k_set_f32(float* p, float v) { *p = v; }
+
+cudaError_t set_f32(float* p, float v, cudaStream_t st) {
+    k_set_f32<<<1, 1, 0, st>>>(p, v);
+    return cudaGetLastError();
+}
+
+cudaError_t range_to_amax(const unsigned long long* rec, float* amax, cudaStream_t st) {
+    k_range_to_amax<<<1, 1, 0, st>>>(rec, amax);
+    return cudaGetLastError();
+}
+
+}  // namespace bq

@@ -1,0 +1,75 @@
+// Internal launch interface between the C ABI (bq_abi.cu) and the kernel
+// translation units. Not installed; not part of the public header.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace bq {
+
+enum class DT { F32 = 0, F64 = 1, F16 = 2, BF16 = 3 };
+
+// Integer code range of a quantize call.
+struct IntCfg {
+    int qmin, qmax;
+    int symmetric;
+    int rhaz;       // 1: ties away from zero
+    int q_signed;   // 1: codes are s8, 0: u8
+};
+
+// Contiguous-group view: n_seg groups of G consecutive elements each.
+struct SegView {
+    int64_t n_seg, G, numel;
+};
+
+enum Op { OP_QUANT = 0, OP_FAKE = 1, OP_QBWD = 2, OP_FBWD = 3, OP_DEQ = 4, OP_DBWD = 5 };
+enum Psrc { PS_STATIC = 0, PS_RANGE = 1 };
+
+int sm_count();
+
+// Single pass: reduction, scale and codes in registers. Returns
+// cudaErrorNotSupported (and launches nothing) when no register-resident
+// configuration covers this view; the caller then takes the two-pass path.
+cudaError_t int_dyn(DT dt, int op, const void* x, SegView sv, IntCfg cfg, void* q, void* y,
+                    float* scale, void* zp, cudaStream_t st);
+
+// Element-wise with per-group parameters (static, or derived from range
+// records). a: x (QUANT, FAKE, QBWD, FBWD), q (DEQ) or dy (DBWD);
+// b: dy (QBWD, FBWD). out: q (QUANT) or a float tensor of type dt.
+cudaError_t int_map(DT dt, int op, int psrc, const void* a, const void* b, SegView sv,
+                    IntCfg cfg, const float* scale_in, const void* zp_in,
+                    const unsigned long long* ranges, float* scale_out, void* zp_out, void* out,
+                    cudaStream_t st);
+
+// Range records of every group (ranges cleared by the caller).
+cudaError_t seg_range(DT dt, const void* x, SegView sv, bool sym, unsigned long long* ranges,
+                      cudaStream_t st);
+
+// Range record of the whole tensor (rec cleared by the caller).
+cudaError_t tensor_range(DT dt, const void* x, int64_t n, bool sym, unsigned long long* rec,
+                         cudaStream_t st);
+// Parameters of groups with no elements (scale 1, zero-point of a zero range).
+cudaError_t empty_groups(int64_t n_seg, IntCfg cfg, float* scale, void* zp, cudaStream_t st);
+// *p = v.
+cudaError_t set_f32(float* p, float v, cudaStream_t st);
+// amax = max(rec[0], rec[1]) as f32.
+cudaError_t range_to_amax(const unsigned long long* rec, float* amax, cudaStream_t st);
+
+// Microscaled formats.
+enum MxFmt { MX_FP8_1x128 = 0, MX_MXFP8 = 1, MX_NVFP4 = 2 };
+cudaError_t mx_quant(DT dt, int fmt, const void* x, int64_t rows, int64_t k, uint8_t* codes,
+                     void* scales, const unsigned long long* amax_rec, float* global_scale,
+                     int static_global, cudaStream_t st);
+cudaError_t mx_dequant(DT ydt, int fmt, const uint8_t* codes, const void* scales,
+                       const float* global_scale, int64_t rows, int64_t k, void* y,
+                       cudaStream_t st);
+cudaError_t fp8_tile_quant(DT dt, const void* x, int64_t rows, int64_t cols, int br, int bc,
+                           uint8_t* e4m3, float* scale, cudaStream_t st);
+cudaError_t fp8_block_dequant(DT ydt, const uint8_t* e4m3, const float* scale, int64_t rows,
+                              int64_t cols, int br, int bc, void* y, cudaStream_t st);
+
+// Byte transpose [rows, cols] -> [cols, stride], columns [rows, stride) zeroed.
+cudaError_t byte_transpose(const uint8_t* in, int64_t rows, int64_t cols, int64_t stride,
+                           uint8_t* out, cudaStream_t st);
+
+}  // namespace bq

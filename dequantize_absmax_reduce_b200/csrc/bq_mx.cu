@@ -1,0 +1,525 @@
+// Microscaled formats: FP8 E4M3 with f32 scales per 1x128 group or 128x128
+// tile (smile llm.quant Fp8BlockGemm / Fp8BlockDequant), MXFP8 with an E8M0
+// scale per 32 (smile llm.quant MxFp8), and NVFP4 with E2M1 codes packed two
+// per byte, an E4M3 scale per 16 and an f32 per-tensor scale (metrale
+// QuantizedWeight).
+//
+// k_mx_quant: contiguous groups of 16 / 32 / 128 elements along a row, one
+//   team of 2..32 lanes per group, 16-byte streaming loads, the group held in
+//   registers between its amax and its codes (one HBM pass; NVFP4 also reads
+//   the per-tensor range record written by a prior amax pass).
+// k_fp8_tile: one CTA per 128x128 tile (or ragged / unaligned 1x128 group).
+// k_mx_deq: element-wise decode with the group's scale.
+#include <type_traits>
+
+#include "bq_device.cuh"
+#include "bq_internal.h"
+
+namespace bq {
+
+template <int FMT> struct MxG;
+template <> struct MxG<MX_FP8_1x128> { static constexpr int G = 128; };
+template <> struct MxG<MX_MXFP8> { static constexpr int G = 32; };
+template <> struct MxG<MX_NVFP4> { static constexpr int G = 16; };
+
+struct MxArgs {
+    const void* x;
+    int64_t n_seg;
+    uint8_t* codes;
+    void* scales;
+    const unsigned long long* amax_rec;
+    float* global_scale;
+    int static_global;
+};
+
+__device__ __forceinline__ void st2(void* p, uint32_t a) {
+    asm volatile("st.global.u16 [%0], %1;" :: "l"(p), "h"((uint16_t)a) : "memory");
+}
+
+// MXFP8 shared exponent: E = clamp(floor(log2 a) - 8, -127, 127), from the
+// bits of a >= 0 (a subnormal a counts its leading zeros; infinity is 2^128;
+// a = 0 gives -127).
+__device__ __forceinline__ int mx_exponent(float a) {
+    const uint32_t b = __float_as_uint(a);
+    const int ex = (int)(b >> 23);
+    int fl2;
+    if (ex == 0) {
+        const uint32_t m = b & 0x7FFFFFu;
+        fl2 = (m == 0) ? -1000 : (31 - __clz((int)m)) - 149;
+    } else if (ex == 255) {
+        fl2 = 128;
+    } else {
+        fl2 = ex - 127;
+    }
+    return min(max(fl2 - 8, -127), 127);
+}
+
+// Codes of one lane's VEC elements (v: values, out: packed bytes).
+template <class T, int FMT, bool FAST>
+__device__ __forceinline__ void mx_emit(const float* v, const Recip& R, float mul, bool zero,
+                                        uint8_t* dst) {
+    constexpr int VEC = Traits<T>::VEC;
+    float t[VEC];
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) {
+        if constexpr (FMT == MX_MXFP8) {
+            t[i] = __fmul_rn(v[i], mul);
+        } else {
+            const float d = FAST ? div_chain(v[i], R) : div_any(v[i], R);
+            t[i] = with_quotient_sign(d, v[i], R.s);
+        }
+    }
+    if constexpr (FMT == MX_NVFP4) {
+        if constexpr (VEC == 8) {
+            const uint32_t w = zero ? 0u : e2m1x8(*reinterpret_cast<const float(*)[8]>(t));
+            st4(dst, w);
+        } else {
+            float t8[8] = {t[0], t[1], t[2], t[3], 0.f, 0.f, 0.f, 0.f};
+            const uint32_t w = zero ? 0u : e2m1x8(t8);
+            st2(dst, w & 0xFFFFu);
+        }
+    } else {
+        if constexpr (VEC == 8) {
+            st8(dst, e4m3x4(t[0], t[1], t[2], t[3]), e4m3x4(t[4], t[5], t[6], t[7]));
+        } else {
+            st4(dst, e4m3x4(t[0], t[1], t[2], t[3]));
+        }
+    }
+}
+
+template <class T, int FMT, int SEGS>
+__global__ void __launch_bounds__(256) k_mx_quant(MxArgs a) {
+    constexpr int VEC = Traits<T>::VEC;
+    constexpr int G = MxG<FMT>::G;
+    constexpr int TEAM = G / VEC;
+    constexpr int TPW = 32 / TEAM;
+    constexpr int CB = (FMT == MX_NVFP4) ? VEC / 2 : VEC;   // code bytes per lane
+    const T* __restrict__ x = (const T*)a.x;
+    const int lane = threadIdx.x & 31;
+    const int tm = lane / TEAM, l = lane % TEAM;
+    const int64_t gwarp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t per_chunk = (int64_t)SEGS * TPW;
+    const int64_t n_chunks = (a.n_seg + per_chunk - 1) / per_chunk;
+
+    float s2 = 1.0f;
+    Recip R6;
+    if constexpr (FMT == MX_NVFP4) {
+        if (a.static_global) {
+            s2 = *a.global_scale;
+        } else {
+            float h, n;
+            range_from_bits(a.amax_rec[0], h);
+            range_from_bits(a.amax_rec[1], n);
+            s2 = __fdiv_rn(fmaxf(h, n), 2688.0f);    // 2688 = 448 * 6
+            if (s2 == 0.0f) s2 = 1.0f;
+            if (blockIdx.x == 0 && threadIdx.x == 0) *a.global_scale = s2;
+        }
+        R6 = make_recip(__fmul_rn(6.0f, s2));
+    }
+
+    for (int64_t c = gwarp; c < n_chunks; c += nwarps) {
+        U4 raw[SEGS];
+#pragma unroll
+        for (int r = 0; r < SEGS; ++r) {
+            const int64_t seg = c * per_chunk + r * TPW + tm;
+            raw[r] = (seg < a.n_seg) ? ld16_stream(x + seg * G + l * VEC) : U4{0u, 0u, 0u, 0u};
+        }
+#pragma unroll
+        for (int r = 0; r < SEGS; ++r) {
+            const int64_t seg = c * per_chunk + r * TPW + tm;
+            float v[VEC];
+            load_vec<T>(raw[r], v);
+            float am = 0.0f;
+#pragma unroll
+            for (int i = 0; i < VEC; ++i) am = fmaxf(am, fabsf(v[i]));
+#pragma unroll
+            for (int o = TEAM / 2; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+            const bool ok = seg < a.n_seg;
+            uint8_t* dst = a.codes + seg * (G * CB / VEC) + l * CB;
+            if constexpr (FMT == MX_FP8_1x128) {
+                float s = __fdiv_rn(am, 448.0f);
+                if (s == 0.0f) s = 1.0f;
+                if (ok && l == 0) ((float*)a.scales)[seg] = s;
+                const Recip R = make_recip(s);
+                if (ok) {
+                    if (R.fast) mx_emit<T, FMT, true>(v, R, 0.f, false, dst);
+                    else mx_emit<T, FMT, false>(v, R, 0.f, false, dst);
+                }
+            } else if constexpr (FMT == MX_MXFP8) {
+                const int E = mx_exponent(am);
+                if (ok && l == 0) ((uint8_t*)a.scales)[seg] = (uint8_t)(E + 127);
+                Recip R{};
+                if (ok) mx_emit<T, FMT, true>(v, R, exp2i(-E), false, dst);
+            } else {
+                const float q6 = div_any(am, R6);                 // a_b / (6 s2)
+                const uint32_t sb = e4m3x2(q6, 0.0f) & 0xFFu;
+                if (ok && l == 0) ((uint8_t*)a.scales)[seg] = (uint8_t)sb;
+                const float eff = __fmul_rn(e4m3_to_f32(sb), s2);
+                const Recip R = make_recip(eff);
+                if (ok) {
+                    if (R.fast && !a.static_global) mx_emit<T, FMT, true>(v, R, 0.f, eff == 0.0f, dst);
+                    else mx_emit<T, FMT, false>(v, R, 0.f, eff == 0.0f, dst);
+                }
+            }
+        }
+    }
+}
+
+// Scalar fallback for unaligned inputs: one thread per group.
+template <class T, int FMT>
+__global__ void __launch_bounds__(256) k_mx_quant_scalar(MxArgs a) {
+    constexpr int G = MxG<FMT>::G;
+    const T* __restrict__ x = (const T*)a.x;
+    float s2 = 1.0f;
+    Recip R6;
+    if constexpr (FMT == MX_NVFP4) {
+        if (a.static_global) {
+            s2 = *a.global_scale;
+        } else {
+            float h, n;
+            range_from_bits(a.amax_rec[0], h);
+            range_from_bits(a.amax_rec[1], n);
+            s2 = __fdiv_rn(fmaxf(h, n), 2688.0f);
+            if (s2 == 0.0f) s2 = 1.0f;
+            if (blockIdx.x == 0 && threadIdx.x == 0) *a.global_scale = s2;
+        }
+        R6 = make_recip(__fmul_rn(6.0f, s2));
+    }
+    for (int64_t seg = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; seg < a.n_seg;
+         seg += (int64_t)gridDim.x * blockDim.x) {
+        const T* p = x + seg * G;
+        float am = 0.0f;
+        for (int i = 0; i < G; ++i) am = fmaxf(am, fabsf(ld1<T>(p + i)));
+        if constexpr (FMT == MX_FP8_1x128) {
+            float s = __fdiv_rn(am, 448.0f);
+            if (s == 0.0f) s = 1.0f;
+            ((float*)a.scales)[seg] = s;
+            const Recip R = make_recip(s);
+            for (int i = 0; i < G; i += 2) {
+                const float v0 = ld1<T>(p + i), v1 = ld1<T>(p + i + 1);
+                const uint32_t w = e4m3x2(with_quotient_sign(div_any(v0, R), v0, s),
+                                          with_quotient_sign(div_any(v1, R), v1, s));
+                a.codes[seg * G + i] = (uint8_t)w;
+                a.codes[seg * G + i + 1] = (uint8_t)(w >> 8);
+            }
+        } else if constexpr (FMT == MX_MXFP8) {
+            const int E = mx_exponent(am);
+            ((uint8_t*)a.scales)[seg] = (uint8_t)(E + 127);
+            const float inv = exp2i(-E);
+            for (int i = 0; i < G; i += 2) {
+                const uint32_t w = e4m3x2(__fmul_rn(ld1<T>(p + i), inv), __fmul_rn(ld1<T>(p + i + 1), inv));
+                a.codes[seg * G + i] = (uint8_t)w;
+                a.codes[seg * G + i + 1] = (uint8_t)(w >> 8);
+            }
+        } else {
+            const uint32_t sb = e4m3x2(div_any(am, R6), 0.0f) & 0xFFu;
+            ((uint8_t*)a.scales)[seg] = (uint8_t)sb;
+            const float eff = __fmul_rn(e4m3_to_f32(sb), s2);
+            const Recip R = make_recip(eff);
+            for (int i = 0; i < G; i += 8) {
+                float t[8];
+                for (int j = 0; j < 8; ++j) {
+                    const float v = ld1<T>(p + i + j);
+                    t[j] = with_quotient_sign(div_any(v, R), v, eff);
+                }
+                const uint32_t w = (eff == 0.0f) ? 0u : e2m1x8(t);
+                uint8_t* d = a.codes + (seg * G + i) / 2;
+                d[0] = (uint8_t)w; d[1] = (uint8_t)(w >> 8); d[2] = (uint8_t)(w >> 16); d[3] = (uint8_t)(w >> 24);
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------ FP8 tiles
+// One CTA per br x 128 block; a block on the bottom / right edge may be
+// partial. VECP: cols % VEC == 0 and x 16-byte aligned.
+template <class T, int BR, int NTH, bool VECP>
+__global__ void __launch_bounds__(NTH) k_fp8_tile(const T* __restrict__ x, int64_t rows,
+                                                  int64_t cols, int64_t nbc, uint8_t* e4m3,
+                                                  float* scale) {
+    constexpr int BC = 128;
+    constexpr int W = VECP ? Traits<T>::VEC : 1;
+    constexpr int IPR = BC / W;                     // items per block row
+    constexpr int NI = (BR * IPR + NTH - 1) / NTH;  // items per thread
+    constexpr int NW = NTH / 32;
+    __shared__ float sh[NW];
+    const int64_t bi = blockIdx.x / nbc, bj = blockIdx.x % nbc;
+    const int tid = threadIdx.x;
+    float v[NI][W];
+    bool ok[NI];
+    float am = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NI; ++i) {
+        const int item = tid + i * NTH;
+        const int64_t r = bi * BR + item / IPR;
+        const int64_t c = bj * BC + (int64_t)(item % IPR) * W;
+        ok[i] = (item < BR * IPR) && (r < rows) && (c < cols);
+        if (ok[i]) {
+            if constexpr (VECP) load_vec<T>(ld16_stream(x + r * cols + c), v[i]);
+            else v[i][0] = ld1<T>(x + r * cols + c);
+        } else {
+#pragma unroll
+            for (int k = 0; k < W; ++k) v[i][k] = 0.0f;
+        }
+#pragma unroll
+        for (int k = 0; k < W; ++k) am = fmaxf(am, fabsf(v[i][k]));
+    }
+    am = warp_max(am);
+    if ((tid & 31) == 0) sh[tid >> 5] = am;
+    __syncthreads();
+    am = sh[0];
+#pragma unroll
+    for (int w = 1; w < NW; ++w) am = fmaxf(am, sh[w]);
+    float s = __fdiv_rn(am, 448.0f);
+    if (s == 0.0f) s = 1.0f;
+    if (tid == 0) scale[blockIdx.x] = s;
+    const Recip R = make_recip(s);
+#pragma unroll
+    for (int i = 0; i < NI; ++i) {
+        if (!ok[i]) continue;
+        const int item = tid + i * NTH;
+        const int64_t r = bi * BR + item / IPR;
+        const int64_t c = bj * BC + (int64_t)(item % IPR) * W;
+        float t[W];
+#pragma unroll
+        for (int k = 0; k < W; ++k) {
+            const float d = R.fast ? div_chain(v[i][k], R) : __fdiv_rn(v[i][k], s);
+            t[k] = with_quotient_sign(d, v[i][k], s);
+        }
+        uint8_t* dst = e4m3 + r * cols + c;
+        if constexpr (W == 8) {
+            st8(dst, e4m3x4(t[0], t[1], t[2], t[3]), e4m3x4(t[4], t[5], t[6], t[7]));
+        } else if constexpr (W == 4) {
+            st4(dst, e4m3x4(t[0], t[1], t[2], t[3]));
+        } else {
+            *dst = (uint8_t)e4m3x2(t[0], 0.0f);
+        }
+    }
+}
+
+// ------------------------------------------------------------ dequantize
+struct DeqArgs {
+    const uint8_t* codes;
+    const void* scales;
+    const float* global_scale;
+    int64_t rows, k;           // row length k (cols for FP8 blocks)
+    int br, bc;                // FP8 block shape
+    int64_t nbc;               // FP8 blocks per row of blocks
+    int64_t numel;
+    FastDiv fk;
+    int use_fd;
+    void* y;
+};
+
+template <int FMT>
+__device__ __forceinline__ float mx_group_mul(const DeqArgs& a, int64_t r, int64_t c, float s2) {
+    if constexpr (FMT == MX_NVFP4) {
+        const uint32_t sb = __ldg(((const uint8_t*)a.scales) + r * (a.k / 16) + c / 16);
+        return __fmul_rn(e4m3_to_f32(sb), s2);
+    } else if constexpr (FMT == MX_MXFP8) {
+        const uint32_t b = __ldg(((const uint8_t*)a.scales) + r * (a.k / 32) + c / 32);
+        return (b == 0xFFu) ? __uint_as_float(0x7FC00000u) : exp2i((int)b - 127);
+    } else {
+        return __ldg(((const float*)a.scales) + (r / a.br) * a.nbc + c / a.bc);
+    }
+}
+
+// FMT as above; MX_FP8_1x128 here covers every FP8 block shape.
+template <class T, int FMT, bool VECP>
+__global__ void __launch_bounds__(256) k_mx_deq(DeqArgs a) {
+    constexpr int W = VECP ? 16 : 1;
+    const float s2 = (FMT == MX_NVFP4) ? __ldg(a.global_scale) : 1.0f;
+    const int64_t n_items = a.numel / W;
+    for (int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; it < n_items;
+         it += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t e0 = it * W;
+        const int64_t r = a.use_fd ? (int64_t)fdiv((uint32_t)e0, a.fk) : e0 / a.k;
+        const int64_t c = e0 - r * a.k;
+        const float mul = mx_group_mul<FMT>(a, r, c, s2);
+        float o[W];
+        if constexpr (FMT == MX_NVFP4) {
+            if constexpr (VECP) {
+                const uint2 w = __ldg(reinterpret_cast<const uint2*>(a.codes + e0 / 2));
+                const uint32_t ws[2] = {w.x, w.y};
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        const float2 f = e2m1x2_to_f32((ws[h] >> (8 * b)) & 0xFFu);
+                        o[h * 8 + 2 * b] = __fmul_rn(f.x, mul);
+                        o[h * 8 + 2 * b + 1] = __fmul_rn(f.y, mul);
+                    }
+            } else {
+                const uint32_t byte = __ldg(a.codes + e0 / 2);
+                const float2 f = e2m1x2_to_f32(byte);
+                o[0] = __fmul_rn((e0 & 1) ? f.y : f.x, mul);
+            }
+        } else {
+            if constexpr (VECP) {
+                const uint4 w = __ldg(reinterpret_cast<const uint4*>(a.codes + e0));
+                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const float2 f0 = e4m3x2_to_f32(ws[h] & 0xFFFFu);
+                    const float2 f1 = e4m3x2_to_f32(ws[h] >> 16);
+                    o[4 * h] = __fmul_rn(f0.x, mul);
+                    o[4 * h + 1] = __fmul_rn(f0.y, mul);
+                    o[4 * h + 2] = __fmul_rn(f1.x, mul);
+                    o[4 * h + 3] = __fmul_rn(f1.y, mul);
+                }
+            } else {
+                o[0] = __fmul_rn(e4m3_to_f32(__ldg(a.codes + e0)), mul);
+            }
+        }
+        T* y = (T*)a.y + e0;
+        if constexpr (VECP) {
+            constexpr int VEC = Traits<T>::VEC;
+#pragma unroll
+            for (int h = 0; h < 16 / VEC; ++h) {
+                float part[VEC];
+#pragma unroll
+                for (int k = 0; k < VEC; ++k) part[k] = o[h * VEC + k];
+                st16(y + h * VEC, pack_vec<T>(part));
+            }
+        } else {
+            *y = to_out<T>(o[0]);
+        }
+    }
+}
+
+// ------------------------------------------------------------ launchers
+static bool al(const void* p, int n) { return ((uintptr_t)p % (uintptr_t)n) == 0; }
+
+static unsigned grid_cap(int64_t need_blocks, int per_sm) {
+    int64_t cap = (int64_t)sm_count() * per_sm;
+    if (need_blocks < 1) need_blocks = 1;
+    return (unsigned)(need_blocks < cap ? need_blocks : cap);
+}
+
+template <class T, int FMT>
+static cudaError_t launch_mx_quant_t(const MxArgs& a, bool vec, cudaStream_t st) {
+    constexpr int VEC = Traits<T>::VEC;
+    constexpr int G = MxG<FMT>::G;
+    constexpr int TPW = 32 / (G / VEC);
+    if (vec) {
+        constexpr int SEGS = (G / VEC >= 16) ? 2 : 4;
+        const int64_t warps = (a.n_seg + (int64_t)SEGS * TPW - 1) / ((int64_t)SEGS * TPW);
+        k_mx_quant<T, FMT, SEGS><<<grid_cap((warps + 7) / 8, 8), 256, 0, st>>>(a);
+    } else {
+        k_mx_quant_scalar<T, FMT><<<grid_cap((a.n_seg + 255) / 256, 8), 256, 0, st>>>(a);
+    }
+    return cudaGetLastError();
+}
+
+template <int FMT>
+static cudaError_t launch_mx_quant_f(DT dt, const MxArgs& a, bool vec, cudaStream_t st) {
+    switch (dt) {
+        case DT::F32: return launch_mx_quant_t<float, FMT>(a, vec, st);
+        case DT::F16: return launch_mx_quant_t<__half, FMT>(a, vec, st);
+        case DT::BF16: return launch_mx_quant_t<__nv_bfloat16, FMT>(a, vec, st);
+        default: return cudaErrorNotSupported;
+    }
+}
+
+cudaError_t mx_quant(DT dt, int fmt, const void* x, int64_t rows, int64_t k, uint8_t* codes,
+                     void* scales, const unsigned long long* amax_rec, float* global_scale,
+                     int static_global, cudaStream_t st) {
+    const int G = fmt == MX_FP8_1x128 ? 128 : (fmt == MX_MXFP8 ? 32 : 16);
+    MxArgs a;
+    a.x = x; a.n_seg = rows * (k / G); a.codes = codes; a.scales = scales;
+    a.amax_rec = amax_rec; a.global_scale = global_scale; a.static_global = static_global;
+    if (a.n_seg == 0) return cudaSuccess;
+    const int VEC = dt == DT::F32 ? 4 : 8;
+    const int cb = (fmt == MX_NVFP4) ? VEC / 2 : VEC;
+    const bool vec = al(x, 16) && al(codes, cb);
+    switch (fmt) {
+        case MX_FP8_1x128: return launch_mx_quant_f<MX_FP8_1x128>(dt, a, vec, st);
+        case MX_MXFP8: return launch_mx_quant_f<MX_MXFP8>(dt, a, vec, st);
+        case MX_NVFP4: return launch_mx_quant_f<MX_NVFP4>(dt, a, vec, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+template <class T>
+static cudaError_t launch_tile_t(const void* x, int64_t rows, int64_t cols, int br, uint8_t* e,
+                                 float* s, cudaStream_t st) {
+    constexpr int VEC = Traits<T>::VEC;
+    const int64_t nbr = (rows + br - 1) / br, nbc = (cols + 127) / 128;
+    const int64_t nb = nbr * nbc;
+    if (nb == 0) return cudaSuccess;
+    if (nb > 0x7FFFFFFFll) return cudaErrorInvalidValue;
+    const bool vec = (cols % VEC == 0) && al(x, 16) && al(e, VEC);
+    if (br == 128) {
+        if (vec) k_fp8_tile<T, 128, 256, true><<<(unsigned)nb, 256, 0, st>>>((const T*)x, rows, cols, nbc, e, s);
+        else k_fp8_tile<T, 128, 256, false><<<(unsigned)nb, 256, 0, st>>>((const T*)x, rows, cols, nbc, e, s);
+    } else {
+        if (vec) k_fp8_tile<T, 1, 32, true><<<(unsigned)nb, 32, 0, st>>>((const T*)x, rows, cols, nbc, e, s);
+        else k_fp8_tile<T, 1, 128, false><<<(unsigned)nb, 128, 0, st>>>((const T*)x, rows, cols, nbc, e, s);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t fp8_tile_quant(DT dt, const void* x, int64_t rows, int64_t cols, int br, int bc,
+                           uint8_t* e4m3, float* scale, cudaStream_t st) {
+    if (bc != 128 || (br != 1 && br != 128)) return cudaErrorNotSupported;
+    switch (dt) {
+        case DT::F32: return launch_tile_t<float>(x, rows, cols, br, e4m3, scale, st);
+        case DT::F16: return launch_tile_t<__half>(x, rows, cols, br, e4m3, scale, st);
+        case DT::BF16: return launch_tile_t<__nv_bfloat16>(x, rows, cols, br, e4m3, scale, st);
+        default: return cudaErrorNotSupported;
+    }
+}
+
+template <class T, int FMT>
+static cudaError_t launch_deq_t(const DeqArgs& a, cudaStream_t st) {
+    const int cin = (FMT == MX_NVFP4) ? 8 : 16;   // code bytes per 16 elements
+    const bool vec = (a.k % 16 == 0) && al(a.y, 16) && al(a.codes, cin);
+    const int64_t items = vec ? a.numel / 16 : a.numel;
+    const unsigned grid = grid_cap((items + 255) / 256, 8);
+    if (vec) k_mx_deq<T, FMT, true><<<grid, 256, 0, st>>>(a);
+    else k_mx_deq<T, FMT, false><<<grid, 256, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+template <int FMT>
+static cudaError_t launch_deq_f(DT dt, const DeqArgs& a, cudaStream_t st) {
+    switch (dt) {
+        case DT::F32: return launch_deq_t<float, FMT>(a, st);
+        case DT::F16: return launch_deq_t<__half, FMT>(a, st);
+        case DT::BF16: return launch_deq_t<__nv_bfloat16, FMT>(a, st);
+        default: return cudaErrorNotSupported;
+    }
+}
+
+static DeqArgs make_deq(const uint8_t* codes, const void* scales, const float* gs, int64_t rows,
+                        int64_t k, void* y) {
+    DeqArgs a;
+    a.codes = codes; a.scales = scales; a.global_scale = gs;
+    a.rows = rows; a.k = k; a.br = 1; a.bc = 128; a.nbc = 1;
+    a.numel = rows * k;
+    a.use_fd = (a.numel < ((int64_t)1 << 32) && k > 0) ? 1 : 0;
+    a.fk = make_fastdiv(a.use_fd ? (uint32_t)k : 1u);
+    a.y = y;
+    return a;
+}
+
+cudaError_t mx_dequant(DT ydt, int fmt, const uint8_t* codes, const void* scales,
+                       const float* global_scale, int64_t rows, int64_t k, void* y,
+                       cudaStream_t st) {
+    DeqArgs a = make_deq(codes, scales, global_scale, rows, k, y);
+    if (a.numel == 0) return cudaSuccess;
+    if (fmt == MX_NVFP4) return launch_deq_f<MX_NVFP4>(ydt, a, st);
+    if (fmt == MX_MXFP8) return launch_deq_f<MX_MXFP8>(ydt, a, st);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t fp8_block_dequant(DT ydt, const uint8_t* e4m3, const float* scale, int64_t rows,
+                              int64_t cols, int br, int bc, void* y, cudaStream_t st) {
+    DeqArgs a = make_deq(e4m3, scale, nullptr, rows, cols, y);
+    a.br = br; a.bc = bc; a.nbc = (cols + bc - 1) / bc;
+    if (a.numel == 0) return cudaSuccess;
+    return launch_deq_f<MX_FP8_1x128>(ydt, a, st);
+}
+
+}  // namespace bq

@@ -1,0 +1,305 @@
+/*
+ * bq — scaled quantize / dequantize on NVIDIA B200 (sm_100a), C ABI.
+ *
+ * Sources of the operations (each declaration below names its own):
+ *   [baracuda]        docs.rs baracuda_kernels::quantize, module index: the
+ *                     per_tensor / per_channel / per_token / per_group quantize
+ *                     and dequantize plans, fake_quantize ("per-tensor, FP
+ *                     roundtrip"), their backwards, the Straight-Through
+ *                     Estimator dx = (dy / scale) * 1[qmin < q < qmax] with the
+ *                     mask recomputed from the saved input, dtype coverage
+ *                     (input f32/f64/f16/bf16, output s8/u8) and default_q_range.
+ *   [granularity]     teenygrad teeny_quant/quant/granularity.rs: Granularity
+ *                     {PerTensor, PerChannel{axis}, Group{axis, group_size}},
+ *                     axis_and_group_size() and strategy_name().
+ *   [QuantizedWeight] docs.metrale.ai QuantizedWeight: NVFP4 weight (packed
+ *                     E2M1 two per byte, FP8 scale per 16, f32 weight_scale_2),
+ *                     transpose_for_gemm(_gs) and transpose_concat_for_gemm_padded.
+ *   [smile.llm.quant] package summary: Fp8BlockGemm / Fp8BlockDequant (E4M3
+ *                     with an f32 scale per 1x128 activation group or per
+ *                     128x128 weight tile) and MxFp8 (E4M3 with an E8M0 scale
+ *                     per 32 elements along the reduction dimension).
+ *
+ * Conventions for every entry point:
+ *   - Pointers named x, q, y, dy, dx, dq, scale, zp, ranges, ws, packed,
+ *     e4m3, e8m0, w, sc, w_t, sc_t are DEVICE pointers owned by the caller.
+ *     Tensors are dense and row-major (C order). The library allocates
+ *     nothing, keeps no state between calls and may be called from several
+ *     host threads at once.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Every call only enqueues work on that stream and returns; it
+ *     never synchronises the host.
+ *   - Arguments are validated on the host before anything is enqueued; on
+ *     any error nothing is launched and the outputs are untouched.
+ *   - Status codes: BQ_OK; BQ_ERR_INVALID_ARG (null pointer where data is
+ *     needed, negative or inconsistent sizes, axis out of range, group_size
+ *     not dividing the axis, qmin >= qmax, workspace too small);
+ *     BQ_ERR_UNSUPPORTED (dtype combination or mode not provided, e.g. a
+ *     symmetric u8 code range); BQ_ERR_MISALIGNED (reserved);
+ *     BQ_ERR_CUDA (a launch failed: cudaGetLastError after the launch);
+ *     BQ_ERR_TIMEOUT (reserved: no kernel here waits on another).
+ *   - Arithmetic: f32/f16/bf16 inputs are widened exactly to f32 and every
+ *     step is one IEEE f32 operation with round-to-nearest-even (a divide is
+ *     the correctly rounded quotient); f64 inputs use f64. Results are
+ *     bit-identical to the plain CPU definition of each op.
+ */
+#ifndef BQ_H
+#define BQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum bq_status {
+    BQ_OK = 0,
+    BQ_ERR_INVALID_ARG = 1,
+    BQ_ERR_UNSUPPORTED = 2,
+    BQ_ERR_MISALIGNED = 3,
+    BQ_ERR_CUDA = 4,
+    BQ_ERR_TIMEOUT = 5
+} bq_status;
+
+typedef enum bq_dtype {
+    BQ_F32 = 0, BQ_F64 = 1, BQ_F16 = 2, BQ_BF16 = 3,
+    BQ_S8 = 4, BQ_U8 = 5,
+    BQ_E4M3 = 6, BQ_E2M1X2 = 7, BQ_E8M0 = 8
+} bq_dtype;
+
+/* Rounding of x/scale to an integer code: nearest with ties to even
+ * (required), or ties away from zero. */
+typedef enum bq_round { BQ_RNE = 0, BQ_RHAZ = 1 } bq_round;
+
+/* [granularity] Granularity. Per-token is PerChannel on the second-to-last
+ * axis and has its own entry points. */
+typedef enum bq_gran { BQ_GRAN_TENSOR = 0, BQ_GRAN_CHANNEL = 1, BQ_GRAN_GROUP = 2 } bq_gran;
+
+/* Where the per-group scale / zero-point come from.
+ *   DYNAMIC:    derived from each group's range and written to scale / zp.
+ *   STATIC:     read from scale / zp (inputs).
+ *   FROM_RANGE: derived from the range records in `ws` (as written by
+ *               bq_group_range, possibly combined across shards with an
+ *               element-wise MAX) and written to scale / zp. */
+typedef enum bq_scale_mode {
+    BQ_SCALE_DYNAMIC = 0, BQ_SCALE_STATIC = 1, BQ_SCALE_FROM_RANGE = 2
+} bq_scale_mode;
+
+/* Description of a quantized tensor x (up to 8 dims) and its code range.
+ * qmin = qmax = 0 selects default_q_range(q_dtype): S8 [-128,127],
+ * U8 [0,255] ([baracuda] default_q_range).
+ * Symmetric: scale = fl(amax / qmax), zero-point 0 (S8 only).
+ * Asymmetric: min' = min(min x, 0), max' = max(max x, 0),
+ *   scale = fl(fl(max' - min') / (qmax - qmin)),
+ *   zp = clamp(qmin - round(fl(min' / scale)), qmin, qmax).
+ * A scale that comes out as 0 is replaced by 1. Ranges ignore NaN.
+ * Quantize: q = clamp(round(fl(x / scale)) + zp, qmin, qmax); a NaN
+ * quotient gives qmin. */
+typedef struct bq_qdesc {
+    int32_t ndim;
+    int64_t shape[8];
+    bq_dtype x_dtype;   /* F32, F64, F16 or BF16 */
+    bq_dtype q_dtype;   /* S8 or U8 */
+    int32_t symmetric;  /* 1: absmax scaling, 0: min/max + zero-point */
+    int32_t qmin, qmax;
+    bq_round rnd;
+} bq_qdesc;
+
+/* ------------------------------------------------------------------ misc */
+
+/* Human-readable name of a status code (static storage). */
+const char* bq_status_string(bq_status s);
+
+/* [granularity] strategy_name(): "tensor", "channel" or "group"; NULL for an
+ * unknown value. */
+const char* bq_granularity_name(bq_gran g);
+
+/* [baracuda] default_q_range: S8 -> [-128, 127], U8 -> [0, 255]. Host only. */
+bq_status bq_default_q_range(bq_dtype q_dtype, int32_t* qmin, int32_t* qmax);
+
+/* [granularity] axis_and_group_size() applied to a shape: number of scale
+ * groups (the length of scale / zp) and elements per group. Group g of outer
+ * index o holds axis indices [g*gs, (g+1)*gs) and every index of the
+ * dimensions after `axis`, i.e. one contiguous run of gs * prod(shape[axis+1:])
+ * elements. PerTensor is one group; PerChannel{axis} is Group{axis, 1}.
+ * Host only. */
+bq_status bq_group_count(const bq_qdesc* d, bq_gran gran, int32_t axis, int64_t group_size,
+                         int64_t* n_groups, int64_t* group_elems);
+
+/* Bytes of device workspace `ws` a quantize / fake_quantize call with these
+ * arguments needs (0 when it runs in one pass over x). Per-tensor dynamic
+ * scaling always needs 16 bytes: one range record. Host only. */
+size_t bq_quantize_workspace_size(const bq_qdesc* d, bq_gran gran, int32_t axis,
+                                  int64_t group_size, bq_scale_mode mode);
+
+/* Per-group range records of x: ranges is uint64[2 * n_groups]; record g is
+ * { bits(max(0, max x)), bits(max(0, -min x)) } over group g, NaN ignored,
+ * where bits() is the IEEE bit pattern of the value as f32 (f64 for f64 x),
+ * zero-extended. Both values are >= 0, so records of shards combine with an
+ * element-wise integer MAX (e.g. an all-reduce MAX over int64). The call
+ * clears `ranges` itself before accumulating. */
+bq_status bq_group_range(const void* x, const bq_qdesc* d, bq_gran gran, int32_t axis,
+                         int64_t group_size, void* ranges, void* stream);
+
+/* Tensor amax: max |x| over n elements of dtype (F32, F16, BF16), NaN
+ * ignored, written as f32 to *amax. ws: 16 bytes of device scratch. This is
+ * the first pass of per-tensor scaling and of the NVFP4 per-tensor scale
+ * ([QuantizedWeight] weight_scale_2). */
+bq_status bq_tensor_amax(const void* x, bq_dtype dtype, int64_t n, float* amax, void* ws,
+                         void* stream);
+
+/* -------------------------------------------------------------- quantize */
+/* [baracuda] quantize_per_tensor / per_channel / per_token / per_group.
+ * x: d->shape, dtype d->x_dtype. q: same shape, dtype d->q_dtype.
+ * scale: f32[n_groups]; zp: q_dtype[n_groups] (may be NULL when symmetric).
+ * ws / ws_bytes: see bq_quantize_workspace_size (FROM_RANGE reads its range
+ * records from ws). Per-token groups are the rows of the last dimension;
+ * per-channel is per-group with group_size 1 along `axis`. */
+bq_status bq_quantize_per_tensor(const void* x, const bq_qdesc* d, void* q, float* scale,
+                                 void* zp, bq_scale_mode mode, void* ws, size_t ws_bytes,
+                                 void* stream);
+bq_status bq_quantize_per_channel(const void* x, const bq_qdesc* d, int32_t axis, void* q,
+                                  float* scale, void* zp, bq_scale_mode mode, void* ws,
+                                  size_t ws_bytes, void* stream);
+bq_status bq_quantize_per_token(const void* x, const bq_qdesc* d, void* q, float* scale,
+                                void* zp, bq_scale_mode mode, void* ws, size_t ws_bytes,
+                                void* stream);
+bq_status bq_quantize_per_group(const void* x, const bq_qdesc* d, int32_t axis,
+                                int64_t group_size, void* q, float* scale, void* zp,
+                                bq_scale_mode mode, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------ dequantize */
+/* [baracuda] dequantize_per_tensor / per_channel / per_token / per_group:
+ * y = RN_y(fl((q - zp) * scale)); y has shape d->shape and dtype y_dtype
+ * (F32, F64, F16, BF16; an F64 y holds the exact product). zp may be NULL
+ * (zero). d->x_dtype is ignored; d->q_dtype gives q's dtype. */
+bq_status bq_dequantize_per_tensor(const void* q, const float* scale, const void* zp,
+                                   const bq_qdesc* d, void* y, bq_dtype y_dtype, void* stream);
+bq_status bq_dequantize_per_channel(const void* q, const float* scale, const void* zp,
+                                    const bq_qdesc* d, int32_t axis, void* y, bq_dtype y_dtype,
+                                    void* stream);
+bq_status bq_dequantize_per_token(const void* q, const float* scale, const void* zp,
+                                  const bq_qdesc* d, void* y, bq_dtype y_dtype, void* stream);
+bq_status bq_dequantize_per_group(const void* q, const float* scale, const void* zp,
+                                  const bq_qdesc* d, int32_t axis, int64_t group_size, void* y,
+                                  bq_dtype y_dtype, void* stream);
+
+/* --------------------------------------------------------- fake quantize */
+/* [baracuda] fake_quantize ("FP roundtrip"): y = dequantize(quantize(x)) in
+ * x's dtype, at any granularity (per-token: BQ_GRAN_CHANNEL with
+ * axis = ndim - 2). scale / zp / mode / ws as for quantize. */
+bq_status bq_fake_quantize(const void* x, const bq_qdesc* d, bq_gran gran, int32_t axis,
+                           int64_t group_size, float* scale, void* zp, bq_scale_mode mode,
+                           void* y, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------- backwards */
+/* [baracuda] quantize_*_backward (Straight-Through Estimator):
+ * dx = RN_x(fl(dy / scale) * m), m = 1 if qmin < round(fl(x/scale)) + zp < qmax
+ * else 0 (the code recomputed from the saved x, before clamping). x, dy and
+ * dx share d->shape and d->x_dtype; scale / zp as saved by the forward. */
+bq_status bq_quantize_per_tensor_backward(const void* x, const void* dy, const float* scale,
+                                          const void* zp, const bq_qdesc* d, void* dx,
+                                          void* stream);
+bq_status bq_quantize_per_channel_backward(const void* x, const void* dy, const float* scale,
+                                           const void* zp, const bq_qdesc* d, int32_t axis,
+                                           void* dx, void* stream);
+bq_status bq_quantize_per_token_backward(const void* x, const void* dy, const float* scale,
+                                         const void* zp, const bq_qdesc* d, void* dx,
+                                         void* stream);
+bq_status bq_quantize_per_group_backward(const void* x, const void* dy, const float* scale,
+                                         const void* zp, const bq_qdesc* d, int32_t axis,
+                                         int64_t group_size, void* dx, void* stream);
+
+/* [baracuda] fake_quantize_backward via STE: dx = dy * m (m as above). */
+bq_status bq_fake_quantize_backward(const void* x, const void* dy, const float* scale,
+                                    const void* zp, const bq_qdesc* d, bq_gran gran,
+                                    int32_t axis, int64_t group_size, void* dx, void* stream);
+
+/* [baracuda] dequantize_*_backward: dq = RN(fl(dy * scale)) (straight-through;
+ * for per-channel dq[i] = dy[i] * scale[c], per-token dy * scale[n]). dy and
+ * dq share d->shape and dtype d->x_dtype. */
+bq_status bq_dequantize_per_tensor_backward(const void* dy, const float* scale,
+                                            const bq_qdesc* d, void* dq, void* stream);
+bq_status bq_dequantize_per_channel_backward(const void* dy, const float* scale,
+                                             const bq_qdesc* d, int32_t axis, void* dq,
+                                             void* stream);
+bq_status bq_dequantize_per_token_backward(const void* dy, const float* scale,
+                                           const bq_qdesc* d, void* dq, void* stream);
+bq_status bq_dequantize_per_group_backward(const void* dy, const float* scale,
+                                           const bq_qdesc* d, int32_t axis, int64_t group_size,
+                                           void* dq, void* stream);
+
+/* ----------------------------------------------------------------- NVFP4 */
+/* [QuantizedWeight] NVFP4 quantize of x [n, k] (F32, F16 or BF16), k % 16 == 0:
+ *   s2 = fl(amax(x) / 2688) (2688 = 448 * 6; 0 -> 1), or *global_scale when
+ *   static_global != 0 (then it is an input);
+ *   per 16 consecutive elements of a row: sb = E4M3(fl(a_b / fl(6 * s2))),
+ *   eff = fl(E4M3(sb) * s2), code = E2M1(fl(x / eff)) (all codes 0 when
+ *   eff == 0).
+ * packed: u8 [n, k/2], element 2j in the low nibble of byte j.
+ * scale_e4m3: u8 [n, k/16]. global_scale: one f32 (device), written when
+ * dynamic. ws: 16 bytes (dynamic only). E4M3 encodes round to nearest even,
+ * saturate to +-448, NaN -> 0x7F; E2M1 encodes saturate to +-6 and keep the
+ * sign; a NaN element encodes as a zero with the NaN's sign bit. */
+bq_status bq_nvfp4_quantize(const void* x, bq_dtype x_dtype, int64_t n, int64_t k,
+                            uint8_t* packed, uint8_t* scale_e4m3, float* global_scale,
+                            int32_t static_global, void* ws, size_t ws_bytes, void* stream);
+
+/* [QuantizedWeight] NVFP4 dequantize: y = RN_y(fl(E2M1(code) * fl(E4M3(sb) * s2))),
+ * y [n, k] of dtype y_dtype (F32, F16, BF16). */
+bq_status bq_nvfp4_dequantize(const uint8_t* packed, const uint8_t* scale_e4m3,
+                              const float* global_scale, int64_t n, int64_t k, void* y,
+                              bq_dtype y_dtype, void* stream);
+
+/* ----------------------------------------------------------------- MXFP8 */
+/* [smile.llm.quant] MxFp8: x [rows, k] (F32, F16, BF16), k % 32 == 0. Per 32
+ * consecutive elements of a row: E = clamp(floor(log2 amax) - 8, -127, 127)
+ * (8 = exponent of 448, the largest E4M3; an all-zero block gives -127, an
+ * infinite amax counts as 2^128), e8m0 byte = E + 127, e4m3 = E4M3(fl(x * 2^-E)).
+ * e4m3: u8 [rows, k]; e8m0: u8 [rows, k/32]. */
+bq_status bq_mxfp8_quantize(const void* x, bq_dtype x_dtype, int64_t rows, int64_t k,
+                            uint8_t* e4m3, uint8_t* e8m0, void* stream);
+
+/* y = RN_y(fl(E4M3(e) * 2^(byte - 127))); byte 0xFF is NaN. */
+bq_status bq_mxfp8_dequantize(const uint8_t* e4m3, const uint8_t* e8m0, int64_t rows, int64_t k,
+                              void* y, bq_dtype y_dtype, void* stream);
+
+/* ------------------------------------------------------------ FP8 blocks */
+/* [smile.llm.quant] Fp8BlockGemm (activations, 1x128 groups) and
+ * Fp8BlockDequant (weights, 128x128 tiles, weight_scale_inv): x [rows, cols]
+ * (F32, F16, BF16); block_rows in {1, 128}, block_cols == 128; blocks on the
+ * bottom / right edge may be partial. Per block: s = fl(amax / 448) (0 -> 1),
+ * e4m3 = E4M3(fl(x / s)). scale: f32 [ceil(rows/block_rows),
+ * ceil(cols/block_cols)] row-major, the dequantize multiplier. */
+bq_status bq_fp8_block_quantize(const void* x, bq_dtype x_dtype, int64_t rows, int64_t cols,
+                                int32_t block_rows, int32_t block_cols, uint8_t* e4m3,
+                                float* scale, void* stream);
+
+/* y = RN_y(fl(E4M3(e) * scale[block])). */
+bq_status bq_fp8_block_dequantize(const uint8_t* e4m3, const float* scale, int64_t rows,
+                                  int64_t cols, int32_t block_rows, int32_t block_cols, void* y,
+                                  bq_dtype y_dtype, void* stream);
+
+/* ------------------------------------------------------- packed transpose */
+/* [QuantizedWeight] transpose_for_gemm(_gs) / transpose_concat_for_gemm_padded
+ * (one part): packed weight w u8 [n, k/2] -> w_t u8 [k/2, stride] and scales
+ * sc u8 [n, k/group_size] -> sc_t u8 [k/group_size, stride], with
+ * stride = align_up(n, align) (align >= 1; 1 means unpadded) and the pad
+ * columns [n, stride) set to 0. Bytes move unchanged (nibbles are not
+ * reordered). sc and sc_t may both be NULL (weight only). k must be even and
+ * divisible by group_size. *out_stride (host pointer, may be NULL) receives
+ * the stride. w_t / sc_t must not overlap w / sc. */
+bq_status bq_packed_transpose(const uint8_t* w, const uint8_t* sc, int64_t n, int64_t k,
+                              int64_t group_size, int64_t align, uint8_t* w_t, uint8_t* sc_t,
+                              int64_t* out_stride, void* stream);
+
+/* align_up(n, align): the row stride bq_packed_transpose uses, for sizing
+ * w_t / sc_t before the call. Returns -1 for n < 0 or align < 1. Host only. */
+int64_t bq_packed_transpose_stride(int64_t n, int64_t align);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BQ_H */

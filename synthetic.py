@@ -138,3 +138,126 @@ def bits_tensor(dtype: str) -> torch.Tensor:
     """Every bit pattern of a 16-bit float dtype, in code order (65,536 values)."""
     codes = torch.arange(0, 65536, dtype=torch.int32).to(torch.int16)
     return codes.view(_TORCH_DTYPES[dtype])
+
+
+# Workloads: the five configurations the benchmark and the full-size parity
+# tests run, as (shape, dtype, distribution) recipes. Every tensor of a
+# workload comes from one Stream seeded 0, drawn in the order listed.
+WORKLOADS = {
+    "per_tensor_f32_64x256": dict(
+        x=dict(shape=(64, 256), dtype="f32"),
+        dy=dict(shape=(64, 256), dtype="f32")),
+    "per_token_bf16_8192x4096": dict(
+        x=dict(shape=(8192, 4096), dtype="bf16", outlier_p=0.001, outlier_factor=20.0),
+        dy=dict(shape=(8192, 4096), dtype="bf16")),
+    "per_group128_f16_11008x4096": dict(
+        x=dict(shape=(11008, 4096), dtype="f16", std=0.02),
+        dy=dict(shape=(11008, 4096), dtype="f16")),
+    "nvfp4_bf16_4096x7168": dict(
+        x=dict(shape=(4096, 7168), dtype="bf16", outlier_p=0.0005, outlier_factor=50.0)),
+    "fp8_blocks_bf16": dict(
+        act=dict(shape=(16384, 7168), dtype="bf16"),
+        w=dict(shape=(7168, 18432), dtype="bf16")),
+    "fp8_blocks_bf16_student_t3": dict(
+        act=dict(shape=(16384, 7168), dtype="bf16", dist="student_t3"),
+        w=dict(shape=(7168, 18432), dtype="bf16", dist="student_t3")),
+}
+
+
+def make_workload(name: str, seed: int = 0, only=None) -> dict:
+    """CPU tensors of a workload; `only` limits which tensors are drawn (the
+    stream still advances past the others, so values do not depend on it)."""
+    st = Stream(seed)
+    out = {}
+    for key, recipe in WORKLOADS[name].items():
+        if only is not None and key not in only:
+            r = dict(recipe)
+            shape = r.pop("shape")
+            n = int(np.prod(shape))
+            dist = r.get("dist", "normal")
+            st._take(2 * ((n + 1) // 2) if dist == "normal" else 4 * n)
+            if r.get("outlier_p", 0.0) > 0.0:
+                st._take(n)
+            continue
+        r = dict(recipe)
+        out[key] = st.tensor(r.pop("shape"), **r)
+    return out
+
+
+# ---------------------------------------------------------------- device draw
+# The same recipe evaluated with torch ops on a CUDA device, for the
+# benchmark's large inputs. Integer steps are exact (int64 arithmetic wraps
+# modulo 2^64 as the uint64 recipe does; logical shifts are masked); the f64
+# transcendental functions of the device may differ from the host's in the
+# last bit, so a device draw can differ from the host draw in rare elements
+# after rounding. Tests that use a device draw hand the oracle a host copy of
+# the very values the kernels saw.
+def _mix64_t(z):
+    def srl(v, k):
+        return (v >> k) & ((1 << (64 - k)) - 1)
+    z = z ^ srl(z, 30)
+    z = z * _signed(0xBF58476D1CE4E5B9)
+    z = z ^ srl(z, 27)
+    z = z * _signed(0x94D049BB133111EB)
+    return z ^ srl(z, 31)
+
+
+def _signed(u: int) -> int:
+    return u - (1 << 64) if u >= (1 << 63) else u
+
+
+def _uniforms_t(seed: int, start: int, count: int, device):
+    idx = torch.arange(start + 1, start + count + 1, dtype=torch.int64, device=device)
+    z = _mix64_t(idx * _signed(int(GAMMA)) + _signed(seed & (2 ** 64 - 1)))
+    top = (z >> 11) & ((1 << 53) - 1)
+    return (top.to(torch.float64) + 0.5) * (2.0 ** -53)
+
+
+def _normals_t(seed: int, start: int, count: int, device):
+    npairs = (count + 1) // 2
+    u = _uniforms_t(seed, start, 2 * npairs, device).reshape(npairs, 2)
+    r = torch.sqrt(-2.0 * torch.log(u[:, 0]))
+    th = (2.0 * math.pi) * u[:, 1]
+    return torch.stack([r * torch.cos(th), r * torch.sin(th)], dim=1).reshape(-1)[:count]
+
+
+def device_tensor(stream: Stream, shape, dtype: str = "f32", std: float = 1.0,
+                  dist: str = "normal", outlier_p: float = 0.0, outlier_factor: float = 1.0,
+                  device="cuda", chunk: int = 1 << 24) -> torch.Tensor:
+    """Stream.tensor's recipe drawn on `device` (chunked to bound memory)."""
+    shape = tuple(int(s) for s in shape)
+    n = int(np.prod(shape, dtype=np.int64)) if shape else 1
+    nuni = 2 * ((n + 1) // 2) if dist == "normal" else 4 * n
+    base = stream._take(nuni)
+    obase = stream._take(n) if outlier_p > 0.0 else 0
+    out = torch.empty(n, dtype=_TORCH_DTYPES[dtype], device=device)
+    for c0 in range(0, n, chunk):
+        m = min(n, c0 + chunk) - c0
+        if dist == "normal":
+            v = _normals_t(stream.seed, base + c0, m, device)
+        else:
+            z = _normals_t(stream.seed, base + 4 * c0, 4 * m, device).reshape(m, 4)
+            v = z[:, 0] / torch.sqrt((z[:, 1] ** 2 + z[:, 2] ** 2 + z[:, 3] ** 2) / 3.0)
+        v = v * std
+        if outlier_p > 0.0:
+            u = _uniforms_t(stream.seed, obase + c0, m, device)
+            v = torch.where(u < outlier_p, v * outlier_factor, v)
+        out[c0:c0 + m] = v if dtype == "f64" else v.to(torch.float32).to(out.dtype)
+        del v
+    return out.reshape(shape)
+
+
+def make_workload_device(name: str, seed: int = 0, device="cuda", only=None) -> dict:
+    st = Stream(seed)
+    out = {}
+    for key, recipe in WORKLOADS[name].items():
+        r = dict(recipe)
+        shape = r.pop("shape")
+        if only is not None and key not in only:
+            n = int(np.prod(shape))
+            st._take(2 * ((n + 1) // 2) if r.get("dist", "normal") == "normal" else 4 * n)
+            if r.get("outlier_p", 0.0) > 0.0:
+                st._take(n)
+            continue
+        out[key] = device_tensor(st, shape, device=device, **r)
+    return out

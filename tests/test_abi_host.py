@@ -1,0 +1,137 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, it
+exports every entry point the public header declares, and argument errors
+come back as status codes before anything is enqueued."""
+
+import ctypes as C
+import os
+import re
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def B():
+    import dequantize_absmax_reduce_b200 as m
+    return m._bq
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "bq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(bq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_symbols()
+    for must in ("bq_quantize_per_tensor", "bq_quantize_per_channel", "bq_quantize_per_token",
+                 "bq_quantize_per_group", "bq_dequantize_per_group", "bq_fake_quantize",
+                 "bq_quantize_per_group_backward", "bq_fake_quantize_backward",
+                 "bq_dequantize_per_token_backward", "bq_nvfp4_quantize", "bq_nvfp4_dequantize",
+                 "bq_mxfp8_quantize", "bq_fp8_block_quantize", "bq_packed_transpose"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(B):
+    lib = C.CDLL(B.LIB_PATH)
+    missing = [n for n in declared_symbols() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_misc_host_functions(B):
+    assert B.bq_default_q_range(torch.int8) == (-128, 127)
+    assert B.bq_default_q_range(torch.uint8) == (0, 255)
+    assert [B.bq_granularity_name(g) for g in ("tensor", "channel", "group")] == ["tensor", "channel", "group"]
+    assert B.lib.bq_granularity_name(7) is None
+    assert B.bq_packed_transpose_stride(4097, 16) == 4112
+    assert B.bq_packed_transpose_stride(4096, 16) == 4096
+    assert B.bq_packed_transpose_stride(5, 1) == 5
+    assert B.bq_packed_transpose_stride(-1, 16) == -1 and B.bq_packed_transpose_stride(5, 0) == -1
+    assert B.bq_status_string(0) == "ok"
+
+
+def test_group_count_matches_reading(B):
+    d = B.make_desc((4, 6, 10), torch.float32)
+    assert B.bq_group_count(d, "tensor") == (1, 240)
+    assert B.bq_group_count(d, "channel", 0) == (4, 60)
+    assert B.bq_group_count(d, "channel", 2) == (240, 1)
+    assert B.bq_group_count(d, "group", 1, 3) == (8, 30)
+    assert B.bq_group_count(d, "group", 2, 5) == (48, 5)
+    with pytest.raises(B.BqError):
+        B.bq_group_count(d, "group", 1, 4)          # 4 does not divide 6
+    with pytest.raises(B.BqError):
+        B.bq_group_count(d, "channel", 3)
+
+
+def test_workspace_size(B):
+    d = B.make_desc((8192, 4096), torch.bfloat16)
+    assert B.bq_quantize_workspace_size(d, "channel", 0) == 0          # one pass per row
+    assert B.bq_quantize_workspace_size(d, "tensor") == 16             # two passes
+    assert B.bq_quantize_workspace_size(d, "group", 1, 128, "static") == 0
+    assert B.bq_quantize_workspace_size(d, "group", 1, 128, "from_range") == 16 * 8192 * 32
+    d64 = B.make_desc((8, 64), torch.float64)
+    assert B.bq_quantize_workspace_size(d64, "channel", 0) == 16 * 8
+    drh = B.make_desc((8, 64), torch.float32, rnd="rhaz")
+    assert B.bq_quantize_workspace_size(drh, "channel", 0) == 16 * 8
+
+
+def _status(fn):
+    try:
+        fn()
+    except Exception as e:  # BqError
+        return getattr(e, "status", None)
+    return 0
+
+
+def test_argument_errors_return_status_without_launching(B):
+    P = 0x10000  # never dereferenced: every call below fails validation first
+    d = B.make_desc((4, 64), torch.float32)
+    st = lambda: B.lib.bq_quantize_per_token(None, C.byref(d), P, P, P, 0, None, 0, None)
+    assert st() == B.BQ_ERR_INVALID_ARG                              # null x
+    du = B.make_desc((4, 64), torch.float32, torch.uint8, symmetric=True)
+    assert B.lib.bq_quantize_per_token(P, C.byref(du), P, P, P, 0, None, 0, None) == B.BQ_ERR_UNSUPPORTED
+    dq = B.make_desc((4, 64), torch.float32, qmin=5, qmax=5)
+    assert B.lib.bq_quantize_per_token(P, C.byref(dq), P, P, P, 0, None, 0, None) == B.BQ_ERR_INVALID_ARG
+    assert B.lib.bq_quantize_per_group(P, C.byref(d), 1, 48, P, P, P, 0, None, 0, None) == B.BQ_ERR_INVALID_ARG
+    assert B.lib.bq_quantize_per_channel(P, C.byref(d), 2, P, P, P, 0, None, 0, None) == B.BQ_ERR_INVALID_ARG
+    assert B.lib.bq_quantize_per_token(P + 1, C.byref(d), P, P, P, 0, None, 0, None) == B.BQ_ERR_MISALIGNED
+    assert B.lib.bq_quantize_per_token(P, C.byref(d), P, P, P, 9, None, 0, None) == B.BQ_ERR_INVALID_ARG
+    # FROM_RANGE without a large enough range buffer
+    assert B.lib.bq_quantize_per_token(P, C.byref(d), P, P, P, 2, P, 16, None) == B.BQ_ERR_INVALID_ARG
+    # asymmetric static scale without a zero-point
+    da = B.make_desc((4, 64), torch.float32, torch.uint8, symmetric=False)
+    assert B.lib.bq_quantize_per_token(P, C.byref(da), P, P, None, 1, None, 0, None) == B.BQ_ERR_INVALID_ARG
+    # dtype errors
+    dbad = B.make_desc((4, 64), B.BQ_E4M3)
+    assert B.lib.bq_quantize_per_token(P, C.byref(dbad), P, P, P, 0, None, 0, None) == B.BQ_ERR_UNSUPPORTED
+    assert B.lib.bq_dequantize_per_token(P, P, None, C.byref(d), P, B.BQ_S8, None) == B.BQ_ERR_UNSUPPORTED
+    # backward of an asymmetric code without a zero-point
+    assert B.lib.bq_quantize_per_token_backward(P, P, P, None, C.byref(da), P, None) == B.BQ_ERR_INVALID_ARG
+    # microscaled formats
+    assert B.lib.bq_nvfp4_quantize(P, B.BQ_BF16, 4, 24, P, P, P, 0, P, 16, None) == B.BQ_ERR_INVALID_ARG
+    assert B.lib.bq_nvfp4_quantize(P, B.BQ_BF16, 4, 32, P, P, P, 0, None, 0, None) == B.BQ_ERR_INVALID_ARG
+    assert B.lib.bq_nvfp4_quantize(P, B.BQ_F64, 4, 32, P, P, P, 1, None, 0, None) == B.BQ_ERR_UNSUPPORTED
+    assert B.lib.bq_mxfp8_quantize(P, B.BQ_BF16, 4, 48, P, P, None) == B.BQ_ERR_INVALID_ARG
+    assert B.lib.bq_fp8_block_quantize(P, B.BQ_BF16, 4, 256, 64, 128, P, P, None) == B.BQ_ERR_UNSUPPORTED
+    assert B.lib.bq_fp8_block_quantize(P, B.BQ_BF16, -1, 256, 1, 128, P, P, None) == B.BQ_ERR_INVALID_ARG
+    st64 = B._I64()
+    assert B.lib.bq_packed_transpose(P, P, 4, 31, 16, 16, P, P, C.byref(st64), None) == B.BQ_ERR_INVALID_ARG
+    assert B.lib.bq_packed_transpose(P, P, 4, 32, 5, 16, P, P, C.byref(st64), None) == B.BQ_ERR_INVALID_ARG
+    assert B.lib.bq_packed_transpose(P, None, 4, 32, 16, 16, P, P, C.byref(st64), None) == B.BQ_ERR_INVALID_ARG
+    # descriptor errors
+    d9 = B.make_desc((4, 64), torch.float32)
+    d9.ndim = 9
+    assert B.lib.bq_quantize_per_token(P, C.byref(d9), P, P, P, 0, None, 0, None) == B.BQ_ERR_INVALID_ARG
+    dneg = B.make_desc((4, 64), torch.float32)
+    dneg.shape[0] = -4
+    assert B.lib.bq_quantize_per_token(P, C.byref(dneg), P, P, P, 0, None, 0, None) == B.BQ_ERR_INVALID_ARG
+
+
+def test_empty_calls_succeed_without_a_device(B):
+    # Nothing to enqueue: an empty tensor returns OK before any CUDA call.
+    d = B.make_desc((0, 64), torch.float32)
+    assert B.lib.bq_quantize_per_token(None, C.byref(d), None, None, None, 0, None, 0, None) == B.BQ_OK
+    assert B.lib.bq_dequantize_per_token(None, None, None, C.byref(d), None, B.BQ_F32, None) == B.BQ_OK
+    assert B.lib.bq_mxfp8_quantize(None, B.BQ_BF16, 0, 64, None, None, None) == B.BQ_OK

@@ -1,0 +1,171 @@
+"""GPU parity of NVFP4, MXFP8, FP8 block scaling and the packed transpose.
+
+Codes, scale bytes, f32 scales, the NVFP4 per-tensor scale and dequantized
+values are compared bit for bit with the CPU oracle.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import synthetic
+from parity import assert_bitwise, cpu, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+DT = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
+
+
+@pytest.fixture(scope="module")
+def bq():
+    import dequantize_absmax_reduce_b200 as m
+    assert torch.cuda.is_available()
+    return m.api
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16", "f32"])
+@pytest.mark.parametrize("shape", [(1, 16), (7, 48), (33, 1024), (64, 7168)])
+def test_nvfp4_parity(bq, orc, dtype, shape):
+    x = synthetic.Stream(11).tensor(shape, dtype, outlier_p=0.01, outlier_factor=50)
+    packed, sc, s2 = bq.nvfp4_quantize(x.cuda())
+    rp, rsc, rs2 = orc.nvfp4_quantize(x)
+    assert cpu(s2).item() == rs2
+    assert_bitwise(packed, rp, "packed")
+    assert_bitwise(sc, rsc, "block scales")
+    for ydt in ("bf16", "f32", "f16"):
+        y = bq.nvfp4_dequantize(packed, sc, s2, DT[ydt])
+        assert_bitwise(y, orc.nvfp4_dequantize(rp, rsc, rs2, *shape, ydtype=ydt), f"deq {ydt}")
+    # static per-tensor scale, including one that saturates block scales
+    for s2v in (rs2, rs2 / 64.0, 1.0):
+        packed, sc, _ = bq.nvfp4_quantize(x.cuda(), s2=s2v)
+        rp, rsc, _ = orc.nvfp4_quantize(x, s2=float(np.float32(s2v)))
+        assert_bitwise(packed, rp, f"static packed {s2v}")
+        assert_bitwise(sc, rsc, f"static scales {s2v}")
+
+
+def test_nvfp4_special_values(bq, orc):
+    vals = [0.0, -0.0, 1e-30, -1e-30, 6.0, -6.0, 5.0, 2.5, 0.25, 0.75, 1e30, -1e30,
+            float("inf"), float("-inf"), float("nan"), -0.1]
+    x = torch.tensor(vals * 4, dtype=torch.float32).reshape(2, 32)
+    x[1] = torch.linspace(-7, 7, 32)
+    packed, sc, s2 = bq.nvfp4_quantize(x.cuda(), s2=1.0)
+    rp, rsc, _ = orc.nvfp4_quantize(x, s2=1.0)
+    assert_bitwise(packed, rp, "packed")
+    assert_bitwise(sc, rsc, "scales")
+    xz = torch.zeros(3, 64, dtype=torch.bfloat16)
+    packed, sc, s2 = bq.nvfp4_quantize(xz.cuda())
+    rp, rsc, rs2 = orc.nvfp4_quantize(xz)
+    assert cpu(s2).item() == rs2 == 1.0
+    assert_bitwise(packed, rp, "zero packed")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16", "f32"])
+@pytest.mark.parametrize("shape", [(1, 32), (5, 96), (40, 7168)])
+def test_mxfp8_parity(bq, orc, dtype, shape):
+    for dist in ("normal", "student_t3"):
+        x = synthetic.Stream(12).tensor(shape, dtype, dist=dist)
+        e, s = bq.mxfp8_quantize(x.cuda())
+        re, rs = orc.mxfp8_quantize(x)
+        assert_bitwise(e, re, "e4m3")
+        assert_bitwise(s, rs, "e8m0")
+        for ydt in ("bf16", "f32"):
+            y = bq.mxfp8_dequantize(e, s, DT[ydt])
+            assert_bitwise(y, orc.mxfp8_dequantize(re, rs, *shape, ydtype=ydt), f"deq {ydt}")
+
+
+def test_mxfp8_special_blocks(bq, orc):
+    x = torch.zeros(2, 128, dtype=torch.float32)
+    x[0, 32] = 1.0
+    x[0, 64] = 2.0 ** -130
+    x[0, 96:] = torch.tensor([float("inf"), -3.0] * 16)
+    x[1] = torch.tensor([-0.0, 448.0, 500.0, 1e-40] * 32)
+    e, s = bq.mxfp8_quantize(x.cuda())
+    re, rs = orc.mxfp8_quantize(x)
+    assert_bitwise(s, rs, "e8m0")
+    assert_bitwise(e, re, "e4m3")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16", "f32"])
+@pytest.mark.parametrize("br,shape", [(1, (3, 384)), (1, (9, 200)), (128, (256, 384)),
+                                      (128, (130, 200)), (128, (1, 128)), (1, (4096, 128))])
+def test_fp8_block_parity(bq, orc, dtype, br, shape):
+    for dist in ("normal", "student_t3"):
+        x = synthetic.Stream(13).tensor(shape, dtype, dist=dist)
+        e, s = bq.fp8_block_quantize(x.cuda(), br)
+        re, rs = orc.fp8_block_quantize(x, br, 128)
+        assert_bitwise(e, re, "e4m3")
+        assert_bitwise(s, rs, "scale")
+        for ydt in ("bf16", "f32"):
+            y = bq.fp8_block_dequantize(e, s, br, 128, DT[ydt])
+            assert_bitwise(y, orc.fp8_block_dequantize(re, rs, *shape, br, 128, ydtype=ydt), f"deq {ydt}")
+
+
+def test_fp8_special_values(bq, orc):
+    vals = [0.0, -0.0, float("inf"), 1.0, -1.0, 1e-30, float("nan"), 448.0]
+    x = torch.tensor(vals * 32, dtype=torch.float32).reshape(2, 128)
+    x[1] = torch.linspace(-1000, 1000, 128)
+    for br in (1, 128):
+        e, s = bq.fp8_block_quantize(x.cuda(), br)
+        re, rs = orc.fp8_block_quantize(x, br, 128)
+        assert_bitwise(s, rs, f"scale {br}")
+        assert_bitwise(e, re, f"e4m3 {br}")
+
+
+@pytest.mark.parametrize("n,k,gs,align", [(8, 32, 16, 1), (7, 32, 16, 16), (33, 64, 32, 16),
+                                          (100, 96, 16, 64), (4096, 256, 16, 16), (1, 2, 2, 1),
+                                          (130, 1000, 8, 16)])
+def test_packed_transpose_parity(bq, orc, n, k, gs, align):
+    g = np.random.default_rng(n + k)
+    w = torch.from_numpy(g.integers(0, 256, (n, k // 2), dtype=np.uint8))
+    sc = torch.from_numpy(g.integers(0, 256, (n, k // gs), dtype=np.uint8))
+    w_t, sc_t, stride = bq.packed_transpose(w.cuda(), sc.cuda(), n, k, gs, align)
+    rw, rsc, rstride = orc.packed_transpose(w, sc, n, k, gs, align)
+    assert stride == rstride
+    assert_bitwise(w_t, rw, "w_t")
+    assert_bitwise(sc_t, rsc, "sc_t")
+
+
+# ---------------------------------------------------------------- full-size workloads
+def test_workload_nvfp4(bq, orc):
+    xg = synthetic.make_workload_device("nvfp4_bf16_4096x7168")["x"]
+    x = cpu(xg)
+    packed, sc, s2 = bq.nvfp4_quantize(xg)
+    A = orc.tensor_amax(x)
+    rs2 = float(np.float32(np.float32(A) / np.float32(2688.0)))
+    assert cpu(s2).item() == rs2
+    rows = sample_rows(4096, 24, seed=3)
+    rp, rsc, _ = orc.nvfp4_quantize(x[rows], s2=rs2)
+    assert_bitwise(cpu(packed)[rows], rp, "packed")
+    assert_bitwise(cpu(sc)[rows], rsc, "block scales")
+    y = bq.nvfp4_dequantize(packed, sc, s2, torch.bfloat16)
+    assert_bitwise(cpu(y)[rows], orc.nvfp4_dequantize(rp, rsc, rs2, len(rows), 7168, "bf16"), "deq")
+    w_t, sc_t, stride = bq.packed_transpose(packed, sc, 4096, 7168, 16, 16)
+    rw, rsct, rstride = orc.packed_transpose(cpu(packed), cpu(sc), 4096, 7168, 16, 16)
+    assert stride == rstride == 4096
+    assert_bitwise(w_t, rw, "w_t")
+    assert_bitwise(sc_t, rsct, "sc_t")
+
+
+@pytest.mark.parametrize("name", ["fp8_blocks_bf16", "fp8_blocks_bf16_student_t3"])
+def test_workload_fp8_blocks(bq, orc, name):
+    act = synthetic.make_workload_device(name, only=["act"])["act"]
+    rows = sample_rows(16384, 16, seed=4)
+    acts = cpu(act[rows.cuda()])
+    e, s = bq.fp8_block_quantize(act, 1)
+    re, rs = orc.fp8_block_quantize(acts, 1, 128)
+    assert_bitwise(cpu(e)[rows], re, "act e4m3")
+    assert_bitwise(cpu(s)[rows], rs, "act scales")
+    me, ms = bq.mxfp8_quantize(act)
+    rme, rms = orc.mxfp8_quantize(acts)
+    assert_bitwise(cpu(me)[rows], rme, "mxfp8 e4m3")
+    assert_bitwise(cpu(ms)[rows], rms, "mxfp8 e8m0")
+    y = bq.fp8_block_dequantize(e, s, 1, 128, torch.bfloat16)
+    assert_bitwise(cpu(y)[rows], orc.fp8_block_dequantize(re, rs, len(rows), 7168, 1, 128, "bf16"), "deq")
+    del act, e, s, me, ms, y
+    wt = synthetic.make_workload_device(name, only=["w"])["w"]
+    e, s = bq.fp8_block_quantize(wt, 128)
+    for band in (0, 27, 55):
+        r0 = band * 128
+        re, rs = orc.fp8_block_quantize(cpu(wt[r0:r0 + 128]), 128, 128)
+        assert_bitwise(cpu(e)[r0:r0 + 128], re, f"w e4m3 band {band}")
+        assert_bitwise(cpu(s)[band], rs[0], f"w scales band {band}")
