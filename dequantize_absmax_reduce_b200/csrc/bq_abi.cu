@@ -433,21 +433,23 @@ bq_status bq_nvfp4_quantize(const void* x, bq_dtype x_dtype, int64_t n, int64_t 
     if (!is_half_or_f32(x_dtype)) return BQ_ERR_UNSUPPORTED;
     if (n < 0 || k < 0 || k % 16 != 0) return BQ_ERR_INVALID_ARG;
     if (!global_scale) return BQ_ERR_INVALID_ARG;
-    if (!static_global && (!ws || ws_bytes < 16)) return BQ_ERR_INVALID_ARG;
+    if (static_global < 0 || static_global > 2) return BQ_ERR_INVALID_ARG;
+    if (static_global != 1 && (!ws || ws_bytes < 16)) return BQ_ERR_INVALID_ARG;
     if (n * k > 0 && (!x || !packed || !scale_e4m3)) return BQ_ERR_INVALID_ARG;
-    if (!aligned(x, esize(x_dtype)) || !aligned(global_scale, 4) || (!static_global && !aligned(ws, 8)))
+    if (!aligned(x, esize(x_dtype)) || !aligned(global_scale, 4) ||
+        (static_global != 1 && !aligned(ws, 8)))
         return BQ_ERR_MISALIGNED;
     cudaStream_t s = S(stream);
     const DT dt = to_dt(x_dtype);
     unsigned long long* rec = (unsigned long long*)ws;
-    if (!static_global) {
+    if (static_global == 0) {
         if (cudaMemsetAsync(rec, 0, 16, s) != cudaSuccess) return BQ_ERR_CUDA;
         if (n * k == 0) return from_cuda(bq::set_f32(global_scale, 1.0f, s));   // zero range
         if (bq::tensor_range(dt, x, n * k, true, rec, s) != cudaSuccess) return BQ_ERR_CUDA;
     }
     if (n * k == 0) return BQ_OK;
     return from_cuda(bq::mx_quant(dt, bq::MX_NVFP4, x, n, k, packed, scale_e4m3, rec, global_scale,
-                                  static_global ? 1 : 0, s));
+                                  static_global == 1 ? 1 : 0, s));
 }
 
 bq_status bq_nvfp4_dequantize(const uint8_t* packed, const uint8_t* scale_e4m3,

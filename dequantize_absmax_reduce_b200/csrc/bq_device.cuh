@@ -22,6 +22,13 @@ template <> struct Traits<double>         { using Acc = double; static constexpr
 
 struct alignas(16) U4 { uint32_t x, y, z, w; };
 
+// Read-only 16-byte load through L1 (neighbouring lanes share sectors).
+__device__ __forceinline__ U4 ld16_nc(const void* p) {
+    U4 r;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
 // Streaming 16-byte load: read once, keep it out of L1.
 __device__ __forceinline__ U4 ld16_stream(const void* p) {
     U4 r;
@@ -156,12 +163,15 @@ __device__ __forceinline__ float div_chain(float x, const Recip& r) {
     const float e1 = __fmaf_rn(-r.s, q1, x);
     return __fmaf_rn(e1, r.y, q1);
 }
+// IEEE division kept out of line: it is the rare path, and inlining it into
+// unrolled loops only costs registers and instruction cache.
+static __device__ __noinline__ float div_slow(float x, float s) { return __fdiv_rn(x, s); }
 // Any x: falls back to IEEE division when the chain produced a NaN
 // (an infinite or overflowing operand); a NaN x stays NaN either way.
 __device__ __forceinline__ float div_any(float x, const Recip& r) {
-    if (!r.fast) return __fdiv_rn(x, r.s);
+    if (!r.fast) return div_slow(x, r.s);
     float q = div_chain(x, r);
-    if (q != q) q = __fdiv_rn(x, r.s);
+    if (q != q) q = div_slow(x, r.s);
     return q;
 }
 // Sign of a quotient of zero: x/s keeps the sign of x * s. The chain returns
@@ -174,38 +184,47 @@ __device__ __forceinline__ float with_quotient_sign(float q, float x, float s) {
 // ---------------------------------------------------------------- int codes
 // Rounding v (an exact f32 quotient) to an integer code with nearest-even:
 // for |v| <= 2^22, fl(v + 1.5*2^23) has unit spacing, so the addition itself
-// rounds v to the nearest integer (ties to even) and the integer sits in the
-// low mantissa bits. Adding (1.5*2^23 + zp) instead puts (round(v) + zp) mod
-// 256 in the low byte.
+// rounds v to the nearest integer (ties to even) and round(v) sits in the low
+// mantissa bits. The zero-point is added afterwards as an integer, so the
+// tie rule applies to round(v) itself, not to round(v) + zp.
 constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
 
 struct IntParams {
     float lo, hi;      // code range shifted by the zero-point: qmin - zp, qmax - zp
-    float magic;       // kMagic + zp
+    int zp;
 };
 __device__ __forceinline__ IntParams make_int_params(int qmin, int qmax, int zp) {
     IntParams p;
     p.lo = (float)(qmin - zp);
     p.hi = (float)(qmax - zp);
-    p.magic = kMagic + (float)zp;
+    p.zp = zp;
     return p;
 }
-// Low byte = clamp(rne(v) + zp, qmin, qmax); a NaN v gives qmin.
-__device__ __forceinline__ uint32_t code_rne(float v, const IntParams& p) {
+// fl(round(clamp(v)) + 1.5*2^23): round(v) clamped to [qmin-zp, qmax-zp], as
+// the low mantissa bits of the result. A NaN v clamps to qmin - zp.
+__device__ __forceinline__ float rounded_rne(float v, const IntParams& p) {
     v = fminf(fmaxf(v, p.lo), p.hi);            // fmaxf(NaN, lo) = lo
-    return __float_as_uint(__fadd_rn(v, p.magic));
+    return __fadd_rn(v, kMagic);
 }
 // Ties away from zero.
-__device__ __forceinline__ uint32_t code_rhaz(float v, const IntParams& p) {
+__device__ __forceinline__ float rounded_rhaz(float v, const IntParams& p) {
     v = fminf(fmaxf(v, p.lo), p.hi);
     const float t = truncf(v);
     const float d = __fsub_rn(v, t);             // exact
     const float k = (fabsf(d) >= 0.5f) ? __fadd_rn(t, copysignf(1.0f, v)) : t;
-    return __float_as_uint(__fadd_rn(k, p.magic));
+    return __fadd_rn(k, kMagic);
 }
 template <bool RHAZ>
-__device__ __forceinline__ uint32_t code_of(float v, const IntParams& p) {
-    if constexpr (RHAZ) return code_rhaz(v, p); else return code_rne(v, p);
+__device__ __forceinline__ float rounded_of(float v, const IntParams& p) {
+    if constexpr (RHAZ) return rounded_rhaz(v, p); else return rounded_rne(v, p);
+}
+// Low byte = the code clamp(round(v) + zp, qmin, qmax).
+__device__ __forceinline__ uint32_t code_from_rounded(float t, int zp) {
+    return __float_as_uint(t) + (uint32_t)zp;
+}
+// The dequantized value fl((q - zp) * s) from the rounded form.
+__device__ __forceinline__ float dequant_from_rounded(float t, float s) {
+    return __fmul_rn(__fsub_rn(t, kMagic), s);
 }
 // round(v) as a float, for the STE mask; v is clamped to [lo-1, hi+1] first
 // so that the result stays exact (a NaN v gives lo - 1: masked).

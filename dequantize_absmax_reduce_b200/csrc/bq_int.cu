@@ -85,7 +85,7 @@ struct DynArgs {
     const void* x;
     int64_t n_seg;
     int G;          // elements per group (multiple of VEC)
-    int team;       // lanes per group when NV == 1 (power of two <= 32)
+    int team;       // lanes per group (power of two <= 32), warp kernels
     IntCfg cfg;
     uint8_t* q;
     void* y;
@@ -93,21 +93,23 @@ struct DynArgs {
     uint8_t* zp;
 };
 
-// One group's codes (and fake-quantized values) from its vectors. `lane_vec`
-// gives the element offset of vector j for this lane.
+// Codes (QUANT) or fake-quantized values (FAKE) of one 16-byte vector.
 template <class T, int OP, bool FAST>
 __device__ __forceinline__ void emit_vec(const U4& raw, const Recip& R, const IntParams& ip,
                                          int64_t off, const DynArgs& a) {
     constexpr int VEC = Traits<T>::VEC;
     float v[VEC];
     load_vec<T>(raw, v);
-    uint32_t cw[VEC];
+    float t[VEC];
 #pragma unroll
     for (int i = 0; i < VEC; ++i) {
-        const float qv = FAST ? div_chain(v[i], R) : __fdiv_rn(v[i], R.s);
-        cw[i] = code_rne(qv, ip);
+        const float qv = FAST ? div_chain(v[i], R) : div_slow(v[i], R.s);
+        t[i] = rounded_rne(qv, ip);
     }
     if constexpr (OP == OP_QUANT) {
+        uint32_t cw[VEC];
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) cw[i] = code_from_rounded(t[i], ip.zp);
         if constexpr (VEC == 8) {
             st8(a.q + off, pack4_lowbytes(cw[0], cw[1], cw[2], cw[3]),
                 pack4_lowbytes(cw[4], cw[5], cw[6], cw[7]));
@@ -117,8 +119,7 @@ __device__ __forceinline__ void emit_vec(const U4& raw, const Recip& R, const In
     } else {
         float o[VEC];
 #pragma unroll
-        for (int i = 0; i < VEC; ++i)
-            o[i] = __fmul_rn(__fsub_rn(__uint_as_float(cw[i]), ip.magic), R.s);
+        for (int i = 0; i < VEC; ++i) o[i] = dequant_from_rounded(t[i], R.s);
         st16((T*)a.y + off, pack_vec<T>(o));
     }
 }
@@ -139,14 +140,13 @@ __device__ __forceinline__ void range_vec(const U4& raw, bool sym, float& hi, fl
     }
 }
 
-// NV vectors per lane; NV == 1 allows teams of `a.team` lanes, NV > 1 uses
-// whole warps. SEGS groups per team per iteration keep several loads in
-// flight when groups are small.
+// Groups of up to team*NV vectors: `a.team` lanes per group, NV vectors per
+// lane, SEGS groups per team per iteration (all their loads issued first).
 template <class T, int OP, int NV, int SEGS, bool SYM>
 __global__ void __launch_bounds__(256) k_int_dyn_warp(DynArgs a) {
     constexpr int VEC = Traits<T>::VEC;
     const T* __restrict__ x = (const T*)a.x;
-    const int team = (NV == 1) ? a.team : 32;
+    const int team = a.team;
     const int tpw = 32 / team;
     const int lane = threadIdx.x & 31;
     const int tm = lane / team;
@@ -164,7 +164,7 @@ __global__ void __launch_bounds__(256) k_int_dyn_warp(DynArgs a) {
 #pragma unroll
             for (int j = 0; j < NV; ++j) {
                 const int e = (j * team + l) * VEC;
-                if (seg < a.n_seg && e < a.G) raw[r][j] = ld16_stream(x + seg * a.G + e);
+                if (seg < a.n_seg && e < a.G) raw[r][j] = ld16_nc(x + seg * a.G + e);
                 else raw[r][j] = U4{0u, 0u, 0u, 0u};
             }
         }
@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(256) k_int_dyn_warp(DynArgs a) {
                 a.scale[seg] = g.s;
                 if (a.zp) a.zp[seg] = (uint8_t)g.zp;
             }
-            const IntParams ip = make_int_params(a.cfg.qmin, a.cfg.qmax, g.zp);
+            const IntParams ip = make_int_params(a.cfg.qmin, a.cfg.qmax, SYM ? 0 : g.zp);
             const Recip R = make_recip(g.s);
             if (R.fast) {
 #pragma unroll
@@ -203,57 +203,74 @@ __global__ void __launch_bounds__(256) k_int_dyn_warp(DynArgs a) {
     }
 }
 
-// A CTA of NTH threads per group, NV vectors per thread.
-template <class T, int OP, int NTH, int NV, bool SYM>
-__global__ void __launch_bounds__(NTH) k_int_dyn_cta(DynArgs a) {
+// A CTA of 256 threads per group, NV vectors per thread; while one group is
+// reduced and written, the loads of the CTA's next group are in flight.
+template <class T, int OP, int NV, bool SYM>
+__device__ __forceinline__ void cta_load(const T* __restrict__ x, int64_t seg, int G, U4 (&raw)[NV]) {
     constexpr int VEC = Traits<T>::VEC;
-    constexpr int NW = NTH / 32;
-    __shared__ float sh_hi[2][NW], sh_nlo[2][NW];
-    const T* __restrict__ x = (const T*)a.x;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+        const int e = (j * 256 + (int)threadIdx.x) * VEC;
+        raw[j] = (e < G) ? ld16_stream(x + seg * G + e) : U4{0u, 0u, 0u, 0u};
+    }
+}
+
+template <class T, int OP, int NV, bool SYM>
+__device__ __forceinline__ void cta_group(const U4 (&raw)[NV], int64_t seg, int par,
+                                          float (*sh)[2][8], const DynArgs& a) {
+    constexpr int VEC = Traits<T>::VEC;
     const int tid = threadIdx.x, wid = tid >> 5, lane = tid & 31;
-    int par = 0;
-    for (int64_t seg = blockIdx.x; seg < a.n_seg; seg += gridDim.x, par ^= 1) {
-        U4 raw[NV];
+    float hi = 0.0f, nlo = 0.0f;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) range_vec<T>(raw[j], SYM, hi, nlo);
+    hi = warp_max(hi);
+    if (!SYM) nlo = warp_max(nlo);
+    if (lane == 0) { sh[par][0][wid] = hi; sh[par][1][wid] = nlo; }
+    __syncthreads();
+    hi = sh[par][0][0];
+    nlo = sh[par][1][0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) {
+        hi = fmaxf(hi, sh[par][0][w]);
+        if (!SYM) nlo = fmaxf(nlo, sh[par][1][w]);
+    }
+    if (SYM) nlo = 0.0f;
+    const GroupF g = derive_f(hi, nlo, a.cfg);
+    if (tid == 0) {
+        a.scale[seg] = g.s;
+        if (a.zp) a.zp[seg] = (uint8_t)g.zp;
+    }
+    const IntParams ip = make_int_params(a.cfg.qmin, a.cfg.qmax, SYM ? 0 : g.zp);
+    const Recip R = make_recip(g.s);
+    if (R.fast) {
 #pragma unroll
         for (int j = 0; j < NV; ++j) {
-            const int e = (j * NTH + tid) * VEC;
-            raw[j] = (e < a.G) ? ld16_stream(x + seg * a.G + e) : U4{0u, 0u, 0u, 0u};
+            const int e = (j * 256 + tid) * VEC;
+            if (e < a.G) emit_vec<T, OP, true>(raw[j], R, ip, seg * a.G + e, a);
         }
-        float hi = 0.0f, nlo = 0.0f;
+    } else {
 #pragma unroll
-        for (int j = 0; j < NV; ++j) range_vec<T>(raw[j], SYM, hi, nlo);
-        hi = warp_max(hi);
-        if (!SYM) nlo = warp_max(nlo);
-        if (lane == 0) { sh_hi[par][wid] = hi; sh_nlo[par][wid] = nlo; }
-        __syncthreads();
-        hi = sh_hi[par][0];
-        nlo = sh_nlo[par][0];
-#pragma unroll
-        for (int w = 1; w < NW; ++w) {
-            hi = fmaxf(hi, sh_hi[par][w]);
-            if (!SYM) nlo = fmaxf(nlo, sh_nlo[par][w]);
+        for (int j = 0; j < NV; ++j) {
+            const int e = (j * 256 + tid) * VEC;
+            if (e < a.G) emit_vec<T, OP, false>(raw[j], R, ip, seg * a.G + e, a);
         }
-        if (SYM) nlo = 0.0f;
-        const GroupF g = derive_f(hi, nlo, a.cfg);
-        if (tid == 0) {
-            a.scale[seg] = g.s;
-            if (a.zp) a.zp[seg] = (uint8_t)g.zp;
-        }
-        const IntParams ip = make_int_params(a.cfg.qmin, a.cfg.qmax, g.zp);
-        const Recip R = make_recip(g.s);
-        if (R.fast) {
-#pragma unroll
-            for (int j = 0; j < NV; ++j) {
-                const int e = (j * NTH + tid) * VEC;
-                if (e < a.G) emit_vec<T, OP, true>(raw[j], R, ip, seg * a.G + e, a);
-            }
-        } else {
-#pragma unroll
-            for (int j = 0; j < NV; ++j) {
-                const int e = (j * NTH + tid) * VEC;
-                if (e < a.G) emit_vec<T, OP, false>(raw[j], R, ip, seg * a.G + e, a);
-            }
-        }
+    }
+}
+
+template <class T, int OP, int NV, bool SYM>
+__global__ void __launch_bounds__(256) k_int_dyn_cta(DynArgs a) {
+    __shared__ float sh[2][2][8];          // [parity][hi / nlo][warp]
+    const T* __restrict__ x = (const T*)a.x;
+    const int64_t G = gridDim.x;
+    U4 A[NV], B[NV];
+    int64_t seg = blockIdx.x;
+    if (seg < a.n_seg) cta_load<T, OP, NV, SYM>(x, seg, a.G, A);
+    for (; seg < a.n_seg; seg += 2 * G) {
+        const int64_t s1 = seg + G, s2 = seg + 2 * G;
+        if (s1 < a.n_seg) cta_load<T, OP, NV, SYM>(x, s1, a.G, B);
+        cta_group<T, OP, NV, SYM>(A, seg, 0, sh, a);
+        if (s2 < a.n_seg) cta_load<T, OP, NV, SYM>(x, s2, a.G, A);
+        if (s1 < a.n_seg) cta_group<T, OP, NV, SYM>(B, s1, 1, sh, a);
     }
 }
 
@@ -315,9 +332,9 @@ template <int OP, bool RHAZ>
 __device__ __forceinline__ float elem_f(float xa, float xb, const GState& st, uint32_t* code) {
     if constexpr (OP == OP_QUANT || OP == OP_FAKE) {
         const float v = div_any(xa, st.R);
-        const uint32_t c = code_of<RHAZ>(v, st.ip);
-        *code = c;
-        if constexpr (OP == OP_FAKE) return __fmul_rn(__fsub_rn(__uint_as_float(c), st.ip.magic), st.s);
+        const float t = rounded_of<RHAZ>(v, st.ip);
+        *code = code_from_rounded(t, st.ip.zp);
+        if constexpr (OP == OP_FAKE) return dequant_from_rounded(t, st.s);
         return 0.0f;
     } else if constexpr (OP == OP_QBWD || OP == OP_FBWD) {
         const float v = div_any(xa, st.R);
@@ -346,7 +363,7 @@ __device__ __forceinline__ double elem_d(double xa, double xb, const GState& st,
         double k = RHAZ ? round(v) : rint(v);
         k = fmin(fmax(k, lo), hi);                  // NaN -> lo
         *code = (uint32_t)((int)k + st.zp);
-        if constexpr (OP == OP_FAKE) return k * s;
+        if constexpr (OP == OP_FAKE) return (double)((int)k) * s;   // (q - zp) as an integer: +0, never -0
         return 0.0;
     } else if constexpr (OP == OP_QBWD || OP == OP_FBWD) {
         const double v = xa / s;
@@ -372,79 +389,122 @@ __device__ __forceinline__ float deq_code_f(uint32_t word, int i, const GState& 
     return __fmul_rn(__fsub_rn(f, off), st.s);
 }
 
+// Items of W elements (one 16-byte vector, or one element); each warp takes
+// contiguous chunks of 32*U items, lane l the items l, l+32, ..., so every
+// load instruction is coalesced and a lane's items rarely change group. All
+// U items' loads are issued before any of them is computed.
 template <class T, int OP, int PSRC, bool VECP, bool RHAZ>
 __global__ void __launch_bounds__(256) k_int_map(MapArgs a) {
     using Acc = typename Traits<T>::Acc;
     constexpr bool WIDE = std::is_same<Acc, double>::value;
     constexpr int W = VECP ? Traits<T>::VEC : 1;
+    constexpr int U = (OP == OP_DEQ) ? 8 : 4;
+    constexpr bool TWO = (OP == OP_QBWD || OP == OP_FBWD);
+    const int lane = threadIdx.x & 31;
+    const int64_t gwarp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     const int64_t n_items = a.numel / W;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t n_chunks = (n_items + 32 * U - 1) / (32 * U);
     GState st;
     st.seg = -1;
-    for (int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; it < n_items; it += stride) {
-        const int64_t e0 = it * W;
-        const int64_t seg = a.use_fd ? (int64_t)fdiv((uint32_t)e0, a.fd) : e0 / a.G;
-        if (seg != st.seg) load_group<T, PSRC>(a, seg, e0 == seg * a.G, st);
-
+    for (int64_t c = gwarp; c < n_chunks; c += nwarps) {
+        const int64_t it0 = c * 32 * U + lane;
         if constexpr (OP == OP_DEQ) {
-            // a: codes (bytes); out: T
-            const uint8_t* qb = (const uint8_t*)a.a + e0;
-            Acc o[W];
-            if constexpr (W == 8) {
-                const uint2 w2 = __ldg(reinterpret_cast<const uint2*>(qb));
+            // codes: W bytes per item
+            uint32_t cw[U][(W + 3) / 4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) o[i] = deq_code_f(w2.x, i, st, a.cfg.q_signed);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) o[4 + i] = deq_code_f(w2.y, i, st, a.cfg.q_signed);
-            } else if constexpr (W == 4) {
-                const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(qb));
-#pragma unroll
-                for (int i = 0; i < 4; ++i) o[i] = deq_code_f(w, i, st, a.cfg.q_signed);
-            } else {
-#pragma unroll
-                for (int i = 0; i < W; ++i) {
-                    const uint8_t b = __ldg(qb + i);
-                    const int qv = a.cfg.q_signed ? (int)(int8_t)b : (int)b;
-                    if constexpr (WIDE) o[i] = (double)(qv - st.zp) * (double)st.s;
-                    else o[i] = __fmul_rn((float)(qv - st.zp), st.s);
+            for (int u = 0; u < U; ++u) {
+                const int64_t it = it0 + (int64_t)u * 32;
+                const uint8_t* qb = (const uint8_t*)a.a + it * W;
+                if (it < n_items) {
+                    if constexpr (W == 8) {
+                        const uint2 w2 = __ldg(reinterpret_cast<const uint2*>(qb));
+                        cw[u][0] = w2.x; cw[u][1] = w2.y;
+                    } else if constexpr (W == 4) {
+                        cw[u][0] = __ldg(reinterpret_cast<const uint32_t*>(qb));
+                    } else if constexpr (W == 2) {
+                        cw[u][0] = __ldg(reinterpret_cast<const unsigned short*>(qb));
+                    } else {
+                        cw[u][0] = __ldg(qb);
+                    }
                 }
             }
-            if constexpr (VECP) {
-                st16((T*)a.out + e0, pack_vec<T>(o));
-            } else {
-                ((T*)a.out)[e0] = to_out<T>(o[0]);
-            }
-        } else {
-            Acc xa[W], xb[W];
-            if constexpr (VECP) {
-                load_vec<T>(ld16_stream((const T*)a.a + e0), xa);
-                if constexpr (OP == OP_QBWD || OP == OP_FBWD)
-                    load_vec<T>(ld16_stream((const T*)a.b + e0), xb);
-            } else {
-                xa[0] = ld1<T>((const T*)a.a + e0);
-                if constexpr (OP == OP_QBWD || OP == OP_FBWD) xb[0] = ld1<T>((const T*)a.b + e0);
-            }
-            Acc o[W];
-            uint32_t cw[W];
 #pragma unroll
-            for (int i = 0; i < W; ++i) {
-                if constexpr (WIDE) o[i] = elem_d<OP, RHAZ>(xa[i], (OP == OP_QBWD || OP == OP_FBWD) ? xb[i] : 0.0, st, &cw[i]);
-                else o[i] = elem_f<OP, RHAZ>(xa[i], (OP == OP_QBWD || OP == OP_FBWD) ? xb[i] : 0.0f, st, &cw[i]);
-            }
-            if constexpr (OP == OP_QUANT) {
-                uint8_t* q = (uint8_t*)a.out + e0;
-                if constexpr (W == 8) {
-                    st8(q, pack4_lowbytes(cw[0], cw[1], cw[2], cw[3]),
-                        pack4_lowbytes(cw[4], cw[5], cw[6], cw[7]));
-                } else if constexpr (W == 4) {
-                    st4(q, pack4_lowbytes(cw[0], cw[1], cw[2], cw[3]));
+            for (int u = 0; u < U; ++u) {
+                const int64_t it = it0 + (int64_t)u * 32;
+                if (it >= n_items) continue;
+                const int64_t e0 = it * W;
+                const int64_t seg = a.use_fd ? (int64_t)fdiv((uint32_t)e0, a.fd) : e0 / a.G;
+                if (seg != st.seg) load_group<T, PSRC>(a, seg, false, st);
+                Acc o[W];
+                if constexpr (!WIDE && (W == 8 || W == 4)) {
+#pragma unroll
+                    for (int i = 0; i < W; ++i) o[i] = deq_code_f(cw[u][i / 4], i % 4, st, a.cfg.q_signed);
                 } else {
 #pragma unroll
-                    for (int i = 0; i < W; ++i) q[i] = (uint8_t)cw[i];
+                    for (int i = 0; i < W; ++i) {
+                        const uint32_t b = (cw[u][0] >> (8 * i)) & 0xFFu;
+                        const int qv = a.cfg.q_signed ? (int)(int8_t)b : (int)b;
+                        if constexpr (WIDE) o[i] = (double)(qv - st.zp) * (double)st.s;
+                        else o[i] = __fmul_rn((float)(qv - st.zp), st.s);
+                    }
                 }
-            } else {
                 if constexpr (VECP) st16((T*)a.out + e0, pack_vec<T>(o));
                 else ((T*)a.out)[e0] = to_out<T>(o[0]);
+            }
+        } else {
+            U4 ra[U], rb[TWO ? U : 1];
+            Acc sa[U], sb[TWO ? U : 1];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t it = it0 + (int64_t)u * 32;
+                if (it < n_items) {
+                    if constexpr (VECP) {
+                        ra[u] = ld16_stream((const T*)a.a + it * W);
+                        if constexpr (TWO) rb[u] = ld16_stream((const T*)a.b + it * W);
+                    } else {
+                        sa[u] = ld1<T>((const T*)a.a + it);
+                        if constexpr (TWO) sb[u] = ld1<T>((const T*)a.b + it);
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t it = it0 + (int64_t)u * 32;
+                if (it >= n_items) continue;
+                const int64_t e0 = it * W;
+                const int64_t seg = a.use_fd ? (int64_t)fdiv((uint32_t)e0, a.fd) : e0 / a.G;
+                if (seg != st.seg) load_group<T, PSRC>(a, seg, e0 == seg * a.G, st);
+                Acc xa[W], xb[W];
+                if constexpr (VECP) {
+                    load_vec<T>(ra[u], xa);
+                    if constexpr (TWO) load_vec<T>(rb[u], xb);
+                } else {
+                    xa[0] = sa[u];
+                    if constexpr (TWO) xb[0] = sb[u];
+                }
+                Acc o[W];
+                uint32_t cw[W];
+#pragma unroll
+                for (int i = 0; i < W; ++i) {
+                    if constexpr (WIDE) o[i] = elem_d<OP, RHAZ>(xa[i], TWO ? xb[i] : 0.0, st, &cw[i]);
+                    else o[i] = elem_f<OP, RHAZ>(xa[i], TWO ? xb[i] : 0.0f, st, &cw[i]);
+                }
+                if constexpr (OP == OP_QUANT) {
+                    uint8_t* q = (uint8_t*)a.out + e0;
+                    if constexpr (W == 8) {
+                        st8(q, pack4_lowbytes(cw[0], cw[1], cw[2], cw[3]),
+                            pack4_lowbytes(cw[4], cw[5], cw[6], cw[7]));
+                    } else if constexpr (W == 4) {
+                        st4(q, pack4_lowbytes(cw[0], cw[1], cw[2], cw[3]));
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < W; ++i) q[i] = (uint8_t)cw[i];
+                    }
+                } else {
+                    if constexpr (VECP) st16((T*)a.out + e0, pack_vec<T>(o));
+                    else ((T*)a.out)[e0] = to_out<T>(o[0]);
+                }
             }
         }
     }
@@ -601,6 +661,26 @@ int sm_count() {
     return v;
 }
 
+// Resident blocks per SM of a kernel at `threads` threads (occupancy API).
+template <class K>
+static int resident_blocks(K kernel, int threads) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0) != cudaSuccess || n < 1) {
+        (void)cudaGetLastError();
+        n = 1;
+    }
+    return n;
+}
+
+// Persistent grid: enough blocks for the work, at most one full wave.
+template <class K>
+static unsigned grid_occ(K kernel, int threads, int64_t need_blocks) {
+    static const int bps = resident_blocks(kernel, threads);
+    const int64_t cap = (int64_t)sm_count() * bps;
+    if (need_blocks < 1) need_blocks = 1;
+    return (unsigned)(need_blocks < cap ? need_blocks : cap);
+}
+
 static unsigned grid_for(int64_t work_items, int per_block, int blocks_per_sm) {
     int64_t need = (work_items + per_block - 1) / per_block;
     int64_t cap = (int64_t)sm_count() * blocks_per_sm;
@@ -608,39 +688,38 @@ static unsigned grid_for(int64_t work_items, int per_block, int blocks_per_sm) {
     return (unsigned)(need < cap ? need : cap);
 }
 
+template <class T, int OP, int NV, int SEGS, bool SYM>
+static void launch_warp(DynArgs a, int team, cudaStream_t st) {
+    a.team = team;
+    const int64_t per_warp = (int64_t)(32 / team) * SEGS;
+    const int64_t warps = (a.n_seg + per_warp - 1) / per_warp;
+    auto k = k_int_dyn_warp<T, OP, NV, SEGS, SYM>;
+    k<<<grid_occ(k, 256, (warps + 7) / 8), 256, 0, st>>>(a);
+}
+
+template <class T, int OP, int NV, bool SYM>
+static void launch_cta(const DynArgs& a, cudaStream_t st) {
+    auto k = k_int_dyn_cta<T, OP, NV, SYM>;
+    k<<<grid_occ(k, 256, a.n_seg), 256, 0, st>>>(a);
+}
+
+// Register-resident configurations by vectors per group U: small groups
+// give each lane several vectors (fewer lanes share a group), large ones a
+// CTA of 256 threads.
 template <class T, int OP, bool SYM>
-static cudaError_t launch_dyn_t(const DynArgs& a0, cudaStream_t st) {
+static cudaError_t launch_dyn_t(const DynArgs& a, cudaStream_t st) {
     constexpr int VEC = Traits<T>::VEC;
-    DynArgs a = a0;
-    const int64_t U = a.G / VEC;          // vectors per group
-    if (U <= 32) {
-        int team = 1;
-        while (team < U) team <<= 1;
-        a.team = team;
-        const int64_t groups_per_warp = (32 / team) * 4;
-        const int64_t warps = (a.n_seg + groups_per_warp - 1) / groups_per_warp;
-        k_int_dyn_warp<T, OP, 1, 4, SYM><<<grid_for(warps * 32, 256, 8), 256, 0, st>>>(a);
-    } else if (U <= 64) {
-        a.team = 32;
-        k_int_dyn_warp<T, OP, 2, 2, SYM><<<grid_for(((a.n_seg + 1) / 2) * 32, 256, 8), 256, 0, st>>>(a);
-    } else if (U <= 128) {
-        a.team = 32;
-        k_int_dyn_warp<T, OP, 4, 1, SYM><<<grid_for(a.n_seg * 32, 256, 8), 256, 0, st>>>(a);
-    } else if (U <= 256) {
-        a.team = 32;
-        k_int_dyn_warp<T, OP, 8, 1, SYM><<<grid_for(a.n_seg * 32, 256, 8), 256, 0, st>>>(a);
-    } else if (U <= 512) {
-        a.team = 32;
-        k_int_dyn_warp<T, OP, 16, 1, SYM><<<grid_for(a.n_seg * 32, 256, 6), 256, 0, st>>>(a);
-    } else if (U <= 1024) {
-        k_int_dyn_cta<T, OP, 256, 4, SYM><<<grid_for(a.n_seg, 1, 8), 256, 0, st>>>(a);
-    } else if (U <= 2048) {
-        k_int_dyn_cta<T, OP, 256, 8, SYM><<<grid_for(a.n_seg, 1, 6), 256, 0, st>>>(a);
-    } else if (U <= 4096) {
-        k_int_dyn_cta<T, OP, 256, 16, SYM><<<grid_for(a.n_seg, 1, 3), 256, 0, st>>>(a);
-    } else {
-        return cudaErrorNotSupported;
-    }
+    const int64_t U = a.G / VEC;
+    auto pow2 = [](int64_t v) { int t = 1; while (t < v) t <<= 1; return t; };
+    if (U == 1)            launch_warp<T, OP, 1, 8, SYM>(a, 1, st);
+    else if (U == 2)       launch_warp<T, OP, 2, 4, SYM>(a, 1, st);
+    else if (U <= 128)     launch_warp<T, OP, 4, 2, SYM>(a, pow2((U + 3) / 4), st);
+    else if (U <= 256)     launch_cta<T, OP, 1, SYM>(a, st);
+    else if (U <= 512)     launch_cta<T, OP, 2, SYM>(a, st);
+    else if (U <= 1024)    launch_cta<T, OP, 4, SYM>(a, st);
+    else if (U <= 2048)    launch_cta<T, OP, 8, SYM>(a, st);
+    else if (U <= 4096)    launch_cta<T, OP, 16, SYM>(a, st);
+    else return cudaErrorNotSupported;
     return cudaGetLastError();
 }
 
@@ -676,9 +755,15 @@ cudaError_t int_dyn(DT dt, int op, const void* x, SegView sv, IntCfg cfg, void* 
 template <class T, int OP, int PSRC, bool VECP>
 static cudaError_t launch_map4(const MapArgs& a, cudaStream_t st) {
     const int W = VECP ? Traits<T>::VEC : 1;
-    const unsigned grid = grid_for(a.numel / W, 256, 8);
-    if (a.cfg.rhaz) k_int_map<T, OP, PSRC, VECP, true><<<grid, 256, 0, st>>>(a);
-    else k_int_map<T, OP, PSRC, VECP, false><<<grid, 256, 0, st>>>(a);
+    const int U = (OP == OP_DEQ) ? 8 : 4;
+    const int64_t chunks = (a.numel / W + 32 * U - 1) / (32 * U);
+    if (a.cfg.rhaz) {
+        auto k = k_int_map<T, OP, PSRC, VECP, true>;
+        k<<<grid_occ(k, 256, (chunks + 7) / 8), 256, 0, st>>>(a);
+    } else {
+        auto k = k_int_map<T, OP, PSRC, VECP, false>;
+        k<<<grid_occ(k, 256, (chunks + 7) / 8), 256, 0, st>>>(a);
+    }
     return cudaGetLastError();
 }
 

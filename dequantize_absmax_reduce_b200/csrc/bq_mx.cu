@@ -54,7 +54,7 @@ __device__ __forceinline__ int mx_exponent(float a) {
     return min(max(fl2 - 8, -127), 127);
 }
 
-// Codes of one lane's VEC elements (v: values, out: packed bytes).
+// Codes of one 16-byte vector (v: its VEC values) written at dst.
 template <class T, int FMT, bool FAST>
 __device__ __forceinline__ void mx_emit(const float* v, const Recip& R, float mul, bool zero,
                                         uint8_t* dst) {
@@ -71,12 +71,11 @@ __device__ __forceinline__ void mx_emit(const float* v, const Recip& R, float mu
     }
     if constexpr (FMT == MX_NVFP4) {
         if constexpr (VEC == 8) {
-            const uint32_t w = zero ? 0u : e2m1x8(*reinterpret_cast<const float(*)[8]>(t));
-            st4(dst, w);
+            const float (&t8)[8] = *reinterpret_cast<const float(*)[8]>(t);
+            st4(dst, zero ? 0u : e2m1x8(t8));
         } else {
             float t8[8] = {t[0], t[1], t[2], t[3], 0.f, 0.f, 0.f, 0.f};
-            const uint32_t w = zero ? 0u : e2m1x8(t8);
-            st2(dst, w & 0xFFFFu);
+            st2(dst, zero ? 0u : (e2m1x8(t8) & 0xFFFFu));
         }
     } else {
         if constexpr (VEC == 8) {
@@ -87,13 +86,24 @@ __device__ __forceinline__ void mx_emit(const float* v, const Recip& R, float mu
     }
 }
 
-template <class T, int FMT, int SEGS>
+// Lanes per group and vectors per lane for each format / element size: each
+// lane holds NV vectors of its group so that the per-group work (amax
+// shuffles, scale, reciprocal) is shared by many elements.
+template <class T, int FMT> struct MxShape {
+    static constexpr int VEC = Traits<T>::VEC;
+    static constexpr int U = MxG<FMT>::G / VEC;              // vectors per group
+    static constexpr int NV = (U >= 4) ? 4 : U;
+    static constexpr int TEAM = U / NV;
+    static constexpr int SEGS = (NV == 2) ? 4 : 2;
+};
+
+template <class T, int FMT>
 __global__ void __launch_bounds__(256) k_mx_quant(MxArgs a) {
-    constexpr int VEC = Traits<T>::VEC;
+    using S = MxShape<T, FMT>;
+    constexpr int VEC = S::VEC, NV = S::NV, TEAM = S::TEAM, SEGS = S::SEGS;
     constexpr int G = MxG<FMT>::G;
-    constexpr int TEAM = G / VEC;
     constexpr int TPW = 32 / TEAM;
-    constexpr int CB = (FMT == MX_NVFP4) ? VEC / 2 : VEC;   // code bytes per lane
+    constexpr int CB = (FMT == MX_NVFP4) ? VEC / 2 : VEC;   // code bytes per vector
     const T* __restrict__ x = (const T*)a.x;
     const int lane = threadIdx.x & 31;
     const int tm = lane / TEAM, l = lane % TEAM;
@@ -119,47 +129,65 @@ __global__ void __launch_bounds__(256) k_mx_quant(MxArgs a) {
     }
 
     for (int64_t c = gwarp; c < n_chunks; c += nwarps) {
-        U4 raw[SEGS];
+        U4 raw[SEGS][NV];
 #pragma unroll
         for (int r = 0; r < SEGS; ++r) {
             const int64_t seg = c * per_chunk + r * TPW + tm;
-            raw[r] = (seg < a.n_seg) ? ld16_stream(x + seg * G + l * VEC) : U4{0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int j = 0; j < NV; ++j)
+                raw[r][j] = (seg < a.n_seg) ? ld16_nc(x + seg * G + (j * TEAM + l) * VEC)
+                                            : U4{0u, 0u, 0u, 0u};
         }
 #pragma unroll
         for (int r = 0; r < SEGS; ++r) {
             const int64_t seg = c * per_chunk + r * TPW + tm;
-            float v[VEC];
-            load_vec<T>(raw[r], v);
+            float v[NV][VEC];
             float am = 0.0f;
 #pragma unroll
-            for (int i = 0; i < VEC; ++i) am = fmaxf(am, fabsf(v[i]));
+            for (int j = 0; j < NV; ++j) {
+                load_vec<T>(raw[r][j], v[j]);
+#pragma unroll
+                for (int i = 0; i < VEC; ++i) am = fmaxf(am, fabsf(v[j][i]));
+            }
 #pragma unroll
             for (int o = TEAM / 2; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
             const bool ok = seg < a.n_seg;
-            uint8_t* dst = a.codes + seg * (G * CB / VEC) + l * CB;
+            uint8_t* base = a.codes + seg * (G / VEC) * CB;
             if constexpr (FMT == MX_FP8_1x128) {
                 float s = __fdiv_rn(am, 448.0f);
                 if (s == 0.0f) s = 1.0f;
                 if (ok && l == 0) ((float*)a.scales)[seg] = s;
                 const Recip R = make_recip(s);
                 if (ok) {
-                    if (R.fast) mx_emit<T, FMT, true>(v, R, 0.f, false, dst);
-                    else mx_emit<T, FMT, false>(v, R, 0.f, false, dst);
+#pragma unroll
+                    for (int j = 0; j < NV; ++j) {
+                        if (R.fast) mx_emit<T, FMT, true>(v[j], R, 0.f, false, base + (j * TEAM + l) * CB);
+                        else mx_emit<T, FMT, false>(v[j], R, 0.f, false, base + (j * TEAM + l) * CB);
+                    }
                 }
             } else if constexpr (FMT == MX_MXFP8) {
                 const int E = mx_exponent(am);
                 if (ok && l == 0) ((uint8_t*)a.scales)[seg] = (uint8_t)(E + 127);
-                Recip R{};
-                if (ok) mx_emit<T, FMT, true>(v, R, exp2i(-E), false, dst);
+                const Recip R{};
+                const float mul = exp2i(-E);
+                if (ok) {
+#pragma unroll
+                    for (int j = 0; j < NV; ++j)
+                        mx_emit<T, FMT, true>(v[j], R, mul, false, base + (j * TEAM + l) * CB);
+                }
             } else {
                 const float q6 = div_any(am, R6);                 // a_b / (6 s2)
                 const uint32_t sb = e4m3x2(q6, 0.0f) & 0xFFu;
                 if (ok && l == 0) ((uint8_t*)a.scales)[seg] = (uint8_t)sb;
                 const float eff = __fmul_rn(e4m3_to_f32(sb), s2);
                 const Recip R = make_recip(eff);
+                const bool fast = R.fast && !a.static_global;
                 if (ok) {
-                    if (R.fast && !a.static_global) mx_emit<T, FMT, true>(v, R, 0.f, eff == 0.0f, dst);
-                    else mx_emit<T, FMT, false>(v, R, 0.f, eff == 0.0f, dst);
+#pragma unroll
+                    for (int j = 0; j < NV; ++j) {
+                        if (fast) mx_emit<T, FMT, true>(v[j], R, 0.f, eff == 0.0f, base + (j * TEAM + l) * CB);
+                        else mx_emit<T, FMT, false>(v[j], R, 0.f, eff == 0.0f, base + (j * TEAM + l) * CB);
+                    }
                 }
             }
         }
@@ -397,15 +425,28 @@ static unsigned grid_cap(int64_t need_blocks, int per_sm) {
     return (unsigned)(need_blocks < cap ? need_blocks : cap);
 }
 
+template <class K>
+static unsigned grid_occ_mx(K kernel, int64_t need_blocks) {
+    static int bps = 0;
+    if (bps == 0) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, 256, 0) != cudaSuccess || n < 1) {
+            (void)cudaGetLastError();
+            n = 1;
+        }
+        bps = n;
+    }
+    return grid_cap(need_blocks, bps);
+}
+
 template <class T, int FMT>
 static cudaError_t launch_mx_quant_t(const MxArgs& a, bool vec, cudaStream_t st) {
-    constexpr int VEC = Traits<T>::VEC;
-    constexpr int G = MxG<FMT>::G;
-    constexpr int TPW = 32 / (G / VEC);
+    using S = MxShape<T, FMT>;
     if (vec) {
-        constexpr int SEGS = (G / VEC >= 16) ? 2 : 4;
-        const int64_t warps = (a.n_seg + (int64_t)SEGS * TPW - 1) / ((int64_t)SEGS * TPW);
-        k_mx_quant<T, FMT, SEGS><<<grid_cap((warps + 7) / 8, 8), 256, 0, st>>>(a);
+        const int64_t per_warp = (int64_t)S::SEGS * (32 / S::TEAM);
+        const int64_t warps = (a.n_seg + per_warp - 1) / per_warp;
+        auto k = k_mx_quant<T, FMT>;
+        k<<<grid_occ_mx(k, (warps + 7) / 8), 256, 0, st>>>(a);
     } else {
         k_mx_quant_scalar<T, FMT><<<grid_cap((a.n_seg + 255) / 256, 8), 256, 0, st>>>(a);
     }
@@ -476,9 +517,13 @@ static cudaError_t launch_deq_t(const DeqArgs& a, cudaStream_t st) {
     const int cin = (FMT == MX_NVFP4) ? 8 : 16;   // code bytes per 16 elements
     const bool vec = (a.k % 16 == 0) && al(a.y, 16) && al(a.codes, cin);
     const int64_t items = vec ? a.numel / 16 : a.numel;
-    const unsigned grid = grid_cap((items + 255) / 256, 8);
-    if (vec) k_mx_deq<T, FMT, true><<<grid, 256, 0, st>>>(a);
-    else k_mx_deq<T, FMT, false><<<grid, 256, 0, st>>>(a);
+    if (vec) {
+        auto k = k_mx_deq<T, FMT, true>;
+        k<<<grid_occ_mx(k, (items + 255) / 256), 256, 0, st>>>(a);
+    } else {
+        auto k = k_mx_deq<T, FMT, false>;
+        k<<<grid_occ_mx(k, (items + 255) / 256), 256, 0, st>>>(a);
+    }
     return cudaGetLastError();
 }
 

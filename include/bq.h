@@ -232,16 +232,19 @@ bq_status bq_dequantize_per_group_backward(const void* dy, const float* scale,
 
 /* ----------------------------------------------------------------- NVFP4 */
 /* [QuantizedWeight] NVFP4 quantize of x [n, k] (F32, F16 or BF16), k % 16 == 0:
- *   s2 = fl(amax(x) / 2688) (2688 = 448 * 6; 0 -> 1), or *global_scale when
- *   static_global != 0 (then it is an input);
+ *   s2 = fl(amax / 2688) (2688 = 448 * 6; 0 -> 1) where amax is that of x
+ *   (static_global == 0) or taken from the range record in ws
+ *   (static_global == 2: as written by bq_group_range with BQ_GRAN_TENSOR,
+ *   possibly combined across shards with an integer MAX); or s2 =
+ *   *global_scale, an input (static_global == 1);
  *   per 16 consecutive elements of a row: sb = E4M3(fl(a_b / fl(6 * s2))),
  *   eff = fl(E4M3(sb) * s2), code = E2M1(fl(x / eff)) (all codes 0 when
  *   eff == 0).
  * packed: u8 [n, k/2], element 2j in the low nibble of byte j.
- * scale_e4m3: u8 [n, k/16]. global_scale: one f32 (device), written when
- * dynamic. ws: 16 bytes (dynamic only). E4M3 encodes round to nearest even,
+ * scale_e4m3: u8 [n, k/16]. global_scale: one f32 (device), written unless
+ * static_global == 1. ws: 16 bytes (static_global 0 and 2). E4M3 encodes round to nearest even,
  * saturate to +-448, NaN -> 0x7F; E2M1 encodes saturate to +-6 and keep the
- * sign; a NaN element encodes as a zero with the NaN's sign bit. */
+ * sign; a NaN element encodes as 0x7 (+6). */
 bq_status bq_nvfp4_quantize(const void* x, bq_dtype x_dtype, int64_t n, int64_t k,
                             uint8_t* packed, uint8_t* scale_e4m3, float* global_scale,
                             int32_t static_global, void* ws, size_t ws_bytes, void* stream);

@@ -44,7 +44,7 @@
 //   * dequantize y = RN_y(fl((q-zp)*s)); f64 outputs keep the exact product.
 //   * E4M3 encode is round-to-nearest-even with saturation to +-448, NaN ->
 //     0x7F; E2M1 encode is round-to-nearest-even with saturation to +-6 and
-//     the sign bit kept, NaN -> a zero carrying the NaN's sign bit; E2M1
+//     the sign bit kept, NaN -> 0x7 (+6, the largest positive code); E2M1
 //     element 2j goes to the low nibble of byte j.
 //   * NVFP4: s2 = fl(A/2688) (2688 = 448*6), sb = E4M3(fl(a_b/fl(6*s2))),
 //     eff = fl(dec(sb)*s2), code = E2M1(fl(x/eff)), all-zero codes when
@@ -152,9 +152,8 @@ uint16_t enc_f16(double v)  { return (uint16_t)mini_encode(fmt_f16(), v, false, 
 uint16_t enc_bf16(double v) { return (uint16_t)mini_encode(fmt_bf16(), v, false, 0x7FC0u); }
 uint8_t  enc_e4m3(double v) { return (uint8_t)mini_encode(fmt_e4m3(), v, true, 0x7Fu); }
 uint8_t  enc_e2m1(double v) {
-    // No NaN in E2M1: a NaN becomes a zero that keeps the NaN's sign bit.
-    if (std::isnan(v)) return std::signbit(v) ? 0x8 : 0x0;
-    return (uint8_t)mini_encode(fmt_e2m1(), v, true, 0u);
+    // No NaN in E2M1: a NaN saturates to the largest positive code (+6).
+    return (uint8_t)mini_encode(fmt_e2m1(), v, true, 0x7u);
 }
 double dec_f16(uint16_t c)  { return mini_decode_fields(fmt_f16(), c); }
 double dec_bf16(uint16_t c) { return mini_decode_fields(fmt_bf16(), c); }

@@ -45,7 +45,7 @@ def test_nvfp4_parity(bq, orc, dtype, shape):
 
 def test_nvfp4_special_values(bq, orc):
     vals = [0.0, -0.0, 1e-30, -1e-30, 6.0, -6.0, 5.0, 2.5, 0.25, 0.75, 1e30, -1e30,
-            float("inf"), float("-inf"), float("nan"), -0.1]
+            float("inf"), float("-inf"), float("nan"), -float("nan")]
     x = torch.tensor(vals * 4, dtype=torch.float32).reshape(2, 32)
     x[1] = torch.linspace(-7, 7, 32)
     packed, sc, s2 = bq.nvfp4_quantize(x.cuda(), s2=1.0)
