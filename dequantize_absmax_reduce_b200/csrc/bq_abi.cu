@@ -322,6 +322,13 @@ bq_status bq_tensor_amax(const void* x, bq_dtype dtype, int64_t n, float* amax, 
     return from_cuda(bq::range_to_amax((const unsigned long long*)ws, amax, s));
 }
 
+bq_status bq_check_device_error(void) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return BQ_ERR_CUDA;
+    unsigned int flag = 0;
+    if (bq::pipe_error_take(&flag) != cudaSuccess) return BQ_ERR_CUDA;
+    return flag ? BQ_ERR_TIMEOUT : BQ_OK;
+}
+
 // ---- quantize
 bq_status bq_quantize_per_tensor(const void* x, const bq_qdesc* d, void* q, float* scale,
                                  void* zp, bq_scale_mode mode, void* ws, size_t ws_bytes,

@@ -22,63 +22,10 @@
 
 #include "bq_device.cuh"
 #include "bq_internal.h"
+#include "bq_quant_ops.cuh"
+#include "bq_map_ops.cuh"
 
 namespace bq {
-
-// ------------------------------------------------------------ group params
-struct GroupF { float s; int zp; };
-struct GroupD { float s; int zp; };
-
-// Scale and zero-point from a group's range (f32 arithmetic). Symmetric:
-// s = fl(amax / qmax). Asymmetric: s = fl(fl(max' - min') / (qmax - qmin)),
-// zp = clamp(qmin - round(fl(min' / s)), qmin, qmax). 0 -> 1.
-__device__ __forceinline__ GroupF derive_f(float hi, float nlo, const IntCfg& c) {
-    GroupF g;
-    if (c.symmetric) {
-        float s = __fdiv_rn(fmaxf(hi, nlo), (float)c.qmax);
-        if (s == 0.0f) s = 1.0f;
-        g.s = s;
-        g.zp = 0;
-    } else {
-        const float span = __fadd_rn(hi, nlo);
-        float s = __fdiv_rn(span, (float)(c.qmax - c.qmin));
-        if (s == 0.0f) s = 1.0f;
-        const float m = __fdiv_rn(-nlo, s);
-        const float r = c.rhaz ? roundf(m) : rintf(m);
-        float z = __fsub_rn((float)c.qmin, r);
-        z = fminf(fmaxf(z, (float)c.qmin), (float)c.qmax);   // NaN -> qmin
-        g.s = s;
-        g.zp = (int)z;
-    }
-    return g;
-}
-// Same in f64 for f64 inputs; the stored scale is still f32.
-__device__ __forceinline__ GroupD derive_d(double hi, double nlo, const IntCfg& c) {
-    GroupD g;
-    if (c.symmetric) {
-        float s = __double2float_rn(fmax(hi, nlo) / (double)c.qmax);
-        if (s == 0.0f) s = 1.0f;
-        g.s = s;
-        g.zp = 0;
-    } else {
-        const double span = hi + nlo;
-        float s = __double2float_rn(span / (double)(c.qmax - c.qmin));
-        if (s == 0.0f) s = 1.0f;
-        const double m = -nlo / (double)s;
-        const double r = c.rhaz ? round(m) : rint(m);
-        double z = (double)c.qmin - r;
-        z = fmin(fmax(z, (double)c.qmin), (double)c.qmax);
-        g.s = s;
-        g.zp = (int)z;
-    }
-    return g;
-}
-
-__device__ __forceinline__ int load_zp(const void* zp, int64_t g, int q_signed) {
-    if (!zp) return 0;
-    const uint8_t b = __ldg((const uint8_t*)zp + g);
-    return q_signed ? (int)(int8_t)b : (int)b;
-}
 
 // ------------------------------------------------------------ dynamic, warp
 struct DynArgs {
@@ -274,121 +221,6 @@ __global__ void __launch_bounds__(256) k_int_dyn_cta(DynArgs a) {
     }
 }
 
-// ------------------------------------------------------------ element-wise
-struct MapArgs {
-    const void* a;      // x, q or dy
-    const void* b;      // dy (backwards)
-    int64_t numel, G, n_seg;
-    FastDiv fd;         // divide by G when numel < 2^32
-    int use_fd;
-    IntCfg cfg;
-    const float* scale_in;
-    const void* zp_in;
-    const unsigned long long* ranges;
-    float* scale_out;
-    uint8_t* zp_out;
-    void* out;
-};
-
-// Per-group state cached by a thread while it walks its elements.
-struct GState {
-    int64_t seg;
-    float s;
-    int zp;
-    Recip R;
-    IntParams ip;
-};
-
-template <class T, int PSRC>
-__device__ __forceinline__ void load_group(const MapArgs& a, int64_t seg, bool writer, GState& st) {
-    using Acc = typename Traits<T>::Acc;
-    st.seg = seg;
-    if (PSRC == PS_RANGE) {
-        Acc hi, nlo;
-        range_from_bits(a.ranges[2 * seg], hi);
-        range_from_bits(a.ranges[2 * seg + 1], nlo);
-        if constexpr (std::is_same<Acc, double>::value) {
-            const GroupD g = derive_d(hi, nlo, a.cfg);
-            st.s = g.s; st.zp = g.zp;
-        } else {
-            const GroupF g = derive_f(hi, nlo, a.cfg);
-            st.s = g.s; st.zp = g.zp;
-        }
-        if (writer) {
-            a.scale_out[seg] = st.s;
-            if (a.zp_out) a.zp_out[seg] = (uint8_t)st.zp;
-        }
-    } else {
-        st.s = __ldg(a.scale_in + seg);
-        st.zp = a.cfg.symmetric ? 0 : load_zp(a.zp_in, seg, a.cfg.q_signed);
-    }
-    st.R = make_recip(st.s);
-    st.ip = make_int_params(a.cfg.qmin, a.cfg.qmax, st.zp);
-}
-
-// One element, f32 arithmetic. Returns the output value (float ops) or the
-// code byte (QUANT) in the low byte of *code.
-template <int OP, bool RHAZ>
-__device__ __forceinline__ float elem_f(float xa, float xb, const GState& st, uint32_t* code) {
-    if constexpr (OP == OP_QUANT || OP == OP_FAKE) {
-        const float v = div_any(xa, st.R);
-        const float t = rounded_of<RHAZ>(v, st.ip);
-        *code = code_from_rounded(t, st.ip.zp);
-        if constexpr (OP == OP_FAKE) return dequant_from_rounded(t, st.s);
-        return 0.0f;
-    } else if constexpr (OP == OP_QBWD || OP == OP_FBWD) {
-        const float v = div_any(xa, st.R);
-        const float k = round_for_mask<RHAZ>(v, st.ip);
-        const float m = (k > st.ip.lo && k < st.ip.hi) ? 1.0f : 0.0f;
-        if constexpr (OP == OP_QBWD) {
-            const float g = with_quotient_sign(div_any(xb, st.R), xb, st.s);
-            return __fmul_rn(g, m);
-        } else {
-            return __fmul_rn(xb, m);
-        }
-    } else if constexpr (OP == OP_DBWD) {
-        return __fmul_rn(xa, st.s);
-    } else {
-        return 0.0f;
-    }
-}
-
-// f64 arithmetic (f64 tensors).
-template <int OP, bool RHAZ>
-__device__ __forceinline__ double elem_d(double xa, double xb, const GState& st, uint32_t* code) {
-    const double s = (double)st.s;
-    const double lo = (double)st.ip.lo, hi = (double)st.ip.hi;
-    if constexpr (OP == OP_QUANT || OP == OP_FAKE) {
-        const double v = xa / s;
-        double k = RHAZ ? round(v) : rint(v);
-        k = fmin(fmax(k, lo), hi);                  // NaN -> lo
-        *code = (uint32_t)((int)k + st.zp);
-        if constexpr (OP == OP_FAKE) return (double)((int)k) * s;   // (q - zp) as an integer: +0, never -0
-        return 0.0;
-    } else if constexpr (OP == OP_QBWD || OP == OP_FBWD) {
-        const double v = xa / s;
-        double k = RHAZ ? round(v) : rint(v);
-        if (v != v) k = lo;
-        const double m = (k > lo && k < hi) ? 1.0 : 0.0;
-        if constexpr (OP == OP_QBWD) return (xb / s) * m;
-        else return xb * m;
-    } else if constexpr (OP == OP_DBWD) {
-        return xa * s;
-    } else {
-        return 0.0;
-    }
-}
-
-// Dequantize one code: (q - zp) * s. The byte goes into the low mantissa of
-// 2^23 so that one f32 subtraction gives q - zp exactly.
-__device__ __forceinline__ float deq_code_f(uint32_t word, int i, const GState& st, int q_signed) {
-    if (q_signed) word ^= 0x80808080u;
-    const uint32_t sel = (uint32_t)i | (4u << 4) | (5u << 8) | (7u << 12);
-    const float f = __uint_as_float(__byte_perm(word, 0x4B000000u, sel));
-    const float off = 8388608.0f + (float)((q_signed ? 128 : 0) + st.zp);
-    return __fmul_rn(__fsub_rn(f, off), st.s);
-}
-
 // Items of W elements (one 16-byte vector, or one element); each warp takes
 // contiguous chunks of 32*U items, lane l the items l, l+32, ..., so every
 // load instruction is coalesced and a lane's items rarely change group. All
@@ -435,7 +267,7 @@ __global__ void __launch_bounds__(256) k_int_map(MapArgs a) {
                 if (it >= n_items) continue;
                 const int64_t e0 = it * W;
                 const int64_t seg = a.use_fd ? (int64_t)fdiv((uint32_t)e0, a.fd) : e0 / a.G;
-                if (seg != st.seg) load_group<T, PSRC>(a, seg, false, st);
+                if (seg != st.seg) load_group<T, PSRC, false, RHAZ>(a, seg, false, st);
                 Acc o[W];
                 if constexpr (!WIDE && (W == 8 || W == 4)) {
 #pragma unroll
@@ -474,7 +306,7 @@ __global__ void __launch_bounds__(256) k_int_map(MapArgs a) {
                 if (it >= n_items) continue;
                 const int64_t e0 = it * W;
                 const int64_t seg = a.use_fd ? (int64_t)fdiv((uint32_t)e0, a.fd) : e0 / a.G;
-                if (seg != st.seg) load_group<T, PSRC>(a, seg, e0 == seg * a.G, st);
+                if (seg != st.seg) load_group<T, PSRC, (OP == OP_QBWD || OP == OP_FBWD), RHAZ>(a, seg, e0 == seg * a.G, st);
                 Acc xa[W], xb[W];
                 if constexpr (VECP) {
                     load_vec<T>(ra[u], xa);
@@ -733,6 +565,8 @@ static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 cudaError_t int_dyn(DT dt, int op, const void* x, SegView sv, IntCfg cfg, void* q, void* y,
                     float* scale, void* zp, cudaStream_t st) {
+    const cudaError_t pe = int_dyn_pipe(dt, op, x, sv, cfg, q, y, scale, zp, st);
+    if (pe != cudaErrorNotSupported) return pe;
     if (dt == DT::F64 || cfg.rhaz) return cudaErrorNotSupported;
     if (op != OP_QUANT && op != OP_FAKE) return cudaErrorNotSupported;
     const int VEC = (dt == DT::F32) ? 4 : 8;
@@ -812,6 +646,10 @@ cudaError_t int_map(DT dt, int op, int psrc, const void* a_ptr, const void* b_pt
         if (op == OP_QBWD || op == OP_FBWD) vecp = vecp && aligned16(b_ptr);
         if (op == OP_QUANT) vecp = vecp && ((uintptr_t)out % VEC == 0);
         else vecp = vecp && aligned16(out);
+    }
+    if (vecp) {
+        const cudaError_t pe = int_map_pipe(dt, op, a, st);
+        if (pe != cudaErrorNotSupported) return pe;
     }
     switch (dt) {
         case DT::F32: return launch_map_dt<float>(op, psrc, a, vecp, st);

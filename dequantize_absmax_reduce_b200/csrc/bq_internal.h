@@ -33,6 +33,18 @@ int sm_count();
 cudaError_t int_dyn(DT dt, int op, const void* x, SegView sv, IntCfg cfg, void* q, void* y,
                     float* scale, void* zp, cudaStream_t st);
 
+// Bulk-copy pipelined variants of int_dyn / mx_quant (bq_pipe.cu); they
+// return cudaErrorNotSupported when the shape or alignment does not fit.
+cudaError_t int_dyn_pipe(DT dt, int op, const void* x, SegView sv, IntCfg cfg, void* q, void* y,
+                         float* scale, void* zp, cudaStream_t st);
+cudaError_t mx_quant_pipe(DT dt, int fmt, const void* x, int64_t rows, int64_t k, uint8_t* codes,
+                          void* scales, const unsigned long long* amax_rec, float* global_scale,
+                          int static_global, cudaStream_t st);
+struct MapArgs;
+cudaError_t int_map_pipe(DT dt, int op, const MapArgs& m, cudaStream_t st);
+// Reads and clears the flag a pipelined kernel sets when a bounded wait gives up.
+cudaError_t pipe_error_take(unsigned int* flag);
+
 // Element-wise with per-group parameters (static, or derived from range
 // records). a: x (QUANT, FAKE, QBWD, FBWD), q (DEQ) or dy (DBWD);
 // b: dy (QBWD, FBWD). out: q (QUANT) or a float tensor of type dt.

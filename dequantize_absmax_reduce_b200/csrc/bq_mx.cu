@@ -14,13 +14,9 @@
 
 #include "bq_device.cuh"
 #include "bq_internal.h"
+#include "bq_quant_ops.cuh"
 
 namespace bq {
-
-template <int FMT> struct MxG;
-template <> struct MxG<MX_FP8_1x128> { static constexpr int G = 128; };
-template <> struct MxG<MX_MXFP8> { static constexpr int G = 32; };
-template <> struct MxG<MX_NVFP4> { static constexpr int G = 16; };
 
 struct MxArgs {
     const void* x;
@@ -31,60 +27,6 @@ struct MxArgs {
     float* global_scale;
     int static_global;
 };
-
-__device__ __forceinline__ void st2(void* p, uint32_t a) {
-    asm volatile("st.global.u16 [%0], %1;" :: "l"(p), "h"((uint16_t)a) : "memory");
-}
-
-// MXFP8 shared exponent: E = clamp(floor(log2 a) - 8, -127, 127), from the
-// bits of a >= 0 (a subnormal a counts its leading zeros; infinity is 2^128;
-// a = 0 gives -127).
-__device__ __forceinline__ int mx_exponent(float a) {
-    const uint32_t b = __float_as_uint(a);
-    const int ex = (int)(b >> 23);
-    int fl2;
-    if (ex == 0) {
-        const uint32_t m = b & 0x7FFFFFu;
-        fl2 = (m == 0) ? -1000 : (31 - __clz((int)m)) - 149;
-    } else if (ex == 255) {
-        fl2 = 128;
-    } else {
-        fl2 = ex - 127;
-    }
-    return min(max(fl2 - 8, -127), 127);
-}
-
-// Codes of one 16-byte vector (v: its VEC values) written at dst.
-template <class T, int FMT, bool FAST>
-__device__ __forceinline__ void mx_emit(const float* v, const Recip& R, float mul, bool zero,
-                                        uint8_t* dst) {
-    constexpr int VEC = Traits<T>::VEC;
-    float t[VEC];
-#pragma unroll
-    for (int i = 0; i < VEC; ++i) {
-        if constexpr (FMT == MX_MXFP8) {
-            t[i] = __fmul_rn(v[i], mul);
-        } else {
-            const float d = FAST ? div_chain(v[i], R) : div_any(v[i], R);
-            t[i] = with_quotient_sign(d, v[i], R.s);
-        }
-    }
-    if constexpr (FMT == MX_NVFP4) {
-        if constexpr (VEC == 8) {
-            const float (&t8)[8] = *reinterpret_cast<const float(*)[8]>(t);
-            st4(dst, zero ? 0u : e2m1x8(t8));
-        } else {
-            float t8[8] = {t[0], t[1], t[2], t[3], 0.f, 0.f, 0.f, 0.f};
-            st2(dst, zero ? 0u : (e2m1x8(t8) & 0xFFFFu));
-        }
-    } else {
-        if constexpr (VEC == 8) {
-            st8(dst, e4m3x4(t[0], t[1], t[2], t[3]), e4m3x4(t[4], t[5], t[6], t[7]));
-        } else {
-            st4(dst, e4m3x4(t[0], t[1], t[2], t[3]));
-        }
-    }
-}
 
 // Lanes per group and vectors per lane for each format / element size: each
 // lane holds NV vectors of its group so that the per-group work (amax
@@ -471,6 +413,9 @@ cudaError_t mx_quant(DT dt, int fmt, const void* x, int64_t rows, int64_t k, uin
     a.x = x; a.n_seg = rows * (k / G); a.codes = codes; a.scales = scales;
     a.amax_rec = amax_rec; a.global_scale = global_scale; a.static_global = static_global;
     if (a.n_seg == 0) return cudaSuccess;
+    const cudaError_t pe = mx_quant_pipe(dt, fmt, x, rows, k, codes, scales, amax_rec, global_scale,
+                                         static_global, st);
+    if (pe != cudaErrorNotSupported) return pe;
     const int VEC = dt == DT::F32 ? 4 : 8;
     const int cb = (fmt == MX_NVFP4) ? VEC / 2 : VEC;
     const bool vec = al(x, 16) && al(codes, cb);

@@ -1,0 +1,891 @@
+// Bulk-copy pipelined quantizers for contiguous groups with dynamic scales:
+// per-token / per-channel / per-group integer quantize and fake-quantize
+// (baracuda_kernels::quantize), FP8 1x128 and MXFP8 (smile llm.quant
+// Fp8BlockGemm, MxFp8) and NVFP4 (metrale QuantizedWeight).
+//
+// A persistent CTA of 256 threads walks tiles of P whole groups. The tiles
+// reach shared memory through cp.async.bulk (the Blackwell / Hopper bulk copy
+// engine, no registers held while in flight) into a ring of STAGES slots,
+// each completed on its own mbarrier; while the threads reduce and encode
+// one tile, the next STAGES-1 are in flight. The CTA splits into 256/TEAM
+// teams, one group per team, each thread holding NV 16-byte vectors of its
+// group; teams of up to 32 lanes reduce with warp shuffles, larger teams
+// also through shared memory. Codes go straight from registers to HBM.
+//
+// Every wait on an mbarrier is bounded: after about two seconds the kernel
+// records the failure in g_pipe_error, waits (bounded again) for the copies
+// it has in flight, and returns.
+#pragma once
+#include <type_traits>
+
+#include "bq_device.cuh"
+#include "bq_internal.h"
+#include "bq_quant_ops.cuh"
+#include "bq_map_ops.cuh"
+#include "bq_pipe_args.h"
+
+namespace bq {
+namespace {   // one copy per dtype translation unit
+
+// Set when a bounded wait gives up (one flag per translation unit).
+__device__ unsigned int g_pipe_error;
+
+
+// ------------------------------------------------------------ PTX helpers
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// One thread: expect `bytes` on the barrier and start the bulk copy.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes) : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 :: "r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(bar), "r"(parity), "r"(1000u) : "memory");
+    return ok != 0;
+}
+// Bounded wait: each try suspends for at most about a microsecond.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    for (uint32_t i = 0; i < (1u << 21); ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+__device__ __forceinline__ U4 ld_shared16(uint32_t addr) {
+    U4 r;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(addr));
+    return r;
+}
+
+// ------------------------------------------------------------ range helpers
+// Range of one 16-byte vector, accumulated without widening: for 16-bit types
+// two lanes per instruction (max.xorsign.abs keeps the larger magnitude; min /
+// max skip a NaN operand), for f32 one.
+template <class T, bool ABS>
+__device__ __forceinline__ void range_acc(const U4& r, uint32_t& ph, uint32_t& pl, float& hi,
+                                          float& nlo) {
+    if constexpr (sizeof(T) == 2) {
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+                if (ABS) {
+                    asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(ph) : "r"(w[i]));
+                } else {
+                    asm("max.bf16x2 %0, %0, %1;" : "+r"(ph) : "r"(w[i]));
+                    asm("min.bf16x2 %0, %0, %1;" : "+r"(pl) : "r"(w[i]));
+                }
+            } else {
+                if (ABS) {
+                    asm("max.xorsign.abs.f16x2 %0, %0, %1;" : "+r"(ph) : "r"(w[i]));
+                } else {
+                    asm("max.f16x2 %0, %0, %1;" : "+r"(ph) : "r"(w[i]));
+                    asm("min.f16x2 %0, %0, %1;" : "+r"(pl) : "r"(w[i]));
+                }
+            }
+        }
+    } else {
+        const float v[4] = {__uint_as_float(r.x), __uint_as_float(r.y), __uint_as_float(r.z),
+                            __uint_as_float(r.w)};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if (ABS) {
+                hi = fmaxf(hi, fabsf(v[i]));
+            } else {
+                hi = fmaxf(hi, v[i]);
+                nlo = fmaxf(nlo, -v[i]);
+            }
+        }
+    }
+}
+// Packed accumulators -> (max(0, max x), max(0, -min x)) or (amax, 0).
+template <class T, bool ABS>
+__device__ __forceinline__ void range_finish(uint32_t ph, uint32_t pl, float& hi, float& nlo) {
+    if constexpr (sizeof(T) == 2) {
+        float h0, h1, l0, l1;
+        if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+            unpack_bf16x2(ph, h0, h1);
+            unpack_bf16x2(pl, l0, l1);
+        } else {
+            unpack_f16x2(ph, h0, h1);
+            unpack_f16x2(pl, l0, l1);
+        }
+        if (ABS) {
+            hi = fmaxf(fabsf(h0), fabsf(h1));
+            nlo = 0.0f;
+        } else {
+            hi = fmaxf(fmaxf(h0, h1), 0.0f);
+            nlo = fmaxf(fmaxf(-l0, -l1), 0.0f);
+        }
+    }
+}
+
+// ------------------------------------------------------------ the kernel
+// Ring depth: 4 slots of up to 16 KB, or 3 of up to 32 KB (NV = 8).
+template <int NV> struct PipeStages { static constexpr int S = NV <= 4 ? 4 : 3; };
+
+template <class T, int PK, int TEAM, int NV, bool SYM>
+__global__ void __launch_bounds__(256) k_seg_pipe(PipeArgs a) {
+    constexpr int VEC = Traits<T>::VEC;
+    constexpr int NW = 8;
+    constexpr int SPAN = TEAM * NV * VEC;          // elements a team covers
+    constexpr bool ABS = (PK != PK_INT_Q && PK != PK_INT_FAKE) || SYM;
+    extern __shared__ __align__(128) uint8_t smem[];
+    float* red = reinterpret_cast<float*>(smem);                     // [2][NW]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 64);         // [stages]
+    uint8_t* ring = smem + 128;                                      // [stages][slot_bytes]
+    const int tid = threadIdx.x;
+    const int team = tid / TEAM, lane = tid % TEAM;
+    const int wid = tid >> 5;
+    constexpr int S = PipeStages<NV>::S;
+    const int64_t grid = gridDim.x;
+    const size_t esz = sizeof(T);
+    const int G = a.G;
+    const bool full_groups = (G == SPAN);
+
+    if (tid == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(smem_addr(&bars[s]), 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    auto tile_bytes = [&](int64_t tile) -> uint32_t {
+        const int64_t segs = min((int64_t)a.P, a.n_seg - tile * a.P);
+        return (uint32_t)(segs * G * esz);
+    };
+    if (tid == 0) {
+        for (int i = 0; i < S; ++i) {
+            const int64_t tile = blockIdx.x + (int64_t)i * grid;
+            if (tile >= a.n_tiles) break;
+            bulk_load(smem_addr(ring + (size_t)i * a.slot_bytes),
+                      (const uint8_t*)a.x + (size_t)tile * a.P * G * esz, tile_bytes(tile),
+                      smem_addr(&bars[i]));
+        }
+    }
+
+    // Launch constants.
+    float s2 = 1.0f;
+    Recip R6, Rq;
+    const float qlo = (float)a.cfg.qmin, qhi = (float)a.cfg.qmax;
+    if constexpr (PK == PK_NV) {
+        if (a.static_global) {
+            s2 = *a.global_scale;
+        } else {
+            float h, n;
+            range_from_bits(a.amax_rec[0], h);
+            range_from_bits(a.amax_rec[1], n);
+            s2 = __fdiv_rn(fmaxf(h, n), 2688.0f);
+            if (s2 == 0.0f) s2 = 1.0f;
+            if (blockIdx.x == 0 && tid == 0) *a.global_scale = s2;
+        }
+        R6 = make_recip(__fmul_rn(6.0f, s2));
+    } else if constexpr (PK == PK_FP8) {
+        Rq = make_recip(448.0f);
+    } else if constexpr (PK == PK_INT_Q || PK == PK_INT_FAKE) {
+        Rq = make_recip(SYM ? qhi : (float)(a.cfg.qmax - a.cfg.qmin));
+    }
+
+    int slot = 0;
+    uint32_t parity = 0;
+    for (int64_t tile = blockIdx.x; tile < a.n_tiles; tile += grid) {
+        const bool ok = mbar_wait(smem_addr(&bars[slot]), parity);
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) {
+                atomicOr(&g_pipe_error, 1u);
+                // Drain the copies still in flight into this CTA's ring.
+                int s2 = slot;
+                uint32_t p2 = parity;
+                for (int i = 0; i < S; ++i) {
+                    const int64_t t2 = tile + (int64_t)i * grid;
+                    if (t2 >= a.n_tiles) break;
+                    mbar_wait(smem_addr(&bars[s2]), p2);
+                    if (++s2 == S) { s2 = 0; p2 ^= 1u; }
+                }
+            }
+            __syncthreads();
+            return;
+        }
+        const uint8_t* slot_ptr = ring + (size_t)slot * a.slot_bytes;
+        const int64_t seg = tile * a.P + team;
+        const bool seg_ok = seg < a.n_seg;
+        const bool full = seg_ok && full_groups;
+
+        // This thread's vectors of its group, straight from shared memory.
+        U4 raw[NV];
+        const uint32_t gbase = smem_addr(slot_ptr + (size_t)team * G * esz) + (uint32_t)(lane * 16);
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+            const int e = (j * TEAM + lane) * VEC;
+            raw[j] = (full || (seg_ok && e < G)) ? ld_shared16(gbase + (uint32_t)(j * TEAM * 16))
+                                                 : U4{0u, 0u, 0u, 0u};
+        }
+        uint32_t ph = 0u, pl = 0u;
+        float hi = 0.0f, nlo = 0.0f;
+#pragma unroll
+        for (int j = 0; j < NV; ++j) range_acc<T, ABS>(raw[j], ph, pl, hi, nlo);
+        range_finish<T, ABS>(ph, pl, hi, nlo);
+        if constexpr (TEAM > 1) {
+#pragma unroll
+            for (int o = (TEAM < 32 ? TEAM : 32) / 2; o > 0; o >>= 1) {
+                hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+                if (!ABS) nlo = fmaxf(nlo, __shfl_xor_sync(0xffffffffu, nlo, o));
+            }
+        }
+        if constexpr (TEAM > 32) {
+            constexpr int WPT = TEAM / 32;
+            if ((tid & 31) == 0) { red[wid] = hi; red[NW + wid] = nlo; }
+            __syncthreads();
+            const int w0 = team * WPT;
+            hi = red[w0];
+            nlo = red[NW + w0];
+#pragma unroll
+            for (int w = 1; w < WPT; ++w) {
+                hi = fmaxf(hi, red[w0 + w]);
+                if (!ABS) nlo = fmaxf(nlo, red[NW + w0 + w]);
+            }
+        }
+
+        if constexpr (PK == PK_INT_Q || PK == PK_INT_FAKE) {
+            constexpr int OP = (PK == PK_INT_Q) ? OP_QUANT : OP_FAKE;
+            // Scale and zero-point: fl(amax/qmax) or fl(fl(max'-min')/(qmax-qmin)),
+            // each quotient by the launch's divisor reciprocal (exact for a
+            // normal dividend; IEEE division below 2^-100).
+            float sc, zf = 0.0f;
+            {
+                const float num = SYM ? fmaxf(hi, nlo) : __fadd_rn(hi, nlo);
+                sc = (num >= 0x1p-100f && num <= 0x1p100f) ? div_chain(num, Rq) : div_slow(num, Rq.s);
+                if (sc == 0.0f) sc = 1.0f;
+                if (!SYM) {
+                    const float m = __fdiv_rn(-nlo, sc);
+                    const float r = a.cfg.rhaz ? roundf(m) : rintf(m);
+                    zf = fminf(fmaxf(__fsub_rn(qlo, r), qlo), qhi);   // NaN -> qmin
+                }
+            }
+            const int zp = (int)zf;
+            if (seg_ok && lane == 0) {
+                a.scale[seg] = sc;
+                if (a.zp) a.zp[seg] = (uint8_t)zp;
+            }
+            IntParams ip;
+            ip.lo = SYM ? qlo : __fsub_rn(qlo, zf);
+            ip.hi = SYM ? qhi : __fsub_rn(qhi, zf);
+            ip.zp = SYM ? 0 : zp;
+            const Recip R = make_recip(sc);
+            uint8_t* qb = a.q + seg * G + lane * VEC;
+            T* yb = (T*)a.y + seg * G + lane * VEC;
+            if (full) {
+                if (R.fast) {
+#pragma unroll
+                    for (int j = 0; j < NV; ++j) {
+                        float v[VEC];
+                        load_vec<T>(raw[j], v);
+                        emit_int<T, OP, true, SYM>(v, R, ip, qb + j * TEAM * VEC, yb + j * TEAM * VEC);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < NV; ++j) {
+                        float v[VEC];
+                        load_vec<T>(raw[j], v);
+                        emit_int<T, OP, false, SYM>(v, R, ip, qb + j * TEAM * VEC, yb + j * TEAM * VEC);
+                    }
+                }
+            } else if (seg_ok) {
+#pragma unroll
+                for (int j = 0; j < NV; ++j) {
+                    if ((j * TEAM + lane) * VEC >= G) continue;
+                    float v[VEC];
+                    load_vec<T>(raw[j], v);
+                    if (R.fast) emit_int<T, OP, true, SYM>(v, R, ip, qb + j * TEAM * VEC, yb + j * TEAM * VEC);
+                    else emit_int<T, OP, false, SYM>(v, R, ip, qb + j * TEAM * VEC, yb + j * TEAM * VEC);
+                }
+            }
+        } else {
+            constexpr int FMT = (PK == PK_FP8) ? MX_FP8_1x128 : (PK == PK_MX ? MX_MXFP8 : MX_NVFP4);
+            constexpr int CB = (PK == PK_NV) ? VEC / 2 : VEC;     // code bytes per vector
+            uint8_t* base = a.q + seg * (G / VEC) * CB + lane * CB;
+            if constexpr (PK == PK_FP8) {
+                float s = (hi >= 0x1p-100f && hi <= 0x1p100f) ? div_chain(hi, Rq) : div_slow(hi, 448.0f);
+                if (s == 0.0f) s = 1.0f;
+                if (seg_ok && lane == 0) a.scale[seg] = s;
+                const Recip R = make_recip(s);
+                if (seg_ok) {
+#pragma unroll
+                    for (int j = 0; j < NV; ++j) {
+                        if (!full && (j * TEAM + lane) * VEC >= G) continue;
+                        float v[VEC];
+                        load_vec<T>(raw[j], v);
+                        if (R.fast) mx_emit<T, FMT, true>(v, R, 0.f, false, base + j * TEAM * CB);
+                        else mx_emit<T, FMT, false>(v, R, 0.f, false, base + j * TEAM * CB);
+                    }
+                }
+            } else if constexpr (PK == PK_MX) {
+                const int E = mx_exponent(hi);
+                if (seg_ok && lane == 0) a.zp[seg] = (uint8_t)(E + 127);
+                const Recip R{};
+                const float mul = exp2i(-E);
+                if (seg_ok) {
+#pragma unroll
+                    for (int j = 0; j < NV; ++j) {
+                        if (!full && (j * TEAM + lane) * VEC >= G) continue;
+                        float v[VEC];
+                        load_vec<T>(raw[j], v);
+                        mx_emit<T, FMT, true>(v, R, mul, false, base + j * TEAM * CB);
+                    }
+                }
+            } else {
+                const uint32_t sb = e4m3x2(div_any(hi, R6), 0.0f) & 0xFFu;
+                if (seg_ok && lane == 0) a.zp[seg] = (uint8_t)sb;
+                const float eff = __fmul_rn(e4m3_to_f32(sb), s2);
+                const Recip R = make_recip(eff);
+                const bool fast = R.fast && !a.static_global;
+                if (seg_ok) {
+#pragma unroll
+                    for (int j = 0; j < NV; ++j) {
+                        if (!full && (j * TEAM + lane) * VEC >= G) continue;
+                        float v[VEC];
+                        load_vec<T>(raw[j], v);
+                        if (fast) mx_emit<T, FMT, true>(v, R, 0.f, eff == 0.0f, base + j * TEAM * CB);
+                        else mx_emit<T, FMT, false>(v, R, 0.f, eff == 0.0f, base + j * TEAM * CB);
+                    }
+                }
+            }
+        }
+
+        // Every thread is done with this slot: refill it with tile it + S.
+        __syncthreads();
+        if (tid == 0) {
+            const int64_t next = tile + (int64_t)S * grid;
+            if (next < a.n_tiles) {
+                fence_proxy_async();
+                bulk_load(smem_addr(ring + (size_t)slot * a.slot_bytes),
+                          (const uint8_t*)a.x + (size_t)next * a.P * G * esz, tile_bytes(next),
+                          smem_addr(&bars[slot]));
+            }
+        }
+        if (++slot == S) { slot = 0; parity ^= 1u; }
+    }
+}
+
+// ------------------------------------------------------------ element-wise
+// Tiles of 256 * ITEMS vectors; both inputs of a backward land in one slot
+// (first the x part, then the dy part). Thread t handles the vectors
+// t, t + 256, ... of its tile: conflict-free shared loads, coalesced stores.
+// Items (16-byte vectors) per thread per tile and ring depth: enough work per
+// tile to amortise the per-tile wait and barrier, within 96 KB of ring.
+template <int OP> struct MapShape {
+    static constexpr bool TWO = (OP == OP_QBWD || OP == OP_FBWD);
+    static constexpr int ITEMS = TWO ? 4 : 8;
+    static constexpr int S = 3;
+};
+
+struct MapPipeArgs {
+    MapArgs m;
+    int64_t n_tiles;
+    int tile_elems;     // 256 * kMapItems * W
+    int in_esz;         // bytes per element of input a (1 for codes)
+    int slot_bytes;
+    int stages;
+};
+
+template <class T, int OP, int PSRC, bool RHAZ>
+__global__ void __launch_bounds__(256) k_map_pipe(MapPipeArgs p) {
+    using Acc = typename Traits<T>::Acc;
+    constexpr int W = Traits<T>::VEC;
+    constexpr int ITEMS = MapShape<OP>::ITEMS;
+    constexpr bool TWO = (OP == OP_QBWD || OP == OP_FBWD);
+    constexpr int ESZ = sizeof(T);
+    const MapArgs& a = p.m;
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 64);
+    uint8_t* ring = smem + 128;
+    const int tid = threadIdx.x;
+    constexpr int S = MapShape<OP>::S;
+    const int64_t grid = gridDim.x;
+    const int E = p.tile_elems;
+
+    if (tid == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(smem_addr(&bars[s]), 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    // Tile `tile` into slot `slot`: input a, then (backwards) input b.
+    auto issue = [&](int64_t tile, int slot) {
+        const int64_t e0 = tile * E;
+        const int64_t n = min((int64_t)E, a.numel - e0);
+        const uint32_t ba = (uint32_t)(n * p.in_esz);
+        const uint32_t bb = TWO ? (uint32_t)(n * ESZ) : 0u;
+        const uint32_t bar = smem_addr(&bars[slot]);
+        uint8_t* dst = ring + (size_t)slot * p.slot_bytes;
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(ba + bb) : "memory");
+        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                     :: "r"(smem_addr(dst)), "l"((const uint8_t*)a.a + e0 * p.in_esz), "r"(ba), "r"(bar) : "memory");
+        if (TWO)
+            asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                         :: "r"(smem_addr(dst + (size_t)E * p.in_esz)), "l"((const uint8_t*)a.b + e0 * ESZ),
+                            "r"(bb), "r"(bar) : "memory");
+    };
+    if (tid == 0) {
+        for (int i = 0; i < S; ++i) {
+            const int64_t tile = blockIdx.x + (int64_t)i * grid;
+            if (tile >= p.n_tiles) break;
+            issue(tile, i);
+        }
+    }
+    GState st;
+    st.seg = -1;
+    int slot = 0;
+    uint32_t parity = 0;
+    for (int64_t tile = blockIdx.x; tile < p.n_tiles; tile += grid) {
+        const bool ok = mbar_wait(smem_addr(&bars[slot]), parity);
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) {
+                atomicOr(&g_pipe_error, 1u);
+                int s2 = slot;
+                uint32_t p2 = parity;
+                for (int i = 0; i < S; ++i) {
+                    const int64_t t2 = tile + (int64_t)i * grid;
+                    if (t2 >= p.n_tiles) break;
+                    mbar_wait(smem_addr(&bars[s2]), p2);
+                    if (++s2 == S) { s2 = 0; p2 ^= 1u; }
+                }
+            }
+            __syncthreads();
+            return;
+        }
+        const uint8_t* sa = ring + (size_t)slot * p.slot_bytes;
+        const uint8_t* sb = sa + (size_t)E * p.in_esz;
+        const int64_t te0 = tile * E;
+#pragma unroll
+        for (int i = 0; i < ITEMS; ++i) {
+            const int le = (i * 256 + tid) * W;               // element offset in the tile
+            const int64_t e0 = te0 + le;
+            if (e0 >= a.numel) continue;
+            const int64_t seg = a.use_fd ? (int64_t)fdiv((uint32_t)e0, a.fd) : e0 / a.G;
+            if (seg != st.seg) load_group<T, PSRC, (OP == OP_QBWD || OP == OP_FBWD), RHAZ>(a, seg, e0 == seg * a.G, st);
+            if constexpr (OP == OP_DEQ) {
+                Acc o[W];
+                if constexpr (W == 8) {
+                    uint32_t w0, w1;
+                    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(smem_addr(sa + le)));
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) o[k] = deq_code_f(w0, k, st, a.cfg.q_signed);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) o[4 + k] = deq_code_f(w1, k, st, a.cfg.q_signed);
+                } else {
+                    uint32_t w0;
+                    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w0) : "r"(smem_addr(sa + le)));
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) o[k] = deq_code_f(w0, k, st, a.cfg.q_signed);
+                }
+                st16((T*)a.out + e0, pack_vec<T>(o));
+            } else {
+                Acc xa[W], xb[W];
+                load_vec<T>(ld_shared16(smem_addr(sa + (size_t)le * ESZ)), xa);
+                if constexpr (TWO) load_vec<T>(ld_shared16(smem_addr(sb + (size_t)le * ESZ)), xb);
+                Acc o[W];
+                uint32_t cw[W];
+#pragma unroll
+                for (int k = 0; k < W; ++k) o[k] = elem_f<OP, RHAZ>(xa[k], TWO ? xb[k] : 0.0f, st, &cw[k]);
+                if constexpr (OP == OP_QUANT) {
+                    uint8_t* q = (uint8_t*)a.out + e0;
+                    if constexpr (W == 8) st8(q, pack4_lowbytes(cw[0], cw[1], cw[2], cw[3]), pack4_lowbytes(cw[4], cw[5], cw[6], cw[7]));
+                    else st4(q, pack4_lowbytes(cw[0], cw[1], cw[2], cw[3]));
+                } else {
+                    st16((T*)a.out + e0, pack_vec<T>(o));
+                }
+            }
+        }
+        __syncthreads();
+        if (tid == 0) {
+            const int64_t next = tile + (int64_t)S * grid;
+            if (next < p.n_tiles) {
+                fence_proxy_async();
+                issue(next, slot);
+            }
+        }
+        if (++slot == S) { slot = 0; parity ^= 1u; }
+    }
+}
+
+// ------------------------------------------------------------ element-wise, by group
+// The element-wise ops on tiles of P whole groups, one team of 256/P threads
+// per group (the layout of k_seg_pipe): each thread loads its group's
+// parameters once and applies them to NV vectors. Backwards stage x and dy of
+// the same groups in one slot.
+struct SegMapArgs {
+    MapArgs m;
+    int P;
+    int64_t n_tiles;
+    int in_esz;         // bytes per element of input a (1 for codes)
+    int part_bytes;     // P * G * in_esz: where the dy part of a slot starts
+    int slot_bytes;
+};
+
+template <int OP> struct SegMapStages { static constexpr int S = 3; };
+
+template <class T, int OP, int PSRC, int TEAM, int NV, bool RHAZ>
+__global__ void __launch_bounds__(256) k_seg_map(SegMapArgs p) {
+    using Acc = typename Traits<T>::Acc;
+    constexpr int W = Traits<T>::VEC;
+    constexpr int ESZ = sizeof(T);
+    constexpr bool TWO = (OP == OP_QBWD || OP == OP_FBWD);
+    constexpr int SPAN = TEAM * NV * W;
+    constexpr int S = SegMapStages<OP>::S;
+    const MapArgs& a = p.m;
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 64);
+    uint8_t* ring = smem + 128;
+    const int tid = threadIdx.x;
+    const int team = tid / TEAM, lane = tid % TEAM;
+    const int64_t grid = gridDim.x;
+    const int G = (int)a.G;
+    const bool full_groups = (G == SPAN);
+
+    if (tid == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(smem_addr(&bars[s]), 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    auto issue = [&](int64_t tile, int slot) {
+        const int64_t segs = min((int64_t)p.P, a.n_seg - tile * p.P);
+        const int64_t e0 = tile * p.P * G;
+        const uint32_t ba = (uint32_t)(segs * G * p.in_esz);
+        const uint32_t bb = TWO ? (uint32_t)(segs * G * ESZ) : 0u;
+        const uint32_t bar = smem_addr(&bars[slot]);
+        uint8_t* dst = ring + (size_t)slot * p.slot_bytes;
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(ba + bb) : "memory");
+        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                     :: "r"(smem_addr(dst)), "l"((const uint8_t*)a.a + e0 * p.in_esz), "r"(ba), "r"(bar) : "memory");
+        if (TWO)
+            asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                         :: "r"(smem_addr(dst + p.part_bytes)), "l"((const uint8_t*)a.b + e0 * ESZ),
+                            "r"(bb), "r"(bar) : "memory");
+    };
+    if (tid == 0) {
+        for (int i = 0; i < S; ++i) {
+            const int64_t tile = blockIdx.x + (int64_t)i * grid;
+            if (tile >= p.n_tiles) break;
+            issue(tile, i);
+        }
+    }
+    GState st;
+    st.seg = -1;
+    int slot = 0;
+    uint32_t parity = 0;
+    for (int64_t tile = blockIdx.x; tile < p.n_tiles; tile += grid) {
+        const bool ok = mbar_wait(smem_addr(&bars[slot]), parity);
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) {
+                atomicOr(&g_pipe_error, 1u);
+                int s2 = slot;
+                uint32_t p2 = parity;
+                for (int i = 0; i < S; ++i) {
+                    const int64_t t2 = tile + (int64_t)i * grid;
+                    if (t2 >= p.n_tiles) break;
+                    mbar_wait(smem_addr(&bars[s2]), p2);
+                    if (++s2 == S) { s2 = 0; p2 ^= 1u; }
+                }
+            }
+            __syncthreads();
+            return;
+        }
+        const int64_t seg = tile * p.P + team;
+        if (seg < a.n_seg) {
+            if constexpr (TWO && TEAM >= 32) load_group_warp_mask<T, PSRC, RHAZ>(a, seg, lane == 0, st);
+            else load_group<T, PSRC, TWO, RHAZ>(a, seg, lane == 0, st);
+            const uint8_t* sa = ring + (size_t)slot * p.slot_bytes + (size_t)team * G * p.in_esz;
+            const uint8_t* sb = ring + (size_t)slot * p.slot_bytes + p.part_bytes + (size_t)team * G * ESZ;
+            const int64_t gbase = seg * G;
+#pragma unroll
+            for (int j = 0; j < NV; ++j) {
+                const int e = (j * TEAM + lane) * W;              // element offset in the group
+                if (!full_groups && e >= G) continue;
+                Acc o[W];
+                if constexpr (OP == OP_DEQ) {
+                    if constexpr (W == 8) {
+                        uint32_t w0, w1;
+                        asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(smem_addr(sa + e)));
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) o[k] = deq_code_f(w0, k, st, a.cfg.q_signed);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) o[4 + k] = deq_code_f(w1, k, st, a.cfg.q_signed);
+                    } else {
+                        uint32_t w0;
+                        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w0) : "r"(smem_addr(sa + e)));
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) o[k] = deq_code_f(w0, k, st, a.cfg.q_signed);
+                    }
+                    st16((T*)a.out + gbase + e, pack_vec<T>(o));
+                } else {
+                    Acc xa[W], xb[W];
+                    load_vec<T>(ld_shared16(smem_addr(sa + (size_t)e * ESZ)), xa);
+                    if constexpr (TWO) load_vec<T>(ld_shared16(smem_addr(sb + (size_t)e * ESZ)), xb);
+                    uint32_t cw[W];
+                    if constexpr (TWO) {
+                        if (st.fast) {
+#pragma unroll
+                            for (int k = 0; k < W; ++k) o[k] = elem_bwd_fast<OP>(xa[k], xb[k], st);
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < W; ++k) o[k] = elem_f<OP, RHAZ>(xa[k], xb[k], st, &cw[k]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < W; ++k) o[k] = elem_f<OP, RHAZ>(xa[k], 0.0f, st, &cw[k]);
+                    }
+                    if constexpr (OP == OP_QUANT) {
+                        uint8_t* q = (uint8_t*)a.out + gbase + e;
+                        if constexpr (W == 8) st8(q, pack4_lowbytes(cw[0], cw[1], cw[2], cw[3]), pack4_lowbytes(cw[4], cw[5], cw[6], cw[7]));
+                        else st4(q, pack4_lowbytes(cw[0], cw[1], cw[2], cw[3]));
+                    } else {
+                        st16((T*)a.out + gbase + e, pack_vec<T>(o));
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        if (tid == 0) {
+            const int64_t next = tile + (int64_t)S * grid;
+            if (next < p.n_tiles) {
+                fence_proxy_async();
+                issue(next, slot);
+            }
+        }
+        if (++slot == S) { slot = 0; parity ^= 1u; }
+    }
+}
+
+// ------------------------------------------------------------ launchers
+// Resident 256-thread blocks per SM of kernel k with `smem` bytes of dynamic
+// shared memory. Each caller passes its own `cache` (a static array in the
+// launcher of one kernel instantiation), which remembers the answer for up to
+// eight distinct ring sizes, so the query runs once per process and size.
+static int occupancy_for(const void* k, size_t smem, unsigned long long (&cache)[8]) {
+    for (int i = 0; i < 8; ++i) {
+        const unsigned long long e = __atomic_load_n(&cache[i], __ATOMIC_RELAXED);
+        if (e == 0) break;
+        if ((e >> 8) == smem) return (int)(e & 0xFFu) - 1;
+    }
+    int v = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, k, 256, smem) != cudaSuccess) {
+        (void)cudaGetLastError();
+        v = 0;
+    }
+    const unsigned long long ent = ((unsigned long long)smem << 8) | (unsigned long long)(v + 1);
+    for (int i = 0; i < 8; ++i) {
+        unsigned long long expected = 0;
+        if (__atomic_compare_exchange_n(&cache[i], &expected, ent, false, __ATOMIC_RELAXED,
+                                        __ATOMIC_RELAXED) || (expected >> 8) == smem)
+            break;
+    }
+    return v;
+}
+
+template <class T, int PK, int TEAM, int NV, bool SYM>
+static cudaError_t launch_pipe_t(PipeArgs a, cudaStream_t st) {
+    constexpr int P = 256 / TEAM;
+    constexpr int S = PipeStages<NV>::S;
+    a.P = P;
+    a.slot_bytes = P * a.G * (int)sizeof(T);
+    a.n_tiles = (a.n_seg + P - 1) / P;
+    a.stages = S;
+    const size_t smem = 128 + (size_t)S * a.slot_bytes;
+    auto k = k_seg_pipe<T, PK, TEAM, NV, SYM>;
+    // Largest ring this instantiation can need: P groups of TEAM*NV vectors.
+    static const cudaError_t attr = cudaFuncSetAttribute(
+        k, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 + S * P * TEAM * NV * 16);
+    if (attr != cudaSuccess) return attr;
+    static unsigned long long occ[8];
+    const int bps = occupancy_for((const void*)k, smem, occ);
+    if (bps < 1) return cudaErrorNotSupported;
+    int64_t grid = (int64_t)sm_count() * bps;
+    if (grid > a.n_tiles) grid = a.n_tiles;
+    k<<<(unsigned)grid, 256, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+// Configuration by vectors per group U (TEAM lanes x NV vectors >= U).
+template <class T, int PK, bool SYM>
+static cudaError_t launch_pipe_u(const PipeArgs& a, cudaStream_t st) {
+    constexpr int VEC = Traits<T>::VEC;
+    const int U = a.G / VEC;
+    if (U <= 1) return launch_pipe_t<T, PK, 1, 1, SYM>(a, st);
+    if (U <= 2) return launch_pipe_t<T, PK, 1, 2, SYM>(a, st);
+    if (U <= 4) return launch_pipe_t<T, PK, 1, 4, SYM>(a, st);
+    if (U <= 8) return launch_pipe_t<T, PK, 2, 4, SYM>(a, st);
+    if (U <= 16) return launch_pipe_t<T, PK, 4, 4, SYM>(a, st);
+    if (U <= 32) return launch_pipe_t<T, PK, 8, 4, SYM>(a, st);
+    if constexpr (PK == PK_INT_Q || PK == PK_INT_FAKE) {
+        if (U <= 64) return launch_pipe_t<T, PK, 16, 4, SYM>(a, st);
+        if (U <= 128) return launch_pipe_t<T, PK, 32, 4, SYM>(a, st);
+        if (U <= 256) return launch_pipe_t<T, PK, 64, 4, SYM>(a, st);
+        if (U <= 512) return launch_pipe_t<T, PK, 64, 8, SYM>(a, st);
+        if (U <= 1024) return launch_pipe_t<T, PK, 128, 8, SYM>(a, st);
+        if (U <= 2048) return launch_pipe_t<T, PK, 256, 8, SYM>(a, st);
+    }
+    return cudaErrorNotSupported;
+}
+
+template <class T>
+static cudaError_t pipe_dt(int pk, bool sym, const PipeArgs& a, cudaStream_t st) {
+    switch (pk) {
+        case PK_INT_Q: return sym ? launch_pipe_u<T, PK_INT_Q, true>(a, st) : launch_pipe_u<T, PK_INT_Q, false>(a, st);
+        case PK_INT_FAKE: return sym ? launch_pipe_u<T, PK_INT_FAKE, true>(a, st) : launch_pipe_u<T, PK_INT_FAKE, false>(a, st);
+        case PK_FP8: return launch_pipe_u<T, PK_FP8, true>(a, st);
+        case PK_MX: return launch_pipe_u<T, PK_MX, true>(a, st);
+        case PK_NV: return launch_pipe_u<T, PK_NV, true>(a, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+template <class T, int OP, int PSRC, bool RHAZ>
+static cudaError_t launch_map_pipe_t(const MapArgs& m, cudaStream_t st) {
+    constexpr int W = Traits<T>::VEC;
+    constexpr int S = MapShape<OP>::S;
+    MapPipeArgs p;
+    p.m = m;
+    p.tile_elems = 256 * MapShape<OP>::ITEMS * W;
+    p.in_esz = (OP == OP_DEQ) ? 1 : (int)sizeof(T);
+    const int two = (OP == OP_QBWD || OP == OP_FBWD) ? (int)sizeof(T) : 0;
+    p.slot_bytes = p.tile_elems * (p.in_esz + two);
+    p.stages = S;
+    p.n_tiles = (m.numel + p.tile_elems - 1) / p.tile_elems;
+    const size_t smem = 128 + (size_t)S * p.slot_bytes;
+    auto k = k_map_pipe<T, OP, PSRC, RHAZ>;
+    static const cudaError_t attr = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (attr != cudaSuccess) return attr;
+    static unsigned long long occ[8];
+    const int bps = occupancy_for((const void*)k, smem, occ);
+    if (bps < 1) return cudaErrorNotSupported;
+    int64_t grid = (int64_t)sm_count() * bps;
+    if (grid > p.n_tiles) grid = p.n_tiles;
+    k<<<(unsigned)grid, 256, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+template <class T, int OP, int PSRC>
+static cudaError_t map_pipe_r(const MapArgs& m, cudaStream_t st) {
+    return m.cfg.rhaz ? launch_map_pipe_t<T, OP, PSRC, true>(m, st) : launch_map_pipe_t<T, OP, PSRC, false>(m, st);
+}
+
+template <class T>
+static cudaError_t map_pipe_dt(int op, int psrc, const MapArgs& m, cudaStream_t st) {
+    switch (op) {
+        case OP_QUANT: return psrc == PS_RANGE ? map_pipe_r<T, OP_QUANT, PS_RANGE>(m, st) : map_pipe_r<T, OP_QUANT, PS_STATIC>(m, st);
+        case OP_FAKE: return psrc == PS_RANGE ? map_pipe_r<T, OP_FAKE, PS_RANGE>(m, st) : map_pipe_r<T, OP_FAKE, PS_STATIC>(m, st);
+        case OP_QBWD: return map_pipe_r<T, OP_QBWD, PS_STATIC>(m, st);
+        case OP_FBWD: return map_pipe_r<T, OP_FBWD, PS_STATIC>(m, st);
+        case OP_DEQ: return map_pipe_r<T, OP_DEQ, PS_STATIC>(m, st);
+        case OP_DBWD: return map_pipe_r<T, OP_DBWD, PS_STATIC>(m, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+template <class T, int OP, int PSRC, int TEAM, int NV, bool RHAZ>
+static cudaError_t launch_seg_map_t(const MapArgs& m, cudaStream_t st) {
+    constexpr int P = 256 / TEAM;
+    constexpr int S = SegMapStages<OP>::S;
+    constexpr bool TWO = (OP == OP_QBWD || OP == OP_FBWD);
+    SegMapArgs p;
+    p.m = m;
+    p.P = P;
+    p.n_tiles = (m.n_seg + P - 1) / P;
+    p.in_esz = (OP == OP_DEQ) ? 1 : (int)sizeof(T);
+    p.part_bytes = P * (int)m.G * p.in_esz;
+    p.slot_bytes = p.part_bytes + (TWO ? P * (int)m.G * (int)sizeof(T) : 0);
+    const size_t smem = 128 + (size_t)S * p.slot_bytes;
+    constexpr int in_max = (OP == OP_DEQ) ? 1 : (int)sizeof(T);
+    constexpr int max_slot = P * TEAM * NV * Traits<T>::VEC * (in_max + (TWO ? (int)sizeof(T) : 0));
+    auto k = k_seg_map<T, OP, PSRC, TEAM, NV, RHAZ>;
+    static const cudaError_t attr = cudaFuncSetAttribute(
+        k, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 + S * max_slot);
+    if (attr != cudaSuccess) return attr;
+    static unsigned long long occ[8];
+    const int bps = occupancy_for((const void*)k, smem, occ);
+    if (bps < 1) return cudaErrorNotSupported;
+    int64_t grid = (int64_t)sm_count() * bps;
+    if (grid > p.n_tiles) grid = p.n_tiles;
+    k<<<(unsigned)grid, 256, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+// (TEAM, NV) by vectors per group U in [5, 1024]; ring slots stay within 32 KB.
+template <class T, int OP, int PSRC, bool RHAZ>
+static cudaError_t seg_map_u(const MapArgs& m, cudaStream_t st) {
+    const int64_t U = m.G / Traits<T>::VEC;
+    if (U <= 4) return cudaErrorNotSupported;
+    if (U <= 8) return launch_seg_map_t<T, OP, PSRC, 2, 4, RHAZ>(m, st);
+    if (U <= 16) return launch_seg_map_t<T, OP, PSRC, 4, 4, RHAZ>(m, st);
+    if (U <= 32) return launch_seg_map_t<T, OP, PSRC, 8, 4, RHAZ>(m, st);
+    if (U <= 64) return launch_seg_map_t<T, OP, PSRC, 16, 4, RHAZ>(m, st);
+    if (U <= 128) return launch_seg_map_t<T, OP, PSRC, 32, 4, RHAZ>(m, st);
+    if (U <= 256) return launch_seg_map_t<T, OP, PSRC, 64, 4, RHAZ>(m, st);
+    if (U <= 512) return launch_seg_map_t<T, OP, PSRC, 128, 4, RHAZ>(m, st);
+    if (U <= 1024) return launch_seg_map_t<T, OP, PSRC, 256, 4, RHAZ>(m, st);
+    return cudaErrorNotSupported;
+}
+
+// Group-tiled element kernels: dequantize and the backwards with nearest-even
+// rounding (other element ops take the flat pipelined kernel).
+template <class T>
+static cudaError_t seg_map_dt(int op, const MapArgs& m, cudaStream_t st) {
+    if (m.cfg.rhaz && (op == OP_QBWD || op == OP_FBWD)) return cudaErrorNotSupported;
+    switch (op) {
+        case OP_QBWD: return seg_map_u<T, OP_QBWD, PS_STATIC, false>(m, st);
+        case OP_FBWD: return seg_map_u<T, OP_FBWD, PS_STATIC, false>(m, st);
+        case OP_DEQ: return seg_map_u<T, OP_DEQ, PS_STATIC, false>(m, st);
+        case OP_DBWD: return seg_map_u<T, OP_DBWD, PS_STATIC, false>(m, st);
+    }
+    return cudaErrorNotSupported;
+}
+
+// Entry points of one dtype's translation unit.
+template <class T>
+cudaError_t pipe_dyn_entry(int pk, bool sym, const PipeArgs& a, cudaStream_t st) {
+    return pipe_dt<T>(pk, sym, a, st);
+}
+
+template <class T>
+cudaError_t pipe_map_entry(int op, const MapArgs& m, cudaStream_t st) {
+    const int in_esz = (op == OP_DEQ) ? 1 : (int)sizeof(T);
+    if (m.n_seg > 0 && (m.G * in_esz) % 16 == 0) {
+        const cudaError_t e = seg_map_dt<T>(op, m, st);
+        if (e != cudaErrorNotSupported) return e;
+    }
+    return map_pipe_dt<T>(op, m.ranges ? PS_RANGE : PS_STATIC, m, st);
+}
+
+template <class T>
+cudaError_t pipe_error_entry(unsigned int* flag) {
+    unsigned int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(flag, g_pipe_error, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    return cudaMemcpyToSymbol(g_pipe_error, &zero, sizeof(unsigned int));
+}
+
+}  // namespace
+
+#define BQ_PIPE_ENTRIES(T, NAME)                                                        \
+    cudaError_t pipe_dyn_##NAME(int pk, bool sym, const PipeArgs& a, cudaStream_t st) { \
+        return pipe_dyn_entry<T>(pk, sym, a, st);                                        \
+    }                                                                                    \
+    cudaError_t pipe_map_##NAME(int op, const MapArgs& m, cudaStream_t st) {            \
+        return pipe_map_entry<T>(op, m, st);                                             \
+    }                                                                                    \
+    cudaError_t pipe_err_##NAME(unsigned int* flag) { return pipe_error_entry<T>(flag); }
+
+}  // namespace bq

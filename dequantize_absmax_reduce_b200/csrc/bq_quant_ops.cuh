@@ -1,0 +1,163 @@
+// Per-group arithmetic shared by the quantize kernels: scale / zero-point
+// derivation of the integer formats, the MXFP8 shared exponent, and the code
+// emitters for one 16-byte vector of values.
+#pragma once
+
+#include "bq_device.cuh"
+#include "bq_internal.h"
+
+namespace bq {
+
+// ------------------------------------------------------------ group params
+struct GroupF { float s; int zp; };
+struct GroupD { float s; int zp; };
+
+// Scale and zero-point from a group's range (f32 arithmetic). Symmetric:
+// s = fl(amax / qmax). Asymmetric: s = fl(fl(max' - min') / (qmax - qmin)),
+// zp = clamp(qmin - round(fl(min' / s)), qmin, qmax). 0 -> 1.
+__device__ __forceinline__ GroupF derive_f(float hi, float nlo, const IntCfg& c) {
+    GroupF g;
+    if (c.symmetric) {
+        float s = __fdiv_rn(fmaxf(hi, nlo), (float)c.qmax);
+        if (s == 0.0f) s = 1.0f;
+        g.s = s;
+        g.zp = 0;
+    } else {
+        const float span = __fadd_rn(hi, nlo);
+        float s = __fdiv_rn(span, (float)(c.qmax - c.qmin));
+        if (s == 0.0f) s = 1.0f;
+        const float m = __fdiv_rn(-nlo, s);
+        const float r = c.rhaz ? roundf(m) : rintf(m);
+        float z = __fsub_rn((float)c.qmin, r);
+        z = fminf(fmaxf(z, (float)c.qmin), (float)c.qmax);   // NaN -> qmin
+        g.s = s;
+        g.zp = (int)z;
+    }
+    return g;
+}
+// Same in f64 for f64 inputs; the stored scale is still f32.
+__device__ __forceinline__ GroupD derive_d(double hi, double nlo, const IntCfg& c) {
+    GroupD g;
+    if (c.symmetric) {
+        float s = __double2float_rn(fmax(hi, nlo) / (double)c.qmax);
+        if (s == 0.0f) s = 1.0f;
+        g.s = s;
+        g.zp = 0;
+    } else {
+        const double span = hi + nlo;
+        float s = __double2float_rn(span / (double)(c.qmax - c.qmin));
+        if (s == 0.0f) s = 1.0f;
+        const double m = -nlo / (double)s;
+        const double r = c.rhaz ? round(m) : rint(m);
+        double z = (double)c.qmin - r;
+        z = fmin(fmax(z, (double)c.qmin), (double)c.qmax);
+        g.s = s;
+        g.zp = (int)z;
+    }
+    return g;
+}
+
+__device__ __forceinline__ int load_zp(const void* zp, int64_t g, int q_signed) {
+    if (!zp) return 0;
+    const uint8_t b = __ldg((const uint8_t*)zp + g);
+    return q_signed ? (int)(int8_t)b : (int)b;
+}
+
+
+// Group sizes of the microscaled formats.
+template <int FMT> struct MxG;
+template <> struct MxG<MX_FP8_1x128> { static constexpr int G = 128; };
+template <> struct MxG<MX_MXFP8> { static constexpr int G = 32; };
+template <> struct MxG<MX_NVFP4> { static constexpr int G = 16; };
+
+
+__device__ __forceinline__ void st2(void* p, uint32_t a) {
+    asm volatile("st.global.u16 [%0], %1;" :: "l"(p), "h"((uint16_t)a) : "memory");
+}
+
+// MXFP8 shared exponent: E = clamp(floor(log2 a) - 8, -127, 127), from the
+// bits of a >= 0 (a subnormal a counts its leading zeros; infinity is 2^128;
+// a = 0 gives -127).
+__device__ __forceinline__ int mx_exponent(float a) {
+    const uint32_t b = __float_as_uint(a);
+    const int ex = (int)(b >> 23);
+    int fl2;
+    if (ex == 0) {
+        const uint32_t m = b & 0x7FFFFFu;
+        fl2 = (m == 0) ? -1000 : (31 - __clz((int)m)) - 149;
+    } else if (ex == 255) {
+        fl2 = 128;
+    } else {
+        fl2 = ex - 127;
+    }
+    return min(max(fl2 - 8, -127), 127);
+}
+
+
+// Codes of one 16-byte vector (v: its VEC values) written at dst.
+template <class T, int FMT, bool FAST>
+__device__ __forceinline__ void mx_emit(const float* v, const Recip& R, float mul, bool zero,
+                                        uint8_t* dst) {
+    constexpr int VEC = Traits<T>::VEC;
+    float t[VEC];
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) {
+        if constexpr (FMT == MX_MXFP8) {
+            t[i] = __fmul_rn(v[i], mul);
+        } else {
+            const float d = FAST ? div_chain(v[i], R) : div_any(v[i], R);
+            t[i] = with_quotient_sign(d, v[i], R.s);
+        }
+    }
+    if constexpr (FMT == MX_NVFP4) {
+        if constexpr (VEC == 8) {
+            const float (&t8)[8] = *reinterpret_cast<const float(*)[8]>(t);
+            st4(dst, zero ? 0u : e2m1x8(t8));
+        } else {
+            float t8[8] = {t[0], t[1], t[2], t[3], 0.f, 0.f, 0.f, 0.f};
+            st2(dst, zero ? 0u : (e2m1x8(t8) & 0xFFFFu));
+        }
+    } else {
+        if constexpr (VEC == 8) {
+            st8(dst, e4m3x4(t[0], t[1], t[2], t[3]), e4m3x4(t[4], t[5], t[6], t[7]));
+        } else {
+            st4(dst, e4m3x4(t[0], t[1], t[2], t[3]));
+        }
+    }
+}
+
+
+// Integer codes (QUANT) or fake-quantized values (FAKE) of one vector of
+// VEC values. SYM_DYN: symmetric scale derived from this group's own range.
+// When that scale is also a normal number (FAST: 2^-64 <= s <= 2^64) it is
+// within 2^-24 of amax/qmax, so |x/s| <= qmax (1 + 2^-23) rounds to at most
+// qmax and only the lower clamp (which also takes a NaN to qmin) can bind.
+template <class T, int OP, bool FAST, bool SYM_DYN>
+__device__ __forceinline__ void emit_int(const float* v, const Recip& R, const IntParams& ip,
+                                         uint8_t* q, T* y) {
+    constexpr int VEC = Traits<T>::VEC;
+    float t[VEC];
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) {
+        const float qv = FAST ? div_chain(v[i], R) : div_slow(v[i], R.s);
+        if constexpr (SYM_DYN && FAST) t[i] = __fadd_rn(fmaxf(qv, ip.lo), kMagic);
+        else t[i] = rounded_rne(qv, ip);
+    }
+    if constexpr (OP == OP_QUANT) {
+        uint32_t cw[VEC];
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) cw[i] = code_from_rounded(t[i], SYM_DYN ? 0 : ip.zp);
+        if constexpr (VEC == 8) {
+            st8(q, pack4_lowbytes(cw[0], cw[1], cw[2], cw[3]), pack4_lowbytes(cw[4], cw[5], cw[6], cw[7]));
+        } else {
+            st4(q, pack4_lowbytes(cw[0], cw[1], cw[2], cw[3]));
+        }
+    } else {
+        float o[VEC];
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) o[i] = dequant_from_rounded(t[i], R.s);
+        st16(y, pack_vec<T>(o));
+    }
+}
+
+}  // namespace bq

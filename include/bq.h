@@ -37,7 +37,8 @@
  *     BQ_ERR_UNSUPPORTED (dtype combination or mode not provided, e.g. a
  *     symmetric u8 code range); BQ_ERR_MISALIGNED (reserved);
  *     BQ_ERR_CUDA (a launch failed: cudaGetLastError after the launch);
- *     BQ_ERR_TIMEOUT (reserved: no kernel here waits on another).
+ *     BQ_ERR_TIMEOUT (from bq_check_device_error only: a bounded wait of a
+ *     kernel on its own bulk copies expired).
  *   - Arithmetic: f32/f16/bf16 inputs are widened exactly to f32 and every
  *     step is one IEEE f32 operation with round-to-nearest-even (a divide is
  *     the correctly rounded quotient); f64 inputs use f64. Results are
@@ -148,6 +149,12 @@ bq_status bq_group_range(const void* x, const bq_qdesc* d, bq_gran gran, int32_t
  * ([QuantizedWeight] weight_scale_2). */
 bq_status bq_tensor_amax(const void* x, bq_dtype dtype, int64_t n, float* amax, void* ws,
                          void* stream);
+
+/* Synchronises the current device, then reports whether a pipelined kernel
+ * gave up waiting for one of its bulk copies since the last call
+ * (BQ_ERR_TIMEOUT; the flag is cleared) — a bounded wait that is never
+ * expected to expire. Host only; the one call here that blocks. */
+bq_status bq_check_device_error(void);
 
 /* -------------------------------------------------------------- quantize */
 /* [baracuda] quantize_per_tensor / per_channel / per_token / per_group.
