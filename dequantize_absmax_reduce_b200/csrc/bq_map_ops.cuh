@@ -137,6 +137,21 @@ __device__ __forceinline__ bool mask_thresholds_warp(const Recip& R, const IntPa
     return true;
 }
 
+// Group state from a known scale and zero-point (static parameters).
+template <class T, bool MASK, bool RHAZ>
+__device__ __forceinline__ void group_set(const MapArgs& a, int64_t seg, float s, int zp, GState& st) {
+    using Acc = typename Traits<T>::Acc;
+    st.seg = seg;
+    st.s = s;
+    st.zp = zp;
+    st.R = make_recip(s);
+    st.ip = make_int_params(a.cfg.qmin, a.cfg.qmax, zp);
+    st.mfast = false;
+    if constexpr (MASK && !std::is_same<Acc, double>::value)
+        st.mfast = mask_thresholds<RHAZ>(st.R, st.ip, &st.x_lo, &st.x_hi);
+    st.fast = st.mfast && st.R.fast;
+}
+
 template <class T, int PSRC, bool MASK = false, bool RHAZ = false>
 __device__ __forceinline__ void load_group(const MapArgs& a, int64_t seg, bool writer, GState& st) {
     using Acc = typename Traits<T>::Acc;

@@ -135,8 +135,24 @@ __device__ __forceinline__ void range_finish(uint32_t ph, uint32_t pl, float& hi
 }
 
 // ------------------------------------------------------------ the kernel
-// Ring depth: 4 slots of up to 16 KB, or 3 of up to 32 KB (NV = 8).
-template <int NV> struct PipeStages { static constexpr int S = NV <= 4 ? 4 : 3; };
+// Tuning constants (compile-time): ring depth of the dynamic quantizer for
+// slots of up to 16 KB (NV <= 4) and 32 KB (NV = 8); team width for groups of
+// 257..512 vectors (the per-token rows of 4096 bf16); ring depth of the
+// group-tiled element kernels.
+#ifndef BQ_SEG_STAGES_16K
+#define BQ_SEG_STAGES_16K 4
+#endif
+#ifndef BQ_SEG_STAGES_32K
+#define BQ_SEG_STAGES_32K 3
+#endif
+#ifndef BQ_SEG_TEAM_512
+#define BQ_SEG_TEAM_512 64
+#endif
+#ifndef BQ_MAP_STAGES
+#define BQ_MAP_STAGES 3
+#endif
+
+template <int NV> struct PipeStages { static constexpr int S = NV <= 4 ? BQ_SEG_STAGES_16K : BQ_SEG_STAGES_32K; };
 
 template <class T, int PK, int TEAM, int NV, bool SYM>
 __global__ void __launch_bounds__(256) k_seg_pipe(PipeArgs a) {
@@ -535,7 +551,7 @@ struct SegMapArgs {
     int slot_bytes;
 };
 
-template <int OP> struct SegMapStages { static constexpr int S = 3; };
+template <int OP> struct SegMapStages { static constexpr int S = BQ_MAP_STAGES; };
 
 template <class T, int OP, int PSRC, int TEAM, int NV, bool RHAZ>
 __global__ void __launch_bounds__(256) k_seg_map(SegMapArgs p) {
@@ -586,6 +602,17 @@ __global__ void __launch_bounds__(256) k_seg_map(SegMapArgs p) {
     st.seg = -1;
     int slot = 0;
     uint32_t parity = 0;
+    // Static group parameters, loaded one tile ahead so their latency hides
+    // behind the current tile's work.
+    auto fetch = [&](int64_t sg, float& s, int& z) {
+        if (sg < a.n_seg) {
+            s = __ldg(a.scale_in + sg);
+            z = a.cfg.symmetric ? 0 : load_zp(a.zp_in, sg, a.cfg.q_signed);
+        }
+    };
+    float pf_s = 1.0f;
+    int pf_z = 0;
+    fetch((int64_t)blockIdx.x * p.P + team, pf_s, pf_z);
     for (int64_t tile = blockIdx.x; tile < p.n_tiles; tile += grid) {
         const bool ok = mbar_wait(smem_addr(&bars[slot]), parity);
         if (__syncthreads_or(!ok)) {
@@ -604,9 +631,17 @@ __global__ void __launch_bounds__(256) k_seg_map(SegMapArgs p) {
             return;
         }
         const int64_t seg = tile * p.P + team;
+        const float cur_s = pf_s;
+        const int cur_z = pf_z;
+        fetch((tile + grid) * p.P + team, pf_s, pf_z);
         if (seg < a.n_seg) {
-            if constexpr (TWO && TEAM >= 32) load_group_warp_mask<T, PSRC, RHAZ>(a, seg, lane == 0, st);
-            else load_group<T, PSRC, TWO, RHAZ>(a, seg, lane == 0, st);
+            if constexpr (TWO && TEAM >= 32) {
+                group_set<T, false, RHAZ>(a, seg, cur_s, cur_z, st);
+                st.mfast = mask_thresholds_warp<RHAZ>(st.R, st.ip, &st.x_lo, &st.x_hi);
+                st.fast = st.mfast && st.R.fast;
+            } else {
+                group_set<T, TWO, RHAZ>(a, seg, cur_s, cur_z, st);
+            }
             const uint8_t* sa = ring + (size_t)slot * p.slot_bytes + (size_t)team * G * p.in_esz;
             const uint8_t* sb = ring + (size_t)slot * p.slot_bytes + p.part_bytes + (size_t)team * G * ESZ;
             const int64_t gbase = seg * G;
@@ -733,7 +768,7 @@ static cudaError_t launch_pipe_u(const PipeArgs& a, cudaStream_t st) {
         if (U <= 64) return launch_pipe_t<T, PK, 16, 4, SYM>(a, st);
         if (U <= 128) return launch_pipe_t<T, PK, 32, 4, SYM>(a, st);
         if (U <= 256) return launch_pipe_t<T, PK, 64, 4, SYM>(a, st);
-        if (U <= 512) return launch_pipe_t<T, PK, 64, 8, SYM>(a, st);
+        if (U <= 512) return launch_pipe_t<T, PK, BQ_SEG_TEAM_512, 512 / BQ_SEG_TEAM_512, SYM>(a, st);
         if (U <= 1024) return launch_pipe_t<T, PK, 128, 8, SYM>(a, st);
         if (U <= 2048) return launch_pipe_t<T, PK, 256, 8, SYM>(a, st);
     }
