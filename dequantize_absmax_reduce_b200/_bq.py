@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libbq.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m dequantize_absmax_reduce_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python dequantize_absmax_reduce_b200/build.py` "
         "(there is no CPU fallback)")
 
 lib = C.CDLL(LIB_PATH)
