@@ -30,6 +30,7 @@ BQ_F32, BQ_F64, BQ_F16, BQ_BF16, BQ_S8, BQ_U8, BQ_E4M3, BQ_E2M1X2, BQ_E8M0 = ran
 BQ_RNE, BQ_RHAZ = 0, 1
 BQ_GRAN_TENSOR, BQ_GRAN_CHANNEL, BQ_GRAN_GROUP = 0, 1, 2
 BQ_SCALE_DYNAMIC, BQ_SCALE_STATIC, BQ_SCALE_FROM_RANGE = 0, 1, 2
+BQ_NOALLOC_MAX_GROUPS = 65536
 
 DTYPE = {torch.float32: BQ_F32, torch.float64: BQ_F64, torch.float16: BQ_F16,
          torch.bfloat16: BQ_BF16, torch.int8: BQ_S8, torch.uint8: BQ_U8}
@@ -62,6 +63,7 @@ _SIGS = {
     "bq_quantize_per_channel": [_P, _DESC, _I32, _P, _P, _P, C.c_int, _P, _SZ, _P],
     "bq_quantize_per_token": [_P, _DESC, _P, _P, _P, C.c_int, _P, _SZ, _P],
     "bq_quantize_per_group": [_P, _DESC, _I32, _I64, _P, _P, _P, C.c_int, _P, _SZ, _P],
+    "bq_quantize_dynamic_noalloc": [_P, _DESC, C.c_int, _I32, _I64, _P, _P, _P, _P],
     "bq_dequantize_per_tensor": [_P, _P, _P, _DESC, _P, C.c_int, _P],
     "bq_dequantize_per_channel": [_P, _P, _P, _DESC, _I32, _P, C.c_int, _P],
     "bq_dequantize_per_token": [_P, _P, _P, _DESC, _P, C.c_int, _P],
@@ -215,6 +217,12 @@ def bq_quantize_per_group(x, d, axis, group_size, q, scale, zp, mode, ws=None, s
     _check(lib.bq_quantize_per_group(_ptr(x), C.byref(d), axis, group_size, _ptr(q), _ptr(scale),
                                      _ptr(zp), _m(mode), _ptr(ws), _nbytes(ws), _stream(stream)),
            "bq_quantize_per_group")
+
+
+def bq_quantize_dynamic_noalloc(x, d, gran, axis, group_size, q, scale, zp, stream=None):
+    _check(lib.bq_quantize_dynamic_noalloc(_ptr(x), C.byref(d), _g(gran), axis, group_size, _ptr(q),
+                                           _ptr(scale), _ptr(zp), _stream(stream)),
+           "bq_quantize_dynamic_noalloc")
 
 
 # ---------------------------------------------------------------- dequantize

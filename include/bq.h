@@ -176,6 +176,37 @@ bq_status bq_quantize_per_group(const void* x, const bq_qdesc* d, int32_t axis,
                                 int64_t group_size, void* q, float* scale, void* zp,
                                 bq_scale_mode mode, void* ws, size_t ws_bytes, void* stream);
 
+/* Dynamic quantize without caller workspace. The sources cited above have no
+ * counterpart: this is a library convenience for callers that cannot hand
+ * the library device memory (a C host with no device allocator of its own
+ * that cannot size `ws` ahead of the call, or a path that must not call
+ * cudaMalloc, which can synchronise the device and fail under pressure).
+ * Same arguments and results as bq_quantize_per_tensor / per_channel /
+ * per_group with mode BQ_SCALE_DYNAMIC (per-token: BQ_GRAN_GROUP with
+ * axis = ndim - 1 and group_size = the last dimension). The range records of
+ * the two-pass path (per-tensor, or groups too long for one pass) live in a
+ * fixed array of BQ_NOALLOC_MAX_GROUPS records (16 bytes each, 1 MiB) in the
+ * library's device memory, one array per device; the call clears the
+ * records it uses on `stream` before filling them, so nothing has to be
+ * zero beforehand.
+ *   - BQ_ERR_INVALID_ARG, with nothing enqueued, when the call needs more
+ *     than BQ_NOALLOC_MAX_GROUPS records
+ *     (bq_quantize_workspace_size(d, gran, axis, group_size, DYNAMIC) >
+ *     16 * BQ_NOALLOC_MAX_GROUPS); other errors as the workspace entries.
+ *   - The first call on each device resolves the array's address there
+ *     (cudaGetSymbolAddress on the current device, done once and cached);
+ *     make that first call before any stream capture starts.
+ *   - The array is shared: calls whose work may overlap on one device (on
+ *     different streams without ordering between them, or from several host
+ *     threads) race on it and may write wrong scales. Calls on one stream,
+ *     or ordered by events, are safe. The library allocates nothing here
+ *     either; unlike every other entry point this one keeps device state
+ *     (the array) between calls. */
+#define BQ_NOALLOC_MAX_GROUPS 65536
+bq_status bq_quantize_dynamic_noalloc(const void* x, const bq_qdesc* d, bq_gran gran,
+                                      int32_t axis, int64_t group_size, void* q, float* scale,
+                                      void* zp, void* stream);
+
 /* ------------------------------------------------------------ dequantize */
 /* [baracuda] dequantize_per_tensor / per_channel / per_token / per_group:
  * y = RN_y(fl((q - zp) * scale)); y has shape d->shape and dtype y_dtype

@@ -1,0 +1,93 @@
+"""bq_quantize_dynamic_noalloc: dynamic quantize with the library's own fixed
+range-record array instead of caller workspace.
+
+Compared bit for bit (codes, scales, zero-points) with the workspace entry
+points on the same inputs. Two calls in a row, the first on a tensor of
+larger magnitude, show that each call starts from cleared records. The file
+is named to be collected last, so it also runs after every other GPU test
+has used the device; it passes alone as well (the first call then does the
+per-device set-up).
+"""
+
+import ctypes
+
+import pytest
+import torch
+
+import synthetic
+from parity import assert_bitwise
+
+DT = {"f32": torch.float32, "f64": torch.float64, "f16": torch.float16, "bf16": torch.bfloat16}
+
+
+@pytest.fixture(scope="module")
+def B():
+    import dequantize_absmax_reduce_b200 as m
+    return m
+
+
+def _reference_call(B, x, gran, axis, gs, qd, sym):
+    """The workspace entry point, with workspace sized by the library."""
+    d = B.make_desc(x.shape, x.dtype, qd, sym)
+    n_groups, _ = B.bq_group_count(d, gran, axis, gs)
+    q = torch.empty(x.shape, dtype=qd, device=x.device)
+    scale = torch.empty(max(n_groups, 1), dtype=torch.float32, device=x.device)
+    zp = torch.empty(max(n_groups, 1), dtype=qd, device=x.device)
+    nbytes = B.bq_quantize_workspace_size(d, gran, axis, gs, "dynamic")
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=x.device)
+    if gran == "tensor":
+        B.bq_quantize_per_tensor(x, d, q, scale, zp, "dynamic", ws)
+    elif gran == "channel":
+        B.bq_quantize_per_channel(x, d, axis, q, scale, zp, "dynamic", ws)
+    else:
+        B.bq_quantize_per_group(x, d, axis, gs, q, scale, zp, "dynamic", ws)
+    return q, scale, zp
+
+
+def _noalloc_call(B, x, gran, axis, gs, qd, sym):
+    d = B.make_desc(x.shape, x.dtype, qd, sym)
+    n_groups, _ = B.bq_group_count(d, gran, axis, gs)
+    q = torch.empty(x.shape, dtype=qd, device=x.device)
+    scale = torch.empty(max(n_groups, 1), dtype=torch.float32, device=x.device)
+    zp = torch.empty(max(n_groups, 1), dtype=qd, device=x.device)
+    B.bq_quantize_dynamic_noalloc(x, d, gran, axis, gs, q, scale, zp)
+    return q, scale, zp
+
+
+CASES = [  # (shape, dtype, gran, axis, group_size, q dtype, symmetric)
+    ((4096, 4096), "bf16", "tensor", 0, 1, torch.int8, True),      # two passes, one record
+    ((1000, 777), "f32", "tensor", 0, 1, torch.uint8, False),      # ragged, asymmetric
+    ((8, 65536), "bf16", "group", 1, 65536, torch.int8, True),     # groups too long for one pass
+    ((6, 40000), "f16", "channel", 0, 1, torch.uint8, False),
+    ((65536,), "f64", "channel", 0, 1, torch.int8, True),          # exactly the maximum record count
+    ((512, 4096), "bf16", "group", 1, 4096, torch.int8, True),     # per-token rows: one pass
+    ((300, 1024), "f32", "group", 1, 128, torch.uint8, False),
+]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("shape,dt,gran,axis,gs,qd,sym", CASES)
+def test_noalloc_matches_workspace_entry_two_calls(B, shape, dt, gran, axis, gs, qd, sym):
+    st = synthetic.Stream(0x5EED0 + len(shape) * 7 + shape[-1])
+    x_big = st.tensor(shape, dt, std=8.0).cuda()
+    x_small = st.tensor(shape, dt, std=0.25).cuda()
+    for x in (x_big, x_small):   # back to back: the second must not see the first's records
+        q, s, z = _noalloc_call(B, x, gran, axis, gs, qd, sym)
+        rq, rs, rz = _reference_call(B, x, gran, axis, gs, qd, sym)
+        torch.cuda.synchronize()
+        assert_bitwise(q, rq, f"codes {gran} {shape}")
+        assert_bitwise(s, rs, f"scales {gran} {shape}")
+        if not sym:
+            assert_bitwise(z, rz, f"zero-points {gran} {shape}")
+
+
+def test_noalloc_rejects_more_records_than_it_holds(B):
+    """65537 f64 groups need the two-pass path and one record more than the
+    array holds: rejected on the host before any CUDA call (so this also
+    runs without a device), while 65536 groups fit exactly."""
+    at_max = B.make_desc((B.BQ_NOALLOC_MAX_GROUPS,), torch.float64, torch.int8, True)
+    assert B.bq_quantize_workspace_size(at_max, "channel", 0, 1, "dynamic") == 16 * B.BQ_NOALLOC_MAX_GROUPS
+    over = B.make_desc((B.BQ_NOALLOC_MAX_GROUPS + 1,), torch.float64, torch.int8, True)
+    status = B.lib.bq_quantize_dynamic_noalloc(None, ctypes.byref(over), B.BQ_GRAN_CHANNEL, 0, 1,
+                                               None, None, None, None)
+    assert status == B.BQ_ERR_INVALID_ARG
