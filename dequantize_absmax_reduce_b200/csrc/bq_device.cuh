@@ -181,6 +181,97 @@ __device__ __forceinline__ float with_quotient_sign(float q, float x, float s) {
                            ((__float_as_uint(x) ^ __float_as_uint(s)) & 0x80000000u));
 }
 
+// ---------------------------------------------------------------- f32 pairs
+// sm_100 issues add / sub / mul / fma on two f32 lanes held in one 64-bit
+// register pair (PTX .f32x2); each lane is rounded exactly as the scalar
+// instruction rounds it (round-to-nearest-even, subnormals kept). The fast
+// per-element paths run their arithmetic on such pairs: the same bits as the
+// scalar sequence, half the issue slots.
+typedef unsigned long long F2;
+__device__ __forceinline__ F2 f2_pack(float lo, float hi) {
+    F2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_split(F2 v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ void f2_split_bits(F2 v, uint32_t& lo, uint32_t& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(v));
+}
+__device__ __forceinline__ F2 f2_bcast(float v) { return f2_pack(v, v); }
+__device__ __forceinline__ F2 f2_add(F2 a, F2 b) {
+    F2 r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ F2 f2_sub(F2 a, F2 b) {
+    F2 r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ F2 f2_mul(F2 a, F2 b) {
+    F2 r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ F2 f2_fma(F2 a, F2 b, F2 c) {
+    F2 r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+// The two 16-bit floats of one word (low half first), widened exactly.
+__device__ __forceinline__ F2 f2_widen_bf16x2(uint32_t w) {
+    F2 r;
+    asm("{\n\t.reg .b32 lo, hi;\n\t"
+        "shl.b32 lo, %1, 16;\n\t"
+        "and.b32 hi, %1, 0xFFFF0000;\n\t"
+        "mov.b64 %0, {lo, hi};\n\t}"
+        : "=l"(r) : "r"(w));
+    return r;
+}
+__device__ __forceinline__ F2 f2_widen_f16x2(uint32_t w) {
+    F2 r;
+    asm("{\n\t.reg .b16 a, b;\n\t.reg .f32 lo, hi;\n\t"
+        "mov.b32 {a, b}, %1;\n\t"
+        "cvt.f32.f16 lo, a;\n\t"
+        "cvt.f32.f16 hi, b;\n\t"
+        "mov.b64 %0, {lo, hi};\n\t}"
+        : "=l"(r) : "r"(w));
+    return r;
+}
+// One 16-byte vector as VEC/2 pairs, in element order.
+template <class T>
+__device__ __forceinline__ void widen_pairs(const U4& u, F2 (&x)[Traits<T>::VEC / 2]) {
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        x[0] = f2_widen_bf16x2(u.x); x[1] = f2_widen_bf16x2(u.y);
+        x[2] = f2_widen_bf16x2(u.z); x[3] = f2_widen_bf16x2(u.w);
+    } else if constexpr (std::is_same<T, __half>::value) {
+        x[0] = f2_widen_f16x2(u.x); x[1] = f2_widen_f16x2(u.y);
+        x[2] = f2_widen_f16x2(u.z); x[3] = f2_widen_f16x2(u.w);
+    } else {
+        x[0] = f2_pack(__uint_as_float(u.x), __uint_as_float(u.y));
+        x[1] = f2_pack(__uint_as_float(u.z), __uint_as_float(u.w));
+    }
+}
+// div_chain on both lanes of a pair: the same five roundings per lane.
+struct Recip2 {
+    F2 y, ns;   // (RN(1/s), RN(1/s)), (-s, -s)
+};
+__device__ __forceinline__ Recip2 make_recip2(const Recip& r) {
+    Recip2 p;
+    p.y = f2_bcast(r.y);
+    p.ns = f2_bcast(-r.s);
+    return p;
+}
+__device__ __forceinline__ F2 div_chain2(F2 x, const Recip2& r) {
+    const F2 q0 = f2_mul(x, r.y);
+    const F2 e0 = f2_fma(r.ns, q0, x);
+    const F2 q1 = f2_fma(e0, r.y, q0);
+    const F2 e1 = f2_fma(r.ns, q1, x);
+    return f2_fma(e1, r.y, q1);
+}
+
 // ---------------------------------------------------------------- int codes
 // Rounding v (an exact f32 quotient) to an integer code with nearest-even:
 // for |v| <= 2^22, fl(v + 1.5*2^23) has unit spacing, so the addition itself

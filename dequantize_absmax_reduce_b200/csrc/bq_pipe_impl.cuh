@@ -73,9 +73,10 @@ __device__ __forceinline__ U4 ld_shared16(uint32_t addr) {
 
 // ------------------------------------------------------------ range helpers
 // Range of one 16-byte vector, accumulated without widening: for 16-bit types
-// two lanes per instruction (max.xorsign.abs keeps the larger magnitude; min /
-// max skip a NaN operand), for f32 one.
-template <class T, bool ABS>
+// two lanes per instruction (max.xorsign.abs keeps the larger magnitude), for
+// f32 one. PROP = true propagates a NaN into the accumulator (to detect one);
+// PROP = false skips NaN operands (the range the formats define).
+template <class T, bool ABS, bool PROP>
 __device__ __forceinline__ void range_acc(const U4& r, uint32_t& ph, uint32_t& pl, float& hi,
                                           float& nlo) {
     if constexpr (sizeof(T) == 2) {
@@ -84,14 +85,22 @@ __device__ __forceinline__ void range_acc(const U4& r, uint32_t& ph, uint32_t& p
         for (int i = 0; i < 4; ++i) {
             if constexpr (std::is_same<T, __nv_bfloat16>::value) {
                 if (ABS) {
-                    asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(ph) : "r"(w[i]));
+                    if (PROP) asm("max.NaN.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(ph) : "r"(w[i]));
+                    else asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(ph) : "r"(w[i]));
+                } else if (PROP) {
+                    asm("max.NaN.bf16x2 %0, %0, %1;" : "+r"(ph) : "r"(w[i]));
+                    asm("min.NaN.bf16x2 %0, %0, %1;" : "+r"(pl) : "r"(w[i]));
                 } else {
                     asm("max.bf16x2 %0, %0, %1;" : "+r"(ph) : "r"(w[i]));
                     asm("min.bf16x2 %0, %0, %1;" : "+r"(pl) : "r"(w[i]));
                 }
             } else {
                 if (ABS) {
-                    asm("max.xorsign.abs.f16x2 %0, %0, %1;" : "+r"(ph) : "r"(w[i]));
+                    if (PROP) asm("max.NaN.xorsign.abs.f16x2 %0, %0, %1;" : "+r"(ph) : "r"(w[i]));
+                    else asm("max.xorsign.abs.f16x2 %0, %0, %1;" : "+r"(ph) : "r"(w[i]));
+                } else if (PROP) {
+                    asm("max.NaN.f16x2 %0, %0, %1;" : "+r"(ph) : "r"(w[i]));
+                    asm("min.NaN.f16x2 %0, %0, %1;" : "+r"(pl) : "r"(w[i]));
                 } else {
                     asm("max.f16x2 %0, %0, %1;" : "+r"(ph) : "r"(w[i]));
                     asm("min.f16x2 %0, %0, %1;" : "+r"(pl) : "r"(w[i]));
@@ -103,7 +112,14 @@ __device__ __forceinline__ void range_acc(const U4& r, uint32_t& ph, uint32_t& p
                             __uint_as_float(r.w)};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            if (ABS) {
+            if (PROP) {
+                if (ABS) {
+                    asm("max.NaN.f32 %0, %0, %1;" : "+f"(hi) : "f"(fabsf(v[i])));
+                } else {
+                    asm("max.NaN.f32 %0, %0, %1;" : "+f"(hi) : "f"(v[i]));
+                    asm("max.NaN.f32 %0, %0, %1;" : "+f"(nlo) : "f"(-v[i]));
+                }
+            } else if (ABS) {
                 hi = fmaxf(hi, fabsf(v[i]));
             } else {
                 hi = fmaxf(hi, v[i]);
@@ -131,6 +147,25 @@ __device__ __forceinline__ void range_finish(uint32_t ph, uint32_t pl, float& hi
             hi = fmaxf(fmaxf(h0, h1), 0.0f);
             nlo = fmaxf(fmaxf(-l0, -l1), 0.0f);
         }
+    }
+}
+// As range_finish after a NaN-propagating accumulation; true if a NaN was met
+// (then hi / nlo are not the range).
+template <class T, bool ABS>
+__device__ __forceinline__ bool range_finish_nan(uint32_t ph, uint32_t pl, float& hi, float& nlo) {
+    if constexpr (sizeof(T) == 2) {
+        // A 16-bit NaN: exponent all ones and a non-zero mantissa.
+        constexpr uint32_t EXP = std::is_same<T, __nv_bfloat16>::value ? 0x7F80u : 0x7C00u;
+        const uint32_t a0 = ph & 0x7FFFu, a1 = (ph >> 16) & 0x7FFFu;
+        bool nan = a0 > EXP || a1 > EXP;
+        if (!ABS) {
+            const uint32_t b0 = pl & 0x7FFFu, b1 = (pl >> 16) & 0x7FFFu;
+            nan = nan || b0 > EXP || b1 > EXP;
+        }
+        range_finish<T, ABS>(ph, pl, hi, nlo);
+        return nan;
+    } else {
+        return (hi != hi) || (nlo != nlo);
     }
 }
 
@@ -172,6 +207,12 @@ __global__ void __launch_bounds__(256) k_seg_pipe(PipeArgs a) {
     const size_t esz = sizeof(T);
     const int G = a.G;
     const bool full_groups = (G == SPAN);
+    // Teams narrower than 8 lanes read their vectors in an order rotated by
+    // team, so that the 8 lanes of one 128-byte shared-memory phase (several
+    // teams) land on distinct banks: vector j of a thread is vidx(j).
+    constexpr int ROT_DIV = (TEAM * NV >= 8) ? 1 : 8 / (TEAM * NV);
+    const int rot = (TEAM >= 8) ? 0 : team / ROT_DIV;
+    auto vidx = [&](int j) { return (TEAM >= 8 || NV == 1) ? j : ((j + rot) & (NV - 1)); };
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) mbar_init(smem_addr(&bars[s]), 1);
@@ -240,20 +281,32 @@ __global__ void __launch_bounds__(256) k_seg_pipe(PipeArgs a) {
         const bool seg_ok = seg < a.n_seg;
         const bool full = seg_ok && full_groups;
 
-        // This thread's vectors of its group, straight from shared memory.
+        // This thread's vectors of its group, straight from shared memory,
+        // in the team's rotated order (vidx).
         U4 raw[NV];
         const uint32_t gbase = smem_addr(slot_ptr + (size_t)team * G * esz) + (uint32_t)(lane * 16);
 #pragma unroll
         for (int j = 0; j < NV; ++j) {
-            const int e = (j * TEAM + lane) * VEC;
-            raw[j] = (full || (seg_ok && e < G)) ? ld_shared16(gbase + (uint32_t)(j * TEAM * 16))
+            const int e = (vidx(j) * TEAM + lane) * VEC;
+            raw[j] = (full || (seg_ok && e < G)) ? ld_shared16(gbase + (uint32_t)(vidx(j) * TEAM * 16))
                                                  : U4{0u, 0u, 0u, 0u};
         }
+        // Range with NaN propagation; a thread that met a NaN recomputes its
+        // part ignoring NaN (the range the formats define) and its warp takes
+        // the general encoders.
         uint32_t ph = 0u, pl = 0u;
         float hi = 0.0f, nlo = 0.0f;
 #pragma unroll
-        for (int j = 0; j < NV; ++j) range_acc<T, ABS>(raw[j], ph, pl, hi, nlo);
-        range_finish<T, ABS>(ph, pl, hi, nlo);
+        for (int j = 0; j < NV; ++j) range_acc<T, ABS, true>(raw[j], ph, pl, hi, nlo);
+        const bool saw_nan = range_finish_nan<T, ABS>(ph, pl, hi, nlo);
+        if (saw_nan) {
+            ph = pl = 0u;
+            hi = nlo = 0.0f;
+#pragma unroll
+            for (int j = 0; j < NV; ++j) range_acc<T, ABS, false>(raw[j], ph, pl, hi, nlo);
+            range_finish<T, ABS>(ph, pl, hi, nlo);
+        }
+        const bool warp_nan = __any_sync(0xffffffffu, saw_nan);
         if constexpr (TEAM > 1) {
 #pragma unroll
             for (int o = (TEAM < 32 ? TEAM : 32) / 2; o > 0; o >>= 1) {
@@ -274,21 +327,24 @@ __global__ void __launch_bounds__(256) k_seg_pipe(PipeArgs a) {
                 if (!ABS) nlo = fmaxf(nlo, red[NW + w0 + w]);
             }
         }
+        // Vector j of this thread: valid, and its offset in the group.
+        auto vok = [&](int j) { return full || (seg_ok && (vidx(j) * TEAM + lane) * VEC < G); };
+        auto voff = [&](int j) { return vidx(j) * TEAM * VEC; };
 
         if constexpr (PK == PK_INT_Q || PK == PK_INT_FAKE) {
             constexpr int OP = (PK == PK_INT_Q) ? OP_QUANT : OP_FAKE;
             // Scale and zero-point: fl(amax/qmax) or fl(fl(max'-min')/(qmax-qmin)),
             // each quotient by the launch's divisor reciprocal (exact for a
             // normal dividend; IEEE division below 2^-100).
-            float sc, zf = 0.0f;
+            float sc, zf = 0.0f, rz = 0.0f;
             {
                 const float num = SYM ? fmaxf(hi, nlo) : __fadd_rn(hi, nlo);
                 sc = (num >= 0x1p-100f && num <= 0x1p100f) ? div_chain(num, Rq) : div_slow(num, Rq.s);
                 if (sc == 0.0f) sc = 1.0f;
                 if (!SYM) {
                     const float m = __fdiv_rn(-nlo, sc);
-                    const float r = a.cfg.rhaz ? roundf(m) : rintf(m);
-                    zf = fminf(fmaxf(__fsub_rn(qlo, r), qlo), qhi);   // NaN -> qmin
+                    rz = a.cfg.rhaz ? roundf(m) : rintf(m);
+                    zf = fminf(fmaxf(__fsub_rn(qlo, rz), qlo), qhi);   // NaN -> qmin
                 }
             }
             const int zp = (int)zf;
@@ -303,84 +359,92 @@ __global__ void __launch_bounds__(256) k_seg_pipe(PipeArgs a) {
             const Recip R = make_recip(sc);
             uint8_t* qb = a.q + seg * G + lane * VEC;
             T* yb = (T*)a.y + seg * G + lane * VEC;
-            if (full) {
-                if (R.fast) {
+            // Fast path: no NaN in the warp's groups, a normal scale, and no
+            // clamp that can bind. Symmetric: |x/s| <= qmax (1 + 2^-23) rounds
+            // into [-qmax, qmax], inside [qmin, qmax] when qmin <= -qmax.
+            // Asymmetric: codes are monotone in x, the smallest is qmin when
+            // the zero-point is unclamped, the largest is round(fl(max'/s)) + zp.
+            bool noclamp;
+            if constexpr (SYM) {
+                noclamp = qlo <= -qhi;
+            } else {
+                const float kmax = R.fast ? __fsub_rn(__fadd_rn(div_chain(hi, R), kMagic), kMagic) : 0.0f;
+                noclamp = (zf == __fsub_rn(qlo, rz)) && (__fadd_rn(kmax, zf) <= qhi);
+            }
+            if (seg_ok && R.fast && noclamp && !warp_nan) {
+                const Recip2 R2 = make_recip2(R);
+                const F2 magic2 = f2_bcast(kMagic), zp2 = f2_bcast(zf), s2v = f2_bcast(sc);
 #pragma unroll
-                    for (int j = 0; j < NV; ++j) {
-                        float v[VEC];
-                        load_vec<T>(raw[j], v);
-                        emit_int<T, OP, true, SYM>(v, R, ip, qb + j * TEAM * VEC, yb + j * TEAM * VEC);
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < NV; ++j) {
-                        float v[VEC];
-                        load_vec<T>(raw[j], v);
-                        emit_int<T, OP, false, SYM>(v, R, ip, qb + j * TEAM * VEC, yb + j * TEAM * VEC);
-                    }
-                }
+                for (int j = 0; j < NV; ++j)
+                    if (vok(j)) emit_int_fast<T, OP, !SYM>(raw[j], R2, magic2, zp2, s2v, qb + voff(j), yb + voff(j));
             } else if (seg_ok) {
 #pragma unroll
                 for (int j = 0; j < NV; ++j) {
-                    if ((j * TEAM + lane) * VEC >= G) continue;
+                    if (!vok(j)) continue;
                     float v[VEC];
                     load_vec<T>(raw[j], v);
-                    if (R.fast) emit_int<T, OP, true, SYM>(v, R, ip, qb + j * TEAM * VEC, yb + j * TEAM * VEC);
-                    else emit_int<T, OP, false, SYM>(v, R, ip, qb + j * TEAM * VEC, yb + j * TEAM * VEC);
+                    if (R.fast) emit_int<T, OP, true, SYM>(v, R, ip, qb + voff(j), yb + voff(j));
+                    else emit_int<T, OP, false, SYM>(v, R, ip, qb + voff(j), yb + voff(j));
                 }
             }
         } else {
             constexpr int FMT = (PK == PK_FP8) ? MX_FP8_1x128 : (PK == PK_MX ? MX_MXFP8 : MX_NVFP4);
             constexpr int CB = (PK == PK_NV) ? VEC / 2 : VEC;     // code bytes per vector
             uint8_t* base = a.q + seg * (G / VEC) * CB + lane * CB;
+            auto coff = [&](int j) { return vidx(j) * TEAM * CB; };
             if constexpr (PK == PK_FP8) {
                 float s = (hi >= 0x1p-100f && hi <= 0x1p100f) ? div_chain(hi, Rq) : div_slow(hi, 448.0f);
                 if (s == 0.0f) s = 1.0f;
                 if (seg_ok && lane == 0) a.scale[seg] = s;
                 const Recip R = make_recip(s);
-                if (seg_ok) {
+                if (seg_ok && R.fast && !warp_nan) {
+                    const Recip2 R2 = make_recip2(R);
+#pragma unroll
+                    for (int j = 0; j < NV; ++j)
+                        if (vok(j)) emit_fp8_fast<T>(raw[j], R2, base + coff(j));
+                } else if (seg_ok) {
 #pragma unroll
                     for (int j = 0; j < NV; ++j) {
-                        if (!full && (j * TEAM + lane) * VEC >= G) continue;
+                        if (!vok(j)) continue;
                         float v[VEC];
                         load_vec<T>(raw[j], v);
-                        if (R.fast) mx_emit<T, FMT, true>(v, R, 0.f, false, base + j * TEAM * CB);
-                        else mx_emit<T, FMT, false>(v, R, 0.f, false, base + j * TEAM * CB);
+                        if (R.fast) mx_emit<T, FMT, true>(v, R, 0.f, false, base + coff(j));
+                        else mx_emit<T, FMT, false>(v, R, 0.f, false, base + coff(j));
                     }
                 }
             } else if constexpr (PK == PK_MX) {
                 const int E = mx_exponent(hi);
                 if (seg_ok && lane == 0) a.zp[seg] = (uint8_t)(E + 127);
-                const Recip R{};
-                const float mul = exp2i(-E);
+                const F2 mul2 = f2_bcast(exp2i(-E));
                 if (seg_ok) {
 #pragma unroll
-                    for (int j = 0; j < NV; ++j) {
-                        if (!full && (j * TEAM + lane) * VEC >= G) continue;
-                        float v[VEC];
-                        load_vec<T>(raw[j], v);
-                        mx_emit<T, FMT, true>(v, R, mul, false, base + j * TEAM * CB);
-                    }
+                    for (int j = 0; j < NV; ++j)
+                        if (vok(j)) emit_mx_fast<T>(raw[j], mul2, base + coff(j));
                 }
             } else {
                 const uint32_t sb = e4m3x2(div_any(hi, R6), 0.0f) & 0xFFu;
                 if (seg_ok && lane == 0) a.zp[seg] = (uint8_t)sb;
                 const float eff = __fmul_rn(e4m3_to_f32(sb), s2);
                 const Recip R = make_recip(eff);
-                const bool fast = R.fast && !a.static_global;
-                if (seg_ok) {
+                // Fast: positive normal divisor, no NaN, quotients far from
+                // overflow (|x| <= hi <= 2^64 eff).
+                const bool fast = R.fast && eff > 0.0f && hi <= __fmul_rn(0x1p64f, eff) && !warp_nan;
+                if (seg_ok && fast) {
+                    const Recip2 R2 = make_recip2(R);
+#pragma unroll
+                    for (int j = 0; j < NV; ++j)
+                        if (vok(j)) emit_nv_fast<T>(raw[j], R2, base + coff(j));
+                } else if (seg_ok) {
 #pragma unroll
                     for (int j = 0; j < NV; ++j) {
-                        if (!full && (j * TEAM + lane) * VEC >= G) continue;
+                        if (!vok(j)) continue;
                         float v[VEC];
                         load_vec<T>(raw[j], v);
-                        if (fast) mx_emit<T, FMT, true>(v, R, 0.f, eff == 0.0f, base + j * TEAM * CB);
-                        else mx_emit<T, FMT, false>(v, R, 0.f, eff == 0.0f, base + j * TEAM * CB);
+                        mx_emit<T, FMT, false>(v, R, 0.f, eff == 0.0f, base + coff(j));
                     }
                 }
             }
         }
-
         // Every thread is done with this slot: refill it with tile it + S.
         __syncthreads();
         if (tid == 0) {

@@ -127,6 +127,123 @@ __device__ __forceinline__ void mx_emit(const float* v, const Recip& R, float mu
 }
 
 
+// ------------------------------------------------------------ fast emitters
+// Per-vector encoders on f32 pairs (one .f32x2 instruction per two values).
+// The caller guarantees, for the whole group: a positive scale in the range
+// where the division chain is exact (Recip::fast), no NaN among the group's
+// values (hence none among the quotients: |x| <= the group's finite range),
+// and, for integer codes, that no clamp can bind. Under those conditions each
+// emitter writes the same bits as the general one.
+
+// Integer codes (QUANT: the low byte of magic + k + zp) or fake-quantized
+// values (FAKE: fl(k * s)), k = round-half-even(fl(x / s)).
+template <class T, int OP, bool ASYM>
+__device__ __forceinline__ void emit_int_fast(const U4& raw, const Recip2& R2, F2 magic2, F2 zp2,
+                                              F2 s2, uint8_t* q, T* y) {
+    constexpr int VEC = Traits<T>::VEC;
+    constexpr int NP = VEC / 2;
+    F2 x[NP];
+    widen_pairs<T>(raw, x);
+    if constexpr (OP == OP_QUANT) {
+        uint32_t c[VEC];
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+            F2 t = f2_add(div_chain2(x[p], R2), magic2);
+            if (ASYM) t = f2_add(t, zp2);            // exact: both integers in the unit-spaced range
+            f2_split_bits(t, c[2 * p], c[2 * p + 1]);
+        }
+        if constexpr (VEC == 8) {
+            st8(q, pack4_lowbytes(c[0], c[1], c[2], c[3]), pack4_lowbytes(c[4], c[5], c[6], c[7]));
+        } else {
+            st4(q, pack4_lowbytes(c[0], c[1], c[2], c[3]));
+        }
+    } else {
+        float o[VEC];
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+            const F2 t = f2_add(div_chain2(x[p], R2), magic2);
+            f2_split(f2_mul(f2_sub(t, magic2), s2), o[2 * p], o[2 * p + 1]);
+        }
+        st16(y, pack_vec<T>(o));
+    }
+}
+
+// Sign bits of a vector's values, one per byte (bit 7 of byte i = sign of
+// value i) for the first four values (HALF = 0) or the next four (HALF = 1).
+template <class T, int HALF>
+__device__ __forceinline__ uint32_t sign_bytes(const U4& raw) {
+    if constexpr (sizeof(T) == 2) {
+        return (HALF == 0 ? __byte_perm(raw.x, raw.y, 0x7531) : __byte_perm(raw.z, raw.w, 0x7531)) &
+               0x80808080u;
+    } else {
+        return __byte_perm(__byte_perm(raw.x, raw.y, 0x0073), __byte_perm(raw.z, raw.w, 0x0073), 0x5410) &
+               0x80808080u;
+    }
+}
+
+// E4M3 codes of fl(x / s). The chain gives +0 for a zero quotient of a
+// negative x; the sign bit of x, OR-ed into each byte afterwards, restores
+// -0 there and changes nothing else (non-zero codes already carry it, and no
+// value is NaN).
+template <class T>
+__device__ __forceinline__ void emit_fp8_fast(const U4& raw, const Recip2& R2, uint8_t* dst) {
+    constexpr int VEC = Traits<T>::VEC;
+    constexpr int NP = VEC / 2;
+    F2 x[NP];
+    widen_pairs<T>(raw, x);
+    float t[VEC];
+#pragma unroll
+    for (int p = 0; p < NP; ++p) f2_split(div_chain2(x[p], R2), t[2 * p], t[2 * p + 1]);
+    if constexpr (VEC == 8) {
+        st8(dst, e4m3x4(t[0], t[1], t[2], t[3]) | sign_bytes<T, 0>(raw),
+            e4m3x4(t[4], t[5], t[6], t[7]) | sign_bytes<T, 1>(raw));
+    } else {
+        st4(dst, e4m3x4(t[0], t[1], t[2], t[3]) | sign_bytes<T, 0>(raw));
+    }
+}
+
+// E2M1 codes of fl(x / s), the sign of each quotient taken from x.
+template <class T>
+__device__ __forceinline__ void emit_nv_fast(const U4& raw, const Recip2& R2, uint8_t* dst) {
+    constexpr int VEC = Traits<T>::VEC;
+    constexpr int NP = VEC / 2;
+    F2 x[NP];
+    widen_pairs<T>(raw, x);
+    float t[8];
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+        uint32_t q0, q1, x0, x1;
+        f2_split_bits(div_chain2(x[p], R2), q0, q1);
+        f2_split_bits(x[p], x0, x1);
+        t[2 * p] = __uint_as_float((q0 & 0x7FFFFFFFu) | (x0 & 0x80000000u));
+        t[2 * p + 1] = __uint_as_float((q1 & 0x7FFFFFFFu) | (x1 & 0x80000000u));
+    }
+    if constexpr (VEC == 8) {
+        st4(dst, e2m1x8(t));
+    } else {
+        t[4] = t[5] = t[6] = t[7] = 0.0f;
+        st2(dst, e2m1x8(t) & 0xFFFFu);
+    }
+}
+
+// MXFP8 codes E4M3(fl(x * 2^-E)): a product, exact for every input (NaN and
+// infinities included), so it needs no guard.
+template <class T>
+__device__ __forceinline__ void emit_mx_fast(const U4& raw, F2 mul2, uint8_t* dst) {
+    constexpr int VEC = Traits<T>::VEC;
+    constexpr int NP = VEC / 2;
+    F2 x[NP];
+    widen_pairs<T>(raw, x);
+    float t[VEC];
+#pragma unroll
+    for (int p = 0; p < NP; ++p) f2_split(f2_mul(x[p], mul2), t[2 * p], t[2 * p + 1]);
+    if constexpr (VEC == 8) {
+        st8(dst, e4m3x4(t[0], t[1], t[2], t[3]), e4m3x4(t[4], t[5], t[6], t[7]));
+    } else {
+        st4(dst, e4m3x4(t[0], t[1], t[2], t[3]));
+    }
+}
+
 // Integer codes (QUANT) or fake-quantized values (FAKE) of one vector of
 // VEC values. SYM_DYN: symmetric scale derived from this group's own range.
 // When that scale is also a normal number (FAST: 2^-64 <= s <= 2^64) it is
