@@ -46,9 +46,9 @@ FLUSH_BYTES = 256 << 20
 # the workload above, with the sha256 of the kernel sources it was taken on;
 # reported as null once the sources change.
 NCU_TRAFFIC = {
-    "quantize_per_token": {"src_sha256": "bff0c6d10b9ef3c22e563d8731cc33a0624a5af4f29b9e782a27546915b7c317", "bytes_per_launch": 71037952},
-    "dequantize_per_token": {"src_sha256": "bff0c6d10b9ef3c22e563d8731cc33a0624a5af4f29b9e782a27546915b7c317", "bytes_per_launch": 38957568},
-    "quantize_per_token_backward": {"src_sha256": "bff0c6d10b9ef3c22e563d8731cc33a0624a5af4f29b9e782a27546915b7c317", "bytes_per_launch": 161623808},
+    "quantize_per_token": {"src_sha256": "78153fee8008be0045a136d071c579da257e0ee37770ac21ade35987138b743b", "bytes_per_launch": 70508800},
+    "dequantize_per_token": {"src_sha256": "78153fee8008be0045a136d071c579da257e0ee37770ac21ade35987138b743b", "bytes_per_launch": 38081024},
+    "quantize_per_token_backward": {"src_sha256": "78153fee8008be0045a136d071c579da257e0ee37770ac21ade35987138b743b", "bytes_per_launch": 161464320},
 }
 
 
