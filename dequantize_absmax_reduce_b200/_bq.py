@@ -100,6 +100,8 @@ lib.bq_quantize_workspace_size.argtypes = [_DESC, C.c_int, _I32, _I64, C.c_int]
 lib.bq_quantize_workspace_size.restype = _SZ
 lib.bq_packed_transpose_stride.argtypes = [_I64, _I64]
 lib.bq_packed_transpose_stride.restype = _I64
+lib.bq_check_device_error.argtypes = []
+lib.bq_check_device_error.restype = C.c_int
 
 
 # ---------------------------------------------------------------- marshalling
@@ -162,6 +164,12 @@ def _g(gran) -> int:
 # ---------------------------------------------------------------- misc
 def bq_status_string(status: int) -> str:
     return lib.bq_status_string(status).decode()
+
+
+def bq_check_device_error() -> int:
+    """Synchronises the device; BQ_ERR_TIMEOUT if a kernel gave up a bounded
+    wait since the last check (the flag is cleared), else BQ_OK / BQ_ERR_CUDA."""
+    return lib.bq_check_device_error()
 
 
 def bq_granularity_name(gran) -> str | None:
@@ -311,7 +319,7 @@ def bq_dequantize_per_group_backward(dy, scale, d, axis, group_size, dq, stream=
 def bq_nvfp4_quantize(x, packed, scale_e4m3, global_scale, static_global=False, ws=None, stream=None):
     n, k = x.shape
     _check(lib.bq_nvfp4_quantize(_ptr(x), DTYPE[x.dtype], n, k, _ptr(packed), _ptr(scale_e4m3),
-                                 _ptr(global_scale), int(bool(static_global)), _ptr(ws), _nbytes(ws),
+                                 _ptr(global_scale), int(static_global), _ptr(ws), _nbytes(ws),
                                  _stream(stream)), "bq_nvfp4_quantize")
 
 

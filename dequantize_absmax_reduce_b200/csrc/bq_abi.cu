@@ -165,7 +165,7 @@ bq_status quant_impl(int op, const void* x, const bq_qdesc* d, int gr, int32_t a
     }
     if (!aligned(ws, 8)) return BQ_ERR_MISALIGNED;
     unsigned long long* ranges = (unsigned long long*)ws;
-    if (cudaMemsetAsync(ranges, 0, need_ranges, s) != cudaSuccess) return BQ_ERR_CUDA;
+    if (bq::clear_records(ranges, 2 * sv.n_seg, s) != cudaSuccess) return BQ_ERR_CUDA;
     e = (sv.n_seg == 1) ? bq::tensor_range(dt, x, sv.numel, cfg.symmetric, ranges, s)
                         : bq::seg_range(dt, x, sv, cfg.symmetric, ranges, s);
     if (e != cudaSuccess) return BQ_ERR_CUDA;
@@ -302,7 +302,7 @@ bq_status bq_group_range(const void* x, const bq_qdesc* d, bq_gran gran, int32_t
     if (!ranges || (sv.numel > 0 && !x)) return BQ_ERR_INVALID_ARG;
     if (!aligned(ranges, 8) || !aligned(x, esize(d->x_dtype))) return BQ_ERR_MISALIGNED;
     cudaStream_t s = S(stream);
-    if (cudaMemsetAsync(ranges, 0, (size_t)sv.n_seg * 16, s) != cudaSuccess) return BQ_ERR_CUDA;
+    if (bq::clear_records((unsigned long long*)ranges, 2 * sv.n_seg, s) != cudaSuccess) return BQ_ERR_CUDA;
     // Both slots are always filled, so the records serve either scaling.
     cudaError_t e = (sv.n_seg == 1)
         ? bq::tensor_range(to_dt(d->x_dtype), x, sv.numel, false, (unsigned long long*)ranges, s)
@@ -316,7 +316,7 @@ bq_status bq_tensor_amax(const void* x, bq_dtype dtype, int64_t n, float* amax, 
     if (n < 0 || !amax || !ws || (n > 0 && !x)) return BQ_ERR_INVALID_ARG;
     if (!aligned(ws, 8) || !aligned(amax, 4) || !aligned(x, esize(dtype))) return BQ_ERR_MISALIGNED;
     cudaStream_t s = S(stream);
-    if (cudaMemsetAsync(ws, 0, 16, s) != cudaSuccess) return BQ_ERR_CUDA;
+    if (bq::clear_records((unsigned long long*)ws, 2, s) != cudaSuccess) return BQ_ERR_CUDA;
     cudaError_t e = bq::tensor_range(to_dt(dtype), x, n, true, (unsigned long long*)ws, s);
     if (e != cudaSuccess) return BQ_ERR_CUDA;
     return from_cuda(bq::range_to_amax((const unsigned long long*)ws, amax, s));
@@ -450,13 +450,13 @@ bq_status bq_nvfp4_quantize(const void* x, bq_dtype x_dtype, int64_t n, int64_t 
     const DT dt = to_dt(x_dtype);
     unsigned long long* rec = (unsigned long long*)ws;
     if (static_global == 0) {
-        if (cudaMemsetAsync(rec, 0, 16, s) != cudaSuccess) return BQ_ERR_CUDA;
+        if (bq::clear_records(rec, 2, s) != cudaSuccess) return BQ_ERR_CUDA;
         if (n * k == 0) return from_cuda(bq::set_f32(global_scale, 1.0f, s));   // zero range
         if (bq::tensor_range(dt, x, n * k, true, rec, s) != cudaSuccess) return BQ_ERR_CUDA;
     }
     if (n * k == 0) return BQ_OK;
     return from_cuda(bq::mx_quant(dt, bq::MX_NVFP4, x, n, k, packed, scale_e4m3, rec, global_scale,
-                                  static_global == 1 ? 1 : 0, s));
+                                  static_global, s));
 }
 
 bq_status bq_nvfp4_dequantize(const uint8_t* packed, const uint8_t* scale_e4m3,

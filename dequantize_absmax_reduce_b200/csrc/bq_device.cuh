@@ -12,6 +12,37 @@
 
 namespace bq {
 
+// ---------------------------------------------------------------- launch order
+// Programmatic dependent launch (sm_90 and later). A kernel launched with the
+// programmatic-serialization attribute (launch_pdl) may start while the
+// kernel before it on the stream is still running: pdl_wait() blocks until
+// that kernel has completed and its writes are visible (it returns at once in
+// a kernel launched the ordinary way), and pdl_trigger() lets the next such
+// kernel start once every block of this grid has called it or exited. The
+// first kernel of every library call is launched the ordinary way, so a call
+// never overlaps the caller's earlier work; a kernel launched with the
+// attribute touches nothing an earlier kernel of the same call writes before
+// its pdl_wait().
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+template <class... KArgs, class... Args>
+static cudaError_t launch_pdl(void (*k)(KArgs...), unsigned grid, unsigned block, size_t smem,
+                              cudaStream_t st, Args... args) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, args...);
+}
+
 // ---------------------------------------------------------------- elements
 // Acc is the arithmetic type: f32 for f32/f16/bf16 storage, f64 for f64.
 template <class T> struct Traits;

@@ -471,6 +471,7 @@ __global__ void k_empty_groups(int64_t n_seg, IntCfg cfg, float* scale, uint8_t*
 }
 
 __global__ void k_range_to_amax(const unsigned long long* rec, float* amax) {
+    pdl_wait();
     float h, n;
     range_from_bits(rec[0], h);
     range_from_bits(rec[1], n);
@@ -707,6 +708,8 @@ static cudaError_t launch_tensor_range_t(const void* x, int64_t n, bool sym,
 cudaError_t tensor_range(DT dt, const void* x, int64_t n, bool sym, unsigned long long* rec,
                          cudaStream_t st) {
     if (n == 0) return cudaSuccess;
+    const cudaError_t pe = tensor_range_pipe(dt, x, n, sym, rec, st);
+    if (pe != cudaErrorNotSupported) return pe;
     switch (dt) {
         case DT::F32: return launch_tensor_range_t<float>(x, n, sym, rec, st);
         case DT::F64: return launch_tensor_range_t<double>(x, n, sym, rec, st);
@@ -730,7 +733,21 @@ cudaError_t set_f32(float* p, float v, cudaStream_t st) {
 }
 
 cudaError_t range_to_amax(const unsigned long long* rec, float* amax, cudaStream_t st) {
-    k_range_to_amax<<<1, 1, 0, st>>>(rec, amax);
+    return launch_pdl(k_range_to_amax, 1u, 1u, 0, st, rec, amax);
+}
+
+// Lets the range kernel after it start at once (it waits for this one before
+// its atomics).
+__global__ void k_clear_records(unsigned long long* rec, int64_t n) {
+    pdl_trigger();
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x)
+        rec[i] = 0ull;
+}
+
+cudaError_t clear_records(unsigned long long* rec, int64_t n, cudaStream_t st) {
+    if (n == 0) return cudaSuccess;
+    k_clear_records<<<grid_for(n, 256, 4), 256, 0, st>>>(rec, n);
     return cudaGetLastError();
 }
 

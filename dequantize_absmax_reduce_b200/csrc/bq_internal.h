@@ -57,17 +57,27 @@ cudaError_t int_map(DT dt, int op, int psrc, const void* a, const void* b, SegVi
 cudaError_t seg_range(DT dt, const void* x, SegView sv, bool sym, unsigned long long* ranges,
                       cudaStream_t st);
 
-// Range record of the whole tensor (rec cleared by the caller).
+// Range record of the whole tensor. rec must be cleared by the kernel just
+// before this one on the stream (clear_records): the range kernel is launched
+// to overlap it and waits for it only before its atomics.
 cudaError_t tensor_range(DT dt, const void* x, int64_t n, bool sym, unsigned long long* rec,
                          cudaStream_t st);
+// The bulk-copy pipelined range kernel behind tensor_range (f32 / f16 / bf16).
+cudaError_t tensor_range_pipe(DT dt, const void* x, int64_t n, bool sym, unsigned long long* rec,
+                              cudaStream_t st);
+// Clears n 64-bit range records; the first kernel of a two-pass call.
+cudaError_t clear_records(unsigned long long* rec, int64_t n, cudaStream_t st);
 // Parameters of groups with no elements (scale 1, zero-point of a zero range).
 cudaError_t empty_groups(int64_t n_seg, IntCfg cfg, float* scale, void* zp, cudaStream_t st);
 // *p = v.
 cudaError_t set_f32(float* p, float v, cudaStream_t st);
-// amax = max(rec[0], rec[1]) as f32.
+// amax = max(rec[0], rec[1]) as f32; launched to overlap the range kernel.
 cudaError_t range_to_amax(const unsigned long long* rec, float* amax, cudaStream_t st);
 
-// Microscaled formats.
+// Microscaled formats. NVFP4 per-tensor scale (static_global): 0 = from the
+// range record that the range kernel just before on the stream writes (the
+// quantizer is launched to overlap it); 1 = *global_scale as given; 2 = from
+// a range record the caller supplies (ordinary launch).
 enum MxFmt { MX_FP8_1x128 = 0, MX_MXFP8 = 1, MX_NVFP4 = 2 };
 cudaError_t mx_quant(DT dt, int fmt, const void* x, int64_t rows, int64_t k, uint8_t* codes,
                      void* scales, const unsigned long long* amax_rec, float* global_scale,
@@ -77,6 +87,10 @@ cudaError_t mx_dequant(DT ydt, int fmt, const uint8_t* codes, const void* scales
                        cudaStream_t st);
 cudaError_t fp8_tile_quant(DT dt, const void* x, int64_t rows, int64_t cols, int br, int bc,
                            uint8_t* e4m3, float* scale, cudaStream_t st);
+// Bulk-copy pipelined 128x128 tiles (16-bit inputs); cudaErrorNotSupported
+// when the shape or alignment does not fit.
+cudaError_t fp8_tile_pipe(DT dt, const void* x, int64_t rows, int64_t cols, uint8_t* e4m3,
+                          float* scale, cudaStream_t st);
 cudaError_t fp8_block_dequant(DT ydt, const uint8_t* e4m3, const float* scale, int64_t rows,
                               int64_t cols, int br, int bc, void* y, cudaStream_t st);
 

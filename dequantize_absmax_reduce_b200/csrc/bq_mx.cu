@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(256) k_mx_quant(MxArgs a) {
     float s2 = 1.0f;
     Recip R6;
     if constexpr (FMT == MX_NVFP4) {
-        if (a.static_global) {
+        if (a.static_global == 1) {
             s2 = *a.global_scale;
         } else {
             float h, n;
@@ -123,7 +123,7 @@ __global__ void __launch_bounds__(256) k_mx_quant(MxArgs a) {
                 if (ok && l == 0) ((uint8_t*)a.scales)[seg] = (uint8_t)sb;
                 const float eff = __fmul_rn(e4m3_to_f32(sb), s2);
                 const Recip R = make_recip(eff);
-                const bool fast = R.fast && !a.static_global;
+                const bool fast = R.fast && a.static_global != 1;
                 if (ok) {
 #pragma unroll
                     for (int j = 0; j < NV; ++j) {
@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(256) k_mx_quant_scalar(MxArgs a) {
     float s2 = 1.0f;
     Recip R6;
     if constexpr (FMT == MX_NVFP4) {
-        if (a.static_global) {
+        if (a.static_global == 1) {
             s2 = *a.global_scale;
         } else {
             float h, n;
@@ -358,6 +358,113 @@ __global__ void __launch_bounds__(256) k_mx_deq(DeqArgs a) {
     }
 }
 
+// ------------------------------------------------------------ dequantize, coalesced
+// Flat stream of items of 8 elements: 4 code bytes (NVFP4) or 8 (FP8), and
+// one 16-byte vector of 16-bit outputs, so that consecutive lanes write
+// consecutive 16 bytes and each warp store covers 512 contiguous bytes. Each
+// thread issues DQ_U item loads, with their scales, before it decodes any.
+// NVFP4 and MXFP8 scales are laid out like the elements ([rows, k/16],
+// [rows, k/32]): the scale of element e is scale[e / 16] or scale[e / 32].
+// FP8 block scales need the row and column of e.
+constexpr int DQ_U = 8;
+
+template <class T>
+__device__ __forceinline__ void st_vals8(T* y, const float (&o)[8]) {
+    if constexpr (sizeof(T) == 2) {
+        st16(y, pack_vec<T>(o));
+    } else {
+        st16(y, U4{__float_as_uint(o[0]), __float_as_uint(o[1]), __float_as_uint(o[2]), __float_as_uint(o[3])});
+        st16(y + 4, U4{__float_as_uint(o[4]), __float_as_uint(o[5]), __float_as_uint(o[6]), __float_as_uint(o[7])});
+    }
+}
+// Eight E2M1 codes (one word, low nibble first) times m, as f32 products.
+__device__ __forceinline__ void e2m1x8_mul(uint32_t w, F2 m2, float (&o)[8]) {
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        const float2 f = e2m1x2_to_f32((w >> (8 * b)) & 0xFFu);
+        f2_split(f2_mul(f2_pack(f.x, f.y), m2), o[2 * b], o[2 * b + 1]);
+    }
+}
+// Eight E4M3 codes (two words, low byte first) times m.
+__device__ __forceinline__ void e4m3x8_mul(uint32_t w0, uint32_t w1, F2 m2, float (&o)[8]) {
+    const uint32_t w[2] = {w0, w1};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const float2 a = e4m3x2_to_f32(w[h] & 0xFFFFu), b = e4m3x2_to_f32(w[h] >> 16);
+        f2_split(f2_mul(f2_pack(a.x, a.y), m2), o[4 * h], o[4 * h + 1]);
+        f2_split(f2_mul(f2_pack(b.x, b.y), m2), o[4 * h + 2], o[4 * h + 3]);
+    }
+}
+// Multiplier of an MXFP8 scale byte: 2^(b-127), NaN for 0xFF.
+__device__ __forceinline__ float e8m0_mul(uint32_t b) {
+    return (b == 0xFFu) ? __uint_as_float(0x7FC00000u) : exp2i((int)b - 127);
+}
+
+// FP8 block scale index of the item starting at element e0. BR: block rows
+// (1 or 128); BR = 0: 1x128 blocks on rows of whole blocks, where the index
+// is e0 / 128. FD: the element count is below 2^32 (32-bit row division).
+template <int BR, bool FD>
+__device__ __forceinline__ int64_t fp8_block_index(const DeqArgs& a, int64_t it) {
+    if constexpr (BR == 0) {
+        return it >> 4;
+    } else if constexpr (FD) {
+        const uint32_t e0 = (uint32_t)it * 8u;
+        const uint32_t r = fdiv(e0, a.fk);
+        const uint32_t c = e0 - r * (uint32_t)a.k;
+        const uint32_t rb = (BR == 1) ? r : (r >> 7);
+        return (int64_t)rb * a.nbc + (c >> 7);
+    } else {
+        const int64_t e0 = it * 8;
+        const int64_t r = e0 / a.k;
+        const int64_t c = e0 - r * a.k;
+        const int64_t rb = (BR == 1) ? r : (r >> 7);
+        return rb * a.nbc + (c >> 7);
+    }
+}
+
+// BR, FD: the FP8 block index variant (fp8_block_index); unused by NVFP4 / MXFP8.
+template <class T, int FMT, int BR, bool FD>
+__global__ void __launch_bounds__(256) k_mx_deq8(DeqArgs a) {
+    const float s2 = (FMT == MX_NVFP4) ? __ldg(a.global_scale) : 1.0f;
+    const int64_t n_items = a.numel / 8;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < n_items;
+         base += stride * DQ_U) {
+        uint2 w[DQ_U];
+        uint32_t sb[DQ_U];
+        float fs[DQ_U];
+#pragma unroll
+        for (int u = 0; u < DQ_U; ++u) {
+            const int64_t it = base + u * stride;
+            if (it < n_items) {
+                if constexpr (FMT == MX_NVFP4) {
+                    w[u].x = __ldg(reinterpret_cast<const uint32_t*>(a.codes) + it);
+                    sb[u] = __ldg((const uint8_t*)a.scales + (it >> 1));
+                } else {
+                    w[u] = __ldg(reinterpret_cast<const uint2*>(a.codes) + it);
+                    if constexpr (FMT == MX_MXFP8) {
+                        sb[u] = __ldg((const uint8_t*)a.scales + (it >> 2));
+                    } else {
+                        fs[u] = __ldg((const float*)a.scales + fp8_block_index<BR, FD>(a, it));
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < DQ_U; ++u) {
+            const int64_t it = base + u * stride;
+            if (it >= n_items) continue;
+            float o[8];
+            if constexpr (FMT == MX_NVFP4) {
+                e2m1x8_mul(w[u].x, f2_bcast(__fmul_rn(e4m3_to_f32(sb[u]), s2)), o);
+            } else {
+                e4m3x8_mul(w[u].x, w[u].y, f2_bcast(FMT == MX_MXFP8 ? e8m0_mul(sb[u]) : fs[u]), o);
+            }
+            st_vals8<T>((T*)a.y + it * 8, o);
+        }
+    }
+}
+
 // ------------------------------------------------------------ launchers
 static bool al(const void* p, int n) { return ((uintptr_t)p % (uintptr_t)n) == 0; }
 
@@ -367,17 +474,18 @@ static unsigned grid_cap(int64_t need_blocks, int per_sm) {
     return (unsigned)(need_blocks < cap ? need_blocks : cap);
 }
 
-template <class K>
-static unsigned grid_occ_mx(K kernel, int64_t need_blocks) {
-    static int bps = 0;
-    if (bps == 0) {
+// Grid of at most one wave of 256-thread blocks of kernel K; the occupancy
+// query runs once per kernel instantiation.
+template <auto K>
+static unsigned grid_occ_mx(int64_t need_blocks) {
+    static const int bps = [] {
         int n = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, 256, 0) != cudaSuccess || n < 1) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, K, 256, 0) != cudaSuccess || n < 1) {
             (void)cudaGetLastError();
             n = 1;
         }
-        bps = n;
-    }
+        return n;
+    }();
     return grid_cap(need_blocks, bps);
 }
 
@@ -388,7 +496,7 @@ static cudaError_t launch_mx_quant_t(const MxArgs& a, bool vec, cudaStream_t st)
         const int64_t per_warp = (int64_t)S::SEGS * (32 / S::TEAM);
         const int64_t warps = (a.n_seg + per_warp - 1) / per_warp;
         auto k = k_mx_quant<T, FMT>;
-        k<<<grid_occ_mx(k, (warps + 7) / 8), 256, 0, st>>>(a);
+        k<<<grid_occ_mx<k_mx_quant<T, FMT>>((warps + 7) / 8), 256, 0, st>>>(a);
     } else {
         k_mx_quant_scalar<T, FMT><<<grid_cap((a.n_seg + 255) / 256, 8), 256, 0, st>>>(a);
     }
@@ -449,6 +557,10 @@ static cudaError_t launch_tile_t(const void* x, int64_t rows, int64_t cols, int 
 cudaError_t fp8_tile_quant(DT dt, const void* x, int64_t rows, int64_t cols, int br, int bc,
                            uint8_t* e4m3, float* scale, cudaStream_t st) {
     if (bc != 128 || (br != 1 && br != 128)) return cudaErrorNotSupported;
+    if (br == 128) {
+        const cudaError_t pe = fp8_tile_pipe(dt, x, rows, cols, e4m3, scale, st);
+        if (pe != cudaErrorNotSupported) return pe;
+    }
     switch (dt) {
         case DT::F32: return launch_tile_t<float>(x, rows, cols, br, e4m3, scale, st);
         case DT::F16: return launch_tile_t<__half>(x, rows, cols, br, e4m3, scale, st);
@@ -459,15 +571,26 @@ cudaError_t fp8_tile_quant(DT dt, const void* x, int64_t rows, int64_t cols, int
 
 template <class T, int FMT>
 static cudaError_t launch_deq_t(const DeqArgs& a, cudaStream_t st) {
-    const int cin = (FMT == MX_NVFP4) ? 8 : 16;   // code bytes per 16 elements
-    const bool vec = (a.k % 16 == 0) && al(a.y, 16) && al(a.codes, cin);
-    const int64_t items = vec ? a.numel / 16 : a.numel;
+    const int cb = (FMT == MX_NVFP4) ? 4 : 8;      // code bytes per 8 elements
+    const bool vec = (a.k % 8 == 0) && al(a.y, 16) && al(a.codes, cb);
     if (vec) {
-        auto k = k_mx_deq<T, FMT, true>;
-        k<<<grid_occ_mx(k, (items + 255) / 256), 256, 0, st>>>(a);
+        const int64_t blocks = (a.numel / 8 + 256 * DQ_U - 1) / (256 * DQ_U);
+        if constexpr (FMT == MX_FP8_1x128) {
+            if (a.br == 1 && a.k % 128 == 0) {
+                k_mx_deq8<T, FMT, 0, true><<<grid_occ_mx<k_mx_deq8<T, FMT, 0, true>>(blocks), 256, 0, st>>>(a);
+            } else if (a.br == 1) {
+                if (a.use_fd) k_mx_deq8<T, FMT, 1, true><<<grid_occ_mx<k_mx_deq8<T, FMT, 1, true>>(blocks), 256, 0, st>>>(a);
+                else k_mx_deq8<T, FMT, 1, false><<<grid_occ_mx<k_mx_deq8<T, FMT, 1, false>>(blocks), 256, 0, st>>>(a);
+            } else {
+                if (a.use_fd) k_mx_deq8<T, FMT, 128, true><<<grid_occ_mx<k_mx_deq8<T, FMT, 128, true>>(blocks), 256, 0, st>>>(a);
+                else k_mx_deq8<T, FMT, 128, false><<<grid_occ_mx<k_mx_deq8<T, FMT, 128, false>>(blocks), 256, 0, st>>>(a);
+            }
+        } else {
+            k_mx_deq8<T, FMT, 0, true><<<grid_occ_mx<k_mx_deq8<T, FMT, 0, true>>(blocks), 256, 0, st>>>(a);
+        }
     } else {
         auto k = k_mx_deq<T, FMT, false>;
-        k<<<grid_occ_mx(k, (items + 255) / 256), 256, 0, st>>>(a);
+        k<<<grid_occ_mx<k_mx_deq<T, FMT, false>>((a.numel + 255) / 256), 256, 0, st>>>(a);
     }
     return cudaGetLastError();
 }

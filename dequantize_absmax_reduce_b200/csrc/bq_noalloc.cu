@@ -12,7 +12,7 @@
 // with cudaGetSymbolAddress, on the first call made with that device current.
 // Nothing here allocates: no cudaMalloc / cudaFree, no allocating library
 // routine. The records a call uses are cleared on its stream before the range
-// kernels accumulate into them (the workspace path's own cudaMemsetAsync).
+// kernels accumulate into them (the workspace path's own clearing kernel).
 #include <mutex>
 
 #include "bq.h"

@@ -16,6 +16,12 @@ cudaError_t pipe_map_bf16(int op, const MapArgs& m, cudaStream_t st);
 cudaError_t pipe_err_f32(unsigned int* flag);
 cudaError_t pipe_err_f16(unsigned int* flag);
 cudaError_t pipe_err_bf16(unsigned int* flag);
+cudaError_t pipe_range_f32(const void* x, int64_t n, bool sym, unsigned long long* rec, cudaStream_t st);
+cudaError_t pipe_range_f16(const void* x, int64_t n, bool sym, unsigned long long* rec, cudaStream_t st);
+cudaError_t pipe_range_bf16(const void* x, int64_t n, bool sym, unsigned long long* rec, cudaStream_t st);
+cudaError_t pipe_tile_f32(const void* x, int64_t rows, int64_t cols, uint8_t* e4m3, float* scale, cudaStream_t st);
+cudaError_t pipe_tile_f16(const void* x, int64_t rows, int64_t cols, uint8_t* e4m3, float* scale, cudaStream_t st);
+cudaError_t pipe_tile_bf16(const void* x, int64_t rows, int64_t cols, uint8_t* e4m3, float* scale, cudaStream_t st);
 
 static cudaError_t pipe_launch(DT dt, int pk, bool sym, const PipeArgs& a, cudaStream_t st) {
     switch (dt) {
@@ -74,6 +80,25 @@ cudaError_t mx_quant_pipe(DT dt, int fmt, const void* x, int64_t rows, int64_t k
     if (a.n_seg == 0) return cudaSuccess;
     const int pk = fmt == MX_FP8_1x128 ? PK_FP8 : (fmt == MX_MXFP8 ? PK_MX : PK_NV);
     return pipe_launch(dt, pk, true, a, st);
+}
+
+cudaError_t tensor_range_pipe(DT dt, const void* x, int64_t n, bool sym, unsigned long long* rec,
+                              cudaStream_t st) {
+    switch (dt) {
+        case DT::F32: return pipe_range_f32(x, n, sym, rec, st);
+        case DT::F16: return pipe_range_f16(x, n, sym, rec, st);
+        case DT::BF16: return pipe_range_bf16(x, n, sym, rec, st);
+        default: return cudaErrorNotSupported;
+    }
+}
+
+cudaError_t fp8_tile_pipe(DT dt, const void* x, int64_t rows, int64_t cols, uint8_t* e4m3, float* scale,
+                          cudaStream_t st) {
+    switch (dt) {
+        case DT::F16: return pipe_tile_f16(x, rows, cols, e4m3, scale, st);
+        case DT::BF16: return pipe_tile_bf16(x, rows, cols, e4m3, scale, st);
+        default: return cudaErrorNotSupported;
+    }
 }
 
 cudaError_t pipe_error_take(unsigned int* flag) {

@@ -25,7 +25,7 @@ struct PipeArgs {
     uint8_t* zp;        // int zero-points, or MXFP8 / NVFP4 scale bytes
     const unsigned long long* amax_rec;
     float* global_scale;
-    int static_global;
+    int static_global;  // 0: record from the range kernel before; 1: static; 2: caller's record
 };
 
 }  // namespace bq

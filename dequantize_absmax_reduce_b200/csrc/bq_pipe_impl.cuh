@@ -16,6 +16,9 @@
 // records the failure in g_pipe_error, waits (bounded again) for the copies
 // it has in flight, and returns.
 #pragma once
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <type_traits>
 
 #include "bq_device.cuh"
@@ -239,9 +242,11 @@ __global__ void __launch_bounds__(256) k_seg_pipe(PipeArgs a) {
     Recip R6, Rq;
     const float qlo = (float)a.cfg.qmin, qhi = (float)a.cfg.qmax;
     if constexpr (PK == PK_NV) {
-        if (a.static_global) {
+        if (a.static_global == 1) {
             s2 = *a.global_scale;
         } else {
+            // The range kernel before this one may still be running (launch_pdl).
+            pdl_wait();
             float h, n;
             range_from_bits(a.amax_rec[0], h);
             range_from_bits(a.amax_rec[1], n);
@@ -457,6 +462,455 @@ __global__ void __launch_bounds__(256) k_seg_pipe(PipeArgs a) {
             }
         }
         if (++slot == S) { slot = 0; parity ^= 1u; }
+    }
+}
+
+// ------------------------------------------------------------ NVFP4, 16-bit inputs
+// One thread per 16-element block (two 16-byte vectors), NV_BPT blocks per
+// thread per tile. A block's codes divide by eff = fl(dec(sb) * s2), where sb
+// is the block's E4M3 scale code: with only 256 codes, RN(1/eff) and the
+// fast-path limits are tabulated once per CTA (NvEntry) instead of being
+// derived once per block. Fast path (the same bits as the general encoder):
+// no NaN in the block, eff a positive normal number in the exact range of
+// the division chain, and |x| <= 2^64 eff (no quotient overflows).
+constexpr int NV_BPT = 2;
+#ifndef BQ_NV_STAGES
+#define BQ_NV_STAGES 3
+#endif
+struct NvEntry {
+    float y;      // RN(1 / eff)
+    float ns;     // -eff
+    float lim;    // 2^64 * eff
+    uint32_t ok;  // eff > 0 and in the exact range of the chain
+};
+
+// E2M1 codes of one vector, fast path: fl(x / eff) by the chain on pairs,
+// the sign of each quotient taken from x (restores -0 for x = -0).
+template <class T>
+__device__ __forceinline__ uint32_t nv_word_fast(const U4& raw, const Recip2& R2) {
+    F2 x[4];
+    widen_pairs<T>(raw, x);
+    float t[8];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        uint32_t q0, q1, x0, x1;
+        f2_split_bits(div_chain2(x[p], R2), q0, q1);
+        f2_split_bits(x[p], x0, x1);
+        t[2 * p] = __uint_as_float((q0 & 0x7FFFFFFFu) | (x0 & 0x80000000u));
+        t[2 * p + 1] = __uint_as_float((q1 & 0x7FFFFFFFu) | (x1 & 0x80000000u));
+    }
+    return e2m1x8(t);
+}
+// General path: IEEE division where the chain cannot be used; all-zero codes
+// when eff == 0.
+template <class T>
+__device__ __forceinline__ uint32_t nv_word_general(const U4& raw, const Recip& R, bool zero) {
+    float v[8];
+    load_vec<T>(raw, v);
+    float t[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) t[i] = with_quotient_sign(div_any(v[i], R), v[i], R.s);
+    return zero ? 0u : e2m1x8(t);
+}
+
+template <class T>
+__global__ void __launch_bounds__(256) k_nv_quant(PipeArgs a) {
+    static_assert(sizeof(T) == 2, "16-bit inputs");
+    constexpr int S = BQ_NV_STAGES;
+    constexpr int P = 256 * NV_BPT;                       // blocks per tile
+    constexpr uint32_t SLOT = P * 32;                     // bytes per tile
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 64);
+    NvEntry* table = reinterpret_cast<NvEntry*>(smem + 128);         // [256]
+    uint8_t* ring = smem + 128 + 256 * sizeof(NvEntry);            // [S][SLOT]
+    const int tid = threadIdx.x;
+    const int64_t grid = gridDim.x;
+    auto tile_bytes = [&](int64_t tile) -> uint32_t {
+        return (uint32_t)(min((int64_t)P, a.n_seg - tile * P) * 32);
+    };
+    if (tid == 0) {
+        for (int i = 0; i < S; ++i) mbar_init(smem_addr(&bars[i]), 1);
+        fence_mbar_init();
+        for (int i = 0; i < S; ++i) {
+            const int64_t tile = blockIdx.x + (int64_t)i * grid;
+            if (tile >= a.n_tiles) break;
+            bulk_load(smem_addr(ring + (size_t)i * SLOT), (const uint8_t*)a.x + (size_t)tile * SLOT,
+                      tile_bytes(tile), smem_addr(&bars[i]));
+        }
+    }
+    // Per-tensor scale: given, or from the range record (written by the range
+    // kernel that may still be running: launch_pdl).
+    float s2;
+    if (a.static_global == 1) {
+        s2 = *a.global_scale;
+    } else {
+        pdl_wait();
+        float h, n;
+        range_from_bits(a.amax_rec[0], h);
+        range_from_bits(a.amax_rec[1], n);
+        s2 = __fdiv_rn(fmaxf(h, n), 2688.0f);
+        if (s2 == 0.0f) s2 = 1.0f;
+        if (blockIdx.x == 0 && tid == 0) *a.global_scale = s2;
+    }
+    const Recip R6 = make_recip(__fmul_rn(6.0f, s2));
+    {
+        const float eff = __fmul_rn(e4m3_to_f32((uint32_t)tid), s2);
+        const Recip r = make_recip(eff);
+        NvEntry e;
+        e.y = r.y;
+        e.ns = -eff;
+        e.lim = __fmul_rn(0x1p64f, eff);
+        e.ok = (r.fast && eff > 0.0f) ? 1u : 0u;
+        table[tid] = e;
+    }
+    __syncthreads();
+
+    // Two 16-byte vectors per block, read in an order rotated every four
+    // lanes so that the eight lanes of one shared-memory phase hit distinct banks.
+    const int rot = (tid >> 2) & 1;
+    int slot = 0;
+    uint32_t parity = 0;
+    for (int64_t tile = blockIdx.x; tile < a.n_tiles; tile += grid) {
+        const bool okw = mbar_wait(smem_addr(&bars[slot]), parity);
+        if (__syncthreads_or(!okw)) {
+            if (tid == 0) {
+                atomicOr(&g_pipe_error, 1u);
+                int s3 = slot;
+                uint32_t p3 = parity;
+                for (int i = 0; i < S; ++i) {
+                    if (tile + (int64_t)i * grid >= a.n_tiles) break;
+                    mbar_wait(smem_addr(&bars[s3]), p3);
+                    if (++s3 == S) { s3 = 0; p3 ^= 1u; }
+                }
+            }
+            __syncthreads();
+            return;
+        }
+        const uint32_t sbase = smem_addr(ring + (size_t)slot * SLOT);
+        // The thread's NV_BPT blocks go through each step together, so that
+        // their serial per-block work (range, block scale, table) overlaps.
+        U4 r0[NV_BPT], r1[NV_BPT];
+        bool okb[NV_BPT], nan[NV_BPT];
+        float hi[NV_BPT];
+        uint32_t sb[NV_BPT];
+#pragma unroll
+        for (int g = 0; g < NV_BPT; ++g) {
+            const int lb = g * 256 + tid;                     // block in the tile
+            okb[g] = tile * P + lb < a.n_seg;
+            const uint32_t ba = sbase + (uint32_t)lb * 32u;
+            r0[g] = okb[g] ? ld_shared16(ba + (uint32_t)(rot * 16)) : U4{0u, 0u, 0u, 0u};
+            r1[g] = okb[g] ? ld_shared16(ba + (uint32_t)((rot ^ 1) * 16)) : U4{0u, 0u, 0u, 0u};
+        }
+#pragma unroll
+        for (int g = 0; g < NV_BPT; ++g) {
+            uint32_t ph = 0u, pl = 0u;
+            float h = 0.0f, nlo = 0.0f;
+            range_acc<T, true, true>(r0[g], ph, pl, h, nlo);
+            range_acc<T, true, true>(r1[g], ph, pl, h, nlo);
+            nan[g] = range_finish_nan<T, true>(ph, pl, h, nlo);
+            if (nan[g]) {
+                ph = 0u;
+                range_acc<T, true, false>(r0[g], ph, pl, h, nlo);
+                range_acc<T, true, false>(r1[g], ph, pl, h, nlo);
+                range_finish<T, true>(ph, pl, h, nlo);
+            }
+            hi[g] = h;
+        }
+#pragma unroll
+        for (int g = 0; g < NV_BPT; ++g) sb[g] = e4m3x2(div_any(hi[g], R6), 0.0f) & 0xFFu;
+#pragma unroll
+        for (int g = 0; g < NV_BPT; ++g) {
+            if (!okb[g]) continue;
+            const int64_t blk = tile * P + g * 256 + tid;
+            a.zp[blk] = (uint8_t)sb[g];
+            const NvEntry e = table[sb[g]];
+            uint32_t w0, w1;     // codes of vectors r0, r1
+            if (e.ok && hi[g] <= e.lim && !nan[g]) {
+                Recip2 R2;
+                R2.y = f2_bcast(e.y);
+                R2.ns = f2_bcast(e.ns);
+                w0 = nv_word_fast<T>(r0[g], R2);
+                w1 = nv_word_fast<T>(r1[g], R2);
+            } else {
+                const float eff = -e.ns;
+                const Recip R = make_recip(eff);
+                w0 = nv_word_general<T>(r0[g], R, eff == 0.0f);
+                w1 = nv_word_general<T>(r1[g], R, eff == 0.0f);
+            }
+            st8(a.q + blk * 8, rot ? w1 : w0, rot ? w0 : w1);
+        }
+        __syncthreads();
+        if (tid == 0) {
+            const int64_t next = tile + (int64_t)S * grid;
+            if (next < a.n_tiles) {
+                fence_proxy_async();
+                bulk_load(smem_addr(ring + (size_t)slot * SLOT), (const uint8_t*)a.x + (size_t)next * SLOT,
+                          tile_bytes(next), smem_addr(&bars[slot]));
+            }
+        }
+        if (++slot == S) { slot = 0; parity ^= 1u; }
+    }
+}
+
+// ------------------------------------------------------------ FP8 128x128 tiles, 16-bit inputs
+// One 128x128 tile per ring slot (32 KB), brought in by one 2D tensor copy
+// (TMA, no multicast): the copy engine fetches the 128 row segments itself
+// and fills the part of an edge tile outside the tensor with zeros, which
+// leaves the tile's amax unchanged. Two passes over the slot: the amax (then
+// one block reduction), then the codes; thread t owns the 16-byte vectors
+// v = t, t + 256, ... of the tile (row v / 16, column chunk v % 16), so the
+// shared loads are conflict-free and each row's codes leave as sixteen
+// consecutive 8-byte stores.
+#ifndef BQ_TILE_STAGES
+#define BQ_TILE_STAGES 2
+#endif
+
+struct TileArgs {
+    int64_t rows, cols, nbc, n_tiles;
+    uint8_t* e4m3;
+    float* scale;
+};
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm, int c0, int c1,
+                                            uint32_t bar) {
+    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                 " [%0], [%1, {%2, %3}], [%4];"
+                 :: "r"(dst), "l"((uint64_t)tm), "r"(c0), "r"(c1), "r"(bar) : "memory");
+}
+
+template <class T>
+__global__ void __launch_bounds__(256) k_fp8_tile_tma(const __grid_constant__ CUtensorMap tm,
+                                                      TileArgs a) {
+    static_assert(sizeof(T) == 2, "16-bit inputs");
+    constexpr int S = BQ_TILE_STAGES;
+    constexpr uint32_t SLOT = 128 * 256;
+    extern __shared__ __align__(128) uint8_t smem[];
+    float* red = reinterpret_cast<float*>(smem);                  // [8] warp maxima
+    uint32_t* rnan = reinterpret_cast<uint32_t*>(smem + 32);      // [8] warp saw a NaN
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 64);      // [S]
+    uint8_t* ring = smem + 128;
+    const int tid = threadIdx.x;
+    const int64_t grid = gridDim.x;
+    auto issue = [&](int64_t tile, int slot) {
+        const int64_t bi = tile / a.nbc, bj = tile - bi * a.nbc;
+        const uint32_t bar = smem_addr(&bars[slot]);
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(SLOT) : "memory");
+        tma_load_2d(smem_addr(ring + (size_t)slot * SLOT), &tm, (int)(bj * 128), (int)(bi * 128), bar);
+    };
+    if (tid == 0) {
+        for (int i = 0; i < S; ++i) mbar_init(smem_addr(&bars[i]), 1);
+        fence_mbar_init();
+        for (int i = 0; i < S; ++i) {
+            const int64_t tile = blockIdx.x + (int64_t)i * grid;
+            if (tile >= a.n_tiles) break;
+            issue(tile, i);
+        }
+    }
+    __syncthreads();
+    const Recip Rq = make_recip(448.0f);
+    int slot = 0;
+    uint32_t parity = 0;
+    for (int64_t tile = blockIdx.x; tile < a.n_tiles; tile += grid) {
+        const bool okw = mbar_wait(smem_addr(&bars[slot]), parity);
+        const uint32_t sbase = smem_addr(ring + (size_t)slot * SLOT);
+        // Pass 1: the tile's amax (NaN propagated to detect one, then ignored).
+        uint32_t ph = 0u, pl = 0u;
+        float hi = 0.0f, nlo = 0.0f;
+        bool nan = false;
+        if (okw) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                range_acc<T, true, true>(ld_shared16(sbase + (uint32_t)(i * 256 + tid) * 16u), ph, pl, hi, nlo);
+            nan = range_finish_nan<T, true>(ph, pl, hi, nlo);
+            if (nan) {
+                ph = 0u;
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    range_acc<T, true, false>(ld_shared16(sbase + (uint32_t)(i * 256 + tid) * 16u), ph, pl, hi, nlo);
+                range_finish<T, true>(ph, pl, hi, nlo);
+            }
+        }
+        hi = warp_max(hi);
+        const bool wnan = __any_sync(0xffffffffu, nan);
+        if ((tid & 31) == 0) {
+            red[tid >> 5] = hi;
+            rnan[tid >> 5] = wnan ? 1u : 0u;
+        }
+        if (__syncthreads_or(!okw)) {
+            if (tid == 0) {
+                atomicOr(&g_pipe_error, 1u);
+                int s3 = slot;
+                uint32_t p3 = parity;
+                for (int i = 0; i < S; ++i) {
+                    if (tile + (int64_t)i * grid >= a.n_tiles) break;
+                    mbar_wait(smem_addr(&bars[s3]), p3);
+                    if (++s3 == S) { s3 = 0; p3 ^= 1u; }
+                }
+            }
+            __syncthreads();
+            return;
+        }
+        float am = red[0];
+        uint32_t any_nan = rnan[0];
+#pragma unroll
+        for (int w = 1; w < 8; ++w) {
+            am = fmaxf(am, red[w]);
+            any_nan |= rnan[w];
+        }
+        float sc = (am >= 0x1p-100f && am <= 0x1p100f) ? div_chain(am, Rq) : div_slow(am, 448.0f);
+        if (sc == 0.0f) sc = 1.0f;
+        if (tid == 0) a.scale[tile] = sc;
+        const Recip R = make_recip(sc);
+        // Pass 2: codes of the valid part of the tile.
+        const int64_t bi = tile / a.nbc, bj = tile - bi * a.nbc;
+        const int nr = (int)min((int64_t)128, a.rows - bi * 128);
+        const int nch = (int)((min((int64_t)128, a.cols - bj * 128)) / 8);
+        const bool full = (nr == 128) && (nch == 16);
+        uint8_t* obase = a.e4m3 + bi * 128 * a.cols + bj * 128;
+        const bool fast = R.fast && !any_nan;
+        const Recip2 R2 = make_recip2(R);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int v = i * 256 + tid;
+            const int r = v >> 4, ch = v & 15;
+            if (!full && (r >= nr || ch >= nch)) continue;
+            const U4 raw = ld_shared16(sbase + (uint32_t)v * 16u);
+            uint8_t* dst = obase + (int64_t)r * a.cols + ch * 8;
+            if (fast) {
+                emit_fp8_fast<T>(raw, R2, dst);
+            } else {
+                float vals[8];
+                load_vec<T>(raw, vals);
+                if (R.fast) mx_emit<T, MX_FP8_1x128, true>(vals, R, 0.f, false, dst);
+                else mx_emit<T, MX_FP8_1x128, false>(vals, R, 0.f, false, dst);
+            }
+        }
+        __syncthreads();
+        if (tid == 0) {
+            const int64_t next = tile + (int64_t)S * grid;
+            if (next < a.n_tiles) {
+                fence_proxy_async();
+                issue(next, slot);
+            }
+        }
+        if (++slot == S) { slot = 0; parity ^= 1u; }
+    }
+}
+
+// ------------------------------------------------------------ tensor range
+// Range record of a whole tensor (per-tensor scaling, the NVFP4 per-tensor
+// scale). The 16-byte aligned body streams through a ring of RANGE_STAGES
+// bulk copies of RANGE_CHUNK bytes per CTA; each thread folds its vectors into
+// a packed running range (two 16-bit lanes per instruction). The few
+// elements before the first 16-byte boundary and after the last one go
+// through scalar loads in block 0. One atomicMax per CTA and record slot, made
+// after pdl_wait(): the kernel before this one on the stream clears the
+// record, and this kernel is launched to overlap it.
+constexpr int RANGE_CHUNK = 16384;
+constexpr int RANGE_STAGES = 4;
+
+struct RangeArgs {
+    const void* x;        // first element
+    int64_t head;         // elements before the 16-byte aligned body
+    int64_t body_bytes;   // multiple of 16
+    int64_t n;            // all elements
+    unsigned long long* rec;
+};
+
+template <class T, bool ABS>
+__global__ void __launch_bounds__(256) k_range_pipe(RangeArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    float* red = reinterpret_cast<float*>(smem);                  // [2][8]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 64);      // [RANGE_STAGES]
+    uint8_t* ring = smem + 128;                                   // [RANGE_STAGES][RANGE_CHUNK]
+    constexpr int S = RANGE_STAGES;
+    const int tid = threadIdx.x;
+    const int64_t grid = gridDim.x;
+    const T* x = (const T*)a.x;
+    const uint8_t* body = (const uint8_t*)(x + a.head);
+    const int64_t n_chunks = (a.body_bytes + RANGE_CHUNK - 1) / RANGE_CHUNK;
+    auto chunk_bytes = [&](int64_t c) -> uint32_t {
+        return (uint32_t)min((int64_t)RANGE_CHUNK, a.body_bytes - c * RANGE_CHUNK);
+    };
+    if (tid == 0) {
+        for (int i = 0; i < S; ++i) mbar_init(smem_addr(&bars[i]), 1);
+        fence_mbar_init();
+        for (int i = 0; i < S; ++i) {
+            const int64_t c = blockIdx.x + (int64_t)i * grid;
+            if (c >= n_chunks) break;
+            bulk_load(smem_addr(ring + (size_t)i * RANGE_CHUNK), body + c * RANGE_CHUNK,
+                      chunk_bytes(c), smem_addr(&bars[i]));
+        }
+    }
+    __syncthreads();
+    uint32_t ph = 0u, pl = 0u;
+    float hi = 0.0f, nlo = 0.0f;
+    int slot = 0;
+    uint32_t parity = 0;
+    for (int64_t c = blockIdx.x; c < n_chunks; c += grid) {
+        const bool ok = mbar_wait(smem_addr(&bars[slot]), parity);
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) {
+                atomicOr(&g_pipe_error, 1u);
+                int s2 = slot;
+                uint32_t p2 = parity;
+                for (int i = 0; i < S; ++i) {
+                    if (c + (int64_t)i * grid >= n_chunks) break;
+                    mbar_wait(smem_addr(&bars[s2]), p2);
+                    if (++s2 == S) { s2 = 0; p2 ^= 1u; }
+                }
+            }
+            __syncthreads();
+            return;
+        }
+        const uint32_t base = smem_addr(ring + (size_t)slot * RANGE_CHUNK);
+        const int nv = (int)(chunk_bytes(c) / 16);
+        if (nv == RANGE_CHUNK / 16) {
+#pragma unroll
+            for (int v = 0; v < RANGE_CHUNK / 16 / 256; ++v)
+                range_acc<T, ABS, false>(ld_shared16(base + (uint32_t)((v * 256 + tid) * 16)), ph, pl, hi, nlo);
+        } else {
+            for (int v = tid; v < nv; v += 256)
+                range_acc<T, ABS, false>(ld_shared16(base + (uint32_t)(v * 16)), ph, pl, hi, nlo);
+        }
+        __syncthreads();
+        if (tid == 0) {
+            const int64_t next = c + (int64_t)S * grid;
+            if (next < n_chunks) {
+                fence_proxy_async();
+                bulk_load(smem_addr(ring + (size_t)slot * RANGE_CHUNK), body + next * RANGE_CHUNK,
+                          chunk_bytes(next), smem_addr(&bars[slot]));
+            }
+        }
+        if (++slot == S) { slot = 0; parity ^= 1u; }
+    }
+    pdl_trigger();
+    range_finish<T, ABS>(ph, pl, hi, nlo);
+    // Unaligned head and tail: fewer than 16 bytes each.
+    if (blockIdx.x == 0) {
+        const int64_t tail0 = a.head + a.body_bytes / (int64_t)sizeof(T);
+        int64_t e = -1;
+        if (tid < a.head) e = tid;
+        else if (tid >= 16 && tid - 16 < a.n - tail0) e = tail0 + (tid - 16);
+        if (e >= 0) {
+            const float v = ld1<T>(x + e);
+            if (ABS) {
+                hi = fmaxf(hi, fabsf(v));
+            } else {
+                hi = fmaxf(hi, v);
+                nlo = fmaxf(nlo, -v);
+            }
+        }
+    }
+    hi = warp_max(hi);
+    if (!ABS) nlo = warp_max(nlo);
+    if ((tid & 31) == 0) { red[tid >> 5] = hi; red[8 + (tid >> 5)] = nlo; }
+    __syncthreads();
+    if (tid == 0) {
+        for (int w = 1; w < 8; ++w) { hi = fmaxf(hi, red[w]); nlo = fmaxf(nlo, red[8 + w]); }
+        pdl_wait();
+        atomicMax(a.rec, range_bits(hi));
+        if (!ABS) atomicMax(a.rec + 1, range_bits(nlo));
     }
 }
 
@@ -813,6 +1267,30 @@ static cudaError_t launch_pipe_t(PipeArgs a, cudaStream_t st) {
     if (bps < 1) return cudaErrorNotSupported;
     int64_t grid = (int64_t)sm_count() * bps;
     if (grid > a.n_tiles) grid = a.n_tiles;
+    // NVFP4 with a per-tensor scale from the range record: overlap the range
+    // kernel's tail (the kernel waits for it before reading the record).
+    if (PK == PK_NV && a.static_global == 0) return launch_pdl(k, (unsigned)grid, 256u, smem, st, a);
+    k<<<(unsigned)grid, 256, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+// NVFP4 of 16-bit inputs (k_nv_quant).
+template <class T>
+static cudaError_t launch_nv_t(PipeArgs a, cudaStream_t st) {
+    constexpr int P = 256 * NV_BPT;
+    constexpr int S = BQ_NV_STAGES;
+    a.P = P;
+    a.n_tiles = (a.n_seg + P - 1) / P;
+    const size_t smem = 128 + 256 * sizeof(NvEntry) + (size_t)S * P * 32;
+    auto k = k_nv_quant<T>;
+    static const cudaError_t attr = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (attr != cudaSuccess) return attr;
+    static unsigned long long occ[8];
+    const int bps = occupancy_for((const void*)k, smem, occ);
+    if (bps < 1) return cudaErrorNotSupported;
+    int64_t grid = (int64_t)sm_count() * bps;
+    if (grid > a.n_tiles) grid = a.n_tiles;
+    if (a.static_global == 0) return launch_pdl(k, (unsigned)grid, 256u, smem, st, a);
     k<<<(unsigned)grid, 256, smem, st>>>(a);
     return cudaGetLastError();
 }
@@ -846,7 +1324,11 @@ static cudaError_t pipe_dt(int pk, bool sym, const PipeArgs& a, cudaStream_t st)
         case PK_INT_FAKE: return sym ? launch_pipe_u<T, PK_INT_FAKE, true>(a, st) : launch_pipe_u<T, PK_INT_FAKE, false>(a, st);
         case PK_FP8: return launch_pipe_u<T, PK_FP8, true>(a, st);
         case PK_MX: return launch_pipe_u<T, PK_MX, true>(a, st);
-        case PK_NV: return launch_pipe_u<T, PK_NV, true>(a, st);
+        case PK_NV:
+            if constexpr (sizeof(T) == 2) {
+                if (((uintptr_t)a.q & 7u) == 0) return launch_nv_t<T>(a, st);
+            }
+            return launch_pipe_u<T, PK_NV, true>(a, st);
     }
     return cudaErrorInvalidValue;
 }
@@ -952,6 +1434,94 @@ static cudaError_t seg_map_dt(int op, const MapArgs& m, cudaStream_t st) {
     return cudaErrorNotSupported;
 }
 
+// Range of a whole tensor into rec (cleared by the kernel before this one on
+// the stream); launched to overlap that kernel (launch_pdl).
+template <class T>
+static cudaError_t range_entry(const void* x, int64_t n, bool sym, unsigned long long* rec,
+                               cudaStream_t st) {
+    RangeArgs a;
+    a.x = x;
+    a.n = n;
+    a.head = 0;
+    const uintptr_t p = (uintptr_t)x;
+    if (p % 16 != 0) a.head = min((int64_t)((16 - p % 16) / sizeof(T)), n);
+    a.body_bytes = (n - a.head) * (int64_t)sizeof(T) / 16 * 16;
+    a.rec = rec;
+    const int64_t n_chunks = (a.body_bytes + RANGE_CHUNK - 1) / RANGE_CHUNK;
+    const size_t smem = 128 + (size_t)RANGE_STAGES * RANGE_CHUNK;
+    auto k = sym ? k_range_pipe<T, true> : k_range_pipe<T, false>;
+    static const cudaError_t attr_s = cudaFuncSetAttribute(
+        k_range_pipe<T, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static const cudaError_t attr_a = cudaFuncSetAttribute(
+        k_range_pipe<T, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (attr_s != cudaSuccess) return attr_s;
+    if (attr_a != cudaSuccess) return attr_a;
+    static unsigned long long occ[8];
+    const int bps = occupancy_for((const void*)k_range_pipe<T, true>, smem, occ);
+    if (bps < 1) return cudaErrorNotSupported;
+    int64_t grid = (int64_t)sm_count() * bps;
+    if (grid > n_chunks) grid = n_chunks;
+    if (grid < 1) grid = 1;
+    return launch_pdl(k, (unsigned)grid, 256u, smem, st, a);
+}
+
+// Tensor map of a row-major [rows, cols] 16-bit tensor in 128x128 boxes, from
+// the driver's encoder (looked up once through the runtime).
+static cudaError_t encode_tile_map(CUtensorMap* tm, const void* x, int64_t rows, int64_t cols) {
+    static const PFN_cuTensorMapEncodeTiled_v12000 encode = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess) {
+            (void)cudaGetLastError();
+            p = nullptr;
+        }
+        return (PFN_cuTensorMapEncodeTiled_v12000)p;
+    }();
+    if (!encode) return cudaErrorNotSupported;
+    const cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t gstride[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {128, 128};
+    const cuuint32_t estride[2] = {1, 1};
+    const CUresult r = encode(tm, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(x), gdim, gstride,
+                              box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorNotSupported;
+}
+
+// FP8 128x128 tiles of 16-bit inputs (k_fp8_tile_tma). Needs cols % 8 == 0
+// (16-byte row stride), x 16-byte and e4m3 8-byte aligned, and dimensions
+// the tensor map can describe.
+template <class T>
+static cudaError_t tile_entry(const void* x, int64_t rows, int64_t cols, uint8_t* e4m3,
+                              float* scale, cudaStream_t st) {
+    if constexpr (sizeof(T) != 2) {
+        return cudaErrorNotSupported;
+    } else {
+        if (cols % 8 != 0 || ((uintptr_t)x & 15u) || ((uintptr_t)e4m3 & 7u)) return cudaErrorNotSupported;
+        if (rows <= 0 || cols <= 0 || rows > 0x7FFFFF80ll || cols > 0x7FFFFF80ll) return cudaErrorNotSupported;
+        TileArgs a;
+        a.rows = rows; a.cols = cols;
+        a.nbc = (cols + 127) / 128;
+        a.n_tiles = ((rows + 127) / 128) * a.nbc;
+        a.e4m3 = e4m3; a.scale = scale;
+        CUtensorMap tm;
+        const cudaError_t me = encode_tile_map(&tm, x, rows, cols);
+        if (me != cudaSuccess) return me;
+        const size_t smem = 128 + (size_t)BQ_TILE_STAGES * 128 * 256;
+        auto k = k_fp8_tile_tma<T>;
+        static const cudaError_t attr = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (attr != cudaSuccess) return attr;
+        static unsigned long long occ[8];
+        const int bps = occupancy_for((const void*)k, smem, occ);
+        if (bps < 1) return cudaErrorNotSupported;
+        int64_t grid = (int64_t)sm_count() * bps;
+        if (grid > a.n_tiles) grid = a.n_tiles;
+        k<<<(unsigned)grid, 256, smem, st>>>(tm, a);
+        return cudaGetLastError();
+    }
+}
+
 // Entry points of one dtype's translation unit.
 template <class T>
 cudaError_t pipe_dyn_entry(int pk, bool sym, const PipeArgs& a, cudaStream_t st) {
@@ -985,6 +1555,14 @@ cudaError_t pipe_error_entry(unsigned int* flag) {
     cudaError_t pipe_map_##NAME(int op, const MapArgs& m, cudaStream_t st) {            \
         return pipe_map_entry<T>(op, m, st);                                             \
     }                                                                                    \
-    cudaError_t pipe_err_##NAME(unsigned int* flag) { return pipe_error_entry<T>(flag); }
+    cudaError_t pipe_err_##NAME(unsigned int* flag) { return pipe_error_entry<T>(flag); }       \
+    cudaError_t pipe_range_##NAME(const void* x, int64_t n, bool sym, unsigned long long* rec,   \
+                                  cudaStream_t st) {                                              \
+        return range_entry<T>(x, n, sym, rec, st);                                               \
+    }                                                                                            \
+    cudaError_t pipe_tile_##NAME(const void* x, int64_t rows, int64_t cols, uint8_t* e4m3,       \
+                                 float* scale, cudaStream_t st) {                                 \
+        return tile_entry<T>(x, rows, cols, e4m3, scale, st);                                    \
+    }
 
 }  // namespace bq

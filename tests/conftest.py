@@ -18,3 +18,15 @@ def orc():
     import oracle
     oracle.lib()
     return oracle
+
+
+@pytest.fixture(autouse=True)
+def _no_abandoned_waits(request):
+    """After every GPU test: no kernel took its bounded-wait exit (which
+    returns without finishing its work)."""
+    yield
+    if request.node.get_closest_marker("gpu") is None:
+        return
+    import dequantize_absmax_reduce_b200 as m
+    st = m._bq.bq_check_device_error()
+    assert st == m._bq.BQ_OK, f"device error flag after the test: {m._bq.bq_status_string(st)}"

@@ -43,6 +43,81 @@ def test_nvfp4_parity(bq, orc, dtype, shape):
         assert_bitwise(sc, rsc, f"static scales {s2v}")
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_nvfp4_all_16bit_patterns(bq, orc, dtype):
+    # Every bit pattern (NaN, infinities, subnormals, -0) in blocks of 16,
+    # with the dynamic scale (infinite: every block takes the general path),
+    # with the finite values only, and with static scales that send blocks
+    # through the fast and the general encoder.
+    x = synthetic.bits_tensor(dtype).reshape(512, 128)
+    finite = torch.where(torch.isfinite(x.float()), x, torch.zeros_like(x))
+    for t in (x, finite):
+        packed, sc, s2 = bq.nvfp4_quantize(t.cuda())
+        rp, rsc, rs2 = orc.nvfp4_quantize(t)
+        assert cpu(s2).item() == rs2
+        assert_bitwise(packed, rp, f"{dtype} packed")
+        assert_bitwise(sc, rsc, f"{dtype} scales")
+        for s2v in (1.0, 2.0 ** -20, 1e-30, 0.0, 3e38):
+            packed, sc, _ = bq.nvfp4_quantize(t.cuda(), s2=s2v)
+            rp, rsc, _ = orc.nvfp4_quantize(t, s2=float(np.float32(s2v)))
+            assert_bitwise(packed, rp, f"{dtype} static packed {s2v}")
+            assert_bitwise(sc, rsc, f"{dtype} static scales {s2v}")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_fp8_tiles_all_16bit_patterns(bq, orc, dtype):
+    x = synthetic.bits_tensor(dtype).reshape(512, 128)
+    finite = torch.where(torch.isfinite(x.float()), x, torch.zeros_like(x))
+    for t in (x, finite, finite[:, :64].contiguous()):
+        for br in (1, 128):
+            e, s = bq.fp8_block_quantize(t.cuda(), br)
+            re, rs = orc.fp8_block_quantize(t, br, 128)
+            assert_bitwise(s, rs, f"{dtype} scale {br}")
+            assert_bitwise(e, re, f"{dtype} e4m3 {br}")
+
+
+def test_nvfp4_from_caller_range_record(bq, orc):
+    # static_global == 2: the per-tensor scale from a range record the caller
+    # made (here by bq_group_range; across shards, after an all-reduce MAX).
+    import dequantize_absmax_reduce_b200 as m
+    x = synthetic.Stream(17).tensor((48, 1024), "bf16", outlier_p=0.01, outlier_factor=50)
+    xg = x.cuda()
+    rp, rsc, rs2 = orc.nvfp4_quantize(x)
+    r = bq.group_range(xg, "tensor")
+    packed = torch.empty((48, 512), dtype=torch.uint8, device="cuda")
+    sc = torch.empty((48, 64), dtype=torch.uint8, device="cuda")
+    s2 = torch.full((1,), -1.0, dtype=torch.float32, device="cuda")
+    m._bq.bq_nvfp4_quantize(xg, packed, sc, s2, 2, r)
+    assert cpu(s2).item() == rs2
+    assert_bitwise(packed, rp, "packed from record")
+    assert_bitwise(sc, rsc, "scales from record")
+    # the sharded helper on one process (no process group: the all-reduce is skipped)
+    from dequantize_absmax_reduce_b200 import shard
+    packed, sc, s2 = shard.nvfp4_quantize_sharded(xg)
+    assert cpu(s2).item() == rs2
+    assert_bitwise(packed, rp, "sharded packed")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16", "f32"])
+def test_tensor_amax_offsets_and_sizes(bq, orc, dtype):
+    # The range kernel streams the 16-byte aligned body and reads the unaligned
+    # head and tail one element at a time: every offset within 16 bytes, sizes
+    # below, at and above one chunk.
+    base = synthetic.Stream(18).tensor((200000,), dtype, outlier_p=0.001, outlier_factor=40)
+    base[123] = float("nan")
+    gb = base.cuda()
+    for n in (1, 7, 8, 9, 8191, 8192 + 5, 65536 * 2 + 3, 199000):
+        for off in range(0, 16 // base.element_size() + 1):
+            if off + n > base.numel():
+                continue
+            a = bq.tensor_amax(gb[off:off + n])
+            ra = orc.tensor_amax(base[off:off + n].contiguous())
+            assert cpu(a).item() == float(np.float32(ra)), (n, off)
+    inf = base.clone()
+    inf[5000] = float("-inf")
+    assert cpu(bq.tensor_amax(inf.cuda())).item() == float("inf")
+
+
 def test_nvfp4_special_values(bq, orc):
     vals = [0.0, -0.0, 1e-30, -1e-30, 6.0, -6.0, 5.0, 2.5, 0.25, 0.75, 1e30, -1e30,
             float("inf"), float("-inf"), float("nan"), -float("nan")]
@@ -87,7 +162,9 @@ def test_mxfp8_special_blocks(bq, orc):
 
 @pytest.mark.parametrize("dtype", ["bf16", "f16", "f32"])
 @pytest.mark.parametrize("br,shape", [(1, (3, 384)), (1, (9, 200)), (128, (256, 384)),
-                                      (128, (130, 200)), (128, (1, 128)), (1, (4096, 128))])
+                                      (128, (130, 200)), (128, (1, 128)), (1, (4096, 128)),
+                                      (128, (130, 208)), (1, (5, 272)), (128, (300, 392)),
+                                      (128, (129, 8)), (128, (384, 1024))])
 def test_fp8_block_parity(bq, orc, dtype, br, shape):
     for dist in ("normal", "student_t3"):
         x = synthetic.Stream(13).tensor(shape, dtype, dist=dist)
