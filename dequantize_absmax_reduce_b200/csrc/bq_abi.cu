@@ -544,9 +544,8 @@ bq_status bq_packed_transpose(const uint8_t* w, const uint8_t* sc, int64_t n, in
     if (k == 0 || stride == 0) return BQ_OK;
     if (!w_t || (n > 0 && !w)) return BQ_ERR_INVALID_ARG;
     cudaStream_t s = S(stream);
-    if (bq::byte_transpose(w, n, k / 2, stride, w_t, s) != cudaSuccess) return BQ_ERR_CUDA;
-    if (sc) return from_cuda(bq::byte_transpose(sc, n, k / group_size, stride, sc_t, s));
-    return BQ_OK;
+    return from_cuda(bq::byte_transpose2(w, n, k / 2, w_t, sc, n, sc ? k / group_size : 0, sc_t,
+                                         stride, s));
 }
 
 }  // extern "C"

@@ -97,5 +97,10 @@ cudaError_t fp8_block_dequant(DT ydt, const uint8_t* e4m3, const float* scale, i
 // Byte transpose [rows, cols] -> [cols, stride], columns [rows, stride) zeroed.
 cudaError_t byte_transpose(const uint8_t* in, int64_t rows, int64_t cols, int64_t stride,
                            uint8_t* out, cudaStream_t st);
+// Two byte transposes with the same output stride (packed weights and their
+// scales) in one launch when both fit the wide-tile kernel; in1 may be null.
+cudaError_t byte_transpose2(const uint8_t* in0, int64_t rows0, int64_t cols0, uint8_t* out0,
+                            const uint8_t* in1, int64_t rows1, int64_t cols1, uint8_t* out1,
+                            int64_t stride, cudaStream_t st);
 
 }  // namespace bq

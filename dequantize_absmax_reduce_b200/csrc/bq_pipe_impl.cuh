@@ -131,6 +131,92 @@ __device__ __forceinline__ void range_acc(const U4& r, uint32_t& ph, uint32_t& p
         }
     }
 }
+// Two-lane 16-bit range steps: the larger magnitude (ABS, sign meaningless),
+// or max / min; PROP propagates a NaN operand instead of skipping it.
+template <class T, bool ABS, bool PROP>
+__device__ __forceinline__ uint32_t pk_hi(uint32_t a, uint32_t b) {
+    uint32_t r;
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        if (ABS && PROP) asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+        else if (ABS) asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+        else if (PROP) asm("max.NaN.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+        else asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    } else {
+        if (ABS && PROP) asm("max.NaN.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+        else if (ABS) asm("max.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+        else if (PROP) asm("max.NaN.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+        else asm("max.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    }
+    return r;
+}
+template <class T, bool PROP>
+__device__ __forceinline__ uint32_t pk_lo(uint32_t a, uint32_t b) {
+    uint32_t r;
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        if (PROP) asm("min.NaN.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+        else asm("min.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    } else {
+        if (PROP) asm("min.NaN.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+        else asm("min.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    }
+    return r;
+}
+template <bool PROP>
+__device__ __forceinline__ float f_hi(float a, float b) {
+    if constexpr (PROP) {
+        float r;
+        asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+        return r;
+    } else {
+        return fmaxf(a, b);
+    }
+}
+// Range of N 16-byte vectors folded into the accumulators of range_acc by a
+// reduction tree: depth 2 + ceil(log2 N) instead of a serial chain of 4N
+// dependent operations. Same result as N calls of range_acc.
+template <class T, bool ABS, bool PROP, int N>
+__device__ __forceinline__ void range_tree(const U4* r, uint32_t& ph, uint32_t& pl, float& hi,
+                                           float& nlo) {
+    if constexpr (sizeof(T) == 2) {
+        uint32_t h[N], l[N];
+#pragma unroll
+        for (int j = 0; j < N; ++j) {
+            h[j] = pk_hi<T, ABS, PROP>(pk_hi<T, ABS, PROP>(r[j].x, r[j].y), pk_hi<T, ABS, PROP>(r[j].z, r[j].w));
+            if (!ABS) l[j] = pk_lo<T, PROP>(pk_lo<T, PROP>(r[j].x, r[j].y), pk_lo<T, PROP>(r[j].z, r[j].w));
+        }
+#pragma unroll
+        for (int st = 1; st < N; st *= 2)
+#pragma unroll
+            for (int i = 0; i + st < N; i += 2 * st) {
+                h[i] = pk_hi<T, ABS, PROP>(h[i], h[i + st]);
+                if (!ABS) l[i] = pk_lo<T, PROP>(l[i], l[i + st]);
+            }
+        ph = pk_hi<T, ABS, PROP>(ph, h[0]);
+        if (!ABS) pl = pk_lo<T, PROP>(pl, l[0]);
+    } else {
+        float h[N], l[N];
+#pragma unroll
+        for (int j = 0; j < N; ++j) {
+            const float a = __uint_as_float(r[j].x), b = __uint_as_float(r[j].y);
+            const float c = __uint_as_float(r[j].z), d = __uint_as_float(r[j].w);
+            if (ABS) {
+                h[j] = f_hi<PROP>(f_hi<PROP>(fabsf(a), fabsf(b)), f_hi<PROP>(fabsf(c), fabsf(d)));
+            } else {
+                h[j] = f_hi<PROP>(f_hi<PROP>(a, b), f_hi<PROP>(c, d));
+                l[j] = f_hi<PROP>(f_hi<PROP>(-a, -b), f_hi<PROP>(-c, -d));
+            }
+        }
+#pragma unroll
+        for (int st = 1; st < N; st *= 2)
+#pragma unroll
+            for (int i = 0; i + st < N; i += 2 * st) {
+                h[i] = f_hi<PROP>(h[i], h[i + st]);
+                if (!ABS) l[i] = f_hi<PROP>(l[i], l[i + st]);
+            }
+        hi = f_hi<PROP>(hi, h[0]);
+        if (!ABS) nlo = f_hi<PROP>(nlo, l[0]);
+    }
+}
 // Packed accumulators -> (max(0, max x), max(0, -min x)) or (amax, 0).
 template <class T, bool ABS>
 __device__ __forceinline__ void range_finish(uint32_t ph, uint32_t pl, float& hi, float& nlo) {
@@ -178,13 +264,16 @@ __device__ __forceinline__ bool range_finish_nan(uint32_t ph, uint32_t pl, float
 // 257..512 vectors (the per-token rows of 4096 bf16); ring depth of the
 // group-tiled element kernels.
 #ifndef BQ_SEG_STAGES_16K
-#define BQ_SEG_STAGES_16K 4
+#define BQ_SEG_STAGES_16K 3
 #endif
 #ifndef BQ_SEG_STAGES_32K
-#define BQ_SEG_STAGES_32K 3
+#define BQ_SEG_STAGES_32K 2
 #endif
 #ifndef BQ_SEG_TEAM_512
 #define BQ_SEG_TEAM_512 64
+#endif
+#ifndef BQ_SEG_TEAM_16
+#define BQ_SEG_TEAM_16 4
 #endif
 #ifndef BQ_MAP_STAGES
 #define BQ_MAP_STAGES 3
@@ -265,6 +354,24 @@ __global__ void __launch_bounds__(256) k_seg_pipe(PipeArgs a) {
     uint32_t parity = 0;
     for (int64_t tile = blockIdx.x; tile < a.n_tiles; tile += grid) {
         const bool ok = mbar_wait(smem_addr(&bars[slot]), parity);
+        const uint8_t* slot_ptr = ring + (size_t)slot * a.slot_bytes;
+        const int64_t seg = tile * a.P + team;
+        const bool seg_ok = seg < a.n_seg;
+        const bool full = seg_ok && full_groups;
+
+        // This thread's vectors of its group, straight from shared memory,
+        // in the team's rotated order (vidx). (After a failed wait the slot
+        // holds stale bytes; they are read but never used.)
+        U4 raw[NV];
+        const uint32_t gbase = smem_addr(slot_ptr + (size_t)team * G * esz) + (uint32_t)(lane * 16);
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+            const int e = (vidx(j) * TEAM + lane) * VEC;
+            raw[j] = (full || (seg_ok && e < G)) ? ld_shared16(gbase + (uint32_t)(vidx(j) * TEAM * 16))
+                                                 : U4{0u, 0u, 0u, 0u};
+        }
+        // One barrier: every thread holds its vectors, so the slot is free
+        // and is refilled with tile + S before this tile is encoded.
         if (__syncthreads_or(!ok)) {
             if (tid == 0) {
                 atomicOr(&g_pipe_error, 1u);
@@ -281,34 +388,27 @@ __global__ void __launch_bounds__(256) k_seg_pipe(PipeArgs a) {
             __syncthreads();
             return;
         }
-        const uint8_t* slot_ptr = ring + (size_t)slot * a.slot_bytes;
-        const int64_t seg = tile * a.P + team;
-        const bool seg_ok = seg < a.n_seg;
-        const bool full = seg_ok && full_groups;
-
-        // This thread's vectors of its group, straight from shared memory,
-        // in the team's rotated order (vidx).
-        U4 raw[NV];
-        const uint32_t gbase = smem_addr(slot_ptr + (size_t)team * G * esz) + (uint32_t)(lane * 16);
-#pragma unroll
-        for (int j = 0; j < NV; ++j) {
-            const int e = (vidx(j) * TEAM + lane) * VEC;
-            raw[j] = (full || (seg_ok && e < G)) ? ld_shared16(gbase + (uint32_t)(vidx(j) * TEAM * 16))
-                                                 : U4{0u, 0u, 0u, 0u};
+        if (tid == 0) {
+            const int64_t next = tile + (int64_t)S * grid;
+            if (next < a.n_tiles) {
+                fence_proxy_async();
+                bulk_load(smem_addr(ring + (size_t)slot * a.slot_bytes),
+                          (const uint8_t*)a.x + (size_t)next * a.P * G * esz, tile_bytes(next),
+                          smem_addr(&bars[slot]));
+            }
         }
+        if (++slot == S) { slot = 0; parity ^= 1u; }
         // Range with NaN propagation; a thread that met a NaN recomputes its
         // part ignoring NaN (the range the formats define) and its warp takes
         // the general encoders.
         uint32_t ph = 0u, pl = 0u;
         float hi = 0.0f, nlo = 0.0f;
-#pragma unroll
-        for (int j = 0; j < NV; ++j) range_acc<T, ABS, true>(raw[j], ph, pl, hi, nlo);
+        range_tree<T, ABS, true, NV>(raw, ph, pl, hi, nlo);
         const bool saw_nan = range_finish_nan<T, ABS>(ph, pl, hi, nlo);
         if (saw_nan) {
             ph = pl = 0u;
             hi = nlo = 0.0f;
-#pragma unroll
-            for (int j = 0; j < NV; ++j) range_acc<T, ABS, false>(raw[j], ph, pl, hi, nlo);
+            range_tree<T, ABS, false, NV>(raw, ph, pl, hi, nlo);
             range_finish<T, ABS>(ph, pl, hi, nlo);
         }
         const bool warp_nan = __any_sync(0xffffffffu, saw_nan);
@@ -379,9 +479,17 @@ __global__ void __launch_bounds__(256) k_seg_pipe(PipeArgs a) {
             if (seg_ok && R.fast && noclamp && !warp_nan) {
                 const Recip2 R2 = make_recip2(R);
                 const F2 magic2 = f2_bcast(kMagic), zp2 = f2_bcast(zf), s2v = f2_bcast(sc);
+                // Whole groups: one branch-free block, so the vectors' division
+                // chains interleave.
+                if (full) {
 #pragma unroll
-                for (int j = 0; j < NV; ++j)
-                    if (vok(j)) emit_int_fast<T, OP, !SYM>(raw[j], R2, magic2, zp2, s2v, qb + voff(j), yb + voff(j));
+                    for (int j = 0; j < NV; ++j)
+                        emit_int_fast<T, OP, !SYM>(raw[j], R2, magic2, zp2, s2v, qb + voff(j), yb + voff(j));
+                } else {
+#pragma unroll
+                    for (int j = 0; j < NV; ++j)
+                        if (vok(j)) emit_int_fast<T, OP, !SYM>(raw[j], R2, magic2, zp2, s2v, qb + voff(j), yb + voff(j));
+                }
             } else if (seg_ok) {
 #pragma unroll
                 for (int j = 0; j < NV; ++j) {
@@ -404,9 +512,14 @@ __global__ void __launch_bounds__(256) k_seg_pipe(PipeArgs a) {
                 const Recip R = make_recip(s);
                 if (seg_ok && R.fast && !warp_nan) {
                     const Recip2 R2 = make_recip2(R);
+                    if (full) {
 #pragma unroll
-                    for (int j = 0; j < NV; ++j)
-                        if (vok(j)) emit_fp8_fast<T>(raw[j], R2, base + coff(j));
+                        for (int j = 0; j < NV; ++j) emit_fp8_fast<T>(raw[j], R2, base + coff(j));
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < NV; ++j)
+                            if (vok(j)) emit_fp8_fast<T>(raw[j], R2, base + coff(j));
+                    }
                 } else if (seg_ok) {
 #pragma unroll
                     for (int j = 0; j < NV; ++j) {
@@ -421,7 +534,10 @@ __global__ void __launch_bounds__(256) k_seg_pipe(PipeArgs a) {
                 const int E = mx_exponent(hi);
                 if (seg_ok && lane == 0) a.zp[seg] = (uint8_t)(E + 127);
                 const F2 mul2 = f2_bcast(exp2i(-E));
-                if (seg_ok) {
+                if (full) {
+#pragma unroll
+                    for (int j = 0; j < NV; ++j) emit_mx_fast<T>(raw[j], mul2, base + coff(j));
+                } else if (seg_ok) {
 #pragma unroll
                     for (int j = 0; j < NV; ++j)
                         if (vok(j)) emit_mx_fast<T>(raw[j], mul2, base + coff(j));
@@ -436,9 +552,14 @@ __global__ void __launch_bounds__(256) k_seg_pipe(PipeArgs a) {
                 const bool fast = R.fast && eff > 0.0f && hi <= __fmul_rn(0x1p64f, eff) && !warp_nan;
                 if (seg_ok && fast) {
                     const Recip2 R2 = make_recip2(R);
+                    if (full) {
 #pragma unroll
-                    for (int j = 0; j < NV; ++j)
-                        if (vok(j)) emit_nv_fast<T>(raw[j], R2, base + coff(j));
+                        for (int j = 0; j < NV; ++j) emit_nv_fast<T>(raw[j], R2, base + coff(j));
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < NV; ++j)
+                            if (vok(j)) emit_nv_fast<T>(raw[j], R2, base + coff(j));
+                    }
                 } else if (seg_ok) {
 #pragma unroll
                     for (int j = 0; j < NV; ++j) {
@@ -450,18 +571,6 @@ __global__ void __launch_bounds__(256) k_seg_pipe(PipeArgs a) {
                 }
             }
         }
-        // Every thread is done with this slot: refill it with tile it + S.
-        __syncthreads();
-        if (tid == 0) {
-            const int64_t next = tile + (int64_t)S * grid;
-            if (next < a.n_tiles) {
-                fence_proxy_async();
-                bulk_load(smem_addr(ring + (size_t)slot * a.slot_bytes),
-                          (const uint8_t*)a.x + (size_t)next * a.P * G * esz, tile_bytes(next),
-                          smem_addr(&bars[slot]));
-            }
-        }
-        if (++slot == S) { slot = 0; parity ^= 1u; }
     }
 }
 
@@ -572,6 +681,23 @@ __global__ void __launch_bounds__(256) k_nv_quant(PipeArgs a) {
     uint32_t parity = 0;
     for (int64_t tile = blockIdx.x; tile < a.n_tiles; tile += grid) {
         const bool okw = mbar_wait(smem_addr(&bars[slot]), parity);
+        const uint32_t sbase = smem_addr(ring + (size_t)slot * SLOT);
+        // The thread's NV_BPT blocks go through each step together, so that
+        // their serial per-block work (range, block scale, table) overlaps.
+        const bool tile_full = (tile + 1) * P <= a.n_seg;
+        U4 r0[NV_BPT], r1[NV_BPT];
+        bool okb[NV_BPT], nan[NV_BPT];
+        float hi[NV_BPT];
+        uint32_t sb[NV_BPT];
+#pragma unroll
+        for (int g = 0; g < NV_BPT; ++g) {
+            const int lb = g * 256 + tid;                     // block in the tile
+            okb[g] = tile_full || tile * P + lb < a.n_seg;
+            const uint32_t ba = sbase + (uint32_t)lb * 32u;
+            r0[g] = okb[g] ? ld_shared16(ba + (uint32_t)(rot * 16)) : U4{0u, 0u, 0u, 0u};
+            r1[g] = okb[g] ? ld_shared16(ba + (uint32_t)((rot ^ 1) * 16)) : U4{0u, 0u, 0u, 0u};
+        }
+        // One barrier: the blocks are in registers, the slot is refilled now.
         if (__syncthreads_or(!okw)) {
             if (tid == 0) {
                 atomicOr(&g_pipe_error, 1u);
@@ -586,32 +712,25 @@ __global__ void __launch_bounds__(256) k_nv_quant(PipeArgs a) {
             __syncthreads();
             return;
         }
-        const uint32_t sbase = smem_addr(ring + (size_t)slot * SLOT);
-        // The thread's NV_BPT blocks go through each step together, so that
-        // their serial per-block work (range, block scale, table) overlaps.
-        U4 r0[NV_BPT], r1[NV_BPT];
-        bool okb[NV_BPT], nan[NV_BPT];
-        float hi[NV_BPT];
-        uint32_t sb[NV_BPT];
-#pragma unroll
-        for (int g = 0; g < NV_BPT; ++g) {
-            const int lb = g * 256 + tid;                     // block in the tile
-            okb[g] = tile * P + lb < a.n_seg;
-            const uint32_t ba = sbase + (uint32_t)lb * 32u;
-            r0[g] = okb[g] ? ld_shared16(ba + (uint32_t)(rot * 16)) : U4{0u, 0u, 0u, 0u};
-            r1[g] = okb[g] ? ld_shared16(ba + (uint32_t)((rot ^ 1) * 16)) : U4{0u, 0u, 0u, 0u};
+        if (tid == 0) {
+            const int64_t next = tile + (int64_t)S * grid;
+            if (next < a.n_tiles) {
+                fence_proxy_async();
+                bulk_load(smem_addr(ring + (size_t)slot * SLOT), (const uint8_t*)a.x + (size_t)next * SLOT,
+                          tile_bytes(next), smem_addr(&bars[slot]));
+            }
         }
+        if (++slot == S) { slot = 0; parity ^= 1u; }
 #pragma unroll
         for (int g = 0; g < NV_BPT; ++g) {
             uint32_t ph = 0u, pl = 0u;
             float h = 0.0f, nlo = 0.0f;
-            range_acc<T, true, true>(r0[g], ph, pl, h, nlo);
-            range_acc<T, true, true>(r1[g], ph, pl, h, nlo);
+            const U4 rr[2] = {r0[g], r1[g]};
+            range_tree<T, true, true, 2>(rr, ph, pl, h, nlo);
             nan[g] = range_finish_nan<T, true>(ph, pl, h, nlo);
             if (nan[g]) {
                 ph = 0u;
-                range_acc<T, true, false>(r0[g], ph, pl, h, nlo);
-                range_acc<T, true, false>(r1[g], ph, pl, h, nlo);
+                range_tree<T, true, false, 2>(rr, ph, pl, h, nlo);
                 range_finish<T, true>(ph, pl, h, nlo);
             }
             hi[g] = h;
@@ -620,7 +739,7 @@ __global__ void __launch_bounds__(256) k_nv_quant(PipeArgs a) {
         for (int g = 0; g < NV_BPT; ++g) sb[g] = e4m3x2(div_any(hi[g], R6), 0.0f) & 0xFFu;
 #pragma unroll
         for (int g = 0; g < NV_BPT; ++g) {
-            if (!okb[g]) continue;
+            if (!tile_full && !okb[g]) continue;
             const int64_t blk = tile * P + g * 256 + tid;
             a.zp[blk] = (uint8_t)sb[g];
             const NvEntry e = table[sb[g]];
@@ -639,16 +758,6 @@ __global__ void __launch_bounds__(256) k_nv_quant(PipeArgs a) {
             }
             st8(a.q + blk * 8, rot ? w1 : w0, rot ? w0 : w1);
         }
-        __syncthreads();
-        if (tid == 0) {
-            const int64_t next = tile + (int64_t)S * grid;
-            if (next < a.n_tiles) {
-                fence_proxy_async();
-                bulk_load(smem_addr(ring + (size_t)slot * SLOT), (const uint8_t*)a.x + (size_t)next * SLOT,
-                          tile_bytes(next), smem_addr(&bars[slot]));
-            }
-        }
-        if (++slot == S) { slot = 0; parity ^= 1u; }
     }
 }
 
@@ -718,15 +827,14 @@ __global__ void __launch_bounds__(256) k_fp8_tile_tma(const __grid_constant__ CU
         float hi = 0.0f, nlo = 0.0f;
         bool nan = false;
         if (okw) {
+            U4 rv[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                range_acc<T, true, true>(ld_shared16(sbase + (uint32_t)(i * 256 + tid) * 16u), ph, pl, hi, nlo);
+            for (int i = 0; i < 8; ++i) rv[i] = ld_shared16(sbase + (uint32_t)(i * 256 + tid) * 16u);
+            range_tree<T, true, true, 8>(rv, ph, pl, hi, nlo);
             nan = range_finish_nan<T, true>(ph, pl, hi, nlo);
             if (nan) {
                 ph = 0u;
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    range_acc<T, true, false>(ld_shared16(sbase + (uint32_t)(i * 256 + tid) * 16u), ph, pl, hi, nlo);
+                range_tree<T, true, false, 8>(rv, ph, pl, hi, nlo);
                 range_finish<T, true>(ph, pl, hi, nlo);
             }
         }
@@ -866,9 +974,11 @@ __global__ void __launch_bounds__(256) k_range_pipe(RangeArgs a) {
         const uint32_t base = smem_addr(ring + (size_t)slot * RANGE_CHUNK);
         const int nv = (int)(chunk_bytes(c) / 16);
         if (nv == RANGE_CHUNK / 16) {
+            constexpr int NVC = RANGE_CHUNK / 16 / 256;
+            U4 rv[NVC];
 #pragma unroll
-            for (int v = 0; v < RANGE_CHUNK / 16 / 256; ++v)
-                range_acc<T, ABS, false>(ld_shared16(base + (uint32_t)((v * 256 + tid) * 16)), ph, pl, hi, nlo);
+            for (int v = 0; v < NVC; ++v) rv[v] = ld_shared16(base + (uint32_t)((v * 256 + tid) * 16));
+            range_tree<T, ABS, false, NVC>(rv, ph, pl, hi, nlo);
         } else {
             for (int v = tid; v < nv; v += 256)
                 range_acc<T, ABS, false>(ld_shared16(base + (uint32_t)(v * 16)), ph, pl, hi, nlo);
@@ -1304,7 +1414,7 @@ static cudaError_t launch_pipe_u(const PipeArgs& a, cudaStream_t st) {
     if (U <= 2) return launch_pipe_t<T, PK, 1, 2, SYM>(a, st);
     if (U <= 4) return launch_pipe_t<T, PK, 1, 4, SYM>(a, st);
     if (U <= 8) return launch_pipe_t<T, PK, 2, 4, SYM>(a, st);
-    if (U <= 16) return launch_pipe_t<T, PK, 4, 4, SYM>(a, st);
+    if (U <= 16) return launch_pipe_t<T, PK, BQ_SEG_TEAM_16, 16 / BQ_SEG_TEAM_16, SYM>(a, st);
     if (U <= 32) return launch_pipe_t<T, PK, 8, 4, SYM>(a, st);
     if constexpr (PK == PK_INT_Q || PK == PK_INT_FAKE) {
         if (U <= 64) return launch_pipe_t<T, PK, 16, 4, SYM>(a, st);

@@ -190,7 +190,8 @@ def test_fp8_special_values(bq, orc):
 
 @pytest.mark.parametrize("n,k,gs,align", [(8, 32, 16, 1), (7, 32, 16, 16), (33, 64, 32, 16),
                                           (100, 96, 16, 64), (4096, 256, 16, 16), (1, 2, 2, 1),
-                                          (130, 1000, 8, 16)])
+                                          (130, 1000, 8, 16), (300, 1024, 16, 16), (33, 8704, 16, 16),
+                                          (64, 512, 32, 16), (200, 1056, 16, 16), (5, 8192, 16, 64)])
 def test_packed_transpose_parity(bq, orc, n, k, gs, align):
     g = np.random.default_rng(n + k)
     w = torch.from_numpy(g.integers(0, 256, (n, k // 2), dtype=np.uint8))
