@@ -260,17 +260,13 @@ __device__ __forceinline__ bool range_finish_nan(uint32_t ph, uint32_t pl, float
 
 // ------------------------------------------------------------ the kernel
 // Tuning constants (compile-time): ring depth of the dynamic quantizer for
-// slots of up to 16 KB (NV <= 4) and 32 KB (NV = 8); team width for groups of
-// 257..512 vectors (the per-token rows of 4096 bf16); ring depth of the
-// group-tiled element kernels.
+// slots of up to 16 KB (NV <= 4) and 32 KB (NV >= 8); team width for groups of
+// 9..16 vectors; ring depth of the group-tiled element kernels.
 #ifndef BQ_SEG_STAGES_16K
 #define BQ_SEG_STAGES_16K 3
 #endif
 #ifndef BQ_SEG_STAGES_32K
 #define BQ_SEG_STAGES_32K 2
-#endif
-#ifndef BQ_SEG_TEAM_512
-#define BQ_SEG_TEAM_512 64
 #endif
 #ifndef BQ_SEG_TEAM_16
 #define BQ_SEG_TEAM_16 4
@@ -281,10 +277,10 @@ __device__ __forceinline__ bool range_finish_nan(uint32_t ph, uint32_t pl, float
 
 template <int NV> struct PipeStages { static constexpr int S = NV <= 4 ? BQ_SEG_STAGES_16K : BQ_SEG_STAGES_32K; };
 
-template <class T, int PK, int TEAM, int NV, bool SYM>
-__global__ void __launch_bounds__(256) k_seg_pipe(PipeArgs a) {
+template <class T, int PK, int TEAM, int NV, bool SYM, int NT>
+__global__ void __launch_bounds__(NT) k_seg_pipe(PipeArgs a) {
     constexpr int VEC = Traits<T>::VEC;
-    constexpr int NW = 8;
+    constexpr int NW = NT / 32;
     constexpr int SPAN = TEAM * NV * VEC;          // elements a team covers
     constexpr bool ABS = (PK != PK_INT_Q && PK != PK_INT_FAKE) || SYM;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -1337,14 +1333,14 @@ __global__ void __launch_bounds__(256) k_seg_map(SegMapArgs p) {
 // shared memory. Each caller passes its own `cache` (a static array in the
 // launcher of one kernel instantiation), which remembers the answer for up to
 // eight distinct ring sizes, so the query runs once per process and size.
-static int occupancy_for(const void* k, size_t smem, unsigned long long (&cache)[8]) {
+static int occupancy_for(const void* k, size_t smem, unsigned long long (&cache)[8], int threads = 256) {
     for (int i = 0; i < 8; ++i) {
         const unsigned long long e = __atomic_load_n(&cache[i], __ATOMIC_RELAXED);
         if (e == 0) break;
         if ((e >> 8) == smem) return (int)(e & 0xFFu) - 1;
     }
     int v = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, k, 256, smem) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, k, threads, smem) != cudaSuccess) {
         (void)cudaGetLastError();
         v = 0;
     }
@@ -1358,29 +1354,29 @@ static int occupancy_for(const void* k, size_t smem, unsigned long long (&cache)
     return v;
 }
 
-template <class T, int PK, int TEAM, int NV, bool SYM>
+template <class T, int PK, int TEAM, int NV, bool SYM, int NT = 256>
 static cudaError_t launch_pipe_t(PipeArgs a, cudaStream_t st) {
-    constexpr int P = 256 / TEAM;
+    constexpr int P = NT / TEAM;
     constexpr int S = PipeStages<NV>::S;
     a.P = P;
     a.slot_bytes = P * a.G * (int)sizeof(T);
     a.n_tiles = (a.n_seg + P - 1) / P;
     a.stages = S;
     const size_t smem = 128 + (size_t)S * a.slot_bytes;
-    auto k = k_seg_pipe<T, PK, TEAM, NV, SYM>;
+    auto k = k_seg_pipe<T, PK, TEAM, NV, SYM, NT>;
     // Largest ring this instantiation can need: P groups of TEAM*NV vectors.
     static const cudaError_t attr = cudaFuncSetAttribute(
         k, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 + S * P * TEAM * NV * 16);
     if (attr != cudaSuccess) return attr;
     static unsigned long long occ[8];
-    const int bps = occupancy_for((const void*)k, smem, occ);
+    const int bps = occupancy_for((const void*)k, smem, occ, NT);
     if (bps < 1) return cudaErrorNotSupported;
     int64_t grid = (int64_t)sm_count() * bps;
     if (grid > a.n_tiles) grid = a.n_tiles;
     // NVFP4 with a per-tensor scale from the range record: overlap the range
     // kernel's tail (the kernel waits for it before reading the record).
-    if (PK == PK_NV && a.static_global == 0) return launch_pdl(k, (unsigned)grid, 256u, smem, st, a);
-    k<<<(unsigned)grid, 256, smem, st>>>(a);
+    if (PK == PK_NV && a.static_global == 0) return launch_pdl(k, (unsigned)grid, (unsigned)NT, smem, st, a);
+    k<<<(unsigned)grid, NT, smem, st>>>(a);
     return cudaGetLastError();
 }
 
@@ -1420,7 +1416,9 @@ static cudaError_t launch_pipe_u(const PipeArgs& a, cudaStream_t st) {
         if (U <= 64) return launch_pipe_t<T, PK, 16, 4, SYM>(a, st);
         if (U <= 128) return launch_pipe_t<T, PK, 32, 4, SYM>(a, st);
         if (U <= 256) return launch_pipe_t<T, PK, 64, 4, SYM>(a, st);
-        if (U <= 512) return launch_pipe_t<T, PK, BQ_SEG_TEAM_512, 512 / BQ_SEG_TEAM_512, SYM>(a, st);
+        // Rows of up to 512 vectors: one warp per group, 16 vectors per lane,
+        // 128-thread CTAs (the reduction stays inside the warp).
+        if (U <= 512) return launch_pipe_t<T, PK, 32, 16, SYM, 128>(a, st);
         if (U <= 1024) return launch_pipe_t<T, PK, 128, 8, SYM>(a, st);
         if (U <= 2048) return launch_pipe_t<T, PK, 256, 8, SYM>(a, st);
     }
