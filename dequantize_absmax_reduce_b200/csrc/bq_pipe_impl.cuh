@@ -272,7 +272,7 @@ __device__ __forceinline__ bool range_finish_nan(uint32_t ph, uint32_t pl, float
 #define BQ_SEG_TEAM_16 4
 #endif
 #ifndef BQ_MAP_STAGES
-#define BQ_MAP_STAGES 3
+#define BQ_MAP_STAGES 2
 #endif
 
 template <int NV> struct PipeStages { static constexpr int S = NV <= 4 ? BQ_SEG_STAGES_16K : BQ_SEG_STAGES_32K; };
@@ -1239,6 +1239,34 @@ __global__ void __launch_bounds__(256) k_seg_map(SegMapArgs p) {
     fetch((int64_t)blockIdx.x * p.P + team, pf_s, pf_z);
     for (int64_t tile = blockIdx.x; tile < p.n_tiles; tile += grid) {
         const bool ok = mbar_wait(smem_addr(&bars[slot]), parity);
+        const int64_t seg = tile * p.P + team;
+        const bool seg_ok = seg < a.n_seg;
+        // This thread's vectors (codes: 8 / 4 bytes per vector; otherwise x and,
+        // for the backwards, dy) copied to registers. (After a failed wait the
+        // slot holds stale bytes; they are read but never used.)
+        const uint8_t* sa = ring + (size_t)slot * p.slot_bytes + (size_t)team * G * p.in_esz;
+        const uint8_t* sb = ring + (size_t)slot * p.slot_bytes + p.part_bytes + (size_t)team * G * ESZ;
+        U4 va[NV], vb[NV];
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+            const int e = (j * TEAM + lane) * W;              // element offset in the group
+            const bool v_ok = seg_ok && (full_groups || e < G);
+            va[j] = U4{0u, 0u, 0u, 0u};
+            vb[j] = U4{0u, 0u, 0u, 0u};
+            if (v_ok) {
+                if constexpr (OP == OP_DEQ) {
+                    if constexpr (W == 8)
+                        asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(va[j].x), "=r"(va[j].y) : "r"(smem_addr(sa + e)));
+                    else
+                        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(va[j].x) : "r"(smem_addr(sa + e)));
+                } else {
+                    va[j] = ld_shared16(smem_addr(sa + (size_t)e * ESZ));
+                    if constexpr (TWO) vb[j] = ld_shared16(smem_addr(sb + (size_t)e * ESZ));
+                }
+            }
+        }
+        // One barrier: the bounded wait's verdict, and the slot is free to be
+        // refilled with tile + S while this tile is computed.
         if (__syncthreads_or(!ok)) {
             if (tid == 0) {
                 atomicOr(&g_pipe_error, 1u);
@@ -1254,11 +1282,18 @@ __global__ void __launch_bounds__(256) k_seg_map(SegMapArgs p) {
             __syncthreads();
             return;
         }
-        const int64_t seg = tile * p.P + team;
+        if (tid == 0) {
+            const int64_t next = tile + (int64_t)S * grid;
+            if (next < p.n_tiles) {
+                fence_proxy_async();
+                issue(next, slot);
+            }
+        }
+        if (++slot == S) { slot = 0; parity ^= 1u; }
         const float cur_s = pf_s;
         const int cur_z = pf_z;
         fetch((tile + grid) * p.P + team, pf_s, pf_z);
-        if (seg < a.n_seg) {
+        if (seg_ok) {
             if constexpr (TWO && TEAM >= 32) {
                 group_set<T, false, RHAZ>(a, seg, cur_s, cur_z, st);
                 st.mfast = mask_thresholds_warp<RHAZ>(st.R, st.ip, &st.x_lo, &st.x_hi);
@@ -1266,8 +1301,6 @@ __global__ void __launch_bounds__(256) k_seg_map(SegMapArgs p) {
             } else {
                 group_set<T, TWO, RHAZ>(a, seg, cur_s, cur_z, st);
             }
-            const uint8_t* sa = ring + (size_t)slot * p.slot_bytes + (size_t)team * G * p.in_esz;
-            const uint8_t* sb = ring + (size_t)slot * p.slot_bytes + p.part_bytes + (size_t)team * G * ESZ;
             const int64_t gbase = seg * G;
 #pragma unroll
             for (int j = 0; j < NV; ++j) {
@@ -1275,24 +1308,17 @@ __global__ void __launch_bounds__(256) k_seg_map(SegMapArgs p) {
                 if (!full_groups && e >= G) continue;
                 Acc o[W];
                 if constexpr (OP == OP_DEQ) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) o[k] = deq_code_f(va[j].x, k, st, a.cfg.q_signed);
                     if constexpr (W == 8) {
-                        uint32_t w0, w1;
-                        asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(smem_addr(sa + e)));
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) o[k] = deq_code_f(w0, k, st, a.cfg.q_signed);
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) o[4 + k] = deq_code_f(w1, k, st, a.cfg.q_signed);
-                    } else {
-                        uint32_t w0;
-                        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w0) : "r"(smem_addr(sa + e)));
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) o[k] = deq_code_f(w0, k, st, a.cfg.q_signed);
+                        for (int k = 0; k < 4; ++k) o[4 + k] = deq_code_f(va[j].y, k, st, a.cfg.q_signed);
                     }
                     st16((T*)a.out + gbase + e, pack_vec<T>(o));
                 } else {
                     Acc xa[W], xb[W];
-                    load_vec<T>(ld_shared16(smem_addr(sa + (size_t)e * ESZ)), xa);
-                    if constexpr (TWO) load_vec<T>(ld_shared16(smem_addr(sb + (size_t)e * ESZ)), xb);
+                    load_vec<T>(va[j], xa);
+                    if constexpr (TWO) load_vec<T>(vb[j], xb);
                     uint32_t cw[W];
                     if constexpr (TWO) {
                         if (st.fast) {
@@ -1316,15 +1342,6 @@ __global__ void __launch_bounds__(256) k_seg_map(SegMapArgs p) {
                 }
             }
         }
-        __syncthreads();
-        if (tid == 0) {
-            const int64_t next = tile + (int64_t)S * grid;
-            if (next < p.n_tiles) {
-                fence_proxy_async();
-                issue(next, slot);
-            }
-        }
-        if (++slot == S) { slot = 0; parity ^= 1u; }
     }
 }
 
@@ -1410,7 +1427,10 @@ static cudaError_t launch_pipe_u(const PipeArgs& a, cudaStream_t st) {
     if (U <= 2) return launch_pipe_t<T, PK, 1, 2, SYM>(a, st);
     if (U <= 4) return launch_pipe_t<T, PK, 1, 4, SYM>(a, st);
     if (U <= 8) return launch_pipe_t<T, PK, 2, 4, SYM>(a, st);
-    if (U <= 16) return launch_pipe_t<T, PK, BQ_SEG_TEAM_16, 16 / BQ_SEG_TEAM_16, SYM>(a, st);
+    if (U <= 16) {
+        if constexpr (BQ_SEG_TEAM_16 == 1) return launch_pipe_t<T, PK, 1, 16, SYM, 128>(a, st);
+        else return launch_pipe_t<T, PK, BQ_SEG_TEAM_16, 16 / BQ_SEG_TEAM_16, SYM>(a, st);
+    }
     if (U <= 32) return launch_pipe_t<T, PK, 8, 4, SYM>(a, st);
     if constexpr (PK == PK_INT_Q || PK == PK_INT_FAKE) {
         if (U <= 64) return launch_pipe_t<T, PK, 16, 4, SYM>(a, st);
