@@ -46,9 +46,9 @@ FLUSH_BYTES = 256 << 20
 # the workload above, with the sha256 of the kernel sources it was taken on;
 # reported as null once the sources change.
 NCU_TRAFFIC = {
-    "quantize_per_token": {"src_sha256": "78153fee8008be0045a136d071c579da257e0ee37770ac21ade35987138b743b", "bytes_per_launch": 70508800},
-    "dequantize_per_token": {"src_sha256": "78153fee8008be0045a136d071c579da257e0ee37770ac21ade35987138b743b", "bytes_per_launch": 38081024},
-    "quantize_per_token_backward": {"src_sha256": "78153fee8008be0045a136d071c579da257e0ee37770ac21ade35987138b743b", "bytes_per_launch": 161464320},
+    "quantize_per_token": {"src_sha256": "b757a10650d3c4d5f0ca25e4c2c51607917146d36db91a995dc853839ad7278d", "bytes_per_launch": 70188800},
+    "dequantize_per_token": {"src_sha256": "b757a10650d3c4d5f0ca25e4c2c51607917146d36db91a995dc853839ad7278d", "bytes_per_launch": 38370304},
+    "quantize_per_token_backward": {"src_sha256": "b757a10650d3c4d5f0ca25e4c2c51607917146d36db91a995dc853839ad7278d", "bytes_per_launch": 158897920},
 }
 
 
@@ -530,7 +530,7 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-breakdown", action="store_true", help="skip the per-granularity table")
