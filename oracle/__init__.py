@@ -41,7 +41,9 @@ def lib() -> C.CDLL:
                      "or_fake_quantize", "or_ste_backward", "or_dequantize_backward",
                      "or_tensor_amax", "or_nvfp4_quantize", "or_nvfp4_dequantize",
                      "or_mxfp8_quantize", "or_mxfp8_dequantize", "or_fp8_block_quantize",
-                     "or_fp8_block_dequantize", "or_packed_transpose"):
+                     "or_fp8_block_dequantize", "or_packed_transpose",
+                     "or_packed_transpose_concat", "or_nvfp4_concat_rows",
+                     "or_nvfp4_predequant_fp8"):
             getattr(_lib, name).restype = C.c_int
         _lib.or_align_up.restype = C.c_int64
         _lib.or_align_up.argtypes = [C.c_int64, C.c_int64]
@@ -312,3 +314,50 @@ def packed_transpose(w: torch.Tensor, sc: torch.Tensor | None, n: int, k: int, g
                                   C.c_int64(k), C.c_int64(gs), C.c_int64(align), _p(w_t), _p(sc_t),
                                   C.byref(st)), "packed_transpose")
     return w_t, sc_t, st.value
+
+
+def packed_transpose_concat(parts, k: int, gs: int, align: int = 1, scales: bool = True):
+    """parts: list of (w [n_i, k/2] u8, sc [n_i, k/gs] u8 or None, n_i) sharing k ->
+    (w_t [k/2, stride], sc_t [k/gs, stride] or None, stride); part i occupies
+    columns [sum of the earlier n, + n_i)."""
+    n_parts = len(parts)
+    ws = [_c(w) for w, _, _ in parts]
+    scs = [_c(s) for _, s, _ in parts] if scales else []
+    ns = [int(n) for _, _, n in parts]
+    total = sum(ns)
+    stride = align_up(total, align) if n_parts else 0
+    w_t = torch.zeros((k // 2, max(stride, 0)), dtype=torch.uint8)
+    sc_t = torch.zeros((k // gs, max(stride, 0)), dtype=torch.uint8) if scales else None
+    WP = (C.c_void_p * max(n_parts, 1))(*[t.data_ptr() for t in ws])
+    SP = (C.c_void_p * max(n_parts, 1))(*[t.data_ptr() for t in scs]) if scales else None
+    NP = (C.c_int64 * max(n_parts, 1))(*ns)
+    st = C.c_int64()
+    _ok(lib().or_packed_transpose_concat(C.c_int(n_parts), WP, SP, NP, C.c_int64(k), C.c_int64(gs),
+                                         C.c_int64(align), _p(w_t), _p(sc_t), C.byref(st)),
+        "packed_transpose_concat")
+    return w_t, sc_t, st.value
+
+
+def nvfp4_concat_rows(w1, sc1, s2_1: float, w2, sc2, s2_2: float, k: int):
+    """Row concatenation of two NVFP4 weights; raises unless the per-tensor
+    scales are bit-identical. Returns (w [n1+n2, k/2], sc [n1+n2, k/16], s2)."""
+    w1, sc1, w2, sc2 = _c(w1), _c(sc1), _c(w2), _c(sc2)
+    n1, n2 = w1.shape[0], w2.shape[0]
+    w = torch.zeros((n1 + n2, k // 2), dtype=torch.uint8)
+    sc = torch.zeros((n1 + n2, k // 16), dtype=torch.uint8)
+    s2o = C.c_float()
+    rc = lib().or_nvfp4_concat_rows(_p(w1), _p(sc1), C.c_float(s2_1), C.c_int64(n1), _p(w2), _p(sc2),
+                                    C.c_float(s2_2), C.c_int64(n2), C.c_int64(k), _p(w), _p(sc),
+                                    C.byref(s2o))
+    if rc == 2:
+        raise OracleError("oracle nvfp4_concat_rows: per-tensor scales differ")
+    _ok(rc, "nvfp4_concat_rows")
+    return w, sc, s2o.value
+
+
+def nvfp4_predequant_fp8(packed, sc, s2: float, n: int, k: int):
+    """NVFP4 [n, k] -> E4M3 codes u8 [n, k] with the per-tensor scale applied."""
+    e = torch.zeros((n, k), dtype=torch.uint8)
+    _ok(lib().or_nvfp4_predequant_fp8(_p(_c(packed)), _p(_c(sc)), C.c_float(s2), C.c_int64(n),
+                                      C.c_int64(k), _p(e)), "nvfp4_predequant_fp8")
+    return e

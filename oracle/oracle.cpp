@@ -17,7 +17,9 @@
 //   [QuantizedWeight] docs.metrale.ai QuantizedWeight — NVFP4 layout: packed
 //               E2M1 two per byte, FP8 scale per 16, f32 per-tensor
 //               weight_scale_2; transpose_for_gemm(_gs) and the padded
-//               transpose (stride = align_up(n, align), pad zeroed).
+//               transpose (stride = align_up(n, align), pad zeroed); the
+//               multi-part transpose_concat_for_gemm(_gs, _padded),
+//               concat_rows and predequant_to_fp8.
 //   [smile.llm.quant] package summary — Fp8BlockGemm / Fp8BlockDequant
 //               (E4M3, f32 scale per 1x128 activation group and per 128x128
 //               weight tile, weight_scale_inv) and MxFp8 (E4M3, E8M0 scale per
@@ -709,6 +711,80 @@ int or_packed_transpose(const uint8_t* w, const uint8_t* sc, int64_t n, int64_t 
                 sc_t[i * stride + j] = (j < n) ? sc[j * ng + i] : 0;
     }
     *stride_out = stride;
+    return 0;
+}
+
+// ---- Multi-part transpose [QuantizedWeight transpose_concat_for_gemm,
+// transpose_concat_for_gemm_gs, transpose_concat_for_gemm_padded]: parts
+// (w_i [n_i, k/2], sc_i [n_i, k/gs]) that share k; part i lands in columns
+// [off_i, off_i + n_i) of w_t [k/2, stride] and sc_t [k/gs, stride], with
+// off_i = n_0 + ... + n_{i-1} and stride = align_up(n_0 + ... + n_{p-1}, align);
+// the pad columns are zero. No parts is an error (the page's rule). sc may be
+// null (weights only); then every sc_i is ignored.
+int or_packed_transpose_concat(int n_parts, const uint8_t* const* w, const uint8_t* const* sc,
+                               const int64_t* n, int64_t k, int64_t gs, int64_t align,
+                               uint8_t* w_t, uint8_t* sc_t, int64_t* stride_out) {
+    if (n_parts < 1 || k < 0 || align < 1 || k % 2 != 0) return 1;
+    if (sc && (gs < 1 || k % gs != 0)) return 1;
+    int64_t total = 0;
+    for (int p = 0; p < n_parts; ++p) {
+        if (n[p] < 0) return 1;
+        total += n[p];
+    }
+    const int64_t stride = or_align_up(total, align);
+    const int64_t kb = k / 2, ng = sc ? k / gs : 0;
+    for (int64_t i = 0; i < kb * stride; ++i) w_t[i] = 0;
+    if (sc) for (int64_t i = 0; i < ng * stride; ++i) sc_t[i] = 0;
+    int64_t off = 0;
+    for (int p = 0; p < n_parts; ++p) {
+        for (int64_t i = 0; i < kb; ++i)
+            for (int64_t j = 0; j < n[p]; ++j) w_t[i * stride + off + j] = w[p][j * kb + i];
+        if (sc)
+            for (int64_t i = 0; i < ng; ++i)
+                for (int64_t j = 0; j < n[p]; ++j) sc_t[i * stride + off + j] = sc[p][j * ng + i];
+        off += n[p];
+    }
+    *stride_out = stride;
+    return 0;
+}
+
+// ---- concat_rows [QuantizedWeight concat_rows]: two NVFP4 weights with the
+// same k, [n1, k/2] + [n2, k/2] -> [n1 + n2, k/2] and their E4M3 scales
+// (group 16) [n1, k/16] + [n2, k/16] -> [n1 + n2, k/16]. The two per-tensor
+// scales must be bit-identical (else an error, 2); the result carries the
+// first one.
+int or_nvfp4_concat_rows(const uint8_t* w1, const uint8_t* sc1, float s2_1, int64_t n1,
+                         const uint8_t* w2, const uint8_t* sc2, float s2_2, int64_t n2, int64_t k,
+                         uint8_t* w_out, uint8_t* sc_out, float* s2_out) {
+    if (n1 < 0 || n2 < 0 || k < 0 || k % 16 != 0) return 1;
+    uint32_t b1, b2;
+    std::memcpy(&b1, &s2_1, 4);
+    std::memcpy(&b2, &s2_2, 4);
+    if (b1 != b2) return 2;
+    const int64_t kb = k / 2, ng = k / 16;
+    for (int64_t i = 0; i < n1 * kb; ++i) w_out[i] = w1[i];
+    for (int64_t i = 0; i < n2 * kb; ++i) w_out[n1 * kb + i] = w2[i];
+    for (int64_t i = 0; i < n1 * ng; ++i) sc_out[i] = sc1[i];
+    for (int64_t i = 0; i < n2 * ng; ++i) sc_out[n1 * ng + i] = sc2[i];
+    *s2_out = s2_1;
+    return 0;
+}
+
+// ---- predequant_to_fp8 [QuantizedWeight predequant_to_fp8]: an NVFP4 weight
+// [n, k] as FP8 E4M3 [n, k] with the per-tensor scale applied: each element is
+// the NVFP4 dequantized value fl(e2m1(code) * fl(dec(sb) * s2)) encoded to
+// E4M3 (round to nearest even, saturating to +-448, NaN -> 0x7F).
+int or_nvfp4_predequant_fp8(const uint8_t* packed, const uint8_t* sc, float s2, int64_t n,
+                            int64_t k, uint8_t* e4m3) {
+    if (n < 0 || k < 0 || k % 16 != 0) return 1;
+    for (int64_t r = 0; r < n; ++r)
+        for (int64_t c = 0; c < k; ++c) {
+            const int64_t idx = r * k + c;
+            const double eff = r32(dec_e4m3(sc[r * (k / 16) + c / 16]) * (double)s2);
+            const uint8_t byte = packed[idx / 2];
+            const uint8_t code = (idx % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+            e4m3[idx] = enc_e4m3(r32(dec_e2m1(code) * eff));
+        }
     return 0;
 }
 
