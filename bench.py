@@ -310,8 +310,24 @@ def per_granularity(B, api, torch, device, peak, reps=5):
     w_t = torch.empty((K // 2, R), dtype=torch.uint8, device=device)
     sc_t = torch.empty((K // 16, R), dtype=torch.uint8, device=device)
     timed(wl, "packed_transpose(weights+scales, align 16)",
-          lambda: B.bq_packed_transpose(packed, sc, R, K, 16, 16, w_t, sc_t), 2 * (n // 2 + n // 16), 2)
-    del x, y, packed, sc, w_t, sc_t
+          lambda: B.bq_packed_transpose(packed, sc, R, K, 16, 16, w_t, sc_t), 2 * (n // 2 + n // 16), 1)
+    # weight preparation: three row blocks transposed into one [K/2, N] twin,
+    # two halves joined by rows, and the FP8 twin with the per-tensor scale applied
+    bounds = [(0, R // 4), (R // 4, 3 * R // 4), (3 * R // 4, R)]
+    parts = [(packed[a:b].contiguous(), sc[a:b].contiguous(), b - a) for a, b in bounds]
+    timed(wl, "packed_transpose_concat(3 parts, align 16)",
+          lambda: B.bq_packed_transpose_concat(parts, K, 16, 16, w_t, sc_t), 2 * (n // 2 + n // 16), 1)
+    h = R // 2
+    p1, p2 = packed[:h].contiguous(), packed[h:].contiguous()
+    c1, c2 = sc[:h].contiguous(), sc[h:].contiguous()
+    wj, cj = torch.empty_like(packed), torch.empty_like(sc)
+    s2v = float(gs.item())
+    timed(wl, "nvfp4_concat_rows",
+          lambda: B.bq_nvfp4_concat_rows(p1, c1, s2v, p2, c2, s2v, K, wj, cj), 2 * (n // 2 + n // 16), 1)
+    e8 = torch.empty((R, K), dtype=torch.uint8, device=device)
+    timed(wl, "nvfp4_predequant_to_fp8", lambda: B.bq_nvfp4_predequant_to_fp8(packed, sc, gs, e8),
+          n // 2 + n // 16 + n, 1)
+    del x, y, packed, sc, w_t, sc_t, parts, p1, p2, c1, c2, wj, cj, e8
 
     # FP8 blocks and MXFP8, bf16 activations [16384, 7168] and weights [7168, 18432]
     wl = "fp8_blocks_bf16"

@@ -85,6 +85,11 @@ _SIGS = {
     "bq_fp8_block_quantize": [_P, C.c_int, _I64, _I64, _I32, _I32, _P, _P, _P],
     "bq_fp8_block_dequantize": [_P, _P, _I64, _I64, _I32, _I32, _P, C.c_int, _P],
     "bq_packed_transpose": [_P, _P, _I64, _I64, _I64, _I64, _P, _P, C.POINTER(_I64), _P],
+    "bq_packed_transpose_concat": [_I32, C.POINTER(_P), C.POINTER(_P), C.POINTER(_I64), _I64, _I64,
+                                   _I64, _P, _P, C.POINTER(_I64), _P],
+    "bq_nvfp4_concat_rows": [_P, _P, C.c_float, _I64, _P, _P, C.c_float, _I64, _I64, _P, _P,
+                             C.POINTER(C.c_float), _P],
+    "bq_nvfp4_predequant_to_fp8": [_P, _P, _P, _I64, _I64, _P, _P],
 }
 for _name, _args in _SIGS.items():
     _f = getattr(lib, _name)
@@ -363,3 +368,32 @@ def bq_packed_transpose(w, sc, n, k, group_size, align, w_t, sc_t, stream=None) 
     _check(lib.bq_packed_transpose(_ptr(w), _ptr(sc), n, k, group_size, align, _ptr(w_t), _ptr(sc_t),
                                    C.byref(st), _stream(stream)), "bq_packed_transpose")
     return st.value
+
+
+def bq_packed_transpose_concat(parts, k, group_size, align, w_t, sc_t, stream=None) -> int:
+    """parts: list of (w, sc or None, n); w_t / sc_t sized [k/2, stride], [k/gs, stride]."""
+    n_parts = len(parts)
+    WP = (_P * max(n_parts, 1))(*[_ptr(w) for w, _, _ in parts])
+    with_sc = sc_t is not None
+    SP = (_P * max(n_parts, 1))(*[_ptr(sc) for _, sc, _ in parts]) if with_sc else None
+    NP = (_I64 * max(n_parts, 1))(*[int(n) for _, _, n in parts])
+    st = _I64()
+    _check(lib.bq_packed_transpose_concat(n_parts, WP, SP, NP, k, group_size, align, _ptr(w_t),
+                                          _ptr(sc_t), C.byref(st), _stream(stream)),
+           "bq_packed_transpose_concat")
+    return st.value
+
+
+def bq_nvfp4_concat_rows(w1, sc1, s2_1, w2, sc2, s2_2, k, w_out, sc_out, stream=None) -> float:
+    n1, n2 = w1.shape[0], w2.shape[0]
+    s2o = C.c_float()
+    _check(lib.bq_nvfp4_concat_rows(_ptr(w1), _ptr(sc1), float(s2_1), n1, _ptr(w2), _ptr(sc2),
+                                    float(s2_2), n2, k, _ptr(w_out), _ptr(sc_out), C.byref(s2o),
+                                    _stream(stream)), "bq_nvfp4_concat_rows")
+    return s2o.value
+
+
+def bq_nvfp4_predequant_to_fp8(packed, scale_e4m3, global_scale, e4m3, stream=None):
+    n, k = e4m3.shape
+    _check(lib.bq_nvfp4_predequant_to_fp8(_ptr(packed), _ptr(scale_e4m3), _ptr(global_scale), n, k,
+                                          _ptr(e4m3), _stream(stream)), "bq_nvfp4_predequant_to_fp8")

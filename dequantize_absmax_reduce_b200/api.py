@@ -218,3 +218,37 @@ def packed_transpose(w, sc, n: int, k: int, group_size: int, align: int = 1, str
                                                device=w.device)
     st = B.bq_packed_transpose(w, sc, n, k, group_size, align, w_t, sc_t, stream)
     return w_t, sc_t, st
+
+
+def packed_transpose_concat(parts, k: int, group_size: int, align: int = 1, scales: bool = True,
+                            stream=None):
+    """parts: list of (w [n_i, k/2], sc [n_i, k/gs] or None, n_i) sharing k ->
+    (w_t [k/2, stride], sc_t [k/gs, stride] or None, stride); part i occupies
+    the columns after the earlier parts'."""
+    total = sum(int(n) for _, _, n in parts)
+    stride = B.bq_packed_transpose_stride(total, align)
+    dev = parts[0][0].device
+    w_t = torch.empty((k // 2, stride), dtype=torch.uint8, device=dev)
+    sc_t = torch.empty((k // group_size, stride), dtype=torch.uint8, device=dev) if scales else None
+    st = B.bq_packed_transpose_concat(parts, k, group_size, align, w_t, sc_t, stream)
+    return w_t, sc_t, st
+
+
+def nvfp4_concat_rows(w1, sc1, s2_1: float, w2, sc2, s2_2: float, k: int, stream=None):
+    """Row concatenation of two NVFP4 weights (per-tensor scales must be
+    bit-identical) -> (w [n1+n2, k/2], sc [n1+n2, k/16], s2)."""
+    n = w1.shape[0] + w2.shape[0]
+    w = torch.empty((n, k // 2), dtype=torch.uint8, device=w1.device)
+    sc = torch.empty((n, k // 16), dtype=torch.uint8, device=w1.device)
+    s2 = B.bq_nvfp4_concat_rows(w1, sc1, s2_1, w2, sc2, s2_2, k, w, sc, stream)
+    return w, sc, s2
+
+
+def nvfp4_predequant_to_fp8(packed, sc, s2, stream=None):
+    """NVFP4 [n, k] -> E4M3 codes u8 [n, k] with the per-tensor scale applied."""
+    n = packed.shape[0]
+    k = packed.shape[1] * 2
+    e = torch.empty((n, k), dtype=torch.uint8, device=packed.device)
+    gs = s2 if isinstance(s2, torch.Tensor) else torch.tensor([float(s2)], device=packed.device)
+    B.bq_nvfp4_predequant_to_fp8(packed, sc, gs, e, stream)
+    return e

@@ -548,4 +548,71 @@ bq_status bq_packed_transpose(const uint8_t* w, const uint8_t* sc, int64_t n, in
                                          stride, s));
 }
 
+bq_status bq_packed_transpose_concat(int32_t n_parts, const uint8_t* const* w,
+                                     const uint8_t* const* sc, const int64_t* n, int64_t k,
+                                     int64_t group_size, int64_t align, uint8_t* w_t,
+                                     uint8_t* sc_t, int64_t* out_stride, void* stream) {
+    if (n_parts < 1 || !w || !n || k < 0 || align < 1 || k % 2 != 0) return BQ_ERR_INVALID_ARG;
+    if ((sc == nullptr) != (sc_t == nullptr)) return BQ_ERR_INVALID_ARG;
+    if (sc && (group_size < 1 || k % group_size != 0)) return BQ_ERR_INVALID_ARG;
+    int64_t total = 0;
+    for (int32_t p = 0; p < n_parts; ++p) {
+        if (n[p] < 0 || total > INT64_MAX - n[p]) return BQ_ERR_INVALID_ARG;
+        total += n[p];
+    }
+    const int64_t stride = bq_packed_transpose_stride(total, align);
+    if (stride < 0) return BQ_ERR_INVALID_ARG;
+    if (out_stride) *out_stride = stride;
+    if (k == 0 || stride == 0) return BQ_OK;
+    if (!w_t) return BQ_ERR_INVALID_ARG;
+    for (int32_t p = 0; p < n_parts; ++p)
+        if (n[p] > 0 && (!w[p] || (sc && !sc[p]))) return BQ_ERR_INVALID_ARG;
+    cudaStream_t s = S(stream);
+    // Four parts (weights and scales: eight transposes) per launch.
+    constexpr int CHUNK = 4;
+    int64_t off = 0;
+    for (int32_t p0 = 0; p0 < n_parts; p0 += CHUNK) {
+        bq::XPart parts[2 * CHUNK];
+        int np = 0;
+        for (int32_t p = p0; p < n_parts && p < p0 + CHUNK; ++p) {
+            const int64_t olim = (p == n_parts - 1) ? stride - off : n[p];
+            parts[np++] = bq::XPart{w[p], n[p], k / 2, w_t + off, olim};
+            if (sc) parts[np++] = bq::XPart{sc[p], n[p], k / group_size, sc_t + off, olim};
+            off += n[p];
+        }
+        if (bq::byte_transpose_parts(parts, np, stride, s) != cudaSuccess) return BQ_ERR_CUDA;
+    }
+    return BQ_OK;
+}
+
+bq_status bq_nvfp4_concat_rows(const uint8_t* w1, const uint8_t* sc1, float s2_1, int64_t n1,
+                               const uint8_t* w2, const uint8_t* sc2, float s2_2, int64_t n2,
+                               int64_t k, uint8_t* w_out, uint8_t* sc_out, float* s2_out,
+                               void* stream) {
+    if (n1 < 0 || n2 < 0 || k < 0 || k % 16 != 0) return BQ_ERR_INVALID_ARG;
+    uint32_t b1, b2;
+    memcpy(&b1, &s2_1, 4);
+    memcpy(&b2, &s2_2, 4);
+    if (b1 != b2) return BQ_ERR_INVALID_ARG;      // the result carries one per-tensor scale
+    if (s2_out) *s2_out = s2_1;
+    if ((n1 + n2) * k == 0) return BQ_OK;
+    if (!w_out || !sc_out || (n1 > 0 && (!w1 || !sc1)) || (n2 > 0 && (!w2 || !sc2)))
+        return BQ_ERR_INVALID_ARG;
+    const int64_t kb = k / 2, ng = k / 16;
+    const void* src[4] = {w1, w2, sc1, sc2};
+    void* dst[4] = {w_out, w_out + n1 * kb, sc_out, sc_out + n1 * ng};
+    const int64_t bytes[4] = {n1 * kb, n2 * kb, n1 * ng, n2 * ng};
+    return from_cuda(bq::copy_segments(src, dst, bytes, 4, S(stream)));
+}
+
+bq_status bq_nvfp4_predequant_to_fp8(const uint8_t* packed, const uint8_t* scale_e4m3,
+                                     const float* global_scale, int64_t n, int64_t k,
+                                     uint8_t* e4m3, void* stream) {
+    if (n < 0 || k < 0 || k % 16 != 0) return BQ_ERR_INVALID_ARG;
+    if (n * k == 0) return BQ_OK;
+    if (!packed || !scale_e4m3 || !global_scale || !e4m3) return BQ_ERR_INVALID_ARG;
+    if (!aligned(global_scale, 4)) return BQ_ERR_MISALIGNED;
+    return from_cuda(bq::nvfp4_predequant_fp8(packed, scale_e4m3, global_scale, n, k, e4m3, S(stream)));
+}
+
 }  // extern "C"

@@ -94,9 +94,28 @@ cudaError_t fp8_tile_pipe(DT dt, const void* x, int64_t rows, int64_t cols, uint
 cudaError_t fp8_block_dequant(DT ydt, const uint8_t* e4m3, const float* scale, int64_t rows,
                               int64_t cols, int br, int bc, void* y, cudaStream_t st);
 
+// NVFP4 [rows, k] -> E4M3 [rows, k] with the per-tensor scale applied.
+cudaError_t nvfp4_predequant_fp8(const uint8_t* codes, const uint8_t* scales, const float* global_scale,
+                                 int64_t rows, int64_t k, uint8_t* out, cudaStream_t st);
+// Up to four byte-range copies in one launch.
+cudaError_t copy_segments(const void* const* src, void* const* dst, const int64_t* bytes, int n,
+                          cudaStream_t st);
+
 // Byte transpose [rows, cols] -> [cols, stride], columns [rows, stride) zeroed.
 cudaError_t byte_transpose(const uint8_t* in, int64_t rows, int64_t cols, int64_t stride,
                            uint8_t* out, cudaStream_t st);
+// One byte transpose of a multi-part concatenation: input [rows, cols] into
+// output rows of `stride` bytes starting at `out` (the part's column offset),
+// writing bytes [0, olim) of each row (input rows past `rows` read as zero).
+struct XPart {
+    const uint8_t* in;
+    int64_t rows, cols;
+    uint8_t* out;
+    int64_t olim;
+};
+// Every part in as few launches as possible (the wide-tile kernel when all
+// widths and bases are multiples of 16 bytes, else byte-wise).
+cudaError_t byte_transpose_parts(const XPart* parts, int n_parts, int64_t stride, cudaStream_t st);
 // Two byte transposes with the same output stride (packed weights and their
 // scales) in one launch when both fit the wide-tile kernel; in1 may be null.
 cudaError_t byte_transpose2(const uint8_t* in0, int64_t rows0, int64_t cols0, uint8_t* out0,

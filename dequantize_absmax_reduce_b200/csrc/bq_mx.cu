@@ -465,6 +465,85 @@ __global__ void __launch_bounds__(256) k_mx_deq8(DeqArgs a) {
     }
 }
 
+// ------------------------------------------------------------ NVFP4 -> FP8
+// predequant_to_fp8 (metrale QuantizedWeight): each element's NVFP4 value
+// fl(e2m1(code) * fl(dec(sb) * s2)) encoded to E4M3 (round to nearest even,
+// saturating). Items of 8 elements: 4 code bytes in, 8 E4M3 bytes out
+// (consecutive lanes write consecutive 8 bytes).
+__global__ void __launch_bounds__(256) k_nv_predeq8(const uint8_t* __restrict__ codes,
+                                                    const uint8_t* __restrict__ scales,
+                                                    const float* __restrict__ global_scale,
+                                                    int64_t numel, uint8_t* __restrict__ out) {
+    const float s2 = __ldg(global_scale);
+    const int64_t n_items = numel / 8;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < n_items;
+         base += stride * DQ_U) {
+        uint32_t w[DQ_U], sb[DQ_U];
+#pragma unroll
+        for (int u = 0; u < DQ_U; ++u) {
+            const int64_t it = base + u * stride;
+            if (it < n_items) {
+                w[u] = __ldg(reinterpret_cast<const uint32_t*>(codes) + it);
+                sb[u] = __ldg(scales + (it >> 1));
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < DQ_U; ++u) {
+            const int64_t it = base + u * stride;
+            if (it >= n_items) continue;
+            float o[8];
+            e2m1x8_mul(w[u], f2_bcast(__fmul_rn(e4m3_to_f32(sb[u]), s2)), o);
+            st8(out + it * 8, e4m3x4(o[0], o[1], o[2], o[3]), e4m3x4(o[4], o[5], o[6], o[7]));
+        }
+    }
+}
+
+// Element-wise fallback (any alignment).
+__global__ void __launch_bounds__(256) k_nv_predeq_scalar(const uint8_t* __restrict__ codes,
+                                                          const uint8_t* __restrict__ scales,
+                                                          const float* __restrict__ global_scale,
+                                                          int64_t numel, uint8_t* __restrict__ out) {
+    const float s2 = __ldg(global_scale);
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < numel;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const uint32_t byte = __ldg(codes + i / 2);
+        const float2 f = e2m1x2_to_f32(byte);
+        const float eff = __fmul_rn(e4m3_to_f32(__ldg(scales + i / 16)), s2);
+        out[i] = (uint8_t)e4m3x2(__fmul_rn((i & 1) ? f.y : f.x, eff), 0.0f);
+    }
+}
+
+// ------------------------------------------------------------ segment copies
+// Up to four (src, dst, bytes) copies in one launch (concat_rows): 16-byte
+// vectors over the aligned part of each segment, bytes for the rest.
+struct CopySeg {
+    const uint8_t* src;
+    uint8_t* dst;
+    int64_t bytes, nvec, vfirst, bfirst;
+};
+struct CopySegs {
+    CopySeg s[4];
+    int n;
+    int64_t nvec, nbytes;     // vector units, byte units over all segments
+};
+
+__global__ void __launch_bounds__(256) k_copy_segs(CopySegs c) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < c.nvec; i += stride) {
+        int q = 0;
+        while (q + 1 < c.n && i >= c.s[q + 1].vfirst) ++q;
+        const int64_t v = i - c.s[q].vfirst;
+        st16(c.s[q].dst + v * 16, ld16_stream(c.s[q].src + v * 16));
+    }
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < c.nbytes; i += stride) {
+        int q = 0;
+        while (q + 1 < c.n && i >= c.s[q + 1].bfirst) ++q;
+        const int64_t b = c.s[q].nvec * 16 + (i - c.s[q].bfirst);
+        c.s[q].dst[b] = __ldg(c.s[q].src + b);
+    }
+}
+
 // ------------------------------------------------------------ launchers
 static bool al(const void* p, int n) { return ((uintptr_t)p % (uintptr_t)n) == 0; }
 
@@ -633,6 +712,43 @@ cudaError_t fp8_block_dequant(DT ydt, const uint8_t* e4m3, const float* scale, i
     a.br = br; a.bc = bc; a.nbc = (cols + bc - 1) / bc;
     if (a.numel == 0) return cudaSuccess;
     return launch_deq_f<MX_FP8_1x128>(ydt, a, st);
+}
+
+cudaError_t nvfp4_predequant_fp8(const uint8_t* codes, const uint8_t* scales, const float* global_scale,
+                                 int64_t rows, int64_t k, uint8_t* out, cudaStream_t st) {
+    const int64_t numel = rows * k;
+    if (numel == 0) return cudaSuccess;
+    if (k % 16 == 0 && al(codes, 4) && al(out, 8)) {
+        const int64_t blocks = (numel / 8 + 256 * DQ_U - 1) / (256 * DQ_U);
+        k_nv_predeq8<<<grid_occ_mx<k_nv_predeq8>(blocks), 256, 0, st>>>(codes, scales, global_scale, numel, out);
+    } else {
+        k_nv_predeq_scalar<<<grid_occ_mx<k_nv_predeq_scalar>((numel + 255) / 256), 256, 0, st>>>(
+            codes, scales, global_scale, numel, out);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t copy_segments(const void* const* src, void* const* dst, const int64_t* bytes, int n,
+                          cudaStream_t st) {
+    CopySegs c{};
+    c.n = 0;
+    for (int i = 0; i < n && i < 4; ++i) {
+        CopySeg g;
+        g.src = (const uint8_t*)src[i];
+        g.dst = (uint8_t*)dst[i];
+        g.bytes = bytes[i];
+        const bool vec = al(g.src, 16) && al(g.dst, 16);
+        g.nvec = vec ? g.bytes / 16 : 0;
+        g.vfirst = c.nvec;
+        g.bfirst = c.nbytes;
+        c.nvec += g.nvec;
+        c.nbytes += g.bytes - g.nvec * 16;
+        c.s[c.n++] = g;
+    }
+    const int64_t work = c.nvec > c.nbytes ? c.nvec : c.nbytes;
+    if (work == 0) return cudaSuccess;
+    k_copy_segs<<<grid_cap((work + 255) / 256, 8), 256, 0, st>>>(c);
+    return cudaGetLastError();
 }
 
 }  // namespace bq

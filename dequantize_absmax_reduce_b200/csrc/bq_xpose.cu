@@ -59,21 +59,31 @@ __global__ void __launch_bounds__(256) k_xpose(const uint8_t* __restrict__ in, i
 // loads; a warp reads 32 full-sector bytes from each of 16 rows), transposes
 // the four 4x4 byte blocks in registers and parks sixteen output words in
 // shared memory (the 32 lanes of one store hit 32 distinct banks); the CTA
-// then writes each of the tile's 256 output rows as four 16-byte runs. Two
-// independent transposes (weights and scales) share one launch: blocks
-// [0, jobs[0].n_tiles) serve the first.
+// then writes each of the tile's 256 output rows as four 16-byte runs. Up to
+// XJOBS independent transposes share one launch (the weights and scales of
+// every part of a concatenation); job j owns blocks [first_j, first_j +
+// n_tiles_j). A job writes bytes [0, olim) of each output row from its base
+// `out` (a part's column offset into the shared rows); input rows beyond
+// `rows` read as zero, which fills the pad columns of the last part.
+constexpr int XJOBS = 8;
 struct XJob {
     const uint8_t* in;
-    int64_t rows, cols, stride, ntr, n_tiles;
+    int64_t rows, cols, stride, olim, ntr, n_tiles, first;
     uint8_t* out;
 };
-struct XJobs { XJob j[2]; };
+struct XJobs {
+    XJob j[XJOBS];
+    int n;
+};
 
 __global__ void __launch_bounds__(256) k_xpose_wide(XJobs jobs) {
     __shared__ uint32_t sm[256][17];                  // [output row][input-row word], padded
-    const bool second = (int64_t)blockIdx.x >= jobs.j[0].n_tiles;
-    const XJob& J = second ? jobs.j[1] : jobs.j[0];
-    const int64_t b = second ? (int64_t)blockIdx.x - jobs.j[0].n_tiles : (int64_t)blockIdx.x;
+    int ji = 0;
+#pragma unroll 1
+    for (int q = 1; q < jobs.n; ++q)
+        if ((int64_t)blockIdx.x >= jobs.j[q].first) ji = q;
+    const XJob& J = jobs.j[ji];
+    const int64_t b = (int64_t)blockIdx.x - J.first;
     const int64_t tr = b % J.ntr, tc = b / J.ntr;
     const int64_t r0 = tr * 64, c0 = tc * 256;
     const int t = threadIdx.x;
@@ -108,7 +118,7 @@ __global__ void __launch_bounds__(256) k_xpose_wide(XJobs jobs) {
         const int orow = 64 * k + (t >> 2), seg = t & 3;
         const int64_t oc = c0 + orow;                 // output row
         const int64_t ob = r0 + 16 * seg;             // output byte column
-        if (oc < J.cols && ob < J.stride) {
+        if (oc < J.cols && ob < J.olim) {
             U4 v;
             v.x = sm[orow][4 * seg + 0];
             v.y = sm[orow][4 * seg + 1];
@@ -119,16 +129,33 @@ __global__ void __launch_bounds__(256) k_xpose_wide(XJobs jobs) {
     }
 }
 
-static bool xpose_wide_ok(const uint8_t* in, int64_t cols, int64_t stride, const uint8_t* out) {
-    return cols % 16 == 0 && stride % 16 == 0 && ((uintptr_t)in % 16 == 0) && ((uintptr_t)out % 16 == 0);
+static bool xpose_wide_ok(const uint8_t* in, int64_t cols, int64_t stride, int64_t olim,
+                          const uint8_t* out) {
+    return cols % 16 == 0 && stride % 16 == 0 && olim % 16 == 0 && ((uintptr_t)in % 16 == 0) &&
+           ((uintptr_t)out % 16 == 0);
 }
-static XJob make_xjob(const uint8_t* in, int64_t rows, int64_t cols, int64_t stride, uint8_t* out) {
+static XJob make_xjob(const uint8_t* in, int64_t rows, int64_t cols, int64_t stride, int64_t olim,
+                      uint8_t* out) {
     XJob j;
-    j.in = in; j.rows = rows; j.cols = cols; j.stride = stride; j.out = out;
-    j.ntr = (stride + 63) / 64;
+    j.in = in; j.rows = rows; j.cols = cols; j.stride = stride; j.olim = olim; j.out = out;
+    j.ntr = (olim + 63) / 64;
     j.n_tiles = j.ntr * ((cols + 255) / 256);
-    if (cols == 0 || stride == 0) j.n_tiles = 0;
+    if (cols == 0 || olim == 0) j.n_tiles = 0;
+    j.first = 0;
     return j;
+}
+
+// Byte-wise transpose of one job (any widths and alignments): output byte
+// (oc, o) for o < olim is in[o][oc] for o < rows, else 0.
+__global__ void __launch_bounds__(256) k_xpose_bytes(const uint8_t* __restrict__ in, int64_t rows,
+                                                     int64_t cols, int64_t stride, int64_t olim,
+                                                     uint8_t* __restrict__ out) {
+    const int64_t n = cols * olim;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t oc = i / olim, o = i - oc * olim;
+        out[oc * stride + o] = (o < rows) ? __ldg(in + o * cols + oc) : (uint8_t)0;
+    }
 }
 
 // Any shape / alignment: one output byte per thread step.
@@ -164,21 +191,50 @@ cudaError_t byte_transpose(const uint8_t* in, int64_t rows, int64_t cols, int64_
 cudaError_t byte_transpose2(const uint8_t* in0, int64_t rows0, int64_t cols0, uint8_t* out0,
                             const uint8_t* in1, int64_t rows1, int64_t cols1, uint8_t* out1,
                             int64_t stride, cudaStream_t st) {
-    const bool wide0 = xpose_wide_ok(in0, cols0, stride, out0);
-    const bool wide1 = !in1 || xpose_wide_ok(in1, cols1, stride, out1);
-    if (wide0 && wide1) {
-        XJobs jobs;
-        jobs.j[0] = make_xjob(in0, rows0, cols0, stride, out0);
-        jobs.j[1] = in1 ? make_xjob(in1, rows1, cols1, stride, out1) : make_xjob(nullptr, 0, 0, 0, nullptr);
-        const int64_t nb = jobs.j[0].n_tiles + jobs.j[1].n_tiles;
-        if (nb == 0) return cudaSuccess;
-        if (nb > 0x7FFFFFFFll) return cudaErrorInvalidValue;
-        k_xpose_wide<<<(unsigned)nb, 256, 0, st>>>(jobs);
-        return cudaGetLastError();
+    XPart parts[2] = {{in0, rows0, cols0, out0, stride}, {in1, rows1, cols1, out1, stride}};
+    return byte_transpose_parts(parts, in1 ? 2 : 1, stride, st);
+}
+
+cudaError_t byte_transpose_parts(const XPart* parts, int n_parts, int64_t stride, cudaStream_t st) {
+    bool wide = stride % 16 == 0;
+    for (int i = 0; i < n_parts && wide; ++i)
+        wide = xpose_wide_ok(parts[i].in, parts[i].cols, stride, parts[i].olim, parts[i].out);
+    if (wide) {
+        for (int i0 = 0; i0 < n_parts; i0 += XJOBS) {
+            XJobs jobs{};
+            int64_t nb = 0;
+            jobs.n = 0;
+            for (int i = i0; i < n_parts && i < i0 + XJOBS; ++i) {
+                XJob j = make_xjob(parts[i].in, parts[i].rows, parts[i].cols, stride, parts[i].olim,
+                                   parts[i].out);
+                j.first = nb;
+                nb += j.n_tiles;
+                jobs.j[jobs.n++] = j;
+            }
+            if (nb == 0) continue;
+            if (nb > 0x7FFFFFFFll) return cudaErrorInvalidValue;
+            k_xpose_wide<<<(unsigned)nb, 256, 0, st>>>(jobs);
+            const cudaError_t e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+        }
+        return cudaSuccess;
     }
-    cudaError_t e = byte_transpose(in0, rows0, cols0, stride, out0, st);
-    if (e == cudaSuccess && in1) e = byte_transpose(in1, rows1, cols1, stride, out1, st);
-    return e;
+    for (int i = 0; i < n_parts; ++i) {
+        const XPart& p = parts[i];
+        if (p.cols == 0 || p.olim == 0) continue;
+        if (p.olim == stride && p.rows <= stride) {
+            const cudaError_t e = byte_transpose(p.in, p.rows, p.cols, stride, p.out, st);
+            if (e != cudaSuccess) return e;
+            continue;
+        }
+        const int64_t need = (p.cols * p.olim + 255) / 256;
+        const int64_t cap = (int64_t)sm_count() * 8;
+        k_xpose_bytes<<<(unsigned)(need < cap ? need : cap), 256, 0, st>>>(p.in, p.rows, p.cols, stride,
+                                                                           p.olim, p.out);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace bq

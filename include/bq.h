@@ -339,6 +339,46 @@ bq_status bq_packed_transpose(const uint8_t* w, const uint8_t* sc, int64_t n, in
  * w_t / sc_t before the call. Returns -1 for n < 0 or align < 1. Host only. */
 int64_t bq_packed_transpose_stride(int64_t n, int64_t align);
 
+/* [QuantizedWeight] transpose_concat_for_gemm / _gs / _padded: n_parts >= 1
+ * packed weights that share k, part p being w[p] u8 [n[p], k/2] with scales
+ * sc[p] u8 [n[p], k/group_size], transposed and concatenated along N into
+ * w_t u8 [k/2, stride] and sc_t u8 [k/group_size, stride]. Part p occupies
+ * columns [off_p, off_p + n[p]) with off_p = n[0] + ... + n[p-1];
+ * stride = align_up(n[0] + ... + n[n_parts-1], align) and the pad columns are
+ * set to 0. w, sc and n are HOST arrays of n_parts entries (device pointers,
+ * row counts); sc (the array) and sc_t may both be NULL (weights only). No
+ * parts (n_parts < 1) is BQ_ERR_INVALID_ARG, as on the page. The parts'
+ * per-tensor scales are the caller's to keep consistent (the page carries
+ * the first part's and checks nothing). *out_stride (host, may be NULL)
+ * receives the stride. Outputs must not overlap inputs. */
+bq_status bq_packed_transpose_concat(int32_t n_parts, const uint8_t* const* w,
+                                     const uint8_t* const* sc, const int64_t* n, int64_t k,
+                                     int64_t group_size, int64_t align, uint8_t* w_t,
+                                     uint8_t* sc_t, int64_t* out_stride, void* stream);
+
+/* [QuantizedWeight] concat_rows: two NVFP4 weights with the same k
+ * (k % 16 == 0) joined by rows into new buffers: w_out u8 [n1+n2, k/2] is
+ * w1 [n1, k/2] then w2 [n2, k/2], sc_out u8 [n1+n2, k/16] likewise. s2_1 and
+ * s2_2 are the host-side per-tensor scales (weight_scale_2): unless their
+ * bits are identical the call returns BQ_ERR_INVALID_ARG and launches
+ * nothing; otherwise *s2_out (host, may be NULL) receives s2_1. Outputs must
+ * not overlap inputs. */
+bq_status bq_nvfp4_concat_rows(const uint8_t* w1, const uint8_t* sc1, float s2_1, int64_t n1,
+                               const uint8_t* w2, const uint8_t* sc2, float s2_2, int64_t n2,
+                               int64_t k, uint8_t* w_out, uint8_t* sc_out, float* s2_out,
+                               void* stream);
+
+/* [QuantizedWeight] predequant_to_fp8: an NVFP4 weight [n, k] (packed
+ * [n, k/2], E4M3 block scales [n, k/16], device f32 *global_scale holding
+ * weight_scale_2) as FP8 E4M3 codes e4m3 u8 [n, k] with the per-tensor scale
+ * applied: code = E4M3(fl(e2m1(c) * fl(dec(sb) * s2))), i.e. the f32 value
+ * bq_nvfp4_dequantize produces, rounded to nearest even and saturating to
+ * +-448 (NaN -> 0x7F). k % 16 == 0. Asynchronous on `stream` (the page's
+ * version synchronises its stream; this one does not). */
+bq_status bq_nvfp4_predequant_to_fp8(const uint8_t* packed, const uint8_t* scale_e4m3,
+                                     const float* global_scale, int64_t n, int64_t k,
+                                     uint8_t* e4m3, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

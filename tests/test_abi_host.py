@@ -30,7 +30,8 @@ def test_header_declares_the_entry_points():
                  "bq_quantize_per_group", "bq_dequantize_per_group", "bq_fake_quantize",
                  "bq_quantize_per_group_backward", "bq_fake_quantize_backward",
                  "bq_dequantize_per_token_backward", "bq_nvfp4_quantize", "bq_nvfp4_dequantize",
-                 "bq_mxfp8_quantize", "bq_fp8_block_quantize", "bq_packed_transpose"):
+                 "bq_mxfp8_quantize", "bq_fp8_block_quantize", "bq_packed_transpose",
+                 "bq_packed_transpose_concat", "bq_nvfp4_concat_rows", "bq_nvfp4_predequant_to_fp8"):
         assert must in names
 
 
@@ -135,3 +136,24 @@ def test_empty_calls_succeed_without_a_device(B):
     assert B.lib.bq_quantize_per_token(None, C.byref(d), None, None, None, 0, None, 0, None) == B.BQ_OK
     assert B.lib.bq_dequantize_per_token(None, None, None, C.byref(d), None, B.BQ_F32, None) == B.BQ_OK
     assert B.lib.bq_mxfp8_quantize(None, B.BQ_BF16, 0, 64, None, None, None) == B.BQ_OK
+
+
+def test_weight_prep_argument_errors(B):
+    P = C.c_void_p(16)
+    NP = (C.c_int64 * 1)(4)
+    WP = (C.c_void_p * 1)(16)
+    st = C.c_int64()
+    # no parts, odd k, scales without sc_t
+    assert B.lib.bq_packed_transpose_concat(0, WP, None, NP, 32, 16, 1, P, None, C.byref(st), None) == B.BQ_ERR_INVALID_ARG
+    assert B.lib.bq_packed_transpose_concat(1, WP, None, NP, 31, 16, 1, P, None, C.byref(st), None) == B.BQ_ERR_INVALID_ARG
+    assert B.lib.bq_packed_transpose_concat(1, WP, WP, NP, 32, 16, 1, P, None, C.byref(st), None) == B.BQ_ERR_INVALID_ARG
+    # different per-tensor scales (bit patterns), k not a multiple of 16
+    s2o = C.c_float()
+    assert B.lib.bq_nvfp4_concat_rows(P, P, 1.0, 2, P, P, 1.0000001, 2, 32, P, P, C.byref(s2o), None) == B.BQ_ERR_INVALID_ARG
+    assert B.lib.bq_nvfp4_concat_rows(P, P, 0.0, 2, P, P, -0.0, 2, 32, P, P, C.byref(s2o), None) == B.BQ_ERR_INVALID_ARG
+    assert B.lib.bq_nvfp4_concat_rows(P, P, 1.0, 2, P, P, 1.0, 2, 24, P, P, C.byref(s2o), None) == B.BQ_ERR_INVALID_ARG
+    assert B.lib.bq_nvfp4_predequant_to_fp8(P, P, P, 4, 24, P, None) == B.BQ_ERR_INVALID_ARG
+    assert B.lib.bq_nvfp4_predequant_to_fp8(None, P, P, 4, 32, P, None) == B.BQ_ERR_INVALID_ARG
+    # zero-sized calls succeed without touching the device
+    assert B.lib.bq_nvfp4_concat_rows(None, None, 1.0, 0, None, None, 1.0, 0, 32, None, None, C.byref(s2o), None) == B.BQ_OK
+    assert s2o.value == 1.0
