@@ -43,7 +43,7 @@ def lib() -> C.CDLL:
                      "or_mxfp8_quantize", "or_mxfp8_dequantize", "or_fp8_block_quantize",
                      "or_fp8_block_dequantize", "or_packed_transpose",
                      "or_packed_transpose_concat", "or_nvfp4_concat_rows",
-                     "or_nvfp4_predequant_fp8"):
+                     "or_nvfp4_predequant_fp8", "or_mxfp4_quantize", "or_mxfp4_dequantize"):
             getattr(_lib, name).restype = C.c_int
         _lib.or_align_up.restype = C.c_int64
         _lib.or_align_up.argtypes = [C.c_int64, C.c_int64]
@@ -361,3 +361,21 @@ def nvfp4_predequant_fp8(packed, sc, s2: float, n: int, k: int):
     _ok(lib().or_nvfp4_predequant_fp8(_p(_c(packed)), _p(_c(sc)), C.c_float(s2), C.c_int64(n),
                                       C.c_int64(k), _p(e)), "nvfp4_predequant_fp8")
     return e
+
+
+def mxfp4_quantize(x: torch.Tensor):
+    """x [rows, k] -> (packed E2M1 u8 [rows, k/2], E8M0 u8 [rows, k/32])."""
+    x = _c(x)
+    rows, k = x.shape
+    p = torch.zeros((rows, k // 2), dtype=torch.uint8)
+    s = torch.zeros((rows, k // 32), dtype=torch.uint8)
+    _ok(lib().or_mxfp4_quantize(_p(x), C.c_int(_dt(x)), C.c_int64(rows), C.c_int64(k), _p(p), _p(s)),
+        "mxfp4_quantize")
+    return p, s
+
+
+def mxfp4_dequantize(p, s, rows: int, k: int, ydtype: str = "bf16"):
+    y = torch.zeros((rows, k), dtype=_TORCH[ydtype])
+    _ok(lib().or_mxfp4_dequantize(_p(_c(p)), _p(_c(s)), C.c_int64(rows), C.c_int64(k), _p(y),
+                                  C.c_int(_T[ydtype])), "mxfp4_dequantize")
+    return y

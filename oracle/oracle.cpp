@@ -52,7 +52,8 @@
 //     eff = fl(dec(sb)*s2), code = E2M1(fl(x/eff)), all-zero codes when
 //     eff == 0.
 //   * MXFP8: E = clamp(floor(log2 a) - 8, -127, 127), byte = E + 127 (an
-//     infinite a counts as 2^128), e = E4M3(fl(x * 2^-E)).
+//     infinite a counts as 2^128), e = E4M3(fl(x * 2^-E)). MXFP4: the same
+//     with 2 (the largest E2M1 exponent) in place of 8 and E2M1 codes.
 //   * FP8 block: s = fl(a/448) (0 -> 1), e = E4M3(fl(x/s)), s is stored.
 
 #include <cmath>
@@ -646,6 +647,55 @@ int or_mxfp8_dequantize(const uint8_t* e4m3, const uint8_t* e8m0, int64_t rows, 
         for (int64_t c = 0; c < k; ++c) {
             const int64_t idx = r * k + c;
             store_f(y, y_t, idx, r32(dec_e4m3(e4m3[idx]) * dec_e8m0(e8m0[r * (k / 32) + c / 32])));
+        }
+    return 0;
+}
+
+// ---- MXFP4 [QuantizedWeight: "E8M0 for native MXFP4"; OCP MX rule as for
+// MXFP8]: E2M1 elements packed two per byte (element 2j in the low nibble),
+// one E8M0 scale per 32 consecutive elements along the last dimension.
+// E = clamp(floor(log2 a) - 2, -127, 127) (2 = the largest E2M1 exponent; an
+// infinite a counts as 2^128, a = 0 gives -127), byte E + 127,
+// code = E2M1(fl(x * 2^-E)).
+int or_mxfp4_quantize(const void* x, int x_t, int64_t rows, int64_t k, uint8_t* packed,
+                      uint8_t* e8m0) {
+    if (x_t != OR_F32 && x_t != OR_F16 && x_t != OR_BF16) return 1;
+    if (rows < 0 || k < 0 || k % 32 != 0) return 1;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < k / 32; ++b) {
+            const int64_t base = r * k + b * 32;
+            double a = 0.0;
+            for (int j = 0; j < 32; ++j) {
+                double v = std::fabs(load_f(x, x_t, base + j));
+                if (v > a) a = v;
+            }
+            int fl2;
+            if (a == 0.0) fl2 = -1000;
+            else if (std::isinf(a)) fl2 = 128;
+            else { int e; std::frexp(a, &e); fl2 = e - 1; }
+            const int E = std::min(std::max(fl2 - 2, -127), 127);
+            e8m0[r * (k / 32) + b] = (uint8_t)(E + 127);
+            const double inv = std::ldexp(1.0, -E);      // exact power of two
+            for (int j = 0; j < 32; j += 2) {
+                const uint8_t c0 = enc_e2m1(r32(load_f(x, x_t, base + j) * inv));
+                const uint8_t c1 = enc_e2m1(r32(load_f(x, x_t, base + j + 1) * inv));
+                packed[(base + j) / 2] = (uint8_t)(c0 | (c1 << 4));
+            }
+        }
+    }
+    return 0;
+}
+
+int or_mxfp4_dequantize(const uint8_t* packed, const uint8_t* e8m0, int64_t rows, int64_t k,
+                        void* y, int y_t) {
+    if (y_t != OR_F32 && y_t != OR_F16 && y_t != OR_BF16) return 1;
+    if (rows < 0 || k < 0 || k % 32 != 0) return 1;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < k; ++c) {
+            const int64_t idx = r * k + c;
+            const uint8_t byte = packed[idx / 2];
+            const uint8_t code = (idx % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+            store_f(y, y_t, idx, r32(dec_e2m1(code) * dec_e8m0(e8m0[r * (k / 32) + c / 32])));
         }
     return 0;
 }

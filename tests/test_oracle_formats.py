@@ -171,3 +171,56 @@ def test_packed_transpose_vs_numpy(orc, n, k, gs, align):
     # Transposing back recovers the original bytes (nibbles untouched).
     back, _, st2 = orc.packed_transpose(w_t[:, :n].contiguous(), None, k // 2, 2 * n, 1, 1)
     assert np.array_equal(back.numpy(), w.numpy())
+
+
+# ---------------------------------------------------------------- MXFP4
+def _e2m1_nearest_even(t: np.ndarray) -> np.ndarray:
+    """Brute-force E2M1 code of f64 values t: nearest grid value, ties to the
+    even mantissa, saturating to +-6, sign kept (NaN -> 0x7)."""
+    mags = E2M1                                   # codes 0..7; odd code = odd mantissa
+    out = np.zeros(t.shape, dtype=np.uint8)
+    for i, v in np.ndenumerate(t):
+        if np.isnan(v):
+            out[i] = 0x7
+            continue
+        a = min(abs(v), 6.0)
+        d = np.abs(mags - a)
+        best = np.flatnonzero(d == d.min())
+        c = best[0] if len(best) == 1 else [b for b in best if b % 2 == 0][0]
+        out[i] = c | (0x8 if np.signbit(v) else 0)
+    return out
+
+
+def test_mxfp4_exact_grid_block_is_lossless(orc):
+    vals = np.concatenate([E2M1, -E2M1[1:], [0.0], E2M1[::-1], -E2M1[1:4], [0.0] * 5])[:32]
+    rows = [vals * 2.0 ** j for j in range(-4, 4)]
+    x = torch.tensor(np.array(rows), dtype=torch.float32)
+    p, s = orc.mxfp4_quantize(x)
+    assert s[:, 0].tolist() == [127 + j for j in range(-4, 4)]     # floor(log2(6*2^j)) - 2 = j
+    y = orc.mxfp4_dequantize(p, s, *x.shape, ydtype="f32")
+    assert torch.equal(y, x)
+
+
+def test_mxfp4_scale_and_codes_vs_frexp_and_brute_force(orc):
+    x = synthetic.Stream(24).tensor((6, 256), "bf16", dist="student_t3")
+    p, s = orc.mxfp4_quantize(x)
+    xv = x.double().numpy().reshape(6, 8, 32)
+    amax = np.abs(xv).max(axis=2)
+    want = np.array([[math.frexp(a)[1] - 1 - 2 + 127 for a in row] for row in amax])
+    assert np.array_equal(s.numpy().astype(np.int64), want)
+    E = (want - 127).astype(np.float64)[:, :, None]
+    t = xv * 2.0 ** -E                      # exact scaling by a power of two
+    assert np.array_equal(_unpack(p).reshape(6, 8, 32), _e2m1_nearest_even(t))
+
+
+def test_mxfp4_special_blocks(orc):
+    x = torch.zeros(1, 96)
+    x[0, 32] = -0.0
+    x[0, 33] = 1.0                          # amax 1 -> E = -2, 1 * 4 = 4: code 6
+    x[0, 64] = float("inf")
+    x[0, 65] = 5.0
+    p, s = orc.mxfp4_quantize(x)
+    assert s[0].tolist() == [0, 125, 127 + 126]       # zero block; E = -2; inf -> 2^128 -> E = 126
+    codes = _unpack(p)[0]
+    assert codes[32] == 0x8 and codes[33] == 0x6
+    assert codes[64] == 0x7                 # inf * 2^-126 saturates to 6
