@@ -327,7 +327,11 @@ def per_granularity(B, api, torch, device, peak, reps=5):
     e8 = torch.empty((R, K), dtype=torch.uint8, device=device)
     timed(wl, "nvfp4_predequant_to_fp8", lambda: B.bq_nvfp4_predequant_to_fp8(packed, sc, gs, e8),
           n // 2 + n // 16 + n, 1)
-    del x, y, packed, sc, w_t, sc_t, parts, p1, p2, c1, c2, wj, cj, e8
+    # MXFP4 of the same weight (E2M1 + E8M0 per 32)
+    sc32 = torch.empty((R, K // 32), dtype=torch.uint8, device=device)
+    timed(wl, "mxfp4_quantize", lambda: B.bq_mxfp4_quantize(x, packed, sc32), 2 * n + n // 2 + n // 32, 1)
+    timed(wl, "mxfp4_dequantize", lambda: B.bq_mxfp4_dequantize(packed, sc32, y), n // 2 + n // 32 + 2 * n, 1)
+    del x, y, packed, sc, w_t, sc_t, parts, p1, p2, c1, c2, wj, cj, e8, sc32
 
     # FP8 blocks and MXFP8, bf16 activations [16384, 7168] and weights [7168, 18432]
     wl = "fp8_blocks_bf16"

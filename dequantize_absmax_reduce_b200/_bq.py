@@ -82,6 +82,8 @@ _SIGS = {
     "bq_nvfp4_dequantize": [_P, _P, _P, _I64, _I64, _P, C.c_int, _P],
     "bq_mxfp8_quantize": [_P, C.c_int, _I64, _I64, _P, _P, _P],
     "bq_mxfp8_dequantize": [_P, _P, _I64, _I64, _P, C.c_int, _P],
+    "bq_mxfp4_quantize": [_P, C.c_int, _I64, _I64, _P, _P, _P],
+    "bq_mxfp4_dequantize": [_P, _P, _I64, _I64, _P, C.c_int, _P],
     "bq_fp8_block_quantize": [_P, C.c_int, _I64, _I64, _I32, _I32, _P, _P, _P],
     "bq_fp8_block_dequantize": [_P, _P, _I64, _I64, _I32, _I32, _P, C.c_int, _P],
     "bq_packed_transpose": [_P, _P, _I64, _I64, _I64, _I64, _P, _P, C.POINTER(_I64), _P],
@@ -397,3 +399,15 @@ def bq_nvfp4_predequant_to_fp8(packed, scale_e4m3, global_scale, e4m3, stream=No
     n, k = e4m3.shape
     _check(lib.bq_nvfp4_predequant_to_fp8(_ptr(packed), _ptr(scale_e4m3), _ptr(global_scale), n, k,
                                           _ptr(e4m3), _stream(stream)), "bq_nvfp4_predequant_to_fp8")
+
+
+def bq_mxfp4_quantize(x, packed, e8m0, stream=None):
+    rows, k = x.shape
+    _check(lib.bq_mxfp4_quantize(_ptr(x), DTYPE[x.dtype], rows, k, _ptr(packed), _ptr(e8m0),
+                                 _stream(stream)), "bq_mxfp4_quantize")
+
+
+def bq_mxfp4_dequantize(packed, e8m0, y, stream=None):
+    rows, k = y.shape
+    _check(lib.bq_mxfp4_dequantize(_ptr(packed), _ptr(e8m0), rows, k, _ptr(y), DTYPE[y.dtype],
+                                   _stream(stream)), "bq_mxfp4_dequantize")

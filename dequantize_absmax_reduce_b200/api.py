@@ -252,3 +252,19 @@ def nvfp4_predequant_to_fp8(packed, sc, s2, stream=None):
     gs = s2 if isinstance(s2, torch.Tensor) else torch.tensor([float(s2)], device=packed.device)
     B.bq_nvfp4_predequant_to_fp8(packed, sc, gs, e, stream)
     return e
+
+
+def mxfp4_quantize(x, stream=None):
+    """x [rows, k] -> (packed E2M1 u8 [rows, k/2], E8M0 u8 [rows, k/32])."""
+    rows, k = x.shape
+    p = torch.empty((rows, k // 2), dtype=torch.uint8, device=x.device)
+    s = torch.empty((rows, k // 32), dtype=torch.uint8, device=x.device)
+    B.bq_mxfp4_quantize(x, p, s, stream)
+    return p, s
+
+
+def mxfp4_dequantize(p, s, ydtype=torch.bfloat16, stream=None):
+    rows, k = p.shape[0], p.shape[1] * 2
+    y = torch.empty((rows, k), dtype=ydtype, device=p.device)
+    B.bq_mxfp4_dequantize(p, s, y, stream)
+    return y

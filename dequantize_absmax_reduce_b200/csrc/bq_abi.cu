@@ -494,6 +494,29 @@ bq_status bq_mxfp8_dequantize(const uint8_t* e4m3, const uint8_t* e8m0, int64_t 
                                     S(stream)));
 }
 
+// ---- MXFP4
+bq_status bq_mxfp4_quantize(const void* x, bq_dtype x_dtype, int64_t rows, int64_t k,
+                            uint8_t* packed, uint8_t* e8m0, void* stream) {
+    if (!is_half_or_f32(x_dtype)) return BQ_ERR_UNSUPPORTED;
+    if (rows < 0 || k < 0 || k % 32 != 0) return BQ_ERR_INVALID_ARG;
+    if (rows * k == 0) return BQ_OK;
+    if (!x || !packed || !e8m0) return BQ_ERR_INVALID_ARG;
+    if (!aligned(x, esize(x_dtype))) return BQ_ERR_MISALIGNED;
+    return from_cuda(bq::mx_quant(to_dt(x_dtype), bq::MX_MXFP4, x, rows, k, packed, e8m0, nullptr,
+                                  nullptr, 0, S(stream)));
+}
+
+bq_status bq_mxfp4_dequantize(const uint8_t* packed, const uint8_t* e8m0, int64_t rows, int64_t k,
+                              void* y, bq_dtype y_dtype, void* stream) {
+    if (!is_half_or_f32(y_dtype)) return BQ_ERR_UNSUPPORTED;
+    if (rows < 0 || k < 0 || k % 32 != 0) return BQ_ERR_INVALID_ARG;
+    if (rows * k == 0) return BQ_OK;
+    if (!packed || !e8m0 || !y) return BQ_ERR_INVALID_ARG;
+    if (!aligned(y, esize(y_dtype))) return BQ_ERR_MISALIGNED;
+    return from_cuda(bq::mx_dequant(to_dt(y_dtype), bq::MX_MXFP4, packed, e8m0, nullptr, rows, k, y,
+                                    S(stream)));
+}
+
 // ---- FP8 blocks
 bq_status bq_fp8_block_quantize(const void* x, bq_dtype x_dtype, int64_t rows, int64_t cols,
                                 int32_t block_rows, int32_t block_cols, uint8_t* e4m3,

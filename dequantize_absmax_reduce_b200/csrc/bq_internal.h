@@ -78,7 +78,7 @@ cudaError_t range_to_amax(const unsigned long long* rec, float* amax, cudaStream
 // range record that the range kernel just before on the stream writes (the
 // quantizer is launched to overlap it); 1 = *global_scale as given; 2 = from
 // a range record the caller supplies (ordinary launch).
-enum MxFmt { MX_FP8_1x128 = 0, MX_MXFP8 = 1, MX_NVFP4 = 2 };
+enum MxFmt { MX_FP8_1x128 = 0, MX_MXFP8 = 1, MX_NVFP4 = 2, MX_MXFP4 = 3 };
 cudaError_t mx_quant(DT dt, int fmt, const void* x, int64_t rows, int64_t k, uint8_t* codes,
                      void* scales, const unsigned long long* amax_rec, float* global_scale,
                      int static_global, cudaStream_t st);

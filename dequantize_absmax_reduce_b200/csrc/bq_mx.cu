@@ -45,7 +45,7 @@ __global__ void __launch_bounds__(256) k_mx_quant(MxArgs a) {
     constexpr int VEC = S::VEC, NV = S::NV, TEAM = S::TEAM, SEGS = S::SEGS;
     constexpr int G = MxG<FMT>::G;
     constexpr int TPW = 32 / TEAM;
-    constexpr int CB = (FMT == MX_NVFP4) ? VEC / 2 : VEC;   // code bytes per vector
+    constexpr int CB = (FMT == MX_NVFP4 || FMT == MX_MXFP4) ? VEC / 2 : VEC;   // code bytes per vector
     const T* __restrict__ x = (const T*)a.x;
     const int lane = threadIdx.x & 31;
     const int tm = lane / TEAM, l = lane % TEAM;
@@ -107,8 +107,8 @@ __global__ void __launch_bounds__(256) k_mx_quant(MxArgs a) {
                         else mx_emit<T, FMT, false>(v[j], R, 0.f, false, base + (j * TEAM + l) * CB);
                     }
                 }
-            } else if constexpr (FMT == MX_MXFP8) {
-                const int E = mx_exponent(am);
+            } else if constexpr (FMT == MX_MXFP8 || FMT == MX_MXFP4) {
+                const int E = mx_exponent(am, FMT == MX_MXFP4 ? 2 : 8);
                 if (ok && l == 0) ((uint8_t*)a.scales)[seg] = (uint8_t)(E + 127);
                 const Recip R{};
                 const float mul = exp2i(-E);
@@ -172,6 +172,17 @@ __global__ void __launch_bounds__(256) k_mx_quant_scalar(MxArgs a) {
                                           with_quotient_sign(div_any(v1, R), v1, s));
                 a.codes[seg * G + i] = (uint8_t)w;
                 a.codes[seg * G + i + 1] = (uint8_t)(w >> 8);
+            }
+        } else if constexpr (FMT == MX_MXFP4) {
+            const int E = mx_exponent(am, 2);
+            ((uint8_t*)a.scales)[seg] = (uint8_t)(E + 127);
+            const float inv = exp2i(-E);
+            for (int i = 0; i < G; i += 8) {
+                float t[8];
+                for (int j = 0; j < 8; ++j) t[j] = __fmul_rn(ld1<T>(p + i + j), inv);
+                const uint32_t w = e2m1x8(t);
+                uint8_t* d = a.codes + (seg * G + i) / 2;
+                d[0] = (uint8_t)w; d[1] = (uint8_t)(w >> 8); d[2] = (uint8_t)(w >> 16); d[3] = (uint8_t)(w >> 24);
             }
         } else if constexpr (FMT == MX_MXFP8) {
             const int E = mx_exponent(am);
@@ -287,7 +298,7 @@ __device__ __forceinline__ float mx_group_mul(const DeqArgs& a, int64_t r, int64
     if constexpr (FMT == MX_NVFP4) {
         const uint32_t sb = __ldg(((const uint8_t*)a.scales) + r * (a.k / 16) + c / 16);
         return __fmul_rn(e4m3_to_f32(sb), s2);
-    } else if constexpr (FMT == MX_MXFP8) {
+    } else if constexpr (FMT == MX_MXFP8 || FMT == MX_MXFP4) {
         const uint32_t b = __ldg(((const uint8_t*)a.scales) + r * (a.k / 32) + c / 32);
         return (b == 0xFFu) ? __uint_as_float(0x7FC00000u) : exp2i((int)b - 127);
     } else {
@@ -308,7 +319,7 @@ __global__ void __launch_bounds__(256) k_mx_deq(DeqArgs a) {
         const int64_t c = e0 - r * a.k;
         const float mul = mx_group_mul<FMT>(a, r, c, s2);
         float o[W];
-        if constexpr (FMT == MX_NVFP4) {
+        if constexpr (FMT == MX_NVFP4 || FMT == MX_MXFP4) {
             if constexpr (VECP) {
                 const uint2 w = __ldg(reinterpret_cast<const uint2*>(a.codes + e0 / 2));
                 const uint32_t ws[2] = {w.x, w.y};
@@ -437,9 +448,9 @@ __global__ void __launch_bounds__(256) k_mx_deq8(DeqArgs a) {
         for (int u = 0; u < DQ_U; ++u) {
             const int64_t it = base + u * stride;
             if (it < n_items) {
-                if constexpr (FMT == MX_NVFP4) {
+                if constexpr (FMT == MX_NVFP4 || FMT == MX_MXFP4) {
                     w[u].x = __ldg(reinterpret_cast<const uint32_t*>(a.codes) + it);
-                    sb[u] = __ldg((const uint8_t*)a.scales + (it >> 1));
+                    sb[u] = __ldg((const uint8_t*)a.scales + (FMT == MX_NVFP4 ? (it >> 1) : (it >> 2)));
                 } else {
                     w[u] = __ldg(reinterpret_cast<const uint2*>(a.codes) + it);
                     if constexpr (FMT == MX_MXFP8) {
@@ -457,6 +468,8 @@ __global__ void __launch_bounds__(256) k_mx_deq8(DeqArgs a) {
             float o[8];
             if constexpr (FMT == MX_NVFP4) {
                 e2m1x8_mul(w[u].x, f2_bcast(__fmul_rn(e4m3_to_f32(sb[u]), s2)), o);
+            } else if constexpr (FMT == MX_MXFP4) {
+                e2m1x8_mul(w[u].x, f2_bcast(e8m0_mul(sb[u])), o);
             } else {
                 e4m3x8_mul(w[u].x, w[u].y, f2_bcast(FMT == MX_MXFP8 ? e8m0_mul(sb[u]) : fs[u]), o);
             }
@@ -595,7 +608,7 @@ static cudaError_t launch_mx_quant_f(DT dt, const MxArgs& a, bool vec, cudaStrea
 cudaError_t mx_quant(DT dt, int fmt, const void* x, int64_t rows, int64_t k, uint8_t* codes,
                      void* scales, const unsigned long long* amax_rec, float* global_scale,
                      int static_global, cudaStream_t st) {
-    const int G = fmt == MX_FP8_1x128 ? 128 : (fmt == MX_MXFP8 ? 32 : 16);
+    const int G = fmt == MX_FP8_1x128 ? 128 : (fmt == MX_NVFP4 ? 16 : 32);
     MxArgs a;
     a.x = x; a.n_seg = rows * (k / G); a.codes = codes; a.scales = scales;
     a.amax_rec = amax_rec; a.global_scale = global_scale; a.static_global = static_global;
@@ -604,12 +617,13 @@ cudaError_t mx_quant(DT dt, int fmt, const void* x, int64_t rows, int64_t k, uin
                                          static_global, st);
     if (pe != cudaErrorNotSupported) return pe;
     const int VEC = dt == DT::F32 ? 4 : 8;
-    const int cb = (fmt == MX_NVFP4) ? VEC / 2 : VEC;
+    const int cb = (fmt == MX_NVFP4 || fmt == MX_MXFP4) ? VEC / 2 : VEC;
     const bool vec = al(x, 16) && al(codes, cb);
     switch (fmt) {
         case MX_FP8_1x128: return launch_mx_quant_f<MX_FP8_1x128>(dt, a, vec, st);
         case MX_MXFP8: return launch_mx_quant_f<MX_MXFP8>(dt, a, vec, st);
         case MX_NVFP4: return launch_mx_quant_f<MX_NVFP4>(dt, a, vec, st);
+        case MX_MXFP4: return launch_mx_quant_f<MX_MXFP4>(dt, a, vec, st);
     }
     return cudaErrorInvalidValue;
 }
@@ -650,7 +664,7 @@ cudaError_t fp8_tile_quant(DT dt, const void* x, int64_t rows, int64_t cols, int
 
 template <class T, int FMT>
 static cudaError_t launch_deq_t(const DeqArgs& a, cudaStream_t st) {
-    const int cb = (FMT == MX_NVFP4) ? 4 : 8;      // code bytes per 8 elements
+    const int cb = (FMT == MX_NVFP4 || FMT == MX_MXFP4) ? 4 : 8;      // code bytes per 8 elements
     const bool vec = (a.k % 8 == 0) && al(a.y, 16) && al(a.codes, cb);
     if (vec) {
         const int64_t blocks = (a.numel / 8 + 256 * DQ_U - 1) / (256 * DQ_U);
@@ -703,6 +717,7 @@ cudaError_t mx_dequant(DT ydt, int fmt, const uint8_t* codes, const void* scales
     if (a.numel == 0) return cudaSuccess;
     if (fmt == MX_NVFP4) return launch_deq_f<MX_NVFP4>(ydt, a, st);
     if (fmt == MX_MXFP8) return launch_deq_f<MX_MXFP8>(ydt, a, st);
+    if (fmt == MX_MXFP4) return launch_deq_f<MX_MXFP4>(ydt, a, st);
     return cudaErrorInvalidValue;
 }
 

@@ -68,9 +68,9 @@ cudaError_t int_dyn_pipe(DT dt, int op, const void* x, SegView sv, IntCfg cfg, v
 cudaError_t mx_quant_pipe(DT dt, int fmt, const void* x, int64_t rows, int64_t k, uint8_t* codes,
                           void* scales, const unsigned long long* amax_rec, float* global_scale,
                           int static_global, cudaStream_t st) {
-    const int G = fmt == MX_FP8_1x128 ? 128 : (fmt == MX_MXFP8 ? 32 : 16);
+    const int G = fmt == MX_FP8_1x128 ? 128 : (fmt == MX_NVFP4 ? 16 : 32);
     const int VEC = (dt == DT::F32) ? 4 : 8;
-    const int cb = (fmt == MX_NVFP4) ? VEC / 2 : VEC;
+    const int cb = (fmt == MX_NVFP4 || fmt == MX_MXFP4) ? VEC / 2 : VEC;
     if (dt == DT::F64 || !al16(x) || ((uintptr_t)codes % cb) != 0) return cudaErrorNotSupported;
     PipeArgs a{};
     a.x = x; a.n_seg = rows * (k / G); a.G = G;
@@ -78,7 +78,8 @@ cudaError_t mx_quant_pipe(DT dt, int fmt, const void* x, int64_t rows, int64_t k
     a.amax_rec = amax_rec; a.global_scale = global_scale; a.static_global = static_global;
     if (fmt == MX_FP8_1x128) a.scale = (float*)scales; else a.zp = (uint8_t*)scales;
     if (a.n_seg == 0) return cudaSuccess;
-    const int pk = fmt == MX_FP8_1x128 ? PK_FP8 : (fmt == MX_MXFP8 ? PK_MX : PK_NV);
+    const int pk = fmt == MX_FP8_1x128 ? PK_FP8
+                 : (fmt == MX_MXFP8 ? PK_MX : (fmt == MX_MXFP4 ? PK_MX4 : PK_NV));
     return pipe_launch(dt, pk, true, a, st);
 }
 

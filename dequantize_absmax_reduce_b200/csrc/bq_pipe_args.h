@@ -8,7 +8,7 @@
 
 namespace bq {
 
-enum PipeKind { PK_INT_Q = 0, PK_INT_FAKE = 1, PK_FP8 = 2, PK_MX = 3, PK_NV = 4 };
+enum PipeKind { PK_INT_Q = 0, PK_INT_FAKE = 1, PK_FP8 = 2, PK_MX = 3, PK_NV = 4, PK_MX4 = 5 };
 
 struct PipeArgs {
     const void* x;

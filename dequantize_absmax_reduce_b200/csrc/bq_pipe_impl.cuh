@@ -497,8 +497,9 @@ __global__ void __launch_bounds__(NT) k_seg_pipe(PipeArgs a) {
                 }
             }
         } else {
-            constexpr int FMT = (PK == PK_FP8) ? MX_FP8_1x128 : (PK == PK_MX ? MX_MXFP8 : MX_NVFP4);
-            constexpr int CB = (PK == PK_NV) ? VEC / 2 : VEC;     // code bytes per vector
+            constexpr int FMT = (PK == PK_FP8) ? MX_FP8_1x128
+                              : (PK == PK_MX ? MX_MXFP8 : (PK == PK_MX4 ? MX_MXFP4 : MX_NVFP4));
+            constexpr int CB = (PK == PK_NV || PK == PK_MX4) ? VEC / 2 : VEC;     // code bytes per vector
             uint8_t* base = a.q + seg * (G / VEC) * CB + lane * CB;
             auto coff = [&](int j) { return vidx(j) * TEAM * CB; };
             if constexpr (PK == PK_FP8) {
@@ -525,6 +526,18 @@ __global__ void __launch_bounds__(NT) k_seg_pipe(PipeArgs a) {
                         if (R.fast) mx_emit<T, FMT, true>(v, R, 0.f, false, base + coff(j));
                         else mx_emit<T, FMT, false>(v, R, 0.f, false, base + coff(j));
                     }
+                }
+            } else if constexpr (PK == PK_MX4) {
+                const int E = mx_exponent(hi, 2);
+                if (seg_ok && lane == 0) a.zp[seg] = (uint8_t)(E + 127);
+                const F2 mul2 = f2_bcast(exp2i(-E));
+                if (full) {
+#pragma unroll
+                    for (int j = 0; j < NV; ++j) emit_mx4_fast<T>(raw[j], mul2, base + coff(j));
+                } else if (seg_ok) {
+#pragma unroll
+                    for (int j = 0; j < NV; ++j)
+                        if (vok(j)) emit_mx4_fast<T>(raw[j], mul2, base + coff(j));
                 }
             } else if constexpr (PK == PK_MX) {
                 const int E = mx_exponent(hi);
@@ -1452,6 +1465,7 @@ static cudaError_t pipe_dt(int pk, bool sym, const PipeArgs& a, cudaStream_t st)
         case PK_INT_FAKE: return sym ? launch_pipe_u<T, PK_INT_FAKE, true>(a, st) : launch_pipe_u<T, PK_INT_FAKE, false>(a, st);
         case PK_FP8: return launch_pipe_u<T, PK_FP8, true>(a, st);
         case PK_MX: return launch_pipe_u<T, PK_MX, true>(a, st);
+        case PK_MX4: return launch_pipe_u<T, PK_MX4, true>(a, st);
         case PK_NV:
             if constexpr (sizeof(T) == 2) {
                 if (((uintptr_t)a.q & 7u) == 0) return launch_nv_t<T>(a, st);

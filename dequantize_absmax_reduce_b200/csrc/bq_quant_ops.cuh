@@ -69,16 +69,18 @@ template <int FMT> struct MxG;
 template <> struct MxG<MX_FP8_1x128> { static constexpr int G = 128; };
 template <> struct MxG<MX_MXFP8> { static constexpr int G = 32; };
 template <> struct MxG<MX_NVFP4> { static constexpr int G = 16; };
+template <> struct MxG<MX_MXFP4> { static constexpr int G = 32; };
 
 
 __device__ __forceinline__ void st2(void* p, uint32_t a) {
     asm volatile("st.global.u16 [%0], %1;" :: "l"(p), "h"((uint16_t)a) : "memory");
 }
 
-// MXFP8 shared exponent: E = clamp(floor(log2 a) - 8, -127, 127), from the
-// bits of a >= 0 (a subnormal a counts its leading zeros; infinity is 2^128;
-// a = 0 gives -127).
-__device__ __forceinline__ int mx_exponent(float a) {
+// MX shared exponent: E = clamp(floor(log2 a) - emax, -127, 127), emax the
+// largest exponent of the element format (8 for E4M3 / MXFP8, 2 for E2M1 /
+// MXFP4), from the bits of a >= 0 (a subnormal a counts its leading zeros;
+// infinity is 2^128; a = 0 gives -127).
+__device__ __forceinline__ int mx_exponent(float a, int emax = 8) {
     const uint32_t b = __float_as_uint(a);
     const int ex = (int)(b >> 23);
     int fl2;
@@ -90,7 +92,7 @@ __device__ __forceinline__ int mx_exponent(float a) {
     } else {
         fl2 = ex - 127;
     }
-    return min(max(fl2 - 8, -127), 127);
+    return min(max(fl2 - emax, -127), 127);
 }
 
 
@@ -102,14 +104,14 @@ __device__ __forceinline__ void mx_emit(const float* v, const Recip& R, float mu
     float t[VEC];
 #pragma unroll
     for (int i = 0; i < VEC; ++i) {
-        if constexpr (FMT == MX_MXFP8) {
+        if constexpr (FMT == MX_MXFP8 || FMT == MX_MXFP4) {
             t[i] = __fmul_rn(v[i], mul);
         } else {
             const float d = FAST ? div_chain(v[i], R) : div_any(v[i], R);
             t[i] = with_quotient_sign(d, v[i], R.s);
         }
     }
-    if constexpr (FMT == MX_NVFP4) {
+    if constexpr (FMT == MX_NVFP4 || FMT == MX_MXFP4) {
         if constexpr (VEC == 8) {
             const float (&t8)[8] = *reinterpret_cast<const float(*)[8]>(t);
             st4(dst, zero ? 0u : e2m1x8(t8));
@@ -241,6 +243,25 @@ __device__ __forceinline__ void emit_mx_fast(const U4& raw, F2 mul2, uint8_t* ds
         st8(dst, e4m3x4(t[0], t[1], t[2], t[3]), e4m3x4(t[4], t[5], t[6], t[7]));
     } else {
         st4(dst, e4m3x4(t[0], t[1], t[2], t[3]));
+    }
+}
+
+// MXFP4 codes E2M1(fl(x * 2^-E)): a product (exact, sign kept for zeros and
+// underflows), so like MXFP8 it needs no guard.
+template <class T>
+__device__ __forceinline__ void emit_mx4_fast(const U4& raw, F2 mul2, uint8_t* dst) {
+    constexpr int VEC = Traits<T>::VEC;
+    constexpr int NP = VEC / 2;
+    F2 x[NP];
+    widen_pairs<T>(raw, x);
+    float t[8];
+#pragma unroll
+    for (int p = 0; p < NP; ++p) f2_split(f2_mul(x[p], mul2), t[2 * p], t[2 * p + 1]);
+    if constexpr (VEC == 8) {
+        st4(dst, e2m1x8(t));
+    } else {
+        t[4] = t[5] = t[6] = t[7] = 0.0f;
+        st2(dst, e2m1x8(t) & 0xFFFFu);
     }
 }
 

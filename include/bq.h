@@ -306,6 +306,21 @@ bq_status bq_mxfp8_quantize(const void* x, bq_dtype x_dtype, int64_t rows, int64
 bq_status bq_mxfp8_dequantize(const uint8_t* e4m3, const uint8_t* e8m0, int64_t rows, int64_t k,
                               void* y, bq_dtype y_dtype, void* stream);
 
+/* [QuantizedWeight] native MXFP4 ("E8M0 for native MXFP4"; OCP MX rule, as for
+ * MXFP8): x [rows, k] (F32, F16 or BF16), k % 32 == 0 -> packed E2M1 codes u8
+ * [rows, k/2] (element 2j in the low nibble of byte j) and one E8M0 scale u8
+ * [rows, k/32] per 32 consecutive elements along k:
+ * E = clamp(floor(log2 amax) - 2, -127, 127) (2 = the largest E2M1 exponent;
+ * amax ignores NaN, an infinite amax counts as 2^128, amax = 0 gives -127),
+ * byte = E + 127, code = E2M1(fl(x * 2^-E)) rounded to nearest even,
+ * saturating to +-6, sign kept, NaN -> 0x7. */
+bq_status bq_mxfp4_quantize(const void* x, bq_dtype x_dtype, int64_t rows, int64_t k,
+                            uint8_t* packed, uint8_t* e8m0, void* stream);
+
+/* y = RN_y(fl(E2M1(code) * 2^(byte - 127))) (NaN for byte 0xFF). */
+bq_status bq_mxfp4_dequantize(const uint8_t* packed, const uint8_t* e8m0, int64_t rows, int64_t k,
+                              void* y, bq_dtype y_dtype, void* stream);
+
 /* ------------------------------------------------------------ FP8 blocks */
 /* [smile.llm.quant] Fp8BlockGemm (activations, 1x128 groups) and
  * Fp8BlockDequant (weights, 128x128 tiles, weight_scale_inv): x [rows, cols]

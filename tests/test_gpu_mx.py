@@ -247,3 +247,64 @@ def test_workload_fp8_blocks(bq, orc, name):
         re, rs = orc.fp8_block_quantize(cpu(wt[r0:r0 + 128]), 128, 128)
         assert_bitwise(cpu(e)[r0:r0 + 128], re, f"w e4m3 band {band}")
         assert_bitwise(cpu(s)[band], rs[0], f"w scales band {band}")
+
+
+# ---------------------------------------------------------------- MXFP4
+@pytest.mark.parametrize("dtype", ["bf16", "f16", "f32"])
+@pytest.mark.parametrize("shape", [(1, 32), (5, 96), (40, 7168)])
+def test_mxfp4_parity(bq, orc, dtype, shape):
+    for dist in ("normal", "student_t3"):
+        x = synthetic.Stream(31).tensor(shape, dtype, dist=dist, outlier_p=0.01, outlier_factor=40)
+        p, s = bq.mxfp4_quantize(x.cuda())
+        rp, rs = orc.mxfp4_quantize(x)
+        assert_bitwise(p, rp, "packed")
+        assert_bitwise(s, rs, "e8m0")
+        for ydt in ("bf16", "f32", "f16"):
+            y = bq.mxfp4_dequantize(p, s, DT[ydt])
+            assert_bitwise(y, orc.mxfp4_dequantize(rp, rs, *shape, ydtype=ydt), f"deq {ydt}")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_mxfp4_all_16bit_patterns_and_unaligned(bq, orc, dtype):
+    x = synthetic.bits_tensor(dtype).reshape(512, 128)
+    p, s = bq.mxfp4_quantize(x.cuda())
+    rp, rs = orc.mxfp4_quantize(x)
+    assert_bitwise(p, rp, "packed")
+    assert_bitwise(s, rs, "e8m0")
+    # an input not 16-byte aligned takes the register kernel
+    buf = torch.zeros(x.numel() + 1, dtype=x.dtype, device="cuda")
+    xg = buf[1:].view(x.shape)
+    xg.copy_(x.cuda())
+    p, s = bq.mxfp4_quantize(xg)
+    assert_bitwise(p, rp, "packed (unaligned x)")
+    assert_bitwise(s, rs, "e8m0 (unaligned x)")
+    # unaligned codes: element-wise dequantize
+    pb = torch.zeros(rp.numel() + 1, dtype=torch.uint8, device="cuda")
+    pk = pb[1:].view(rp.shape)
+    pk.copy_(rp.cuda())
+    y = bq.mxfp4_dequantize(pk, rs.cuda(), torch.float32)
+    assert_bitwise(y, orc.mxfp4_dequantize(rp, rs, 512, 128, ydtype="f32"), "deq (unaligned codes)")
+
+
+def test_mxfp4_special_values(bq, orc):
+    vals = [0.0, -0.0, 1e-30, -1e-30, 6.0, -6.0, 5.0, 2.5, 0.25, 0.75, 1e30, -1e30,
+            float("inf"), float("-inf"), float("nan"), -float("nan")]
+    x = torch.tensor(vals * 6, dtype=torch.float32).reshape(3, 32)
+    x[1] = torch.linspace(-7, 7, 32)
+    x[2] = 0.0
+    p, s = bq.mxfp4_quantize(x.cuda())
+    rp, rs = orc.mxfp4_quantize(x)
+    assert_bitwise(p, rp, "packed")
+    assert_bitwise(s, rs, "e8m0")
+
+
+def test_workload_mxfp4(bq, orc):
+    xg = synthetic.make_workload_device("nvfp4_bf16_4096x7168")["x"]
+    p, s = bq.mxfp4_quantize(xg)
+    rows = sample_rows(4096, 16, seed=5)
+    xs = cpu(xg[rows.cuda()])
+    rp, rs = orc.mxfp4_quantize(xs)
+    assert_bitwise(cpu(p)[rows], rp, "packed")
+    assert_bitwise(cpu(s)[rows], rs, "e8m0")
+    y = bq.mxfp4_dequantize(p, s, torch.bfloat16)
+    assert_bitwise(cpu(y)[rows], orc.mxfp4_dequantize(rp, rs, len(rows), 7168, "bf16"), "deq")
