@@ -43,7 +43,8 @@ def lib() -> C.CDLL:
                      "or_mxfp8_quantize", "or_mxfp8_dequantize", "or_fp8_block_quantize",
                      "or_fp8_block_dequantize", "or_packed_transpose",
                      "or_packed_transpose_concat", "or_nvfp4_concat_rows",
-                     "or_nvfp4_predequant_fp8", "or_mxfp4_quantize", "or_mxfp4_dequantize"):
+                     "or_nvfp4_predequant_fp8", "or_mxfp4_quantize", "or_mxfp4_dequantize",
+                     "or_fp8_tensor_quantize", "or_fp8_tensor_dequantize"):
             getattr(_lib, name).restype = C.c_int
         _lib.or_align_up.restype = C.c_int64
         _lib.or_align_up.argtypes = [C.c_int64, C.c_int64]
@@ -378,4 +379,22 @@ def mxfp4_dequantize(p, s, rows: int, k: int, ydtype: str = "bf16"):
     y = torch.zeros((rows, k), dtype=_TORCH[ydtype])
     _ok(lib().or_mxfp4_dequantize(_p(_c(p)), _p(_c(s)), C.c_int64(rows), C.c_int64(k), _p(y),
                                   C.c_int(_T[ydtype])), "mxfp4_dequantize")
+    return y
+
+
+def fp8_tensor_quantize(x: torch.Tensor, scale: float | None = None):
+    """FP8 per-tensor store: x (any shape) -> (E4M3 codes u8 of x's shape, scale)."""
+    x = _c(x)
+    e = torch.zeros(x.shape, dtype=torch.uint8)
+    sc = C.c_float(0.0 if scale is None else scale)
+    _ok(lib().or_fp8_tensor_quantize(_p(x), C.c_int(_dt(x)), C.c_int64(x.numel()), _p(e), C.byref(sc),
+                                     C.c_int(int(scale is not None))), "fp8_tensor_quantize")
+    return e, sc.value
+
+
+def fp8_tensor_dequantize(e: torch.Tensor, scale: float, ydtype: str = "bf16"):
+    e = _c(e)
+    y = torch.zeros(e.shape, dtype=_TORCH[ydtype])
+    _ok(lib().or_fp8_tensor_dequantize(_p(e), C.c_float(scale), C.c_int64(e.numel()), _p(y),
+                                       C.c_int(_T[ydtype])), "fp8_tensor_dequantize")
     return y

@@ -23,7 +23,8 @@
 //   [smile.llm.quant] package summary — Fp8BlockGemm / Fp8BlockDequant
 //               (E4M3, f32 scale per 1x128 activation group and per 128x128
 //               weight tile, weight_scale_inv) and MxFp8 (E4M3, E8M0 scale per
-//               32 consecutive elements along the reduction dimension).
+//               32 consecutive elements along the reduction dimension) and
+//               Fp8KvCodec (FP8 KV store / load with per-tensor scales).
 //
 // Precision. The pages fix no precision. Every result of this path ends in a
 // discrete encoding (an integer code, an FP8/FP4 code, a bf16/f16/f32 value),
@@ -737,6 +738,35 @@ int or_fp8_block_dequantize(const uint8_t* e4m3, const float* scale, int64_t row
         for (int64_t c = 0; c < cols; ++c)
             store_f(y, y_t, r * cols + c,
                     r32(dec_e4m3(e4m3[r * cols + c]) * (double)scale[(r / br) * nbc + c / bc]));
+    return 0;
+}
+
+// ---- FP8 per-tensor codec [smile.llm.quant Fp8KvCodec: FP8 KV store / load
+// with per-tensor scales]: one f32 scale for the whole tensor, the dequantize
+// multiplier as in the FP8 block formats: s = fl(amax / 448) (0 -> 1, amax
+// ignores NaN) or given; e = E4M3(fl(x / s)); load y = RN_y(fl(dec(e) * s)).
+int or_fp8_tensor_quantize(const void* x, int x_t, int64_t n, uint8_t* e4m3, float* s_io,
+                           int static_s) {
+    if (x_t != OR_F32 && x_t != OR_F16 && x_t != OR_BF16) return 1;
+    if (n < 0) return 1;
+    float s;
+    if (static_s) {
+        s = *s_io;
+    } else {
+        double a;
+        or_tensor_amax(x, x_t, n, &a);
+        s = (float)(a / 448.0);
+        if (s == 0.0f) s = 1.0f;
+        *s_io = s;
+    }
+    for (int64_t i = 0; i < n; ++i) e4m3[i] = enc_e4m3(r32(load_f(x, x_t, i) / (double)s));
+    return 0;
+}
+
+int or_fp8_tensor_dequantize(const uint8_t* e4m3, float s, int64_t n, void* y, int y_t) {
+    if (y_t != OR_F32 && y_t != OR_F16 && y_t != OR_BF16) return 1;
+    if (n < 0) return 1;
+    for (int64_t i = 0; i < n; ++i) store_f(y, y_t, i, r32(dec_e4m3(e4m3[i]) * (double)s));
     return 0;
 }
 

@@ -224,3 +224,35 @@ def test_mxfp4_special_blocks(orc):
     codes = _unpack(p)[0]
     assert codes[32] == 0x8 and codes[33] == 0x6
     assert codes[64] == 0x7                 # inf * 2^-126 saturates to 6
+
+
+# ---------------------------------------------------------------- FP8 per-tensor (KV codec)
+def test_fp8_tensor_codec_scale_and_codes(orc):
+    x = synthetic.Stream(25).tensor((4, 8, 96), "bf16", dist="student_t3")
+    e, s = orc.fp8_tensor_quantize(x)
+    amax = float(np.abs(x.double().numpy()).max())
+    assert s == float(np.float32(amax / 448.0))
+    # the amax element lands on 448 (or within one rounding of it)
+    top = orc.decode("e4m3", e.numpy().reshape(-1))
+    assert 416.0 <= np.abs(top).max() <= 448.0
+    # power-of-two static scale: x / s is exact, so the codes are torch's cast
+    e2, s2 = orc.fp8_tensor_quantize(x, scale=0.125)
+    assert s2 == 0.125
+    t = (x.float() / 0.125)
+    inr = t.abs() <= 448
+    ref = t.clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+    assert torch.equal(e2[inr], ref[inr])
+    assert torch.all(e2[~inr] == torch.where(t[~inr] > 0, 0x7E, 0xFE).to(torch.uint8))
+    # load: exact products for a power-of-two scale
+    y = orc.fp8_tensor_dequantize(e2, 0.125, ydtype="f32")
+    assert torch.equal(y, e2.view(torch.float8_e4m3fn).float() * 0.125)
+
+
+def test_fp8_tensor_codec_is_one_block(orc):
+    x = synthetic.Stream(26).tensor((37, 200), "f16")
+    e, s = orc.fp8_tensor_quantize(x)
+    eb, sb = orc.fp8_block_quantize(x, 37, 200)        # one block covering the tensor
+    assert torch.equal(e, eb) and s == sb.item()
+    z = torch.zeros(5, 7)
+    ez, sz = orc.fp8_tensor_quantize(z)
+    assert sz == 1.0 and torch.all(ez == 0)
