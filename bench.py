@@ -259,6 +259,21 @@ def per_granularity(B, api, torch, device, peak, reps=5):
     timed(wl, "quantize_per_tensor_backward",
           lambda: B.bq_quantize_per_tensor_backward(x, dy, s, None, d, dx), 12 * n + 4, 1)
 
+    # FP8 per-tensor codec (KV store / load) of the per-token bf16 [8192, 4096] tensor
+    wl = "per_token_bf16_8192x4096"
+    x = synthetic.make_workload_device(wl, device=device)["x"]
+    n = x.numel()
+    e = torch.empty(x.shape, dtype=torch.uint8, device=device)
+    s = torch.empty(1, dtype=torch.float32, device=device)
+    ws = torch.empty(2, dtype=torch.int64, device=device)
+    y = torch.empty_like(x)
+    timed(wl, "fp8_tensor_quantize(KV store, dynamic: amax + codes)",
+          lambda: B.bq_fp8_tensor_quantize(x, e, s, False, ws), 2 * n + 2 * n + n, 3)
+    timed(wl, "fp8_tensor_quantize(KV store, static scale)",
+          lambda: B.bq_fp8_tensor_quantize(x, e, s, True, None), 2 * n + n, 1)
+    timed(wl, "fp8_tensor_dequantize(KV load)", lambda: B.bq_fp8_tensor_dequantize(e, s, y), n + 2 * n, 1)
+    del x, e, y
+
     # per-group 128 asymmetric u8 and per-channel s8, f16 [11008, 4096]
     wl = "per_group128_f16_11008x4096"
     w = synthetic.make_workload_device(wl, device=device)

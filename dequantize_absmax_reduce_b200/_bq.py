@@ -83,6 +83,8 @@ _SIGS = {
     "bq_mxfp8_quantize": [_P, C.c_int, _I64, _I64, _P, _P, _P],
     "bq_mxfp8_dequantize": [_P, _P, _I64, _I64, _P, C.c_int, _P],
     "bq_mxfp4_quantize": [_P, C.c_int, _I64, _I64, _P, _P, _P],
+    "bq_fp8_tensor_quantize": [_P, C.c_int, _I64, _P, _P, _I32, _P, _SZ, _P],
+    "bq_fp8_tensor_dequantize": [_P, _P, _I64, _P, C.c_int, _P],
     "bq_mxfp4_dequantize": [_P, _P, _I64, _I64, _P, C.c_int, _P],
     "bq_fp8_block_quantize": [_P, C.c_int, _I64, _I64, _I32, _I32, _P, _P, _P],
     "bq_fp8_block_dequantize": [_P, _P, _I64, _I64, _I32, _I32, _P, C.c_int, _P],
@@ -411,3 +413,14 @@ def bq_mxfp4_dequantize(packed, e8m0, y, stream=None):
     rows, k = y.shape
     _check(lib.bq_mxfp4_dequantize(_ptr(packed), _ptr(e8m0), rows, k, _ptr(y), DTYPE[y.dtype],
                                    _stream(stream)), "bq_mxfp4_dequantize")
+
+
+def bq_fp8_tensor_quantize(x, e4m3, scale, static_scale=False, ws=None, stream=None):
+    _check(lib.bq_fp8_tensor_quantize(_ptr(x), DTYPE[x.dtype], x.numel(), _ptr(e4m3), _ptr(scale),
+                                      int(bool(static_scale)), _ptr(ws), _nbytes(ws), _stream(stream)),
+           "bq_fp8_tensor_quantize")
+
+
+def bq_fp8_tensor_dequantize(e4m3, scale, y, stream=None):
+    _check(lib.bq_fp8_tensor_dequantize(_ptr(e4m3), _ptr(scale), y.numel(), _ptr(y), DTYPE[y.dtype],
+                                        _stream(stream)), "bq_fp8_tensor_dequantize")

@@ -268,3 +268,24 @@ def mxfp4_dequantize(p, s, ydtype=torch.bfloat16, stream=None):
     y = torch.empty((rows, k), dtype=ydtype, device=p.device)
     B.bq_mxfp4_dequantize(p, s, y, stream)
     return y
+
+
+def fp8_tensor_quantize(x, scale=None, stream=None):
+    """FP8 per-tensor store (KV codec): x (any shape) -> (E4M3 codes u8 of x's
+    shape, scale f32 [1]); scale given (static) or amax / 448 (dynamic)."""
+    e = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if scale is None:
+        sc = torch.empty(1, dtype=torch.float32, device=x.device)
+        ws = torch.empty(2, dtype=torch.int64, device=x.device)
+        B.bq_fp8_tensor_quantize(x, e, sc, False, ws, stream)
+    else:
+        sc = scale if isinstance(scale, torch.Tensor) else torch.tensor([float(scale)], device=x.device)
+        B.bq_fp8_tensor_quantize(x, e, sc, True, None, stream)
+    return e, sc
+
+
+def fp8_tensor_dequantize(e, scale, ydtype=torch.bfloat16, stream=None):
+    y = torch.empty(e.shape, dtype=ydtype, device=e.device)
+    sc = scale if isinstance(scale, torch.Tensor) else torch.tensor([float(scale)], device=e.device)
+    B.bq_fp8_tensor_dequantize(e, sc, y, stream)
+    return y

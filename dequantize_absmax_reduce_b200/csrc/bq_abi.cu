@@ -517,6 +517,38 @@ bq_status bq_mxfp4_dequantize(const uint8_t* packed, const uint8_t* e8m0, int64_
                                     S(stream)));
 }
 
+// ---- FP8 per-tensor codec
+bq_status bq_fp8_tensor_quantize(const void* x, bq_dtype x_dtype, int64_t n, uint8_t* e4m3,
+                                 float* scale, int32_t static_scale, void* ws, size_t ws_bytes,
+                                 void* stream) {
+    if (!is_half_or_f32(x_dtype)) return BQ_ERR_UNSUPPORTED;
+    if (n < 0 || !scale || (static_scale != 0 && static_scale != 1)) return BQ_ERR_INVALID_ARG;
+    if (static_scale == 0 && (!ws || ws_bytes < 16)) return BQ_ERR_INVALID_ARG;
+    if (n > 0 && (!x || !e4m3)) return BQ_ERR_INVALID_ARG;
+    if (!aligned(x, esize(x_dtype)) || !aligned(scale, 4) || (static_scale == 0 && !aligned(ws, 8)))
+        return BQ_ERR_MISALIGNED;
+    cudaStream_t s = S(stream);
+    const DT dt = to_dt(x_dtype);
+    unsigned long long* rec = (unsigned long long*)ws;
+    if (static_scale == 0) {
+        if (bq::clear_records(rec, 2, s) != cudaSuccess) return BQ_ERR_CUDA;
+        if (n == 0) return from_cuda(bq::set_f32(scale, 1.0f, s));       // zero range
+        if (bq::tensor_range(dt, x, n, true, rec, s) != cudaSuccess) return BQ_ERR_CUDA;
+    }
+    if (n == 0) return BQ_OK;
+    return from_cuda(bq::fp8_tensor_quant(dt, x, n, e4m3, scale, rec, static_scale == 0 ? 1 : 0, s));
+}
+
+bq_status bq_fp8_tensor_dequantize(const uint8_t* e4m3, const float* scale, int64_t n, void* y,
+                                   bq_dtype y_dtype, void* stream) {
+    if (!is_half_or_f32(y_dtype)) return BQ_ERR_UNSUPPORTED;
+    if (n < 0) return BQ_ERR_INVALID_ARG;
+    if (n == 0) return BQ_OK;
+    if (!e4m3 || !scale || !y) return BQ_ERR_INVALID_ARG;
+    if (!aligned(scale, 4) || !aligned(y, esize(y_dtype))) return BQ_ERR_MISALIGNED;
+    return from_cuda(bq::fp8_tensor_dequant(to_dt(y_dtype), e4m3, scale, n, y, S(stream)));
+}
+
 // ---- FP8 blocks
 bq_status bq_fp8_block_quantize(const void* x, bq_dtype x_dtype, int64_t rows, int64_t cols,
                                 int32_t block_rows, int32_t block_cols, uint8_t* e4m3,

@@ -94,6 +94,14 @@ cudaError_t fp8_tile_pipe(DT dt, const void* x, int64_t rows, int64_t cols, uint
 cudaError_t fp8_block_dequant(DT ydt, const uint8_t* e4m3, const float* scale, int64_t rows,
                               int64_t cols, int br, int bc, void* y, cudaStream_t st);
 
+// FP8 per-tensor store: e = E4M3(fl(x / s)); s = *scale (from_rec = 0) or
+// fl(amax / 448) from the range record rec written by the range kernel just
+// before on the stream (from_rec = 1; s is then written to *scale).
+cudaError_t fp8_tensor_quant(DT dt, const void* x, int64_t n, uint8_t* e4m3, float* scale,
+                             const unsigned long long* rec, int from_rec, cudaStream_t st);
+// FP8 per-tensor load: y = RN_y(fl(dec(e) * *scale)).
+cudaError_t fp8_tensor_dequant(DT ydt, const uint8_t* e4m3, const float* scale, int64_t n, void* y,
+                               cudaStream_t st);
 // NVFP4 [rows, k] -> E4M3 [rows, k] with the per-tensor scale applied.
 cudaError_t nvfp4_predequant_fp8(const uint8_t* codes, const uint8_t* scales, const float* global_scale,
                                  int64_t rows, int64_t k, uint8_t* out, cudaStream_t st);

@@ -416,7 +416,9 @@ __device__ __forceinline__ float e8m0_mul(uint32_t b) {
 // is e0 / 128. FD: the element count is below 2^32 (32-bit row division).
 template <int BR, bool FD>
 __device__ __forceinline__ int64_t fp8_block_index(const DeqArgs& a, int64_t it) {
-    if constexpr (BR == 0) {
+    if constexpr (BR < 0) {
+        return 0;                 // one scale for the whole tensor
+    } else if constexpr (BR == 0) {
         return it >> 4;
     } else if constexpr (FD) {
         const uint32_t e0 = (uint32_t)it * 8u;
@@ -669,7 +671,9 @@ static cudaError_t launch_deq_t(const DeqArgs& a, cudaStream_t st) {
     if (vec) {
         const int64_t blocks = (a.numel / 8 + 256 * DQ_U - 1) / (256 * DQ_U);
         if constexpr (FMT == MX_FP8_1x128) {
-            if (a.br == 1 && a.k % 128 == 0) {
+            if (a.br < 0) {
+                k_mx_deq8<T, FMT, -1, true><<<grid_occ_mx<k_mx_deq8<T, FMT, -1, true>>(blocks), 256, 0, st>>>(a);
+            } else if (a.br == 1 && a.k % 128 == 0) {
                 k_mx_deq8<T, FMT, 0, true><<<grid_occ_mx<k_mx_deq8<T, FMT, 0, true>>(blocks), 256, 0, st>>>(a);
             } else if (a.br == 1) {
                 if (a.use_fd) k_mx_deq8<T, FMT, 1, true><<<grid_occ_mx<k_mx_deq8<T, FMT, 1, true>>(blocks), 256, 0, st>>>(a);
@@ -725,6 +729,18 @@ cudaError_t fp8_block_dequant(DT ydt, const uint8_t* e4m3, const float* scale, i
                               int64_t cols, int br, int bc, void* y, cudaStream_t st) {
     DeqArgs a = make_deq(e4m3, scale, nullptr, rows, cols, y);
     a.br = br; a.bc = bc; a.nbc = (cols + bc - 1) / bc;
+    if (a.numel == 0) return cudaSuccess;
+    return launch_deq_f<MX_FP8_1x128>(ydt, a, st);
+}
+
+cudaError_t fp8_tensor_dequant(DT ydt, const uint8_t* e4m3, const float* scale, int64_t n, void* y,
+                               cudaStream_t st) {
+    // One row of n elements; a block of one row and n columns (the scalar
+    // path's index) or the single-scale index (the vector path).
+    DeqArgs a = make_deq(e4m3, scale, nullptr, 1, n, y);
+    a.br = (n % 8 == 0) ? -1 : 1;
+    a.bc = n > 0 ? n : 1;
+    a.nbc = 1;
     if (a.numel == 0) return cudaSuccess;
     return launch_deq_f<MX_FP8_1x128>(ydt, a, st);
 }

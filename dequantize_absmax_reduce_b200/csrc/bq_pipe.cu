@@ -22,6 +22,9 @@ cudaError_t pipe_range_bf16(const void* x, int64_t n, bool sym, unsigned long lo
 cudaError_t pipe_tile_f32(const void* x, int64_t rows, int64_t cols, uint8_t* e4m3, float* scale, cudaStream_t st);
 cudaError_t pipe_tile_f16(const void* x, int64_t rows, int64_t cols, uint8_t* e4m3, float* scale, cudaStream_t st);
 cudaError_t pipe_tile_bf16(const void* x, int64_t rows, int64_t cols, uint8_t* e4m3, float* scale, cudaStream_t st);
+cudaError_t pipe_fp8t_f32(const void* x, int64_t n, uint8_t* e4m3, float* scale, const unsigned long long* rec, int from_rec, cudaStream_t st);
+cudaError_t pipe_fp8t_f16(const void* x, int64_t n, uint8_t* e4m3, float* scale, const unsigned long long* rec, int from_rec, cudaStream_t st);
+cudaError_t pipe_fp8t_bf16(const void* x, int64_t n, uint8_t* e4m3, float* scale, const unsigned long long* rec, int from_rec, cudaStream_t st);
 
 static cudaError_t pipe_launch(DT dt, int pk, bool sym, const PipeArgs& a, cudaStream_t st) {
     switch (dt) {
@@ -98,6 +101,17 @@ cudaError_t fp8_tile_pipe(DT dt, const void* x, int64_t rows, int64_t cols, uint
     switch (dt) {
         case DT::F16: return pipe_tile_f16(x, rows, cols, e4m3, scale, st);
         case DT::BF16: return pipe_tile_bf16(x, rows, cols, e4m3, scale, st);
+        default: return cudaErrorNotSupported;
+    }
+}
+
+cudaError_t fp8_tensor_quant(DT dt, const void* x, int64_t n, uint8_t* e4m3, float* scale,
+                             const unsigned long long* rec, int from_rec, cudaStream_t st) {
+    if (n == 0) return cudaSuccess;
+    switch (dt) {
+        case DT::F32: return pipe_fp8t_f32(x, n, e4m3, scale, rec, from_rec, st);
+        case DT::F16: return pipe_fp8t_f16(x, n, e4m3, scale, rec, from_rec, st);
+        case DT::BF16: return pipe_fp8t_bf16(x, n, e4m3, scale, rec, from_rec, st);
         default: return cudaErrorNotSupported;
     }
 }

@@ -914,6 +914,158 @@ __global__ void __launch_bounds__(256) k_fp8_tile_tma(const __grid_constant__ CU
     }
 }
 
+// ------------------------------------------------------------ FP8 per-tensor
+// FP8 per-tensor store (smile llm.quant Fp8KvCodec): e = E4M3(fl(x / s)) with
+// one f32 scale s for the whole tensor, given (*scale) or fl(amax / 448) from
+// the range record written by the range kernel just before this one (launched
+// to overlap it: the first copies go out before the wait). A vector with a
+// NaN or an element beyond 2^64 s takes the general encoder.
+struct Fp8TArgs {
+    const void* x;
+    int64_t n;
+    uint8_t* e4m3;
+    float* scale;
+    const unsigned long long* rec;
+    int from_rec;
+};
+
+// The same store, pipelined: chunks of FP8T_CHUNK bytes of x reach shared
+// memory by bulk copy into a ring of FP8T_STAGES slots; each thread copies its
+// vectors of a chunk to registers, one barrier frees the slot for the chunk S
+// ahead, then the vectors are encoded. x 16-byte and e4m3 8-byte aligned.
+constexpr int FP8T_CHUNK = 32768;
+constexpr int FP8T_STAGES = 2;
+
+template <class T>
+__global__ void __launch_bounds__(256) k_fp8t_pipe(Fp8TArgs a) {
+    constexpr int VEC = Traits<T>::VEC;
+    constexpr int S = FP8T_STAGES;
+    constexpr int NVT = FP8T_CHUNK / 16 / 256;            // vectors per thread per chunk
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 64);
+    uint8_t* ring = smem + 128;
+    const int tid = threadIdx.x;
+    const int64_t grid = gridDim.x;
+    const T* x = (const T*)a.x;
+    const int64_t nvec = a.n / VEC;                        // whole 16-byte vectors
+    const int64_t body = nvec * 16;
+    const int64_t n_chunks = (body + FP8T_CHUNK - 1) / FP8T_CHUNK;
+    auto chunk_bytes = [&](int64_t c) -> uint32_t {
+        return (uint32_t)min((int64_t)FP8T_CHUNK, body - c * FP8T_CHUNK);
+    };
+    if (tid == 0) {
+        for (int i = 0; i < S; ++i) mbar_init(smem_addr(&bars[i]), 1);
+        fence_mbar_init();
+        for (int i = 0; i < S; ++i) {
+            const int64_t c = blockIdx.x + (int64_t)i * grid;
+            if (c >= n_chunks) break;
+            bulk_load(smem_addr(ring + (size_t)i * FP8T_CHUNK), (const uint8_t*)x + c * FP8T_CHUNK,
+                      chunk_bytes(c), smem_addr(&bars[i]));
+        }
+    }
+    __syncthreads();
+    float s;
+    if (a.from_rec) {
+        pdl_wait();
+        float h, nl;
+        range_from_bits(a.rec[0], h);
+        range_from_bits(a.rec[1], nl);
+        s = __fdiv_rn(fmaxf(h, nl), 448.0f);
+        if (s == 0.0f) s = 1.0f;
+        if (blockIdx.x == 0 && tid == 0) *a.scale = s;
+    } else {
+        s = *a.scale;
+    }
+    const Recip R = make_recip(s);
+    const bool fast_s = R.fast && s > 0.0f;
+    const Recip2 R2 = make_recip2(R);
+    const float lim = __fmul_rn(0x1p64f, s);
+    int slot = 0;
+    uint32_t parity = 0;
+    for (int64_t c = blockIdx.x; c < n_chunks; c += grid) {
+        const bool ok = mbar_wait(smem_addr(&bars[slot]), parity);
+        const uint32_t base = smem_addr(ring + (size_t)slot * FP8T_CHUNK);
+        const int nv = (int)(chunk_bytes(c) / 16);
+        U4 raw[NVT];
+#pragma unroll
+        for (int v = 0; v < NVT; ++v) {
+            const int vi = v * 256 + tid;
+            raw[v] = (vi < nv) ? ld_shared16(base + (uint32_t)vi * 16u) : U4{0u, 0u, 0u, 0u};
+        }
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) {
+                atomicOr(&g_pipe_error, 1u);
+                int s3 = slot;
+                uint32_t p3 = parity;
+                for (int i = 0; i < S; ++i) {
+                    if (c + (int64_t)i * grid >= n_chunks) break;
+                    mbar_wait(smem_addr(&bars[s3]), p3);
+                    if (++s3 == S) { s3 = 0; p3 ^= 1u; }
+                }
+            }
+            __syncthreads();
+            return;
+        }
+        if (tid == 0) {
+            const int64_t next = c + (int64_t)S * grid;
+            if (next < n_chunks) {
+                fence_proxy_async();
+                bulk_load(smem_addr(ring + (size_t)slot * FP8T_CHUNK), (const uint8_t*)x + next * FP8T_CHUNK,
+                          chunk_bytes(next), smem_addr(&bars[slot]));
+            }
+        }
+        if (++slot == S) { slot = 0; parity ^= 1u; }
+        const int64_t v0 = c * (FP8T_CHUNK / 16);            // first vector of the chunk
+#pragma unroll
+        for (int v = 0; v < NVT; ++v) {
+            const int vi = v * 256 + tid;
+            if (vi >= nv) continue;
+            uint32_t ph = 0u, pl = 0u;
+            float hi = 0.0f, nlo = 0.0f;
+            range_tree<T, true, true, 1>(&raw[v], ph, pl, hi, nlo);
+            const bool nan = range_finish_nan<T, true>(ph, pl, hi, nlo);
+            uint8_t* dst = a.e4m3 + (v0 + vi) * VEC;
+            if (fast_s && !nan && hi <= lim) {
+                emit_fp8_fast<T>(raw[v], R2, dst);
+            } else {
+                float vals[VEC];
+                load_vec<T>(raw[v], vals);
+                mx_emit<T, MX_FP8_1x128, false>(vals, R, 0.f, false, dst);
+            }
+        }
+    }
+    // elements after the last whole vector
+    if (blockIdx.x == 0 && tid < a.n - nvec * VEC) {
+        const int64_t i = nvec * VEC + tid;
+        const float v = ld1<T>(x + i);
+        a.e4m3[i] = (uint8_t)(e4m3x2(with_quotient_sign(div_any(v, R), v, s), 0.0f) & 0xFFu);
+    }
+}
+
+// Any alignment: one element per thread step.
+template <class T>
+__global__ void __launch_bounds__(256) k_fp8_tensor_scalar(Fp8TArgs a) {
+    float s;
+    if (a.from_rec) {
+        pdl_wait();
+        float h, nl;
+        range_from_bits(a.rec[0], h);
+        range_from_bits(a.rec[1], nl);
+        s = __fdiv_rn(fmaxf(h, nl), 448.0f);
+        if (s == 0.0f) s = 1.0f;
+        if (blockIdx.x == 0 && threadIdx.x == 0) *a.scale = s;
+    } else {
+        s = *a.scale;
+    }
+    const Recip R = make_recip(s);
+    const T* x = (const T*)a.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < a.n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const float v = ld1<T>(x + i);
+        a.e4m3[i] = (uint8_t)(e4m3x2(with_quotient_sign(div_any(v, R), v, s), 0.0f) & 0xFFu);
+    }
+}
+
 // ------------------------------------------------------------ tensor range
 // Range record of a whole tensor (per-tensor scaling, the NVFP4 per-tensor
 // scale). The 16-byte aligned body streams through a ring of RANGE_STAGES
@@ -1664,6 +1816,40 @@ static cudaError_t tile_entry(const void* x, int64_t rows, int64_t cols, uint8_t
     }
 }
 
+// FP8 per-tensor store (k_fp8t_pipe); the consumer of the range kernel when
+// the scale is dynamic (launch_pdl).
+template <class T>
+static cudaError_t fp8t_entry(const void* x, int64_t n, uint8_t* e4m3, float* scale,
+                              const unsigned long long* rec, int from_rec, cudaStream_t st) {
+    constexpr int VEC = Traits<T>::VEC;
+    Fp8TArgs a{x, n, e4m3, scale, rec, from_rec};
+    const bool vec = (((uintptr_t)x & 15u) == 0) && (((uintptr_t)e4m3 % VEC) == 0);
+    if (vec) {
+        const size_t smem = 128 + (size_t)FP8T_STAGES * FP8T_CHUNK;
+        auto k = k_fp8t_pipe<T>;
+        static const cudaError_t attr = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (attr != cudaSuccess) return attr;
+        static unsigned long long occ[8];
+        const int bps = occupancy_for((const void*)k, smem, occ);
+        if (bps < 1) return cudaErrorNotSupported;
+        const int64_t n_chunks = (n / VEC * 16 + FP8T_CHUNK - 1) / FP8T_CHUNK;
+        int64_t grid = (int64_t)sm_count() * bps;
+        if (grid > n_chunks) grid = n_chunks;
+        if (grid < 1) grid = 1;
+        if (from_rec) return launch_pdl(k, (unsigned)grid, 256u, smem, st, a);
+        k<<<(unsigned)grid, 256, smem, st>>>(a);
+        return cudaGetLastError();
+    }
+    int64_t grid = (n + 255) / 256;
+    const int64_t cap = (int64_t)sm_count() * 8;
+    if (grid > cap) grid = cap;
+    if (grid < 1) grid = 1;
+    auto k = k_fp8_tensor_scalar<T>;
+    if (from_rec) return launch_pdl(k, (unsigned)grid, 256u, 0, st, a);
+    k<<<(unsigned)grid, 256, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
 // Entry points of one dtype's translation unit.
 template <class T>
 cudaError_t pipe_dyn_entry(int pk, bool sym, const PipeArgs& a, cudaStream_t st) {
@@ -1705,6 +1891,10 @@ cudaError_t pipe_error_entry(unsigned int* flag) {
     cudaError_t pipe_tile_##NAME(const void* x, int64_t rows, int64_t cols, uint8_t* e4m3,       \
                                  float* scale, cudaStream_t st) {                                 \
         return tile_entry<T>(x, rows, cols, e4m3, scale, st);                                    \
+    }                                                                                            \
+    cudaError_t pipe_fp8t_##NAME(const void* x, int64_t n, uint8_t* e4m3, float* scale,           \
+                                 const unsigned long long* rec, int from_rec, cudaStream_t st) {  \
+        return fp8t_entry<T>(x, n, e4m3, scale, rec, from_rec, st);                              \
     }
 
 }  // namespace bq

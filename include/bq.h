@@ -337,6 +337,22 @@ bq_status bq_fp8_block_dequantize(const uint8_t* e4m3, const float* scale, int64
                                   int64_t cols, int32_t block_rows, int32_t block_cols, void* y,
                                   bq_dtype y_dtype, void* stream);
 
+/* --------------------------------------------------- FP8 per-tensor codec */
+/* [smile.llm.quant] Fp8KvCodec (FP8 KV store / load with per-tensor scales):
+ * one f32 scale for the whole tensor, the dequantize multiplier as in the FP8
+ * block formats. Store: e4m3 u8 [n] = E4M3(fl(x / s)) (round to nearest even,
+ * saturating to +-448, NaN -> 0x7F) for x of dtype F32, F16 or BF16 and n
+ * elements. static_scale == 1: s = *scale (device, input). static_scale == 0:
+ * s = fl(amax / 448) (amax ignores NaN; 0 -> 1), written to *scale; ws: 16
+ * bytes of device scratch (the range record). */
+bq_status bq_fp8_tensor_quantize(const void* x, bq_dtype x_dtype, int64_t n, uint8_t* e4m3,
+                                 float* scale, int32_t static_scale, void* ws, size_t ws_bytes,
+                                 void* stream);
+
+/* Load: y [n] = RN_y(fl(E4M3(e) * *scale)). */
+bq_status bq_fp8_tensor_dequantize(const uint8_t* e4m3, const float* scale, int64_t n, void* y,
+                                   bq_dtype y_dtype, void* stream);
+
 /* ------------------------------------------------------- packed transpose */
 /* [QuantizedWeight] transpose_for_gemm(_gs) / transpose_concat_for_gemm_padded
  * (one part): packed weight w u8 [n, k/2] -> w_t u8 [k/2, stride] and scales

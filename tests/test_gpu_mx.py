@@ -308,3 +308,51 @@ def test_workload_mxfp4(bq, orc):
     assert_bitwise(cpu(s)[rows], rs, "e8m0")
     y = bq.mxfp4_dequantize(p, s, torch.bfloat16)
     assert_bitwise(cpu(y)[rows], orc.mxfp4_dequantize(rp, rs, len(rows), 7168, "bf16"), "deq")
+
+
+# ---------------------------------------------------------------- FP8 per-tensor (KV codec)
+@pytest.mark.parametrize("dtype", ["bf16", "f16", "f32"])
+@pytest.mark.parametrize("shape", [(1,), (7,), (3, 37), (16, 8, 128), (1001, 77)])
+def test_fp8_tensor_codec_parity(bq, orc, dtype, shape):
+    x = synthetic.Stream(41).tensor(shape, dtype, dist="student_t3", outlier_p=0.01, outlier_factor=30)
+    e, s = bq.fp8_tensor_quantize(x.cuda())
+    re, rs = orc.fp8_tensor_quantize(x)
+    assert cpu(s).item() == rs
+    assert_bitwise(e, re, "codes (dynamic)")
+    for sv in (rs, 2.0 ** -9, 1e-30, 7.5):      # static; 2^-9 and 1e-30 saturate, 7.5 underflows
+        svf = float(np.float32(sv))
+        e, _ = bq.fp8_tensor_quantize(x.cuda(), scale=svf)
+        re, _ = orc.fp8_tensor_quantize(x, scale=svf)
+        assert_bitwise(e, re, f"codes (static {svf})")
+        for ydt in ("f32", "bf16", "f16"):
+            y = bq.fp8_tensor_dequantize(e, svf, DT[ydt])
+            assert_bitwise(y, orc.fp8_tensor_dequantize(re, svf, ydtype=ydt), f"load {ydt}")
+
+
+def test_fp8_tensor_codec_special_values_and_unaligned(bq, orc):
+    vals = [0.0, -0.0, 1e-30, -1e-30, 448.0, -448.0, 500.0, float("inf"), float("-inf"),
+            float("nan"), -float("nan"), 1.0, -1.0, 3.4e38, -3.4e38, 0.001]
+    x = torch.tensor(vals * 8, dtype=torch.float32)
+    for sv in (None, 1.0, -2.0, 0.0):
+        e, s = bq.fp8_tensor_quantize(x.cuda(), scale=sv)
+        re, rs = orc.fp8_tensor_quantize(x, scale=sv)
+        assert_bitwise(e, re, f"codes {sv}")
+    xb = synthetic.Stream(42).tensor((4099,), "bf16")
+    buf = torch.zeros(xb.numel() + 1, dtype=xb.dtype, device="cuda")
+    xg = buf[1:]
+    xg.copy_(xb.cuda())
+    e, s = bq.fp8_tensor_quantize(xg)
+    re, rs = orc.fp8_tensor_quantize(xb)
+    assert cpu(s).item() == rs
+    assert_bitwise(e, re, "codes (unaligned x)")
+
+
+def test_workload_fp8_tensor_codec(bq, orc):
+    xg = synthetic.make_workload_device("per_token_bf16_8192x4096")["x"]
+    x = cpu(xg)
+    e, s = bq.fp8_tensor_quantize(xg)
+    re, rs = orc.fp8_tensor_quantize(x)
+    assert cpu(s).item() == rs
+    assert_bitwise(e, re, "codes")
+    y = bq.fp8_tensor_dequantize(e, s, torch.bfloat16)
+    assert_bitwise(y, orc.fp8_tensor_dequantize(re, rs, ydtype="bf16"), "load")
