@@ -438,12 +438,17 @@ __global__ void __launch_bounds__(NT) k_seg_pipe(PipeArgs a) {
             // each quotient by the launch's divisor reciprocal (exact for a
             // normal dividend; IEEE division below 2^-100).
             float sc, zf = 0.0f, rz = 0.0f;
+            Recip R;
             {
                 const float num = SYM ? fmaxf(hi, nlo) : __fadd_rn(hi, nlo);
                 sc = (num >= 0x1p-100f && num <= 0x1p100f) ? div_chain(num, Rq) : div_slow(num, Rq.s);
                 if (sc == 0.0f) sc = 1.0f;
+                R = make_recip(sc);
                 if (!SYM) {
-                    const float m = __fdiv_rn(-nlo, sc);
+                    // fl(min'/s) through the group's reciprocal: |min'/s| <= qmax - qmin,
+                    // so the chain cannot overflow, and it is exact wherever the
+                    // rounding to an integer can depend on it (|min'/s| >= 1/2).
+                    const float m = R.fast ? div_chain(-nlo, R) : __fdiv_rn(-nlo, sc);
                     rz = a.cfg.rhaz ? roundf(m) : rintf(m);
                     zf = fminf(fmaxf(__fsub_rn(qlo, rz), qlo), qhi);   // NaN -> qmin
                 }
@@ -457,7 +462,6 @@ __global__ void __launch_bounds__(NT) k_seg_pipe(PipeArgs a) {
             ip.lo = SYM ? qlo : __fsub_rn(qlo, zf);
             ip.hi = SYM ? qhi : __fsub_rn(qhi, zf);
             ip.zp = SYM ? 0 : zp;
-            const Recip R = make_recip(sc);
             uint8_t* qb = a.q + seg * G + lane * VEC;
             T* yb = (T*)a.y + seg * G + lane * VEC;
             // Fast path: no NaN in the warp's groups, a normal scale, and no
