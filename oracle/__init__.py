@@ -8,7 +8,8 @@ nothing from it: the two sides share no code.
 Tensors in and out are contiguous CPU ``torch.Tensor`` objects (torch is only
 used here as a typed buffer that can hold bf16); all arithmetic happens in
 ``oracle.cpp``. Dtype names: f32 f64 f16 bf16 s8 u8. Granularity names:
-tensor channel group token.
+tensor channel group token column_group (groups along `axis` at one index of
+the dimensions after it).
 """
 
 from __future__ import annotations
@@ -25,7 +26,7 @@ _T = {"f32": 0, "f64": 1, "f16": 2, "bf16": 3, "s8": 4, "u8": 5}
 _TORCH = {"f32": torch.float32, "f64": torch.float64, "f16": torch.float16,
           "bf16": torch.bfloat16, "s8": torch.int8, "u8": torch.uint8}
 _NAME = {v: k for k, v in _TORCH.items()}
-_GRAN = {"tensor": 0, "channel": 1, "group": 2, "token": 3}
+_GRAN = {"tensor": 0, "channel": 1, "group": 2, "token": 3, "column_group": 4}
 _FMT = {"f16": 0, "bf16": 1, "e4m3": 2, "e2m1": 3, "e8m0": 4}
 
 _lib = None

@@ -224,12 +224,20 @@ double round_rhaz(double v) {
 // Group g of outer index o covers axis indices [g*gs, (g+1)*gs) and all inner
 // indices: with x viewed as [outer, L, inner] the element (o, l, i) sits at
 // (o*L + l)*inner + i.
-enum OrGran { GRAN_TENSOR = 0, GRAN_CHANNEL = 1, GRAN_GROUP = 2, GRAN_TOKEN = 3 };
+// Column groups (GRAN_COLUMN): the Group granularity read as blocks of gs
+// consecutive indices along `axis` at one fixed index of the dimensions after
+// it (the [K, N]-stored weight of a GPTQ-style quantizer grouped along K):
+// group (o, b, i) holds the elements (o, l, i) for l in [b*gs, (b+1)*gs), and
+// groups are numbered (o*(L/gs) + b)*inner + i, i.e. a scale array of shape
+// [outer, L/gs, inner].
+enum OrGran { GRAN_TENSOR = 0, GRAN_CHANNEL = 1, GRAN_GROUP = 2, GRAN_TOKEN = 3, GRAN_COLUMN = 4 };
 
 struct Layout {
     int64_t outer = 1, L = 1, inner = 1, gs = 1;   // groups per outer = L / gs
+    bool column = false;                           // one group per inner index
     bool ok = true;
-    int64_t n_groups() const { return outer * (gs ? L / gs : 0); }
+    int64_t n_groups() const { return outer * (gs ? L / gs : 0) * (column ? inner : 1); }
+    int64_t group_elems() const { return column ? gs : gs * inner; }
     int64_t numel() const { return outer * L * inner; }
 };
 
@@ -254,7 +262,9 @@ Layout make_layout(int ndim, const int64_t* shape, int gran, int axis, int64_t g
     }
     if (axis < 0 || axis >= ndim) { lay.ok = false; return lay; }
     if (gran == GRAN_CHANNEL) gs = 1;          // PerChannel{axis} -> (axis, 1)
+    if (gran != GRAN_CHANNEL && gran != GRAN_GROUP && gran != GRAN_COLUMN) { lay.ok = false; return lay; }
     if (gs < 1) { lay.ok = false; return lay; }
+    lay.column = (gran == GRAN_COLUMN);
     lay.outer = 1; lay.inner = 1;
     for (int d = 0; d < axis; ++d) lay.outer *= shape[d];
     for (int d = axis + 1; d < ndim; ++d) lay.inner *= shape[d];
@@ -267,6 +277,12 @@ Layout make_layout(int ndim, const int64_t* shape, int gran, int axis, int64_t g
 template <class F>
 void for_each_in_group(const Layout& lay, int64_t group, F&& fn) {
     const int64_t per_outer = lay.L / lay.gs;
+    if (lay.column) {
+        const int64_t i = group % lay.inner, ob = group / lay.inner;
+        const int64_t o = ob / per_outer, b = ob % per_outer;
+        for (int64_t l = b * lay.gs; l < (b + 1) * lay.gs; ++l) fn((o * lay.L + l) * lay.inner + i);
+        return;
+    }
     const int64_t o = group / per_outer, g = group % per_outer;
     for (int64_t l = g * lay.gs; l < (g + 1) * lay.gs; ++l)
         for (int64_t i = 0; i < lay.inner; ++i)
@@ -400,7 +416,7 @@ int or_group_count(int ndim, const int64_t* shape, int gran, int axis, int64_t g
     Layout lay = make_layout(ndim, shape, gran, axis, gs);
     if (!lay.ok) return 1;
     *n_groups = lay.n_groups();
-    *group_elems = lay.gs * lay.inner;
+    *group_elems = lay.group_elems();
     return 0;
 }
 

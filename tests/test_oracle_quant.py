@@ -310,3 +310,101 @@ def test_empty_tensors(orc):
         assert q.shape == x.shape and s.numel() == shape[0] * (1 if shape[1] else 0) or True
         q, s, _ = orc.quantize(x, "tensor")
         assert s.item() == 1.0
+
+
+# ---------------------------------------------------------------- column groups
+# granularity.rs Group{axis, group_size}: "one scale / zero-point per
+# contiguous group_size-element block along axis", read here for a tensor
+# stored [K, N] with the groups along K (the GPTQ/AWQ convention the page names):
+# one group per (outer, block, inner index), scales shaped [outer, L/gs, inner].
+COL_CASES = [((8, 6), 0, 4), ((8, 6), 0, 8), ((2, 6, 5), 1, 3), ((3, 4, 2, 2), 1, 2),
+             ((256, 48), 0, 128), ((6, 1), 0, 2), ((5, 7), 1, 7)]
+
+
+def _col_view(shape, axis, gs):
+    outer = int(np.prod(shape[:axis], dtype=np.int64))
+    inner = int(np.prod(shape[axis + 1:], dtype=np.int64))
+    return outer, shape[axis] // gs, gs, inner
+
+
+@pytest.mark.parametrize("shape,axis,gs", COL_CASES)
+def test_column_group_scales_and_codes_vs_numpy(orc, shape, axis, gs):
+    # Symmetric s8: s = fl(amax / 127) per (o, b, i); asymmetric u8: the
+    # min' / max' closed form; codes = clamp(rne(fl(x / s)) + zp), numpy f32.
+    x = synthetic.Stream(40).tensor(shape, "f32", outlier_p=0.05, outlier_factor=20)
+    v = _col_view(shape, axis, gs)
+    xv = x.numpy().reshape(v)
+    ng, ge = orc.group_count(shape, "column_group", axis, gs)
+    assert (ng, ge) == (v[0] * v[1] * v[3], gs)
+    q, s, _ = orc.quantize(x, "column_group", axis, gs)
+    amax = np.abs(xv).max(axis=2)
+    s_np = (amax.astype(np.float64) / 127.0).astype(np.float32)
+    assert np.array_equal(s.numpy().reshape(amax.shape), s_np)
+    sb = s_np[:, :, None, :]
+    want = np.clip(np.rint(xv / sb), -128, 127).astype(np.int64)
+    assert np.array_equal(q.numpy().astype(np.int64).reshape(v), want)
+    # Asymmetric u8.
+    qa, sa, za = orc.quantize(x, "column_group", axis, gs, qdtype="u8", symmetric=False)
+    hi = np.maximum(xv.max(axis=2), np.float32(0))
+    nlo = np.maximum(-xv.min(axis=2), np.float32(0))
+    span = (hi + nlo).astype(np.float32)
+    s_a = (span / np.float32(255)).astype(np.float32)
+    s_a = np.where(s_a == 0, np.float32(1), s_a)
+    zp = np.clip(0 - np.rint((-nlo / s_a).astype(np.float32)), 0, 255).astype(np.int64)
+    assert np.array_equal(sa.numpy().reshape(s_a.shape), s_a)
+    assert np.array_equal(za.numpy().astype(np.int64).reshape(zp.shape), zp)
+    wa = np.clip(np.rint(xv / s_a[:, :, None, :]) + zp[:, :, None, :], 0, 255).astype(np.int64)
+    assert np.array_equal(qa.numpy().astype(np.int64).reshape(v), wa)
+
+
+def test_column_group_over_whole_axis_is_per_token_of_transpose(orc):
+    # Blocks as long as the axis: one scale per column of a [K, N] tensor,
+    # the per-row (per-token) scaling of its transpose.
+    x = synthetic.Stream(41).tensor((64, 24), "bf16")
+    for sym, qd in ((True, "s8"), (False, "u8")):
+        a = orc.quantize(x, "column_group", 0, 64, qdtype=qd, symmetric=sym)
+        b = orc.quantize(x.t().contiguous(), "token", qdtype=qd, symmetric=sym)
+        assert torch.equal(a[0], b[0].t())
+        for u, w in zip(a[1:], b[1:]):
+            assert torch.equal(u, w)
+
+
+def test_column_group_on_last_axis_is_contiguous_group(orc):
+    # Nothing after the axis: a column group is the contiguous group.
+    x = synthetic.Stream(42).tensor((3, 5, 32), "f16")
+    a = orc.quantize(x, "column_group", 2, 8, qdtype="u8", symmetric=False)
+    b = orc.quantize(x, "group", 2, 8, qdtype="u8", symmetric=False)
+    for u, w in zip(a, b):
+        assert torch.equal(u, w)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f64"])
+def test_column_group_is_group_of_the_transpose(orc, dtype):
+    # x [K, N] grouped along K per column == x^T [N, K] grouped contiguously
+    # along its last axis, transposed back; scales [K/gs, N] == ([N, K/gs])^T.
+    K, N, gs = 32, 10, 8
+    x = synthetic.Stream(43).tensor((K, N), dtype, outlier_p=0.05, outlier_factor=10)
+    xt = x.t().contiguous()
+    dy = synthetic.Stream(44).tensor((K, N), dtype)
+    for sym, qd in ((True, "s8"), (False, "u8")):
+        q, s, z = orc.quantize(x, "column_group", 0, gs, qdtype=qd, symmetric=sym)
+        qt, st, zt = orc.quantize(xt, "group", 1, gs, qdtype=qd, symmetric=sym)
+        assert torch.equal(q, qt.t())
+        assert torch.equal(s.reshape(K // gs, N), st.reshape(N, K // gs).t())
+        if not sym:
+            assert torch.equal(z.reshape(K // gs, N), zt.reshape(N, K // gs).t())
+        zz = None if sym else z
+        y = orc.dequantize(q, s, zz, "column_group", 0, gs, ydtype=dtype)
+        yt = orc.dequantize(qt, st, None if sym else zt, "group", 1, gs, ydtype=dtype)
+        assert torch.equal(y, yt.t())
+        f, _, _ = orc.fake_quantize(x, "column_group", 0, gs, qdtype=qd, symmetric=sym)
+        ft, _, _ = orc.fake_quantize(xt, "group", 1, gs, qdtype=qd, symmetric=sym)
+        assert torch.equal(f, ft.t())
+        dyt = dy.t().contiguous()
+        for bwd in (orc.quantize_backward, orc.fake_quantize_backward):
+            a = bwd(x, dy, s, zz, "column_group", 0, gs, qdtype=qd, symmetric=sym)
+            b = bwd(xt, dyt, st, None if sym else zt, "group", 1, gs, qdtype=qd, symmetric=sym)
+            assert torch.equal(a, b.t())
+        a = orc.dequantize_backward(dy, s, "column_group", 0, gs)
+        b = orc.dequantize_backward(dyt, st, "group", 1, gs)
+        assert torch.equal(a, b.t())
