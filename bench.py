@@ -301,6 +301,17 @@ def per_granularity(B, api, torch, device, peak, reps=5):
           lambda: B.bq_quantize_per_group_backward(x, dy, s, z, du, 1, 128, dx), 6 * n + 5 * ng, 1)
     timed(wl, "fake_quantize_backward(group)",
           lambda: B.bq_fake_quantize_backward(x, dy, s, z, du, "group", 1, 128, dx), 6 * n + 5 * ng, 1)
+    # The same tensor as a [K, N] weight grouped along K (column groups, GPTQ layout).
+    wlc = "column_group128_f16_11008x4096"
+    timed(wlc, "quantize_per_column_group(axis=0,gs=128,u8 asym)",
+          lambda: B.bq_quantize_per_column_group(x, du, 0, 128, q, s, z, "dynamic"), 3 * n + 5 * ng, 1)
+    timed(wlc, "dequantize_per_column_group",
+          lambda: B.bq_dequantize_per_column_group(q, s, z, du, 0, 128, y), 3 * n + 5 * ng, 1)
+    timed(wlc, "fake_quantize(column_group,dynamic)",
+          lambda: B.bq_fake_quantize(x, du, "column_group", 0, 128, s, z, "dynamic", y, None),
+          4 * n + 5 * ng, 1)
+    timed(wlc, "quantize_per_column_group_backward",
+          lambda: B.bq_quantize_per_column_group_backward(x, dy, s, z, du, 0, 128, dx), 6 * n + 5 * ng, 1)
     del w, x, dy, q, qs, y, dx
 
     # NVFP4 bf16 [4096, 7168]

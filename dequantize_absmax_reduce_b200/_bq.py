@@ -28,13 +28,14 @@ lib = C.CDLL(LIB_PATH)
 BQ_OK, BQ_ERR_INVALID_ARG, BQ_ERR_UNSUPPORTED, BQ_ERR_MISALIGNED, BQ_ERR_CUDA, BQ_ERR_TIMEOUT = range(6)
 BQ_F32, BQ_F64, BQ_F16, BQ_BF16, BQ_S8, BQ_U8, BQ_E4M3, BQ_E2M1X2, BQ_E8M0 = range(9)
 BQ_RNE, BQ_RHAZ = 0, 1
-BQ_GRAN_TENSOR, BQ_GRAN_CHANNEL, BQ_GRAN_GROUP = 0, 1, 2
+BQ_GRAN_TENSOR, BQ_GRAN_CHANNEL, BQ_GRAN_GROUP, BQ_GRAN_COLUMN_GROUP = 0, 1, 2, 3
 BQ_SCALE_DYNAMIC, BQ_SCALE_STATIC, BQ_SCALE_FROM_RANGE = 0, 1, 2
 BQ_NOALLOC_MAX_GROUPS = 65536
 
 DTYPE = {torch.float32: BQ_F32, torch.float64: BQ_F64, torch.float16: BQ_F16,
          torch.bfloat16: BQ_BF16, torch.int8: BQ_S8, torch.uint8: BQ_U8}
-GRAN = {"tensor": BQ_GRAN_TENSOR, "channel": BQ_GRAN_CHANNEL, "group": BQ_GRAN_GROUP}
+GRAN = {"tensor": BQ_GRAN_TENSOR, "channel": BQ_GRAN_CHANNEL, "group": BQ_GRAN_GROUP,
+        "column_group": BQ_GRAN_COLUMN_GROUP}
 MODE = {"dynamic": BQ_SCALE_DYNAMIC, "static": BQ_SCALE_STATIC, "from_range": BQ_SCALE_FROM_RANGE}
 ROUND = {"rne": BQ_RNE, "rhaz": BQ_RHAZ}
 
@@ -63,21 +64,25 @@ _SIGS = {
     "bq_quantize_per_channel": [_P, _DESC, _I32, _P, _P, _P, C.c_int, _P, _SZ, _P],
     "bq_quantize_per_token": [_P, _DESC, _P, _P, _P, C.c_int, _P, _SZ, _P],
     "bq_quantize_per_group": [_P, _DESC, _I32, _I64, _P, _P, _P, C.c_int, _P, _SZ, _P],
+    "bq_quantize_per_column_group": [_P, _DESC, _I32, _I64, _P, _P, _P, C.c_int, _P],
     "bq_quantize_dynamic_noalloc": [_P, _DESC, C.c_int, _I32, _I64, _P, _P, _P, _P],
     "bq_dequantize_per_tensor": [_P, _P, _P, _DESC, _P, C.c_int, _P],
     "bq_dequantize_per_channel": [_P, _P, _P, _DESC, _I32, _P, C.c_int, _P],
     "bq_dequantize_per_token": [_P, _P, _P, _DESC, _P, C.c_int, _P],
     "bq_dequantize_per_group": [_P, _P, _P, _DESC, _I32, _I64, _P, C.c_int, _P],
+    "bq_dequantize_per_column_group": [_P, _P, _P, _DESC, _I32, _I64, _P, C.c_int, _P],
     "bq_fake_quantize": [_P, _DESC, C.c_int, _I32, _I64, _P, _P, C.c_int, _P, _P, _SZ, _P],
     "bq_quantize_per_tensor_backward": [_P, _P, _P, _P, _DESC, _P, _P],
     "bq_quantize_per_channel_backward": [_P, _P, _P, _P, _DESC, _I32, _P, _P],
     "bq_quantize_per_token_backward": [_P, _P, _P, _P, _DESC, _P, _P],
     "bq_quantize_per_group_backward": [_P, _P, _P, _P, _DESC, _I32, _I64, _P, _P],
+    "bq_quantize_per_column_group_backward": [_P, _P, _P, _P, _DESC, _I32, _I64, _P, _P],
     "bq_fake_quantize_backward": [_P, _P, _P, _P, _DESC, C.c_int, _I32, _I64, _P, _P],
     "bq_dequantize_per_tensor_backward": [_P, _P, _DESC, _P, _P],
     "bq_dequantize_per_channel_backward": [_P, _P, _DESC, _I32, _P, _P],
     "bq_dequantize_per_token_backward": [_P, _P, _DESC, _P, _P],
     "bq_dequantize_per_group_backward": [_P, _P, _DESC, _I32, _I64, _P, _P],
+    "bq_dequantize_per_column_group_backward": [_P, _P, _DESC, _I32, _I64, _P, _P],
     "bq_nvfp4_quantize": [_P, C.c_int, _I64, _I64, _P, _P, _P, _I32, _P, _SZ, _P],
     "bq_nvfp4_dequantize": [_P, _P, _P, _I64, _I64, _P, C.c_int, _P],
     "bq_mxfp8_quantize": [_P, C.c_int, _I64, _I64, _P, _P, _P],
@@ -236,6 +241,12 @@ def bq_quantize_per_group(x, d, axis, group_size, q, scale, zp, mode, ws=None, s
            "bq_quantize_per_group")
 
 
+def bq_quantize_per_column_group(x, d, axis, group_size, q, scale, zp, mode, stream=None):
+    _check(lib.bq_quantize_per_column_group(_ptr(x), C.byref(d), axis, group_size, _ptr(q),
+                                            _ptr(scale), _ptr(zp), _m(mode), _stream(stream)),
+           "bq_quantize_per_column_group")
+
+
 def bq_quantize_dynamic_noalloc(x, d, gran, axis, group_size, q, scale, zp, stream=None):
     _check(lib.bq_quantize_dynamic_noalloc(_ptr(x), C.byref(d), _g(gran), axis, group_size, _ptr(q),
                                            _ptr(scale), _ptr(zp), _stream(stream)),
@@ -262,6 +273,12 @@ def bq_dequantize_per_group(q, scale, zp, d, axis, group_size, y, stream=None):
     _check(lib.bq_dequantize_per_group(_ptr(q), _ptr(scale), _ptr(zp), C.byref(d), axis, group_size,
                                        _ptr(y), DTYPE[y.dtype], _stream(stream)),
            "bq_dequantize_per_group")
+
+
+def bq_dequantize_per_column_group(q, scale, zp, d, axis, group_size, y, stream=None):
+    _check(lib.bq_dequantize_per_column_group(_ptr(q), _ptr(scale), _ptr(zp), C.byref(d), axis,
+                                              group_size, _ptr(y), DTYPE[y.dtype], _stream(stream)),
+           "bq_dequantize_per_column_group")
 
 
 # ---------------------------------------------------------------- fake quantize
@@ -296,6 +313,13 @@ def bq_quantize_per_group_backward(x, dy, scale, zp, d, axis, group_size, dx, st
            "bq_quantize_per_group_backward")
 
 
+def bq_quantize_per_column_group_backward(x, dy, scale, zp, d, axis, group_size, dx, stream=None):
+    _check(lib.bq_quantize_per_column_group_backward(_ptr(x), _ptr(dy), _ptr(scale), _ptr(zp),
+                                                     C.byref(d), axis, group_size, _ptr(dx),
+                                                     _stream(stream)),
+           "bq_quantize_per_column_group_backward")
+
+
 def bq_fake_quantize_backward(x, dy, scale, zp, d, gran, axis, group_size, dx, stream=None):
     _check(lib.bq_fake_quantize_backward(_ptr(x), _ptr(dy), _ptr(scale), _ptr(zp), C.byref(d),
                                          _g(gran), axis, group_size, _ptr(dx), _stream(stream)),
@@ -322,6 +346,12 @@ def bq_dequantize_per_group_backward(dy, scale, d, axis, group_size, dq, stream=
     _check(lib.bq_dequantize_per_group_backward(_ptr(dy), _ptr(scale), C.byref(d), axis, group_size,
                                                 _ptr(dq), _stream(stream)),
            "bq_dequantize_per_group_backward")
+
+
+def bq_dequantize_per_column_group_backward(dy, scale, d, axis, group_size, dq, stream=None):
+    _check(lib.bq_dequantize_per_column_group_backward(_ptr(dy), _ptr(scale), C.byref(d), axis,
+                                                       group_size, _ptr(dq), _stream(stream)),
+           "bq_dequantize_per_column_group_backward")
 
 
 # ---------------------------------------------------------------- microscaled formats

@@ -1,8 +1,10 @@
 """Allocating helpers over the C ABI: each allocates its outputs (and any
 workspace) with torch on the input's device, then makes one binding call.
 
-Granularity names: "tensor", "channel", "group" (the granularity.rs enum)
-and "token" (one scale per row of the last dimension). Every helper returns
+Granularity names: "tensor", "channel", "group" (the granularity.rs enum),
+"token" (one scale per row of the last dimension) and "column_group" (blocks
+of group_size along `axis` at one index of the dimensions after it: the
+[K, N]-stored weight grouped along K; scales [outer, L/gs, inner]). Every helper returns
 torch tensors; no value is computed in Python.
 """
 
@@ -49,15 +51,21 @@ def quantize(x: torch.Tensor, gran: str, axis: int = 0, group_size: int = 1,
         zp = torch.empty(ng, dtype=qdtype, device=x.device)
         if ranges is not None:
             mode, ws = "from_range", ranges
-        else:
+        elif gran != "column_group":
             mode = "dynamic"
             ws = torch.empty(max(1, 2 * ng), dtype=torch.int64, device=x.device)
+        else:
+            mode = "dynamic"
     if gran == "tensor":
         B.bq_quantize_per_tensor(x, d, q, scale, zp, mode, ws, stream)
     elif gran == "token":
         B.bq_quantize_per_token(x, d, q, scale, zp, mode, ws, stream)
     elif gran == "channel":
         B.bq_quantize_per_channel(x, d, axis, q, scale, zp, mode, ws, stream)
+    elif gran == "column_group":
+        if mode == "from_range":
+            raise ValueError("column groups take no range records")
+        B.bq_quantize_per_column_group(x, d, axis, group_size, q, scale, zp, mode, stream)
     else:
         B.bq_quantize_per_group(x, d, axis, group_size, q, scale, zp, mode, ws, stream)
     return q, scale, zp
@@ -73,6 +81,8 @@ def dequantize(q: torch.Tensor, scale, zp, gran: str, axis: int = 0, group_size:
         B.bq_dequantize_per_token(q, scale, zp, d, y, stream)
     elif gran == "channel":
         B.bq_dequantize_per_channel(q, scale, zp, d, axis, y, stream)
+    elif gran == "column_group":
+        B.bq_dequantize_per_column_group(q, scale, zp, d, axis, group_size, y, stream)
     else:
         B.bq_dequantize_per_group(q, scale, zp, d, axis, group_size, y, stream)
     return y
@@ -112,6 +122,8 @@ def quantize_backward(x, dy, scale, zp, gran: str, axis: int = 0, group_size: in
         B.bq_quantize_per_token_backward(x, dy, scale, zp, d, dx, stream)
     elif gran == "channel":
         B.bq_quantize_per_channel_backward(x, dy, scale, zp, d, axis, dx, stream)
+    elif gran == "column_group":
+        B.bq_quantize_per_column_group_backward(x, dy, scale, zp, d, axis, group_size, dx, stream)
     else:
         B.bq_quantize_per_group_backward(x, dy, scale, zp, d, axis, group_size, dx, stream)
     return dx
@@ -136,6 +148,8 @@ def dequantize_backward(dy, scale, gran: str, axis: int = 0, group_size: int = 1
         B.bq_dequantize_per_token_backward(dy, scale, d, dq, stream)
     elif gran == "channel":
         B.bq_dequantize_per_channel_backward(dy, scale, d, axis, dq, stream)
+    elif gran == "column_group":
+        B.bq_dequantize_per_column_group_backward(dy, scale, d, axis, group_size, dq, stream)
     else:
         B.bq_dequantize_per_group_backward(dy, scale, d, axis, group_size, dq, stream)
     return dq

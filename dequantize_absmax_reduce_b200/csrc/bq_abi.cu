@@ -35,10 +35,13 @@ bq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BQ_OK : BQ_ERR_CU
 cudaStream_t S(void* s) { return (cudaStream_t)s; }
 
 // Granularities as the kernels see them (per-token is its own case).
-enum Gr { GR_TENSOR = 0, GR_CHANNEL = 1, GR_GROUP = 2, GR_TOKEN = 3 };
+enum Gr { GR_TENSOR = 0, GR_CHANNEL = 1, GR_GROUP = 2, GR_TOKEN = 3, GR_COLUMN = 4 };
 
 struct Layout {
-    bq::SegView sv;   // n_seg groups of G contiguous elements
+    bq::SegView sv;   // n_seg groups of G contiguous elements (column groups:
+                      // n_seg groups of G = gs elements, inner apart)
+    bool column = false;
+    bq::ColView cv{}; // column groups only
 };
 
 // Shape checks shared by every entry point: ndim in [0, 8], sizes >= 0 and
@@ -82,8 +85,16 @@ bq_status make_layout(const bq_qdesc* d, int gr, int32_t axis, int64_t gs, Layou
         for (int i = axis + 1; i < d->ndim; ++i) inner *= d->shape[i];
         const int64_t L = d->shape[axis];
         if (L % gs != 0) return BQ_ERR_INVALID_ARG;
-        sv.n_seg = outer * (L / gs);
-        sv.G = gs * inner;
+        if (gr == GR_COLUMN) {
+            // One group per (outer, block, inner index): gs elements, inner apart.
+            out->column = true;
+            out->cv = bq::ColView{outer, L, inner, gs};
+            sv.n_seg = outer * (L / gs) * inner;
+            sv.G = gs;
+        } else {
+            sv.n_seg = outer * (L / gs);
+            sv.G = gs * inner;
+        }
     }
     out->sv = sv;
     return BQ_OK;
@@ -128,6 +139,7 @@ bq_status quant_impl(int op, const void* x, const bq_qdesc* d, int gr, int32_t a
     if ((st = make_cfg(d, true, &cfg)) != BQ_OK) return st;
     if (mode != BQ_SCALE_DYNAMIC && mode != BQ_SCALE_STATIC && mode != BQ_SCALE_FROM_RANGE)
         return BQ_ERR_INVALID_ARG;
+    if (lay.column && mode == BQ_SCALE_FROM_RANGE) return BQ_ERR_UNSUPPORTED;
     const bq::SegView sv = lay.sv;
     const bool asym = !cfg.symmetric;
     if (sv.numel > 0 && !x) return BQ_ERR_INVALID_ARG;
@@ -144,6 +156,15 @@ bq_status quant_impl(int op, const void* x, const bq_qdesc* d, int gr, int32_t a
     }
     const DT dt = to_dt(d->x_dtype);
     cudaStream_t s = S(stream);
+    if (lay.column) {
+        // Column groups run in one pass over x for either mode; there are
+        // no range records to derive them from.
+        if (sv.n_seg == 0) return BQ_OK;
+        void* out = (op == bq::OP_QUANT) ? q : y;
+        const bool dyn = mode == BQ_SCALE_DYNAMIC;
+        return from_cuda(bq::col_groups(dt, op, dyn ? 1 : 0, x, nullptr, lay.cv, cfg, scale, zp,
+                                        dyn ? scale : nullptr, dyn ? zp : nullptr, out, s));
+    }
     if (sv.n_seg == 0) return BQ_OK;
     if (mode == BQ_SCALE_DYNAMIC && sv.G == 0) {
         return from_cuda(bq::empty_groups(sv.n_seg, cfg, scale, zp, s));
@@ -187,6 +208,9 @@ bq_status dequant_impl(const void* q, const float* scale, const void* zp, const 
     if (sv.numel == 0) return BQ_OK;
     if (!q || !scale || !y) return BQ_ERR_INVALID_ARG;
     if (!aligned(scale, 4) || !aligned(y, esize(y_dtype))) return BQ_ERR_MISALIGNED;
+    if (lay.column)
+        return from_cuda(bq::col_groups(to_dt(y_dtype), bq::OP_DEQ, 0, q, nullptr, lay.cv, cfg, scale,
+                                        zp, nullptr, nullptr, y, S(stream)));
     return from_cuda(bq::int_map(to_dt(y_dtype), bq::OP_DEQ, bq::PS_STATIC, q, nullptr, sv, cfg,
                                  scale, zp, nullptr, nullptr, nullptr, y, S(stream)));
 }
@@ -206,6 +230,9 @@ bq_status ste_impl(int op, const void* x, const void* dy, const float* scale, co
     const int64_t es = esize(d->x_dtype);
     if (!aligned(x, es) || !aligned(dy, es) || !aligned(dx, es) || !aligned(scale, 4))
         return BQ_ERR_MISALIGNED;
+    if (lay.column)
+        return from_cuda(bq::col_groups(to_dt(d->x_dtype), op, 0, x, dy, lay.cv, cfg, scale, zp,
+                                        nullptr, nullptr, dx, S(stream)));
     return from_cuda(bq::int_map(to_dt(d->x_dtype), op, bq::PS_STATIC, x, dy, sv, cfg, scale, zp,
                                  nullptr, nullptr, nullptr, dx, S(stream)));
 }
@@ -222,6 +249,9 @@ bq_status dequant_bwd_impl(const void* dy, const float* scale, const bq_qdesc* d
     if (!dy || !scale || !dq) return BQ_ERR_INVALID_ARG;
     const int64_t es = esize(d->x_dtype);
     if (!aligned(dy, es) || !aligned(dq, es) || !aligned(scale, 4)) return BQ_ERR_MISALIGNED;
+    if (lay.column)
+        return from_cuda(bq::col_groups(to_dt(d->x_dtype), bq::OP_DBWD, 0, dy, nullptr, lay.cv, cfg,
+                                        scale, nullptr, nullptr, nullptr, dq, S(stream)));
     return from_cuda(bq::int_map(to_dt(d->x_dtype), bq::OP_DBWD, bq::PS_STATIC, dy, nullptr, sv,
                                  cfg, scale, nullptr, nullptr, nullptr, nullptr, dq, S(stream)));
 }
@@ -231,6 +261,7 @@ int gran_to_gr(bq_gran g) {
         case BQ_GRAN_TENSOR: return GR_TENSOR;
         case BQ_GRAN_CHANNEL: return GR_CHANNEL;
         case BQ_GRAN_GROUP: return GR_GROUP;
+        case BQ_GRAN_COLUMN_GROUP: return GR_COLUMN;
     }
     return -1;
 }
@@ -256,6 +287,7 @@ const char* bq_granularity_name(bq_gran g) {
         case BQ_GRAN_TENSOR: return "tensor";
         case BQ_GRAN_CHANNEL: return "channel";
         case BQ_GRAN_GROUP: return "group";
+        case BQ_GRAN_COLUMN_GROUP: return "column_group";
     }
     return nullptr;
 }
@@ -284,7 +316,7 @@ size_t bq_quantize_workspace_size(const bq_qdesc* d, bq_gran gran, int32_t axis,
     const int gr = gran_to_gr(gran);
     Layout lay;
     if (gr < 0 || make_layout(d, gr, axis, group_size, &lay) != BQ_OK) return 0;
-    if (mode == BQ_SCALE_STATIC) return 0;
+    if (mode == BQ_SCALE_STATIC || lay.column) return 0;
     if (mode == BQ_SCALE_FROM_RANGE) return (size_t)lay.sv.n_seg * 16;
     return single_pass_possible(d, lay.sv) ? 0 : (size_t)lay.sv.n_seg * 16;
 }
@@ -296,7 +328,7 @@ bq_status bq_group_range(const void* x, const bq_qdesc* d, bq_gran gran, int32_t
     Layout lay;
     bq_status st = make_layout(d, gr, axis, group_size, &lay);
     if (st != BQ_OK) return st;
-    if (!is_float(d->x_dtype)) return BQ_ERR_UNSUPPORTED;
+    if (!is_float(d->x_dtype) || lay.column) return BQ_ERR_UNSUPPORTED;
     const bq::SegView sv = lay.sv;
     if (sv.n_seg == 0) return BQ_OK;
     if (!ranges || (sv.numel > 0 && !x)) return BQ_ERR_INVALID_ARG;
@@ -354,6 +386,12 @@ bq_status bq_quantize_per_group(const void* x, const bq_qdesc* d, int32_t axis,
     return quant_impl(bq::OP_QUANT, x, d, GR_GROUP, axis, group_size, q, scale, zp, mode,
                       nullptr, ws, ws_bytes, stream);
 }
+bq_status bq_quantize_per_column_group(const void* x, const bq_qdesc* d, int32_t axis,
+                                       int64_t group_size, void* q, float* scale, void* zp,
+                                       bq_scale_mode mode, void* stream) {
+    return quant_impl(bq::OP_QUANT, x, d, GR_COLUMN, axis, group_size, q, scale, zp, mode,
+                      nullptr, nullptr, 0, stream);
+}
 
 // ---- dequantize
 bq_status bq_dequantize_per_tensor(const void* q, const float* scale, const void* zp,
@@ -373,6 +411,11 @@ bq_status bq_dequantize_per_group(const void* q, const float* scale, const void*
                                   const bq_qdesc* d, int32_t axis, int64_t group_size, void* y,
                                   bq_dtype y_dtype, void* stream) {
     return dequant_impl(q, scale, zp, d, GR_GROUP, axis, group_size, y, y_dtype, stream);
+}
+bq_status bq_dequantize_per_column_group(const void* q, const float* scale, const void* zp,
+                                         const bq_qdesc* d, int32_t axis, int64_t group_size,
+                                         void* y, bq_dtype y_dtype, void* stream) {
+    return dequant_impl(q, scale, zp, d, GR_COLUMN, axis, group_size, y, y_dtype, stream);
 }
 
 // ---- fake quantize
@@ -406,6 +449,11 @@ bq_status bq_quantize_per_group_backward(const void* x, const void* dy, const fl
                                          int64_t group_size, void* dx, void* stream) {
     return ste_impl(bq::OP_QBWD, x, dy, scale, zp, d, GR_GROUP, axis, group_size, dx, stream);
 }
+bq_status bq_quantize_per_column_group_backward(const void* x, const void* dy, const float* scale,
+                                                const void* zp, const bq_qdesc* d, int32_t axis,
+                                                int64_t group_size, void* dx, void* stream) {
+    return ste_impl(bq::OP_QBWD, x, dy, scale, zp, d, GR_COLUMN, axis, group_size, dx, stream);
+}
 bq_status bq_fake_quantize_backward(const void* x, const void* dy, const float* scale,
                                     const void* zp, const bq_qdesc* d, bq_gran gran,
                                     int32_t axis, int64_t group_size, void* dx, void* stream) {
@@ -431,6 +479,11 @@ bq_status bq_dequantize_per_group_backward(const void* dy, const float* scale,
                                            const bq_qdesc* d, int32_t axis, int64_t group_size,
                                            void* dq, void* stream) {
     return dequant_bwd_impl(dy, scale, d, GR_GROUP, axis, group_size, dq, stream);
+}
+bq_status bq_dequantize_per_column_group_backward(const void* dy, const float* scale,
+                                                  const bq_qdesc* d, int32_t axis,
+                                                  int64_t group_size, void* dq, void* stream) {
+    return dequant_bwd_impl(dy, scale, d, GR_COLUMN, axis, group_size, dq, stream);
 }
 
 // ---- NVFP4

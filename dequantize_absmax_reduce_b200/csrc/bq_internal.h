@@ -53,6 +53,18 @@ cudaError_t int_map(DT dt, int op, int psrc, const void* a, const void* b, SegVi
                     const unsigned long long* ranges, float* scale_out, void* zp_out, void* out,
                     cudaStream_t st);
 
+// Column groups: x viewed as [outer, L, inner]; group (o, b, i) holds the gs
+// elements (o, b*gs + r, i), r < gs; scale / zp are [outer, L/gs, inner].
+struct ColView {
+    int64_t outer, L, inner, gs;
+};
+// Any op of int_map over column groups. dyn (OP_QUANT / OP_FAKE): the scale
+// and zero-point come from each group's range and are written to scale_out /
+// zp_out; otherwise they are read from scale_in / zp_in.
+cudaError_t col_groups(DT dt, int op, int dyn, const void* a, const void* b, ColView v, IntCfg cfg,
+                       const float* scale_in, const void* zp_in, float* scale_out, void* zp_out,
+                       void* out, cudaStream_t st);
+
 // Range records of every group (ranges cleared by the caller).
 cudaError_t seg_range(DT dt, const void* x, SegView sv, bool sym, unsigned long long* ranges,
                       cudaStream_t st);

@@ -46,8 +46,13 @@ bq_status scratch_on_current_device(void** out) {
 extern "C" bq_status bq_quantize_dynamic_noalloc(const void* x, const bq_qdesc* d, bq_gran gran,
                                                  int32_t axis, int64_t group_size, void* q,
                                                  float* scale, void* zp, void* stream) {
-    if (gran != BQ_GRAN_TENSOR && gran != BQ_GRAN_CHANNEL && gran != BQ_GRAN_GROUP)
+    if (gran != BQ_GRAN_TENSOR && gran != BQ_GRAN_CHANNEL && gran != BQ_GRAN_GROUP &&
+        gran != BQ_GRAN_COLUMN_GROUP)
         return BQ_ERR_INVALID_ARG;
+    // Column groups take one pass over x and no records.
+    if (gran == BQ_GRAN_COLUMN_GROUP)
+        return bq_quantize_per_column_group(x, d, axis, group_size, q, scale, zp, BQ_SCALE_DYNAMIC,
+                                            stream);
     int64_t n_groups = 0, group_elems = 0;
     bq_status st = bq_group_count(d, gran, axis, group_size, &n_groups, &group_elems);
     if (st != BQ_OK) return st;

@@ -28,4 +28,15 @@ struct PipeArgs {
     int static_global;  // 0: record from the range kernel before; 1: static; 2: caller's record
 };
 
+// Column groups with dynamic scales through the 2D-TMA ring (k_col_tma): x
+// row-major [rows, inner], groups of gs consecutive rows at one column.
+struct ColPipeArgs {
+    const void* x;
+    int64_t rows, inner, gs;
+    IntCfg cfg;
+    float* scale;       // [rows / gs, inner]
+    uint8_t* zp;        // [rows / gs, inner] or null
+    void* out;          // codes (quantize) or x's dtype (fake-quantize)
+};
+
 }  // namespace bq

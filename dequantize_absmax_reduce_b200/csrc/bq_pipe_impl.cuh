@@ -1870,6 +1870,392 @@ cudaError_t pipe_map_entry(int op, const MapArgs& m, cudaStream_t st) {
     return map_pipe_dt<T>(op, m.ranges ? PS_RANGE : PS_STATIC, m, st);
 }
 
+// ------------------------------------------------------------ column groups
+// Column groups (groups of GS consecutive rows at one column of a row-major
+// [rows, inner] tensor: the [K, N]-stored weight grouped along K) with
+// dynamic scales. Tiles of GS rows x CW columns (16 KB) reach shared memory
+// through 2D TMA into a ring of BQ_COL_STAGES slots; columns past `inner`
+// read as zero. A thread holds COL_RPT rows of one 16-byte column vector
+// (RS = GS / 4 lanes down the rows, CVN = 256 / RS vectors across), so a
+// tile's values sit in registers once and its slot is refilled before the
+// tile is reduced. The range runs down each column: packed 16-bit max / min
+// per thread, shuffles between the lanes of a column within a warp, then the
+// warps' partials through shared memory; one thread per column (pair)
+// derives the scale and zero-point, and the codes are encoded on f32 pairs.
+#ifndef BQ_COL_STAGES
+#define BQ_COL_STAGES 3
+#endif
+#ifndef BQ_COL_MINB
+#define BQ_COL_MINB 1
+#endif
+constexpr int COLT_RPT = 4;
+
+struct ColTileArgs {
+    int64_t inner, n_ct, n_tiles;
+    IntCfg cfg;
+    float* scale;
+    uint8_t* zp;
+    void* out;
+};
+
+template <class T, int GS> struct ColTileGeom {
+    static constexpr int W = Traits<T>::VEC;
+    static constexpr int RS = GS / COLT_RPT;            // lanes down the rows
+    static constexpr int CVN = 256 / RS;                // vectors across a tile row
+    static constexpr int CW = CVN * W;                  // columns per tile
+    static constexpr bool H = sizeof(T) == 2;
+    static constexpr int NP = H ? W / 2 : W;            // range words per thread
+    static constexpr int NWORDS = CVN * NP;             // range words per tile row
+    static constexpr uint32_t SLOT = (uint32_t)GS * CW * sizeof(T);
+    static constexpr int RED_OFF = 64;
+    static constexpr int PAR_OFF = RED_OFF + 2 * 8 * NWORDS * 4;
+    static constexpr int NPAR = 6;                      // per-column parameter arrays
+    static constexpr int RING_OFF = ((PAR_OFF + NPAR * CW * 4) + 1023) / 1024 * 1024;
+    static_assert(CW <= 256 && (CW * sizeof(T)) % 16 == 0, "TMA box");
+    static_assert(SLOT == 16384, "slot size");
+};
+
+template <class T>
+__device__ __forceinline__ uint32_t col_pk_max(uint32_t a, uint32_t b) {
+    if constexpr (sizeof(T) == 2) return pk_hi<T, false, false>(a, b);
+    else return __float_as_uint(fmaxf(__uint_as_float(a), __uint_as_float(b)));
+}
+template <class T>
+__device__ __forceinline__ uint32_t col_pk_min(uint32_t a, uint32_t b) {
+    if constexpr (sizeof(T) == 2) return pk_lo<T, false>(a, b);
+    else return __float_as_uint(fminf(__uint_as_float(a), __uint_as_float(b)));
+}
+// The two (16-bit) or one (f32) values of a range word.
+template <class T>
+__device__ __forceinline__ void col_word_vals(uint32_t w, float& v0, float& v1) {
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) unpack_bf16x2(w, v0, v1);
+    else if constexpr (std::is_same<T, __half>::value) unpack_f16x2(w, v0, v1);
+    else { v0 = __uint_as_float(w); v1 = 0.0f; }
+}
+
+template <class T, int OP, int GS>
+__global__ void __launch_bounds__(256, BQ_COL_MINB) k_col_tma(const __grid_constant__ CUtensorMap tm, ColTileArgs a) {
+    using G = ColTileGeom<T, GS>;
+    constexpr int W = G::W, RS = G::RS, CVN = G::CVN, CW = G::CW, NP = G::NP, NWORDS = G::NWORDS;
+    constexpr int S = BQ_COL_STAGES;
+    constexpr uint32_t SLOT = G::SLOT;
+    constexpr int NW = 8;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
+    uint32_t* red_hi = reinterpret_cast<uint32_t*>(smem + G::RED_OFF);      // [NW][NWORDS]
+    uint32_t* red_lo = red_hi + NW * NWORDS;
+    // Per-column parameters, each array [CW]: scale, -scale, RN(1/scale),
+    // qmin - zp, qmax - zp, zp (floats; a column pair reads as one 8-byte load).
+    float* cs = reinterpret_cast<float*>(smem + G::PAR_OFF);
+    float* cns = cs + CW;
+    float* cy = cns + CW;
+    float* clo = cy + CW;
+    float* chi = clo + CW;
+    float* czf = chi + CW;
+    uint8_t* ring = smem + G::RING_OFF;
+    const int tid = threadIdx.x;
+    const int cv = tid % CVN, rl = tid / CVN;
+    const int wid = tid >> 5, lane = tid & 31;
+    const int64_t grid = gridDim.x;
+    const float qlo = (float)a.cfg.qmin, qhi = (float)a.cfg.qmax;
+    const bool sym = a.cfg.symmetric != 0;
+    // Divisor of the scale: qmax (symmetric) or qmax - qmin.
+    const Recip Rq = make_recip(sym ? qhi : (float)(a.cfg.qmax - a.cfg.qmin));
+
+    if (tid == 0) {
+        for (int i = 0; i < S; ++i) mbar_init(smem_addr(&bars[i]), 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    auto issue = [&](int slot_i, int64_t tile) {
+        const uint32_t bar = smem_addr(&bars[slot_i]);
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(SLOT) : "memory");
+        tma_load_2d(smem_addr(ring + (size_t)slot_i * SLOT), &tm, (int)((tile % a.n_ct) * CW),
+                    (int)((tile / a.n_ct) * GS), bar);
+    };
+    if (tid == 0) {
+        for (int i = 0; i < S; ++i) {
+            const int64_t t = blockIdx.x + (int64_t)i * grid;
+            if (t >= a.n_tiles) break;
+            issue(i, t);
+        }
+    }
+
+    int slot = 0;
+    uint32_t parity = 0;
+    for (int64_t tile = blockIdx.x; tile < a.n_tiles; tile += grid) {
+        const bool ok = mbar_wait(smem_addr(&bars[slot]), parity);
+        const uint32_t sbase = smem_addr(ring + (size_t)slot * SLOT) + (uint32_t)(cv * 16);
+        U4 raw[COLT_RPT];
+#pragma unroll
+        for (int j = 0; j < COLT_RPT; ++j)
+            raw[j] = ld_shared16(sbase + (uint32_t)((rl + j * RS) * CW * (int)sizeof(T)));
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) {
+                atomicOr(&g_pipe_error, 1u);
+                int s2 = slot;
+                uint32_t p2 = parity;
+                for (int i = 0; i < S; ++i) {
+                    const int64_t t2 = tile + (int64_t)i * grid;
+                    if (t2 >= a.n_tiles) break;
+                    mbar_wait(smem_addr(&bars[s2]), p2);
+                    if (++s2 == S) { s2 = 0; p2 ^= 1u; }
+                }
+            }
+            __syncthreads();
+            return;
+        }
+        // Every thread holds its vectors: refill the slot with tile + S now.
+        if (tid == 0) {
+            const int64_t next = tile + (int64_t)S * grid;
+            if (next < a.n_tiles) {
+                fence_proxy_async();
+                issue(slot, next);
+            }
+        }
+        if (++slot == S) { slot = 0; parity ^= 1u; }
+
+        const int64_t ct = tile % a.n_ct, ob = tile / a.n_ct;
+        const int64_t col0 = ct * CW;
+        // ---- range of this thread's columns over its rows (NaN skipped)
+        uint32_t hw[NP], lw[NP];
+#pragma unroll
+        for (int p = 0; p < NP; ++p) {
+            uint32_t h = 0u, l = 0u;
+#pragma unroll
+            for (int j = 0; j < COLT_RPT; ++j) {
+                const uint32_t wj[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+                h = col_pk_max<T>(h, wj[p]);
+                l = col_pk_min<T>(l, wj[p]);
+            }
+            hw[p] = h;
+            lw[p] = l;
+        }
+#pragma unroll
+        for (int o = CVN; o < 32; o <<= 1) {
+#pragma unroll
+            for (int p = 0; p < NP; ++p) {
+                hw[p] = col_pk_max<T>(hw[p], __shfl_xor_sync(0xffffffffu, hw[p], o));
+                lw[p] = col_pk_min<T>(lw[p], __shfl_xor_sync(0xffffffffu, lw[p], o));
+            }
+        }
+        if (lane < CVN) {
+#pragma unroll
+            for (int p = 0; p < NP; ++p) {
+                red_hi[wid * NWORDS + cv * NP + p] = hw[p];
+                red_lo[wid * NWORDS + cv * NP + p] = lw[p];
+            }
+        }
+        __syncthreads();
+        // ---- one thread per range word: the tile's column parameters
+        bool slow_col = false;
+        if (tid < NWORDS) {
+            uint32_t h = red_hi[tid], l = red_lo[tid];
+#pragma unroll
+            for (int w = 1; w < NW; ++w) {
+                h = col_pk_max<T>(h, red_hi[w * NWORDS + tid]);
+                l = col_pk_min<T>(l, red_lo[w * NWORDS + tid]);
+            }
+            float h0, h1, l0, l1;
+            col_word_vals<T>(h, h0, h1);
+            col_word_vals<T>(l, l0, l1);
+            constexpr int CPW = G::H ? 2 : 1;     // columns per word
+#pragma unroll
+            for (int u = 0; u < CPW; ++u) {
+                const int c = tid * CPW + u;
+                // Scale fl(amax/qmax) or fl(fl(max'-min')/(qmax-qmin)) and
+                // zero-point, each quotient through a reciprocal chain
+                // (exact for a normal dividend; IEEE division outside).
+                const float hi = u ? h1 : h0, nlo = -(u ? l1 : l0);
+                const float num = sym ? fmaxf(hi, nlo) : __fadd_rn(hi, nlo);
+                float sc = (num >= 0x1p-100f && num <= 0x1p100f) ? div_chain(num, Rq) : div_slow(num, Rq.s);
+                if (sc == 0.0f) sc = 1.0f;
+                const Recip R = make_recip(sc);
+                int zp = 0;
+                if (!sym) {
+                    const float m = R.fast ? div_chain(-nlo, R) : __fdiv_rn(-nlo, sc);
+                    const float zf = fminf(fmaxf(__fsub_rn(qlo, rintf(m)), qlo), qhi);   // NaN -> qmin
+                    zp = (int)zf;
+                }
+                cs[c] = sc;
+                cns[c] = -sc;
+                cy[c] = R.y;
+                clo[c] = qlo - (float)zp;
+                chi[c] = qhi - (float)zp;
+                czf[c] = (float)zp;
+                slow_col = slow_col || !R.fast;
+                if (col0 + c < a.inner) {
+                    a.scale[ob * a.inner + col0 + c] = sc;
+                    if (a.zp) a.zp[ob * a.inner + col0 + c] = (uint8_t)zp;
+                }
+            }
+        }
+        // The barrier also tells every thread whether a scale of this tile
+        // lies outside the reciprocal chain's range.
+        const bool tile_slow = __syncthreads_or(slow_col) != 0;
+        if (col0 + cv * W >= a.inner) continue;
+
+        // ---- codes: each column pair on f32 pairs
+        const int64_t obase = (ob * GS + rl) * a.inner + col0 + cv * W;
+        if (!tile_slow) {
+            uint32_t cwd[COLT_RPT][(W + 3) / 4];
+            uint32_t ow[COLT_RPT][4];
+            const F2 magic2 = f2_bcast(kMagic);
+#pragma unroll
+            for (int p = 0; p < W / 2; ++p) {
+                const int c = cv * W + 2 * p;
+                const float2 lo = *reinterpret_cast<const float2*>(clo + c);
+                const float2 hi = *reinterpret_cast<const float2*>(chi + c);
+                Recip2 R2;
+                R2.y = *reinterpret_cast<const F2*>(cy + c);
+                R2.ns = *reinterpret_cast<const F2*>(cns + c);
+                const F2 zf2 = *reinterpret_cast<const F2*>(czf + c);
+                const F2 s2 = *reinterpret_cast<const F2*>(cs + c);
+#pragma unroll
+                for (int j = 0; j < COLT_RPT; ++j) {
+                    F2 xp[W / 2];
+                    widen_pairs<T>(raw[j], xp);
+                    float q0, q1;
+                    f2_split(div_chain2(xp[p], R2), q0, q1);
+                    q0 = fminf(fmaxf(q0, lo.x), hi.x);        // NaN -> qmin
+                    q1 = fminf(fmaxf(q1, lo.y), hi.y);
+                    const F2 t = f2_add(f2_pack(q0, q1), magic2);   // round(q) + 1.5 * 2^23
+                    if constexpr (OP == OP_QUANT) {
+                        uint32_t b0, b1;
+                        f2_split_bits(f2_add(t, zf2), b0, b1);      // + zp, exact; low byte = code
+                        const uint32_t pair = __byte_perm(b0, b1, 0x0040);  // codes in bytes 0, 1
+                        uint32_t& wd = cwd[j][(2 * p) / 4];
+                        wd = ((2 * p) % 4 == 0) ? pair : __byte_perm(wd, pair, 0x5410);
+                    } else {
+                        float o0, o1;
+                        f2_split(f2_mul(f2_sub(t, magic2), s2), o0, o1);
+                        if constexpr (sizeof(T) == 2) {
+                            ow[j][p] = std::is_same<T, __nv_bfloat16>::value ? pack_bf16x2(o0, o1) : pack_f16x2(o0, o1);
+                        } else {
+                            ow[j][2 * p] = __float_as_uint(o0);
+                            ow[j][2 * p + 1] = __float_as_uint(o1);
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < COLT_RPT; ++j) {
+                const int64_t e = obase + (int64_t)j * RS * a.inner;
+                if constexpr (OP == OP_QUANT) {
+                    if constexpr (W == 8) st8((uint8_t*)a.out + e, cwd[j][0], cwd[j][1]);
+                    else st4((uint8_t*)a.out + e, cwd[j][0]);
+                } else {
+                    st16((T*)a.out + e, U4{ow[j][0], ow[j][1], ow[j][2], ow[j][3]});
+                }
+            }
+        } else {
+            // A scale outside the reciprocal chain's range (tiny or infinite):
+            // IEEE division per element.
+#pragma unroll
+            for (int j = 0; j < COLT_RPT; ++j) {
+                float v[W], o[W];
+                uint32_t code[W];
+                load_vec<T>(raw[j], v);
+#pragma unroll
+                for (int k = 0; k < W; ++k) {
+                    const int c = cv * W + k;
+                    IntParams ip = make_int_params(a.cfg.qmin, a.cfg.qmax, (int)czf[c]);
+                    Recip R;
+                    R.s = cs[c];
+                    R.y = cy[c];
+                    const float m = fabsf(R.s);
+                    R.fast = (m >= 0x1p-64f) && (m <= 0x1p64f);
+                    const float t = rounded_rne(div_any(v[k], R), ip);
+                    code[k] = code_from_rounded(t, ip.zp);
+                    o[k] = dequant_from_rounded(t, R.s);
+                }
+                const int64_t e = obase + (int64_t)j * RS * a.inner;
+                if constexpr (OP == OP_QUANT) {
+                    if constexpr (W == 8) st8((uint8_t*)a.out + e, pack4_lowbytes(code[0], code[1], code[2], code[3]),
+                                              pack4_lowbytes(code[4], code[5], code[6], code[7]));
+                    else st4((uint8_t*)a.out + e, pack4_lowbytes(code[0], code[1], code[2], code[3]));
+                } else {
+                    st16((T*)a.out + e, pack_vec<T>(o));
+                }
+            }
+        }
+    }
+}
+
+// Tensor map of a row-major [rows, cols] tensor of 2- or 4-byte elements in
+// boxes of box_rows x box_cols, zero fill outside (no multicast).
+static cudaError_t encode_map_2d(CUtensorMap* tm, const void* x, int64_t rows, int64_t cols, int esz,
+                                 uint32_t box_cols, uint32_t box_rows) {
+    static const PFN_cuTensorMapEncodeTiled_v12000 encode = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess) {
+            (void)cudaGetLastError();
+            p = nullptr;
+        }
+        return (PFN_cuTensorMapEncodeTiled_v12000)p;
+    }();
+    if (!encode) return cudaErrorNotSupported;
+    const cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t gstride[1] = {(cuuint64_t)cols * (cuuint64_t)esz};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estride[2] = {1, 1};
+    const CUresult r = encode(tm, esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT32,
+                              2, const_cast<void*>(x), gdim, gstride, box, estride,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorNotSupported;
+}
+
+template <class T, int OP, int GS>
+static cudaError_t col_tma_launch(const ColPipeArgs& p, cudaStream_t st) {
+    using G = ColTileGeom<T, GS>;
+    ColTileArgs a;
+    a.inner = p.inner;
+    a.n_ct = (p.inner + G::CW - 1) / G::CW;
+    a.n_tiles = (p.rows / GS) * a.n_ct;
+    a.cfg = p.cfg;
+    a.scale = p.scale;
+    a.zp = p.zp;
+    a.out = p.out;
+    CUtensorMap tm;
+    const cudaError_t me = encode_map_2d(&tm, p.x, p.rows, p.inner, (int)sizeof(T), G::CW, GS);
+    if (me != cudaSuccess) return me;
+    const size_t smem = (size_t)G::RING_OFF + (size_t)BQ_COL_STAGES * G::SLOT;
+    auto k = k_col_tma<T, OP, GS>;
+    static const cudaError_t attr = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (attr != cudaSuccess) return attr;
+    static unsigned long long occ[8];
+    const int bps = occupancy_for((const void*)k, smem, occ);
+    if (bps < 1) return cudaErrorNotSupported;
+    int64_t grid = (int64_t)sm_count() * bps;
+    if (grid > a.n_tiles) grid = a.n_tiles;
+    if (grid < 1) grid = 1;
+    k<<<(unsigned)grid, 256, smem, st>>>(tm, a);
+    return cudaGetLastError();
+}
+
+// Column groups with dynamic scales through k_col_tma: 16-bit or f32 x, gs
+// in {32, 64, 128, 256}, round-to-nearest-even, whole vectors per row,
+// aligned operands; cudaErrorNotSupported otherwise.
+template <class T>
+static cudaError_t col_tma_entry(int op, const ColPipeArgs& p, cudaStream_t st) {
+    constexpr int W = Traits<T>::VEC;
+    if (sizeof(T) == 8 || p.cfg.rhaz || (op != OP_QUANT && op != OP_FAKE)) return cudaErrorNotSupported;
+    if (p.inner % W != 0 || ((uintptr_t)p.x & 15u)) return cudaErrorNotSupported;
+    if (op == OP_QUANT ? ((uintptr_t)p.out % W) != 0 : ((uintptr_t)p.out & 15u) != 0) return cudaErrorNotSupported;
+    if (p.rows <= 0 || p.inner <= 0 || p.rows > 0x7FFFFF00ll || p.inner > 0x7FFFFF00ll) return cudaErrorNotSupported;
+    if (p.rows % p.gs != 0) return cudaErrorNotSupported;
+    switch (p.gs) {
+        case 32: return op == OP_QUANT ? col_tma_launch<T, OP_QUANT, 32>(p, st) : col_tma_launch<T, OP_FAKE, 32>(p, st);
+        case 64: return op == OP_QUANT ? col_tma_launch<T, OP_QUANT, 64>(p, st) : col_tma_launch<T, OP_FAKE, 64>(p, st);
+        case 128: return op == OP_QUANT ? col_tma_launch<T, OP_QUANT, 128>(p, st) : col_tma_launch<T, OP_FAKE, 128>(p, st);
+        case 256: return op == OP_QUANT ? col_tma_launch<T, OP_QUANT, 256>(p, st) : col_tma_launch<T, OP_FAKE, 256>(p, st);
+    }
+    return cudaErrorNotSupported;
+}
+
 template <class T>
 cudaError_t pipe_error_entry(unsigned int* flag) {
     unsigned int zero = 0;
@@ -1899,6 +2285,9 @@ cudaError_t pipe_error_entry(unsigned int* flag) {
     cudaError_t pipe_fp8t_##NAME(const void* x, int64_t n, uint8_t* e4m3, float* scale,           \
                                  const unsigned long long* rec, int from_rec, cudaStream_t st) {  \
         return fp8t_entry<T>(x, n, e4m3, scale, rec, from_rec, st);                              \
+    }                                                                                            \
+    cudaError_t pipe_col_##NAME(int op, const ColPipeArgs& p, cudaStream_t st) {                 \
+        return col_tma_entry<T>(op, p, st);                                                      \
     }
 
 }  // namespace bq

@@ -74,8 +74,20 @@ typedef enum bq_dtype {
 typedef enum bq_round { BQ_RNE = 0, BQ_RHAZ = 1 } bq_round;
 
 /* [granularity] Granularity. Per-token is PerChannel on the second-to-last
- * axis and has its own entry points. */
-typedef enum bq_gran { BQ_GRAN_TENSOR = 0, BQ_GRAN_CHANNEL = 1, BQ_GRAN_GROUP = 2 } bq_gran;
+ * axis and has its own entry points.
+ * BQ_GRAN_COLUMN_GROUP: the Group granularity read for a weight stored
+ * [K, N] and grouped along K (the GPTQ / AWQ layout of the baracuda quantize
+ * module's per-group weight quantization): with x viewed as [outer, L, inner]
+ * around `axis`, group (o, b, i) holds the group_size elements
+ * x[o, b*gs + r, i], r < gs, which lie `inner` elements apart; scale / zp are
+ * [outer, L/gs, inner] row-major. Accepted by bq_group_count,
+ * bq_quantize_workspace_size (always 0), bq_fake_quantize (DYNAMIC and
+ * STATIC), bq_fake_quantize_backward, bq_quantize_dynamic_noalloc and the
+ * *_per_column_group entry points; bq_group_range and FROM_RANGE scaling
+ * return BQ_ERR_UNSUPPORTED for it. */
+typedef enum bq_gran {
+    BQ_GRAN_TENSOR = 0, BQ_GRAN_CHANNEL = 1, BQ_GRAN_GROUP = 2, BQ_GRAN_COLUMN_GROUP = 3
+} bq_gran;
 
 /* Where the per-group scale / zero-point come from.
  *   DYNAMIC:    derived from each group's range and written to scale / zp.
@@ -112,8 +124,8 @@ typedef struct bq_qdesc {
 /* Human-readable name of a status code (static storage). */
 const char* bq_status_string(bq_status s);
 
-/* [granularity] strategy_name(): "tensor", "channel" or "group"; NULL for an
- * unknown value. */
+/* [granularity] strategy_name(): "tensor", "channel" or "group"
+ * ("column_group" for BQ_GRAN_COLUMN_GROUP); NULL for an unknown value. */
 const char* bq_granularity_name(bq_gran g);
 
 /* [baracuda] default_q_range: S8 -> [-128, 127], U8 -> [0, 255]. Host only. */
@@ -124,6 +136,7 @@ bq_status bq_default_q_range(bq_dtype q_dtype, int32_t* qmin, int32_t* qmax);
  * index o holds axis indices [g*gs, (g+1)*gs) and every index of the
  * dimensions after `axis`, i.e. one contiguous run of gs * prod(shape[axis+1:])
  * elements. PerTensor is one group; PerChannel{axis} is Group{axis, 1}.
+ * Column groups: outer * (L/gs) * inner groups of gs elements each.
  * Host only. */
 bq_status bq_group_count(const bq_qdesc* d, bq_gran gran, int32_t axis, int64_t group_size,
                          int64_t* n_groups, int64_t* group_elems);
@@ -175,6 +188,12 @@ bq_status bq_quantize_per_token(const void* x, const bq_qdesc* d, void* q, float
 bq_status bq_quantize_per_group(const void* x, const bq_qdesc* d, int32_t axis,
                                 int64_t group_size, void* q, float* scale, void* zp,
                                 bq_scale_mode mode, void* ws, size_t ws_bytes, void* stream);
+/* Column groups (BQ_GRAN_COLUMN_GROUP): scale / zp [outer, L/gs, inner];
+ * mode DYNAMIC or STATIC (FROM_RANGE: BQ_ERR_UNSUPPORTED). One pass over x,
+ * no workspace. Otherwise as bq_quantize_per_group. */
+bq_status bq_quantize_per_column_group(const void* x, const bq_qdesc* d, int32_t axis,
+                                       int64_t group_size, void* q, float* scale, void* zp,
+                                       bq_scale_mode mode, void* stream);
 
 /* Dynamic quantize without caller workspace. The sources cited above have no
  * counterpart: this is a library convenience for callers that cannot hand
@@ -222,6 +241,9 @@ bq_status bq_dequantize_per_token(const void* q, const float* scale, const void*
 bq_status bq_dequantize_per_group(const void* q, const float* scale, const void* zp,
                                   const bq_qdesc* d, int32_t axis, int64_t group_size, void* y,
                                   bq_dtype y_dtype, void* stream);
+bq_status bq_dequantize_per_column_group(const void* q, const float* scale, const void* zp,
+                                         const bq_qdesc* d, int32_t axis, int64_t group_size,
+                                         void* y, bq_dtype y_dtype, void* stream);
 
 /* --------------------------------------------------------- fake quantize */
 /* [baracuda] fake_quantize ("FP roundtrip"): y = dequantize(quantize(x)) in
@@ -248,6 +270,9 @@ bq_status bq_quantize_per_token_backward(const void* x, const void* dy, const fl
 bq_status bq_quantize_per_group_backward(const void* x, const void* dy, const float* scale,
                                          const void* zp, const bq_qdesc* d, int32_t axis,
                                          int64_t group_size, void* dx, void* stream);
+bq_status bq_quantize_per_column_group_backward(const void* x, const void* dy, const float* scale,
+                                                const void* zp, const bq_qdesc* d, int32_t axis,
+                                                int64_t group_size, void* dx, void* stream);
 
 /* [baracuda] fake_quantize_backward via STE: dx = dy * m (m as above). */
 bq_status bq_fake_quantize_backward(const void* x, const void* dy, const float* scale,
@@ -267,6 +292,9 @@ bq_status bq_dequantize_per_token_backward(const void* dy, const float* scale,
 bq_status bq_dequantize_per_group_backward(const void* dy, const float* scale,
                                            const bq_qdesc* d, int32_t axis, int64_t group_size,
                                            void* dq, void* stream);
+bq_status bq_dequantize_per_column_group_backward(const void* dy, const float* scale,
+                                                  const bq_qdesc* d, int32_t axis,
+                                                  int64_t group_size, void* dq, void* stream);
 
 /* ----------------------------------------------------------------- NVFP4 */
 /* [QuantizedWeight] NVFP4 quantize of x [n, k] (F32, F16 or BF16), k % 16 == 0:

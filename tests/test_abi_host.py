@@ -60,6 +60,13 @@ def test_group_count_matches_reading(B):
     assert B.bq_group_count(d, "channel", 2) == (240, 1)
     assert B.bq_group_count(d, "group", 1, 3) == (8, 30)
     assert B.bq_group_count(d, "group", 2, 5) == (48, 5)
+    # column groups: one per (outer, block, inner index), gs elements each
+    assert B.bq_group_count(d, "column_group", 1, 3) == (4 * 2 * 10, 3)
+    assert B.bq_group_count(d, "column_group", 0, 2) == (2 * 60, 2)
+    assert B.bq_group_count(d, "column_group", 2, 5) == B.bq_group_count(d, "group", 2, 5)
+    assert B.bq_granularity_name("column_group") == "column_group"
+    with pytest.raises(B.BqError):
+        B.bq_group_count(d, "column_group", 1, 4)
     with pytest.raises(B.BqError):
         B.bq_group_count(d, "group", 1, 4)          # 4 does not divide 6
     with pytest.raises(B.BqError):
@@ -76,6 +83,8 @@ def test_workspace_size(B):
     assert B.bq_quantize_workspace_size(d64, "channel", 0) == 16 * 8
     drh = B.make_desc((8, 64), torch.float32, rnd="rhaz")
     assert B.bq_quantize_workspace_size(drh, "channel", 0) == 16 * 8
+    for mode in ("dynamic", "static", "from_range"):           # one pass, no records
+        assert B.bq_quantize_workspace_size(d, "column_group", 0, 128, mode) == 0
 
 
 def _status(fn):
@@ -121,6 +130,17 @@ def test_argument_errors_return_status_without_launching(B):
     assert B.lib.bq_packed_transpose(P, P, 4, 31, 16, 16, P, P, C.byref(st64), None) == B.BQ_ERR_INVALID_ARG
     assert B.lib.bq_packed_transpose(P, P, 4, 32, 5, 16, P, P, C.byref(st64), None) == B.BQ_ERR_INVALID_ARG
     assert B.lib.bq_packed_transpose(P, None, 4, 32, 16, 16, P, P, C.byref(st64), None) == B.BQ_ERR_INVALID_ARG
+    # column groups: no range records, group_size must divide the axis
+    dc = B.make_desc((64, 48), torch.float32)
+    assert B.lib.bq_quantize_per_column_group(P, C.byref(dc), 0, 16, P, P, P, 2, None) == B.BQ_ERR_UNSUPPORTED
+    assert B.lib.bq_quantize_per_column_group(P, C.byref(dc), 0, 48, P, P, P, 0, None) == B.BQ_ERR_INVALID_ARG
+    assert B.lib.bq_quantize_per_column_group(P, C.byref(dc), 2, 1, P, P, P, 0, None) == B.BQ_ERR_INVALID_ARG
+    assert B.lib.bq_quantize_per_column_group(P + 2, C.byref(dc), 0, 16, P, P, P, 0, None) == B.BQ_ERR_MISALIGNED
+    assert B.lib.bq_group_range(P, C.byref(dc), B.BQ_GRAN_COLUMN_GROUP, 0, 16, P, None) == B.BQ_ERR_UNSUPPORTED
+    assert B.lib.bq_dequantize_per_column_group(P, P, None, C.byref(dc), 0, 48, P, B.BQ_F32, None) == B.BQ_ERR_INVALID_ARG
+    assert B.lib.bq_quantize_per_column_group_backward(P, P, P, None, C.byref(da), 0, 3, P, None) == B.BQ_ERR_INVALID_ARG
+    assert B.lib.bq_dequantize_per_column_group_backward(P, P, C.byref(dc), 0, 5, P, None) == B.BQ_ERR_INVALID_ARG
+    assert B.lib.bq_quantize_dynamic_noalloc(P, C.byref(dc), 9, 0, 16, P, P, P, None) == B.BQ_ERR_INVALID_ARG
     # descriptor errors
     d9 = B.make_desc((4, 64), torch.float32)
     d9.ndim = 9
@@ -136,6 +156,8 @@ def test_empty_calls_succeed_without_a_device(B):
     assert B.lib.bq_quantize_per_token(None, C.byref(d), None, None, None, 0, None, 0, None) == B.BQ_OK
     assert B.lib.bq_dequantize_per_token(None, None, None, C.byref(d), None, B.BQ_F32, None) == B.BQ_OK
     assert B.lib.bq_mxfp8_quantize(None, B.BQ_BF16, 0, 64, None, None, None) == B.BQ_OK
+    assert B.lib.bq_quantize_per_column_group(None, C.byref(d), 0, 1, None, None, None, 0, None) == B.BQ_OK
+    assert B.lib.bq_dequantize_per_column_group(None, None, None, C.byref(d), 1, 4, None, B.BQ_F32, None) == B.BQ_OK
 
 
 def test_weight_prep_argument_errors(B):
