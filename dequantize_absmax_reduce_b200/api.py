@@ -187,6 +187,16 @@ def nvfp4_quantize(x, s2=None, stream=None):
     return packed, sc, gs
 
 
+def nvfp4_quantize_activation(x, input_scale, stream=None):
+    """NVFP4 activations with a static per-tensor input scale (the f32 device
+    tensor a checkpoint holds as input_scale): (packed, scale_e4m3)."""
+    n, k = x.shape
+    packed = torch.empty((n, k // 2), dtype=torch.uint8, device=x.device)
+    sc = torch.empty((n, k // 16), dtype=torch.uint8, device=x.device)
+    B.bq_nvfp4_quantize(x, packed, sc, input_scale, True, None, stream)
+    return packed, sc
+
+
 def nvfp4_dequantize(packed, sc, s2, ydtype=torch.bfloat16, stream=None):
     n, kb = packed.shape
     y = torch.empty((n, 2 * kb), dtype=ydtype, device=packed.device)

@@ -302,7 +302,10 @@ bq_status bq_dequantize_per_column_group_backward(const void* dy, const float* s
  *   (static_global == 0) or taken from the range record in ws
  *   (static_global == 2: as written by bq_group_range with BQ_GRAN_TENSOR,
  *   possibly combined across shards with an integer MAX); or s2 =
- *   *global_scale, an input (static_global == 1);
+ *   *global_scale, an input (static_global == 1): this is also how NVFP4
+ *   activations are quantized with a static [QuantizedWeight] input_scale
+ *   ("input activation scale on the device"): pass that device pointer as
+ *   global_scale; it is read, never written;
  *   per 16 consecutive elements of a row: sb = E4M3(fl(a_b / fl(6 * s2))),
  *   eff = fl(E4M3(sb) * s2), code = E2M1(fl(x / eff)) (all codes 0 when
  *   eff == 0).

@@ -356,3 +356,20 @@ def test_workload_fp8_tensor_codec(bq, orc):
     assert_bitwise(e, re, "codes")
     y = bq.fp8_tensor_dequantize(e, s, torch.bfloat16)
     assert_bitwise(y, orc.fp8_tensor_dequantize(re, rs, ydtype="bf16"), "load")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_nvfp4_activation_with_static_input_scale(bq, orc, dtype):
+    # QuantizedWeight input_scale: a per-tensor activation scale calibrated
+    # beforehand (here from another batch, amax / 2688) and held on the
+    # device; this batch has larger outliers, so some blocks saturate.
+    st = synthetic.Stream(61)
+    calib = st.tensor((64, 512), dtype)
+    x = st.tensor((96, 512), dtype, outlier_p=0.01, outlier_factor=40)
+    s_in = float(np.float32(orc.tensor_amax(calib) / 2688.0))
+    input_scale = torch.tensor([s_in], dtype=torch.float32, device="cuda")
+    packed, sc = bq.nvfp4_quantize_activation(x.cuda(), input_scale)
+    rp, rsc, _ = orc.nvfp4_quantize(x, s2=s_in)
+    assert_bitwise(packed, rp, "packed")
+    assert_bitwise(sc, rsc, "block scales")
+    assert input_scale.item() == s_in          # read, never written
