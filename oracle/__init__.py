@@ -22,7 +22,12 @@ import torch
 
 from . import build as _build
 
-_T = {"f32": 0, "f64": 1, "f16": 2, "bf16": 3, "s8": 4, "u8": 5}
+_T = {"f32": 0, "f64": 1, "f16": 2, "bf16": 3, "s8": 4, "u8": 5, "s4": 6, "u4": 7}
+# s4 / u4: two codes per byte (element 2j in the low nibble), held in a u8
+# tensor whose last dimension is half the logical one; zero-points one byte
+# per group (s8 for s4, u8 for u4).
+_PACKED = ("s4", "u4")
+_ZP = {"s8": torch.int8, "u8": torch.uint8, "s4": torch.int8, "u4": torch.uint8}
 _TORCH = {"f32": torch.float32, "f64": torch.float64, "f16": torch.float16,
           "bf16": torch.bfloat16, "s8": torch.int8, "u8": torch.uint8}
 _NAME = {v: k for k, v in _TORCH.items()}
@@ -140,7 +145,12 @@ def quantize(x: torch.Tensor, gran: str, axis: int = 0, gs: int = 1, qdtype: str
     (hi, neg_lo) f64 tensors per group to derive the scale from them."""
     x = _c(x)
     ng, _ = group_count(tuple(x.shape), gran, axis, gs)
-    q = torch.zeros(x.shape, dtype=_TORCH[qdtype])
+    if qdtype in _PACKED:
+        if x.dim() < 1 or x.shape[-1] % 2:
+            raise OracleError("packed 4-bit codes need an even last dimension")
+        q = torch.zeros(tuple(x.shape[:-1]) + (x.shape[-1] // 2,), dtype=torch.uint8)
+    else:
+        q = torch.zeros(x.shape, dtype=_TORCH[qdtype])
     mode = 0
     if scale is not None:
         mode = 1
@@ -148,7 +158,7 @@ def quantize(x: torch.Tensor, gran: str, axis: int = 0, gs: int = 1, qdtype: str
         zp = None if zp is None else _c(zp).clone()
     else:
         scale = torch.zeros(ng, dtype=torch.float32)
-        zp = torch.zeros(ng, dtype=_TORCH[qdtype])
+        zp = torch.zeros(ng, dtype=_ZP[qdtype])
         if ranges is not None:
             mode = 2
     hi = nlo = None
@@ -163,11 +173,18 @@ def quantize(x: torch.Tensor, gran: str, axis: int = 0, gs: int = 1, qdtype: str
 
 
 def dequantize(q: torch.Tensor, scale: torch.Tensor, zp: torch.Tensor | None, gran: str,
-               axis: int = 0, gs: int = 1, ydtype: str = "f32") -> torch.Tensor:
+               axis: int = 0, gs: int = 1, ydtype: str = "f32", qdtype: str | None = None) -> torch.Tensor:
+    """qdtype "s4" / "u4": q holds packed codes (last dimension halved)."""
     q = _c(q)
-    y = torch.zeros(q.shape, dtype=_TORCH[ydtype])
-    nd, sh = _shape(q)
-    _ok(lib().or_dequantize(_p(q), C.c_int(_dt(q)), _p(_c(scale)), _p(None if zp is None else _c(zp)),
+    if qdtype in _PACKED:
+        shape = tuple(q.shape[:-1]) + (2 * q.shape[-1],)
+        qt = _T[qdtype]
+    else:
+        shape = tuple(q.shape)
+        qt = _dt(q)
+    y = torch.zeros(shape, dtype=_TORCH[ydtype])
+    nd, sh = _shape(y)
+    _ok(lib().or_dequantize(_p(q), C.c_int(qt), _p(_c(scale)), _p(None if zp is None else _c(zp)),
                             nd, sh, C.c_int(_GRAN[gran]), C.c_int(axis), C.c_int64(gs), _p(y),
                             C.c_int(_T[ydtype])), "dequantize")
     return y
@@ -187,7 +204,7 @@ def fake_quantize(x: torch.Tensor, gran: str, axis: int = 0, gs: int = 1, qdtype
         zp = None if zp is None else _c(zp).clone()
     else:
         scale = torch.zeros(ng, dtype=torch.float32)
-        zp = torch.zeros(ng, dtype=_TORCH[qdtype])
+        zp = torch.zeros(ng, dtype=_ZP[qdtype])
         if ranges is not None:
             mode = 2
     hi = nlo = None

@@ -67,7 +67,10 @@ namespace {
 
 // ---------------------------------------------------------------------------
 // Element types understood by the oracle (its own numbering).
-enum OrType { OR_F32 = 0, OR_F64 = 1, OR_F16 = 2, OR_BF16 = 3, OR_S8 = 4, OR_U8 = 5 };
+// OR_S4 / OR_U4: 4-bit codes packed two per byte, element 2j in the low
+// nibble of byte j (the nibble order of packed E2M1 on the QuantizedWeight
+// page); their zero-points are stored one per byte (s8 / u8).
+enum OrType { OR_F32 = 0, OR_F64 = 1, OR_F16 = 2, OR_BF16 = 3, OR_S8 = 4, OR_U8 = 5, OR_S4 = 6, OR_U4 = 7 };
 
 // ---------------------------------------------------------------------------
 // Small floating-point formats, decoded from their bit-field definitions:
@@ -193,11 +196,24 @@ void store_f(void* p, int t, int64_t i, double v) {
     }
 }
 int64_t load_i(const void* p, int t, int64_t i) {
+    if (t == OR_S4 || t == OR_U4) {
+        const int nib = (((const uint8_t*)p)[i / 2] >> (4 * (i % 2))) & 0xF;
+        return (t == OR_S4 && nib >= 8) ? nib - 16 : nib;
+    }
     return t == OR_S8 ? (int64_t)((const int8_t*)p)[i] : (int64_t)((const uint8_t*)p)[i];
 }
 void store_i(void* p, int t, int64_t i, int64_t v) {
+    if (t == OR_S4 || t == OR_U4) {
+        uint8_t& b = ((uint8_t*)p)[i / 2];
+        const int sh = 4 * (int)(i % 2);
+        b = (uint8_t)((b & ~(0xF << sh)) | (((int)v & 0xF) << sh));
+        return;
+    }
     if (t == OR_S8) ((int8_t*)p)[i] = (int8_t)v; else ((uint8_t*)p)[i] = (uint8_t)v;
 }
+bool is_int_type(int t) { return t == OR_S8 || t == OR_U8 || t == OR_S4 || t == OR_U4; }
+// Zero-points of a code type: one byte per group (s8 for signed codes).
+int zp_type(int q_t) { return (q_t == OR_S8 || q_t == OR_S4) ? OR_S8 : OR_U8; }
 
 // ---------------------------------------------------------------------------
 // Rounding a real value to an integer.
@@ -300,6 +316,10 @@ bool default_range(int q_t, int64_t* qmin, int64_t* qmax) {
     // [baracuda] default_q_range: S8 -> [-128, 127], U8 -> [0, 255].
     if (q_t == OR_S8) { *qmin = -128; *qmax = 127; return true; }
     if (q_t == OR_U8) { *qmin = 0; *qmax = 255; return true; }
+    // s4 / u4 (deferred to a later milestone on the baracuda page): the
+    // two's-complement and unsigned 4-bit ranges.
+    if (q_t == OR_S4) { *qmin = -8; *qmax = 7; return true; }
+    if (q_t == OR_U4) { *qmin = 0; *qmax = 15; return true; }
     return false;
 }
 
@@ -357,12 +377,12 @@ double dequant_one(int64_t q, int64_t zp, float s, int y_t) {
 
 bool check_params(QParams& P, int64_t qmin, int64_t qmax) {
     if (!is_float_type(P.x_t)) return false;
-    if (P.q_t != OR_S8 && P.q_t != OR_U8) return false;
+    if (!is_int_type(P.q_t)) return false;
     int64_t dmin, dmax;
     default_range(P.q_t, &dmin, &dmax);
     if (qmin == 0 && qmax == 0) { qmin = dmin; qmax = dmax; }
     if (qmin < dmin || qmax > dmax || qmin >= qmax) return false;
-    if (P.symmetric && (P.q_t == OR_U8 || qmax <= 0)) return false;
+    if (P.symmetric && (P.q_t == OR_U8 || P.q_t == OR_U4 || qmax <= 0)) return false;
     P.qmin = qmin; P.qmax = qmax;
     return true;
 }
@@ -447,14 +467,14 @@ int or_quantize(const void* x, int x_t, int ndim, const int64_t* shape, int gran
         float s; int64_t z;
         if (scale_mode == 1) {
             s = scale[g];
-            z = (zp && !symmetric) ? load_i(zp, q_t, g) : 0;
+            z = (zp && !symmetric) ? load_i(zp, zp_type(q_t), g) : 0;
         } else {
             double hi, nlo;
             if (scale_mode == 2) { hi = range_hi[g]; nlo = range_neg_lo[g]; }
             else group_range(x, x_t, lay, g, &hi, &nlo);
             derive_scale(P, wide, hi, nlo, &s, &z);
             scale[g] = s;
-            if (zp) store_i(zp, q_t, g, z);
+            if (zp) store_i(zp, zp_type(q_t), g, z);
         }
         for_each_in_group(lay, g, [&](int64_t idx) {
             store_i(q, q_t, idx, quant_one(P, wide, load_f(x, x_t, idx), s, z));
@@ -466,13 +486,13 @@ int or_quantize(const void* x, int x_t, int ndim, const int64_t* shape, int gran
 // [baracuda] dequantize_per_{tensor,channel,token,group}: y = (q - zp) * scale.
 int or_dequantize(const void* q, int q_t, const float* scale, const void* zp, int ndim,
                   const int64_t* shape, int gran, int axis, int64_t gs, void* y, int y_t) {
-    if (q_t != OR_S8 && q_t != OR_U8) return 1;
+    if (!is_int_type(q_t)) return 1;
     if (!is_float_type(y_t)) return 1;
     Layout lay = make_layout(ndim, shape, gran, axis, gs);
     if (!lay.ok) return 1;
     for (int64_t g = 0; g < lay.n_groups(); ++g) {
         const float s = scale[g];
-        const int64_t z = zp ? load_i(zp, q_t, g) : 0;
+        const int64_t z = zp ? load_i(zp, zp_type(q_t), g) : 0;
         for_each_in_group(lay, g, [&](int64_t idx) {
             store_f(y, y_t, idx, dequant_one(load_i(q, q_t, idx), z, s, y_t));
         });
@@ -495,14 +515,14 @@ int or_fake_quantize(const void* x, int x_t, int ndim, const int64_t* shape, int
         float s; int64_t z;
         if (scale_mode == 1) {
             s = scale[g];
-            z = (zp && !symmetric) ? load_i(zp, q_t, g) : 0;
+            z = (zp && !symmetric) ? load_i(zp, zp_type(q_t), g) : 0;
         } else {
             double hi, nlo;
             if (scale_mode == 2) { hi = range_hi[g]; nlo = range_neg_lo[g]; }
             else group_range(x, x_t, lay, g, &hi, &nlo);
             derive_scale(P, wide, hi, nlo, &s, &z);
             scale[g] = s;
-            if (zp) store_i(zp, q_t, g, z);
+            if (zp) store_i(zp, zp_type(q_t), g, z);
         }
         for_each_in_group(lay, g, [&](int64_t idx) {
             int64_t qq = quant_one(P, wide, load_f(x, x_t, idx), s, z);
@@ -528,7 +548,7 @@ int or_ste_backward(int kind, const void* x, const void* dy, int x_t, const floa
     auto rnd = [&](double v) { return wide ? v : r32(v); };
     for (int64_t g = 0; g < lay.n_groups(); ++g) {
         const float s = scale[g];
-        const int64_t z = (zp && !symmetric) ? load_i(zp, q_t, g) : 0;
+        const int64_t z = (zp && !symmetric) ? load_i(zp, zp_type(q_t), g) : 0;
         for_each_in_group(lay, g, [&](int64_t idx) {
             double k = quant_unclamped(P, wide, load_f(x, x_t, idx), s, z);
             double m = ((double)P.qmin < k && k < (double)P.qmax) ? 1.0 : 0.0;

@@ -408,3 +408,67 @@ def test_column_group_is_group_of_the_transpose(orc, dtype):
         a = orc.dequantize_backward(dy, s, "column_group", 0, gs)
         b = orc.dequantize_backward(dyt, st, "group", 1, gs)
         assert torch.equal(a, b.t())
+
+
+# ---------------------------------------------------------------- s4 / u4
+# baracuda quantize module: "Sub-byte packed types (s4 / u4) are deferred to a
+# later milestone". Read here as 4-bit two's-complement / unsigned codes in
+# [-8, 7] / [0, 15], two per byte with element 2j in the low nibble (the order
+# of packed E2M1 on the QuantizedWeight page), zero-points one byte per group.
+def _nibble_pack(codes):
+    c = codes.astype(np.int64).reshape(-1) & 0xF
+    return (c[0::2] | (c[1::2] << 4)).astype(np.uint8)
+
+
+def test_s4_u4_default_ranges(orc):
+    assert orc.default_q_range("s4") == (-8, 7)
+    assert orc.default_q_range("u4") == (0, 15)
+
+
+def test_s4_u4_nibble_order_hand_computed(orc):
+    x = torch.tensor([[1.0, -1.0, 7.0, -8.0, 0.4, 3.0]])
+    q, _, _ = orc.quantize(x, "tensor", qdtype="s4", scale=torch.tensor([1.0]))
+    assert q.tolist() == [[0xF1, 0x87, 0x30]]          # (1, -1), (7, -8), (0, 3)
+    xu = torch.tensor([[-8.0, -1.0, 0.0, 7.0, 3.5, 100.0]])
+    qu, _, _ = orc.quantize(xu, "tensor", qdtype="u4", symmetric=False, scale=torch.tensor([1.0]),
+                            zp=torch.tensor([8], dtype=torch.uint8))
+    assert qu.tolist() == [[0x70, 0xF8, 0xFC]]         # codes 0, 7, 8, 15, 12, 15 (clamped)
+    y = orc.dequantize(q, torch.tensor([1.0]), None, "tensor", qdtype="s4")
+    assert y.tolist() == [[1.0, -1.0, 7.0, -8.0, 0.0, 3.0]]
+
+
+@pytest.mark.parametrize("gran,axis,gs,shape", [("token", 0, 1, (6, 64)), ("group", 1, 32, (5, 128)),
+                                                ("channel", 0, 1, (4, 10)), ("tensor", 0, 1, (3, 8)),
+                                                ("column_group", 0, 8, (16, 6))])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_s4_u4_are_packed_4bit_ranges(orc, gran, axis, gs, shape, dtype):
+    # Codes, scales and zero-points equal those of the byte codes restricted
+    # to the 4-bit range; the packing is numpy's nibble pack of those codes.
+    x = synthetic.Stream(50).tensor(shape, dtype, outlier_p=0.05, outlier_factor=10)
+    dy = synthetic.Stream(51).tensor(shape, dtype)
+    for q4, q8, sym, lo, hi in (("s4", "s8", True, -8, 7), ("u4", "u8", False, 0, 15),
+                                ("s4", "s8", False, -8, 7)):
+        q, s, z = orc.quantize(x, gran, axis, gs, q4, sym)
+        r, rs, rz = orc.quantize(x, gran, axis, gs, q8, sym, qmin=lo, qmax=hi)
+        assert q.shape == shape[:-1] + (shape[-1] // 2,)
+        assert np.array_equal(q.numpy().reshape(-1), _nibble_pack(r.numpy()))
+        assert torch.equal(s, rs)
+        if not sym:
+            assert torch.equal(z, rz)
+        zz = None if sym else z
+        y = orc.dequantize(q, s, zz, gran, axis, gs, ydtype=dtype, qdtype=q4)
+        ry = orc.dequantize(r, rs, None if sym else rz, gran, axis, gs, ydtype=dtype)
+        assert torch.equal(y, ry)
+        f, _, _ = orc.fake_quantize(x, gran, axis, gs, q4, sym)
+        rf, _, _ = orc.fake_quantize(x, gran, axis, gs, q8, sym, qmin=lo, qmax=hi)
+        assert torch.equal(f, rf)
+        a = orc.quantize_backward(x, dy, s, zz, gran, axis, gs, q4, sym)
+        b = orc.quantize_backward(x, dy, s, zz, gran, axis, gs, q8, sym, qmin=lo, qmax=hi)
+        assert torch.equal(a, b)
+
+
+def test_s4_u4_invalid(orc):
+    with pytest.raises(orc.OracleError):
+        orc.quantize(torch.zeros(3, 5), "token", qdtype="s4")          # odd last dimension
+    with pytest.raises(orc.OracleError):
+        orc.quantize(torch.zeros(3, 4), "token", qdtype="u4", symmetric=True)
