@@ -26,14 +26,15 @@ lib = C.CDLL(LIB_PATH)
 
 # ---------------------------------------------------------------- enums
 BQ_OK, BQ_ERR_INVALID_ARG, BQ_ERR_UNSUPPORTED, BQ_ERR_MISALIGNED, BQ_ERR_CUDA, BQ_ERR_TIMEOUT = range(6)
-BQ_F32, BQ_F64, BQ_F16, BQ_BF16, BQ_S8, BQ_U8, BQ_E4M3, BQ_E2M1X2, BQ_E8M0 = range(9)
+BQ_F32, BQ_F64, BQ_F16, BQ_BF16, BQ_S8, BQ_U8, BQ_E4M3, BQ_E2M1X2, BQ_E8M0, BQ_S4X2, BQ_U4X2 = range(11)
 BQ_RNE, BQ_RHAZ = 0, 1
 BQ_GRAN_TENSOR, BQ_GRAN_CHANNEL, BQ_GRAN_GROUP, BQ_GRAN_COLUMN_GROUP = 0, 1, 2, 3
 BQ_SCALE_DYNAMIC, BQ_SCALE_STATIC, BQ_SCALE_FROM_RANGE = 0, 1, 2
 BQ_NOALLOC_MAX_GROUPS = 65536
 
 DTYPE = {torch.float32: BQ_F32, torch.float64: BQ_F64, torch.float16: BQ_F16,
-         torch.bfloat16: BQ_BF16, torch.int8: BQ_S8, torch.uint8: BQ_U8}
+         torch.bfloat16: BQ_BF16, torch.int8: BQ_S8, torch.uint8: BQ_U8,
+         "s4": BQ_S4X2, "u4": BQ_U4X2}   # 4-bit codes, two per byte
 GRAN = {"tensor": BQ_GRAN_TENSOR, "channel": BQ_GRAN_CHANNEL, "group": BQ_GRAN_GROUP,
         "column_group": BQ_GRAN_COLUMN_GROUP}
 MODE = {"dynamic": BQ_SCALE_DYNAMIC, "static": BQ_SCALE_STATIC, "from_range": BQ_SCALE_FROM_RANGE}

@@ -15,6 +15,18 @@ import torch
 from . import _bq as B
 
 _SIGNED = {torch.int8: True, torch.uint8: False}
+# "s4" / "u4": 4-bit codes two per byte (element 2j in the low nibble) in a
+# uint8 tensor whose last dimension is half the logical one; zero-points one
+# byte per group (int8 for s4, uint8 for u4).
+_PACKED = ("s4", "u4")
+_ZP = {"s4": torch.int8, "u4": torch.uint8}
+
+
+def _codes_like(shape, qdtype, device):
+    if qdtype in _PACKED:
+        shape = tuple(shape)
+        return torch.empty(shape[:-1] + (shape[-1] // 2,), dtype=torch.uint8, device=device)
+    return torch.empty(shape, dtype=qdtype, device=device)
 
 
 def _axis_gs(gran: str, shape, axis: int, group_size: int):
@@ -42,13 +54,13 @@ def quantize(x: torch.Tensor, gran: str, axis: int = 0, group_size: int = 1,
     (int64 [n_groups, 2] range records) selects FROM_RANGE."""
     d = B.make_desc(x.shape, x.dtype, qdtype, symmetric, qmin, qmax, rnd)
     ng, _ = group_count(tuple(x.shape), x.dtype, gran, axis, group_size)
-    q = torch.empty(x.shape, dtype=qdtype, device=x.device)
+    q = _codes_like(x.shape, qdtype, x.device)
     ws = None
     if scale is not None:
         mode = "static"
     else:
         scale = torch.empty(ng, dtype=torch.float32, device=x.device)
-        zp = torch.empty(ng, dtype=qdtype, device=x.device)
+        zp = torch.empty(ng, dtype=_ZP.get(qdtype, qdtype), device=x.device)
         if ranges is not None:
             mode, ws = "from_range", ranges
         elif gran != "column_group":
@@ -72,9 +84,14 @@ def quantize(x: torch.Tensor, gran: str, axis: int = 0, group_size: int = 1,
 
 
 def dequantize(q: torch.Tensor, scale, zp, gran: str, axis: int = 0, group_size: int = 1,
-               ydtype=torch.float32, stream=None):
-    d = B.make_desc(q.shape, torch.float32, q.dtype, zp is None)
-    y = torch.empty(q.shape, dtype=ydtype, device=q.device)
+               ydtype=torch.float32, qdtype=None, stream=None):
+    """qdtype "s4" / "u4": q holds packed codes (last dimension halved)."""
+    if qdtype in _PACKED:
+        shape = tuple(q.shape[:-1]) + (2 * q.shape[-1],)
+    else:
+        shape, qdtype = tuple(q.shape), q.dtype
+    d = B.make_desc(shape, torch.float32, qdtype, zp is None)
+    y = torch.empty(shape, dtype=ydtype, device=q.device)
     if gran == "tensor":
         B.bq_dequantize_per_tensor(q, scale, zp, d, y, stream)
     elif gran == "token":
@@ -101,7 +118,7 @@ def fake_quantize(x: torch.Tensor, gran: str, axis: int = 0, group_size: int = 1
         mode = "static"
     else:
         scale = torch.empty(ng, dtype=torch.float32, device=x.device)
-        zp = torch.empty(ng, dtype=qdtype, device=x.device)
+        zp = torch.empty(ng, dtype=_ZP.get(qdtype, qdtype), device=x.device)
         if ranges is not None:
             mode, ws = "from_range", ranges
         else:

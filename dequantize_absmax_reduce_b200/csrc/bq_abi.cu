@@ -14,6 +14,8 @@ namespace {
 
 bool is_float(bq_dtype t) { return t == BQ_F32 || t == BQ_F64 || t == BQ_F16 || t == BQ_BF16; }
 bool is_half_or_f32(bq_dtype t) { return t == BQ_F32 || t == BQ_F16 || t == BQ_BF16; }
+bool is_packed_code(bq_dtype t) { return t == BQ_S4X2 || t == BQ_U4X2; }
+bool is_int_code(bq_dtype t) { return t == BQ_S8 || t == BQ_U8 || is_packed_code(t); }
 DT to_dt(bq_dtype t) {
     switch (t) {
         case BQ_F32: return DT::F32;
@@ -103,20 +105,35 @@ bq_status make_layout(const bq_qdesc* d, int gr, int32_t axis, int64_t gs, Layou
 // Code range: validates dtypes and resolves qmin = qmax = 0 to the defaults.
 bq_status make_cfg(const bq_qdesc* d, bool need_x, bq::IntCfg* c) {
     if (need_x && !is_float(d->x_dtype)) return BQ_ERR_UNSUPPORTED;
-    if (d->q_dtype != BQ_S8 && d->q_dtype != BQ_U8) return BQ_ERR_UNSUPPORTED;
+    if (!is_int_code(d->q_dtype)) return BQ_ERR_UNSUPPORTED;
     if (d->rnd != BQ_RNE && d->rnd != BQ_RHAZ) return BQ_ERR_INVALID_ARG;
     int32_t lo, hi;
     bq_default_q_range(d->q_dtype, &lo, &hi);
     int32_t qmin = d->qmin, qmax = d->qmax;
     if (qmin == 0 && qmax == 0) { qmin = lo; qmax = hi; }
     if (qmin < lo || qmax > hi || qmin >= qmax) return BQ_ERR_INVALID_ARG;
-    if (d->symmetric && d->q_dtype == BQ_U8) return BQ_ERR_UNSUPPORTED;
+    if (d->symmetric && (d->q_dtype == BQ_U8 || d->q_dtype == BQ_U4X2)) return BQ_ERR_UNSUPPORTED;
     if (d->symmetric && qmax <= 0) return BQ_ERR_INVALID_ARG;
     c->qmin = qmin;
     c->qmax = qmax;
     c->symmetric = d->symmetric ? 1 : 0;
     c->rhaz = d->rnd == BQ_RHAZ ? 1 : 0;
-    c->q_signed = d->q_dtype == BQ_S8 ? 1 : 0;
+    c->q_signed = (d->q_dtype == BQ_S8 || d->q_dtype == BQ_S4X2) ? 1 : 0;
+    c->packed = is_packed_code(d->q_dtype) ? 1 : 0;
+    return BQ_OK;
+}
+
+// Packed 4-bit codes go through the vector paths only (whole bytes per
+// vector): an even last dimension, groups (column groups: rows) of whole
+// 16-byte vectors of the float tensor, 16-byte aligned operands.
+bq_status check_packed(const bq_qdesc* d, const Layout& lay, bq_dtype float_dtype, const void* fp,
+                       const void* codes) {
+    if (lay.sv.numel == 0) return BQ_OK;
+    if (d->ndim < 1 || d->shape[d->ndim - 1] % 2 != 0) return BQ_ERR_UNSUPPORTED;
+    const int64_t vec = 16 / esize(float_dtype);
+    const int64_t len = lay.column ? lay.cv.inner : lay.sv.G;
+    if (len % vec != 0) return BQ_ERR_UNSUPPORTED;
+    if (!aligned(fp, 16) || !aligned(codes, 16)) return BQ_ERR_MISALIGNED;
     return BQ_OK;
 }
 
@@ -149,6 +166,8 @@ bq_status quant_impl(int op, const void* x, const bq_qdesc* d, int gr, int32_t a
     if (mode == BQ_SCALE_STATIC && asym && sv.n_seg > 0 && !zp) return BQ_ERR_INVALID_ARG;
     const int64_t es = esize(d->x_dtype);
     if (!aligned(x, es) || !aligned(scale, 4) || (y && !aligned(y, es))) return BQ_ERR_MISALIGNED;
+    if (cfg.packed && op == bq::OP_QUANT && (st = check_packed(d, lay, d->x_dtype, x, q)) != BQ_OK)
+        return st;
     const size_t need_ranges = (size_t)sv.n_seg * 16;
     if (mode == BQ_SCALE_FROM_RANGE) {
         if (sv.n_seg > 0 && (!ws || ws_bytes < need_ranges)) return BQ_ERR_INVALID_ARG;
@@ -208,6 +227,7 @@ bq_status dequant_impl(const void* q, const float* scale, const void* zp, const 
     if (sv.numel == 0) return BQ_OK;
     if (!q || !scale || !y) return BQ_ERR_INVALID_ARG;
     if (!aligned(scale, 4) || !aligned(y, esize(y_dtype))) return BQ_ERR_MISALIGNED;
+    if (cfg.packed && (st = check_packed(d, lay, y_dtype, y, q)) != BQ_OK) return st;
     if (lay.column)
         return from_cuda(bq::col_groups(to_dt(y_dtype), bq::OP_DEQ, 0, q, nullptr, lay.cv, cfg, scale,
                                         zp, nullptr, nullptr, y, S(stream)));
@@ -296,6 +316,8 @@ bq_status bq_default_q_range(bq_dtype q_dtype, int32_t* qmin, int32_t* qmax) {
     if (!qmin || !qmax) return BQ_ERR_INVALID_ARG;
     if (q_dtype == BQ_S8) { *qmin = -128; *qmax = 127; return BQ_OK; }
     if (q_dtype == BQ_U8) { *qmin = 0; *qmax = 255; return BQ_OK; }
+    if (q_dtype == BQ_S4X2) { *qmin = -8; *qmax = 7; return BQ_OK; }
+    if (q_dtype == BQ_U4X2) { *qmin = 0; *qmax = 15; return BQ_OK; }
     return BQ_ERR_UNSUPPORTED;
 }
 

@@ -34,6 +34,7 @@ cudaError_t col_groups(DT dt, int op, int dyn, const void* a, const void* b, Col
     if (op == OP_DEQ) vec = vec && al(a, vec_n) && al(out, 16);
     else if (op == OP_QUANT) vec = vec && al(a, 16) && al(out, vec_n);
     else vec = vec && al(a, 16) && al(b, 16) && al(out, 16);
+    if (cfg.packed && !vec && (op == OP_QUANT || op == OP_DEQ)) return cudaErrorNotSupported;
     ColArgs c;
     c.a = a;
     c.b = b;

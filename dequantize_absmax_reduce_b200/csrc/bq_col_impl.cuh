@@ -80,20 +80,6 @@ __device__ __forceinline__ typename Traits<T>::Acc col_elem(const ColRaw<T, W>& 
         return k == 0 ? __hiloint2double((int)r.u.y, (int)r.u.x) : __hiloint2double((int)r.u.w, (int)r.u.z);
     }
 }
-// W code bytes from q, as little-endian words.
-template <int W>
-__device__ __forceinline__ void col_load_code_words(const uint8_t* q, uint32_t (&w)[(W + 3) / 4]) {
-    if constexpr (W == 8) {
-        const uint2 v = __ldg(reinterpret_cast<const uint2*>(q));
-        w[0] = v.x; w[1] = v.y;
-    } else if constexpr (W == 4) {
-        w[0] = __ldg(reinterpret_cast<const uint32_t*>(q));
-    } else if constexpr (W == 2) {
-        w[0] = __ldg(reinterpret_cast<const unsigned short*>(q));
-    } else {
-        w[0] = __ldg(q);
-    }
-}
 // One row's W outputs, packed as they are produced: code bytes (CODES), or
 // values narrowed to T in pairs (16-bit T) or kept (f32 / f64).
 template <class T, int W, bool CODES> struct ColOut {
@@ -119,10 +105,17 @@ template <class T, int W, bool CODES> struct ColOut {
             v[k] = o;
         }
     }
-    __device__ __forceinline__ void store_codes(uint8_t* q) const {
-        if constexpr (W == 8) st8(q, cw[0], cw[1]);
-        else if constexpr (W == 4) st4(q, cw[0]);
-        else {
+    __device__ __forceinline__ void store_codes(uint8_t* q, int packed) const {
+        if (packed) {
+            if constexpr (W == 8) st4(q, nib_pack4(cw[0]) | (nib_pack4(cw[1]) << 16));
+            else if constexpr (W == 4) *reinterpret_cast<unsigned short*>(q) = (unsigned short)nib_pack4(cw[0]);
+            else if constexpr (W == 2) q[0] = (uint8_t)nib_pack4(cw[0]);
+            else q[0] = (uint8_t)cw[0];          // single codes: never packed
+        } else if constexpr (W == 8) {
+            st8(q, cw[0], cw[1]);
+        } else if constexpr (W == 4) {
+            st4(q, cw[0]);
+        } else {
 #pragma unroll
             for (int i = 0; i < W; ++i) q[i] = (uint8_t)(cw[0] >> (8 * i));
         }
@@ -307,7 +300,8 @@ __global__ void __launch_bounds__(256) k_col(ColArgs a) {
                     if (r >= gs) continue;
                     const int64_t e = (row0 + r) * inner + c0;
                     if constexpr (OP == OP_DEQ) {
-                        col_load_code_words<W>((const uint8_t*)a.a + e, cq[j]);
+                        ld_codes<W>(code_ptr((const uint8_t*)a.a, e, a.cfg.packed), a.cfg.packed,
+                                    a.cfg.q_signed, cq[j]);
                     } else {
                         raw[j] = col_fetch<T, W>((const T*)a.a + e, false);
                         if constexpr (TWO) rb[j] = col_fetch<T, W>((const T*)a.b + e, false);
@@ -350,7 +344,7 @@ __global__ void __launch_bounds__(256) k_col(ColArgs a) {
                 const int64_t r = r0 + (int64_t)j * RS;
                 if (r >= gs) continue;
                 const int64_t e = (row0 + r) * inner + c0;
-                if constexpr (OP == OP_QUANT) res[j].store_codes((uint8_t*)a.out + e);
+                if constexpr (OP == OP_QUANT) res[j].store_codes(code_ptr((uint8_t*)a.out, e, a.cfg.packed), a.cfg.packed);
                 else res[j].store((T*)a.out + e);
             }
         }

@@ -367,10 +367,97 @@ __device__ __forceinline__ double round_rne_d(double v) { return rint(v); }
 __device__ __forceinline__ double round_rhaz_d(double v) { return round(v); }
 
 // Pack four low bytes into one word: byte i of the result = low byte of w[i].
+__device__ __forceinline__ uint32_t pack4_lowbytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d);
+
+// ---------------------------------------------------------------- code storage
+// Integer codes are one byte each, or (packed) two 4-bit codes per byte with
+// element 2j in the low nibble of byte j. Vectors of codes always start at an
+// even element, so a packed vector covers whole bytes.
+__device__ __forceinline__ uint8_t* code_ptr(uint8_t* q, int64_t e, int packed) {
+    return q + (packed ? (e >> 1) : e);
+}
+__device__ __forceinline__ const uint8_t* code_ptr(const uint8_t* q, int64_t e, int packed) {
+    return q + (packed ? (e >> 1) : e);
+}
+// Low nibbles of the four bytes of w as two bytes (bytes 0, 1 of the result).
+__device__ __forceinline__ uint32_t nib_pack4(uint32_t w) {
+    uint32_t t = w & 0x0F0F0F0Fu;
+    t |= t >> 4;                                   // bytes 0 and 2 hold the pairs
+    return __byte_perm(t, 0u, 0x4420);
+}
+// Bytes 0, 1 of x as four 4-bit codes widened to bytes (sign-extended when
+// q_signed).
+__device__ __forceinline__ uint32_t nib_spread(uint32_t x, int q_signed) {
+    const uint32_t y = __byte_perm(x, 0u, 0x1100);
+    uint32_t w = (y & 0x000F000Fu) | ((y >> 4) & 0x0F000F00u);
+    if (q_signed) w = __vsub4(w ^ 0x08080808u, 0x08080808u);
+    return w;
+}
+template <int W>
+__device__ __forceinline__ void st_codes(uint8_t* q, const uint32_t (&c)[W], int packed);
+template <int W>
+__device__ __forceinline__ void ld_codes(const uint8_t* q, int packed, int q_signed,
+                                         uint32_t (&w)[(W + 3) / 4]);
+
 __device__ __forceinline__ uint32_t pack4_lowbytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
     const uint32_t ab = __byte_perm(a, b, 0x0040);   // [a0, b0, a0, a0]
     const uint32_t cd = __byte_perm(c, d, 0x0040);   // [c0, d0, ...]
     return __byte_perm(ab, cd, 0x5410);              // [a0, b0, c0, d0]
+}
+
+// W codes (the low bytes of c[]) at q (from code_ptr): W bytes, or W/2 bytes
+// of two 4-bit codes.
+template <int W>
+__device__ __forceinline__ void st_codes(uint8_t* q, const uint32_t (&c)[W], int packed) {
+    if constexpr (W == 8) {
+        const uint32_t lo = pack4_lowbytes(c[0], c[1], c[2], c[3]);
+        const uint32_t hi = pack4_lowbytes(c[4], c[5], c[6], c[7]);
+        if (packed) st4(q, nib_pack4(lo) | (nib_pack4(hi) << 16));
+        else st8(q, lo, hi);
+    } else if constexpr (W == 4) {
+        const uint32_t w = pack4_lowbytes(c[0], c[1], c[2], c[3]);
+        if (packed) *reinterpret_cast<unsigned short*>(q) = (unsigned short)nib_pack4(w);
+        else st4(q, w);
+    } else if constexpr (W == 2) {
+        if (packed) {
+            q[0] = (uint8_t)((c[0] & 0xFu) | ((c[1] & 0xFu) << 4));
+        } else {
+            q[0] = (uint8_t)c[0];
+            q[1] = (uint8_t)c[1];
+        }
+    } else {
+        q[0] = (uint8_t)c[0];     // single codes: never packed (the callers' shapes rule it out)
+    }
+}
+// W codes at q (from code_ptr) as bytes, four per word; packed 4-bit codes
+// are widened to bytes (sign-extended when q_signed).
+template <int W>
+__device__ __forceinline__ void ld_codes(const uint8_t* q, int packed, int q_signed,
+                                         uint32_t (&w)[(W + 3) / 4]) {
+    if (packed) {
+        if constexpr (W == 8) {
+            const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(q));
+            w[0] = nib_spread(v & 0xFFFFu, q_signed);
+            w[1] = nib_spread(v >> 16, q_signed);
+        } else if constexpr (W == 4) {
+            w[0] = nib_spread(__ldg(reinterpret_cast<const unsigned short*>(q)), q_signed);
+        } else if constexpr (W == 2) {
+            w[0] = nib_spread(__ldg(q), q_signed);
+        } else {
+            w[0] = __ldg(q);
+        }
+        return;
+    }
+    if constexpr (W == 8) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(q));
+        w[0] = v.x; w[1] = v.y;
+    } else if constexpr (W == 4) {
+        w[0] = __ldg(reinterpret_cast<const uint32_t*>(q));
+    } else if constexpr (W == 2) {
+        w[0] = __ldg(reinterpret_cast<const unsigned short*>(q));
+    } else {
+        w[0] = __ldg(q);
+    }
 }
 
 // ---------------------------------------------------------------- FP8 / FP4

@@ -57,12 +57,7 @@ __device__ __forceinline__ void emit_vec(const U4& raw, const Recip& R, const In
         uint32_t cw[VEC];
 #pragma unroll
         for (int i = 0; i < VEC; ++i) cw[i] = code_from_rounded(t[i], ip.zp);
-        if constexpr (VEC == 8) {
-            st8(a.q + off, pack4_lowbytes(cw[0], cw[1], cw[2], cw[3]),
-                pack4_lowbytes(cw[4], cw[5], cw[6], cw[7]));
-        } else {
-            st4(a.q + off, pack4_lowbytes(cw[0], cw[1], cw[2], cw[3]));
-        }
+        st_codes<VEC>(code_ptr(a.q, off, a.cfg.packed), cw, a.cfg.packed);
     } else {
         float o[VEC];
 #pragma unroll
@@ -247,19 +242,9 @@ __global__ void __launch_bounds__(256) k_int_map(MapArgs a) {
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int64_t it = it0 + (int64_t)u * 32;
-                const uint8_t* qb = (const uint8_t*)a.a + it * W;
-                if (it < n_items) {
-                    if constexpr (W == 8) {
-                        const uint2 w2 = __ldg(reinterpret_cast<const uint2*>(qb));
-                        cw[u][0] = w2.x; cw[u][1] = w2.y;
-                    } else if constexpr (W == 4) {
-                        cw[u][0] = __ldg(reinterpret_cast<const uint32_t*>(qb));
-                    } else if constexpr (W == 2) {
-                        cw[u][0] = __ldg(reinterpret_cast<const unsigned short*>(qb));
-                    } else {
-                        cw[u][0] = __ldg(qb);
-                    }
-                }
+                if (it < n_items)
+                    ld_codes<W>(code_ptr((const uint8_t*)a.a, it * W, a.cfg.packed), a.cfg.packed,
+                                a.cfg.q_signed, cw[u]);
             }
 #pragma unroll
             for (int u = 0; u < U; ++u) {
@@ -323,16 +308,7 @@ __global__ void __launch_bounds__(256) k_int_map(MapArgs a) {
                     else o[i] = elem_f<OP, RHAZ>(xa[i], TWO ? xb[i] : 0.0f, st, &cw[i]);
                 }
                 if constexpr (OP == OP_QUANT) {
-                    uint8_t* q = (uint8_t*)a.out + e0;
-                    if constexpr (W == 8) {
-                        st8(q, pack4_lowbytes(cw[0], cw[1], cw[2], cw[3]),
-                            pack4_lowbytes(cw[4], cw[5], cw[6], cw[7]));
-                    } else if constexpr (W == 4) {
-                        st4(q, pack4_lowbytes(cw[0], cw[1], cw[2], cw[3]));
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < W; ++i) q[i] = (uint8_t)cw[i];
-                    }
+                    st_codes<W>(code_ptr((uint8_t*)a.out, e0, a.cfg.packed), cw, a.cfg.packed);
                 } else {
                     if constexpr (VECP) st16((T*)a.out + e0, pack_vec<T>(o));
                     else ((T*)a.out)[e0] = to_out<T>(o[0]);
@@ -648,7 +624,10 @@ cudaError_t int_map(DT dt, int op, int psrc, const void* a_ptr, const void* b_pt
         if (op == OP_QUANT) vecp = vecp && ((uintptr_t)out % VEC == 0);
         else vecp = vecp && aligned16(out);
     }
-    if (vecp) {
+    // Packed 4-bit codes are written and read a whole vector (whole bytes) at
+    // a time; the callers only pass shapes and pointers that allow it.
+    if (cfg.packed && !vecp && (op == OP_QUANT || op == OP_DEQ)) return cudaErrorNotSupported;
+    if (vecp && !(cfg.packed && (op == OP_QUANT || op == OP_DEQ))) {
         const cudaError_t pe = int_map_pipe(dt, op, a, st);
         if (pe != cudaErrorNotSupported) return pe;
     }

@@ -14,7 +14,8 @@ struct IntCfg {
     int qmin, qmax;
     int symmetric;
     int rhaz;       // 1: ties away from zero
-    int q_signed;   // 1: codes are s8, 0: u8
+    int q_signed;   // 1: codes are s8 (or s4), 0: u8 (or u4)
+    int packed;     // 1: 4-bit codes, two per byte (element 2j in the low nibble)
 };
 
 // Contiguous-group view: n_seg groups of G consecutive elements each.

@@ -462,7 +462,8 @@ __global__ void __launch_bounds__(NT) k_seg_pipe(PipeArgs a) {
             ip.lo = SYM ? qlo : __fsub_rn(qlo, zf);
             ip.hi = SYM ? qhi : __fsub_rn(qhi, zf);
             ip.zp = SYM ? 0 : zp;
-            uint8_t* qb = a.q + seg * G + lane * VEC;
+            const int64_t qe = seg * G + lane * VEC;          // element offset of the codes
+            const int pk = a.cfg.packed;
             T* yb = (T*)a.y + seg * G + lane * VEC;
             // Fast path: no NaN in the warp's groups, a normal scale, and no
             // clamp that can bind. Symmetric: |x/s| <= qmax (1 + 2^-23) rounds
@@ -484,11 +485,11 @@ __global__ void __launch_bounds__(NT) k_seg_pipe(PipeArgs a) {
                 if (full) {
 #pragma unroll
                     for (int j = 0; j < NV; ++j)
-                        emit_int_fast<T, OP, !SYM>(raw[j], R2, magic2, zp2, s2v, qb + voff(j), yb + voff(j));
+                        emit_int_fast<T, OP, !SYM>(raw[j], R2, magic2, zp2, s2v, code_ptr(a.q, qe + voff(j), pk), pk, yb + voff(j));
                 } else {
 #pragma unroll
                     for (int j = 0; j < NV; ++j)
-                        if (vok(j)) emit_int_fast<T, OP, !SYM>(raw[j], R2, magic2, zp2, s2v, qb + voff(j), yb + voff(j));
+                        if (vok(j)) emit_int_fast<T, OP, !SYM>(raw[j], R2, magic2, zp2, s2v, code_ptr(a.q, qe + voff(j), pk), pk, yb + voff(j));
                 }
             } else if (seg_ok) {
 #pragma unroll
@@ -496,8 +497,8 @@ __global__ void __launch_bounds__(NT) k_seg_pipe(PipeArgs a) {
                     if (!vok(j)) continue;
                     float v[VEC];
                     load_vec<T>(raw[j], v);
-                    if (R.fast) emit_int<T, OP, true, SYM>(v, R, ip, qb + voff(j), yb + voff(j));
-                    else emit_int<T, OP, false, SYM>(v, R, ip, qb + voff(j), yb + voff(j));
+                    if (R.fast) emit_int<T, OP, true, SYM>(v, R, ip, code_ptr(a.q, qe + voff(j), pk), pk, yb + voff(j));
+                    else emit_int<T, OP, false, SYM>(v, R, ip, code_ptr(a.q, qe + voff(j), pk), pk, yb + voff(j));
                 }
             }
         } else {
@@ -2142,8 +2143,14 @@ __global__ void __launch_bounds__(256, BQ_COL_MINB) k_col_tma(const __grid_const
             for (int j = 0; j < COLT_RPT; ++j) {
                 const int64_t e = obase + (int64_t)j * RS * a.inner;
                 if constexpr (OP == OP_QUANT) {
-                    if constexpr (W == 8) st8((uint8_t*)a.out + e, cwd[j][0], cwd[j][1]);
-                    else st4((uint8_t*)a.out + e, cwd[j][0]);
+                    uint8_t* q = code_ptr((uint8_t*)a.out, e, a.cfg.packed);
+                    if (a.cfg.packed) {
+                        if constexpr (W == 8) st4(q, nib_pack4(cwd[j][0]) | (nib_pack4(cwd[j][1]) << 16));
+                        else *reinterpret_cast<unsigned short*>(q) = (unsigned short)nib_pack4(cwd[j][0]);
+                    } else {
+                        if constexpr (W == 8) st8(q, cwd[j][0], cwd[j][1]);
+                        else st4(q, cwd[j][0]);
+                    }
                 } else {
                     st16((T*)a.out + e, U4{ow[j][0], ow[j][1], ow[j][2], ow[j][3]});
                 }
@@ -2171,9 +2178,7 @@ __global__ void __launch_bounds__(256, BQ_COL_MINB) k_col_tma(const __grid_const
                 }
                 const int64_t e = obase + (int64_t)j * RS * a.inner;
                 if constexpr (OP == OP_QUANT) {
-                    if constexpr (W == 8) st8((uint8_t*)a.out + e, pack4_lowbytes(code[0], code[1], code[2], code[3]),
-                                              pack4_lowbytes(code[4], code[5], code[6], code[7]));
-                    else st4((uint8_t*)a.out + e, pack4_lowbytes(code[0], code[1], code[2], code[3]));
+                    st_codes<W>(code_ptr((uint8_t*)a.out, e, a.cfg.packed), code, a.cfg.packed);
                 } else {
                     st16((T*)a.out + e, pack_vec<T>(o));
                 }

@@ -141,7 +141,7 @@ __device__ __forceinline__ void mx_emit(const float* v, const Recip& R, float mu
 // values (FAKE: fl(k * s)), k = round-half-even(fl(x / s)).
 template <class T, int OP, bool ASYM>
 __device__ __forceinline__ void emit_int_fast(const U4& raw, const Recip2& R2, F2 magic2, F2 zp2,
-                                              F2 s2, uint8_t* q, T* y) {
+                                              F2 s2, uint8_t* q, int packed, T* y) {
     constexpr int VEC = Traits<T>::VEC;
     constexpr int NP = VEC / 2;
     F2 x[NP];
@@ -154,11 +154,7 @@ __device__ __forceinline__ void emit_int_fast(const U4& raw, const Recip2& R2, F
             if (ASYM) t = f2_add(t, zp2);            // exact: both integers in the unit-spaced range
             f2_split_bits(t, c[2 * p], c[2 * p + 1]);
         }
-        if constexpr (VEC == 8) {
-            st8(q, pack4_lowbytes(c[0], c[1], c[2], c[3]), pack4_lowbytes(c[4], c[5], c[6], c[7]));
-        } else {
-            st4(q, pack4_lowbytes(c[0], c[1], c[2], c[3]));
-        }
+        st_codes<VEC>(q, c, packed);
     } else {
         float o[VEC];
 #pragma unroll
@@ -272,7 +268,7 @@ __device__ __forceinline__ void emit_mx4_fast(const U4& raw, F2 mul2, uint8_t* d
 // qmax and only the lower clamp (which also takes a NaN to qmin) can bind.
 template <class T, int OP, bool FAST, bool SYM_DYN>
 __device__ __forceinline__ void emit_int(const float* v, const Recip& R, const IntParams& ip,
-                                         uint8_t* q, T* y) {
+                                         uint8_t* q, int packed, T* y) {
     constexpr int VEC = Traits<T>::VEC;
     float t[VEC];
 #pragma unroll
@@ -285,11 +281,7 @@ __device__ __forceinline__ void emit_int(const float* v, const Recip& R, const I
         uint32_t cw[VEC];
 #pragma unroll
         for (int i = 0; i < VEC; ++i) cw[i] = code_from_rounded(t[i], SYM_DYN ? 0 : ip.zp);
-        if constexpr (VEC == 8) {
-            st8(q, pack4_lowbytes(cw[0], cw[1], cw[2], cw[3]), pack4_lowbytes(cw[4], cw[5], cw[6], cw[7]));
-        } else {
-            st4(q, pack4_lowbytes(cw[0], cw[1], cw[2], cw[3]));
-        }
+        st_codes<VEC>(q, cw, packed);
     } else {
         float o[VEC];
 #pragma unroll

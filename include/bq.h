@@ -63,10 +63,16 @@ typedef enum bq_status {
     BQ_ERR_TIMEOUT = 5
 } bq_status;
 
+/* BQ_S4X2 / BQ_U4X2: 4-bit integer codes (the s4 / u4 the baracuda quantize
+ * module defers to a later milestone), two per byte with element 2j in the
+ * low nibble of byte j (the order of packed E2M1); a code tensor of n
+ * elements is n/2 bytes. Their zero-points are one byte per group: s8 for
+ * S4X2, u8 for U4X2. */
 typedef enum bq_dtype {
     BQ_F32 = 0, BQ_F64 = 1, BQ_F16 = 2, BQ_BF16 = 3,
     BQ_S8 = 4, BQ_U8 = 5,
-    BQ_E4M3 = 6, BQ_E2M1X2 = 7, BQ_E8M0 = 8
+    BQ_E4M3 = 6, BQ_E2M1X2 = 7, BQ_E8M0 = 8,
+    BQ_S4X2 = 9, BQ_U4X2 = 10
 } bq_dtype;
 
 /* Rounding of x/scale to an integer code: nearest with ties to even
@@ -101,7 +107,13 @@ typedef enum bq_scale_mode {
 
 /* Description of a quantized tensor x (up to 8 dims) and its code range.
  * qmin = qmax = 0 selects default_q_range(q_dtype): S8 [-128,127],
- * U8 [0,255] ([baracuda] default_q_range).
+ * U8 [0,255] ([baracuda] default_q_range), S4X2 [-8,7], U4X2 [0,15].
+ * Packed codes (S4X2, U4X2) are written and read whole bytes at a time:
+ * quantize and dequantize with them need an even last dimension, groups
+ * (column groups: rows) whose length is a multiple of the float tensor's
+ * 16-byte vector (8 elements for F16 / BF16, 4 for F32, 2 for F64;
+ * BQ_ERR_UNSUPPORTED otherwise) and 16-byte aligned float and code tensors
+ * (BQ_ERR_MISALIGNED otherwise).
  * Symmetric: scale = fl(amax / qmax), zero-point 0 (S8 only).
  * Asymmetric: min' = min(min x, 0), max' = max(max x, 0),
  *   scale = fl(fl(max' - min') / (qmax - qmin)),
@@ -113,7 +125,7 @@ typedef struct bq_qdesc {
     int32_t ndim;
     int64_t shape[8];
     bq_dtype x_dtype;   /* F32, F64, F16 or BF16 */
-    bq_dtype q_dtype;   /* S8 or U8 */
+    bq_dtype q_dtype;   /* S8, U8, S4X2 or U4X2 */
     int32_t symmetric;  /* 1: absmax scaling, 0: min/max + zero-point */
     int32_t qmin, qmax;
     bq_round rnd;
@@ -128,7 +140,8 @@ const char* bq_status_string(bq_status s);
  * ("column_group" for BQ_GRAN_COLUMN_GROUP); NULL for an unknown value. */
 const char* bq_granularity_name(bq_gran g);
 
-/* [baracuda] default_q_range: S8 -> [-128, 127], U8 -> [0, 255]. Host only. */
+/* [baracuda] default_q_range: S8 -> [-128, 127], U8 -> [0, 255]; S4X2 ->
+ * [-8, 7], U4X2 -> [0, 15]. Host only. */
 bq_status bq_default_q_range(bq_dtype q_dtype, int32_t* qmin, int32_t* qmax);
 
 /* [granularity] axis_and_group_size() applied to a shape: number of scale

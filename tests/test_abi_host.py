@@ -44,6 +44,7 @@ def test_library_exports_every_declared_symbol(B):
 def test_misc_host_functions(B):
     assert B.bq_default_q_range(torch.int8) == (-128, 127)
     assert B.bq_default_q_range(torch.uint8) == (0, 255)
+    assert B.bq_default_q_range("s4") == (-8, 7) and B.bq_default_q_range("u4") == (0, 15)
     assert [B.bq_granularity_name(g) for g in ("tensor", "channel", "group")] == ["tensor", "channel", "group"]
     assert B.lib.bq_granularity_name(7) is None
     assert B.bq_packed_transpose_stride(4097, 16) == 4112
@@ -141,6 +142,16 @@ def test_argument_errors_return_status_without_launching(B):
     assert B.lib.bq_quantize_per_column_group_backward(P, P, P, None, C.byref(da), 0, 3, P, None) == B.BQ_ERR_INVALID_ARG
     assert B.lib.bq_dequantize_per_column_group_backward(P, P, C.byref(dc), 0, 5, P, None) == B.BQ_ERR_INVALID_ARG
     assert B.lib.bq_quantize_dynamic_noalloc(P, C.byref(dc), 9, 0, 16, P, P, P, None) == B.BQ_ERR_INVALID_ARG
+    # s4 / u4: packed codes need whole vectors and aligned tensors
+    d4 = B.make_desc((4, 7), torch.float32, "s4")
+    assert B.lib.bq_quantize_per_token(P, C.byref(d4), P, P, P, 0, None, 0, None) == B.BQ_ERR_UNSUPPORTED
+    d4 = B.make_desc((4, 12), torch.bfloat16, "s4")                 # 12 % 8: not whole bf16 vectors
+    assert B.lib.bq_quantize_per_token(P, C.byref(d4), P, P, P, 0, None, 0, None) == B.BQ_ERR_UNSUPPORTED
+    d4 = B.make_desc((4, 16), torch.bfloat16, "u4", symmetric=True)
+    assert B.lib.bq_quantize_per_token(P, C.byref(d4), P, P, P, 0, None, 0, None) == B.BQ_ERR_UNSUPPORTED
+    d4 = B.make_desc((4, 16), torch.bfloat16, "s4")
+    assert B.lib.bq_quantize_per_token(P, C.byref(d4), P + 8, P, P, 0, None, 0, None) == B.BQ_ERR_MISALIGNED
+    assert B.lib.bq_dequantize_per_token(P + 4, P, None, C.byref(d4), P, B.BQ_BF16, None) == B.BQ_ERR_MISALIGNED
     # descriptor errors
     d9 = B.make_desc((4, 64), torch.float32)
     d9.ndim = 9
