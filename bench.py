@@ -312,7 +312,16 @@ def per_granularity(B, api, torch, device, peak, reps=5):
           4 * n + 5 * ng, 1)
     timed(wlc, "quantize_per_column_group_backward",
           lambda: B.bq_quantize_per_column_group_backward(x, dy, s, z, du, 0, 128, dx), 6 * n + 5 * ng, 1)
-    del w, x, dy, q, qs, y, dx
+    # 4-bit weights of the same tensor (u4 asymmetric, two codes per byte).
+    d4 = B.make_desc(x.shape, x.dtype, "u4", symmetric=False)
+    q4 = torch.empty((R, K // 2), dtype=torch.uint8, device=device)
+    timed(wl, "quantize_per_group(axis=1,gs=128,u4 asym, packed)",
+          lambda: B.bq_quantize_per_group(x, d4, 1, 128, q4, s, z, "dynamic", None), 2 * n + n // 2 + 5 * ng, 1)
+    timed(wl, "dequantize_per_group(u4 packed)",
+          lambda: B.bq_dequantize_per_group(q4, s, z, d4, 1, 128, y), 2 * n + n // 2 + 5 * ng, 1)
+    timed(wlc, "quantize_per_column_group(axis=0,gs=128,u4 asym, packed)",
+          lambda: B.bq_quantize_per_column_group(x, d4, 0, 128, q4, s, z, "dynamic"), 2 * n + n // 2 + 5 * ng, 1)
+    del w, x, dy, q, qs, y, dx, q4
 
     # NVFP4 bf16 [4096, 7168]
     wl = "nvfp4_bf16_4096x7168"
