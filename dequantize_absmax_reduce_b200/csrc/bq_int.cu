@@ -627,7 +627,7 @@ cudaError_t int_map(DT dt, int op, int psrc, const void* a_ptr, const void* b_pt
     // Packed 4-bit codes are written and read a whole vector (whole bytes) at
     // a time; the callers only pass shapes and pointers that allow it.
     if (cfg.packed && !vecp && (op == OP_QUANT || op == OP_DEQ)) return cudaErrorNotSupported;
-    if (vecp && !(cfg.packed && (op == OP_QUANT || op == OP_DEQ))) {
+    if (vecp && !(cfg.packed && op == OP_QUANT)) {
         const cudaError_t pe = int_map_pipe(dt, op, a, st);
         if (pe != cudaErrorNotSupported) return pe;
     }

@@ -44,7 +44,7 @@ cudaError_t int_map_pipe(DT dt, int op, const MapArgs& m, cudaStream_t st) {
     const int VEC = dt == DT::F32 ? 4 : 8;
     if (m.G % VEC != 0 || !al16(m.a) || !al16(m.out)) return cudaErrorNotSupported;
     if ((op == OP_QBWD || op == OP_FBWD) && !al16(m.b)) return cudaErrorNotSupported;
-    if (op == OP_DEQ && m.numel % 16 != 0) return cudaErrorNotSupported;
+    if (op == OP_DEQ && m.numel % (m.cfg.packed ? 32 : 16) != 0) return cudaErrorNotSupported;
     if (op == OP_QUANT && ((uintptr_t)m.out % VEC) != 0) return cudaErrorNotSupported;
     switch (dt) {
         case DT::F32: return pipe_map_f32(op, m, st);

@@ -1341,6 +1341,7 @@ struct SegMapArgs {
     int P;
     int64_t n_tiles;
     int in_esz;         // bytes per element of input a (1 for codes)
+    int code_shift;     // 1: 4-bit codes two per byte (byte counts of a halved)
     int part_bytes;     // P * G * in_esz: where the dy part of a slot starts
     int slot_bytes;
 };
@@ -1373,13 +1374,13 @@ __global__ void __launch_bounds__(256) k_seg_map(SegMapArgs p) {
     auto issue = [&](int64_t tile, int slot) {
         const int64_t segs = min((int64_t)p.P, a.n_seg - tile * p.P);
         const int64_t e0 = tile * p.P * G;
-        const uint32_t ba = (uint32_t)(segs * G * p.in_esz);
+        const uint32_t ba = (uint32_t)((segs * G * p.in_esz) >> p.code_shift);
         const uint32_t bb = TWO ? (uint32_t)(segs * G * ESZ) : 0u;
         const uint32_t bar = smem_addr(&bars[slot]);
         uint8_t* dst = ring + (size_t)slot * p.slot_bytes;
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(ba + bb) : "memory");
         asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                     :: "r"(smem_addr(dst)), "l"((const uint8_t*)a.a + e0 * p.in_esz), "r"(ba), "r"(bar) : "memory");
+                     :: "r"(smem_addr(dst)), "l"((const uint8_t*)a.a + ((e0 * p.in_esz) >> p.code_shift)), "r"(ba), "r"(bar) : "memory");
         if (TWO)
             asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                          :: "r"(smem_addr(dst + p.part_bytes)), "l"((const uint8_t*)a.b + e0 * ESZ),
@@ -1414,7 +1415,7 @@ __global__ void __launch_bounds__(256) k_seg_map(SegMapArgs p) {
         // This thread's vectors (codes: 8 / 4 bytes per vector; otherwise x and,
         // for the backwards, dy) copied to registers. (After a failed wait the
         // slot holds stale bytes; they are read but never used.)
-        const uint8_t* sa = ring + (size_t)slot * p.slot_bytes + (size_t)team * G * p.in_esz;
+        const uint8_t* sa = ring + (size_t)slot * p.slot_bytes + (((size_t)team * G * p.in_esz) >> p.code_shift);
         const uint8_t* sb = ring + (size_t)slot * p.slot_bytes + p.part_bytes + (size_t)team * G * ESZ;
         U4 va[NV], vb[NV];
 #pragma unroll
@@ -1425,10 +1426,23 @@ __global__ void __launch_bounds__(256) k_seg_map(SegMapArgs p) {
             vb[j] = U4{0u, 0u, 0u, 0u};
             if (v_ok) {
                 if constexpr (OP == OP_DEQ) {
-                    if constexpr (W == 8)
+                    if (p.code_shift) {
+                        // two 4-bit codes per byte, widened to one per byte
+                        if constexpr (W == 8) {
+                            uint32_t v;
+                            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_addr(sa + (e >> 1))));
+                            va[j].x = nib_spread(v & 0xFFFFu, a.cfg.q_signed);
+                            va[j].y = nib_spread(v >> 16, a.cfg.q_signed);
+                        } else {
+                            unsigned short v;
+                            asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(smem_addr(sa + (e >> 1))));
+                            va[j].x = nib_spread(v, a.cfg.q_signed);
+                        }
+                    } else if constexpr (W == 8) {
                         asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(va[j].x), "=r"(va[j].y) : "r"(smem_addr(sa + e)));
-                    else
+                    } else {
                         asm volatile("ld.shared.u32 %0, [%1];" : "=r"(va[j].x) : "r"(smem_addr(sa + e)));
+                    }
                 } else {
                     va[j] = ld_shared16(smem_addr(sa + (size_t)e * ESZ));
                     if constexpr (TWO) vb[j] = ld_shared16(smem_addr(sb + (size_t)e * ESZ));
@@ -1685,7 +1699,8 @@ static cudaError_t launch_seg_map_t(const MapArgs& m, cudaStream_t st) {
     p.P = P;
     p.n_tiles = (m.n_seg + P - 1) / P;
     p.in_esz = (OP == OP_DEQ) ? 1 : (int)sizeof(T);
-    p.part_bytes = P * (int)m.G * p.in_esz;
+    p.code_shift = (OP == OP_DEQ && m.cfg.packed) ? 1 : 0;
+    p.part_bytes = (P * (int)m.G * p.in_esz) >> p.code_shift;
     p.slot_bytes = p.part_bytes + (TWO ? P * (int)m.G * (int)sizeof(T) : 0);
     const size_t smem = 128 + (size_t)S * p.slot_bytes;
     constexpr int in_max = (OP == OP_DEQ) ? 1 : (int)sizeof(T);
@@ -1864,10 +1879,16 @@ cudaError_t pipe_dyn_entry(int pk, bool sym, const PipeArgs& a, cudaStream_t st)
 template <class T>
 cudaError_t pipe_map_entry(int op, const MapArgs& m, cudaStream_t st) {
     const int in_esz = (op == OP_DEQ) ? 1 : (int)sizeof(T);
-    if (m.n_seg > 0 && (m.G * in_esz) % 16 == 0) {
+    // Packed 4-bit codes: only the group-tiled dequantize reads them (whole
+    // 16-byte runs of codes per group); packed quantize stays element-wise.
+    const bool packed = m.cfg.packed && (op == OP_DEQ || op == OP_QUANT);
+    if (packed && op != OP_DEQ) return cudaErrorNotSupported;
+    const int64_t a_bytes = (m.G * in_esz) >> (packed ? 1 : 0);
+    if (m.n_seg > 0 && a_bytes % 16 == 0) {
         const cudaError_t e = seg_map_dt<T>(op, m, st);
-        if (e != cudaErrorNotSupported) return e;
+        if (e != cudaErrorNotSupported || packed) return e;
     }
+    if (packed) return cudaErrorNotSupported;
     return map_pipe_dt<T>(op, m.ranges ? PS_RANGE : PS_STATIC, m, st);
 }
 
