@@ -13,6 +13,12 @@ cudaError_t col_groups_f64(int op, int dyn, const ColArgs& a, bool vec, cudaStre
 cudaError_t pipe_col_f32(int op, const ColPipeArgs& p, cudaStream_t st);
 cudaError_t pipe_col_f16(int op, const ColPipeArgs& p, cudaStream_t st);
 cudaError_t pipe_col_bf16(int op, const ColPipeArgs& p, cudaStream_t st);
+cudaError_t pipe_colmap_f32(int op, const void* a, const void* b, int64_t rows, int64_t inner, int64_t gs,
+                            IntCfg cfg, const float* scale, const uint8_t* zp, void* out, cudaStream_t st);
+cudaError_t pipe_colmap_f16(int op, const void* a, const void* b, int64_t rows, int64_t inner, int64_t gs,
+                            IntCfg cfg, const float* scale, const uint8_t* zp, void* out, cudaStream_t st);
+cudaError_t pipe_colmap_bf16(int op, const void* a, const void* b, int64_t rows, int64_t inner, int64_t gs,
+                             IntCfg cfg, const float* scale, const uint8_t* zp, void* out, cudaStream_t st);
 
 static bool al(const void* p, int n) { return !p || ((uintptr_t)p % (uintptr_t)n) == 0; }
 
@@ -25,6 +31,15 @@ cudaError_t col_groups(DT dt, int op, int dyn, const void* a, const void* b, Col
         ColPipeArgs p{a, v.outer * v.L, v.inner, v.gs, cfg, scale_out, (uint8_t*)zp_out, out};
         const cudaError_t e = dt == DT::F32 ? pipe_col_f32(op, p, st)
                             : dt == DT::F16 ? pipe_col_f16(op, p, st) : pipe_col_bf16(op, p, st);
+        if (e != cudaErrorNotSupported) return e;
+    }
+    if (!dyn && dt != DT::F64) {
+        // Static parameters: the 2D-TMA pipelined kernel for the sizes it covers.
+        const int64_t rows = v.outer * v.L;
+        const uint8_t* z = (const uint8_t*)zp_in;
+        const cudaError_t e = dt == DT::F32 ? pipe_colmap_f32(op, a, b, rows, v.inner, v.gs, cfg, scale_in, z, out, st)
+                            : dt == DT::F16 ? pipe_colmap_f16(op, a, b, rows, v.inner, v.gs, cfg, scale_in, z, out, st)
+                                            : pipe_colmap_bf16(op, a, b, rows, v.inner, v.gs, cfg, scale_in, z, out, st);
         if (e != cudaErrorNotSupported) return e;
     }
     const int vec_n = dt == DT::F32 ? 4 : (dt == DT::F64 ? 2 : 8);

@@ -181,11 +181,11 @@ __global__ void __launch_bounds__(256) k_col(ColArgs a) {
     constexpr int CVN = G::CVN, RS = G::RS, CW = G::CW, NW = G::NW;
     constexpr bool NEEDR = !WIDE && OP != OP_DEQ && OP != OP_DBWD;   // reciprocal used
     __shared__ Acc red_hi[DYN ? NW : 1][CW], red_lo[DYN ? NW : 1][CW];
-    // The tile's column parameters, double-buffered by tile parity: a thread
-    // writing tile t+2's entries has passed a barrier that every reader of
-    // tile t's entries reached after reading them.
-    __shared__ float col_s[2][CW], col_y[2][CW];
-    __shared__ int col_z[2][CW];
+    // The tile's column parameters (dynamic scaling), double-buffered by tile
+    // parity: a thread writing tile t+2's entries has passed a barrier that
+    // every reader of tile t's entries reached after reading them.
+    __shared__ float col_s[DYN ? 2 : 1][CW], col_y[DYN ? 2 : 1][CW];
+    __shared__ int col_z[DYN ? 2 : 1][CW];
 
     const int tid = threadIdx.x;
     const int cv = tid % CVN, rl = tid / CVN;
@@ -270,21 +270,8 @@ __global__ void __launch_bounds__(256) k_col(ColArgs a) {
                     if (a.zp_out) a.zp_out[ob * inner + c] = (uint8_t)z;
                 }
             }
-        } else {
-            if (tid < CW) {
-                const int64_t c = ct * CW + tid;
-                float s = 1.0f;
-                int z = 0;
-                if (c < inner) {
-                    s = __ldg(a.scale_in + ob * inner + c);
-                    if (OP != OP_DBWD && !a.cfg.symmetric) z = load_zp(a.zp_in, ob * inner + c, a.cfg.q_signed);
-                }
-                col_s[par][tid] = s;
-                col_z[par][tid] = z;
-                if constexpr (NEEDR) col_y[par][tid] = __frcp_rn(s);
-            }
+            __syncthreads();
         }
-        __syncthreads();
         if (!col_ok) continue;      // no barrier below this point
 
         // ---- element pass over the block's rows, one column at a time (one
@@ -312,7 +299,21 @@ __global__ void __launch_bounds__(256) k_col(ColArgs a) {
 #pragma unroll
             for (int k = 0; k < W; ++k) {
                 const int c = cv * W + k;
-                const GState stk = col_state(a.cfg, col_s[par][c], NEEDR ? col_y[par][c] : 0.0f, col_z[par][c]);
+                float sk, yk = 0.0f;
+                int zk;
+                if constexpr (DYN) {
+                    sk = col_s[par][c];
+                    if constexpr (NEEDR) yk = col_y[par][c];
+                    zk = col_z[par][c];
+                } else {
+                    // Static parameters: each thread reads its own columns' (the
+                    // rows of a block share them; L1 / L2 serve the repeats).
+                    const int64_t g = ob * inner + c0 + k;
+                    sk = __ldg(a.scale_in + g);
+                    if constexpr (NEEDR) yk = __frcp_rn(sk);
+                    zk = (OP == OP_DBWD || a.cfg.symmetric) ? 0 : load_zp(a.zp_in, g, a.cfg.q_signed);
+                }
+                const GState stk = col_state(a.cfg, sk, yk, zk);
 #pragma unroll
                 for (int j = 0; j < COL_RPT; ++j) {
                     if (r0 + (int64_t)j * RS >= gs) continue;

@@ -2208,8 +2208,8 @@ __global__ void __launch_bounds__(256, BQ_COL_MINB) k_col_tma(const __grid_const
     }
 }
 
-// Tensor map of a row-major [rows, cols] tensor of 2- or 4-byte elements in
-// boxes of box_rows x box_cols, zero fill outside (no multicast).
+// Tensor map of a row-major [rows, cols] tensor of 1-, 2- or 4-byte elements
+// in boxes of box_rows x box_cols, zero fill outside (no multicast).
 static cudaError_t encode_map_2d(CUtensorMap* tm, const void* x, int64_t rows, int64_t cols, int esz,
                                  uint32_t box_cols, uint32_t box_rows) {
     static const PFN_cuTensorMapEncodeTiled_v12000 encode = [] {
@@ -2227,7 +2227,8 @@ static cudaError_t encode_map_2d(CUtensorMap* tm, const void* x, int64_t rows, i
     const cuuint64_t gstride[1] = {(cuuint64_t)cols * (cuuint64_t)esz};
     const cuuint32_t box[2] = {box_cols, box_rows};
     const cuuint32_t estride[2] = {1, 1};
-    const CUresult r = encode(tm, esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT32,
+    const CUresult r = encode(tm, esz == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                  : (esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT32),
                               2, const_cast<void*>(x), gdim, gstride, box, estride,
                               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -2282,6 +2283,338 @@ static cudaError_t col_tma_entry(int op, const ColPipeArgs& p, cudaStream_t st) 
     return cudaErrorNotSupported;
 }
 
+// ------------------------------------------------------------ column groups, static parameters
+// Every column-group op whose parameters are given (static quantize and
+// fake-quantize, dequantize, the STE backwards, dequantize backward): tiles of
+// gs rows x CW columns of the input (and of dy for the backwards) through 2D
+// TMA into a ring of BQ_COLM_STAGES slots. The geometry is set per launch:
+// RS = min(32, gs) lanes down the rows (a power of two), CVN = 256 / RS
+// 16-byte column vectors across (CW = CVN * VEC columns <= 256, the widest
+// box). A thread reads its W columns' scale / zero-point once per tile,
+// walks its rows of the slot (shared memory), and writes its outputs; the
+// slot is refilled once every thread is done with it. The ring holds as
+// many slots (2..6) as fit in about BQ_COLM_RING_BYTES, so that three CTAs
+// share an SM whatever the slot size.
+#ifndef BQ_COLM_RING_BYTES
+#define BQ_COLM_RING_BYTES 65536
+#endif
+
+struct ColMapArgs {
+    int64_t inner, n_ct, n_tiles;
+    int gs, rs_log2, cvn, cw;       // rows per group, log2(RS), vectors across, columns per tile
+    uint32_t slot_a, slot_b;        // bytes of input a / dy in one slot (as copied)
+    uint32_t off_b, slot_bytes;     // dy's offset in a slot and the slot stride (128-byte multiples)
+    uint32_t off_s, off_z;          // the tile's scales (CW f32) and zero-points (CW bytes) in a slot
+    int has_zp;                     // zero-points are copied (asymmetric codes)
+    int stages;                     // ring slots
+    IntCfg cfg;
+    const float* scale;
+    const uint8_t* zp;
+    void* out;
+};
+
+template <class T, int OP>
+__global__ void __launch_bounds__(256) k_col_tma_map(const __grid_constant__ CUtensorMap tma,
+                                                     const __grid_constant__ CUtensorMap tmb,
+                                                     const __grid_constant__ CUtensorMap tms,
+                                                     const __grid_constant__ CUtensorMap tmz,
+                                                     ColMapArgs a) {
+    constexpr int W = Traits<T>::VEC;
+    constexpr bool TWO = (OP == OP_QBWD || OP == OP_FBWD);
+    constexpr bool NEEDR = (OP != OP_DEQ && OP != OP_DBWD);
+    const int S = a.stages;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
+    uint8_t* ring = smem + 1024;
+    const uint32_t slot_bytes = a.slot_bytes;
+    const uint32_t tx_bytes = a.slot_a + a.slot_b + (uint32_t)a.cw * 4u + (a.has_zp ? (uint32_t)a.cw : 0u);
+    const int tid = threadIdx.x;
+    const int RS = 1 << a.rs_log2;
+    const int cv = tid & (a.cvn - 1), rl = tid / a.cvn;
+    const int64_t grid = gridDim.x;
+    const int pk = a.cfg.packed;
+    // bytes per element of input a in shared memory, as a right shift of
+    // (elements * sizeof(T)): codes 1 byte (or half a byte when packed)
+    const int a_row_bytes = (OP == OP_DEQ) ? (a.cw >> pk) : a.cw * (int)sizeof(T);
+    const int b_row_bytes = a.cw * (int)sizeof(T);
+
+    if (tid == 0) {
+        for (int i = 0; i < S; ++i) mbar_init(smem_addr(&bars[i]), 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    auto issue = [&](int slot_i, int64_t tile) {
+        const uint32_t bar = smem_addr(&bars[slot_i]);
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(tx_bytes) : "memory");
+        const int c0 = (int)((tile % a.n_ct) * a.cw);
+        const int r0 = (int)((tile / a.n_ct) * a.gs);
+        uint8_t* dst = ring + (size_t)slot_i * slot_bytes;
+        tma_load_2d(smem_addr(dst), &tma, (OP == OP_DEQ) ? (c0 >> pk) : c0, r0, bar);
+        if (TWO) tma_load_2d(smem_addr(dst + a.off_b), &tmb, c0, r0, bar);
+        // the block's row of scales (and zero-points) for these columns
+        tma_load_2d(smem_addr(dst + a.off_s), &tms, c0, (int)(tile / a.n_ct), bar);
+        if (a.has_zp) tma_load_2d(smem_addr(dst + a.off_z), &tmz, c0, (int)(tile / a.n_ct), bar);
+    };
+    if (tid == 0) {
+        for (int i = 0; i < S; ++i) {
+            const int64_t t = blockIdx.x + (int64_t)i * grid;
+            if (t >= a.n_tiles) break;
+            issue(i, t);
+        }
+    }
+
+    int slot = 0;
+    uint32_t parity = 0;
+    for (int64_t tile = blockIdx.x; tile < a.n_tiles; tile += grid) {
+        const int64_t ct = tile % a.n_ct, ob = tile / a.n_ct;
+        const int64_t col = ct * a.cw + (int64_t)cv * W;         // this thread's first column
+        const bool col_ok = col < a.inner;
+        const bool ok = mbar_wait(smem_addr(&bars[slot]), parity);
+        if (ok && col_ok) {
+            // This thread's columns' parameters, copied in with the tile.
+            const uint8_t* sp = ring + (size_t)slot * slot_bytes;
+            float sk[W], yk[W];
+            int zk[W];
+#pragma unroll
+            for (int k = 0; k < W; ++k) {
+                sk[k] = reinterpret_cast<const float*>(sp + a.off_s)[cv * W + k];
+                const uint8_t zb = a.has_zp ? sp[a.off_z + cv * W + k] : (uint8_t)0;
+                zk[k] = (OP == OP_DBWD) ? 0 : (a.cfg.q_signed ? (int)(int8_t)zb : (int)zb);
+            }
+            GState st[W];
+#pragma unroll
+            for (int k = 0; k < W; ++k) {
+                if constexpr (NEEDR) yk[k] = __frcp_rn(sk[k]);
+                else yk[k] = 0.0f;
+                st[k].seg = 0;
+                st[k].s = sk[k];
+                st[k].zp = zk[k];
+                st[k].R.s = sk[k];
+                st[k].R.y = yk[k];
+                const float m = fabsf(sk[k]);
+                st[k].R.fast = (m >= 0x1p-64f) && (m <= 0x1p64f);
+                st[k].ip = make_int_params(a.cfg.qmin, a.cfg.qmax, zk[k]);
+                st[k].x_lo = st[k].x_hi = 0.0f;
+                st[k].mfast = false;
+                st[k].fast = false;
+            }
+            const uint8_t* sa = ring + (size_t)slot * slot_bytes;
+            const uint8_t* sb = sa + a.off_b;
+            bool all_fast = true;
+#pragma unroll
+            for (int k = 0; k < W; ++k) all_fast = all_fast && st[k].R.fast;
+            bool lean = false;
+            if constexpr (TWO) {
+                if (all_fast && !a.cfg.rhaz) {
+                    // STE backwards on f32 pairs: the mask from the exact quotient
+                    // (the reciprocal chain; a NaN or overflowing quotient clamps
+                    // below the code range: masked, as the exact quotient would be).
+                    Recip2 R2[W / 2];
+                    float lo[W];
+#pragma unroll
+                    for (int p = 0; p < W / 2; ++p) {
+                        R2[p].y = f2_pack(yk[2 * p], yk[2 * p + 1]);
+                        R2[p].ns = f2_pack(-sk[2 * p], -sk[2 * p + 1]);
+                    }
+#pragma unroll
+                    for (int k = 0; k < W; ++k) lo[k] = st[k].ip.lo;
+                    const float span = (float)(a.cfg.qmax - a.cfg.qmin);
+                    const F2 magic2 = f2_bcast(kMagic);
+                    for (int r = rl; r < a.gs; r += RS) {
+                        const int64_t e = (ob * a.gs + r) * a.inner + col;
+                        F2 xp[W / 2], dp[W / 2];
+                        widen_pairs<T>(ld_shared16(smem_addr(sa + r * a_row_bytes + cv * 16)), xp);
+                        widen_pairs<T>(ld_shared16(smem_addr(sb + r * b_row_bytes + cv * 16)), dp);
+                        float o[W];
+#pragma unroll
+                        for (int p = 0; p < W / 2; ++p) {
+                            float q0, q1;
+                            f2_split(div_chain2(xp[p], R2[p]), q0, q1);
+                            const float l0 = lo[2 * p], l1 = lo[2 * p + 1];
+                            q0 = fminf(fmaxf(q0, l0 - 1.0f), l0 + span + 1.0f);      // NaN -> below the range
+                            q1 = fminf(fmaxf(q1, l1 - 1.0f), l1 + span + 1.0f);
+                            float k0, k1;
+                            f2_split(f2_sub(f2_add(f2_pack(q0, q1), magic2), magic2), k0, k1);   // round half even
+                            const float m0 = (k0 > l0 && k0 < l0 + span) ? 1.0f : 0.0f;
+                            const float m1 = (k1 > l1 && k1 < l1 + span) ? 1.0f : 0.0f;
+                            F2 g = dp[p];
+                            if constexpr (OP == OP_QBWD) g = f2_mul(g, R2[p].y);
+                            f2_split(f2_mul(g, f2_pack(m0, m1)), o[2 * p], o[2 * p + 1]);
+                        }
+                        st16((T*)a.out + e, pack_vec<T>(o));
+                    }
+                    lean = true;
+                }
+            }
+            for (int r = lean ? a.gs : rl; r < a.gs; r += RS) {
+                const int64_t e = (ob * a.gs + r) * a.inner + col;
+                float o[W];
+                uint32_t cw[W];
+                if constexpr (OP == OP_DEQ) {
+                    uint32_t w[2];
+                    const uint32_t ad = smem_addr(sa + r * a_row_bytes + ((cv * W) >> pk));
+                    if (pk) {
+                        if constexpr (W == 8) {
+                            uint32_t v;
+                            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(ad));
+                            w[0] = nib_spread(v & 0xFFFFu, a.cfg.q_signed);
+                            w[1] = nib_spread(v >> 16, a.cfg.q_signed);
+                        } else {
+                            unsigned short v;
+                            asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(ad));
+                            w[0] = nib_spread(v, a.cfg.q_signed);
+                            w[1] = 0u;
+                        }
+                    } else if constexpr (W == 8) {
+                        asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "r"(ad));
+                    } else {
+                        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w[0]) : "r"(ad));
+                        w[1] = 0u;
+                    }
+#pragma unroll
+                    for (int k = 0; k < W; ++k) o[k] = deq_code_f(w[k / 4], k % 4, st[k], a.cfg.q_signed);
+                } else {
+                    float xa[W], xb[W];
+                    load_vec<T>(ld_shared16(smem_addr(sa + r * a_row_bytes + cv * 16)), xa);
+                    if constexpr (TWO) load_vec<T>(ld_shared16(smem_addr(sb + r * b_row_bytes + cv * 16)), xb);
+#pragma unroll
+                    for (int k = 0; k < W; ++k) {
+                        if (a.cfg.rhaz) o[k] = elem_f<OP, true>(xa[k], TWO ? xb[k] : 0.0f, st[k], &cw[k]);
+                        else o[k] = elem_f<OP, false>(xa[k], TWO ? xb[k] : 0.0f, st[k], &cw[k]);
+                    }
+                }
+                if constexpr (OP == OP_QUANT) st_codes<W>(code_ptr((uint8_t*)a.out, e, pk), cw, pk);
+                else st16((T*)a.out + e, pack_vec<T>(o));
+            }
+        }
+        // Every thread is done with the slot: refill it with tile + S (and a
+        // wait that gave up ends the kernel).
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) {
+                atomicOr(&g_pipe_error, 1u);
+                int s2 = slot;
+                uint32_t p2 = parity;
+                for (int i = 0; i < S; ++i) {
+                    const int64_t t2 = tile + (int64_t)i * grid;
+                    if (t2 >= a.n_tiles) break;
+                    mbar_wait(smem_addr(&bars[s2]), p2);
+                    if (++s2 == S) { s2 = 0; p2 ^= 1u; }
+                }
+            }
+            __syncthreads();
+            return;
+        }
+        if (tid == 0) {
+            const int64_t next = tile + (int64_t)S * grid;
+            if (next < a.n_tiles) {
+                fence_proxy_async();
+                issue(slot, next);
+            }
+        }
+        if (++slot == S) { slot = 0; parity ^= 1u; }
+    }
+}
+
+// Column groups with static parameters through k_col_tma_map: f32 / f16 /
+// bf16 float tensors, 8 <= gs <= 256, whole vectors per row, 16-byte aligned
+// operands; cudaErrorNotSupported otherwise. a: x, codes (OP_DEQ) or dy
+// (OP_DBWD); b: dy (OP_QBWD, OP_FBWD); out: codes (OP_QUANT) or a tensor of T.
+template <class T>
+static cudaError_t col_map_entry(int op, const void* ap, const void* bp, int64_t rows, int64_t inner,
+                                 int64_t gs, IntCfg cfg, const float* scale, const uint8_t* zp,
+                                 void* out, cudaStream_t st) {
+    constexpr int W = Traits<T>::VEC;
+    if constexpr (sizeof(T) == 8) {
+        return cudaErrorNotSupported;
+    } else {
+        const bool two = (op == OP_QBWD || op == OP_FBWD);
+        if (gs < 8 || gs > 256 || rows % gs != 0 || inner % W != 0) return cudaErrorNotSupported;
+        if (rows <= 0 || inner <= 0 || rows > 0x7FFFFF00ll || inner > 0x7FFFFF00ll) return cudaErrorNotSupported;
+        if (((uintptr_t)ap & 15u) || (two && ((uintptr_t)bp & 15u)) || ((uintptr_t)out & 15u))
+            return cudaErrorNotSupported;
+        int rs_log2 = 0;
+        while ((2 << rs_log2) <= gs && (1 << (rs_log2 + 1)) <= 32) ++rs_log2;   // RS = largest power of two <= min(gs, 32)
+        const int RS = 1 << rs_log2;
+        const int cvn = 256 / RS;
+        const int cw = cvn * W;
+        if (cw > 256) return cudaErrorNotSupported;
+        const int pk = cfg.packed;
+        const int a_esz = (op == OP_DEQ) ? 1 : (int)sizeof(T);
+        const int a_box_cols = (op == OP_DEQ) ? (cw >> pk) : cw;
+        if ((a_box_cols * a_esz) % 16 != 0) return cudaErrorNotSupported;
+        if (op == OP_DEQ && pk && (inner % 2 != 0)) return cudaErrorNotSupported;
+        // Scales [rows / gs, inner] f32 and zero-points [rows / gs, inner]
+        // bytes come in by TMA as well: 16-byte aligned, rows of whole 16 bytes.
+        const bool has_zp = zp != nullptr && !cfg.symmetric && op != OP_DBWD;
+        if (((uintptr_t)scale & 15u) || (has_zp && (((uintptr_t)zp & 15u) || inner % 16 != 0)))
+            return cudaErrorNotSupported;
+        ColMapArgs a;
+        a.inner = inner;
+        a.n_ct = (inner + cw - 1) / cw;
+        a.n_tiles = (rows / gs) * a.n_ct;
+        a.gs = (int)gs;
+        a.rs_log2 = rs_log2;
+        a.cvn = cvn;
+        a.cw = cw;
+        a.slot_a = (uint32_t)((int64_t)gs * a_box_cols * a_esz);
+        a.slot_b = two ? (uint32_t)((int64_t)gs * cw * sizeof(T)) : 0u;
+        a.off_b = (a.slot_a + 127u) & ~127u;                 // TMA destinations on 128-byte boundaries
+        a.off_s = (a.off_b + a.slot_b + 127u) & ~127u;
+        a.off_z = (a.off_s + (uint32_t)cw * 4u + 127u) & ~127u;
+        a.has_zp = has_zp ? 1 : 0;
+        a.slot_bytes = (a.off_z + (uint32_t)cw + 127u) & ~127u;
+        a.stages = (int)(BQ_COLM_RING_BYTES / a.slot_bytes);
+        if (a.stages > 6) a.stages = 6;
+        if (a.stages < 2) a.stages = 2;
+        a.cfg = cfg;
+        a.scale = scale;
+        a.zp = zp;
+        a.out = out;
+        CUtensorMap ta, tb, ts, tz;
+        const int64_t a_cols = (op == OP_DEQ) ? (inner >> pk) : inner;
+        cudaError_t e = encode_map_2d(&ta, ap, rows, a_cols, a_esz, (uint32_t)a_box_cols, (uint32_t)gs);
+        if (e != cudaSuccess) return e;
+        if (two) {
+            e = encode_map_2d(&tb, bp, rows, inner, (int)sizeof(T), (uint32_t)cw, (uint32_t)gs);
+            if (e != cudaSuccess) return e;
+        } else {
+            tb = ta;
+        }
+        e = encode_map_2d(&ts, scale, rows / gs, inner, 4, (uint32_t)cw, 1u);
+        if (e != cudaSuccess) return e;
+        if (has_zp) {
+            e = encode_map_2d(&tz, zp, rows / gs, inner, 1, (uint32_t)cw, 1u);
+            if (e != cudaSuccess) return e;
+        } else {
+            tz = ts;
+        }
+        const size_t smem = 1024 + (size_t)a.stages * a.slot_bytes;
+        if (smem > 200 * 1024) return cudaErrorNotSupported;
+        void (*k)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, ColMapArgs) = nullptr;
+        switch (op) {
+            case OP_QUANT: k = k_col_tma_map<T, OP_QUANT>; break;
+            case OP_FAKE: k = k_col_tma_map<T, OP_FAKE>; break;
+            case OP_QBWD: k = k_col_tma_map<T, OP_QBWD>; break;
+            case OP_FBWD: k = k_col_tma_map<T, OP_FBWD>; break;
+            case OP_DEQ: k = k_col_tma_map<T, OP_DEQ>; break;
+            case OP_DBWD: k = k_col_tma_map<T, OP_DBWD>; break;
+            default: return cudaErrorNotSupported;
+        }
+        if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+            return cudaErrorNotSupported;
+        int bps = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, k, 256, smem) != cudaSuccess || bps < 1) {
+            (void)cudaGetLastError();
+            return cudaErrorNotSupported;
+        }
+        int64_t grid = (int64_t)sm_count() * bps;
+        if (grid > a.n_tiles) grid = a.n_tiles;
+        if (grid < 1) grid = 1;
+        k<<<(unsigned)grid, 256, smem, st>>>(ta, tb, ts, tz, a);
+        return cudaGetLastError();
+    }
+}
+
 template <class T>
 cudaError_t pipe_error_entry(unsigned int* flag) {
     unsigned int zero = 0;
@@ -2314,6 +2647,11 @@ cudaError_t pipe_error_entry(unsigned int* flag) {
     }                                                                                            \
     cudaError_t pipe_col_##NAME(int op, const ColPipeArgs& p, cudaStream_t st) {                 \
         return col_tma_entry<T>(op, p, st);                                                      \
+    }                                                                                            \
+    cudaError_t pipe_colmap_##NAME(int op, const void* a, const void* b, int64_t rows,           \
+                                   int64_t inner, int64_t gs, IntCfg cfg, const float* scale,    \
+                                   const uint8_t* zp, void* out, cudaStream_t st) {              \
+        return col_map_entry<T>(op, a, b, rows, inner, gs, cfg, scale, zp, out, st);             \
     }
 
 }  // namespace bq
