@@ -1895,10 +1895,11 @@ cudaError_t pipe_map_entry(int op, const MapArgs& m, cudaStream_t st) {
 // ------------------------------------------------------------ column groups
 // Column groups (groups of GS consecutive rows at one column of a row-major
 // [rows, inner] tensor: the [K, N]-stored weight grouped along K) with
-// dynamic scales. Tiles of GS rows x CW columns (16 KB) reach shared memory
+// dynamic scales. Tiles of GS rows x CW columns (NT * 64 bytes: 8 KB with
+// 128-thread CTAs, so that a block barrier holds four warps) reach shared memory
 // through 2D TMA into a ring of BQ_COL_STAGES slots; columns past `inner`
 // read as zero. A thread holds COL_RPT rows of one 16-byte column vector
-// (RS = GS / 4 lanes down the rows, CVN = 256 / RS vectors across), so a
+// (RS = GS / 4 lanes down the rows, CVN = NT / RS vectors across), so a
 // tile's values sit in registers once and its slot is refilled before the
 // tile is reduced. The range runs down each column: packed 16-bit max / min
 // per thread, shuffles between the lanes of a column within a warp, then the
@@ -1920,10 +1921,14 @@ struct ColTileArgs {
     void* out;
 };
 
+#ifndef BQ_COLT_NT
+#define BQ_COLT_NT 128
+#endif
 template <class T, int GS> struct ColTileGeom {
+    static constexpr int NT = BQ_COLT_NT;               // threads per CTA
     static constexpr int W = Traits<T>::VEC;
     static constexpr int RS = GS / COLT_RPT;            // lanes down the rows
-    static constexpr int CVN = 256 / RS;                // vectors across a tile row
+    static constexpr int CVN = NT / RS;                 // vectors across a tile row
     static constexpr int CW = CVN * W;                  // columns per tile
     static constexpr bool H = sizeof(T) == 2;
     static constexpr int NP = H ? W / 2 : W;            // range words per thread
@@ -1934,7 +1939,7 @@ template <class T, int GS> struct ColTileGeom {
     static constexpr int NPAR = 6;                      // per-column parameter arrays
     static constexpr int RING_OFF = ((PAR_OFF + NPAR * CW * 4) + 1023) / 1024 * 1024;
     static_assert(CW <= 256 && (CW * sizeof(T)) % 16 == 0, "TMA box");
-    static_assert(SLOT == 16384, "slot size");
+    static_assert(SLOT == (uint32_t)NT * 64, "slot size");
 };
 
 template <class T>
@@ -1956,12 +1961,12 @@ __device__ __forceinline__ void col_word_vals(uint32_t w, float& v0, float& v1) 
 }
 
 template <class T, int OP, int GS>
-__global__ void __launch_bounds__(256, BQ_COL_MINB) k_col_tma(const __grid_constant__ CUtensorMap tm, ColTileArgs a) {
+__global__ void __launch_bounds__(BQ_COLT_NT, BQ_COL_MINB) k_col_tma(const __grid_constant__ CUtensorMap tm, ColTileArgs a) {
     using G = ColTileGeom<T, GS>;
     constexpr int W = G::W, RS = G::RS, CVN = G::CVN, CW = G::CW, NP = G::NP, NWORDS = G::NWORDS;
     constexpr int S = BQ_COL_STAGES;
     constexpr uint32_t SLOT = G::SLOT;
-    constexpr int NW = 8;
+    constexpr int NW = G::NT / 32;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
     uint32_t* red_hi = reinterpret_cast<uint32_t*>(smem + G::RED_OFF);      // [NW][NWORDS]
@@ -2254,12 +2259,12 @@ static cudaError_t col_tma_launch(const ColPipeArgs& p, cudaStream_t st) {
     static const cudaError_t attr = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (attr != cudaSuccess) return attr;
     static unsigned long long occ[8];
-    const int bps = occupancy_for((const void*)k, smem, occ);
+    const int bps = occupancy_for((const void*)k, smem, occ, G::NT);
     if (bps < 1) return cudaErrorNotSupported;
     int64_t grid = (int64_t)sm_count() * bps;
     if (grid > a.n_tiles) grid = a.n_tiles;
     if (grid < 1) grid = 1;
-    k<<<(unsigned)grid, 256, smem, st>>>(tm, a);
+    k<<<(unsigned)grid, G::NT, smem, st>>>(tm, a);
     return cudaGetLastError();
 }
 
