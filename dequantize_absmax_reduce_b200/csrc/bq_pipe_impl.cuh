@@ -2295,9 +2295,11 @@ static cudaError_t col_tma_entry(int op, const ColPipeArgs& p, cudaStream_t st) 
 // TMA into a ring of BQ_COLM_STAGES slots. The geometry is set per launch:
 // RS = min(32, gs) lanes down the rows (a power of two), CVN = 256 / RS
 // 16-byte column vectors across (CW = CVN * VEC columns <= 256, the widest
-// box). A thread reads its W columns' scale / zero-point once per tile,
+// box). The tile's CW scales (and zero-points) come into the same slot by
+// TMA; a thread reads its W columns' parameters from there once per tile,
 // walks its rows of the slot (shared memory), and writes its outputs; the
-// slot is refilled once every thread is done with it. The ring holds as
+// slot is refilled once every thread is done with it. The STE backwards with
+// normal scales take the mask from the exact quotient on f32 pairs. The ring holds as
 // many slots (2..6) as fit in about BQ_COLM_RING_BYTES, so that three CTAs
 // share an SM whatever the slot size.
 #ifndef BQ_COLM_RING_BYTES
@@ -2313,8 +2315,6 @@ struct ColMapArgs {
     int has_zp;                     // zero-points are copied (asymmetric codes)
     int stages;                     // ring slots
     IntCfg cfg;
-    const float* scale;
-    const uint8_t* zp;
     void* out;
 };
 
@@ -2572,8 +2572,6 @@ static cudaError_t col_map_entry(int op, const void* ap, const void* bp, int64_t
         if (a.stages > 6) a.stages = 6;
         if (a.stages < 2) a.stages = 2;
         a.cfg = cfg;
-        a.scale = scale;
-        a.zp = zp;
         a.out = out;
         CUtensorMap ta, tb, ts, tz;
         const int64_t a_cols = (op == OP_DEQ) ? (inner >> pk) : inner;
