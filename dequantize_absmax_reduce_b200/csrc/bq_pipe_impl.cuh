@@ -2074,22 +2074,25 @@ __global__ void __launch_bounds__(BQ_COLT_NT, BQ_COL_MINB) k_col_tma(const __gri
             }
         }
         __syncthreads();
-        // ---- one thread per range word: the tile's column parameters
+        // ---- one thread per column: the tile's column parameters (the two
+        // threads of a 16-bit column pair reduce the same range words)
         bool slow_col = false;
-        if (tid < NWORDS) {
-            uint32_t h = red_hi[tid], l = red_lo[tid];
+        constexpr int CPW = G::H ? 2 : 1;     // columns per range word
+        static_assert(NWORDS * CPW <= G::NT, "one thread per column");
+        if (tid < NWORDS * CPW) {
+            const int wd = tid / CPW;
+            uint32_t h = red_hi[wd], l = red_lo[wd];
 #pragma unroll
             for (int w = 1; w < NW; ++w) {
-                h = col_pk_max<T>(h, red_hi[w * NWORDS + tid]);
-                l = col_pk_min<T>(l, red_lo[w * NWORDS + tid]);
+                h = col_pk_max<T>(h, red_hi[w * NWORDS + wd]);
+                l = col_pk_min<T>(l, red_lo[w * NWORDS + wd]);
             }
             float h0, h1, l0, l1;
             col_word_vals<T>(h, h0, h1);
             col_word_vals<T>(l, l0, l1);
-            constexpr int CPW = G::H ? 2 : 1;     // columns per word
-#pragma unroll
-            for (int u = 0; u < CPW; ++u) {
-                const int c = tid * CPW + u;
+            {
+                const int u = tid % CPW;
+                const int c = tid;
                 // Scale fl(amax/qmax) or fl(fl(max'-min')/(qmax-qmin)) and
                 // zero-point, each quotient through a reciprocal chain
                 // (exact for a normal dividend; IEEE division outside).
