@@ -371,7 +371,9 @@ bq_status bq_tensor_amax(const void* x, bq_dtype dtype, int64_t n, float* amax, 
     if (!aligned(ws, 8) || !aligned(amax, 4) || !aligned(x, esize(dtype))) return BQ_ERR_MISALIGNED;
     cudaStream_t s = S(stream);
     if (bq::clear_records((unsigned long long*)ws, 2, s) != cudaSuccess) return BQ_ERR_CUDA;
-    cudaError_t e = bq::tensor_range(to_dt(dtype), x, n, true, (unsigned long long*)ws, s);
+    cudaError_t e = bq::tensor_amax_pipe(to_dt(dtype), x, n, (unsigned long long*)ws, amax, s);
+    if (e != cudaErrorNotSupported) return from_cuda(e);
+    e = bq::tensor_range(to_dt(dtype), x, n, true, (unsigned long long*)ws, s);
     if (e != cudaSuccess) return BQ_ERR_CUDA;
     return from_cuda(bq::range_to_amax((const unsigned long long*)ws, amax, s));
 }

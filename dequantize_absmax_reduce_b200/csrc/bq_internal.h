@@ -78,6 +78,11 @@ cudaError_t tensor_range(DT dt, const void* x, int64_t n, bool sym, unsigned lon
 // The bulk-copy pipelined range kernel behind tensor_range (f32 / f16 / bf16).
 cudaError_t tensor_range_pipe(DT dt, const void* x, int64_t n, bool sym, unsigned long long* rec,
                               cudaStream_t st);
+// Tensor amax in one pass after the clearing kernel: the pipelined range
+// kernel's last CTA writes max |x| to *amax (rec: two cleared records, the
+// second used as a CTA counter). cudaErrorNotSupported for f64.
+cudaError_t tensor_amax_pipe(DT dt, const void* x, int64_t n, unsigned long long* rec, float* amax,
+                             cudaStream_t st);
 // Clears n 64-bit range records; the first kernel of a two-pass call.
 cudaError_t clear_records(unsigned long long* rec, int64_t n, cudaStream_t st);
 // Parameters of groups with no elements (scale 1, zero-point of a zero range).

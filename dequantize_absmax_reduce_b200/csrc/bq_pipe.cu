@@ -19,6 +19,9 @@ cudaError_t pipe_err_bf16(unsigned int* flag);
 cudaError_t pipe_range_f32(const void* x, int64_t n, bool sym, unsigned long long* rec, cudaStream_t st);
 cudaError_t pipe_range_f16(const void* x, int64_t n, bool sym, unsigned long long* rec, cudaStream_t st);
 cudaError_t pipe_range_bf16(const void* x, int64_t n, bool sym, unsigned long long* rec, cudaStream_t st);
+cudaError_t pipe_amax_f32(const void* x, int64_t n, unsigned long long* rec, float* amax, cudaStream_t st);
+cudaError_t pipe_amax_f16(const void* x, int64_t n, unsigned long long* rec, float* amax, cudaStream_t st);
+cudaError_t pipe_amax_bf16(const void* x, int64_t n, unsigned long long* rec, float* amax, cudaStream_t st);
 cudaError_t pipe_tile_f32(const void* x, int64_t rows, int64_t cols, uint8_t* e4m3, float* scale, cudaStream_t st);
 cudaError_t pipe_tile_f16(const void* x, int64_t rows, int64_t cols, uint8_t* e4m3, float* scale, cudaStream_t st);
 cudaError_t pipe_tile_bf16(const void* x, int64_t rows, int64_t cols, uint8_t* e4m3, float* scale, cudaStream_t st);
@@ -92,6 +95,16 @@ cudaError_t tensor_range_pipe(DT dt, const void* x, int64_t n, bool sym, unsigne
         case DT::F32: return pipe_range_f32(x, n, sym, rec, st);
         case DT::F16: return pipe_range_f16(x, n, sym, rec, st);
         case DT::BF16: return pipe_range_bf16(x, n, sym, rec, st);
+        default: return cudaErrorNotSupported;
+    }
+}
+
+cudaError_t tensor_amax_pipe(DT dt, const void* x, int64_t n, unsigned long long* rec, float* amax,
+                             cudaStream_t st) {
+    switch (dt) {
+        case DT::F32: return pipe_amax_f32(x, n, rec, amax, st);
+        case DT::F16: return pipe_amax_f16(x, n, rec, amax, st);
+        case DT::BF16: return pipe_amax_bf16(x, n, rec, amax, st);
         default: return cudaErrorNotSupported;
     }
 }

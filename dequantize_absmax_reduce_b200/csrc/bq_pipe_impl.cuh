@@ -1089,6 +1089,7 @@ struct RangeArgs {
     int64_t body_bytes;   // multiple of 16
     int64_t n;            // all elements
     unsigned long long* rec;
+    float* amax;          // tensor amax: written by the last CTA (ABS only; rec[1] counts CTAs)
 };
 
 template <class T, bool ABS>
@@ -1187,6 +1188,20 @@ __global__ void __launch_bounds__(256) k_range_pipe(RangeArgs a) {
         pdl_wait();
         atomicMax(a.rec, range_bits(hi));
         if (!ABS) atomicMax(a.rec + 1, range_bits(nlo));
+        if (ABS && a.amax) {
+            // The last CTA to finish turns the record into the amax: rec[1]
+            // (unused by an absolute range, zeroed by the clearing kernel)
+            // counts finished CTAs; each CTA's maximum is visible before its
+            // count (fence), so the last one reads the final record.
+            __threadfence();
+            const unsigned long long done = atomicAdd(a.rec + 1, 1ull);
+            if (done == (unsigned long long)gridDim.x - 1ull) {
+                __threadfence();
+                float h;
+                range_from_bits(atomicAdd(a.rec, 0ull), h);
+                *a.amax = h;
+            }
+        }
     }
 }
 
@@ -1752,8 +1767,9 @@ static cudaError_t seg_map_dt(int op, const MapArgs& m, cudaStream_t st) {
 // the stream); launched to overlap that kernel (launch_pdl).
 template <class T>
 static cudaError_t range_entry(const void* x, int64_t n, bool sym, unsigned long long* rec,
-                               cudaStream_t st) {
+                               cudaStream_t st, float* amax = nullptr) {
     RangeArgs a;
+    a.amax = sym ? amax : nullptr;
     a.x = x;
     a.n = n;
     a.head = 0;
@@ -2642,6 +2658,10 @@ cudaError_t pipe_error_entry(unsigned int* flag) {
     cudaError_t pipe_range_##NAME(const void* x, int64_t n, bool sym, unsigned long long* rec,   \
                                   cudaStream_t st) {                                              \
         return range_entry<T>(x, n, sym, rec, st);                                               \
+    }                                                                                            \
+    cudaError_t pipe_amax_##NAME(const void* x, int64_t n, unsigned long long* rec, float* amax,  \
+                                 cudaStream_t st) {                                               \
+        return range_entry<T>(x, n, true, rec, st, amax);                                        \
     }                                                                                            \
     cudaError_t pipe_tile_##NAME(const void* x, int64_t rows, int64_t cols, uint8_t* e4m3,       \
                                  float* scale, cudaStream_t st) {                                 \

@@ -170,9 +170,11 @@ bq_status bq_group_range(const void* x, const bq_qdesc* d, bq_gran gran, int32_t
                          int64_t group_size, void* ranges, void* stream);
 
 /* Tensor amax: max |x| over n elements of dtype (F32, F16, BF16), NaN
- * ignored, written as f32 to *amax. ws: 16 bytes of device scratch. This is
- * the first pass of per-tensor scaling and of the NVFP4 per-tensor scale
- * ([QuantizedWeight] weight_scale_2). */
+ * ignored, written as f32 to *amax. ws: 16 bytes of device scratch (cleared
+ * by the call; afterwards it holds no range record). This is the first pass
+ * of per-tensor scaling and of the NVFP4 per-tensor scale ([QuantizedWeight]
+ * weight_scale_2). Two kernels: a clearing kernel, then the range kernel,
+ * whose last CTA writes *amax. */
 bq_status bq_tensor_amax(const void* x, bq_dtype dtype, int64_t n, float* amax, void* ws,
                          void* stream);
 
