@@ -39,6 +39,9 @@ CASES = [  # (shape, axis, gs)
     ((64, 7), 0, 1),               # every element its own group
     ((40, 1), 0, 8),               # one column
     ((9, 33, 40), 2, 5),           # nothing after the axis: contiguous groups
+    ((48, 40), 0, 24),             # 24 rows: 16 lanes down, ragged column tile
+    ((36, 136), 0, 12),            # 12 rows: 8 lanes down, the widest tile
+    ((2, 16, 72), 1, 8),           # the shortest groups the TMA kernels take
 ]
 
 
