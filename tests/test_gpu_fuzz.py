@@ -2,7 +2,7 @@
 shapes, axes, group lengths (contiguous and column groups), dtypes, code
 types (s8 / u8 / s4 / u4), symmetric or not, rounding mode and a pointer
 offset that makes the input misaligned. Each case runs quantize (dynamic and
-static), dequantize, fake-quantize and the STE backward, so every dispatch
+static), dequantize, fake-quantize and the three backwards, so every dispatch
 decision (vector or element paths, pipelined, TMA or fallback kernels) meets
 a variety of sizes. Cases a kernel does not take (packed codes on shapes
 without whole vectors) must be refused with a status, never computed wrong.
@@ -95,3 +95,9 @@ def test_random_integer_case(bq, orc, case):
                                gs, QD[qd], sym, rnd=rnd)
     assert_ulp(dx, orc.quantize_backward(x, dy, s2, rzz, gran, axis, gs, qd, sym, rhaz=rhaz), 1,
                "STE backward")
+    fdx = api.fake_quantize_backward(xg, dyg, s2.cuda(), None if rzz is None else rzz.cuda(), gran,
+                                     axis, gs, QD[qd], sym, rnd=rnd)
+    assert_bitwise(fdx, orc.fake_quantize_backward(x, dy, s2, rzz, gran, axis, gs, qd, sym, rhaz=rhaz),
+                   "fake-quantize backward")
+    dq = api.dequantize_backward(dyg, s2.cuda(), gran, axis, gs)
+    assert_bitwise(dq, orc.dequantize_backward(dy, s2, gran, axis, gs), "dequantize backward")
