@@ -304,7 +304,7 @@ def per_granularity(B, api, torch, device, peak, reps=5):
     # The same tensor as a [K, N] weight grouped along K (column groups, GPTQ layout).
     wlc = "column_group128_f16_11008x4096"
     timed(wlc, "quantize_per_column_group(axis=0,gs=128,u8 asym)",
-          lambda: B.bq_quantize_per_column_group(x, du, 0, 128, q, s, z, "dynamic"), 3 * n + 5 * ng, 1)
+          lambda: B.bq_quantize_per_column_group(x, du, 0, 128, q, s, z, "dynamic", None), 3 * n + 5 * ng, 1)
     timed(wlc, "dequantize_per_column_group",
           lambda: B.bq_dequantize_per_column_group(q, s, z, du, 0, 128, y), 3 * n + 5 * ng, 1)
     timed(wlc, "fake_quantize(column_group,dynamic)",
@@ -320,7 +320,7 @@ def per_granularity(B, api, torch, device, peak, reps=5):
     timed(wl, "dequantize_per_group(u4 packed)",
           lambda: B.bq_dequantize_per_group(q4, s, z, d4, 1, 128, y), 2 * n + n // 2 + 5 * ng, 1)
     timed(wlc, "quantize_per_column_group(axis=0,gs=128,u4 asym, packed)",
-          lambda: B.bq_quantize_per_column_group(x, d4, 0, 128, q4, s, z, "dynamic"), 2 * n + n // 2 + 5 * ng, 1)
+          lambda: B.bq_quantize_per_column_group(x, d4, 0, 128, q4, s, z, "dynamic", None), 2 * n + n // 2 + 5 * ng, 1)
     del w, x, dy, q, qs, y, dx, q4
 
     # NVFP4 bf16 [4096, 7168]

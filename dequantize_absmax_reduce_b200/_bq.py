@@ -65,7 +65,7 @@ _SIGS = {
     "bq_quantize_per_channel": [_P, _DESC, _I32, _P, _P, _P, C.c_int, _P, _SZ, _P],
     "bq_quantize_per_token": [_P, _DESC, _P, _P, _P, C.c_int, _P, _SZ, _P],
     "bq_quantize_per_group": [_P, _DESC, _I32, _I64, _P, _P, _P, C.c_int, _P, _SZ, _P],
-    "bq_quantize_per_column_group": [_P, _DESC, _I32, _I64, _P, _P, _P, C.c_int, _P],
+    "bq_quantize_per_column_group": [_P, _DESC, _I32, _I64, _P, _P, _P, C.c_int, _P, _SZ, _P],
     "bq_quantize_dynamic_noalloc": [_P, _DESC, C.c_int, _I32, _I64, _P, _P, _P, _P],
     "bq_dequantize_per_tensor": [_P, _P, _P, _DESC, _P, C.c_int, _P],
     "bq_dequantize_per_channel": [_P, _P, _P, _DESC, _I32, _P, C.c_int, _P],
@@ -242,9 +242,10 @@ def bq_quantize_per_group(x, d, axis, group_size, q, scale, zp, mode, ws=None, s
            "bq_quantize_per_group")
 
 
-def bq_quantize_per_column_group(x, d, axis, group_size, q, scale, zp, mode, stream=None):
+def bq_quantize_per_column_group(x, d, axis, group_size, q, scale, zp, mode, ws=None, stream=None):
     _check(lib.bq_quantize_per_column_group(_ptr(x), C.byref(d), axis, group_size, _ptr(q),
-                                            _ptr(scale), _ptr(zp), _m(mode), _stream(stream)),
+                                            _ptr(scale), _ptr(zp), _m(mode), _ptr(ws), _nbytes(ws),
+                                            _stream(stream)),
            "bq_quantize_per_column_group")
 
 

@@ -75,9 +75,7 @@ def quantize(x: torch.Tensor, gran: str, axis: int = 0, group_size: int = 1,
     elif gran == "channel":
         B.bq_quantize_per_channel(x, d, axis, q, scale, zp, mode, ws, stream)
     elif gran == "column_group":
-        if mode == "from_range":
-            raise ValueError("column groups take no range records")
-        B.bq_quantize_per_column_group(x, d, axis, group_size, q, scale, zp, mode, stream)
+        B.bq_quantize_per_column_group(x, d, axis, group_size, q, scale, zp, mode, ws, stream)
     else:
         B.bq_quantize_per_group(x, d, axis, group_size, q, scale, zp, mode, ws, stream)
     return q, scale, zp

@@ -156,7 +156,6 @@ bq_status quant_impl(int op, const void* x, const bq_qdesc* d, int gr, int32_t a
     if ((st = make_cfg(d, true, &cfg)) != BQ_OK) return st;
     if (mode != BQ_SCALE_DYNAMIC && mode != BQ_SCALE_STATIC && mode != BQ_SCALE_FROM_RANGE)
         return BQ_ERR_INVALID_ARG;
-    if (lay.column && mode == BQ_SCALE_FROM_RANGE) return BQ_ERR_UNSUPPORTED;
     const bq::SegView sv = lay.sv;
     const bool asym = !cfg.symmetric;
     if (sv.numel > 0 && !x) return BQ_ERR_INVALID_ARG;
@@ -176,10 +175,12 @@ bq_status quant_impl(int op, const void* x, const bq_qdesc* d, int gr, int32_t a
     const DT dt = to_dt(d->x_dtype);
     cudaStream_t s = S(stream);
     if (lay.column) {
-        // Column groups run in one pass over x for either mode; there are
-        // no range records to derive them from.
+        // Column groups run in one pass over x in every mode.
         if (sv.n_seg == 0) return BQ_OK;
         void* out = (op == bq::OP_QUANT) ? q : y;
+        if (mode == BQ_SCALE_FROM_RANGE)
+            return from_cuda(bq::col_groups_from_range(dt, op, x, lay.cv, cfg, (const unsigned long long*)ws,
+                                                       scale, zp, out, s));
         const bool dyn = mode == BQ_SCALE_DYNAMIC;
         return from_cuda(bq::col_groups(dt, op, dyn ? 1 : 0, x, nullptr, lay.cv, cfg, scale, zp,
                                         dyn ? scale : nullptr, dyn ? zp : nullptr, out, s));
@@ -338,7 +339,8 @@ size_t bq_quantize_workspace_size(const bq_qdesc* d, bq_gran gran, int32_t axis,
     const int gr = gran_to_gr(gran);
     Layout lay;
     if (gr < 0 || make_layout(d, gr, axis, group_size, &lay) != BQ_OK) return 0;
-    if (mode == BQ_SCALE_STATIC || lay.column) return 0;
+    if (mode == BQ_SCALE_STATIC) return 0;
+    if (lay.column) return mode == BQ_SCALE_FROM_RANGE ? (size_t)lay.sv.n_seg * 16 : 0;
     if (mode == BQ_SCALE_FROM_RANGE) return (size_t)lay.sv.n_seg * 16;
     return single_pass_possible(d, lay.sv) ? 0 : (size_t)lay.sv.n_seg * 16;
 }
@@ -350,12 +352,14 @@ bq_status bq_group_range(const void* x, const bq_qdesc* d, bq_gran gran, int32_t
     Layout lay;
     bq_status st = make_layout(d, gr, axis, group_size, &lay);
     if (st != BQ_OK) return st;
-    if (!is_float(d->x_dtype) || lay.column) return BQ_ERR_UNSUPPORTED;
+    if (!is_float(d->x_dtype)) return BQ_ERR_UNSUPPORTED;
     const bq::SegView sv = lay.sv;
     if (sv.n_seg == 0) return BQ_OK;
     if (!ranges || (sv.numel > 0 && !x)) return BQ_ERR_INVALID_ARG;
     if (!aligned(ranges, 8) || !aligned(x, esize(d->x_dtype))) return BQ_ERR_MISALIGNED;
     cudaStream_t s = S(stream);
+    if (lay.column)     // one record pair per column group, written once (no clearing)
+        return from_cuda(bq::col_groups_range(to_dt(d->x_dtype), x, lay.cv, (unsigned long long*)ranges, s));
     if (bq::clear_records((unsigned long long*)ranges, 2 * sv.n_seg, s) != cudaSuccess) return BQ_ERR_CUDA;
     // Both slots are always filled, so the records serve either scaling.
     cudaError_t e = (sv.n_seg == 1)
@@ -412,9 +416,10 @@ bq_status bq_quantize_per_group(const void* x, const bq_qdesc* d, int32_t axis,
 }
 bq_status bq_quantize_per_column_group(const void* x, const bq_qdesc* d, int32_t axis,
                                        int64_t group_size, void* q, float* scale, void* zp,
-                                       bq_scale_mode mode, void* stream) {
+                                       bq_scale_mode mode, void* ws, size_t ws_bytes,
+                                       void* stream) {
     return quant_impl(bq::OP_QUANT, x, d, GR_COLUMN, axis, group_size, q, scale, zp, mode,
-                      nullptr, nullptr, 0, stream);
+                      nullptr, ws, ws_bytes, stream);
 }
 
 // ---- dequantize

@@ -22,6 +22,11 @@ cudaError_t pipe_colmap_bf16(int op, const void* a, const void* b, int64_t rows,
 
 static bool al(const void* p, int n) { return !p || ((uintptr_t)p % (uintptr_t)n) == 0; }
 
+cudaError_t col_generic(DT dt, int op, int dyn, const void* a, const void* b, ColView v, IntCfg cfg,
+                        const float* scale_in, const void* zp_in, float* scale_out, void* zp_out,
+                        void* out, const unsigned long long* ranges_in, unsigned long long* ranges_out,
+                        cudaStream_t st);
+
 cudaError_t col_groups(DT dt, int op, int dyn, const void* a, const void* b, ColView v, IntCfg cfg,
                        const float* scale_in, const void* zp_in, float* scale_out, void* zp_out,
                        void* out, cudaStream_t st) {
@@ -42,6 +47,17 @@ cudaError_t col_groups(DT dt, int op, int dyn, const void* a, const void* b, Col
                                             : pipe_colmap_bf16(op, a, b, rows, v.inner, v.gs, cfg, scale_in, z, out, st);
         if (e != cudaErrorNotSupported) return e;
     }
+    return col_generic(dt, op, dyn, a, b, v, cfg, scale_in, zp_in, scale_out, zp_out, out, nullptr,
+                       nullptr, st);
+}
+
+// The element-tiled kernel (k_col) for every case, FROM_RANGE parameters
+// (ranges_in) and range records (op COL_OP_RANGE, ranges_out) included.
+cudaError_t col_generic(DT dt, int op, int dyn, const void* a, const void* b, ColView v, IntCfg cfg,
+                        const float* scale_in, const void* zp_in, float* scale_out, void* zp_out,
+                        void* out, const unsigned long long* ranges_in, unsigned long long* ranges_out,
+                        cudaStream_t st) {
+    if (v.outer == 0 || v.L == 0 || v.inner == 0) return cudaSuccess;
     const int vec_n = dt == DT::F32 ? 4 : (dt == DT::F64 ? 2 : 8);
     // Vectors need whole vectors per row and aligned operands: 16 bytes for
     // float tensors, one vector's worth of bytes for code tensors.
@@ -53,6 +69,8 @@ cudaError_t col_groups(DT dt, int op, int dyn, const void* a, const void* b, Col
     ColArgs c;
     c.a = a;
     c.b = b;
+    c.ranges_in = ranges_in;
+    c.ranges_out = ranges_out;
     c.inner = v.inner;
     c.gs = v.gs;
     c.n_ct = 0;
@@ -70,6 +88,20 @@ cudaError_t col_groups(DT dt, int op, int dyn, const void* a, const void* b, Col
         case DT::F64: return col_groups_f64(op, dyn, c, vec, st);
     }
     return cudaErrorInvalidValue;
+}
+
+cudaError_t col_groups_range(DT dt, const void* x, ColView v, unsigned long long* ranges,
+                             cudaStream_t st) {
+    IntCfg cfg{-128, 127, 0, 0, 1, 0};
+    return col_generic(dt, COL_OP_RANGE, 1, x, nullptr, v, cfg, nullptr, nullptr, nullptr, nullptr,
+                       nullptr, nullptr, ranges, st);
+}
+
+cudaError_t col_groups_from_range(DT dt, int op, const void* x, ColView v, IntCfg cfg,
+                                  const unsigned long long* ranges, float* scale_out, void* zp_out,
+                                  void* out, cudaStream_t st) {
+    return col_generic(dt, op, 0, x, nullptr, v, cfg, nullptr, nullptr, scale_out, zp_out, out, ranges,
+                       nullptr, st);
 }
 
 }  // namespace bq

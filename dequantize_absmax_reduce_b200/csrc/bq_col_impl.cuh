@@ -23,9 +23,15 @@
 
 namespace bq {
 
+// Range records of every column group (bq_group_range): the dynamic
+// kernel's reduction with the two records written in place of the codes.
+constexpr int COL_OP_RANGE = 16;
+
 struct ColArgs {
     const void* a;          // x, q or dy
     const void* b;          // dy (STE backwards)
+    const unsigned long long* ranges_in;   // FROM_RANGE: parameters derived from these records
+    unsigned long long* ranges_out;        // COL_OP_RANGE: the records written
     int64_t inner, gs;      // row width (columns) and group length (rows)
     int64_t n_ct;           // column tiles per row
     int64_t n_tiles;        // outer * (L / gs) * n_ct
@@ -266,12 +272,21 @@ __global__ void __launch_bounds__(256) k_col(ColArgs a) {
                 if constexpr (NEEDR) col_y[par][tid] = __frcp_rn(s);
                 const int64_t c = ct * CW + tid;
                 if (c < inner) {
-                    a.scale_out[ob * inner + c] = s;
-                    if (a.zp_out) a.zp_out[ob * inner + c] = (uint8_t)z;
+                    if constexpr (OP == COL_OP_RANGE) {
+                        // max(0, max x) and max(0, -min x) as non-negative IEEE
+                        // bits (a zero of either sign becomes +0), so that records
+                        // combine with an integer MAX
+                        a.ranges_out[2 * (ob * inner + c)] = range_bits(h + (Acc)0);
+                        a.ranges_out[2 * (ob * inner + c) + 1] = range_bits((Acc)0 - l);
+                    } else {
+                        a.scale_out[ob * inner + c] = s;
+                        if (a.zp_out) a.zp_out[ob * inner + c] = (uint8_t)z;
+                    }
                 }
             }
             __syncthreads();
         }
+        if constexpr (OP == COL_OP_RANGE) continue;
         if (!col_ok) continue;      // no barrier below this point
 
         // ---- element pass over the block's rows, one column at a time (one
@@ -305,6 +320,25 @@ __global__ void __launch_bounds__(256) k_col(ColArgs a) {
                     sk = col_s[par][c];
                     if constexpr (NEEDR) yk = col_y[par][c];
                     zk = col_z[par][c];
+                } else if (a.ranges_in) {
+                    // Parameters from range records (FROM_RANGE), written out by
+                    // the first lane of each column.
+                    const int64_t g = ob * inner + c0 + k;
+                    Acc h, n;
+                    range_from_bits(a.ranges_in[2 * g], h);
+                    range_from_bits(a.ranges_in[2 * g + 1], n);
+                    if constexpr (WIDE) {
+                        const GroupD gp = derive_d(h, n, a.cfg);
+                        sk = gp.s; zk = gp.zp;
+                    } else {
+                        const GroupF gp = derive_f(h, n, a.cfg);
+                        sk = gp.s; zk = gp.zp;
+                    }
+                    if constexpr (NEEDR) yk = __frcp_rn(sk);
+                    if (rl == 0 && r0 == rl) {
+                        a.scale_out[g] = sk;
+                        if (a.zp_out) a.zp_out[g] = (uint8_t)zk;
+                    }
                 } else {
                     // Static parameters: each thread reads its own columns' (the
                     // rows of a block share them; L1 / L2 serve the repeats).
@@ -420,6 +454,7 @@ static cudaError_t col_entry(int op, int dyn, const ColArgs& a, bool vec, cudaSt
                         : col_launch_r<T, OP_FBWD, false, false>(a, vec, st);
         case OP_DEQ: return col_launch_r<T, OP_DEQ, false, false>(a, vec, st);
         case OP_DBWD: return col_launch_r<T, OP_DBWD, false, false>(a, vec, st);
+        case COL_OP_RANGE: return col_launch_r<T, COL_OP_RANGE, true, false>(a, vec, st);
     }
     return cudaErrorInvalidValue;
 }

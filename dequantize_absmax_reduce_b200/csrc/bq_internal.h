@@ -65,6 +65,15 @@ struct ColView {
 cudaError_t col_groups(DT dt, int op, int dyn, const void* a, const void* b, ColView v, IntCfg cfg,
                        const float* scale_in, const void* zp_in, float* scale_out, void* zp_out,
                        void* out, cudaStream_t st);
+// Range records of every column group ([outer, L/gs, inner] x 2 uint64, the
+// layout bq_group_range documents), written directly (no clearing needed).
+cudaError_t col_groups_range(DT dt, const void* x, ColView v, unsigned long long* ranges,
+                             cudaStream_t st);
+// Quantize / fake-quantize of column groups with parameters derived from
+// range records (FROM_RANGE), written to scale_out / zp_out.
+cudaError_t col_groups_from_range(DT dt, int op, const void* x, ColView v, IntCfg cfg,
+                                  const unsigned long long* ranges, float* scale_out, void* zp_out,
+                                  void* out, cudaStream_t st);
 
 // Range records of every group (ranges cleared by the caller).
 cudaError_t seg_range(DT dt, const void* x, SegView sv, bool sym, unsigned long long* ranges,

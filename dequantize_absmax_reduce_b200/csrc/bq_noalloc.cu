@@ -52,7 +52,7 @@ extern "C" bq_status bq_quantize_dynamic_noalloc(const void* x, const bq_qdesc* 
     // Column groups take one pass over x and no records.
     if (gran == BQ_GRAN_COLUMN_GROUP)
         return bq_quantize_per_column_group(x, d, axis, group_size, q, scale, zp, BQ_SCALE_DYNAMIC,
-                                            stream);
+                                            nullptr, 0, stream);
     int64_t n_groups = 0, group_elems = 0;
     bq_status st = bq_group_count(d, gran, axis, group_size, &n_groups, &group_elems);
     if (st != BQ_OK) return st;

@@ -87,10 +87,10 @@ typedef enum bq_round { BQ_RNE = 0, BQ_RHAZ = 1 } bq_round;
  * around `axis`, group (o, b, i) holds the group_size elements
  * x[o, b*gs + r, i], r < gs, which lie `inner` elements apart; scale / zp are
  * [outer, L/gs, inner] row-major. Accepted by bq_group_count,
- * bq_quantize_workspace_size (always 0), bq_fake_quantize (DYNAMIC and
- * STATIC), bq_fake_quantize_backward, bq_quantize_dynamic_noalloc and the
- * *_per_column_group entry points; bq_group_range and FROM_RANGE scaling
- * return BQ_ERR_UNSUPPORTED for it. */
+ * bq_quantize_workspace_size (16 bytes per group for FROM_RANGE, else 0),
+ * bq_group_range (records written directly, one pair per column group),
+ * bq_fake_quantize (every mode), bq_fake_quantize_backward,
+ * bq_quantize_dynamic_noalloc and the *_per_column_group entry points. */
 typedef enum bq_gran {
     BQ_GRAN_TENSOR = 0, BQ_GRAN_CHANNEL = 1, BQ_GRAN_GROUP = 2, BQ_GRAN_COLUMN_GROUP = 3
 } bq_gran;
@@ -203,12 +203,14 @@ bq_status bq_quantize_per_token(const void* x, const bq_qdesc* d, void* q, float
 bq_status bq_quantize_per_group(const void* x, const bq_qdesc* d, int32_t axis,
                                 int64_t group_size, void* q, float* scale, void* zp,
                                 bq_scale_mode mode, void* ws, size_t ws_bytes, void* stream);
-/* Column groups (BQ_GRAN_COLUMN_GROUP): scale / zp [outer, L/gs, inner];
- * mode DYNAMIC or STATIC (FROM_RANGE: BQ_ERR_UNSUPPORTED). One pass over x,
- * no workspace. Otherwise as bq_quantize_per_group. */
+/* Column groups (BQ_GRAN_COLUMN_GROUP): scale / zp [outer, L/gs, inner]. One
+ * pass over x in every mode; ws is read only with FROM_RANGE (the records of
+ * bq_group_range with BQ_GRAN_COLUMN_GROUP) and may be NULL otherwise.
+ * Otherwise as bq_quantize_per_group. */
 bq_status bq_quantize_per_column_group(const void* x, const bq_qdesc* d, int32_t axis,
                                        int64_t group_size, void* q, float* scale, void* zp,
-                                       bq_scale_mode mode, void* stream);
+                                       bq_scale_mode mode, void* ws, size_t ws_bytes,
+                                       void* stream);
 
 /* Dynamic quantize without caller workspace. The sources cited above have no
  * counterpart: this is a library convenience for callers that cannot hand

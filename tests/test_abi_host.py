@@ -84,8 +84,9 @@ def test_workspace_size(B):
     assert B.bq_quantize_workspace_size(d64, "channel", 0) == 16 * 8
     drh = B.make_desc((8, 64), torch.float32, rnd="rhaz")
     assert B.bq_quantize_workspace_size(drh, "channel", 0) == 16 * 8
-    for mode in ("dynamic", "static", "from_range"):           # one pass, no records
+    for mode in ("dynamic", "static"):                          # one pass, no records
         assert B.bq_quantize_workspace_size(d, "column_group", 0, 128, mode) == 0
+    assert B.bq_quantize_workspace_size(d, "column_group", 0, 128, "from_range") == 16 * 64 * 4096
 
 
 def _status(fn):
@@ -133,11 +134,12 @@ def test_argument_errors_return_status_without_launching(B):
     assert B.lib.bq_packed_transpose(P, None, 4, 32, 16, 16, P, P, C.byref(st64), None) == B.BQ_ERR_INVALID_ARG
     # column groups: no range records, group_size must divide the axis
     dc = B.make_desc((64, 48), torch.float32)
-    assert B.lib.bq_quantize_per_column_group(P, C.byref(dc), 0, 16, P, P, P, 2, None) == B.BQ_ERR_UNSUPPORTED
-    assert B.lib.bq_quantize_per_column_group(P, C.byref(dc), 0, 48, P, P, P, 0, None) == B.BQ_ERR_INVALID_ARG
-    assert B.lib.bq_quantize_per_column_group(P, C.byref(dc), 2, 1, P, P, P, 0, None) == B.BQ_ERR_INVALID_ARG
-    assert B.lib.bq_quantize_per_column_group(P + 2, C.byref(dc), 0, 16, P, P, P, 0, None) == B.BQ_ERR_MISALIGNED
-    assert B.lib.bq_group_range(P, C.byref(dc), B.BQ_GRAN_COLUMN_GROUP, 0, 16, P, None) == B.BQ_ERR_UNSUPPORTED
+    # FROM_RANGE without a large enough record buffer
+    assert B.lib.bq_quantize_per_column_group(P, C.byref(dc), 0, 16, P, P, P, 2, P, 16, None) == B.BQ_ERR_INVALID_ARG
+    assert B.lib.bq_quantize_per_column_group(P, C.byref(dc), 0, 48, P, P, P, 0, None, 0, None) == B.BQ_ERR_INVALID_ARG
+    assert B.lib.bq_quantize_per_column_group(P, C.byref(dc), 2, 1, P, P, P, 0, None, 0, None) == B.BQ_ERR_INVALID_ARG
+    assert B.lib.bq_quantize_per_column_group(P + 2, C.byref(dc), 0, 16, P, P, P, 0, None, 0, None) == B.BQ_ERR_MISALIGNED
+    assert B.lib.bq_group_range(P + 2, C.byref(dc), B.BQ_GRAN_COLUMN_GROUP, 0, 16, P, None) == B.BQ_ERR_MISALIGNED
     assert B.lib.bq_dequantize_per_column_group(P, P, None, C.byref(dc), 0, 48, P, B.BQ_F32, None) == B.BQ_ERR_INVALID_ARG
     assert B.lib.bq_quantize_per_column_group_backward(P, P, P, None, C.byref(da), 0, 3, P, None) == B.BQ_ERR_INVALID_ARG
     assert B.lib.bq_dequantize_per_column_group_backward(P, P, C.byref(dc), 0, 5, P, None) == B.BQ_ERR_INVALID_ARG
@@ -167,7 +169,7 @@ def test_empty_calls_succeed_without_a_device(B):
     assert B.lib.bq_quantize_per_token(None, C.byref(d), None, None, None, 0, None, 0, None) == B.BQ_OK
     assert B.lib.bq_dequantize_per_token(None, None, None, C.byref(d), None, B.BQ_F32, None) == B.BQ_OK
     assert B.lib.bq_mxfp8_quantize(None, B.BQ_BF16, 0, 64, None, None, None) == B.BQ_OK
-    assert B.lib.bq_quantize_per_column_group(None, C.byref(d), 0, 1, None, None, None, 0, None) == B.BQ_OK
+    assert B.lib.bq_quantize_per_column_group(None, C.byref(d), 0, 1, None, None, None, 0, None, 0, None) == B.BQ_OK
     assert B.lib.bq_dequantize_per_column_group(None, None, None, C.byref(d), 1, 4, None, B.BQ_F32, None) == B.BQ_OK
 
 

@@ -196,3 +196,37 @@ def test_workload_column_groups_f16(bq, orc):
     dx = bq.quantize_backward(xg, dyg, s, z, "column_group", 0, gs, torch.uint8, False)
     rdx = orc.quantize_backward(xs, dys, rs, rz, "column_group", 0, gs, "u8", False)
     assert_ulp(cpu(dx)[:, cols].contiguous(), rdx, 1, "backward")
+
+
+def _records_as_float(r, dtype):
+    r = cpu(r).reshape(-1, 2)
+    assert bool((r >= 0).all()), "range records must be non-negative bit patterns"
+    if dtype == "f64":
+        return r[:, 0].view(torch.float64), r[:, 1].view(torch.float64)
+    lo32 = (r & 0xFFFFFFFF).to(torch.int32)
+    return lo32[:, 0].view(torch.float32), lo32[:, 1].view(torch.float32)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16", "f32", "f64"])
+def test_column_group_ranges_and_from_range(bq, orc, dtype):
+    # bq_group_range with column groups: one record pair per (block, column),
+    # max(0, max x) and max(0, -min x); FROM_RANGE scaling from those records
+    # gives the dynamic result.
+    for shape, axis, gs in (((256, 96), 0, 128), ((3, 12, 5, 6), 1, 4), ((64, 7), 0, 8)):
+        x = synthetic.Stream(35).tensor(shape, dtype, outlier_p=0.05, outlier_factor=20)
+        x.view(-1)[::7] = 0.0
+        xg = x.cuda()
+        r = bq.group_range(xg, "column_group", axis, gs)
+        hi, nlo = _records_as_float(r, dtype)
+        rhi, rnlo = orc.group_range(x, "column_group", axis, gs)
+        want = torch.float64 if dtype == "f64" else torch.float32
+        assert torch.equal(hi, rhi.to(want).abs()) and torch.equal(nlo, rnlo.to(want).abs())
+        for qd, sym in (("s8", True), ("u8", False)):
+            q, s, z = bq.quantize(xg, "column_group", axis, gs, QD[qd], sym, ranges=r)
+            rq, rs, rz = orc.quantize(x, "column_group", axis, gs, qd, sym)
+            assert_bitwise(q, rq, "FROM_RANGE codes")
+            assert_bitwise(s, rs, "FROM_RANGE scales")
+            if not sym:
+                assert_bitwise(z, rz, "FROM_RANGE zero-points")
+            f, fs, _ = bq.fake_quantize(xg, "column_group", axis, gs, QD[qd], sym, ranges=r)
+            assert_bitwise(f, orc.fake_quantize(x, "column_group", axis, gs, qd, sym)[0], "FROM_RANGE fake")
