@@ -46,9 +46,9 @@ FLUSH_BYTES = 256 << 20
 # the workload above, with the sha256 of the kernel sources it was taken on;
 # reported as null once the sources change.
 NCU_TRAFFIC = {
-    "quantize_per_token": {"src_sha256": "bd915fd8ad68d907e75d4053b483cb53489a1a4e7ae09f7e25dbce49cbe9e8a9", "bytes_per_launch": 70145024},
-    "dequantize_per_token": {"src_sha256": "bd915fd8ad68d907e75d4053b483cb53489a1a4e7ae09f7e25dbce49cbe9e8a9", "bytes_per_launch": 39525632},
-    "quantize_per_token_backward": {"src_sha256": "bd915fd8ad68d907e75d4053b483cb53489a1a4e7ae09f7e25dbce49cbe9e8a9", "bytes_per_launch": 159273216},
+    "quantize_per_token": {"src_sha256": "174acbcfca9b0fd077a568a1ad14d6bef656864cef247f71dade71d450b52b24", "bytes_per_launch": 70312704},
+    "dequantize_per_token": {"src_sha256": "174acbcfca9b0fd077a568a1ad14d6bef656864cef247f71dade71d450b52b24", "bytes_per_launch": 40218368},
+    "quantize_per_token_backward": {"src_sha256": "174acbcfca9b0fd077a568a1ad14d6bef656864cef247f71dade71d450b52b24", "bytes_per_launch": 159534848},
 }
 
 
