@@ -61,6 +61,7 @@ _SIGS = {
     "bq_group_count": [_DESC, C.c_int, _I32, _I64, C.POINTER(_I64), C.POINTER(_I64)],
     "bq_group_range": [_P, _DESC, C.c_int, _I32, _I64, _P, _P],
     "bq_tensor_amax": [_P, C.c_int, _I64, _P, _P, _P],
+    "bq_diag_wait_timeout": [C.c_uint32, _P],
     "bq_quantize_per_tensor": [_P, _DESC, _P, _P, _P, C.c_int, _P, _SZ, _P],
     "bq_quantize_per_channel": [_P, _DESC, _I32, _P, _P, _P, C.c_int, _P, _SZ, _P],
     "bq_quantize_per_token": [_P, _DESC, _P, _P, _P, C.c_int, _P, _SZ, _P],
@@ -212,6 +213,10 @@ def bq_quantize_workspace_size(d: bq_qdesc, gran, axis=0, group_size=1, mode="dy
 def bq_group_range(x, d, gran, axis, group_size, ranges, stream=None):
     _check(lib.bq_group_range(_ptr(x), C.byref(d), _g(gran), axis, group_size, _ptr(ranges),
                               _stream(stream)), "bq_group_range")
+
+
+def bq_diag_wait_timeout(tries, stream=None):
+    _check(lib.bq_diag_wait_timeout(int(tries), _stream(stream)), "bq_diag_wait_timeout")
 
 
 def bq_tensor_amax(x, amax, ws, stream=None):

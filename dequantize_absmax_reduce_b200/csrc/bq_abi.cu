@@ -382,6 +382,11 @@ bq_status bq_tensor_amax(const void* x, bq_dtype dtype, int64_t n, float* amax, 
     return from_cuda(bq::range_to_amax((const unsigned long long*)ws, amax, s));
 }
 
+bq_status bq_diag_wait_timeout(uint32_t tries, void* stream) {
+    if (tries == 0 || tries > (1u << 20)) return BQ_ERR_INVALID_ARG;
+    return from_cuda(bq::wait_diag(tries, S(stream)));
+}
+
 bq_status bq_check_device_error(void) {
     if (cudaDeviceSynchronize() != cudaSuccess) return BQ_ERR_CUDA;
     unsigned int flag = 0;

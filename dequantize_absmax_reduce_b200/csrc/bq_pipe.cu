@@ -16,6 +16,7 @@ cudaError_t pipe_map_bf16(int op, const MapArgs& m, cudaStream_t st);
 cudaError_t pipe_err_f32(unsigned int* flag);
 cudaError_t pipe_err_f16(unsigned int* flag);
 cudaError_t pipe_err_bf16(unsigned int* flag);
+cudaError_t pipe_wait_diag_f32(uint32_t tries, cudaStream_t st);
 cudaError_t pipe_range_f32(const void* x, int64_t n, bool sym, unsigned long long* rec, cudaStream_t st);
 cudaError_t pipe_range_f16(const void* x, int64_t n, bool sym, unsigned long long* rec, cudaStream_t st);
 cudaError_t pipe_range_bf16(const void* x, int64_t n, bool sym, unsigned long long* rec, cudaStream_t st);
@@ -98,6 +99,8 @@ cudaError_t tensor_range_pipe(DT dt, const void* x, int64_t n, bool sym, unsigne
         default: return cudaErrorNotSupported;
     }
 }
+
+cudaError_t wait_diag(uint32_t tries, cudaStream_t st) { return pipe_wait_diag_f32(tries, st); }
 
 cudaError_t tensor_amax_pipe(DT dt, const void* x, int64_t n, unsigned long long* rec, float* amax,
                              cudaStream_t st) {

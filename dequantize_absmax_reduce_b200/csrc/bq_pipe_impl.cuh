@@ -1073,8 +1073,11 @@ __global__ void __launch_bounds__(256) k_fp8_tensor_scalar(Fp8TArgs a) {
 
 // ------------------------------------------------------------ tensor range
 // Range record of a whole tensor (per-tensor scaling, the NVFP4 per-tensor
-// scale). The 16-byte aligned body streams through a ring of RANGE_STAGES
-// bulk copies of RANGE_CHUNK bytes per CTA; each thread folds its vectors into
+// scale). The 16-byte aligned body is cut into units of RANGE_UNIT bytes (one
+// 16-byte vector per thread); CTA b takes the contiguous units
+// [b*U/grid, (b+1)*U/grid), so no CTA streams more than one unit above the
+// mean, and streams them through a ring of RANGE_STAGES bulk copies of up to
+// RANGE_CHUNK bytes; each thread folds its vectors into
 // a packed running range (two 16-bit lanes per instruction). The few
 // elements before the first 16-byte boundary and after the last one go
 // through scalar loads in block 0. One atomicMax per CTA and record slot, made
@@ -1082,6 +1085,7 @@ __global__ void __launch_bounds__(256) k_fp8_tensor_scalar(Fp8TArgs a) {
 // record, and this kernel is launched to overlap it.
 constexpr int RANGE_CHUNK = 16384;
 constexpr int RANGE_STAGES = 4;
+constexpr int RANGE_UNIT = 4096;
 
 struct RangeArgs {
     const void* x;        // first element
@@ -1103,26 +1107,28 @@ __global__ void __launch_bounds__(256) k_range_pipe(RangeArgs a) {
     const int64_t grid = gridDim.x;
     const T* x = (const T*)a.x;
     const uint8_t* body = (const uint8_t*)(x + a.head);
-    const int64_t n_chunks = (a.body_bytes + RANGE_CHUNK - 1) / RANGE_CHUNK;
+    const int64_t n_units = (a.body_bytes + RANGE_UNIT - 1) / RANGE_UNIT;
+    const int64_t b0 = (int64_t)blockIdx.x * n_units / grid * RANGE_UNIT;
+    const int64_t b1 = min(((int64_t)blockIdx.x + 1) * n_units / grid * RANGE_UNIT, a.body_bytes);
+    const int64_t my_bytes = max(b1 - b0, (int64_t)0);
+    const uint8_t* mine = body + b0;
+    const int64_t n_chunks = (my_bytes + RANGE_CHUNK - 1) / RANGE_CHUNK;
     auto chunk_bytes = [&](int64_t c) -> uint32_t {
-        return (uint32_t)min((int64_t)RANGE_CHUNK, a.body_bytes - c * RANGE_CHUNK);
+        return (uint32_t)min((int64_t)RANGE_CHUNK, my_bytes - c * RANGE_CHUNK);
     };
     if (tid == 0) {
         for (int i = 0; i < S; ++i) mbar_init(smem_addr(&bars[i]), 1);
         fence_mbar_init();
-        for (int i = 0; i < S; ++i) {
-            const int64_t c = blockIdx.x + (int64_t)i * grid;
-            if (c >= n_chunks) break;
-            bulk_load(smem_addr(ring + (size_t)i * RANGE_CHUNK), body + c * RANGE_CHUNK,
-                      chunk_bytes(c), smem_addr(&bars[i]));
-        }
+        for (int i = 0; i < S && i < n_chunks; ++i)
+            bulk_load(smem_addr(ring + (size_t)i * RANGE_CHUNK), mine + (int64_t)i * RANGE_CHUNK,
+                      chunk_bytes(i), smem_addr(&bars[i]));
     }
     __syncthreads();
     uint32_t ph = 0u, pl = 0u;
     float hi = 0.0f, nlo = 0.0f;
     int slot = 0;
     uint32_t parity = 0;
-    for (int64_t c = blockIdx.x; c < n_chunks; c += grid) {
+    for (int64_t c = 0; c < n_chunks; ++c) {
         const bool ok = mbar_wait(smem_addr(&bars[slot]), parity);
         if (__syncthreads_or(!ok)) {
             if (tid == 0) {
@@ -1130,7 +1136,7 @@ __global__ void __launch_bounds__(256) k_range_pipe(RangeArgs a) {
                 int s2 = slot;
                 uint32_t p2 = parity;
                 for (int i = 0; i < S; ++i) {
-                    if (c + (int64_t)i * grid >= n_chunks) break;
+                    if (c + i >= n_chunks) break;
                     mbar_wait(smem_addr(&bars[s2]), p2);
                     if (++s2 == S) { s2 = 0; p2 ^= 1u; }
                 }
@@ -1152,10 +1158,10 @@ __global__ void __launch_bounds__(256) k_range_pipe(RangeArgs a) {
         }
         __syncthreads();
         if (tid == 0) {
-            const int64_t next = c + (int64_t)S * grid;
+            const int64_t next = c + S;
             if (next < n_chunks) {
                 fence_proxy_async();
-                bulk_load(smem_addr(ring + (size_t)slot * RANGE_CHUNK), body + next * RANGE_CHUNK,
+                bulk_load(smem_addr(ring + (size_t)slot * RANGE_CHUNK), mine + next * RANGE_CHUNK,
                           chunk_bytes(next), smem_addr(&bars[slot]));
             }
         }
@@ -1777,7 +1783,7 @@ static cudaError_t range_entry(const void* x, int64_t n, bool sym, unsigned long
     if (p % 16 != 0) a.head = min((int64_t)((16 - p % 16) / sizeof(T)), n);
     a.body_bytes = (n - a.head) * (int64_t)sizeof(T) / 16 * 16;
     a.rec = rec;
-    const int64_t n_chunks = (a.body_bytes + RANGE_CHUNK - 1) / RANGE_CHUNK;
+    const int64_t n_units = (a.body_bytes + RANGE_UNIT - 1) / RANGE_UNIT;
     const size_t smem = 128 + (size_t)RANGE_STAGES * RANGE_CHUNK;
     auto k = sym ? k_range_pipe<T, true> : k_range_pipe<T, false>;
     static const cudaError_t attr_s = cudaFuncSetAttribute(
@@ -1790,7 +1796,7 @@ static cudaError_t range_entry(const void* x, int64_t n, bool sym, unsigned long
     const int bps = occupancy_for((const void*)k_range_pipe<T, true>, smem, occ);
     if (bps < 1) return cudaErrorNotSupported;
     int64_t grid = (int64_t)sm_count() * bps;
-    if (grid > n_chunks) grid = n_chunks;
+    if (grid > n_units) grid = n_units;
     if (grid < 1) grid = 1;
     return launch_pdl(k, (unsigned)grid, 256u, smem, st, a);
 }
@@ -2637,6 +2643,21 @@ static cudaError_t col_map_entry(int op, const void* ap, const void* bp, int64_t
     }
 }
 
+// ------------------------------------------------------------ bounded-wait diagnostic
+// One CTA waits on an mbarrier that nothing will ever complete, `tries` times
+// (each try suspends for at most about a microsecond), then records the
+// give-up in g_pipe_error exactly as the pipelined kernels do and returns: the
+// host-visible path of a bounded wait that runs out, with no fault and no hang.
+__global__ void k_wait_diag(uint32_t tries) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(smem_addr(&bar), 1);
+    fence_mbar_init();
+    bool done = false;
+    for (uint32_t i = 0; i < tries && !done; ++i) done = mbar_try_wait(smem_addr(&bar), 0u);
+    if (!done) atomicOr(&g_pipe_error, 1u);
+}
+
 template <class T>
 cudaError_t pipe_error_entry(unsigned int* flag) {
     unsigned int zero = 0;
@@ -2655,6 +2676,10 @@ cudaError_t pipe_error_entry(unsigned int* flag) {
         return pipe_map_entry<T>(op, m, st);                                             \
     }                                                                                    \
     cudaError_t pipe_err_##NAME(unsigned int* flag) { return pipe_error_entry<T>(flag); }       \
+    cudaError_t pipe_wait_diag_##NAME(uint32_t tries, cudaStream_t st) {                         \
+        k_wait_diag<<<1, 32, 0, st>>>(tries);                                                    \
+        return cudaGetLastError();                                                               \
+    }                                                                                            \
     cudaError_t pipe_range_##NAME(const void* x, int64_t n, bool sym, unsigned long long* rec,   \
                                   cudaStream_t st) {                                              \
         return range_entry<T>(x, n, sym, rec, st);                                               \

@@ -184,6 +184,15 @@ bq_status bq_tensor_amax(const void* x, bq_dtype dtype, int64_t n, float* amax, 
  * expected to expire. Host only; the one call here that blocks. */
 bq_status bq_check_device_error(void);
 
+/* Diagnostic of the bounded-wait error path (no counterpart on the pages):
+ * enqueues one small kernel that waits `tries` times (1 <= tries <= 2^20,
+ * each try at most about a microsecond) on an mbarrier nothing completes,
+ * then records the give-up exactly as the pipelined kernels do and returns.
+ * The next bq_check_device_error reports BQ_ERR_TIMEOUT; the context stays
+ * usable. No fault, no unbounded wait. BQ_ERR_INVALID_ARG for tries out of
+ * range. */
+bq_status bq_diag_wait_timeout(uint32_t tries, void* stream);
+
 /* -------------------------------------------------------------- quantize */
 /* [baracuda] quantize_per_tensor / per_channel / per_token / per_group.
  * x: d->shape, dtype d->x_dtype. q: same shape, dtype d->q_dtype.

@@ -163,6 +163,12 @@ def test_argument_errors_return_status_without_launching(B):
     assert B.lib.bq_quantize_per_token(P, C.byref(dneg), P, P, P, 0, None, 0, None) == B.BQ_ERR_INVALID_ARG
 
 
+def test_wait_diagnostic_refuses_out_of_range_tries(B):
+    # Checked before any launch, so it runs without a device.
+    assert B.lib.bq_diag_wait_timeout(0, None) == B.BQ_ERR_INVALID_ARG
+    assert B.lib.bq_diag_wait_timeout((1 << 20) + 1, None) == B.BQ_ERR_INVALID_ARG
+
+
 def test_empty_calls_succeed_without_a_device(B):
     # Nothing to enqueue: an empty tensor returns OK before any CUDA call.
     d = B.make_desc((0, 64), torch.float32)
