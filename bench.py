@@ -228,8 +228,19 @@ def measure_e2e(B, torch, device, x, dy, steps, warmup, chunks=8, nstreams=3):
     return ms, h2d, d2h, ok
 
 
-def per_granularity(B, api, torch, device, peak, reps=5):
-    """Every other workload's kernels, each timed alone with a cold L2."""
+def _trimmed_mean(xs, cut=0.1):
+    xs = sorted(xs)
+    k = int(len(xs) * cut)
+    xs = xs[k:len(xs) - k] if len(xs) > 2 * k else xs
+    return sum(xs) / len(xs)
+
+
+def per_granularity(B, api, torch, device, peak, reps=40):
+    """Every other workload's kernels, each timed alone with a cold L2. The
+    event timer reads in steps of about a microsecond, a large part of one
+    launch of 10-60 us, so each figure is the mean of `reps` launches with the
+    highest and lowest tenth dropped: the tick averages out where a median
+    would keep it."""
     import synthetic
     out = []
     T = Timer(torch, device)
@@ -239,7 +250,7 @@ def per_granularity(B, api, torch, device, peak, reps=5):
         T.collect()
         for _ in range(reps):
             T.run(name, fn)
-        ms = statistics.median(T.collect()[name])
+        ms = _trimmed_mean(T.collect()[name])
         out.append({"workload": workload, "kernel": name, "us": round(ms * 1e3, 2),
                     "GB_s": round(nbytes / (ms * 1e-3) / 1e9, 1),
                     "frac": round(nbytes / (ms * 1e-3) / 1e9 / peak, 3), "bytes": int(nbytes),
