@@ -258,6 +258,18 @@ __device__ __forceinline__ bool range_finish_nan(uint32_t ph, uint32_t pl, float
     }
 }
 
+// The general encoder of one vector (a clamp that can bind, a NaN, a scale
+// outside the fast range), kept out of line: it is the rare path, and
+// inlining it into the unrolled loops only adds instruction-cache pressure
+// to the fast one.
+template <class T, int OP, bool SYM>
+__device__ __noinline__ void emit_int_general(U4 raw, Recip R, IntParams ip, uint8_t* q, int packed, T* y) {
+    float v[Traits<T>::VEC];
+    load_vec<T>(raw, v);
+    if (R.fast) emit_int<T, OP, true, SYM>(v, R, ip, q, packed, y);
+    else emit_int<T, OP, false, SYM>(v, R, ip, q, packed, y);
+}
+
 // ------------------------------------------------------------ the kernel
 // Tuning constants (compile-time): ring depth of the dynamic quantizer for
 // slots of up to 16 KB (NV <= 4) and 32 KB (NV >= 8); team width for groups of
@@ -493,13 +505,8 @@ __global__ void __launch_bounds__(NT) k_seg_pipe(PipeArgs a) {
                 }
             } else if (seg_ok) {
 #pragma unroll
-                for (int j = 0; j < NV; ++j) {
-                    if (!vok(j)) continue;
-                    float v[VEC];
-                    load_vec<T>(raw[j], v);
-                    if (R.fast) emit_int<T, OP, true, SYM>(v, R, ip, code_ptr(a.q, qe + voff(j), pk), pk, yb + voff(j));
-                    else emit_int<T, OP, false, SYM>(v, R, ip, code_ptr(a.q, qe + voff(j), pk), pk, yb + voff(j));
-                }
+                for (int j = 0; j < NV; ++j)
+                    if (vok(j)) emit_int_general<T, OP, SYM>(raw[j], R, ip, code_ptr(a.q, qe + voff(j), pk), pk, yb + voff(j));
             }
         } else {
             constexpr int FMT = (PK == PK_FP8) ? MX_FP8_1x128
