@@ -106,3 +106,10 @@ def test_predequant_fp8_matches_dequantize_then_encode(orc):
     e = orc.nvfp4_predequant_fp8(packed, sc, s2, 8, 64)
     ref = y.clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
     assert torch.equal(e, ref)
+
+
+def test_align_up_is_the_next_multiple(orc):
+    for a in (1, 2, 16, 128):
+        for n in (0, 1, 15, 16, 17, 4095, 4096, 4097):
+            got = orc.align_up(n, a)
+            assert got % a == 0 and n <= got < n + a
