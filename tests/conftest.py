@@ -11,6 +11,21 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running CPU test")
+    _build_library_if_missing()
+
+
+def _build_library_if_missing():
+    """A fresh checkout has no libbq.so (built files are not committed):
+    compile it with the package's own build script before any test imports
+    the package. nvcc cross-compiles for sm_100a without a GPU."""
+    import importlib.util
+    pkg = os.path.join(ROOT, "dequantize_absmax_reduce_b200")
+    if os.path.exists(os.path.join(pkg, "libbq.so")):
+        return
+    spec = importlib.util.spec_from_file_location("_bq_build", os.path.join(pkg, "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
 
 
 @pytest.fixture(scope="session")
