@@ -318,6 +318,24 @@ def fp8_block_dequantize(e, s, rows: int, cols: int, br: int, bc: int, ydtype: s
     return y
 
 
+def fp8_block_gemm(a: torch.Tensor, ew: torch.Tensor, sw: torch.Tensor):
+    """W8A8 block-FP8 matrix multiply (smile.llm.quant Fp8BlockGemm): a [m, k]
+    quantized on the fly to E4M3 with a scale per 1x128 group, times the E4M3
+    weights ew [n, k] with a scale per 128x128 tile (sw [ceil(n/128),
+    ceil(k/128)]). Returns (C f64 [m, n], activation codes u8 [m, k],
+    activation scales f32 [m, ceil(k/128)])."""
+    a = _c(a)
+    m, k = a.shape
+    n = ew.shape[0]
+    assert tuple(ew.shape) == (n, k) and tuple(sw.shape) == ((n + 127) // 128, (k + 127) // 128)
+    c = torch.zeros((m, n), dtype=torch.float64)
+    ea = torch.zeros((m, k), dtype=torch.uint8)
+    sa = torch.zeros((m, (k + 127) // 128), dtype=torch.float32)
+    _ok(lib().or_fp8_block_gemm(_p(a), C.c_int(_dt(a)), _p(_c(ew)), _p(_c(sw)), C.c_int64(m),
+                                C.c_int64(n), C.c_int64(k), _p(c), _p(ea), _p(sa)), "fp8_block_gemm")
+    return c, ea, sa
+
+
 def align_up(n: int, align: int) -> int:
     return int(lib().or_align_up(n, align))
 

@@ -777,6 +777,43 @@ int or_fp8_block_dequantize(const uint8_t* e4m3, const float* scale, int64_t row
     return 0;
 }
 
+// ---- W8A8 block-FP8 matrix multiply [smile.llm.quant Fp8BlockGemm]: the
+// activations a [m, k] are quantized on the fly to E4M3 with one f32 scale
+// per 1x128 group (or_fp8_block_quantize with a 1 x 128 block); the weights
+// are E4M3 [n, k] with one f32 scale per 128x128 tile (sw is
+// [ceil(n/128), ceil(k/128)]); then
+//   C[i, j] = sum over k-blocks b of sa[i, b] * sw[j / 128, b] * S(i, j, b),
+//   S(i, j, b) = sum over the k in block b of dec(ea[i, k]) * dec(ew[j, k]).
+// Every E4M3 value is an integer multiple of 2^-9 below 2^18 such units, so a
+// product of two is a multiple of 2^-18 below 2^36 units and a block's 128
+// products add exactly in binary64; the two scale products and the sum over
+// blocks round in binary64. The pages fix no output precision: C is returned
+// in binary64 (a tensor-core f32 accumulation is compared with it within a
+// bound). ea / sa, when given, receive the activation codes and scales.
+int or_fp8_block_gemm(const void* a, int a_t, const uint8_t* ew, const float* sw, int64_t m,
+                      int64_t n, int64_t k, double* c, uint8_t* ea_out, float* sa_out) {
+    if (a_t != OR_F32 && a_t != OR_F16 && a_t != OR_BF16) return 1;
+    if (m < 0 || n < 0 || k < 0) return 1;
+    const int64_t nkb = (k + 127) / 128;
+    std::vector<uint8_t> ea((size_t)(m * k));
+    std::vector<float> sa((size_t)(m * nkb));
+    if (or_fp8_block_quantize(a, a_t, m, k, 1, 128, ea.data(), sa.data()) != 0) return 1;
+    for (int64_t i = 0; i < m; ++i)
+        for (int64_t j = 0; j < n; ++j) {
+            double acc = 0.0;
+            for (int64_t b = 0; b < nkb; ++b) {
+                double blk = 0.0;
+                for (int64_t kk = b * 128; kk < std::min(k, (b + 1) * 128); ++kk)
+                    blk += dec_e4m3(ea[i * k + kk]) * dec_e4m3(ew[j * k + kk]);
+                acc += (double)sa[i * nkb + b] * (double)sw[(j / 128) * nkb + b] * blk;
+            }
+            c[i * n + j] = acc;
+        }
+    if (ea_out) std::copy(ea.begin(), ea.end(), ea_out);
+    if (sa_out) std::copy(sa.begin(), sa.end(), sa_out);
+    return 0;
+}
+
 // ---- FP8 per-tensor codec [smile.llm.quant Fp8KvCodec: FP8 KV store / load
 // with per-tensor scales]: one f32 scale for the whole tensor, the dequantize
 // multiplier as in the FP8 block formats: s = fl(amax / 448) (0 -> 1, amax
