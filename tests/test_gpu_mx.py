@@ -118,6 +118,26 @@ def test_tensor_amax_offsets_and_sizes(bq, orc, dtype):
     assert cpu(bq.tensor_amax(inf.cuda())).item() == float("inf")
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_tensor_amax_finds_a_lone_maximum_anywhere(bq, dtype):
+    # More 4 KB units than CTAs, split unevenly into contiguous runs: a single
+    # element of magnitude 4096 (the rest N(0,1)) must be found wherever it
+    # sits: on either side of unit boundaries, in the ragged last unit, in
+    # the unaligned tail, at random places.
+    n = (4096 * 1339 + 48) // (2 if dtype == "bf16" else 4) + 3
+    x = synthetic.Stream(31).tensor((n,), dtype).cuda()
+    per_unit = 4096 // x.element_size()
+    rng = np.random.default_rng(2)
+    pos = [0, 1, n - 1, n - 2, n - 4, per_unit - 1, per_unit, 700 * per_unit - 1, 700 * per_unit,
+           1338 * per_unit, 1338 * per_unit + 5] + [int(p) for p in rng.integers(0, n, 12)]
+    for i, p in enumerate(pos):
+        v = 4096.0 if i % 2 == 0 else -4096.0
+        old = x[p].item()
+        x[p] = v
+        assert cpu(bq.tensor_amax(x)).item() == 4096.0, (p, v)
+        x[p] = old
+
+
 def test_nvfp4_special_values(bq, orc):
     vals = [0.0, -0.0, 1e-30, -1e-30, 6.0, -6.0, 5.0, 2.5, 0.25, 0.75, 1e30, -1e30,
             float("inf"), float("-inf"), float("nan"), -float("nan")]
