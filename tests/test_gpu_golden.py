@@ -42,3 +42,15 @@ def test_mxfp8_worked_block(bq, dtype):
     e, s = bq.mxfp8_quantize(x)
     assert s.cpu().tolist() == [[int(g["scale_byte"][0])]]
     assert e[0].cpu().tolist() == [int(v) for v in g["codes"]]
+
+
+@pytest.mark.parametrize("name", ["nvfp4_block.txt", "nvfp4_block_scaled.txt"])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_nvfp4_worked_block(bq, name, dtype):
+    g = load(name)
+    x = torch.tensor([g["x"]], dtype=dtype, device="cuda")
+    p, sc, s2 = bq.nvfp4_quantize(x, s2=g["s2"][0])
+    assert sc.cpu().tolist() == [[int(g["scale_byte"][0])]]
+    assert p[0].cpu().tolist() == [int(v) for v in g["packed"]]
+    y = bq.nvfp4_dequantize(p, sc, s2, torch.float32)
+    assert y[0].cpu().tolist() == g["dequantized"]

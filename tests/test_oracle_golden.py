@@ -2,6 +2,7 @@
 names the passage it follows and shows its arithmetic)."""
 
 import numpy as np
+import pytest
 import torch
 
 from golden_fixtures import load
@@ -36,3 +37,15 @@ def test_mxfp8_worked_block(orc):
     # and back: every element here is exact in E4M3 * 2^3
     y = orc.mxfp8_dequantize(e, s, 1, 32, "f32")
     assert np.array_equal(y.numpy()[0], np.array(g["x"], dtype=np.float32))
+
+
+@pytest.mark.parametrize("name", ["nvfp4_block.txt", "nvfp4_block_scaled.txt"])
+def test_nvfp4_worked_block(orc, name):
+    g = load(name)
+    x = torch.tensor([g["x"]], dtype=torch.bfloat16)            # every value exact in bf16
+    p, sc, s2 = orc.nvfp4_quantize(x, s2=g["s2"][0])
+    assert s2 == g["s2"][0]
+    assert sc.tolist() == [[int(g["scale_byte"][0])]]
+    assert p[0].tolist() == [int(v) for v in g["packed"]]
+    y = orc.nvfp4_dequantize(p, sc, s2, 1, 16, "f32")
+    assert y[0].tolist() == g["dequantized"]
