@@ -42,7 +42,7 @@ def lib() -> C.CDLL:
     if _lib is None:
         path = _build.build()
         _lib = C.CDLL(path)
-        for name in ("or_encode", "or_decode", "or_round_int", "or_default_q_range",
+        for name in ("or_encode", "or_encode_f32_bits", "or_decode", "or_round_int", "or_default_q_range",
                      "or_group_count", "or_group_range", "or_quantize", "or_dequantize",
                      "or_fake_quantize", "or_ste_backward", "or_dequantize_backward",
                      "or_tensor_amax", "or_nvfp4_quantize", "or_nvfp4_dequantize",
@@ -90,6 +90,20 @@ def encode(fmt: str, values) -> np.ndarray:
     out = np.zeros(v.shape, dtype=np.uint16 if fmt in ("f16", "bf16") else np.uint8)
     _ok(lib().or_encode(_FMT[fmt], v.ctypes.data_as(C.c_void_p), C.c_int64(v.size),
                         out.ctypes.data_as(C.c_void_p)), "encode")
+    return out
+
+
+def encode_f32_bits(fmt: str, first: int, count: int, out: np.ndarray | None = None) -> np.ndarray:
+    """Encode the f32 values whose bit patterns are first, first+1, ...,
+    first+count-1 (one code per element; e2m1 one code per byte). Writes into
+    `out` when given (a contiguous array of the code type); the C loop runs
+    without the GIL, so threads may fill disjoint slices at once."""
+    dt = np.uint16 if fmt in ("f16", "bf16") else np.uint8
+    if out is None:
+        out = np.empty(count, dtype=dt)
+    assert out.dtype == dt and out.flags.c_contiguous and out.size == count
+    _ok(lib().or_encode_f32_bits(C.c_int(_FMT[fmt]), C.c_uint32(first), C.c_int64(count),
+                                 out.ctypes.data_as(C.c_void_p)), "encode_f32_bits")
     return out
 
 

@@ -47,8 +47,10 @@
 //   * dequantize y = RN_y(fl((q-zp)*s)); f64 outputs keep the exact product.
 //   * E4M3 encode is round-to-nearest-even with saturation to +-448, NaN ->
 //     0x7F; E2M1 encode is round-to-nearest-even with saturation to +-6 and
-//     the sign bit kept, NaN -> 0x7 (+6, the largest positive code); E2M1
-//     element 2j goes to the low nibble of byte j.
+//     the sign bit kept, NaN -> 0x0 (+0: E2M1 has no NaN, and IEEE 754-2019
+//     6.3 gives a NaN's sign bit no meaning, so the code carries no sign,
+//     as E4M3's single NaN code carries none); E2M1 element 2j goes to the
+//     low nibble of byte j.
 //   * NVFP4: s2 = fl(A/2688) (2688 = 448*6), sb = E4M3(fl(a_b/fl(6*s2))),
 //     eff = fl(dec(sb)*s2), code = E2M1(fl(x/eff)), all-zero codes when
 //     eff == 0.
@@ -159,8 +161,8 @@ uint16_t enc_f16(double v)  { return (uint16_t)mini_encode(fmt_f16(), v, false, 
 uint16_t enc_bf16(double v) { return (uint16_t)mini_encode(fmt_bf16(), v, false, 0x7FC0u); }
 uint8_t  enc_e4m3(double v) { return (uint8_t)mini_encode(fmt_e4m3(), v, true, 0x7Fu); }
 uint8_t  enc_e2m1(double v) {
-    // No NaN in E2M1: a NaN saturates to the largest positive code (+6).
-    return (uint8_t)mini_encode(fmt_e2m1(), v, true, 0x7u);
+    // No NaN in E2M1: a NaN of either sign becomes +0 (code 0x0).
+    return (uint8_t)mini_encode(fmt_e2m1(), v, true, 0x0u);
 }
 double dec_f16(uint16_t c)  { return mini_decode_fields(fmt_f16(), c); }
 double dec_bf16(uint16_t c) { return mini_decode_fields(fmt_bf16(), c); }
@@ -403,6 +405,24 @@ int or_encode(int fmt, const double* v, int64_t n, void* out) {
             case 2: ((uint8_t*)out)[i] = enc_e4m3(v[i]); break;
             case 3: ((uint8_t*)out)[i] = enc_e2m1(v[i]); break;
             default: return 1;
+        }
+    }
+    return 0;
+}
+// The same encoders over a run of f32 bit patterns: value i is the f32 whose
+// bits are first + i (count <= 2^32 - first), so a caller can sweep every f32.
+int or_encode_f32_bits(int fmt, uint32_t first, int64_t count, void* out) {
+    if (fmt < 0 || fmt > 3 || count < 0 || (uint64_t)first + (uint64_t)count > (1ull << 32)) return 1;
+    for (int64_t i = 0; i < count; ++i) {
+        const uint32_t bits = first + (uint32_t)i;
+        float f;
+        std::memcpy(&f, &bits, 4);
+        const double v = f;
+        switch (fmt) {
+            case 0: ((uint16_t*)out)[i] = enc_f16(v); break;
+            case 1: ((uint16_t*)out)[i] = enc_bf16(v); break;
+            case 2: ((uint8_t*)out)[i] = enc_e4m3(v); break;
+            default: ((uint8_t*)out)[i] = enc_e2m1(v); break;
         }
     }
     return 0;

@@ -33,9 +33,22 @@ def test_e2m1_encode_ties_and_saturation(orc):
     neg = orc.encode("e2m1", [-v for v in cases])
     assert list(neg) == [c | 8 for c in cases.values()]
     assert list(orc.encode("e2m1", [-0.0, -1e-9])) == [8, 8]
-    # Reading: E2M1 has no NaN; a NaN saturates to +6 whatever its sign.
-    assert orc.encode("e2m1", [float("nan")])[0] == 7
-    assert orc.encode("e2m1", [-float("nan")])[0] == 7
+
+
+def test_e2m1_nan_encodes_as_positive_zero(orc):
+    # Reading: the OCP E2M1 element has no NaN (all 16 codes are finite, table
+    # above), and IEEE 754-2019 section 6.3 gives no meaning to the sign bit of
+    # a NaN, so every NaN, whatever its sign and payload, encodes as the code
+    # of +0: the code whose OCP magnitude is 0 and whose sign bit (bit 3) is
+    # clear. Checked on quiet and signalling NaNs of both signs.
+    ocp = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    bits = np.array([0x7FF8000000000000, 0xFFF8000000000000, 0x7FF0000000000001,
+                     0xFFF0000000000001, 0x7FFFFFFFFFFFFFFF, 0xFFF4000000000000], dtype=np.uint64)
+    nans = bits.view(np.float64)
+    assert np.isnan(nans).all()
+    codes = orc.encode("e2m1", nans)
+    for c in codes:
+        assert (int(c) & 8) == 0 and ocp[int(c) & 7] == 0.0
 
 
 def test_e4m3_decode_all_codes_vs_torch(orc):

@@ -176,12 +176,13 @@ def test_packed_transpose_vs_numpy(orc, n, k, gs, align):
 # ---------------------------------------------------------------- MXFP4
 def _e2m1_nearest_even(t: np.ndarray) -> np.ndarray:
     """Brute-force E2M1 code of f64 values t: nearest grid value, ties to the
-    even mantissa, saturating to +-6, sign kept (NaN -> 0x7)."""
+    even mantissa, saturating to +-6, sign kept (NaN -> 0x0: E2M1 has no
+    NaN, and a NaN's sign bit means nothing)."""
     mags = E2M1                                   # codes 0..7; odd code = odd mantissa
     out = np.zeros(t.shape, dtype=np.uint8)
     for i, v in np.ndenumerate(t):
         if np.isnan(v):
-            out[i] = 0x7
+            out[i] = 0x0
             continue
         a = min(abs(v), 6.0)
         d = np.abs(mags - a)
