@@ -62,6 +62,7 @@ _SIGS = {
     "bq_group_range": [_P, _DESC, C.c_int, _I32, _I64, _P, _P],
     "bq_tensor_amax": [_P, C.c_int, _I64, _P, _P, _P],
     "bq_diag_wait_timeout": [C.c_uint32, _P],
+    "bq_diag_encode_f32": [_P, _I64, C.c_int, _P, _P],
     "bq_quantize_per_tensor": [_P, _DESC, _P, _P, _P, C.c_int, _P, _SZ, _P],
     "bq_quantize_per_channel": [_P, _DESC, _I32, _P, _P, _P, C.c_int, _P, _SZ, _P],
     "bq_quantize_per_token": [_P, _DESC, _P, _P, _P, C.c_int, _P, _SZ, _P],
@@ -217,6 +218,13 @@ def bq_group_range(x, d, gran, axis, group_size, ranges, stream=None):
 
 def bq_diag_wait_timeout(tries, stream=None):
     _check(lib.bq_diag_wait_timeout(int(tries), _stream(stream)), "bq_diag_wait_timeout")
+
+
+def bq_diag_encode_f32(x, fmt, out, stream=None):
+    """x: f32 device tensor; fmt: BQ_E4M3, BQ_E2M1X2, BQ_BF16 or BQ_F16 (the
+    enum values); out: device buffer of n, n/2 or 2n bytes."""
+    _check(lib.bq_diag_encode_f32(_ptr(x), x.numel(), int(fmt), _ptr(out), _stream(stream)),
+           "bq_diag_encode_f32")
 
 
 def bq_tensor_amax(x, amax, ws, stream=None):

@@ -472,8 +472,9 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
     return e4m3x2(a, b) | (e4m3x2(c, d) << 16);
 }
 // E2M1 (OCP FP4), round to nearest even, saturating to +-6: eight values
-// into one word, value i in nibble i (low nibble first).
-__device__ __forceinline__ uint32_t e2m1x8(const float (&v)[8]) {
+// into one word, value i in nibble i (low nibble first). For NaN-free
+// inputs only: the conversion instruction gives a NaN the code of +6.
+__device__ __forceinline__ uint32_t e2m1x8_finite(const float (&v)[8]) {
     uint32_t r;
     asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
         "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
@@ -484,6 +485,14 @@ __device__ __forceinline__ uint32_t e2m1x8(const float (&v)[8]) {
         : "=r"(r)
         : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
     return r;
+}
+// E2M1 of any f32: E2M1 has no NaN, so a NaN of either sign encodes as +0
+// (code 0); every other value as e2m1x8_finite.
+__device__ __forceinline__ uint32_t e2m1x8(const float (&v)[8]) {
+    float t[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) t[i] = isnan(v[i]) ? 0.0f : v[i];
+    return e2m1x8_finite(t);
 }
 // Decode two E4M3 bytes (low byte first) to f32 exactly (via f16, which
 // holds every E4M3 value).

@@ -542,14 +542,25 @@ __global__ void __launch_bounds__(NT) k_seg_pipe(PipeArgs a) {
             } else if constexpr (PK == PK_MX4) {
                 const int E = mx_exponent(hi, 2);
                 if (seg_ok && lane == 0) a.zp[seg] = (uint8_t)(E + 127);
-                const F2 mul2 = f2_bcast(exp2i(-E));
-                if (full) {
+                const float mul = exp2i(-E);
+                const F2 mul2 = f2_bcast(mul);
+                if (full && !warp_nan) {
 #pragma unroll
                     for (int j = 0; j < NV; ++j) emit_mx4_fast<T>(raw[j], mul2, base + coff(j));
-                } else if (seg_ok) {
+                } else if (seg_ok && !warp_nan) {
 #pragma unroll
                     for (int j = 0; j < NV; ++j)
                         if (vok(j)) emit_mx4_fast<T>(raw[j], mul2, base + coff(j));
+                } else if (seg_ok) {
+                    // A NaN in the warp's groups: the general encoder (NaN -> code 0).
+                    const Recip R{};
+#pragma unroll
+                    for (int j = 0; j < NV; ++j) {
+                        if (!vok(j)) continue;
+                        float v[VEC];
+                        load_vec<T>(raw[j], v);
+                        mx_emit<T, FMT, true>(v, R, mul, false, base + coff(j));
+                    }
                 }
             } else if constexpr (PK == PK_MX) {
                 const int E = mx_exponent(hi);
@@ -629,7 +640,7 @@ __device__ __forceinline__ uint32_t nv_word_fast(const U4& raw, const Recip2& R2
         t[2 * p] = __uint_as_float((q0 & 0x7FFFFFFFu) | (x0 & 0x80000000u));
         t[2 * p + 1] = __uint_as_float((q1 & 0x7FFFFFFFu) | (x1 & 0x80000000u));
     }
-    return e2m1x8(t);
+    return e2m1x8_finite(t);
 }
 // General path: IEEE division where the chain cannot be used; all-zero codes
 // when eff == 0.

@@ -200,7 +200,8 @@ __device__ __forceinline__ void emit_fp8_fast(const U4& raw, const Recip2& R2, u
     }
 }
 
-// E2M1 codes of fl(x / s), the sign of each quotient taken from x.
+// E2M1 codes of fl(x / s), the sign of each quotient taken from x (no NaN
+// among the values: the caller's guarantee above).
 template <class T>
 __device__ __forceinline__ void emit_nv_fast(const U4& raw, const Recip2& R2, uint8_t* dst) {
     constexpr int VEC = Traits<T>::VEC;
@@ -217,10 +218,10 @@ __device__ __forceinline__ void emit_nv_fast(const U4& raw, const Recip2& R2, ui
         t[2 * p + 1] = __uint_as_float((q1 & 0x7FFFFFFFu) | (x1 & 0x80000000u));
     }
     if constexpr (VEC == 8) {
-        st4(dst, e2m1x8(t));
+        st4(dst, e2m1x8_finite(t));
     } else {
         t[4] = t[5] = t[6] = t[7] = 0.0f;
-        st2(dst, e2m1x8(t) & 0xFFFFu);
+        st2(dst, e2m1x8_finite(t) & 0xFFFFu);
     }
 }
 
@@ -243,7 +244,8 @@ __device__ __forceinline__ void emit_mx_fast(const U4& raw, F2 mul2, uint8_t* ds
 }
 
 // MXFP4 codes E2M1(fl(x * 2^-E)): a product (exact, sign kept for zeros and
-// underflows), so like MXFP8 it needs no guard.
+// underflows). The caller guarantees no NaN among the values (a NaN takes
+// the general encoder, which gives it code 0).
 template <class T>
 __device__ __forceinline__ void emit_mx4_fast(const U4& raw, F2 mul2, uint8_t* dst) {
     constexpr int VEC = Traits<T>::VEC;
@@ -254,10 +256,10 @@ __device__ __forceinline__ void emit_mx4_fast(const U4& raw, F2 mul2, uint8_t* d
 #pragma unroll
     for (int p = 0; p < NP; ++p) f2_split(f2_mul(x[p], mul2), t[2 * p], t[2 * p + 1]);
     if constexpr (VEC == 8) {
-        st4(dst, e2m1x8(t));
+        st4(dst, e2m1x8_finite(t));
     } else {
         t[4] = t[5] = t[6] = t[7] = 0.0f;
-        st2(dst, e2m1x8(t) & 0xFFFFu);
+        st2(dst, e2m1x8_finite(t) & 0xFFFFu);
     }
 }
 
