@@ -24,8 +24,11 @@
  *   - Pointers named x, q, y, dy, dx, dq, scale, zp, ranges, ws, packed,
  *     e4m3, e8m0, w, sc, w_t, sc_t are DEVICE pointers owned by the caller.
  *     Tensors are dense and row-major (C order). The library allocates
- *     nothing, keeps no state between calls and may be called from several
- *     host threads at once.
+ *     nothing and may be called from several host threads at once. The
+ *     only device state it keeps between calls is one flag per device that
+ *     records a bounded wait that gave up (shared by every stream on that
+ *     device: see bq_check_device_error) and the range-record array of
+ *     bq_quantize_dynamic_noalloc.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream). Every call only enqueues work on that stream and returns; it
  *     never synchronises the host.
@@ -181,7 +184,9 @@ bq_status bq_tensor_amax(const void* x, bq_dtype dtype, int64_t n, float* amax, 
 /* Synchronises the current device, then reports whether a pipelined kernel
  * gave up waiting for one of its bulk copies since the last call
  * (BQ_ERR_TIMEOUT; the flag is cleared) — a bounded wait that is never
- * expected to expire. Host only; the one call here that blocks. */
+ * expected to expire. The flag is per device, not per stream: a give-up on
+ * any stream of the device is reported to whichever caller checks next.
+ * Host only; the one call here that blocks. */
 bq_status bq_check_device_error(void);
 
 /* Diagnostic of the bounded-wait error path (no counterpart on the pages):
@@ -192,6 +197,24 @@ bq_status bq_check_device_error(void);
  * usable. No fault, no unbounded wait. BQ_ERR_INVALID_ARG for tries out of
  * range. */
 bq_status bq_diag_wait_timeout(uint32_t tries, void* stream);
+
+/* Diagnostic of the element encoders (no counterpart on the pages): encodes
+ * n f32 values x (device) into `out` (device) with the very
+ * device functions the quantize kernels use for that format:
+ *   BQ_E4M3   one byte per value: round to nearest even, saturating to
+ *             +-448, NaN -> 0x7F (the OCP FP8 E4M3 element of
+ *             [smile.llm.quant] Fp8BlockGemm / MxFp8 and [QuantizedWeight]);
+ *   BQ_E2M1X2 two values per byte, value 2j in the low nibble of byte j
+ *             (n even): round to nearest even, saturating to +-6, sign kept,
+ *             NaN -> 0x0 ([QuantizedWeight] NVFP4 element);
+ *   BQ_BF16 / BQ_F16  two bytes per value: round to nearest even (the
+ *             narrowing of every bf16 / f16 output).
+ * One launch; out must hold n (E4M3), n/2 (E2M1X2) or 2n (BF16, F16) bytes.
+ * x must be 16-byte aligned and out aligned to 8 (E4M3), 4 (E2M1X2) or 16
+ * (BF16, F16) bytes (BQ_ERR_MISALIGNED otherwise). BQ_ERR_UNSUPPORTED for
+ * another format, BQ_ERR_INVALID_ARG for n < 0, an odd n with E2M1X2 or a
+ * NULL pointer with n > 0. */
+bq_status bq_diag_encode_f32(const float* x, int64_t n, bq_dtype fmt, void* out, void* stream);
 
 /* -------------------------------------------------------------- quantize */
 /* [baracuda] quantize_per_tensor / per_channel / per_token / per_group.
@@ -237,10 +260,18 @@ bq_status bq_quantize_per_column_group(const void* x, const bq_qdesc* d, int32_t
  *   - BQ_ERR_INVALID_ARG, with nothing enqueued, when the call needs more
  *     than BQ_NOALLOC_MAX_GROUPS records
  *     (bq_quantize_workspace_size(d, gran, axis, group_size, DYNAMIC) >
- *     16 * BQ_NOALLOC_MAX_GROUPS); other errors as the workspace entries.
- *   - The first call on each device resolves the array's address there
- *     (cudaGetSymbolAddress on the current device, done once and cached);
- *     make that first call before any stream capture starts.
+ *     16 * BQ_NOALLOC_MAX_GROUPS), and when it has more groups than that
+ *     and x or q is not 16-byte aligned (the single-pass kernels, which
+ *     need no records, take only aligned tensors); other errors as the
+ *     workspace entries.
+ *   - The array exists once per CUDA context, i.e. once per device for
+ *     runtime-API callers (the device's primary context). The first call
+ *     made in a context resolves the array's address there
+ *     (cudaGetSymbolAddress with that context current) and caches it under
+ *     the context's ID, so a context created later on the same device
+ *     (after cudaDeviceReset, or a driver-API caller's own context) gets
+ *     its own address; make each context's first call before any stream
+ *     capture starts.
  *   - The array is shared: calls whose work may overlap on one device (on
  *     different streams without ordering between them, or from several host
  *     threads) race on it and may write wrong scales. Calls on one stream,
@@ -339,7 +370,7 @@ bq_status bq_dequantize_per_column_group_backward(const void* dy, const float* s
  * scale_e4m3: u8 [n, k/16]. global_scale: one f32 (device), written unless
  * static_global == 1. ws: 16 bytes (static_global 0 and 2). E4M3 encodes round to nearest even,
  * saturate to +-448, NaN -> 0x7F; E2M1 encodes saturate to +-6 and keep the
- * sign; a NaN element encodes as 0x7 (+6). */
+ * sign; a NaN element of either sign encodes as 0x0 (+0: E2M1 has no NaN). */
 bq_status bq_nvfp4_quantize(const void* x, bq_dtype x_dtype, int64_t n, int64_t k,
                             uint8_t* packed, uint8_t* scale_e4m3, float* global_scale,
                             int32_t static_global, void* ws, size_t ws_bytes, void* stream);
@@ -370,7 +401,7 @@ bq_status bq_mxfp8_dequantize(const uint8_t* e4m3, const uint8_t* e8m0, int64_t 
  * E = clamp(floor(log2 amax) - 2, -127, 127) (2 = the largest E2M1 exponent;
  * amax ignores NaN, an infinite amax counts as 2^128, amax = 0 gives -127),
  * byte = E + 127, code = E2M1(fl(x * 2^-E)) rounded to nearest even,
- * saturating to +-6, sign kept, NaN -> 0x7. */
+ * saturating to +-6, sign kept, NaN -> 0x0. */
 bq_status bq_mxfp4_quantize(const void* x, bq_dtype x_dtype, int64_t rows, int64_t k,
                             uint8_t* packed, uint8_t* e8m0, void* stream);
 

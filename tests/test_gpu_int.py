@@ -174,6 +174,43 @@ def test_all_16bit_patterns(bq, orc):
                 assert_ulp(dx, rdx, 1, f"{dtype} ste {s}")
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f16", "f32"])
+def test_ste_backward_every_dy_at_limit_scales(bq, orc, dtype):
+    """The STE gradient is dy * RN(1/s) on the GPU and fl(dy / s) in the oracle
+    (both narrowed to dy's dtype): within one step of the output dtype for
+    every dy. Every 16-bit pattern serves as dy (subnormals, infinities and
+    NaN included; for f32, the widened 16-bit values plus random f32 words),
+    against x holding every pattern in another order, at scales at and
+    around the ends of the range where the reciprocal is used (2^-64 and
+    2^64), just outside it (IEEE division), near the f32 subnormal range and
+    at ordinary values."""
+    if dtype == "f32":
+        base = synthetic.bits_tensor("bf16").float()
+        rnd = torch.from_numpy(np.random.default_rng(5).integers(0, 2**32, 65536, dtype=np.uint64)
+                               .astype(np.uint32).view(np.int32)).view(torch.float32)
+        dy = torch.cat([base, rnd]).reshape(32, 4096)
+        x = torch.cat([base.flip(0), base.roll(12345)]).reshape(32, 4096)
+    else:
+        dy = synthetic.bits_tensor(dtype).reshape(16, 4096)
+        perm = torch.from_numpy(np.random.default_rng(3).permutation(65536))
+        x = synthetic.bits_tensor(dtype)[perm].reshape(16, 4096)
+    for s in (2.0 ** -64, 1.37 * 2.0 ** -64, 2.0 ** 64, 1.9 * 2.0 ** 63, 0.99 * 2.0 ** -64,
+              1.01 * 2.0 ** 64, 2.0 ** -126, 1.2e-40, 3.0, 0.0173):
+        for qd, sym in (("s8", True), ("u8", False)):
+            sc = torch.full((x.shape[0],), s, dtype=torch.float32)
+            zp = None if sym else torch.full((x.shape[0],), 131, dtype=torch.uint8)
+            dx = bq.quantize_backward(x.cuda(), dy.cuda(), sc.cuda(), None if zp is None else zp.cuda(),
+                                      "token", qdtype=QD[qd], symmetric=sym)
+            rdx = orc.quantize_backward(x, dy, sc, zp, "token", qdtype=qd, symmetric=sym)
+            assert_ulp(dx, rdx, 1, f"{dtype} ste s={s!r} {qd}")
+            st = sc[:1]
+            dx = bq.quantize_backward(x.cuda(), dy.cuda(), st.cuda(), None if zp is None else zp[:1].cuda(),
+                                      "tensor", qdtype=QD[qd], symmetric=sym)
+            rdx = orc.quantize_backward(x, dy, st, None if zp is None else zp[:1], "tensor",
+                                        qdtype=qd, symmetric=sym)
+            assert_ulp(dx, rdx, 1, f"{dtype} ste per-tensor s={s!r} {qd}")
+
+
 def test_special_values_f32(bq, orc):
     vals = [0.0, -0.0, 1e-45, -1e-45, 1.17e-38, 3.4e38, -3.4e38, float("inf"), float("-inf"),
             float("nan"), 1.0, -1.0, 0.5, -0.5, 127.5, -128.5]

@@ -5,6 +5,9 @@ included. About 40 GB of device memory at a time; inputs are seeded normal
 draws made on the device, and the oracle gets host copies of exactly the rows
 it checks."""
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import pytest
 import torch
 
@@ -62,12 +65,18 @@ def test_per_tensor_and_fp8_blocks_past_2_32(bq, orc):
     x = _draw(R, K, torch.bfloat16, 13)
     rows = _rows(R)
     xs = cpu(x[rows.cuda()])
-    # Per-tensor: two passes over 4.3e9 elements; the scale is amax / 127 with
-    # the amax taken by torch here, the codes of the sampled rows by the oracle.
+    # Per-tensor: two passes over 4.3e9 elements. The oracle takes the tensor
+    # amax chunk by chunk on the host cores (the max of the chunks' maxima),
+    # derives the scale from that range (fl(amax / 127)) and gives the codes
+    # of the sampled rows with it.
     q, s, _ = bq.quantize(x, "tensor")
-    amax = float(x.abs().max().float())
-    rq, rs, _ = orc.quantize(xs, "tensor", scale=torch.tensor([amax]) / 127.0)
-    assert s.item() == torch.tensor(amax / 127.0, dtype=torch.float32).item()
+    flat = x.reshape(-1)
+    with ThreadPoolExecutor(max_workers=max(1, os.cpu_count() or 1)) as pool:
+        futs = [pool.submit(orc.tensor_amax, cpu(c)) for c in flat.split(1 << 27)]
+        amax = max(f.result() for f in futs)
+    r = torch.tensor([amax], dtype=torch.float64)
+    rq, rs, _ = orc.quantize(xs, "tensor", ranges=(r, r))
+    assert_bitwise(s, rs, "per-tensor scale")
     assert_bitwise(cpu(q[rows.cuda()]), rq, "per-tensor codes")
     del q
     # FP8 1x128: codes and scales of the sampled rows.

@@ -259,14 +259,20 @@ def test_workload_fp8_blocks(bq, orc, name):
     assert_bitwise(cpu(ms)[rows], rms, "mxfp8 e8m0")
     y = bq.fp8_block_dequantize(e, s, 1, 128, torch.bfloat16)
     assert_bitwise(cpu(y)[rows], orc.fp8_block_dequantize(re, rs, len(rows), 7168, 1, 128, "bf16"), "deq")
-    del act, e, s, me, ms, y
+    del y
+    my = bq.mxfp8_dequantize(me, ms, torch.bfloat16)
+    assert_bitwise(cpu(my)[rows], orc.mxfp8_dequantize(rme, rms, len(rows), 7168, "bf16"), "mxfp8 deq")
+    del act, e, s, me, ms, my
     wt = synthetic.make_workload_device(name, only=["w"])["w"]
     e, s = bq.fp8_block_quantize(wt, 128)
+    wy = bq.fp8_block_dequantize(e, s, 128, 128, torch.bfloat16)
     for band in (0, 27, 55):
         r0 = band * 128
         re, rs = orc.fp8_block_quantize(cpu(wt[r0:r0 + 128]), 128, 128)
         assert_bitwise(cpu(e)[r0:r0 + 128], re, f"w e4m3 band {band}")
         assert_bitwise(cpu(s)[band], rs[0], f"w scales band {band}")
+        ry = orc.fp8_block_dequantize(re, rs, 128, 18432, 128, 128, "bf16")
+        assert_bitwise(cpu(wy[r0:r0 + 128]), ry, f"w 128x128 deq band {band}")
 
 
 # ---------------------------------------------------------------- MXFP4
