@@ -35,7 +35,11 @@ def _reference_call(B, x, gran, axis, gs, qd, sym):
     q = torch.empty(x.shape, dtype=qd, device=x.device)
     scale = torch.empty(max(n_groups, 1), dtype=torch.float32, device=x.device)
     zp = torch.empty(max(n_groups, 1), dtype=qd, device=x.device)
+    # The size query judges from the shape; a misaligned x falls back to two
+    # passes, which need one record per group.
     nbytes = B.bq_quantize_workspace_size(d, gran, axis, gs, "dynamic")
+    if x.data_ptr() % 16:
+        nbytes = max(nbytes, 16 * n_groups)
     ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=x.device)
     if gran == "tensor":
         B.bq_quantize_per_tensor(x, d, q, scale, zp, "dynamic", ws)
