@@ -405,7 +405,52 @@ def per_granularity(B, api, torch, device, peak, reps=40):
           3 * n + 4 * s.numel(), 1)
     timed(wl, "fp8_block_dequantize(128x128 weight)",
           lambda: B.bq_fp8_block_dequantize(e, s, 128, 128, y), 3 * n + 4 * s.numel(), 1)
+    del e, s, y
+    out.append(gemm_bench(B, torch, device, wt, T))
     return out
+
+
+def _fp8_peak_tflops():
+    """Dense FP8 tensor peak: twice the measured bf16 GEMM rate (burst), the
+    nominal FP8 : BF16 ratio of the B200 (4.5 : 2.25 PFLOP/s)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return 2.0 * float(json.load(f)["bf16_tflops"]), "derived: 2 x measured bf16 burst"
+    return 2.0 * 1590.0, "derived: 2 x fallback bf16"
+
+
+def gemm_bench(B, torch, device, wt, T, reps=10):
+    """Block-FP8 GEMM with the fused activation quantization on the FP8
+    workload: activations bf16 [16384, 7168] quantized on the fly (1x128),
+    the workload's weight read as W[n, k] = w[k, n] (the [7168, 18432] tensor
+    transposed, then quantized in 128x128 tiles outside the timed region),
+    C bf16 [16384, 18432]. TFLOP/s = 2 m n k / time."""
+    import synthetic
+    a = synthetic.make_workload_device("fp8_blocks_bf16", device=device, only=["act"])["act"]
+    m, k = a.shape
+    w_nk = wt.t().contiguous()
+    n = w_nk.shape[0]
+    ew = torch.empty((n, k), dtype=torch.uint8, device=device)
+    sw = torch.empty((n // 128, k // 128), dtype=torch.float32, device=device)
+    B.bq_fp8_block_quantize(w_nk, 128, 128, ew, sw)
+    del w_nk
+    c = torch.empty((m, n), dtype=torch.bfloat16, device=device)
+    name = "fp8_block_gemm(bf16 act quantized 1x128 in the prologue, 128x128 E4M3 w, bf16 C)"
+    fn = lambda: B.bq_fp8_block_gemm(a, ew, sw, c)   # noqa: E731
+    fn()
+    T.collect()
+    for _ in range(reps):
+        T.run(name, fn)
+    ms = _trimmed_mean(T.collect()[name])
+    flops = 2.0 * m * n * k
+    tf = flops / (ms * 1e-3) / 1e12
+    peak, src = _fp8_peak_tflops()
+    nbytes = m * k * 2 + n * k + 4 * sw.numel() + m * n * 2
+    return {"workload": "fp8_blocks_bf16", "kernel": name, "us": round(ms * 1e3, 2),
+            "TFLOP_s": round(tf, 1), "frac": round(tf / peak, 3), "bound": "tensor",
+            "peak_TFLOP_s": round(peak, 1), "peak_source": src, "flops": flops,
+            "shape_mnk": [m, n, k], "bytes": int(nbytes), "launches": 1}
 
 
 def cpu_baseline_oracle(rows_sample=ROWS):

@@ -242,6 +242,21 @@ def fp8_block_quantize(x, block_rows: int, block_cols: int = 128, stream=None):
     return e, s
 
 
+def fp8_block_gemm(a, w_e4m3, w_scale, out_dtype=torch.bfloat16, operands: bool = False, stream=None):
+    """C = a @ w^T in W8A8 block FP8: a [m, k] bf16 / f16 quantized on the fly
+    (1x128 E4M3), w_e4m3 [n, k] with 128x128 tile scales w_scale. Returns C
+    [m, n] (out_dtype f32 or bf16), or (C, a_e4m3, a_scale) with operands=True."""
+    m, k = a.shape
+    n = w_e4m3.shape[0]
+    c = torch.empty((m, n), dtype=out_dtype, device=a.device)
+    ea = sa = None
+    if operands:
+        ea = torch.empty((m, k), dtype=torch.uint8, device=a.device)
+        sa = torch.empty((m, k // 128), dtype=torch.float32, device=a.device)
+    B.bq_fp8_block_gemm(a, w_e4m3, w_scale, c, ea, sa, stream)
+    return (c, ea, sa) if operands else c
+
+
 def fp8_block_dequantize(e, s, block_rows: int, block_cols: int = 128, ydtype=torch.bfloat16,
                          stream=None):
     y = torch.empty(e.shape, dtype=ydtype, device=e.device)

@@ -45,6 +45,8 @@ struct MapArgs;
 cudaError_t int_map_pipe(DT dt, int op, const MapArgs& m, cudaStream_t st);
 // Reads and clears the flag a pipelined kernel sets when a bounded wait gives up.
 cudaError_t pipe_error_take(unsigned int* flag);
+// Reads and clears the flag the block-FP8 GEMM sets when a bounded wait gives up.
+cudaError_t gemm_error_take(unsigned int* flag);
 // A one-CTA kernel whose bounded wait always runs out (bq_diag_wait_timeout).
 cudaError_t wait_diag(uint32_t tries, cudaStream_t st);
 

@@ -133,11 +133,12 @@ cudaError_t fp8_tensor_quant(DT dt, const void* x, int64_t n, uint8_t* e4m3, flo
 }
 
 cudaError_t pipe_error_take(unsigned int* flag) {
-    unsigned int a = 0, b = 0, c = 0;
+    unsigned int a = 0, b = 0, c = 0, d = 0;
     cudaError_t e = pipe_err_f32(&a);
     if (e == cudaSuccess) e = pipe_err_f16(&b);
     if (e == cudaSuccess) e = pipe_err_bf16(&c);
-    *flag = a | b | c;
+    if (e == cudaSuccess) e = gemm_error_take(&d);
+    *flag = a | b | c | d;
     return e;
 }
 

@@ -183,8 +183,9 @@ __device__ __forceinline__ uint32_t sign_bytes(const U4& raw) {
 // negative x; the sign bit of x, OR-ed into each byte afterwards, restores
 // -0 there and changes nothing else (non-zero codes already carry it, and no
 // value is NaN).
+// The codes of one vector as words (VEC / 4 of them: byte i = value i).
 template <class T>
-__device__ __forceinline__ void emit_fp8_fast(const U4& raw, const Recip2& R2, uint8_t* dst) {
+__device__ __forceinline__ uint2 fp8_words_fast(const U4& raw, const Recip2& R2) {
     constexpr int VEC = Traits<T>::VEC;
     constexpr int NP = VEC / 2;
     F2 x[NP];
@@ -192,12 +193,30 @@ __device__ __forceinline__ void emit_fp8_fast(const U4& raw, const Recip2& R2, u
     float t[VEC];
 #pragma unroll
     for (int p = 0; p < NP; ++p) f2_split(div_chain2(x[p], R2), t[2 * p], t[2 * p + 1]);
-    if constexpr (VEC == 8) {
-        st8(dst, e4m3x4(t[0], t[1], t[2], t[3]) | sign_bytes<T, 0>(raw),
-            e4m3x4(t[4], t[5], t[6], t[7]) | sign_bytes<T, 1>(raw));
-    } else {
-        st4(dst, e4m3x4(t[0], t[1], t[2], t[3]) | sign_bytes<T, 0>(raw));
+    uint2 w;
+    w.x = e4m3x4(t[0], t[1], t[2], t[3]) | sign_bytes<T, 0>(raw);
+    if constexpr (VEC == 8) w.y = e4m3x4(t[4], t[5], t[6], t[7]) | sign_bytes<T, 1>(raw);
+    else w.y = 0u;
+    return w;
+}
+template <class T>
+__device__ __forceinline__ void emit_fp8_fast(const U4& raw, const Recip2& R2, uint8_t* dst) {
+    const uint2 w = fp8_words_fast<T>(raw, R2);
+    if constexpr (Traits<T>::VEC == 8) st8(dst, w.x, w.y);
+    else st4(dst, w.x);
+}
+// E4M3 codes of fl(x / s) for any values and scale (the general encoder of
+// the FP8 block formats: IEEE division where the chain cannot be used, the
+// sign of a zero quotient restored), eight values into two words.
+template <bool FAST>
+__device__ __forceinline__ uint2 fp8_words_general8(const float (&v)[8], const Recip& R) {
+    float t[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float d = FAST ? div_chain(v[i], R) : div_any(v[i], R);
+        t[i] = with_quotient_sign(d, v[i], R.s);
     }
+    return make_uint2(e4m3x4(t[0], t[1], t[2], t[3]), e4m3x4(t[4], t[5], t[6], t[7]));
 }
 
 // E2M1 codes of fl(x / s), the sign of each quotient taken from x (no NaN

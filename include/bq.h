@@ -425,6 +425,35 @@ bq_status bq_fp8_block_dequantize(const uint8_t* e4m3, const float* scale, int64
                                   int64_t cols, int32_t block_rows, int32_t block_cols, void* y,
                                   bq_dtype y_dtype, void* stream);
 
+/* [smile.llm.quant] Fp8BlockGemm, with the activation quantization as the
+ * GEMM's prologue: C[i, j] = sum over k-blocks b of
+ *   sa[i, b] * sw[j / 128, b] * sum_{k in b} E4M3(ea[i, k]) * E4M3(w[j, k]),
+ * where ea / sa are the 1x128 E4M3 codes and scales of a (exactly those
+ * bq_fp8_block_quantize writes with block_rows = 1) and w / sw the E4M3
+ * weights with one f32 scale per 128x128 tile (bq_fp8_block_quantize with
+ * block_rows = 128).
+ *   a        [m, k] BF16 or F16, 16-byte aligned (quantized on the fly: the
+ *            codes never leave the chip unless a_e4m3 is given);
+ *   w_e4m3   [n, k] u8, 16-byte aligned (K-major: row j holds output column j);
+ *   w_scale  [ceil(n/128), k/128] f32;
+ *   c        [m, n] F32 or BF16 (c_dtype), 16-byte aligned, overwritten;
+ *   a_e4m3 / a_scale  optional ([m, k] u8 16-byte aligned, [m, k/128] f32;
+ *            both or neither): the activation operand bytes as the tensor
+ *            core reads them (read back from shared memory) and the scales.
+ * k % 128 == 0; m, n, k < 2^31 (BQ_ERR_INVALID_ARG otherwise); m or n = 0
+ * is a no-op. The products of E4M3 values are exact; each k-block's sum is
+ * accumulated by the tensor core in f32, scaled by fl(sa * sw) and added
+ * into an f32 accumulator with one fused multiply-add per block, so C
+ * differs from the exact sum by at most about 2^-16 of
+ * sum_b |sa * sw| * sum_k |ea * w|, plus 2^-150 per block sum where
+ * fl(sa * sw) or C falls below the normal f32 range, plus the final
+ * rounding to BF16. One
+ * launch of a persistent kernel (tcgen05 tensor cores, TMA, one CTA per SM)
+ * on `stream`. BQ_ERR_UNSUPPORTED for other dtypes. */
+bq_status bq_fp8_block_gemm(const void* a, bq_dtype a_dtype, int64_t m, int64_t k,
+                            const uint8_t* w_e4m3, const float* w_scale, int64_t n, void* c,
+                            bq_dtype c_dtype, uint8_t* a_e4m3, float* a_scale, void* stream);
+
 /* --------------------------------------------------- FP8 per-tensor codec */
 /* [smile.llm.quant] Fp8KvCodec (FP8 KV store / load with per-tensor scales):
  * one f32 scale for the whole tensor, the dequantize multiplier as in the FP8

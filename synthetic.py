@@ -133,6 +133,28 @@ class Stream:
                 fill(c0)
         return out.reshape(shape)
 
+    def codes8(self, shape, exclude=(0x7F, 0xFF)) -> torch.Tensor:
+        """Uniformly drawn bytes (uint8) of ``shape``, never one of ``exclude``
+        (by default the two E4M3 NaN codes): byte = the floor(u * K)-th of the
+        K allowed values in increasing order, one uniform per element."""
+        shape = tuple(int(s) for s in shape)
+        n = int(np.prod(shape, dtype=np.int64)) if shape else 1
+        allowed = np.array([b for b in range(256) if b not in exclude], dtype=np.uint8)
+        base = self._take(n)
+        out = np.empty(n, dtype=np.uint8)
+        for c0 in range(0, n, _CHUNK):
+            c1 = min(n, c0 + _CHUNK)
+            u = uniforms(self.seed, base + c0, c1 - c0)
+            out[c0:c1] = allowed[np.minimum((u * len(allowed)).astype(np.int64), len(allowed) - 1)]
+        return torch.from_numpy(out).reshape(shape)
+
+    def uniform_f32(self, shape, lo: float, hi: float) -> torch.Tensor:
+        """f32 values lo + (hi - lo) * u, rounded to f32 (one uniform each)."""
+        shape = tuple(int(s) for s in shape)
+        n = int(np.prod(shape, dtype=np.int64)) if shape else 1
+        u = uniforms(self.seed, self._take(n), n)
+        return torch.from_numpy((lo + (hi - lo) * u).astype(np.float32)).reshape(shape)
+
 
 def bits_tensor(dtype: str) -> torch.Tensor:
     """Every bit pattern of a 16-bit float dtype, in code order (65,536 values)."""
