@@ -198,9 +198,27 @@ __device__ __forceinline__ void fence_async_shared_cluster() {
 // early once another role (of any CTA of the cluster) has set the abort
 // flag. On giving up by itself it sets the flag in every CTA of the cluster
 // and the device error.
+// Non-blocking probe of a phase (no suspension): the common case of a
+// barrier that has already completed costs one instruction.
+template <bool CLUSTER_SCOPE>
+__device__ __forceinline__ bool bar_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    if (CLUSTER_SCOPE)
+        asm volatile("{\n\t.reg .pred p;\n\t"
+                     "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t}"
+                     : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    else
+        asm volatile("{\n\t.reg .pred p;\n\t"
+                     "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t}"
+                     : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
 template <int CL, bool CLUSTER_SCOPE>
 __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
                                          uint32_t abort_addr) {
+    if (bar_test<CLUSTER_SCOPE>(bar, parity)) return true;
     for (uint32_t i = 0; i < (1u << 21); ++i) {
         if (CLUSTER_SCOPE ? bar_try_wait_cl(bar, parity) : bar_try_wait(bar, parity)) return true;
         if ((i & 15u) == 15u && *abort_flag) return false;
