@@ -638,8 +638,86 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# Single-kernel cases for profiler captures (`--ncu-case NAME`): inputs sized
+# above the 126 MB L2 where the kernel streams HBM (so DRAM counters mean
+# something), prepared untimed, then the op launched `--ncu-reps` times.
+NCU_CASES = ("xpose", "nvfp4_quant", "nvfp4_deq", "mxfp8_quant", "mxfp8_deq", "mxfp4_quant",
+             "fp8_1x128_quant", "fp8_block_deq", "tensor_amax", "fp8_tensor_store", "predeq_fp8",
+             "concat_rows", "gemm")
+
+
+def ncu_case(name, reps):
+    import torch
+    import dequantize_absmax_reduce_b200 as m
+    import synthetic
+    A, B = m.api, m._bq
+    torch.cuda.set_device(0)
+    dev = "cuda"
+    st = synthetic.Stream(0)
+    R, K = 16384, 7168                                  # 235 MB of bf16
+    big = lambda: synthetic.device_tensor(st, (R, K), "bf16")   # noqa: E731
+    if name == "xpose":
+        x = synthetic.device_tensor(st, (32768, K), "bf16")    # packed weights 117 MB + scales 15 MB
+        packed, sc, _ = A.nvfp4_quantize(x, s2=1.0)
+        del x
+        fn = lambda: A.packed_transpose(packed, sc, 32768, K, 16, 16)   # noqa: E731
+    elif name == "nvfp4_quant":
+        x = big()
+        fn = lambda: A.nvfp4_quantize(x, s2=1.0)   # noqa: E731
+    elif name == "nvfp4_deq":
+        packed, sc, s2 = A.nvfp4_quantize(big())
+        fn = lambda: A.nvfp4_dequantize(packed, sc, s2)   # noqa: E731
+    elif name == "mxfp8_quant":
+        x = big()
+        fn = lambda: A.mxfp8_quantize(x)   # noqa: E731
+    elif name == "mxfp8_deq":
+        e, s8 = A.mxfp8_quantize(big())
+        fn = lambda: A.mxfp8_dequantize(e, s8)   # noqa: E731
+    elif name == "mxfp4_quant":
+        x = big()
+        fn = lambda: A.mxfp4_quantize(x)   # noqa: E731
+    elif name == "fp8_1x128_quant":
+        x = big()
+        fn = lambda: A.fp8_block_quantize(x, 1, 128)   # noqa: E731
+    elif name == "fp8_block_deq":
+        e, s = A.fp8_block_quantize(big(), 1, 128)
+        fn = lambda: A.fp8_block_dequantize(e, s, 1, 128)   # noqa: E731
+    elif name == "tensor_amax":
+        x = big()
+        fn = lambda: A.tensor_amax(x)   # noqa: E731
+    elif name == "fp8_tensor_store":
+        x = big()
+        sc = torch.tensor([0.01], dtype=torch.float32, device=dev)
+        fn = lambda: A.fp8_tensor_quantize(x, scale=sc)   # noqa: E731
+    elif name == "predeq_fp8":
+        packed, sc, s2 = A.nvfp4_quantize(big())
+        fn = lambda: A.nvfp4_predequant_to_fp8(packed, sc, s2)   # noqa: E731
+    elif name == "concat_rows":
+        p1, s1, _ = A.nvfp4_quantize(big(), s2=1.0)
+        p2, s2_, _ = A.nvfp4_quantize(big(), s2=1.0)
+        fn = lambda: A.nvfp4_concat_rows(p1, s1, 1.0, p2, s2_, 1.0, K)   # noqa: E731
+    elif name == "gemm":
+        a = synthetic.device_tensor(st, (2048, K), "bf16")
+        w = synthetic.device_tensor(st, (4608, K), "bf16", std=0.05)
+        ew, sw = A.fp8_block_quantize(w, 128, 128)
+        fn = lambda: A.fp8_block_gemm(a, ew, sw)   # noqa: E731
+    else:
+        raise SystemExit(f"unknown case {name}")
+    torch.cuda.synchronize()
+    for _ in range(reps):
+        fn()
+    torch.cuda.synchronize()
+    st_ = B.bq_check_device_error()
+    print(f"ncu case {name}: {reps} launches, device status {B.bq_status_string(st_)}", flush=True)
+    if st_ != B.BQ_OK:
+        raise SystemExit(1)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--ncu-case", choices=NCU_CASES, default=None,
+                    help="run one op on a profiling-size input and exit (for ncu captures)")
+    ap.add_argument("--ncu-reps", type=int, default=2)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
@@ -647,6 +725,9 @@ def main():
     ap.add_argument("--no-breakdown", action="store_true", help="skip the per-granularity table")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
+    if args.ncu_case:
+        ncu_case(args.ncu_case, args.ncu_reps)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
