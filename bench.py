@@ -406,7 +406,7 @@ def per_granularity(B, api, torch, device, peak, reps=40):
     timed(wl, "fp8_block_dequantize(128x128 weight)",
           lambda: B.bq_fp8_block_dequantize(e, s, 128, 128, y), 3 * n + 4 * s.numel(), 1)
     del e, s, y
-    out.append(gemm_bench(B, torch, device, wt, T))
+    out.extend(gemm_bench(B, torch, device, wt, T))
     return out
 
 
@@ -447,10 +447,36 @@ def gemm_bench(B, torch, device, wt, T, reps=10):
     tf = flops / (ms * 1e-3) / 1e12
     peak, src = _fp8_peak_tflops()
     nbytes = m * k * 2 + n * k + 4 * sw.numel() + m * n * 2
-    return {"workload": "fp8_blocks_bf16", "kernel": name, "us": round(ms * 1e3, 2),
+    out = [{"workload": "fp8_blocks_bf16", "kernel": name, "us": round(ms * 1e3, 2),
             "TFLOP_s": round(tf, 1), "frac": round(tf / peak, 3), "bound": "tensor",
             "peak_TFLOP_s": round(peak, 1), "peak_source": src, "flops": flops,
-            "shape_mnk": [m, n, k], "bytes": int(nbytes), "launches": 1}
+            "shape_mnk": [m, n, k], "bytes": int(nbytes), "launches": 1}]
+    # Two passes: quantize the activations once (1x128), then the GEMM on the
+    # codes; timed together (both launches between one event pair) and alone.
+    ea = torch.empty((m, k), dtype=torch.uint8, device=device)
+    sa = torch.empty((m, k // 128), dtype=torch.float32, device=device)
+    name2 = "fp8_block_gemm_quantized(activations quantized by a separate 1x128 pass, timed together)"
+    name3 = "fp8_block_gemm_quantized(GEMM alone, activations already quantized)"
+
+    def two_pass():
+        B.bq_fp8_block_quantize(a, 1, 128, ea, sa)
+        B.bq_fp8_block_gemm_quantized(ea, sa, ew, sw, c)
+
+    two_pass()
+    T.collect()
+    for _ in range(reps):
+        T.run(name2, two_pass)
+    for _ in range(reps):
+        T.run(name3, lambda: B.bq_fp8_block_gemm_quantized(ea, sa, ew, sw, c))
+    col = T.collect()
+    for nm, launches in ((name2, 2), (name3, 1)):
+        ms2 = _trimmed_mean(col[nm])
+        tf2 = flops / (ms2 * 1e-3) / 1e12
+        out.append({"workload": "fp8_blocks_bf16", "kernel": nm, "us": round(ms2 * 1e3, 2),
+                    "TFLOP_s": round(tf2, 1), "frac": round(tf2 / peak, 3), "bound": "tensor",
+                    "peak_TFLOP_s": round(peak, 1), "peak_source": src, "flops": flops,
+                    "shape_mnk": [m, n, k], "launches": launches})
+    return out
 
 
 def cpu_baseline_oracle(rows_sample=ROWS):

@@ -97,6 +97,7 @@ _SIGS = {
     "bq_fp8_block_quantize": [_P, C.c_int, _I64, _I64, _I32, _I32, _P, _P, _P],
     "bq_fp8_block_dequantize": [_P, _P, _I64, _I64, _I32, _I32, _P, C.c_int, _P],
     "bq_fp8_block_gemm": [_P, C.c_int, _I64, _I64, _P, _P, _I64, _P, C.c_int, _P, _P, _P],
+    "bq_fp8_block_gemm_quantized": [_P, _P, _I64, _I64, _P, _P, _I64, _P, C.c_int, _P],
     "bq_packed_transpose": [_P, _P, _I64, _I64, _I64, _I64, _P, _P, C.POINTER(_I64), _P],
     "bq_packed_transpose_concat": [_I32, C.POINTER(_P), C.POINTER(_P), C.POINTER(_I64), _I64, _I64,
                                    _I64, _P, _P, C.POINTER(_I64), _P],
@@ -408,6 +409,14 @@ def bq_fp8_block_gemm(a, w_e4m3, w_scale, c, a_e4m3=None, a_scale=None, stream=N
     _check(lib.bq_fp8_block_gemm(_ptr(a), DTYPE[a.dtype], m, k, _ptr(w_e4m3), _ptr(w_scale), n, _ptr(c),
                                  DTYPE[c.dtype], _ptr(a_e4m3), _ptr(a_scale), _stream(stream)),
            "bq_fp8_block_gemm")
+
+
+def bq_fp8_block_gemm_quantized(a_e4m3, a_scale, w_e4m3, w_scale, c, stream=None):
+    m, k = a_e4m3.shape
+    n = w_e4m3.shape[0]
+    _check(lib.bq_fp8_block_gemm_quantized(_ptr(a_e4m3), _ptr(a_scale), m, k, _ptr(w_e4m3), _ptr(w_scale), n,
+                                           _ptr(c), DTYPE[c.dtype], _stream(stream)),
+           "bq_fp8_block_gemm_quantized")
 
 
 def bq_fp8_block_dequantize(e4m3, scale, block_rows, block_cols, y, stream=None):

@@ -257,6 +257,16 @@ def fp8_block_gemm(a, w_e4m3, w_scale, out_dtype=torch.bfloat16, operands: bool 
     return (c, ea, sa) if operands else c
 
 
+def fp8_block_gemm_quantized(a_e4m3, a_scale, w_e4m3, w_scale, out_dtype=torch.bfloat16, stream=None):
+    """C = A @ W^T from activations already quantized (1x128 E4M3 codes
+    a_e4m3 [m, k] and scales a_scale [m, k/128])."""
+    m = a_e4m3.shape[0]
+    n = w_e4m3.shape[0]
+    c = torch.empty((m, n), dtype=out_dtype, device=a_e4m3.device)
+    B.bq_fp8_block_gemm_quantized(a_e4m3, a_scale, w_e4m3, w_scale, c, stream)
+    return c
+
+
 def fp8_block_dequantize(e, s, block_rows: int, block_cols: int = 128, ydtype=torch.bfloat16,
                          stream=None):
     y = torch.empty(e.shape, dtype=ydtype, device=e.device)

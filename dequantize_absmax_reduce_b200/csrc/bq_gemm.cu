@@ -107,6 +107,7 @@ struct GemmArgs {
     int c_bf16;
     uint8_t* dump_q;    // optional [m, k]: operand bytes read back from shared memory
     float* dump_s;      // optional [m, nkb]
+    const float* sa;    // activation scales [m, nkb] (pre-quantized activations only)
 };
 
 // ------------------------------------------------------------ PTX helpers
@@ -315,6 +316,55 @@ __device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr) {
 // Instruction descriptor: f32 accumulator, E4M3 x E4M3, both K-major,
 // N = BN, M = BM, dense, no negation.
 constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+
+// One k-block of promotion for one thread (a TMEM lane = a row of the tile,
+// 128 columns from `ta`): acc[i] += partial[i] * cf, one fused multiply-add
+// per column, on column pairs.
+__device__ __forceinline__ void promote_block(F2 (&acc)[64], uint32_t ta, F2 cf) {
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+        F2 p[16];
+        tmem_ld32(ta + 32 * ch, p);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[16 * ch + i] = f2_fma(p[i], cf, acc[16 * ch + i]);
+    }
+}
+// The thread's 128 columns of C (row `row`, from column col0), in C's dtype;
+// columns past n are skipped.
+__device__ __forceinline__ void store_c_half(const GemmArgs& g, int64_t row, int64_t col0, const F2 (&acc)[64]) {
+    const int64_t ncols = min((int64_t)128, g.n - col0);
+    float v[128];
+#pragma unroll
+    for (int i = 0; i < 64; ++i) f2_split(acc[i], v[2 * i], v[2 * i + 1]);
+    if (g.c_bf16) {
+        __nv_bfloat16* cr = reinterpret_cast<__nv_bfloat16*>(g.c) + row * g.n + col0;
+        if (ncols == 128 && (g.n & 7) == 0) {
+#pragma unroll
+            for (int i = 0; i < 128; i += 8) {
+                U4 o;
+                o.x = pack_bf16x2(v[i], v[i + 1]); o.y = pack_bf16x2(v[i + 2], v[i + 3]);
+                o.z = pack_bf16x2(v[i + 4], v[i + 5]); o.w = pack_bf16x2(v[i + 6], v[i + 7]);
+                *reinterpret_cast<U4*>(cr + i) = o;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 128; ++i)
+                if (i < ncols) cr[i] = __float2bfloat16_rn(v[i]);
+        }
+    } else {
+        float* cr = reinterpret_cast<float*>(g.c) + row * g.n + col0;
+        if (ncols == 128 && (g.n & 3) == 0) {
+#pragma unroll
+            for (int i = 0; i < 128; i += 4)
+                *reinterpret_cast<float4*>(cr + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 128; ++i)
+                if (i < ncols) cr[i] = v[i];
+        }
+    }
+}
 
 // Cluster tile u -> (M tile, cluster tile along N): bands of `band` M tiles,
 // walked down M first, so the clusters working at one time share a few
@@ -528,14 +578,7 @@ __global__ void __launch_bounds__(NT, 1) k_fp8_gemm(const __grid_constant__ CUte
                 if (!(ok = bar_wait<CL, false>(bar(P::B_TFULL + buf), (uint32_t)(it >> 1) & 1u, abort_flag, abort_addr))) break;
                 tc_fence_after();
                 const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN + 128 * h);
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    F2 p[16];
-                    tmem_ld32(ta + 32 * ch, p);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) acc[16 * ch + i] = f2_fma(p[i], cf, acc[16 * ch + i]);
-                }
+                promote_block(acc, ta, cf);
                 tc_fence_before();
                 bar_arrive(bar(P::B_TEMPTY + buf));
                 ++it;
@@ -544,39 +587,7 @@ __global__ void __launch_bounds__(NT, 1) k_fp8_gemm(const __grid_constant__ CUte
             }
             if (!ok) break;
             const int64_t row = (int64_t)mt * BM + rloc;
-            if (row < g.m && half_in) {
-                const int64_t ncols = min((int64_t)128, g.n - col0);
-                float v[128];
-#pragma unroll
-                for (int i = 0; i < 64; ++i) f2_split(acc[i], v[2 * i], v[2 * i + 1]);
-                if (g.c_bf16) {
-                    __nv_bfloat16* cr = reinterpret_cast<__nv_bfloat16*>(g.c) + row * g.n + col0;
-                    if (ncols == 128 && (g.n & 7) == 0) {
-#pragma unroll
-                        for (int i = 0; i < 128; i += 8) {
-                            U4 o;
-                            o.x = pack_bf16x2(v[i], v[i + 1]); o.y = pack_bf16x2(v[i + 2], v[i + 3]);
-                            o.z = pack_bf16x2(v[i + 4], v[i + 5]); o.w = pack_bf16x2(v[i + 6], v[i + 7]);
-                            *reinterpret_cast<U4*>(cr + i) = o;
-                        }
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 128; ++i)
-                            if (i < ncols) cr[i] = __float2bfloat16_rn(v[i]);
-                    }
-                } else {
-                    float* cr = reinterpret_cast<float*>(g.c) + row * g.n + col0;
-                    if (ncols == 128 && (g.n & 3) == 0) {
-#pragma unroll
-                        for (int i = 0; i < 128; i += 4)
-                            *reinterpret_cast<float4*>(cr + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 128; ++i)
-                            if (i < ncols) cr[i] = v[i];
-                    }
-                }
-            }
+            if (row < g.m && half_in) store_c_half(g, row, col0, acc);
         }
     } else {
         // ---------------------------------------------------- control warps
@@ -703,6 +714,180 @@ __global__ void __launch_bounds__(NT, 1) k_fp8_gemm(const __grid_constant__ CUte
     }
 }
 
+// ------------------------------------------------------------ activations
+// already quantized
+// The same matrix multiply for activations given as 1x128 E4M3 codes and
+// scales (as bq_fp8_block_quantize writes them): no prologue, so every CTA
+// works alone. 384 threads: warp 0 loads activation code tiles
+// [128 rows x 128 bytes] and warp 1 weight tiles [256 rows x 128 bytes] by TMA
+// (128-byte swizzle: the operand layout the MMA reads), warp 2 allocates TMEM
+// and issues the MMAs, warps 4-11 promote as in k_fp8_gemm with the
+// activation scales read from global memory two blocks ahead. Register
+// split: warps 0-3 keep 56, warps 4-11 take 224 (128*56 + 256*224 =
+// 384 * 168, the launch count).
+struct PlanQ {
+    static constexpr int SQ = 4, SW = 4;
+    static constexpr uint32_t OFF_AQ = 0;
+    static constexpr uint32_t OFF_W = OFF_AQ + SQ * AQ_BYTES;
+    static constexpr uint32_t OFF_BAR = OFF_W + SW * W_BYTES;
+    static constexpr int B_FULL_Q = 0, B_EMPTY_Q = B_FULL_Q + SQ, B_FULL_W = B_EMPTY_Q + SQ,
+                         B_EMPTY_W = B_FULL_W + SW, B_TFULL = B_EMPTY_W + SW, B_TEMPTY = B_TFULL + 2,
+                         B_MMA_DONE = B_TEMPTY + 2, N_BAR = B_MMA_DONE + 1;
+    static constexpr uint32_t OFF_MISC = OFF_BAR + N_BAR * 8;
+    static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+constexpr int NT_Q = 384;
+constexpr int REGQ_LAUNCH = 168, REGQ_CTL = 56, REGQ_ACC = 224;
+static_assert(128 * REGQ_CTL + 256 * REGQ_ACC <= NT_Q * REGQ_LAUNCH, "register split");
+
+__global__ void __launch_bounds__(NT_Q, 1) k_fp8_gemm_q(const __grid_constant__ CUtensorMap tm_a,
+                                                         const __grid_constant__ CUtensorMap tm_w,
+                                                         const GemmArgs g) {
+    using P = PlanQ;
+    constexpr int SQ = P::SQ, SW = P::SW;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = sm_addr(smem_raw);
+    const uint32_t base = (raw_base + 1023u) & ~1023u;
+    uint8_t* sb = smem_raw + (base - raw_base);
+    volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(sb + P::OFF_MISC);
+    volatile uint32_t* abort_flag = misc + 1;
+    const uint32_t abort_addr = base + P::OFF_MISC + 4;
+    auto bar = [&](int i) -> uint32_t { return base + P::OFF_BAR + 8u * (uint32_t)i; };
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < SQ; ++i) { bar_init(bar(P::B_FULL_Q + i), 1); bar_init(bar(P::B_EMPTY_Q + i), 1); }
+        for (int i = 0; i < SW; ++i) { bar_init(bar(P::B_FULL_W + i), 1); bar_init(bar(P::B_EMPTY_W + i), 1); }
+        for (int i = 0; i < 2; ++i) { bar_init(bar(P::B_TFULL + i), 1); bar_init(bar(P::B_TEMPTY + i), 256); }
+        bar_init(bar(P::B_MMA_DONE), 1);
+        misc[1] = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0 && lane == 0) prefetch_map(&tm_a);
+    if (warp == 1 && lane == 0) prefetch_map(&tm_w);
+    if (warp == 2) tmem_alloc(base + P::OFF_MISC, TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc[0];
+    const int nkb = g.nkb;
+    const int64_t cid = blockIdx.x, ncl = gridDim.x;
+
+    if (warp < 4) {
+        set_max_regs_dec<REGQ_CTL>();
+        if (warp == 0 && lane == 0) {
+            // Activation code tiles.
+            int iq = 0;
+            bool ok = true;
+            for (int64_t u = cid; ok && u < g.n_ctiles; u += ncl) {
+                int mt, nt;
+                ctile_coords(g, u, mt, nt);
+                for (int kb = 0; kb < nkb; ++kb) {
+                    const int sq = iq % SQ;
+                    if (!(ok = bar_wait<1, false>(bar(P::B_EMPTY_Q + sq), ((uint32_t)(iq / SQ) & 1u) ^ 1u, abort_flag, abort_addr))) break;
+                    const uint32_t fb = bar(P::B_FULL_Q + sq);
+                    bar_expect_tx(fb, AQ_BYTES);
+                    tma_2d(base + P::OFF_AQ + (uint32_t)sq * AQ_BYTES, &tm_a, kb * BK, mt * BM, fb);
+                    ++iq;
+                }
+            }
+            for (int i = max(0, iq - SQ); i < iq; ++i) bar_drain(bar(P::B_FULL_Q + i % SQ), (uint32_t)(i / SQ) & 1u);
+        } else if (warp == 1 && lane == 0) {
+            // Weight tiles.
+            int iw = 0;
+            bool ok = true;
+            for (int64_t u = cid; ok && u < g.n_ctiles; u += ncl) {
+                int mt, nt;
+                ctile_coords(g, u, mt, nt);
+                for (int kb = 0; kb < nkb; ++kb) {
+                    const int sw = iw % SW;
+                    if (!(ok = bar_wait<1, false>(bar(P::B_EMPTY_W + sw), ((uint32_t)(iw / SW) & 1u) ^ 1u, abort_flag, abort_addr))) break;
+                    const uint32_t fb = bar(P::B_FULL_W + sw);
+                    bar_expect_tx(fb, W_BYTES);
+                    tma_2d(base + P::OFF_W + (uint32_t)sw * W_BYTES, &tm_w, kb * BK, nt * BN, fb);
+                    ++iw;
+                }
+            }
+            for (int i = max(0, iw - SW); i < iw; ++i) bar_drain(bar(P::B_FULL_W + i % SW), (uint32_t)(i / SW) & 1u);
+        } else if (warp == 2 && lane == 0) {
+            // MMA issue.
+            int iq = 0, iw = 0, it = 0;
+            bool ok = true;
+            for (int64_t u = cid; ok && u < g.n_ctiles; u += ncl) {
+                for (int kb = 0; kb < nkb; ++kb) {
+                    const int buf = it & 1;
+                    if (!(ok = bar_wait<1, false>(bar(P::B_TEMPTY + buf), ((uint32_t)(it >> 1) & 1u) ^ 1u, abort_flag, abort_addr))) break;
+                    const int sq = iq % SQ, sw = iw % SW;
+                    if (!(ok = bar_wait<1, false>(bar(P::B_FULL_Q + sq), (uint32_t)(iq / SQ) & 1u, abort_flag, abort_addr))) break;
+                    if (!(ok = bar_wait<1, false>(bar(P::B_FULL_W + sw), (uint32_t)(iw / SW) & 1u, abort_flag, abort_addr))) break;
+                    tc_fence_after();
+                    const uint64_t da = desc_k_sw128(base + P::OFF_AQ + (uint32_t)sq * AQ_BYTES);
+                    const uint64_t dw = desc_k_sw128(base + P::OFF_W + (uint32_t)sw * W_BYTES);
+                    const uint32_t d = tmem + (uint32_t)(buf * BN);
+#pragma unroll
+                    for (int k4 = 0; k4 < BK / 32; ++k4)
+                        mma_f8(d, da + (uint64_t)(2 * k4), dw + (uint64_t)(2 * k4), kIdesc, k4 > 0 ? 1u : 0u);
+                    mma_commit(bar(P::B_TFULL + buf));
+                    mma_commit(bar(P::B_EMPTY_W + sw));
+                    mma_commit(bar(P::B_EMPTY_Q + sq));
+                    ++iq; ++iw; ++it;
+                }
+            }
+            mma_commit(bar(P::B_MMA_DONE));
+            bar_drain(bar(P::B_MMA_DONE), 0u);
+        }
+    } else {
+        // ---------------------------------------------------- promotion
+        set_max_regs_inc<REGQ_ACC>();
+        const int q = warp & 3, h = (warp - 4) >> 2;
+        const int rloc = 32 * q + lane;
+        int it = 0;
+        bool ok = true;
+        F2 acc[64];
+        for (int64_t u = cid; ok && u < g.n_ctiles; u += ncl) {
+            int mt, nt;
+            ctile_coords(g, u, mt, nt);
+#pragma unroll
+            for (int i = 0; i < 64; ++i) acc[i] = 0ull;
+            const int64_t col0 = (int64_t)nt * BN + 128 * h;
+            const bool half_in = col0 < g.n;
+            const int64_t row = (int64_t)mt * BM + rloc;
+            const bool row_in = row < g.m;
+            const float* swp = g.sw + (half_in ? (col0 / 128) * nkb : 0);
+            const float* sap = g.sa + (row_in ? row * nkb : 0);
+            // Both scales two blocks ahead.
+            float sw0 = half_in ? __ldg(swp) : 0.0f, sa0 = row_in ? __ldg(sap) : 0.0f;
+            float sw1 = (half_in && nkb > 1) ? __ldg(swp + 1) : 0.0f;
+            float sa1 = (row_in && nkb > 1) ? __ldg(sap + 1) : 0.0f;
+            for (int kb = 0; kb < nkb; ++kb) {
+                const bool more = kb + 2 < nkb;
+                const float sw2 = (half_in && more) ? __ldg(swp + kb + 2) : 0.0f;
+                const float sa2 = (row_in && more) ? __ldg(sap + kb + 2) : 0.0f;
+                const F2 cf = f2_bcast(__fmul_rn(sa0, sw0));
+                const int buf = it & 1;
+                if (!(ok = bar_wait<1, false>(bar(P::B_TFULL + buf), (uint32_t)(it >> 1) & 1u, abort_flag, abort_addr))) break;
+                tc_fence_after();
+                promote_block(acc, tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN + 128 * h), cf);
+                tc_fence_before();
+                bar_arrive(bar(P::B_TEMPTY + buf));
+                ++it;
+                sw0 = sw1; sw1 = sw2;
+                sa0 = sa1; sa1 = sa2;
+            }
+            if (!ok) break;
+            if (row_in && half_in) store_c_half(g, row, col0, acc);
+        }
+    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
 cudaError_t encode_map(CUtensorMap* tm, CUtensorMapDataType dt, const void* p, uint64_t inner,
                        uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
     static const PFN_cuTensorMapEncodeTiled_v12000 encode = [] {
@@ -814,6 +999,44 @@ cudaError_t launch_gemm(const void* a, int64_t m, int64_t k, const uint8_t* w, c
     return cudaGetLastError();
 }
 
+cudaError_t launch_gemm_q(const uint8_t* ea, const float* sa, int64_t m, int64_t k, const uint8_t* w,
+                          const float* sw, int64_t n, void* c, int c_bf16, cudaStream_t st) {
+    static int ready[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorUnknown;
+    if (dev < 0 || dev >= 64) return cudaErrorNotSupported;
+    if (!__atomic_load_n(&ready[dev], __ATOMIC_ACQUIRE)) {
+        cudaFuncAttributes fa;
+        cudaError_t e = cudaFuncGetAttributes(&fa, k_fp8_gemm_q);
+        if (e != cudaSuccess) return e;
+        if (fa.numRegs != REGQ_LAUNCH) return cudaErrorNotSupported;
+        e = cudaFuncSetAttribute(k_fp8_gemm_q, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PlanQ::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        __atomic_store_n(&ready[dev], 1, __ATOMIC_RELEASE);
+    }
+    CUtensorMap ta, tw;
+    cudaError_t e;
+    if ((e = encode_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, ea, (uint64_t)k, (uint64_t)m, (uint64_t)k, BK, BM)) !=
+        cudaSuccess)
+        return e;
+    if ((e = encode_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, (uint64_t)k, (uint64_t)n, (uint64_t)k, BK, BN)) !=
+        cudaSuccess)
+        return e;
+    GemmArgs g = {};
+    g.m = m; g.n = n; g.k = k;
+    g.nkb = (int)(k / BK);
+    g.mtiles = (int)((m + BM - 1) / BM);
+    g.ntiles = (int)((n + BN - 1) / BN);
+    g.nct = g.ntiles;
+    g.band = min(16, g.mtiles);
+    g.n_ctiles = (int64_t)g.mtiles * g.nct;
+    g.sw = sw; g.c = c; g.c_bf16 = c_bf16; g.sa = sa;
+    int64_t grid = sm_count();
+    if (grid > g.n_ctiles) grid = g.n_ctiles;
+    k_fp8_gemm_q<<<(unsigned)grid, NT_Q, PlanQ::SMEM_BYTES, st>>>(ta, tw, g);
+    return cudaGetLastError();
+}
+
 // Cluster size: activations are quantized once per cluster of CL CTAs that
 // share them; CL = 4 when the tile row holds at least four N tiles.
 template <class T>
@@ -872,6 +1095,23 @@ extern "C" bq_status bq_fp8_block_gemm(const void* a, bq_dtype a_dtype, int64_t 
     const cudaError_t e = (a_dtype == BQ_BF16)
         ? bq::launch_gemm_any<__nv_bfloat16>(a, m, k, w_e4m3, w_scale, n, c, c_dtype == BQ_BF16, a_e4m3, a_scale, st, cl)
         : bq::launch_gemm_any<__half>(a, m, k, w_e4m3, w_scale, n, c, c_dtype == BQ_BF16, a_e4m3, a_scale, st, cl);
+    if (e == cudaErrorNotSupported) return BQ_ERR_UNSUPPORTED;
+    return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+}
+
+extern "C" bq_status bq_fp8_block_gemm_quantized(const uint8_t* a_e4m3, const float* a_scale, int64_t m,
+                                                 int64_t k, const uint8_t* w_e4m3, const float* w_scale,
+                                                 int64_t n, void* c, bq_dtype c_dtype, void* stream) {
+    if (c_dtype != BQ_F32 && c_dtype != BQ_BF16) return BQ_ERR_UNSUPPORTED;
+    if (m < 0 || n < 0 || k <= 0 || k % 128 != 0) return BQ_ERR_INVALID_ARG;
+    if (m >= (1ll << 31) || n >= (1ll << 31) || k >= (1ll << 31)) return BQ_ERR_INVALID_ARG;
+    if (m == 0 || n == 0) return BQ_OK;
+    if (!a_e4m3 || !a_scale || !w_e4m3 || !w_scale || !c) return BQ_ERR_INVALID_ARG;
+    if (((uintptr_t)a_e4m3 & 15u) || ((uintptr_t)w_e4m3 & 15u) || ((uintptr_t)w_scale & 3u) ||
+        ((uintptr_t)a_scale & 3u) || ((uintptr_t)c & 15u))
+        return BQ_ERR_MISALIGNED;
+    const cudaError_t e = bq::launch_gemm_q(a_e4m3, a_scale, m, k, w_e4m3, w_scale, n, c, c_dtype == BQ_BF16,
+                                            (cudaStream_t)stream);
     if (e == cudaErrorNotSupported) return BQ_ERR_UNSUPPORTED;
     return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }

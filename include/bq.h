@@ -454,6 +454,20 @@ bq_status bq_fp8_block_gemm(const void* a, bq_dtype a_dtype, int64_t m, int64_t 
                             const uint8_t* w_e4m3, const float* w_scale, int64_t n, void* c,
                             bq_dtype c_dtype, uint8_t* a_e4m3, float* a_scale, void* stream);
 
+/* [smile.llm.quant] Fp8BlockGemm on activations already quantized: the same
+ * product as bq_fp8_block_gemm with the activation codes and scales given
+ *   a_e4m3  [m, k] u8, 16-byte aligned; a_scale [m, k/128] f32 (exactly what
+ *           bq_fp8_block_quantize writes with block_rows = 1, or the a_e4m3 /
+ *           a_scale outputs of bq_fp8_block_gemm),
+ * and the same weights, output, shape rules, errors and accuracy bound. For
+ * activations that several weights multiply, and for large n, quantizing
+ * once (bq_fp8_block_quantize) and calling this entry is cheaper than the
+ * fused prologue, which requantizes a tile row for every group of N tiles.
+ * One launch of a persistent kernel (one CTA per SM, TMA, tcgen05). */
+bq_status bq_fp8_block_gemm_quantized(const uint8_t* a_e4m3, const float* a_scale, int64_t m, int64_t k,
+                                      const uint8_t* w_e4m3, const float* w_scale, int64_t n, void* c,
+                                      bq_dtype c_dtype, void* stream);
+
 /* --------------------------------------------------- FP8 per-tensor codec */
 /* [smile.llm.quant] Fp8KvCodec (FP8 KV store / load with per-tensor scales):
  * one f32 scale for the whole tensor, the dequantize multiplier as in the FP8

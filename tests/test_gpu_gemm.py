@@ -109,6 +109,24 @@ def test_gemm_parity(bq, orc, a_dtype, c_dtype, m, n, k):
     _check_c(orc, c, c_ref, ea, sa, ew, sw, f"C {m}x{n}x{k}")
 
 
+@pytest.mark.parametrize("c_dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("m,n,k", [(1, 16, 128), (300, 520, 512), (257, 384, 1024), (64, 1000, 384)])
+def test_gemm_quantized_parity(bq, orc, c_dtype, m, n, k):
+    """Activations given as 1x128 codes and scales (the oracle's own): C
+    within the bound, and bit-identical to the fused kernel's C (same
+    operands, same block sums, same promotion order)."""
+    st = synthetic.Stream(3000 + m + n + k)
+    a = st.tensor((m, k), "bf16", outlier_p=0.01, outlier_factor=30.0)
+    ew, sw = _weights_from_oracle(orc, n, k, 4000 + n + k)
+    ea, sa = orc.fp8_block_quantize(a, 1, 128)
+    c = bq.api.fp8_block_gemm_quantized(ea.cuda(), sa.cuda(), ew.cuda(), sw.cuda(), out_dtype=c_dtype)
+    c_ref, ea_r, sa_r = orc.fp8_block_gemm(a, ew, sw)
+    assert_bitwise(ea, ea_r, "oracle codes")
+    _check_c(orc, c, c_ref, ea, sa, ew, sw, f"C quantized {m}x{n}x{k}")
+    c_fused = bq.api.fp8_block_gemm(a.cuda(), ew.cuda(), sw.cuda(), out_dtype=c_dtype)
+    assert_bitwise(c, c_fused, "quantized-activation GEMM vs fused prologue")
+
+
 def test_gemm_special_rows(bq, orc):
     # Rows of zeros, of subnormals only, of values at the bf16 range's top, a
     # row with one huge outlier, a NaN, and an infinity (whose block scale is
@@ -177,6 +195,9 @@ def test_gemm_workload_full_size(bq, orc):
     assert_bitwise(cpu(ea_g)[rows], ea, "codes vs oracle")
     assert_bitwise(cpu(sa_g)[rows], sa, "scales vs oracle")
     _check_c(orc, cpu(c)[rows], c_ref, ea, sa, ew, sw, "full size")
+    # The same product from the quantized activations: bit-identical C.
+    cq = bq.api.fp8_block_gemm_quantized(ea_g, sa_g, ew.cuda(), sw.cuda(), out_dtype=torch.bfloat16)
+    assert_bitwise(cq, c, "full size: quantized-activation GEMM vs fused prologue")
 
 
 def test_gemm_arguments(bq):
@@ -203,3 +224,11 @@ def test_gemm_arguments(bq):
     assert e.value.status == B.BQ_ERR_MISALIGNED
     # m = 0 is a no-op
     B.bq_fp8_block_gemm(a[:0], w, s, c[:0])
+    ea = torch.zeros((4, 128), dtype=torch.uint8, device="cuda")
+    sa = torch.ones((4, 1), dtype=torch.float32, device="cuda")
+    with pytest.raises(B.BqError) as e:
+        B.bq_fp8_block_gemm_quantized(ea, sa, w, s, c.half())
+    assert e.value.status == B.BQ_ERR_UNSUPPORTED
+    with pytest.raises(B.BqError) as e:
+        B.bq_fp8_block_gemm_quantized(ea[:, :100].contiguous(), sa, w[:, :100].contiguous(), s, c)
+    assert e.value.status == B.BQ_ERR_INVALID_ARG
