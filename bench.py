@@ -669,7 +669,7 @@ def run_reference(args):
 # something), prepared untimed, then the op launched `--ncu-reps` times.
 NCU_CASES = ("xpose", "nvfp4_quant", "nvfp4_deq", "mxfp8_quant", "mxfp8_deq", "mxfp4_quant",
              "fp8_1x128_quant", "fp8_block_deq", "tensor_amax", "fp8_tensor_store", "predeq_fp8",
-             "concat_rows", "gemm")
+             "concat_rows", "gemm", "gemm_q")
 
 
 def ncu_case(name, reps):
@@ -727,6 +727,12 @@ def ncu_case(name, reps):
         w = synthetic.device_tensor(st, (4608, K), "bf16", std=0.05)
         ew, sw = A.fp8_block_quantize(w, 128, 128)
         fn = lambda: A.fp8_block_gemm(a, ew, sw)   # noqa: E731
+    elif name == "gemm_q":
+        a = synthetic.device_tensor(st, (4096, K), "bf16")
+        w = synthetic.device_tensor(st, (9216, K), "bf16", std=0.05)
+        ea, sa = A.fp8_block_quantize(a, 1, 128)
+        ew, sw = A.fp8_block_quantize(w, 128, 128)
+        fn = lambda: A.fp8_block_gemm_quantized(ea, sa, ew, sw)   # noqa: E731
     else:
         raise SystemExit(f"unknown case {name}")
     torch.cuda.synchronize()
