@@ -285,21 +285,19 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                  :: "r"(bar) : "memory");
 }
-// 32 consecutive f32 columns of this thread's TMEM lane, as 16 pairs.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, F2 (&v)[16]) {
-    uint32_t r[32];
+// 32 consecutive f32 columns of this thread's TMEM lane (raw bits). The
+// registers hold the values only after tmem_ld_wait and tmem_regs_ready.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-                 "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-                 "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-                   "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-                   "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-                   "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-                   "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-                   "=r"(r[31])
+                 "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
                  : "r"(taddr));
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = f2_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+}
+// Placed after tcgen05.wait::ld: no use of the loaded registers is moved
+// above it (the compiler sees them written here).
+__device__ __forceinline__ void tmem_regs_ready(uint32_t (&r)[32]) {
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
 }
 __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
@@ -319,15 +317,39 @@ constexpr uint32_t kIdesc = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t
 
 // One k-block of promotion for one thread (a TMEM lane = a row of the tile,
 // 128 columns from `ta`): acc[i] += partial[i] * cf, one fused multiply-add
-// per column, on column pairs.
+// per column, on column pairs. Four loads of 32 columns, each waited for.
 __device__ __forceinline__ void promote_block(F2 (&acc)[64], uint32_t ta, F2 cf) {
 #pragma unroll
     for (int ch = 0; ch < 4; ++ch) {
-        F2 p[16];
-        tmem_ld32(ta + 32 * ch, p);
+        uint32_t r[32];
+        tmem_ld32(ta + 32 * ch, r);
         tmem_ld_wait();
+        tmem_regs_ready(r);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) acc[16 * ch + i] = f2_fma(p[i], cf, acc[16 * ch + i]);
+        for (int i = 0; i < 16; ++i)
+            acc[16 * ch + i] = f2_fma(f2_pack(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), cf,
+                                      acc[16 * ch + i]);
+    }
+}
+// The same with two loads in flight per wait (64 more registers): half the
+// TMEM round trips per k-block.
+__device__ __forceinline__ void promote_block_2x(F2 (&acc)[64], uint32_t ta, F2 cf) {
+#pragma unroll
+    for (int hb = 0; hb < 2; ++hb) {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(ta + 64 * hb, r0);
+        tmem_ld32(ta + 64 * hb + 32, r1);
+        tmem_ld_wait();
+        tmem_regs_ready(r0);
+        tmem_regs_ready(r1);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            acc[32 * hb + i] = f2_fma(f2_pack(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1])), cf,
+                                      acc[32 * hb + i]);
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            acc[32 * hb + 16 + i] = f2_fma(f2_pack(__uint_as_float(r1[2 * i]), __uint_as_float(r1[2 * i + 1])),
+                                           cf, acc[32 * hb + 16 + i]);
     }
 }
 // The thread's 128 columns of C (row `row`, from column col0), in C's dtype;
@@ -868,7 +890,7 @@ __global__ void __launch_bounds__(NT_Q, 1) k_fp8_gemm_q(const __grid_constant__ 
                 const int buf = it & 1;
                 if (!(ok = bar_wait<1, false>(bar(P::B_TFULL + buf), (uint32_t)(it >> 1) & 1u, abort_flag, abort_addr))) break;
                 tc_fence_after();
-                promote_block(acc, tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN + 128 * h), cf);
+                promote_block_2x(acc, tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN + 128 * h), cf);
                 tc_fence_before();
                 bar_arrive(bar(P::B_TEMPTY + buf));
                 ++it;
@@ -886,6 +908,223 @@ __global__ void __launch_bounds__(NT_Q, 1) k_fp8_gemm_q(const __grid_constant__ 
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
+}
+
+// ---------------------------------------------------------------------------
+// The same product for activations already quantized, on CTA pairs: a
+// cluster of two CTAs (one per SM) computes a 256 x 256 tile of C with
+// tcgen05.mma.cta_group::2 (M 256, N 256, K 32). CTA r of the pair loads
+// activation rows [128 r, 128 r + 128) and weight rows [128 r, 128 r + 128)
+// of the tile into its own shared memory; the MMA, issued by CTA 0, reads A
+// split by rows and B split by columns across the pair and writes each
+// CTA's 128 rows x 256 columns of the k-block's partial into that CTA's
+// TMEM. Per k-block and SM, shared memory then takes 32 KB of TMA writes and
+// serves 32 KB of operand reads (the one-CTA form: 48 KB and 48 KB), L2
+// serves a third less, and one MMA instruction carries twice the work, so
+// the issuing thread's per-block overhead is spread over twice the FLOPs.
+// (Issuing each block as two N = 128 halves into four TMEM quarters, to give
+// the promotion more slack, measured 23 % slower: twice the instructions and
+// activation reads.)
+// Roles (384 threads in each CTA):
+//   warp 0       TMA: both operand tiles of the k-block into one ring stage;
+//                the copies of both CTAs complete on the stage's barrier in
+//                CTA 0, whose producer expects the pair's 64 KB;
+//   warp 2       TMEM allocation for the pair (512 columns in each CTA); in
+//                CTA 0 one thread issues the MMAs and commits each k-block to
+//                the barriers of both CTAs (ring stage free, partial ready);
+//   warps 4-11   promotion as in k_fp8_gemm_q, for this CTA's 128 rows;
+//                each warp frees a TMEM buffer with one arrival on CTA 0's
+//                barrier (16 per k-block).
+struct PlanQ2 {
+    static constexpr int S = 6;
+    static constexpr uint32_t HALF = 128 * BK;                   // 128 rows x 128 bytes
+    static constexpr uint32_t STAGE = 2 * HALF;                  // A half, then B half
+    static constexpr uint32_t PAIR_TX = 2 * STAGE;               // both CTAs' bytes
+    static constexpr uint32_t OFF_RING = 0;
+    static constexpr uint32_t OFF_BAR = OFF_RING + S * STAGE;
+    static constexpr int B_FULL = 0, B_EMPTY = B_FULL + S, B_TFULL = B_EMPTY + S, B_TEMPTY = B_TFULL + 2,
+                         B_MMA_DONE = B_TEMPTY + 2, N_BAR = B_MMA_DONE + 1;
+    static constexpr uint32_t OFF_MISC = OFF_BAR + N_BAR * 8;   // [0] TMEM base, [1] abort flag
+    static constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+    static_assert(PAIR_TX < (1u << 20), "transaction count range");
+};
+// f32 accumulator, E4M3 x E4M3, both K-major, N 256, M 256 (the pair).
+constexpr uint32_t kIdescPair = (1u << 4) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t cols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(dst_smem), "r"(cols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t cols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" :: "r"(taddr), "r"(cols) : "memory");
+}
+__device__ __forceinline__ void mma_f8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+                 :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+// One arrival on the barrier at the same offset in both CTAs of the pair
+// when the pair's MMAs issued before by this thread have completed.
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+                 :: "r"(bar), "h"((uint16_t)3) : "memory");
+}
+// Tiled TMA load into this CTA's shared memory whose completion is counted on
+// an mbarrier of either CTA of the pair (`cl_bar`, a cluster address).
+__device__ __forceinline__ void tma_2d_pair(uint32_t dst, const CUtensorMap* tm, int x, int y, uint32_t cl_bar) {
+    asm volatile("cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                 " [%0], [%1, {%2, %3}], [%4];"
+                 :: "r"(dst), "l"((uint64_t)tm), "r"(x), "r"(y), "r"(cl_bar) : "memory");
+}
+// Bounded pause (about `us` microseconds).
+__device__ __forceinline__ void pause_us(uint32_t us) {
+    for (uint32_t i = 0; i < us; ++i) __nanosleep(1000);
+}
+
+__global__ void __launch_bounds__(NT_Q, 1) k_fp8_gemm_q2(const __grid_constant__ CUtensorMap tm_a,
+                                                          const __grid_constant__ CUtensorMap tm_w,
+                                                          const GemmArgs g) {
+    using P = PlanQ2;
+    constexpr int S = P::S;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = sm_addr(smem_raw);
+    const uint32_t base = (raw_base + 1023u) & ~1023u;
+    uint8_t* sb = smem_raw + (base - raw_base);
+    volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(sb + P::OFF_MISC);
+    volatile uint32_t* abort_flag = misc + 1;
+    const uint32_t abort_addr = base + P::OFF_MISC + 4;
+    auto bar = [&](int i) -> uint32_t { return base + P::OFF_BAR + 8u * (uint32_t)i; };
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < S; ++i) { bar_init(bar(P::B_FULL + i), 1); bar_init(bar(P::B_EMPTY + i), 1); }
+        for (int i = 0; i < 2; ++i) { bar_init(bar(P::B_TFULL + i), 1); bar_init(bar(P::B_TEMPTY + i), 16); }
+        bar_init(bar(P::B_MMA_DONE), 1);
+        misc[1] = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0 && lane == 0) { prefetch_map(&tm_a); prefetch_map(&tm_w); }
+    if (warp == 2) tmem_alloc_pair(base + P::OFF_MISC, TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();                                   // both CTAs' barriers initialised
+    tc_fence_after();
+    const uint32_t tmem = misc[0];
+    const int nkb = g.nkb;
+    const int64_t cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+
+    if (warp < 4) {
+        set_max_regs_dec<REGQ_CTL>();
+        if (warp == 0 && lane == 0) {
+            // Both operand halves of this CTA, completing on CTA 0's stage barrier.
+            int i = 0;
+            bool ok = true;
+            for (int64_t u = cid; ok && u < g.n_ctiles; u += ncl) {
+                int mt, nt;
+                ctile_coords(g, u, mt, nt);
+                for (int kb = 0; kb < nkb; ++kb) {
+                    const int s = i % S;
+                    if (!(ok = bar_wait<2, true>(bar(P::B_EMPTY + s), ((uint32_t)(i / S) & 1u) ^ 1u, abort_flag, abort_addr))) break;
+                    const uint32_t fb = bar(P::B_FULL + s);
+                    if (leader) bar_expect_tx(fb, P::PAIR_TX);
+                    const uint32_t cl_fb = map_rank(fb, 0u);
+                    const uint32_t dst = base + P::OFF_RING + (uint32_t)s * P::STAGE;
+                    tma_2d_pair(dst, &tm_a, kb * BK, mt * 256 + (int)rank * 128, cl_fb);
+                    tma_2d_pair(dst + P::HALF, &tm_w, kb * BK, nt * 256 + (int)rank * 128, cl_fb);
+                    ++i;
+                }
+            }
+        } else if (warp == 2 && lane == 0) {
+            if (leader) {
+                // MMA issue for the pair.
+                int i = 0, it = 0;
+                bool ok = true;
+                for (int64_t u = cid; ok && u < g.n_ctiles; u += ncl) {
+                    for (int kb = 0; kb < nkb; ++kb) {
+                        const int buf = it & 1;
+                        if (!(ok = bar_wait<2, true>(bar(P::B_TEMPTY + buf), ((uint32_t)(it >> 1) & 1u) ^ 1u, abort_flag, abort_addr))) break;
+                        const int s = i % S;
+                        if (!(ok = bar_wait<2, true>(bar(P::B_FULL + s), (uint32_t)(i / S) & 1u, abort_flag, abort_addr))) break;
+                        tc_fence_after();
+                        const uint32_t st = base + P::OFF_RING + (uint32_t)s * P::STAGE;
+                        const uint64_t da = desc_k_sw128(st);
+                        const uint64_t dw = desc_k_sw128(st + P::HALF);
+                        const uint32_t d = tmem + (uint32_t)(buf * BN);
+#pragma unroll
+                        for (int k4 = 0; k4 < BK / 32; ++k4)
+                            mma_f8_pair(d, da + (uint64_t)(2 * k4), dw + (uint64_t)(2 * k4), kIdescPair, k4 > 0 ? 1u : 0u);
+                        mma_commit_pair(bar(P::B_TFULL + buf));
+                        mma_commit_pair(bar(P::B_EMPTY + s));
+                        ++i; ++it;
+                    }
+                }
+                mma_commit_pair(bar(P::B_MMA_DONE));
+            }
+            // Both CTAs: the pair's MMAs (which write this CTA's TMEM) are done.
+            bar_drain(bar(P::B_MMA_DONE), 0u);
+        }
+    } else {
+        // ---------------------------------------------------- promotion
+        set_max_regs_inc<REGQ_ACC>();
+        const int q = warp & 3, h = (warp - 4) >> 2;
+        const int rloc = 32 * q + lane;
+        const uint32_t tempty0 = map_rank(bar(P::B_TEMPTY), 0u);
+        int it = 0;
+        bool ok = true;
+        F2 acc[64];
+        for (int64_t u = cid; ok && u < g.n_ctiles; u += ncl) {
+            int mt, nt;
+            ctile_coords(g, u, mt, nt);
+#pragma unroll
+            for (int i = 0; i < 64; ++i) acc[i] = 0ull;
+            const int64_t col0 = (int64_t)nt * BN + 128 * h;
+            const bool half_in = col0 < g.n;
+            const int64_t row = (int64_t)mt * 256 + (int64_t)rank * 128 + rloc;
+            const bool row_in = row < g.m;
+            const float* swp = g.sw + (half_in ? (col0 / 128) * nkb : 0);
+            const float* sap = g.sa + (row_in ? row * nkb : 0);
+            float sw0 = half_in ? __ldg(swp) : 0.0f, sa0 = row_in ? __ldg(sap) : 0.0f;
+            float sw1 = (half_in && nkb > 1) ? __ldg(swp + 1) : 0.0f;
+            float sa1 = (row_in && nkb > 1) ? __ldg(sap + 1) : 0.0f;
+            for (int kb = 0; kb < nkb; ++kb) {
+                const bool more = kb + 2 < nkb;
+                const float sw2 = (half_in && more) ? __ldg(swp + kb + 2) : 0.0f;
+                const float sa2 = (row_in && more) ? __ldg(sap + kb + 2) : 0.0f;
+                const F2 cf = f2_bcast(__fmul_rn(sa0, sw0));
+                const int buf = it & 1;
+                if (!(ok = bar_wait<2, true>(bar(P::B_TFULL + buf), (uint32_t)(it >> 1) & 1u, abort_flag, abort_addr))) break;
+                tc_fence_after();
+                promote_block_2x(acc, tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN + 128 * h), cf);
+                tc_fence_before();
+                __syncwarp();
+                // The warp's TMEM reads have completed (tcgen05.wait::ld): the
+                // arrival only has to follow them, so it needs no release (a
+                // release at cluster scope would also wait for the scale loads
+                // issued above for later blocks: measured 2x slower).
+                if (lane == 0) {
+                    if (leader) bar_arrive(bar(P::B_TEMPTY + buf));
+                    else bar_arrive_remote_relaxed(tempty0 + 8u * (uint32_t)buf);
+                }
+                ++it;
+                sw0 = sw1; sw1 = sw2;
+                sa0 = sa1; sa1 = sa2;
+            }
+            if (!ok) break;
+            if (row_in && half_in) store_c_half(g, row, col0, acc);
+        }
+    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();                                   // no TMEM access or remote arrival left in the pair
+    tc_fence_after();
+    if (warp == 2) tmem_dealloc_pair(tmem, TMEM_COLS);
 }
 
 cudaError_t encode_map(CUtensorMap* tm, CUtensorMapDataType dt, const void* p, uint64_t inner,
@@ -1037,6 +1276,65 @@ cudaError_t launch_gemm_q(const uint8_t* ea, const float* sa, int64_t m, int64_t
     return cudaGetLastError();
 }
 
+cudaError_t launch_gemm_q2(const uint8_t* ea, const float* sa, int64_t m, int64_t k, const uint8_t* w,
+                           const float* sw, int64_t n, void* c, int c_bf16, cudaStream_t st) {
+    static int ready[64] = {0};
+    static int pairs[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorUnknown;
+    if (dev < 0 || dev >= 64) return cudaErrorNotSupported;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(NT_Q);
+    cfg.dynamicSmemBytes = PlanQ2::SMEM_BYTES;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (!__atomic_load_n(&ready[dev], __ATOMIC_ACQUIRE)) {
+        cudaFuncAttributes fa;
+        cudaError_t e = cudaFuncGetAttributes(&fa, k_fp8_gemm_q2);
+        if (e != cudaSuccess) return e;
+        if (fa.numRegs != REGQ_LAUNCH) return cudaErrorNotSupported;
+        e = cudaFuncSetAttribute(k_fp8_gemm_q2, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)PlanQ2::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        cfg.gridDim = dim3((unsigned)(sm_count() & ~1));
+        int cnum = 0;
+        e = cudaOccupancyMaxActiveClusters(&cnum, k_fp8_gemm_q2, &cfg);
+        if (e != cudaSuccess) return e;
+        if (cnum < 1) return cudaErrorNotSupported;
+        pairs[dev] = cnum;
+        __atomic_store_n(&ready[dev], 1, __ATOMIC_RELEASE);
+    }
+    CUtensorMap ta, tw;
+    cudaError_t e;
+    if ((e = encode_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, ea, (uint64_t)k, (uint64_t)m, (uint64_t)k, BK, 128)) !=
+        cudaSuccess)
+        return e;
+    if ((e = encode_map(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, (uint64_t)k, (uint64_t)n, (uint64_t)k, BK, 128)) !=
+        cudaSuccess)
+        return e;
+    GemmArgs g = {};
+    g.m = m; g.n = n; g.k = k;
+    g.nkb = (int)(k / BK);
+    g.mtiles = (int)((m + 255) / 256);             // pair tiles of 256 rows
+    g.ntiles = (int)((n + BN - 1) / BN);
+    g.nct = g.ntiles;
+    g.band = min(16, g.mtiles);
+    g.n_ctiles = (int64_t)g.mtiles * g.nct;
+    g.sw = sw; g.c = c; g.c_bf16 = c_bf16; g.sa = sa;
+    int64_t np = pairs[dev];
+    if (np > g.n_ctiles) np = g.n_ctiles;
+    cfg.gridDim = dim3((unsigned)(2 * np));
+    cfg.stream = st;
+    e = cudaLaunchKernelEx(&cfg, k_fp8_gemm_q2, ta, tw, g);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
 // Cluster size: activations are quantized once per cluster of CL CTAs that
 // share them; CL = 4 when the tile row holds at least four N tiles.
 template <class T>
@@ -1052,6 +1350,19 @@ cudaError_t launch_gemm_any(const void* a, int64_t m, int64_t k, const uint8_t* 
 }
 
 }  // namespace
+
+// Kernel for bq_fp8_block_gemm_quantized: BQ_GEMM_PAIR = 0 forces the
+// one-CTA kernel, 1 the CTA-pair kernel (for measurement); otherwise the
+// pair kernel takes every m above 128.
+int gemm_pair_override() {
+    static const int v = [] {
+        const char* e = getenv("BQ_GEMM_PAIR");
+        if (!e) return -1;
+        const int x = atoi(e);
+        return (x == 0 || x == 1) ? x : -1;
+    }();
+    return v;
+}
 
 // Cluster size for bq_fp8_block_gemm: BQ_GEMM_CLUSTER = 1, 2 or 4 forces one
 // (for measurement); unset or anything else lets the shape decide.
@@ -1110,8 +1421,11 @@ extern "C" bq_status bq_fp8_block_gemm_quantized(const uint8_t* a_e4m3, const fl
     if (((uintptr_t)a_e4m3 & 15u) || ((uintptr_t)w_e4m3 & 15u) || ((uintptr_t)w_scale & 3u) ||
         ((uintptr_t)a_scale & 3u) || ((uintptr_t)c & 15u))
         return BQ_ERR_MISALIGNED;
-    const cudaError_t e = bq::launch_gemm_q(a_e4m3, a_scale, m, k, w_e4m3, w_scale, n, c, c_dtype == BQ_BF16,
-                                            (cudaStream_t)stream);
+    const int pair = bq::gemm_pair_override();
+    const bool use_pair = pair < 0 ? m > 128 : pair == 1;
+    const cudaError_t e = use_pair
+        ? bq::launch_gemm_q2(a_e4m3, a_scale, m, k, w_e4m3, w_scale, n, c, c_dtype == BQ_BF16, (cudaStream_t)stream)
+        : bq::launch_gemm_q(a_e4m3, a_scale, m, k, w_e4m3, w_scale, n, c, c_dtype == BQ_BF16, (cudaStream_t)stream);
     if (e == cudaErrorNotSupported) return BQ_ERR_UNSUPPORTED;
     return e == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }

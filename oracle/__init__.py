@@ -350,6 +350,19 @@ def fp8_block_gemm(a: torch.Tensor, ew: torch.Tensor, sw: torch.Tensor):
     return c, ea, sa
 
 
+def fp8_block_gemm_codes(ea: torch.Tensor, sa: torch.Tensor, ew: torch.Tensor, sw: torch.Tensor):
+    """The same product for activations already quantized: E4M3 codes ea
+    [m, k] with f32 scales sa [m, ceil(k/128)]. Returns C f64 [m, n]."""
+    m, k = ea.shape
+    n = ew.shape[0]
+    assert tuple(ew.shape) == (n, k) and tuple(sa.shape) == (m, (k + 127) // 128)
+    assert tuple(sw.shape) == ((n + 127) // 128, (k + 127) // 128)
+    c = torch.zeros((m, n), dtype=torch.float64)
+    _ok(lib().or_fp8_block_gemm_codes(_p(_c(ea)), _p(_c(sa)), _p(_c(ew)), _p(_c(sw)), C.c_int64(m),
+                                      C.c_int64(n), C.c_int64(k), _p(c)), "fp8_block_gemm_codes")
+    return c
+
+
 def align_up(n: int, align: int) -> int:
     return int(lib().or_align_up(n, align))
 

@@ -810,14 +810,12 @@ int or_fp8_block_dequantize(const uint8_t* e4m3, const float* scale, int64_t row
 // blocks round in binary64. The pages fix no output precision: C is returned
 // in binary64 (a tensor-core f32 accumulation is compared with it within a
 // bound). ea / sa, when given, receive the activation codes and scales.
-int or_fp8_block_gemm(const void* a, int a_t, const uint8_t* ew, const float* sw, int64_t m,
-                      int64_t n, int64_t k, double* c, uint8_t* ea_out, float* sa_out) {
-    if (a_t != OR_F32 && a_t != OR_F16 && a_t != OR_BF16) return 1;
+// The product alone, for activations already quantized: ea [m, k] E4M3 codes
+// with sa [m, ceil(k/128)] scales.
+int or_fp8_block_gemm_codes(const uint8_t* ea, const float* sa, const uint8_t* ew, const float* sw,
+                            int64_t m, int64_t n, int64_t k, double* c) {
     if (m < 0 || n < 0 || k < 0) return 1;
     const int64_t nkb = (k + 127) / 128;
-    std::vector<uint8_t> ea((size_t)(m * k));
-    std::vector<float> sa((size_t)(m * nkb));
-    if (or_fp8_block_quantize(a, a_t, m, k, 1, 128, ea.data(), sa.data()) != 0) return 1;
     for (int64_t i = 0; i < m; ++i)
         for (int64_t j = 0; j < n; ++j) {
             double acc = 0.0;
@@ -829,6 +827,18 @@ int or_fp8_block_gemm(const void* a, int a_t, const uint8_t* ew, const float* sw
             }
             c[i * n + j] = acc;
         }
+    return 0;
+}
+
+int or_fp8_block_gemm(const void* a, int a_t, const uint8_t* ew, const float* sw, int64_t m,
+                      int64_t n, int64_t k, double* c, uint8_t* ea_out, float* sa_out) {
+    if (a_t != OR_F32 && a_t != OR_F16 && a_t != OR_BF16) return 1;
+    if (m < 0 || n < 0 || k < 0) return 1;
+    const int64_t nkb = (k + 127) / 128;
+    std::vector<uint8_t> ea((size_t)(m * k));
+    std::vector<float> sa((size_t)(m * nkb));
+    if (or_fp8_block_quantize(a, a_t, m, k, 1, 128, ea.data(), sa.data()) != 0) return 1;
+    if (or_fp8_block_gemm_codes(ea.data(), sa.data(), ew, sw, m, n, k, c) != 0) return 1;
     if (ea_out) std::copy(ea.begin(), ea.end(), ea_out);
     if (sa_out) std::copy(sa.begin(), sa.end(), sa_out);
     return 0;

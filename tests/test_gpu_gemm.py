@@ -110,11 +110,15 @@ def test_gemm_parity(bq, orc, a_dtype, c_dtype, m, n, k):
 
 
 @pytest.mark.parametrize("c_dtype", [torch.float32, torch.bfloat16])
-@pytest.mark.parametrize("m,n,k", [(1, 16, 128), (300, 520, 512), (257, 384, 1024), (64, 1000, 384)])
+@pytest.mark.parametrize("m,n,k", [(1, 16, 128), (64, 1000, 384), (128, 1536, 256),
+                                   (129, 256, 128), (300, 520, 512), (257, 384, 1024)])
 def test_gemm_quantized_parity(bq, orc, c_dtype, m, n, k):
     """Activations given as 1x128 codes and scales (the oracle's own): C
     within the bound, and bit-identical to the fused kernel's C (same
-    operands, same block sums, same promotion order)."""
+    operands, same block sums, same promotion order). m <= 128 runs the
+    one-CTA kernel, larger m the CTA-pair kernel (256 x 256 tiles: with
+    m = 129 or 300 the second CTA of a pair, with n = 520 the weight half of
+    the second CTA, lie wholly or partly past the matrix)."""
     st = synthetic.Stream(3000 + m + n + k)
     a = st.tensor((m, k), "bf16", outlier_p=0.01, outlier_factor=30.0)
     ew, sw = _weights_from_oracle(orc, n, k, 4000 + n + k)
@@ -125,6 +129,21 @@ def test_gemm_quantized_parity(bq, orc, c_dtype, m, n, k):
     _check_c(orc, c, c_ref, ea, sa, ew, sw, f"C quantized {m}x{n}x{k}")
     c_fused = bq.api.fp8_block_gemm(a.cuda(), ew.cuda(), sw.cuda(), out_dtype=c_dtype)
     assert_bitwise(c, c_fused, "quantized-activation GEMM vs fused prologue")
+
+
+def test_gemm_quantized_many_tiles_per_pair(bq, orc):
+    # 8 x 16 = 128 pair tiles of 256 x 256 (more than the 74 pairs that fit):
+    # pairs walk several tiles through the same ring and TMEM buffers.
+    m, n, k = 2048, 4096, 1024
+    st = synthetic.Stream(502)
+    ea = st.codes8((m, k))
+    sa = st.uniform_f32((m, k // 128), 2.0 ** -10, 2.0 ** -6)
+    ew = st.codes8((n, k))
+    sw = st.uniform_f32((n // 128, k // 128), 2.0 ** -12, 2.0 ** -8)
+    c = bq.api.fp8_block_gemm_quantized(ea.cuda(), sa.cuda(), ew.cuda(), sw.cuda(), out_dtype=torch.float32)
+    rows = torch.tensor([0, 127, 128, 255, 256, 700, 1023, 1024, 1151, 1280, 1919, 2047])
+    c_ref = orc.fp8_block_gemm_codes(ea[rows].contiguous(), sa[rows].contiguous(), ew, sw)
+    _check_c(orc, cpu(c)[rows], c_ref, ea[rows], sa[rows], ew, sw, "quantized, many tiles per pair")
 
 
 def test_gemm_special_rows(bq, orc):

@@ -83,3 +83,27 @@ def test_rows_are_independent(orc):
     for i in (0, 3, 6):
         ci, _, _ = orc.fp8_block_gemm(a[i:i + 1].clone(), ew, sw)
         assert torch.equal(ci[0], c[i])
+
+
+@pytest.mark.parametrize("m,n,k", [(4, 130, 300), (2, 256, 128)])
+def test_codes_product_matches_numpy(orc, m, n, k):
+    # Activations given as arbitrary codes and scales (not from a quantizer).
+    rng = np.random.default_rng(m * 7 + n + k)
+    ea, _ = _weights(rng, m, k)
+    sa = torch.from_numpy(rng.uniform(1e-3, 4.0, size=(m, (k + 127) // 128)).astype(np.float32))
+    ew, sw = _weights(rng, n, k)
+    c = orc.fp8_block_gemm_codes(ea, sa, ew, sw)
+    kb = np.arange(k) // 128
+    a_deq = _dec(ea) * sa.numpy().astype(np.float64)[:, kb]
+    w_deq = _dec(ew) * sw.numpy().astype(np.float64)[(np.arange(n) // 128)[:, None], kb[None, :]]
+    ref = a_deq @ w_deq.T
+    bound = 2.0 ** -40 * (np.abs(a_deq) @ np.abs(w_deq).T) + 1e-300
+    assert np.all(np.abs(c.numpy() - ref) <= bound)
+
+
+def test_codes_product_of_quantized_activations_is_the_fused_product(orc):
+    rng = np.random.default_rng(8)
+    a = synthetic.Stream(10).tensor((3, 384), "bf16", outlier_p=0.05, outlier_factor=20)
+    ew, sw = _weights(rng, 96, 384)
+    c, ea, sa = orc.fp8_block_gemm(a, ew, sw)
+    assert torch.equal(orc.fp8_block_gemm_codes(ea, sa, ew, sw), c)
