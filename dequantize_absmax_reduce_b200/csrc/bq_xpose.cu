@@ -54,18 +54,24 @@ __global__ void __launch_bounds__(256) k_xpose(const uint8_t* __restrict__ in, i
 }
 
 // Wide tiles for the common case (cols % 16 == 0, stride % 16 == 0, 16-byte
-// aligned buffers): a CTA moves a 64-row x 256-byte tile. Thread (rb, cb) =
-// (t % 16, t / 16) loads rows 4rb..4rb+3 at bytes 16cb..16cb+15 (four 16-byte
-// loads; a warp reads 32 full-sector bytes from each of 16 rows), transposes
-// the four 4x4 byte blocks in registers and parks sixteen output words in
-// shared memory (the 32 lanes of one store hit 32 distinct banks); the CTA
-// then writes each of the tile's 256 output rows as four 16-byte runs. Up to
-// XJOBS independent transposes share one launch (the weights and scales of
-// every part of a concatenation); job j owns blocks [first_j, first_j +
-// n_tiles_j). A job writes bytes [0, olim) of each output row from its base
-// `out` (a part's column offset into the shared rows); input rows beyond
-// `rows` read as zero, which fills the pad columns of the last part.
+// aligned buffers): a CTA of 128 threads moves a 64-row x 512-byte tile.
+// Warp w holds input rows 16w..16w+15 and lane l the 16 bytes 16l..16l+15 of
+// each (sixteen 16-byte loads; one load instruction reads 512 contiguous
+// bytes of one row). The lane's 16 x 16 byte block is transposed in
+// registers (sixteen 4 x 4 byte transposes by byte permutes) into sixteen
+// 16-byte pieces of output rows 16l..16l+15, stored to shared memory whole;
+// the CTA then writes each output row's 64 bytes as four 16-byte runs.
+// Shared memory holds the 512 output rows x 64 bytes as pairs of rows per
+// 128-byte line, the eight 16-byte slots of a line permuted by XOR with
+// bits 4-6 of the row: the eight lanes of a store phase (rows 16 apart) and
+// of a load phase (two rows of one line) then touch eight distinct slots.
+// Up to XJOBS independent transposes share one launch (the weights and
+// scales of every part of a concatenation); job j owns blocks [first_j,
+// first_j + n_tiles_j). A job writes bytes [0, olim) of each output row from
+// its base `out` (a part's column offset into the shared rows); input rows
+// beyond `rows` read as zero, which fills the pad columns of the last part.
 constexpr int XJOBS = 8;
+constexpr int XT_ROWS = 64, XT_COLS = 512, XT_THREADS = 128;
 struct XJob {
     const uint8_t* in;
     int64_t rows, cols, stride, olim, ntr, n_tiles, first;
@@ -76,8 +82,14 @@ struct XJobs {
     int n;
 };
 
-__global__ void __launch_bounds__(256) k_xpose_wide(XJobs jobs) {
-    __shared__ uint32_t sm[256][17];                  // [output row][input-row word], padded
+// Byte offset in the staging tile of output row `orow`, 16-byte piece `c`
+// (input rows 16c..16c+15 of the tile).
+__device__ __forceinline__ uint32_t xt_slot(int orow, int c) {
+    return (uint32_t)(orow >> 1) * 128u + 16u * (uint32_t)((c + 4 * (orow & 1)) ^ ((orow >> 4) & 7));
+}
+
+__global__ void __launch_bounds__(XT_THREADS) k_xpose_wide(XJobs jobs) {
+    __shared__ __align__(128) uint8_t sm[XT_COLS * XT_ROWS];
     int ji = 0;
 #pragma unroll 1
     for (int q = 1; q < jobs.n; ++q)
@@ -85,45 +97,51 @@ __global__ void __launch_bounds__(256) k_xpose_wide(XJobs jobs) {
     const XJob& J = jobs.j[ji];
     const int64_t b = (int64_t)blockIdx.x - J.first;
     const int64_t tr = b % J.ntr, tc = b / J.ntr;
-    const int64_t r0 = tr * 64, c0 = tc * 256;
-    const int t = threadIdx.x;
+    const int64_t r0 = tr * XT_ROWS, c0 = tc * XT_COLS;
+    const int t = threadIdx.x, lane = t & 31, rg = t >> 5;
+    const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(sm);
     {
-        const int rb = t & 15, cb = t >> 4;
-        const int64_t c = c0 + 16 * cb;
-        U4 w[4];
+        const int64_t c = c0 + 16 * lane;
+        U4 w[16];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int64_t r = r0 + 4 * rb + i;
+        for (int i = 0; i < 16; ++i) {
+            const int64_t r = r0 + 16 * rg + i;
             w[i] = (r < J.rows && c < J.cols) ? ld16_stream(J.in + r * J.cols + c) : U4{0u, 0u, 0u, 0u};
         }
-        const uint32_t x0[4] = {w[0].x, w[0].y, w[0].z, w[0].w};
-        const uint32_t x1[4] = {w[1].x, w[1].y, w[1].z, w[1].w};
-        const uint32_t x2[4] = {w[2].x, w[2].y, w[2].z, w[2].w};
-        const uint32_t x3[4] = {w[3].x, w[3].y, w[3].z, w[3].w};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            // 4x4 bytes: rows 4rb+i, columns 16cb+4q+j -> word j holds byte j of each row.
-            const uint32_t a_lo = __byte_perm(x0[q], x1[q], 0x5140), a_hi = __byte_perm(x0[q], x1[q], 0x7362);
-            const uint32_t b_lo = __byte_perm(x2[q], x3[q], 0x5140), b_hi = __byte_perm(x2[q], x3[q], 0x7362);
-            const int orow = 16 * cb + 4 * q;
-            sm[orow + 0][rb] = __byte_perm(a_lo, b_lo, 0x5410);
-            sm[orow + 1][rb] = __byte_perm(a_lo, b_lo, 0x7632);
-            sm[orow + 2][rb] = __byte_perm(a_hi, b_hi, 0x5410);
-            sm[orow + 3][rb] = __byte_perm(a_hi, b_hi, 0x7632);
+        for (int bb = 0; bb < 4; ++bb) {               // input bytes 4bb..4bb+3 of the lane's 16
+            uint32_t o[4][4];                          // [j][ib]: output row 4bb + j, input rows 4ib..4ib+3
+#pragma unroll
+            for (int ib = 0; ib < 4; ++ib) {
+                const uint32_t x0 = (&w[4 * ib + 0].x)[bb], x1 = (&w[4 * ib + 1].x)[bb];
+                const uint32_t x2 = (&w[4 * ib + 2].x)[bb], x3 = (&w[4 * ib + 3].x)[bb];
+                const uint32_t a_lo = __byte_perm(x0, x1, 0x5140), a_hi = __byte_perm(x0, x1, 0x7362);
+                const uint32_t b_lo = __byte_perm(x2, x3, 0x5140), b_hi = __byte_perm(x2, x3, 0x7362);
+                o[0][ib] = __byte_perm(a_lo, b_lo, 0x5410);
+                o[1][ib] = __byte_perm(a_lo, b_lo, 0x7632);
+                o[2][ib] = __byte_perm(a_hi, b_hi, 0x5410);
+                o[3][ib] = __byte_perm(a_hi, b_hi, 0x7632);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int orow = 16 * lane + 4 * bb + j;
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};"
+                             :: "r"(sbase + xt_slot(orow, rg)), "r"(o[j][0]), "r"(o[j][1]), "r"(o[j][2]),
+                                "r"(o[j][3]) : "memory");
+            }
         }
     }
     __syncthreads();
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int orow = 64 * k + (t >> 2), seg = t & 3;
+#pragma unroll 4
+    for (int k = 0; k < XT_COLS * XT_ROWS / 16 / XT_THREADS; ++k) {
+        const int idx = k * XT_THREADS + t;
+        const int orow = idx >> 2, seg = idx & 3;
         const int64_t oc = c0 + orow;                 // output row
         const int64_t ob = r0 + 16 * seg;             // output byte column
         if (oc < J.cols && ob < J.olim) {
             U4 v;
-            v.x = sm[orow][4 * seg + 0];
-            v.y = sm[orow][4 * seg + 1];
-            v.z = sm[orow][4 * seg + 2];
-            v.w = sm[orow][4 * seg + 3];
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(sbase + xt_slot(orow, seg)));
             st16(J.out + oc * J.stride + ob, v);
         }
     }
@@ -138,8 +156,8 @@ static XJob make_xjob(const uint8_t* in, int64_t rows, int64_t cols, int64_t str
                       uint8_t* out) {
     XJob j;
     j.in = in; j.rows = rows; j.cols = cols; j.stride = stride; j.olim = olim; j.out = out;
-    j.ntr = (olim + 63) / 64;
-    j.n_tiles = j.ntr * ((cols + 255) / 256);
+    j.ntr = (olim + XT_ROWS - 1) / XT_ROWS;
+    j.n_tiles = j.ntr * ((cols + XT_COLS - 1) / XT_COLS);
     if (cols == 0 || olim == 0) j.n_tiles = 0;
     j.first = 0;
     return j;
@@ -213,7 +231,7 @@ cudaError_t byte_transpose_parts(const XPart* parts, int n_parts, int64_t stride
             }
             if (nb == 0) continue;
             if (nb > 0x7FFFFFFFll) return cudaErrorInvalidValue;
-            k_xpose_wide<<<(unsigned)nb, 256, 0, st>>>(jobs);
+            k_xpose_wide<<<(unsigned)nb, XT_THREADS, 0, st>>>(jobs);
             const cudaError_t e = cudaGetLastError();
             if (e != cudaSuccess) return e;
         }
