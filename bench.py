@@ -45,6 +45,13 @@ FLUSH_BYTES = 256 << 20
 # DRAM bytes (read + write) per launch from one ncu capture of each kernel on
 # the workload above, with the sha256 of the kernel sources it was taken on;
 # reported as null once the sources change.
+# The sources hashed: every file the step's kernels and their host dispatch
+# are compiled from (the include closure of the bf16 pipeline translation
+# unit and of the dispatch units, from nvcc -M), so that edits to unrelated
+# kernels (GEMM, transpose, column groups, ...) leave the figures valid.
+TRAFFIC_SOURCES = ("bq_abi.cu", "bq_int.cu", "bq_pipe.cu", "bq_pipe_bf16.cu", "bq_pipe_impl.cuh",
+                   "bq_pipe_args.h", "bq_device.cuh", "bq_internal.h", "bq_map_ops.cuh",
+                   "bq_quant_ops.cuh", "bq_range.cuh")
 NCU_TRAFFIC = {
     "quantize_per_token": {"src_sha256": "771710426153cdec45e8e95d1a636ac540d766f27a13b288289f50f623f0bed2", "bytes_per_launch": 70402048},
     "dequantize_per_token": {"src_sha256": "771710426153cdec45e8e95d1a636ac540d766f27a13b288289f50f623f0bed2", "bytes_per_launch": 38783744},
@@ -55,9 +62,10 @@ NCU_TRAFFIC = {
 def _kernel_source_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "dequantize_absmax_reduce_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode())
+    paths = [os.path.join(csrc, n) for n in sorted(TRAFFIC_SOURCES)] + [os.path.join(ROOT, "include", "bq.h")]
+    for path in paths:
+        with open(path, "rb") as f:
+            h.update(os.path.basename(path).encode())
             h.update(f.read())
     return h.hexdigest()
 
