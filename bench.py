@@ -53,9 +53,9 @@ TRAFFIC_SOURCES = ("bq_abi.cu", "bq_int.cu", "bq_pipe.cu", "bq_pipe_bf16.cu", "b
                    "bq_pipe_args.h", "bq_device.cuh", "bq_internal.h", "bq_map_ops.cuh",
                    "bq_quant_ops.cuh", "bq_range.cuh")
 NCU_TRAFFIC = {
-    "quantize_per_token": {"src_sha256": "771710426153cdec45e8e95d1a636ac540d766f27a13b288289f50f623f0bed2", "bytes_per_launch": 70402048},
-    "dequantize_per_token": {"src_sha256": "771710426153cdec45e8e95d1a636ac540d766f27a13b288289f50f623f0bed2", "bytes_per_launch": 38783744},
-    "quantize_per_token_backward": {"src_sha256": "771710426153cdec45e8e95d1a636ac540d766f27a13b288289f50f623f0bed2", "bytes_per_launch": 159154432},
+    "quantize_per_token": {"src_sha256": "59cf6d1666d435e466ad225b69d990414f1b93108845f50c8fd3d321ee0686a6", "bytes_per_launch": 71384320},
+    "dequantize_per_token": {"src_sha256": "59cf6d1666d435e466ad225b69d990414f1b93108845f50c8fd3d321ee0686a6", "bytes_per_launch": 39869952},
+    "quantize_per_token_backward": {"src_sha256": "59cf6d1666d435e466ad225b69d990414f1b93108845f50c8fd3d321ee0686a6", "bytes_per_launch": 159439360},
 }
 
 
