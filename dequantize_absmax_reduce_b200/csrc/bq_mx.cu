@@ -545,11 +545,31 @@ struct CopySegs {
 
 __global__ void __launch_bounds__(256) k_copy_segs(CopySegs c) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < c.nvec; i += stride) {
+    // Four 16-byte vectors per thread and step, all four loads issued before
+    // any store, so that one step keeps four times the bytes in flight.
+    constexpr int U = 4;
+    auto seg_of = [&](int64_t i) {
         int q = 0;
         while (q + 1 < c.n && i >= c.s[q + 1].vfirst) ++q;
-        const int64_t v = i - c.s[q].vfirst;
-        st16(c.s[q].dst + v * 16, ld16_stream(c.s[q].src + v * 16));
+        return q;
+    };
+    for (int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i0 < c.nvec; i0 += U * stride) {
+        U4 v[U];
+        int qs[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = i0 + u * stride;
+            qs[u] = 0;
+            if (i < c.nvec) {
+                qs[u] = seg_of(i);
+                v[u] = ld16_stream(c.s[qs[u]].src + (i - c.s[qs[u]].vfirst) * 16);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = i0 + u * stride;
+            if (i < c.nvec) st16(c.s[qs[u]].dst + (i - c.s[qs[u]].vfirst) * 16, v[u]);
+        }
     }
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < c.nbytes; i += stride) {
         int q = 0;
