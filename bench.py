@@ -44,7 +44,7 @@ FLUSH_BYTES = 256 << 20
 
 # DRAM bytes (read + write) per launch from one ncu capture of each kernel on
 # the workload above, with the sha256 of the kernel sources it was taken on;
-# reported as null once the sources change.
+# reported as null once the sources change (comments excluded).
 # The sources hashed: every file the step's kernels and their host dispatch
 # are compiled from (the include closure of the bf16 pipeline translation
 # unit and of the dispatch units, from nvcc -M), so that edits to unrelated
@@ -53,10 +53,34 @@ TRAFFIC_SOURCES = ("bq_abi.cu", "bq_int.cu", "bq_pipe.cu", "bq_pipe_bf16.cu", "b
                    "bq_pipe_args.h", "bq_device.cuh", "bq_internal.h", "bq_map_ops.cuh",
                    "bq_quant_ops.cuh", "bq_range.cuh")
 NCU_TRAFFIC = {
-    "quantize_per_token": {"src_sha256": "59cf6d1666d435e466ad225b69d990414f1b93108845f50c8fd3d321ee0686a6", "bytes_per_launch": 71384320},
-    "dequantize_per_token": {"src_sha256": "59cf6d1666d435e466ad225b69d990414f1b93108845f50c8fd3d321ee0686a6", "bytes_per_launch": 39869952},
-    "quantize_per_token_backward": {"src_sha256": "59cf6d1666d435e466ad225b69d990414f1b93108845f50c8fd3d321ee0686a6", "bytes_per_launch": 159439360},
+    "quantize_per_token": {"src_sha256": "d96cb38586416c7132f23bb2b1660feb113243a94fe0c3128fea3b6a7172a5f7", "bytes_per_launch": 71384320},
+    "dequantize_per_token": {"src_sha256": "d96cb38586416c7132f23bb2b1660feb113243a94fe0c3128fea3b6a7172a5f7", "bytes_per_launch": 39869952},
+    "quantize_per_token_backward": {"src_sha256": "d96cb38586416c7132f23bb2b1660feb113243a94fe0c3128fea3b6a7172a5f7", "bytes_per_launch": 159439360},
 }
+
+
+def _strip_comments(src: str) -> str:
+    """C / C++ source without its comments (string and character literals
+    kept), so that comment edits leave the hash unchanged."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return "".join(out)
 
 
 def _kernel_source_hash() -> str:
@@ -64,9 +88,9 @@ def _kernel_source_hash() -> str:
     csrc = os.path.join(ROOT, "dequantize_absmax_reduce_b200", "csrc")
     paths = [os.path.join(csrc, n) for n in sorted(TRAFFIC_SOURCES)] + [os.path.join(ROOT, "include", "bq.h")]
     for path in paths:
-        with open(path, "rb") as f:
+        with open(path, encoding="utf-8") as f:
             h.update(os.path.basename(path).encode())
-            h.update(f.read())
+            h.update(_strip_comments(f.read()).encode())
     return h.hexdigest()
 
 

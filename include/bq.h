@@ -463,7 +463,12 @@ bq_status bq_fp8_block_gemm(const void* a, bq_dtype a_dtype, int64_t m, int64_t 
  * activations that several weights multiply, and for large n, quantizing
  * once (bq_fp8_block_quantize) and calling this entry is cheaper than the
  * fused prologue, which requantizes a tile row for every group of N tiles.
- * One launch of a persistent kernel (one CTA per SM, TMA, tcgen05). */
+ * One launch of a persistent kernel: for m > 128, clusters of two CTAs (one
+ * per SM) that compute 256 x 256 tiles with tcgen05.mma.cta_group::2; for
+ * m <= 128, one CTA per SM and 128 x 256 tiles (both sum each k-block in
+ * the same order, and the tests find the same C bits from both and from
+ * bq_fp8_block_gemm). The environment variable BQ_GEMM_PAIR (read once per
+ * process) = 0 or 1 forces one of them, for measurement. */
 bq_status bq_fp8_block_gemm_quantized(const uint8_t* a_e4m3, const float* a_scale, int64_t m, int64_t k,
                                       const uint8_t* w_e4m3, const float* w_scale, int64_t n, void* c,
                                       bq_dtype c_dtype, void* stream);
