@@ -63,6 +63,7 @@ _SIGS = {
     "bq_tensor_amax": [_P, C.c_int, _I64, _P, _P, _P],
     "bq_diag_wait_timeout": [C.c_uint32, _P],
     "bq_diag_encode_f32": [_P, _I64, C.c_int, _P, _P],
+    "bq_diag_divide_f32": [_P, _I64, C.c_float, C.c_int, _P, _P],
     "bq_quantize_per_tensor": [_P, _DESC, _P, _P, _P, C.c_int, _P, _SZ, _P],
     "bq_quantize_per_channel": [_P, _DESC, _I32, _P, _P, _P, C.c_int, _P, _SZ, _P],
     "bq_quantize_per_token": [_P, _DESC, _P, _P, _P, C.c_int, _P, _SZ, _P],
@@ -227,6 +228,13 @@ def bq_diag_encode_f32(x, fmt, out, stream=None):
     enum values); out: device buffer of n, n/2 or 2n bytes."""
     _check(lib.bq_diag_encode_f32(_ptr(x), x.numel(), int(fmt), _ptr(out), _stream(stream)),
            "bq_diag_encode_f32")
+
+
+def bq_diag_divide_f32(x, s, chain, out, stream=None):
+    """out = x / s (f32 device tensors of even length) through the kernels'
+    reciprocal chain: chain 0 five roundings, 1 four (two-term reciprocal)."""
+    _check(lib.bq_diag_divide_f32(_ptr(x), x.numel(), float(s), int(chain), _ptr(out), _stream(stream)),
+           "bq_diag_divide_f32")
 
 
 def bq_tensor_amax(x, amax, ws, stream=None):

@@ -289,18 +289,36 @@ __device__ __forceinline__ void widen_pairs(const U4& u, F2 (&x)[Traits<T>::VEC 
 struct Recip2 {
     F2 y, ns;   // (RN(1/s), RN(1/s)), (-s, -s)
 };
-__device__ __forceinline__ Recip2 make_recip2(const Recip& r) {
-    Recip2 p;
-    p.y = f2_bcast(r.y);
-    p.ns = f2_bcast(-r.s);
-    return p;
-}
 __device__ __forceinline__ F2 div_chain2(F2 x, const Recip2& r) {
     const F2 q0 = f2_mul(x, r.y);
     const F2 e0 = f2_fma(r.ns, q0, x);
     const F2 q1 = f2_fma(e0, r.y, q0);
     const F2 e1 = f2_fma(r.ns, q1, x);
     return f2_fma(e1, r.y, q1);
+}
+// fl(x / s) on pairs in four roundings, from a two-term reciprocal: with
+// y = RN(1/s), the residual e = 1 - s*y is exact in an FMA and
+// 1/s = y (1 + e + e^2 + ...), |e| <= 2^-23, so y + ylo, ylo = RN(e * y),
+// is 1/s to a relative 2^-45. Then q0 = RN(x*y + RN(x*ylo)) (one FMA) lies
+// within 2^-44 |x/s| + half an ulp of x/s, i.e. within one ulp, and one
+// remainder correction RN(q0 + (x - s*q0) * y) is RN(x/s) (Markstein's
+// theorem, the hypotheses of div_chain's last step; the remainder is exact
+// in an FMA). Same domain as div_chain: Recip::fast and no overflow.
+struct Recip2T {
+    F2 y, ylo, ns;   // RN(1/s), RN((1 - s*y) * y), -s, on both lanes
+};
+__device__ __forceinline__ Recip2T make_recip2(const Recip& r) {
+    Recip2T p;
+    const float e = __fmaf_rn(-r.s, r.y, 1.0f);
+    p.y = f2_bcast(r.y);
+    p.ylo = f2_bcast(__fmul_rn(e, r.y));
+    p.ns = f2_bcast(-r.s);
+    return p;
+}
+__device__ __forceinline__ F2 div_chain2(F2 x, const Recip2T& r) {
+    const F2 q0 = f2_fma(x, r.y, f2_mul(x, r.ylo));
+    const F2 e0 = f2_fma(r.ns, q0, x);
+    return f2_fma(e0, r.y, q0);
 }
 
 // ---------------------------------------------------------------- int codes

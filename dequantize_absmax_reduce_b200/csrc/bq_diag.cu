@@ -1,4 +1,4 @@
-// Encoder diagnostic (bq_diag_encode_f32): f32 values encoded by the same
+// Encoder and divider diagnostics. bq_diag_encode_f32: f32 values encoded by the same
 // device functions the quantize and dequantize kernels call — the E4M3 and
 // E2M1 conversions of the microscaled formats and the round-to-nearest-even
 // narrowing to bf16 / f16 of every float output — so that the encoders can
@@ -84,5 +84,53 @@ extern "C" bq_status bq_diag_encode_f32(const float* x, int64_t n, bq_dtype fmt,
     if (blocks < 1) blocks = 1;
     if (blocks > 148 * 8) blocks = 148 * 8;
     k_diag_encode<<<(unsigned)blocks, kThreads, 0, (cudaStream_t)stream>>>(x, n, f, (uint8_t*)out);
+    return cudaGetLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+}
+
+namespace {
+
+// fl(x / s) on pairs through the kernels' reciprocal chains (CHAIN 0: five
+// roundings, 1: four from a two-term reciprocal).
+template <int CHAIN>
+__global__ void __launch_bounds__(kThreads) k_diag_divide(const float2* __restrict__ x, int64_t n2, float s,
+                                                           float2* __restrict__ out) {
+    const bq::Recip r = bq::make_recip(s);
+    for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < n2; i += (int64_t)gridDim.x * kThreads) {
+        const float2 v = x[i];
+        const bq::F2 xv = bq::f2_pack(v.x, v.y);
+        bq::F2 q;
+        if (CHAIN == 0) {
+            bq::Recip2 r2;
+            r2.y = bq::f2_bcast(r.y);
+            r2.ns = bq::f2_bcast(-r.s);
+            q = bq::div_chain2(xv, r2);
+        } else {
+            q = bq::div_chain2(xv, bq::make_recip2(r));
+        }
+        float a, b;
+        bq::f2_split(q, a, b);
+        out[i] = make_float2(a, b);
+    }
+}
+
+}  // namespace
+
+extern "C" bq_status bq_diag_divide_f32(const float* x, int64_t n, float s, int chain, float* out,
+                                        void* stream) {
+    if (n < 0 || (n & 1) || (chain != 0 && chain != 1)) return BQ_ERR_INVALID_ARG;
+    const float as = fabsf(s);
+    if (!(as >= 0x1p-64f && as <= 0x1p64f)) return BQ_ERR_INVALID_ARG;
+    if (n == 0) return BQ_OK;
+    if (!x || !out) return BQ_ERR_INVALID_ARG;
+    if (((uintptr_t)x % 8) != 0 || ((uintptr_t)out % 8) != 0) return BQ_ERR_MISALIGNED;
+    const int64_t n2 = n / 2;
+    int64_t blocks = (n2 + kThreads - 1) / kThreads;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    if (chain == 0)
+        k_diag_divide<0><<<(unsigned)blocks, kThreads, 0, (cudaStream_t)stream>>>(
+            reinterpret_cast<const float2*>(x), n2, s, reinterpret_cast<float2*>(out));
+    else
+        k_diag_divide<1><<<(unsigned)blocks, kThreads, 0, (cudaStream_t)stream>>>(
+            reinterpret_cast<const float2*>(x), n2, s, reinterpret_cast<float2*>(out));
     return cudaGetLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }

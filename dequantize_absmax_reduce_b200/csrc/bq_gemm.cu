@@ -507,7 +507,7 @@ __global__ void __launch_bounds__(NT, 1) k_fp8_gemm(const __grid_constant__ CUte
                 if (!(ok = bar_wait<CL, true>(bar(P::B_EMPTY_Q + sq), ((uint32_t)(iq / SQ) & 1u) ^ 1u, abort_flag, abort_addr))) break;
                 const uint32_t aq_row = base + P::OFF_AQ + (uint32_t)sq * AQ_BYTES + (uint32_t)R * 128u;
                 const bool fast = R1.fast && !nan;
-                const Recip2 R2 = make_recip2(R1);
+                const Recip2T R2 = make_recip2(R1);
 #pragma unroll
                 for (int jj = 0; jj < CPT / 2; ++jj) {
                     // Codes of input chunks c0, c0 + 1 (16 values) -> code chunk c0 / 2.

@@ -307,7 +307,7 @@ __global__ void __launch_bounds__(NT) k_seg_pipe(PipeArgs a) {
                 noclamp = (zf == __fsub_rn(qlo, rz)) && (__fadd_rn(kmax, zf) <= qhi);
             }
             if (seg_ok && R.fast && noclamp && !warp_nan) {
-                const Recip2 R2 = make_recip2(R);
+                const Recip2T R2 = make_recip2(R);
                 const F2 magic2 = f2_bcast(kMagic), zp2 = f2_bcast(zf), s2v = f2_bcast(sc);
                 // Whole groups: one branch-free block, so the vectors' division
                 // chains interleave.
@@ -337,7 +337,7 @@ __global__ void __launch_bounds__(NT) k_seg_pipe(PipeArgs a) {
                 if (seg_ok && lane == 0) a.scale[seg] = s;
                 const Recip R = make_recip(s);
                 if (seg_ok && R.fast && !warp_nan) {
-                    const Recip2 R2 = make_recip2(R);
+                    const Recip2T R2 = make_recip2(R);
                     if (full) {
 #pragma unroll
                         for (int j = 0; j < NV; ++j) emit_fp8_fast<T>(raw[j], R2, base + coff(j));
@@ -400,7 +400,7 @@ __global__ void __launch_bounds__(NT) k_seg_pipe(PipeArgs a) {
                 // overflow (|x| <= hi <= 2^64 eff).
                 const bool fast = R.fast && eff > 0.0f && hi <= __fmul_rn(0x1p64f, eff) && !warp_nan;
                 if (seg_ok && fast) {
-                    const Recip2 R2 = make_recip2(R);
+                    const Recip2T R2 = make_recip2(R);
                     if (full) {
 #pragma unroll
                         for (int j = 0; j < NV; ++j) emit_nv_fast<T>(raw[j], R2, base + coff(j));
@@ -725,7 +725,7 @@ __global__ void __launch_bounds__(256) k_fp8_tile_tma(const __grid_constant__ CU
         const bool full = (nr == 128) && (nch == 16);
         uint8_t* obase = a.e4m3 + bi * 128 * a.cols + bj * 128;
         const bool fast = R.fast && !any_nan;
-        const Recip2 R2 = make_recip2(R);
+        const Recip2T R2 = make_recip2(R);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int v = i * 256 + tid;
@@ -818,7 +818,7 @@ __global__ void __launch_bounds__(256) k_fp8t_pipe(Fp8TArgs a) {
     }
     const Recip R = make_recip(s);
     const bool fast_s = R.fast && s > 0.0f;
-    const Recip2 R2 = make_recip2(R);
+    const Recip2T R2 = make_recip2(R);
     const float lim = __fmul_rn(0x1p64f, s);
     int slot = 0;
     uint32_t parity = 0;

@@ -139,8 +139,8 @@ __device__ __forceinline__ void mx_emit(const float* v, const Recip& R, float mu
 
 // Integer codes (QUANT: the low byte of magic + k + zp) or fake-quantized
 // values (FAKE: fl(k * s)), k = round-half-even(fl(x / s)).
-template <class T, int OP, bool ASYM>
-__device__ __forceinline__ void emit_int_fast(const U4& raw, const Recip2& R2, F2 magic2, F2 zp2,
+template <class T, int OP, bool ASYM, class R2T>
+__device__ __forceinline__ void emit_int_fast(const U4& raw, const R2T& R2, F2 magic2, F2 zp2,
                                               F2 s2, uint8_t* q, int packed, T* y) {
     constexpr int VEC = Traits<T>::VEC;
     constexpr int NP = VEC / 2;
@@ -184,8 +184,8 @@ __device__ __forceinline__ uint32_t sign_bytes(const U4& raw) {
 // -0 there and changes nothing else (non-zero codes already carry it, and no
 // value is NaN).
 // The codes of one vector as words (VEC / 4 of them: byte i = value i).
-template <class T>
-__device__ __forceinline__ uint2 fp8_words_fast(const U4& raw, const Recip2& R2) {
+template <class T, class R2T>
+__device__ __forceinline__ uint2 fp8_words_fast(const U4& raw, const R2T& R2) {
     constexpr int VEC = Traits<T>::VEC;
     constexpr int NP = VEC / 2;
     F2 x[NP];
@@ -199,8 +199,8 @@ __device__ __forceinline__ uint2 fp8_words_fast(const U4& raw, const Recip2& R2)
     else w.y = 0u;
     return w;
 }
-template <class T>
-__device__ __forceinline__ void emit_fp8_fast(const U4& raw, const Recip2& R2, uint8_t* dst) {
+template <class T, class R2T>
+__device__ __forceinline__ void emit_fp8_fast(const U4& raw, const R2T& R2, uint8_t* dst) {
     const uint2 w = fp8_words_fast<T>(raw, R2);
     if constexpr (Traits<T>::VEC == 8) st8(dst, w.x, w.y);
     else st4(dst, w.x);
@@ -221,8 +221,8 @@ __device__ __forceinline__ uint2 fp8_words_general8(const float (&v)[8], const R
 
 // E2M1 codes of fl(x / s), the sign of each quotient taken from x (no NaN
 // among the values: the caller's guarantee above).
-template <class T>
-__device__ __forceinline__ void emit_nv_fast(const U4& raw, const Recip2& R2, uint8_t* dst) {
+template <class T, class R2T>
+__device__ __forceinline__ void emit_nv_fast(const U4& raw, const R2T& R2, uint8_t* dst) {
     constexpr int VEC = Traits<T>::VEC;
     constexpr int NP = VEC / 2;
     F2 x[NP];

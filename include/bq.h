@@ -216,6 +216,17 @@ bq_status bq_diag_wait_timeout(uint32_t tries, void* stream);
  * NULL pointer with n > 0. */
 bq_status bq_diag_encode_f32(const float* x, int64_t n, bq_dtype fmt, void* out, void* stream);
 
+/* Diagnostic of the quotient fl(x / s) the quantizers divide by (no
+ * counterpart on the pages): out[i] = x[i] / s for n f32 values, computed
+ * on f32 pairs by the kernels' own reciprocal chain: chain = 0 the
+ * five-rounding chain (the reciprocal and two remainder corrections), 1 the
+ * four-rounding chain from a two-term reciprocal (one correction), which
+ * the per-row quantizers use. Both are exact (IEEE round to nearest) for
+ * 2^-64 <= |s| <= 2^64 and quotients that neither overflow nor fall below
+ * 2^-100; s outside that range is BQ_ERR_INVALID_ARG. n even, x and out
+ * 8-byte aligned (BQ_ERR_MISALIGNED), one launch. */
+bq_status bq_diag_divide_f32(const float* x, int64_t n, float s, int chain, float* out, void* stream);
+
 /* -------------------------------------------------------------- quantize */
 /* [baracuda] quantize_per_tensor / per_channel / per_token / per_group.
  * x: d->shape, dtype d->x_dtype. q: same shape, dtype d->q_dtype.
