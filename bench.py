@@ -53,9 +53,9 @@ TRAFFIC_SOURCES = ("bq_abi.cu", "bq_int.cu", "bq_pipe.cu", "bq_pipe_bf16.cu", "b
                    "bq_pipe_args.h", "bq_device.cuh", "bq_internal.h", "bq_map_ops.cuh",
                    "bq_quant_ops.cuh", "bq_range.cuh")
 NCU_TRAFFIC = {
-    "quantize_per_token": {"src_sha256": "d96cb38586416c7132f23bb2b1660feb113243a94fe0c3128fea3b6a7172a5f7", "bytes_per_launch": 71384320},
-    "dequantize_per_token": {"src_sha256": "d96cb38586416c7132f23bb2b1660feb113243a94fe0c3128fea3b6a7172a5f7", "bytes_per_launch": 39869952},
-    "quantize_per_token_backward": {"src_sha256": "d96cb38586416c7132f23bb2b1660feb113243a94fe0c3128fea3b6a7172a5f7", "bytes_per_launch": 159439360},
+    "quantize_per_token": {"src_sha256": "2bf6b8b499754285996e108397c1dabcabc17323f69129310851b1ab2d38e18f", "bytes_per_launch": 70334464},
+    "dequantize_per_token": {"src_sha256": "2bf6b8b499754285996e108397c1dabcabc17323f69129310851b1ab2d38e18f", "bytes_per_launch": 39076096},
+    "quantize_per_token_backward": {"src_sha256": "2bf6b8b499754285996e108397c1dabcabc17323f69129310851b1ab2d38e18f", "bytes_per_launch": 159325952},
 }
 
 
