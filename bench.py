@@ -53,15 +53,16 @@ TRAFFIC_SOURCES = ("bq_abi.cu", "bq_int.cu", "bq_pipe.cu", "bq_pipe_bf16.cu", "b
                    "bq_pipe_args.h", "bq_device.cuh", "bq_internal.h", "bq_map_ops.cuh",
                    "bq_quant_ops.cuh", "bq_range.cuh")
 NCU_TRAFFIC = {
-    "quantize_per_token": {"src_sha256": "2bf6b8b499754285996e108397c1dabcabc17323f69129310851b1ab2d38e18f", "bytes_per_launch": 70334464},
-    "dequantize_per_token": {"src_sha256": "2bf6b8b499754285996e108397c1dabcabc17323f69129310851b1ab2d38e18f", "bytes_per_launch": 39076096},
-    "quantize_per_token_backward": {"src_sha256": "2bf6b8b499754285996e108397c1dabcabc17323f69129310851b1ab2d38e18f", "bytes_per_launch": 159325952},
+    "quantize_per_token": {"src_sha256": "f6951c07fdda335427e2696a504b022566d727d7a8ffd5b9cdf01f716552b362", "bytes_per_launch": 70334464},
+    "dequantize_per_token": {"src_sha256": "f6951c07fdda335427e2696a504b022566d727d7a8ffd5b9cdf01f716552b362", "bytes_per_launch": 39076096},
+    "quantize_per_token_backward": {"src_sha256": "f6951c07fdda335427e2696a504b022566d727d7a8ffd5b9cdf01f716552b362", "bytes_per_launch": 159325952},
 }
 
 
 def _strip_comments(src: str) -> str:
     """C / C++ source without its comments (string and character literals
-    kept), so that comment edits leave the hash unchanged."""
+    kept), trailing blanks or blank lines, so that comment edits leave the
+    hash unchanged."""
     out, i, n = [], 0, len(src)
     while i < n:
         c = src[i]
@@ -80,7 +81,8 @@ def _strip_comments(src: str) -> str:
         else:
             out.append(c)
             i += 1
-    return "".join(out)
+    # trailing blanks left by a removed comment and comment-only lines go too
+    return "\n".join(ln.rstrip() for ln in "".join(out).split("\n") if ln.strip())
 
 
 def _kernel_source_hash() -> str:

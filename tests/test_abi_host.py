@@ -198,3 +198,33 @@ def test_weight_prep_argument_errors(B):
     # zero-sized calls succeed without touching the device
     assert B.lib.bq_nvfp4_concat_rows(None, None, 1.0, 0, None, None, 1.0, 0, 32, None, None, C.byref(s2o), None) == B.BQ_OK
     assert s2o.value == 1.0
+
+
+def test_gemm_and_diagnostic_argument_errors(B):
+    # Every call below fails validation (or is empty) before any CUDA call.
+    P = 0x10000
+    L = B.lib
+    # fused-prologue GEMM: dtypes, k, sizes, operand outputs, alignment
+    assert L.bq_fp8_block_gemm(P, B.BQ_F32, 4, 128, P, P, 16, P, B.BQ_F32, None, None, None) == B.BQ_ERR_UNSUPPORTED
+    assert L.bq_fp8_block_gemm(P, B.BQ_BF16, 4, 128, P, P, 16, P, B.BQ_F16, None, None, None) == B.BQ_ERR_UNSUPPORTED
+    assert L.bq_fp8_block_gemm(P, B.BQ_BF16, 4, 100, P, P, 16, P, B.BQ_F32, None, None, None) == B.BQ_ERR_INVALID_ARG
+    assert L.bq_fp8_block_gemm(P, B.BQ_BF16, -1, 128, P, P, 16, P, B.BQ_F32, None, None, None) == B.BQ_ERR_INVALID_ARG
+    assert L.bq_fp8_block_gemm(P, B.BQ_BF16, 4, 128, P, P, 16, P, B.BQ_F32, P, None, None) == B.BQ_ERR_INVALID_ARG
+    assert L.bq_fp8_block_gemm(P + 2, B.BQ_BF16, 4, 128, P, P, 16, P, B.BQ_F32, None, None, None) == B.BQ_ERR_MISALIGNED
+    assert L.bq_fp8_block_gemm(None, B.BQ_BF16, 0, 128, None, None, 16, None, B.BQ_F32, None, None, None) == B.BQ_OK
+    # the same product on quantized activations
+    assert L.bq_fp8_block_gemm_quantized(P, P, 4, 128, P, P, 16, P, B.BQ_F16, None) == B.BQ_ERR_UNSUPPORTED
+    assert L.bq_fp8_block_gemm_quantized(P, P, 4, 100, P, P, 16, P, B.BQ_F32, None) == B.BQ_ERR_INVALID_ARG
+    assert L.bq_fp8_block_gemm_quantized(P, None, 4, 128, P, P, 16, P, B.BQ_F32, None) == B.BQ_ERR_INVALID_ARG
+    assert L.bq_fp8_block_gemm_quantized(P + 8, P, 4, 128, P, P, 16, P, B.BQ_F32, None) == B.BQ_ERR_MISALIGNED
+    assert L.bq_fp8_block_gemm_quantized(None, None, 4, 128, None, None, 0, None, B.BQ_F32, None) == B.BQ_OK
+    # the encoder and divider diagnostics
+    assert L.bq_diag_encode_f32(P, 8, B.BQ_S8, P, None) == B.BQ_ERR_UNSUPPORTED
+    assert L.bq_diag_encode_f32(P, 7, B.BQ_E2M1X2, P, None) == B.BQ_ERR_INVALID_ARG
+    assert L.bq_diag_encode_f32(P + 4, 8, B.BQ_E4M3, P, None) == B.BQ_ERR_MISALIGNED
+    assert L.bq_diag_divide_f32(P, 8, 0.0, 1, P, None) == B.BQ_ERR_INVALID_ARG
+    assert L.bq_diag_divide_f32(P, 8, 2.0 ** 65, 0, P, None) == B.BQ_ERR_INVALID_ARG
+    assert L.bq_diag_divide_f32(P, 7, 3.0, 1, P, None) == B.BQ_ERR_INVALID_ARG
+    assert L.bq_diag_divide_f32(P, 8, 3.0, 2, P, None) == B.BQ_ERR_INVALID_ARG
+    assert L.bq_diag_divide_f32(P + 4, 8, 3.0, 1, P, None) == B.BQ_ERR_MISALIGNED
+    assert L.bq_diag_divide_f32(None, 0, 3.0, 1, None, None) == B.BQ_OK
