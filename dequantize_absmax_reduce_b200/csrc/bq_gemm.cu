@@ -167,13 +167,6 @@ __device__ __forceinline__ void arrive_all_ranks(uint32_t bar, int lane) {
         else bar_arrive_remote_relaxed(a);
     }
 }
-__device__ __forceinline__ void st_cluster16(uint32_t cl_addr, const U4& v) {
-    asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};"
-                 :: "r"(cl_addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
-}
-__device__ __forceinline__ void st_cluster_f32(uint32_t cl_addr, float v) {
-    asm volatile("st.shared::cluster.f32 [%0], %1;" :: "r"(cl_addr), "f"(v) : "memory");
-}
 __device__ __forceinline__ void st_cluster_u32(uint32_t cl_addr, uint32_t v) {
     asm volatile("st.shared::cluster.u32 [%0], %1;" :: "r"(cl_addr), "r"(v) : "memory");
 }
@@ -191,9 +184,6 @@ __device__ __forceinline__ uint32_t cluster_rank() {
 }
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void fence_async_shared_cluster() {
-    asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
 }
 // Bounded wait (each try suspends for at most about a microsecond); gives up
 // early once another role (of any CTA of the cluster) has set the abort
@@ -1125,6 +1115,11 @@ __global__ void __launch_bounds__(NT_Q, 1) k_fp8_gemm_q2(const __grid_constant__
     cluster_sync();                                   // no TMEM access or remote arrival left in the pair
     tc_fence_after();
     if (warp == 2) tmem_dealloc_pair(tmem, TMEM_COLS);
+    // Every stage loaded was consumed unless the pair gave up (the flag is
+    // visible here after the cluster barrier); then copies may still be in
+    // flight to this CTA's ring or CTA 0's barriers: keep the shared memory
+    // alive until they have landed.
+    if (threadIdx.x == 0 && *abort_flag) pause_us(1000);
 }
 
 cudaError_t encode_map(CUtensorMap* tm, CUtensorMapDataType dt, const void* p, uint64_t inner,
