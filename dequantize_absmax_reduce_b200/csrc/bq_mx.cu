@@ -514,6 +514,52 @@ __global__ void __launch_bounds__(256) k_nv_predeq8(const uint8_t* __restrict__ 
     }
 }
 
+// The same on 16-byte code chunks (32 elements, two scale blocks): one
+// 16-byte code load and one 2-byte scale load per chunk, two 16-byte stores;
+// PQ_U chunks loaded per thread before any is decoded. Needs numel % 32 == 0,
+// codes and out 16-byte aligned and scales 2-byte aligned.
+constexpr int PQ_U = 4;
+__global__ void __launch_bounds__(256) k_nv_predeq16(const uint8_t* __restrict__ codes,
+                                                     const uint8_t* __restrict__ scales,
+                                                     const float* __restrict__ global_scale,
+                                                     int64_t numel, uint8_t* __restrict__ out) {
+    const float s2 = __ldg(global_scale);
+    const int64_t n_items = numel / 32;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < n_items;
+         base += stride * PQ_U) {
+        U4 w[PQ_U];
+        uint32_t sb[PQ_U];
+#pragma unroll
+        for (int u = 0; u < PQ_U; ++u) {
+            const int64_t it = base + u * stride;
+            if (it < n_items) {
+                w[u] = ld16_stream(codes + it * 16);
+                sb[u] = __ldg(reinterpret_cast<const unsigned short*>(scales) + it);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < PQ_U; ++u) {
+            const int64_t it = base + u * stride;
+            if (it >= n_items) continue;
+            const F2 m0 = f2_bcast(__fmul_rn(e4m3_to_f32(sb[u] & 0xFFu), s2));   // block 2 it
+            const F2 m1 = f2_bcast(__fmul_rn(e4m3_to_f32(sb[u] >> 8), s2));      // block 2 it + 1
+            float o[8];
+            U4 r0, r1;
+            e2m1x8_mul(w[u].x, m0, o);
+            r0.x = e4m3x4(o[0], o[1], o[2], o[3]); r0.y = e4m3x4(o[4], o[5], o[6], o[7]);
+            e2m1x8_mul(w[u].y, m0, o);
+            r0.z = e4m3x4(o[0], o[1], o[2], o[3]); r0.w = e4m3x4(o[4], o[5], o[6], o[7]);
+            e2m1x8_mul(w[u].z, m1, o);
+            r1.x = e4m3x4(o[0], o[1], o[2], o[3]); r1.y = e4m3x4(o[4], o[5], o[6], o[7]);
+            e2m1x8_mul(w[u].w, m1, o);
+            r1.z = e4m3x4(o[0], o[1], o[2], o[3]); r1.w = e4m3x4(o[4], o[5], o[6], o[7]);
+            st16(out + it * 32, r0);
+            st16(out + it * 32 + 16, r1);
+        }
+    }
+}
+
 // Element-wise fallback (any alignment).
 __global__ void __launch_bounds__(256) k_nv_predeq_scalar(const uint8_t* __restrict__ codes,
                                                           const uint8_t* __restrict__ scales,
@@ -769,7 +815,10 @@ cudaError_t nvfp4_predequant_fp8(const uint8_t* codes, const uint8_t* scales, co
                                  int64_t rows, int64_t k, uint8_t* out, cudaStream_t st) {
     const int64_t numel = rows * k;
     if (numel == 0) return cudaSuccess;
-    if (k % 16 == 0 && al(codes, 4) && al(out, 8)) {
+    if (numel % 32 == 0 && k % 16 == 0 && al(codes, 16) && al(out, 16) && al(scales, 2)) {
+        const int64_t blocks = (numel / 32 + 256 * PQ_U - 1) / (256 * PQ_U);
+        k_nv_predeq16<<<grid_occ_mx<k_nv_predeq16>(blocks), 256, 0, st>>>(codes, scales, global_scale, numel, out);
+    } else if (k % 16 == 0 && al(codes, 4) && al(out, 8)) {
         const int64_t blocks = (numel / 8 + 256 * DQ_U - 1) / (256 * DQ_U);
         k_nv_predeq8<<<grid_occ_mx<k_nv_predeq8>(blocks), 256, 0, st>>>(codes, scales, global_scale, numel, out);
     } else {
